@@ -1,0 +1,176 @@
+"""CPU oracle for paged-KV GQA decode attention with split-KV scheduling.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+bench's CPU-baseline / reference arm may import this module; the product path
+(``paged_kv_decode_29_b200``) never does. It shares no code with the CUDA
+path; both only read inputs drawn by ``workloads``.
+
+Everything is computed in fp64 by ``oracle.c``:
+
+* ``decode`` / ``decode_rows`` / ``attend``: scaled-dot-product attention of
+  each query row over the paged KV cache, with an explicit full softmax and the
+  bottom-right causal mask of speculative multi-token queries ("PaddlePaddle/
+  HALOps" README, Highlights, GQA attention item).
+* ``plan``: the greedy bin-packing of uniform KV tiles onto CTAs ("HPC-Ops:
+  Tencent's CUDA Kernel Library for LLM Inference Hot Paths", "How the kernels
+  are organized around specific workload shapes"), as a literal sequential
+  greedy over the tiles sorted by cost.
+* ``e4m3_value``: the OCP E4M3 "fn" code table.
+
+Parity pins for each function live in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into oracle/_build/liboracle.so (gcc, -O2, OpenMP)."""
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Problem(C.Structure):
+    _fields_ = [
+        ("batch", C.c_int32), ("q_tokens", C.c_int32), ("n_q_heads", C.c_int32), ("n_kv_heads", C.c_int32),
+        ("head_dim", C.c_int32), ("page_size", C.c_int32), ("num_pages", C.c_int32),
+        ("max_pages_per_seq", C.c_int32), ("kv_fp8", C.c_int32), ("pad_", C.c_int32),
+        ("sm_scale", C.c_double),
+        ("q", C.c_void_p), ("k_pages", C.c_void_p), ("v_pages", C.c_void_p), ("kv_scales", C.c_void_p),
+        ("page_table", C.c_void_p), ("seq_lens", C.c_void_p),
+    ]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = C.CDLL(build())
+            P = C.POINTER(_Problem)
+            lib.oracle_decode.argtypes = [P, C.c_void_p, C.c_void_p, C.c_int]
+            lib.oracle_decode_rows.argtypes = [P, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_int]
+            lib.oracle_attend.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int64, C.c_int64,
+                                          C.c_void_p, C.c_void_p, C.c_void_p]
+            lib.oracle_attend.restype = C.c_int64
+            lib.oracle_plan.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int64,
+                                        C.c_void_p, C.c_void_p, C.c_void_p]
+            lib.oracle_plan.restype = C.c_int64
+            lib.oracle_e4m3_value.argtypes = [C.c_uint8]
+            lib.oracle_e4m3_value.restype = C.c_double
+            lib.oracle_max_threads.restype = C.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+class _Bound:
+    """Keeps the numpy arrays alive while the C struct points at them."""
+
+    def __init__(self, pr):
+        self.arrs = dict(
+            q=np.ascontiguousarray(pr.q, dtype=np.uint16),
+            k=np.ascontiguousarray(pr.k_pages),
+            v=np.ascontiguousarray(pr.v_pages),
+            s=None if pr.kv_scales is None else np.ascontiguousarray(pr.kv_scales, dtype=np.float32),
+            t=np.ascontiguousarray(pr.page_table, dtype=np.int32),
+            L=np.ascontiguousarray(pr.seq_lens, dtype=np.int32),
+        )
+        a = self.arrs
+        fp8 = pr.kv_dtype == "fp8e4m3"
+        if fp8 and a["s"] is None:
+            raise ValueError("FP8 KV needs kv_scales")
+        self.s = _Problem(pr.batch, pr.q_tokens, pr.n_q_heads, pr.n_kv_heads, pr.head_dim, pr.page_size,
+                          int(a["k"].shape[0]), int(a["t"].shape[1]), int(fp8), 0, float(pr.sm_scale),
+                          _ptr(a["q"]), _ptr(a["k"]), _ptr(a["v"]), _ptr(a["s"]), _ptr(a["t"]), _ptr(a["L"]))
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def decode(pr, nthreads: int = 0):
+    """All rows. Returns out float64 [B][T][Hq][d] and lse float64 [B][T][Hq] (natural log)."""
+    lib = _load()
+    bd = _Bound(pr)
+    out = np.zeros((pr.batch, pr.q_tokens, pr.n_q_heads, pr.head_dim), dtype=np.float64)
+    lse = np.zeros((pr.batch, pr.q_tokens, pr.n_q_heads), dtype=np.float64)
+    lib.oracle_decode(C.byref(bd.s), out.ctypes.data, lse.ctypes.data, int(nthreads))
+    return out, lse
+
+
+def decode_rows(pr, rows, nthreads: int = 0):
+    """Selected rows, ``rows`` an int array [n][3] of (b, t, qh)."""
+    lib = _load()
+    bd = _Bound(pr)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+    n = rows.shape[0]
+    out = np.zeros((n, pr.head_dim), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    lib.oracle_decode_rows(C.byref(bd.s), rows.ctypes.data, n, out.ctypes.data, lse.ctypes.data, int(nthreads))
+    return out, lse
+
+
+def attend(pr, b, t, qh, j_lo=0, j_hi=None, weights=False):
+    """One row over keys [j_lo, j_hi) (clipped to the causal limit).
+
+    Returns (out[d], lse, n_visible[, weights[n_visible]])."""
+    lib = _load()
+    bd = _Bound(pr)
+    if j_hi is None:
+        j_hi = int(pr.seq_lens[b])
+    out = np.zeros(pr.head_dim, dtype=np.float64)
+    lse = np.zeros(1, dtype=np.float64)
+    w = np.zeros(max(1, int(j_hi) - int(j_lo)), dtype=np.float64) if weights else None
+    n = lib.oracle_attend(C.byref(bd.s), int(b), int(t), int(qh), int(j_lo), int(j_hi),
+                          out.ctypes.data, lse.ctypes.data, _ptr(w))
+    if weights:
+        return out, float(lse[0]), int(n), w[:n]
+    return out, float(lse[0]), int(n)
+
+
+UNIT_FIELDS = ("b", "h", "tok_begin", "tok_end", "seq_len", "slot", "tile", "zero")
+
+
+def plan(seq_lens, n_kv_heads: int, tile_len: int, n_bins: int, capacity: int | None = None):
+    """Greedy bin-packing of uniform KV tiles. Returns dict(n_units, bin_off, units[U][8], pair_off)
+    or None when the tile count exceeds ``capacity``."""
+    lib = _load()
+    L = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    B = L.shape[0]
+    U_max = int(n_kv_heads * ((L.astype(np.int64) + tile_len - 1) // tile_len).sum())
+    cap = U_max if capacity is None else int(capacity)
+    bin_off = np.zeros(n_bins + 1, dtype=np.int32)
+    units = np.zeros((max(U_max, 1), 8), dtype=np.int32)
+    pair_off = np.zeros(B * n_kv_heads + 1, dtype=np.int32)
+    U = lib.oracle_plan(L.ctypes.data, B, int(n_kv_heads), int(tile_len), int(n_bins), cap,
+                        bin_off.ctypes.data, units.ctypes.data, pair_off.ctypes.data)
+    if U < 0:
+        return None
+    return dict(n_units=int(U), bin_off=bin_off, units=units[:U], pair_off=pair_off)
+
+
+def e4m3_value(code: int) -> float:
+    return float(_load().oracle_e4m3_value(int(code) & 0xFF))
+
+
+def e4m3_table() -> np.ndarray:
+    return np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
