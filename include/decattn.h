@@ -1,0 +1,173 @@
+/*
+ * decattn.h -- C ABI of libdecattn.so: GQA decode attention over a paged KV
+ * cache with dynamic split-KV scheduling, for NVIDIA B200 (sm_100a).
+ *
+ * The operation ("PaddlePaddle/HALOps" README, Highlights, GQA attention item):
+ * paged-KV decode attention with BF16 or FP8 KV cache, grouped-query heads and
+ * speculative decoding (several query tokens per request), with split-KV
+ * parallelism and an adaptive reduction.
+ * The scheduling ("HPC-Ops: Tencent's CUDA Kernel Library for LLM Inference Hot
+ * Paths", section "How the kernels are organized around specific workload
+ * shapes"): before each decode step the requests are cut into uniform KV tiles,
+ * the tiles are balanced across CTAs by greedy bin-packing, and a combine
+ * kernel merges the split results.
+ *
+ * For query row (b, t, qh) with h = qh / (n_q_heads / n_kv_heads) and KV length
+ * Lb = seq_lens[b], the visible keys are j = 0 .. Lb - T + t (the T query
+ * tokens are the last T tokens of the cache; bottom-right causal). With
+ * s_j = sm_scale * <q[b][t][qh], K[b,h,j]>:
+ *     out[b][t][qh] = sum_j softmax(s)_j * V[b,h,j],   lse[b][t][qh] = ln sum_j e^{s_j}.
+ * K[b,h,j] is row (j % P) of block [page_table[b][j / P]][h] of k_pages (FP8:
+ * the code's value times kv_scales[0][page][h]; V likewise with kv_scales[1]).
+ * A row with no visible key gets out = 0 and lse = -inf.
+ *
+ * Conventions for every call:
+ *  - "device" pointers are CUDA device memory on the current device; "host"
+ *    pointers are ordinary host memory. The caller allocates and owns every
+ *    buffer; the library never allocates, never frees and keeps no state
+ *    between calls other than per-device attributes it caches.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). dec_attn_plan and
+ *    dec_attn_run only enqueue work on it: they never synchronise, so both may
+ *    be captured into a CUDA graph.
+ *  - Errors that the host can see (null or misaligned pointers, unsupported
+ *    shapes, buffers too small) return a negative decattn_status and enqueue
+ *    nothing. Errors only the device can see (a page id outside the pool, more
+ *    tiles than the plan can hold, a pipeline wait that gives up) never trap:
+ *    they set a status word in the plan or workspace, which
+ *    dec_attn_read_status() returns.
+ */
+#ifndef DECATTN_H
+#define DECATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DECATTN_API __attribute__((visibility("default")))
+#else
+#define DECATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DECATTN_OK = 0,
+  DECATTN_EINVAL = -1,   /* invalid argument: null pointer, negative size, inconsistent plan/shape */
+  DECATTN_ENOTSUP = -2,  /* valid but unsupported: head_dim, page size, tile length, group size, dtype */
+  DECATTN_ESMALL = -3,   /* a caller buffer (plan or workspace) is too small */
+  DECATTN_ECUDA = -4,    /* a CUDA runtime call failed (launch, attribute query) */
+  DECATTN_ETIMEOUT = -5, /* device: a pipeline wait gave up (the kernel returned early) */
+  DECATTN_EDEVICE = -6,  /* device: bad input seen by a kernel (page id outside the pool, negative
+                            seq_len, seq_len beyond the page-table row) */
+  DECATTN_EALIGN = -7,   /* a pointer is not 16-byte aligned */
+  DECATTN_ECAPACITY = -8 /* device: the tiles of seq_lens exceed the plan's capacity */
+} decattn_status;
+
+typedef enum { DECATTN_KV_BF16 = 0, DECATTN_KV_FP8E4M3 = 1 } decattn_kv_dtype;
+
+/* Host-side handle of a plan. dec_attn_plan fills it; dec_attn_run reads it. The
+ * work list itself lives in the caller's device buffer `buf`. */
+typedef struct {
+  void *buf;          /* device: plan buffer (header + tile list), caller-owned */
+  size_t buf_bytes;
+  int32_t batch;
+  int32_t n_kv_heads;
+  int32_t tile_len;   /* tokens per uniform KV tile */
+  int32_t n_bins;     /* CTAs of the split kernel; one bin of tiles per CTA */
+  int64_t max_units;  /* capacity of the tile list */
+} dec_attn_plan_t;
+
+/* Problem shape shared by dec_attn_workspace_bytes and dec_attn_run. */
+typedef struct {
+  int32_t batch;              /* B >= 0 requests */
+  int32_t n_q_heads;          /* Hq, a multiple of n_kv_heads */
+  int32_t n_kv_heads;         /* Hkv */
+  int32_t head_dim;           /* d: 64 or 128 */
+  int32_t q_tokens;           /* T >= 1 query tokens per request (T > 1: speculative decode) */
+  int32_t page_size;          /* P tokens per page: a multiple of 16, at most 256 */
+  int32_t num_pages;          /* pages in the pool */
+  int32_t max_pages_per_seq;  /* row stride of page_table */
+  int32_t kv_dtype;           /* decattn_kv_dtype */
+  float sm_scale;             /* softmax scale; <= 0 selects 1/sqrt(head_dim) */
+} dec_attn_shape;
+
+/* Number of bins (split-kernel CTAs) the library uses on `device` when a plan is
+ * made with n_bins = 0: SM count x CTAs resident per SM. Returns < 0 on error. */
+DECATTN_API int dec_attn_default_bins(int device);
+
+/* Bytes of the device plan buffer for a plan of `batch` requests whose KV lengths
+ * sum to at most max_total_kv_tokens. n_bins = 0 selects dec_attn_default_bins of
+ * the current device. Returns 0 for invalid arguments. */
+DECATTN_API size_t dec_attn_plan_bytes(int batch, int n_kv_heads, int tile_len, int64_t max_total_kv_tokens, int n_bins);
+
+/* Planner ("HPC-Ops ...", "How the kernels are organized around specific workload
+ * shapes": uniform KV tiles assigned before each decode step and balanced across
+ * CTAs by greedy bin-packing). One single-block kernel on `stream`:
+ *   1. each pair (b, h) is cut into n_b = ceil(Lb / tile_len) tiles
+ *      [i*tl, min((i+1)*tl, Lb)); cost of a tile = its token count;
+ *   2. tiles are stably sorted by cost, largest first ((b, h, i) order on ties);
+ *   3. in that order each tile goes to the least-loaded bin (lowest index on ties);
+ *   4. a bin keeps its tiles in assignment order.
+ * A tile of a pair with n_b > 1 writes its partial result to slot
+ * pair_off[b*Hkv+h] + i; a pair with n_b == 1 writes the final output directly.
+ *   seq_lens  device int32 [batch]: KV length of each request (>= 0).
+ *   tile_len  > 0 and a multiple of 16; dec_attn_run further needs it to be a
+ *             multiple of the page size.
+ *   plan_buf  device, plan_bytes >= dec_attn_plan_bytes(...), 16-byte aligned.
+ *   plan      host, filled on success.
+ * Device-side failures (sum of tiles above capacity, negative seq_len) set the
+ * plan's status (DECATTN_ECAPACITY / DECATTN_EDEVICE); a later dec_attn_run then
+ * writes nothing and reports the same status. */
+DECATTN_API int dec_attn_plan(const int32_t *seq_lens, int batch, int n_kv_heads, int tile_len, int64_t max_total_kv_tokens,
+                  int n_bins, void *plan_buf, size_t plan_bytes, dec_attn_plan_t *plan, void *stream);
+
+/* Bytes of the device workspace dec_attn_run needs: a status word plus room for
+ * the partial (o, lse) of every tile the plan can hold (fp32, [tiles][G*T][d+1]).
+ * Returns 0 for invalid arguments. */
+DECATTN_API size_t dec_attn_workspace_bytes(const dec_attn_shape *shape, const dec_attn_plan_t *plan);
+
+/* Split + combine ("PaddlePaddle/HALOps" README, Highlights, GQA attention item;
+ * "HPC-Ops ...", "How the kernels are organized around specific workload
+ * shapes": a combine kernel merges the split results). Enqueues, on `stream`:
+ *   - the split kernel: CTA k walks bin k of the plan; for each tile it stages the
+ *     page-table-indirected K/V rows through a shared-memory pipeline (TMA), computes
+ *     the G*T query rows of its KV head against them with an online softmax in
+ *     fp32 and writes the tile's normalised partial (o, lse) -- or, for a request
+ *     held in one tile, the final out/lse;
+ *   - the combine kernel: merges the partials of every row by log-sum-exp:
+ *     M = max_i lse_i, w_i = e^{lse_i - M}, out = sum_i w_i o_i / sum_i w_i,
+ *     lse = M + ln sum_i w_i (a partial with no visible key has lse -inf, weight 0).
+ * Arguments (all device pointers 16-byte aligned, except page_table, seq_lens, lse):
+ *   q          bf16 [B][T][Hq][d]
+ *   k_pages    [num_pages][Hkv][P][d], bf16 or FP8 E4M3 ("fn") codes
+ *   v_pages    same layout as k_pages
+ *   page_table int32 [B][max_pages_per_seq]: physical page of logical page p of
+ *              request b (entries past ceil(Lb/P) are not read)
+ *   seq_lens   int32 [B]: must hold the values the plan was made from
+ *   kv_scales  fp32 [2][num_pages][Hkv] (K scales, then V scales); FP8 only, else NULL
+ *   plan       host handle from dec_attn_plan (same batch and n_kv_heads)
+ *   workspace  device, workspace_bytes >= dec_attn_workspace_bytes(shape, plan)
+ *   out        fp32 [B][T][Hq][d];  lse  fp32 [B][T][Hq] (natural log)
+ * Supported: head_dim 64 or 128; page_size a multiple of 16 up to 256;
+ * tile_len a multiple of page_size; G*T <= 16. Anything else returns
+ * DECATTN_ENOTSUP before any launch. */
+DECATTN_API int dec_attn_run(const dec_attn_shape *shape, const void *q, const void *k_pages, const void *v_pages,
+                 const int32_t *page_table, const int32_t *seq_lens, const float *kv_scales,
+                 const dec_attn_plan_t *plan, void *workspace, size_t workspace_bytes, float *out, float *lse,
+                 void *stream);
+
+/* Synchronises `stream`, then returns the first device-detected status recorded in
+ * the plan header and (if not NULL) the workspace, or DECATTN_OK. Either pointer
+ * may be NULL. For tests and diagnostics, not for the hot path. */
+DECATTN_API int dec_attn_read_status(const dec_attn_plan_t *plan, const void *workspace, void *stream);
+
+/* Static text for a decattn_status value. */
+DECATTN_API const char *dec_attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DECATTN_H */

@@ -1,0 +1,221 @@
+"""GQA decode attention over a paged KV cache with dynamic split-KV scheduling, for
+NVIDIA B200 (sm_100a).
+
+This module is the Python face of ``libdecattn.so`` (C ABI in ``include/decattn.h``):
+it only marshals torch tensors into pointers and sizes. Every step of the work --
+planning, the split kernel, the combine -- runs in the library's CUDA kernels. If the
+library is missing, every call raises; there is no fallback.
+
+Typical use (one plan per decode step, reused by every layer)::
+
+    pl = plan(seq_lens, n_kv_heads=8, tile_len=256, max_total_kv_tokens=total)
+    out, lse = run(q, k_pages, v_pages, page_table, seq_lens, pl)
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdecattn.so")
+
+OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1, -2, -3, -4, -5, -6, -7, -8
+KV_BF16, KV_FP8E4M3 = 0, 1
+API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_workspace_bytes",
+       "dec_attn_run", "dec_attn_read_status", "dec_attn_status_string")
+
+
+class DecAttnError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)} ({code})" if what else f"{status_string(code)} ({code})")
+
+
+class PlanT(C.Structure):
+    _fields_ = [("buf", C.c_void_p), ("buf_bytes", C.c_size_t), ("batch", C.c_int32), ("n_kv_heads", C.c_int32),
+                ("tile_len", C.c_int32), ("n_bins", C.c_int32), ("max_units", C.c_int64)]
+
+
+class ShapeT(C.Structure):
+    _fields_ = [("batch", C.c_int32), ("n_q_heads", C.c_int32), ("n_kv_heads", C.c_int32), ("head_dim", C.c_int32),
+                ("q_tokens", C.c_int32), ("page_size", C.c_int32), ("num_pages", C.c_int32),
+                ("max_pages_per_seq", C.c_int32), ("kv_dtype", C.c_int32), ("sm_scale", C.c_float)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads libdecattn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m paged_kv_decode_29_b200.build` "
+                               "(or __graft_entry__.build()); there is no fallback path")
+        lib = C.CDLL(path)
+        vp, i32, i64, sz = C.c_void_p, C.c_int, C.c_int64, C.c_size_t
+        lib.dec_attn_default_bins.argtypes = [i32]
+        lib.dec_attn_default_bins.restype = i32
+        lib.dec_attn_plan_bytes.argtypes = [i32, i32, i32, i64, i32]
+        lib.dec_attn_plan_bytes.restype = sz
+        lib.dec_attn_plan.argtypes = [vp, i32, i32, i32, i64, i32, vp, sz, C.POINTER(PlanT), vp]
+        lib.dec_attn_plan.restype = i32
+        lib.dec_attn_workspace_bytes.argtypes = [C.POINTER(ShapeT), C.POINTER(PlanT)]
+        lib.dec_attn_workspace_bytes.restype = sz
+        lib.dec_attn_run.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, C.POINTER(PlanT), vp, sz, vp, vp, vp]
+        lib.dec_attn_run.restype = i32
+        lib.dec_attn_read_status.argtypes = [C.POINTER(PlanT), vp, vp]
+        lib.dec_attn_read_status.restype = i32
+        lib.dec_attn_status_string.argtypes = [i32]
+        lib.dec_attn_status_string.restype = C.c_char_p
+        _lib = lib
+        return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().dec_attn_status_string(int(code)).decode()
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    h = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return h or None
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+@dataclass
+class Plan:
+    """A plan: the device buffer holding the work list and its host handle."""
+    buf: torch.Tensor
+    handle: PlanT
+
+    @property
+    def n_bins(self) -> int:
+        return int(self.handle.n_bins)
+
+    @property
+    def tile_len(self) -> int:
+        return int(self.handle.tile_len)
+
+
+def default_bins(device: int | None = None) -> int:
+    dev = torch.cuda.current_device() if device is None else int(device)
+    n = load_library().dec_attn_default_bins(dev)
+    if n <= 0:
+        raise DecAttnError(ECUDA, "dec_attn_default_bins")
+    return n
+
+
+def plan_bytes(batch: int, n_kv_heads: int, tile_len: int, max_total_kv_tokens: int, n_bins: int = 0) -> int:
+    return int(load_library().dec_attn_plan_bytes(batch, n_kv_heads, tile_len, int(max_total_kv_tokens), n_bins))
+
+
+def plan(seq_lens: torch.Tensor, n_kv_heads: int, tile_len: int, max_total_kv_tokens: int | None = None,
+         n_bins: int = 0, buf: torch.Tensor | None = None, stream=None) -> Plan:
+    """Enqueues the planner (one single-block kernel) on ``stream``.
+
+    ``seq_lens``: int32 CUDA tensor [B]. ``max_total_kv_tokens`` bounds sum(seq_lens) and sizes the
+    plan buffer (None: read it from ``seq_lens``, which synchronises)."""
+    lib = load_library()
+    assert seq_lens.is_cuda and seq_lens.dtype == torch.int32 and seq_lens.is_contiguous()
+    B = int(seq_lens.numel())
+    if max_total_kv_tokens is None:
+        max_total_kv_tokens = int(seq_lens.sum().item()) if B else 0
+    nbytes = lib.dec_attn_plan_bytes(B, n_kv_heads, tile_len, int(max_total_kv_tokens), n_bins)
+    if nbytes == 0:
+        raise DecAttnError(ENOTSUP, "dec_attn_plan_bytes")
+    if buf is None:
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=seq_lens.device)
+    h = PlanT()
+    rc = lib.dec_attn_plan(_ptr(seq_lens), B, n_kv_heads, tile_len, int(max_total_kv_tokens), n_bins,
+                           buf.data_ptr(), buf.numel(), C.byref(h), _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_plan")
+    return Plan(buf=buf, handle=h)
+
+
+def make_shape(q: torch.Tensor, k_pages: torch.Tensor, page_table: torch.Tensor, kv_dtype: int,
+               sm_scale: float = 0.0) -> ShapeT:
+    B, T, Hq, d = q.shape
+    num_pages, Hkv, P, d2 = k_pages.shape
+    assert d == d2
+    return ShapeT(B, Hq, Hkv, d, T, P, num_pages, int(page_table.shape[1]), kv_dtype, float(sm_scale))
+
+
+def kv_dtype_of(k_pages: torch.Tensor) -> int:
+    if k_pages.dtype == torch.bfloat16:
+        return KV_BF16
+    if k_pages.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return KV_FP8E4M3
+    raise TypeError(f"KV pool dtype {k_pages.dtype} is not bf16 / e4m3")
+
+
+def workspace_bytes(shape: ShapeT, pl: Plan) -> int:
+    n = load_library().dec_attn_workspace_bytes(C.byref(shape), C.byref(pl.handle))
+    if n == 0:
+        raise DecAttnError(ENOTSUP, "dec_attn_workspace_bytes")
+    return int(n)
+
+
+def run(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_table: torch.Tensor,
+        seq_lens: torch.Tensor, pl: Plan, *, kv_scales: torch.Tensor | None = None, sm_scale: float = 0.0,
+        workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+        stream=None):
+    """Enqueues split + combine on ``stream``; returns (out fp32 [B][T][Hq][d], lse fp32 [B][T][Hq]).
+
+    q: bf16 [B][T][Hq][d]; k_pages / v_pages: [num_pages][Hkv][P][d] bf16, or uint8 / float8_e4m3fn
+    E4M3 codes with ``kv_scales`` fp32 [2][num_pages][Hkv]; page_table: int32 [B][max_pages_per_seq];
+    seq_lens: int32 [B] (the values the plan was made from)."""
+    lib = load_library()
+    kvt = kv_dtype_of(k_pages)
+    shape = make_shape(q, k_pages, page_table, kvt, sm_scale)
+    B, T, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, T, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, T, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(shape, pl), dtype=torch.uint8, device=q.device)
+    rc = lib.dec_attn_run(C.byref(shape), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(seq_lens),
+                          _ptr(kv_scales), C.byref(pl.handle), _ptr(workspace), workspace.numel(), _ptr(out),
+                          _ptr(lse), _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_run")
+    return out, lse
+
+
+def read_status(pl: Plan | None = None, workspace: torch.Tensor | None = None, stream=None) -> int:
+    """Synchronises the stream and returns the first device-side status (0 = ok)."""
+    lib = load_library()
+    return int(lib.dec_attn_read_status(None if pl is None else C.byref(pl.handle), _ptr(workspace),
+                                        _stream_handle(stream)))
+
+
+def plan_contents(pl: Plan) -> dict:
+    """Copies the work list back to the host (layout: the plan header of csrc/common.cuh)."""
+    import numpy as np
+    raw = pl.buf.cpu().numpy()
+    hdr = raw[:64].view(np.int32)
+    magic, status, n_bins, batch, hkv, tl, n_units, n_pairs = (int(x) for x in hdr[:8])
+    off_bin_off, off_pair_off, off_units = (int(x) for x in hdr[10:13])
+    bin_off = raw[off_bin_off:off_bin_off + 4 * (n_bins + 1)].view(np.int32).copy()
+    pair_off = raw[off_pair_off:off_pair_off + 4 * (n_pairs + 1)].view(np.int32).copy()
+    units = raw[off_units:off_units + 32 * n_units].view(np.int32).reshape(n_units, 8).copy()
+    return dict(magic=magic, status=status, n_bins=n_bins, n_units=n_units, tile_len=tl,
+                bin_off=bin_off, pair_off=pair_off, units=units)
+
+
+def sm_scale_default(head_dim: int) -> float:
+    return 1.0 / math.sqrt(head_dim)

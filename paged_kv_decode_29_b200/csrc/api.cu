@@ -1,0 +1,232 @@
+// api.cu -- the C ABI front end: argument checks, workspace layout, TMA tensor maps and
+// the launches of the split and combine kernels. See include/decattn.h for the contract.
+#include <math.h>
+
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "common.cuh"
+
+namespace decattn {
+
+static std::mutex g_mu;
+
+int default_bins(int device) {
+  static std::map<int, int> cache;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = cache.find(device);
+  if (it != cache.end()) return it->second;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0) return -1;
+  const int n = sms * split_ctas_per_sm();
+  cache[device] = n;
+  return n;
+}
+
+bool ensure_smem_attr(const void* kernel, int bytes) {
+  static std::map<std::pair<const void*, int>, int> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto key = std::make_pair(kernel, dev);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  done[key] = bytes;
+  return true;
+}
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// K or V pool viewed as a 2-D tensor: x = head_dim elements, y = (page * Hkv + h) * P + slot.
+// A box is 16 rows of 128 (or 64) bytes, swizzled to match the kernel's ldmatrix reads.
+static bool make_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int D, int64_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int esz = kv_dtype == DECATTN_KV_BF16 ? 2 : 1;
+  const int row_bytes = D * esz;
+  const int box_bytes = row_bytes >= 128 ? 128 : row_bytes;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)(box_bytes / esz), 16};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      kv_dtype == DECATTN_KV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapSwizzle sw = box_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct WsLayout {
+  int64_t off_part_lse, off_part_o, total;
+};
+
+static WsLayout ws_layout(int64_t max_units, int GT, int D) {
+  WsLayout w;
+  int64_t o = sizeof(WorkspaceHeader);
+  w.off_part_lse = o; o = align_up(o + 4 * max_units * GT, 256);
+  w.off_part_o = o; o = align_up(o + 4 * max_units * GT * D, 256);
+  w.total = o;
+  return w;
+}
+
+// Same layout arithmetic as dec_attn_plan (plan.cu).
+static void plan_offsets(const dec_attn_plan_t* pl, int64_t* off_bin_off, int64_t* off_pair_off,
+                         int64_t* off_units) {
+  int64_t o = sizeof(PlanHeader);
+  *off_bin_off = o; o = align_up(o + 4 * (int64_t)(pl->n_bins + 1), 32);
+  *off_pair_off = o; o = align_up(o + 4 * ((int64_t)pl->batch * pl->n_kv_heads + 1), 32);
+  *off_units = o;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static int check_shape(const dec_attn_shape* s, const dec_attn_plan_t* pl) {
+  if (!s || !pl) return DECATTN_EINVAL;
+  if (s->batch < 0 || s->n_q_heads <= 0 || s->n_kv_heads <= 0 || s->q_tokens <= 0 || s->page_size <= 0 ||
+      s->num_pages < 0 || s->max_pages_per_seq < 0 || s->head_dim <= 0)
+    return DECATTN_EINVAL;
+  if (s->n_q_heads % s->n_kv_heads != 0) return DECATTN_EINVAL;
+  if (pl->batch != s->batch || pl->n_kv_heads != s->n_kv_heads || pl->tile_len <= 0 || pl->n_bins <= 0 ||
+      pl->max_units < 0 || !pl->buf)
+    return DECATTN_EINVAL;
+  const int G = s->n_q_heads / s->n_kv_heads;
+  const int64_t GT = (int64_t)G * s->q_tokens;
+  if (s->head_dim != 64 && s->head_dim != 128) return DECATTN_ENOTSUP;
+  if (s->page_size % 16 != 0 || s->page_size > 256) return DECATTN_ENOTSUP;
+  if (pl->tile_len % s->page_size != 0) return DECATTN_ENOTSUP;
+  if (GT > 16 || !split_supported(s->kv_dtype, s->head_dim, (int)GT)) return DECATTN_ENOTSUP;
+  if ((int64_t)s->num_pages * s->n_kv_heads * s->page_size >= (1ll << 31)) return DECATTN_ENOTSUP;
+  if ((int64_t)s->batch * s->q_tokens * s->n_q_heads >= (1ll << 31)) return DECATTN_ENOTSUP;
+  return DECATTN_OK;
+}
+
+}  // namespace decattn
+
+using namespace decattn;
+
+extern "C" int dec_attn_default_bins(int device) { return default_bins(device); }
+
+extern "C" size_t dec_attn_workspace_bytes(const dec_attn_shape* shape, const dec_attn_plan_t* plan) {
+  if (check_shape(shape, plan) != DECATTN_OK) return 0;
+  const int GT = shape->n_q_heads / shape->n_kv_heads * shape->q_tokens;
+  return (size_t)ws_layout(plan->max_units, GT, shape->head_dim).total;
+}
+
+extern "C" int dec_attn_run(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
+                            const int32_t* page_table, const int32_t* seq_lens, const float* kv_scales,
+                            const dec_attn_plan_t* plan, void* workspace, size_t workspace_bytes, float* out,
+                            float* lse, void* stream) {
+  int rc = check_shape(shape, plan);
+  if (rc != DECATTN_OK) return rc;
+  const dec_attn_shape& s = *shape;
+  if (!workspace) return DECATTN_EINVAL;
+  if (s.batch == 0) return DECATTN_OK;
+  if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !out || !lse) return DECATTN_EINVAL;
+  if (s.kv_dtype == DECATTN_KV_FP8E4M3 && !kv_scales) return DECATTN_EINVAL;
+  if (s.num_pages <= 0 || s.max_pages_per_seq <= 0) return DECATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out) || !aligned16(workspace) ||
+      !aligned16(plan->buf))
+    return DECATTN_EALIGN;
+  if (((reinterpret_cast<uintptr_t>(page_table) | reinterpret_cast<uintptr_t>(seq_lens) |
+        reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(kv_scales)) & 3) != 0)
+    return DECATTN_EALIGN;
+  const int G = s.n_q_heads / s.n_kv_heads;
+  const int GT = G * s.q_tokens;
+  const int D = s.head_dim;
+  const WsLayout wl = ws_layout(plan->max_units, GT, D);
+  if ((int64_t)workspace_bytes < wl.total) return DECATTN_ESMALL;
+
+  CUtensorMap tmK, tmV;
+  const int64_t rows = (int64_t)s.num_pages * s.n_kv_heads * s.page_size;
+  if (!make_kv_map(&tmK, k_pages, s.kv_dtype, D, rows) || !make_kv_map(&tmV, v_pages, s.kv_dtype, D, rows))
+    return DECATTN_ECUDA;
+
+  int64_t off_bin_off, off_pair_off, off_units;
+  plan_offsets(plan, &off_bin_off, &off_pair_off, &off_units);
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess) return DECATTN_ECUDA;
+
+  const float scale = s.sm_scale > 0.f ? s.sm_scale : 1.0f / sqrtf((float)D);
+  SplitParams sp;
+  sp.q = static_cast<const uint16_t*>(q);
+  sp.page_table = page_table;
+  sp.kv_scales = kv_scales;
+  sp.plan = static_cast<const char*>(plan->buf);
+  sp.out = out;
+  sp.lse = lse;
+  sp.part_o = reinterpret_cast<float*>(ws + wl.off_part_o);
+  sp.part_lse = reinterpret_cast<float*>(ws + wl.off_part_lse);
+  sp.status = reinterpret_cast<int32_t*>(ws);
+  sp.B = s.batch; sp.T = s.q_tokens; sp.Hq = s.n_q_heads; sp.Hkv = s.n_kv_heads; sp.G = G; sp.GT = GT;
+  sp.P = s.page_size; sp.num_pages = s.num_pages; sp.mpps = s.max_pages_per_seq; sp.n_bins = plan->n_bins;
+  sp.off_bin_off = (int)off_bin_off;
+  sp.off_units = (int)off_units;
+  sp.qk_scale_log2 = scale * 1.4426950408889634f;
+  if (launch_split(sp, tmK, tmV, s.kv_dtype, D, st) != cudaSuccess) return DECATTN_ECUDA;
+
+  CombineParams cp;
+  cp.plan = sp.plan;
+  cp.seq_lens = seq_lens;
+  cp.part_o = sp.part_o;
+  cp.part_lse = sp.part_lse;
+  cp.out = out;
+  cp.lse = lse;
+  cp.T = s.q_tokens; cp.Hq = s.n_q_heads; cp.Hkv = s.n_kv_heads; cp.G = G; cp.GT = GT; cp.D = D;
+  cp.tl = plan->tile_len;
+  cp.off_pair_off = (int)off_pair_off;
+  if (launch_combine(cp, s.batch * s.q_tokens * s.n_q_heads, st) != cudaSuccess) return DECATTN_ECUDA;
+  return DECATTN_OK;
+}
+
+extern "C" int dec_attn_read_status(const dec_attn_plan_t* plan, const void* workspace, void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DECATTN_ECUDA;
+  if (plan && plan->buf) {
+    PlanHeader h;
+    if (cudaMemcpy(&h, plan->buf, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return DECATTN_ECUDA;
+    if (h.magic != kPlanMagic) return DECATTN_EINVAL;
+    if (h.status != DECATTN_OK) return h.status;
+  }
+  if (workspace) {
+    int32_t w = 0;
+    if (cudaMemcpy(&w, workspace, sizeof w, cudaMemcpyDeviceToHost) != cudaSuccess) return DECATTN_ECUDA;
+    if (w != DECATTN_OK) return w;
+  }
+  return DECATTN_OK;
+}
+
+extern "C" const char* dec_attn_status_string(int status) {
+  switch (status) {
+    case DECATTN_OK: return "ok";
+    case DECATTN_EINVAL: return "invalid argument";
+    case DECATTN_ENOTSUP: return "unsupported shape or dtype";
+    case DECATTN_ESMALL: return "buffer too small";
+    case DECATTN_ECUDA: return "CUDA runtime error";
+    case DECATTN_ETIMEOUT: return "device pipeline wait timed out";
+    case DECATTN_EDEVICE: return "device detected invalid input (page id, seq_len)";
+    case DECATTN_EALIGN: return "pointer not 16-byte aligned";
+    case DECATTN_ECAPACITY: return "more tiles than the plan can hold";
+    default: return "unknown status";
+  }
+}

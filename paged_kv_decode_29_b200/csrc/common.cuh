@@ -1,0 +1,265 @@
+// common.cuh -- device helpers shared by the planner, split and combine kernels
+// (sm_100a): mbarriers, TMA / bulk copies, ldmatrix, mma.sync, movmatrix,
+// bounded waits and the plan-buffer layout.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/decattn.h"
+
+namespace decattn {
+
+// ------------------------------------------------------------------ plan layout
+// The plan buffer starts with this header; the arrays follow at the byte offsets it
+// records. All offsets are multiples of 32.
+struct PlanHeader {
+  int32_t magic;        // kPlanMagic once the planner kernel has written the plan
+  int32_t status;       // DECATTN_OK or a negative device-detected status
+  int32_t n_bins;       // CTAs of the split kernel; bin k is run by CTA k
+  int32_t batch;
+  int32_t n_kv_heads;
+  int32_t tile_len;
+  int32_t n_units;      // tiles in the work list
+  int32_t n_pairs;      // batch * n_kv_heads
+  int64_t max_units;    // capacity of units[]
+  int32_t off_bin_off;  // int32 [n_bins + 1]: CSR offsets of each bin's tiles in units[]
+  int32_t off_pair_off; // int32 [n_pairs + 1]: first partial slot of each (b, h)
+  int32_t off_units;    // Unit [max_units]
+  int32_t off_scratch;  // planner scratch
+  int32_t reserved[2];
+};
+static_assert(sizeof(PlanHeader) == 64, "plan header is 64 bytes");
+constexpr int32_t kPlanMagic = 0x31504144;  // "DAP1"
+
+// One tile of the work list (32 bytes).
+struct Unit {
+  int32_t b, h, tok_begin, tok_end, seq_len, slot, tile, zero;
+};
+static_assert(sizeof(Unit) == 32, "unit is 32 bytes");
+
+// Workspace: a status word, then partial outputs and their LSEs.
+struct WorkspaceHeader {
+  int32_t status;
+  int32_t reserved[63];
+};
+static_assert(sizeof(WorkspaceHeader) == 256, "workspace header is 256 bytes");
+
+// Arguments of the split kernel (one CTA per bin of the plan).
+struct SplitParams {
+  const uint16_t* q;        // bf16 [B][T][Hq][D]
+  const int32_t* page_table;
+  const float* kv_scales;   // [2][num_pages][Hkv] or null
+  const char* plan;
+  float* out;               // [B][T][Hq][D]
+  float* lse;               // [B][T][Hq]
+  float* part_o;            // [max_units][GT][D]
+  float* part_lse;          // [max_units][GT]
+  int32_t* status;          // workspace status word
+  int B, T, Hq, Hkv, G, GT, P, num_pages, mpps, n_bins;
+  int off_bin_off, off_units;
+  float qk_scale_log2;      // sm_scale * log2(e)
+};
+
+// Arguments of the combine kernel (one CTA per query row).
+struct CombineParams {
+  const char* plan;
+  const int32_t* seq_lens;
+  const float* part_o;
+  const float* part_lse;
+  float* out;
+  float* lse;
+  int T, Hq, Hkv, G, GT, D, tl;
+  int off_pair_off;
+};
+
+__host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ status
+__device__ __forceinline__ void set_status(int32_t* st, int32_t code) {
+  if (st) atomicCAS(st, 0, code);
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// A pipeline wait gives up after this long; a healthy pipeline waits microseconds.
+constexpr uint64_t kWaitLimitNs = 2000ull * 1000 * 1000;
+
+// ------------------------------------------------------------------ shared-memory addresses
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ------------------------------------------------------------------ mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete. Returns false (after setting
+// DECATTN_ETIMEOUT) if it has not completed within kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    #pragma unroll 1
+    for (int i = 0; i < 256; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_status(status, DECATTN_ETIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Lane 0 waits and tells the rest of the warp (used where only lane 0 touches the staged
+// data afterwards, e.g. the thread that issues the next copy into a freed stage).
+__device__ __forceinline__ bool warp_wait_lane0(uint64_t* bar, uint32_t parity, int32_t* status) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// ------------------------------------------------------------------ async copies
+// 2-D tiled TMA load into shared memory, completion signalled on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Plain bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// 4-byte asynchronous copy global -> shared (LDGSTS) ...
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// ... whose completion is folded into an mbarrier phase: the pending count is raised now
+// and lowered when this thread's earlier cp.async copies have landed.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------------ warp-level matrix ops
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+// D (16x8 fp32) += A (16x16) * B (16x8); bf16 or f16 operands, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Two OCP E4M3 codes sitting in bytes 1 and 3 of x -> f16x2 holding code * 2^-8 each
+// (low half from byte 1, high half from byte 3); bytes 0 and 2 are ignored.
+// An E4M3 code s.eeee.mmm and the f16 s.0eeee.mmm0000000 have the same sign, exponent
+// field and mantissa bits; the exponent biases (7 vs 15) differ by 8, so the f16 value
+// is exactly code * 2^-8, subnormals included (both formats read exponent field 0 as
+// 2^(1-bias) with no implicit bit). The 2^8 goes into the per-page scale.
+__device__ __forceinline__ uint32_t e4m3x2_hi_bytes_to_f16x2(uint32_t x) {
+  return (x & 0x80008000u) | ((x >> 1) & 0x3F803F80u);
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ------------------------------------------------------------------ host-side launchers
+int default_bins(int device);                                     // api.cu
+bool ensure_smem_attr(const void* kernel, int bytes);             // api.cu
+bool split_supported(int kv_dtype, int D, int GT);                // split.cu
+cudaError_t launch_split(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int kv_dtype,
+                         int D, cudaStream_t st);                 // split.cu
+int split_ctas_per_sm();                                          // split.cu
+cudaError_t launch_combine(const CombineParams& p, int rows, cudaStream_t st);  // combine.cu
+
+}  // namespace decattn

@@ -1,0 +1,531 @@
+// split.cu -- the split kernel: one persistent CTA per bin of the plan; it walks its
+// tiles, streams the page-table-indirected K/V rows of each tile through a shared-memory
+// ring filled by TMA, and computes the tile's partial attention for the G*T query rows
+// of its KV head.
+//
+// Method ("PaddlePaddle/HALOps" README, Highlights, GQA attention item: paged-KV decode,
+// BF16/FP8 KV, GQA, speculative decoding, split-KV; "HPC-Ops: Tencent's CUDA Kernel
+// Library for LLM Inference Hot Paths", "How the kernels are organized around specific
+// workload shapes": uniform tiles balanced across CTAs, a combine merges the splits).
+//
+// CTA = 2 warps.
+//  * warp 0 (producer): reads the bin's tile list and page-table rows, and for every
+//    16-key block issues two 2-D TMA copies (K rows, V rows) of one (page, KV head) into
+//    the next ring stage; the tile's q rows go to a double-buffered q slot by bulk copy;
+//    FP8 page scales ride along as 4-byte cp.async copies folded into the stage's
+//    mbarrier. It waits only on "stage empty" barriers, so it runs ahead of the math.
+//  * warp 1 (consumer): per 16-key block, S^T = K Q^T on tensor cores with the keys on
+//    the MMA's M side ("SwapAB", as in the pages' Attention SwapAB), so a G*T of 4..16
+//    query rows fills N = 8 or 16 instead of padding M to 16; then an online softmax in
+//    fp32 (log2 domain), then O^T += V^T P^T (again keys as the contraction, head_dim on
+//    M). Probabilities go to the MMA as bf16 hi + bf16 lo (BF16 KV: two columns of the
+//    same MMA when G*T <= 4, two N tiles otherwise), or as f16 scaled by the page's V
+//    scale (FP8 KV).
+//  * the tile ends with either the final output (the tile covers its whole request) or
+//    a normalised partial (o, lse) in the workspace for the combine kernel.
+//
+// Shared-memory staging uses the TMA 128-byte (or 64-byte) swizzle, so every ldmatrix
+// below reads 8 distinct 16-byte bank groups.
+#include "common.cuh"
+
+namespace decattn {
+
+
+constexpr int kSplitThreads = 64;
+constexpr int kCtasPerSm = 4;
+
+template <int KVT, int D>
+struct Geo {
+  static constexpr int ESZ = KVT == 0 ? 2 : 1;                  // bytes per KV element
+  static constexpr int ROW = D * ESZ;                           // bytes of one key row
+  static constexpr int RB = ROW >= 128 ? 128 : ROW;             // bytes of one TMA box row
+  static constexpr int CPB = RB / 16;                           // 16-byte chunks per box row
+  static constexpr int NBOX = ROW / RB;                         // boxes per 16-row block
+  static constexpr int BOX_ELEMS = RB / ESZ;
+  static constexpr int BOX_BYTES = 16 * RB;
+  static constexpr int TILE = 16 * ROW;                         // K (or V) bytes per stage
+  static constexpr int STAGES = (40 * 1024) / (2 * TILE);
+  static_assert(RB == 128 || RB == 64, "box rows are 64 or 128 bytes");
+  // byte offset of (row r, 16-byte chunk cg of the full row) in a stage buffer
+  __device__ static __forceinline__ uint32_t off(int r, int cg) {
+    const int box = cg / CPB, c = cg % CPB;
+    const int sw = RB == 128 ? (c ^ (r & 7)) : (c ^ ((r >> 1) & 3));
+    return (uint32_t)(box * BOX_BYTES + r * RB + (sw << 4));
+  }
+};
+
+template <int KVT, int D, int NQ>
+struct Smem {
+  using G_ = Geo<KVT, D>;
+  static constexpr int QBYTES = 8 * NQ * D * 2;
+  static constexpr int OFF_Q = G_::STAGES * 2 * G_::TILE;
+  static constexpr int OFF_BAR = OFF_Q + 2 * QBYTES;
+  static constexpr int NBAR = 2 * G_::STAGES + 4;
+  static constexpr int OFF_META = OFF_BAR + 8 * NBAR;            // per stage: pad, K scale, V scale, pad
+  static constexpr int OFF_QMETA = OFF_META + 16 * G_::STAGES;   // Unit x 2
+  static constexpr int BYTES = OFF_QMETA + 2 * (int)sizeof(Unit);
+  static constexpr int ALLOC = BYTES + 1024;                     // slack to align the base to 1024
+};
+
+// Row of the staged q slot feeding MMA column n, or -1 for a zero column.
+template <bool DUP>
+__device__ __forceinline__ int qrow_of_col(int n, int GT) {
+  if (DUP) {
+    const int r = n & 3;  // columns 4..7 repeat rows 0..3 (they carry the low bf16 half of P)
+    return r < GT ? r : -1;
+  }
+  return n < GT ? n : -1;
+}
+
+// KVT: 0 = bf16 KV, 1 = FP8 E4M3 KV.  NQ: 8-column tiles of S^T.  NPV: 8-column tiles of
+// O^T.  DUP: bf16 with G*T <= 4 (hi in columns 0..3, lo in 4..7 of one tile).
+template <int KVT, int D, int NQ, int NPV, bool DUP>
+__global__ void __launch_bounds__(kSplitThreads, kCtasPerSm)
+split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+  using G_ = Geo<KVT, D>;
+  using S_ = Smem<KVT, D, NQ>;
+  constexpr int STAGES = G_::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_::OFF_BAR);
+  uint64_t* full = bar;
+  uint64_t* empty = bar + STAGES;
+  uint64_t* qfull = bar + 2 * STAGES;
+  uint64_t* qempty = bar + 2 * STAGES + 2;
+  float* meta_sc = reinterpret_cast<float*>(sm + S_::OFF_META);      // [s*4 + 1] = K scale, [s*4 + 2] = V scale
+  Unit* qmeta = reinterpret_cast<Unit*>(sm + S_::OFF_QMETA);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
+  if (hdr->magic != kPlanMagic || hdr->status != DECATTN_OK || hdr->n_bins != (int)gridDim.x ||
+      hdr->batch != p.B || hdr->n_kv_heads != p.Hkv) {
+    if (threadIdx.x == 0 && blockIdx.x == 0)
+      set_status(p.status, hdr->magic != kPlanMagic ? DECATTN_EINVAL
+                           : hdr->status != DECATTN_OK ? hdr->status : DECATTN_EINVAL);
+    return;
+  }
+  const int32_t* bin_off = reinterpret_cast<const int32_t*>(p.plan + p.off_bin_off);
+  const Unit* units = reinterpret_cast<const Unit*>(p.plan + p.off_units);
+  const int u0 = bin_off[blockIdx.x], u1 = bin_off[blockIdx.x + 1];
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 32); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 32); }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (u0 >= u1) return;
+
+  if (warp == 0) {
+    // ===================================================================== producer
+    if (lane == 0) { prefetch_tensormap(&tmK); prefetch_tensormap(&tmV); }
+    const int P = p.P, kb_per_page = P / 16;
+    int s = 0; uint32_t eph = 1;
+    int qs = 0; uint32_t qeph = 1;
+    bool ok = true;
+    int64_t n_fill = 0, n_qfill = 0;  // copies issued so far (ring stages, q slots)
+    // tile descriptors run two tiles ahead and page ids one tile ahead of the copies
+    Unit dn = units[u0];
+    Unit dnn = u0 + 1 < u1 ? units[u0 + 1] : dn;
+    int pid_next;
+    {
+      const int pg0 = dn.tok_begin / P, npg = (dn.tok_end - dn.tok_begin + P - 1) / P;
+      pid_next = lane < npg ? p.page_table[(int64_t)dn.b * p.mpps + min(pg0 + lane, p.mpps - 1)] : 0;
+    }
+    for (int u = u0; u < u1 && ok; ++u) {
+      const Unit d = dn;
+      int pid_l = pid_next;
+      dn = dnn;
+      if (u + 2 < u1) dnn = units[u + 2];
+      if (u + 1 < u1) {
+        const int pg0 = dn.tok_begin / P, npg = (dn.tok_end - dn.tok_begin + P - 1) / P;
+        pid_next = lane < npg ? p.page_table[(int64_t)dn.b * p.mpps + min(pg0 + lane, p.mpps - 1)] : 0;
+      }
+      // q rows of this tile: T bulk copies of G consecutive heads each
+      if (!warp_wait_lane0(&qempty[qs], qeph, p.status)) { ok = false; break; }
+      if (lane == 0) {
+        qmeta[qs] = d;
+        const uint32_t bytes = (uint32_t)(p.G * D * 2);
+        mbar_arrive_expect_tx(&qfull[qs], bytes * p.T);
+        uint8_t* dst = sm + S_::OFF_Q + qs * S_::QBYTES;
+        for (int t = 0; t < p.T; ++t)
+          bulk_load(dst + t * bytes, p.q + (((int64_t)d.b * p.T + t) * p.Hq + (int64_t)d.h * p.G) * D, bytes,
+                    &qfull[qs]);
+      }
+      ++n_qfill;
+      qs ^= 1; if (qs == 0) qeph ^= 1;
+      const int pg0 = d.tok_begin / P;
+      const int npg = (d.tok_end - d.tok_begin + P - 1) / P;
+      if (lane == 0 && pg0 + npg > p.mpps) set_status(p.status, DECATTN_EDEVICE);  // row too short
+      for (int c0 = 0; c0 < npg && ok; c0 += 32) {
+        if (c0 > 0)
+          pid_l = c0 + lane < npg ? p.page_table[(int64_t)d.b * p.mpps + min(pg0 + c0 + lane, p.mpps - 1)] : 0;
+        if (c0 + lane < npg && (pid_l < 0 || pid_l >= p.num_pages)) {
+          set_status(p.status, DECATTN_EDEVICE);
+          pid_l = 0;  // keeps the copy inside the pool; the result is flagged invalid
+        }
+        const int n_here = min(32, npg - c0);
+        for (int i = 0; i < n_here && ok; ++i) {
+          const int pid = __shfl_sync(0xffffffffu, pid_l, i);
+          const int ip = c0 + i;
+          for (int kb = 0; kb < kb_per_page; ++kb) {
+            const int tok = d.tok_begin + ip * P + kb * 16;
+            if (tok >= d.tok_end) break;
+            if (!warp_wait_lane0(&empty[s], eph, p.status)) { ok = false; break; }
+            if (lane == 0) {
+              if (KVT == 1) {
+                const int64_t si = (int64_t)pid * p.Hkv + d.h;
+                cp_async_4(&meta_sc[s * 4 + 1], p.kv_scales + si);
+                cp_async_4(&meta_sc[s * 4 + 2], p.kv_scales + (int64_t)p.num_pages * p.Hkv + si);
+                cp_async_mbar_arrive(&full[s]);
+              }
+              mbar_arrive_expect_tx(&full[s], 2 * G_::TILE);
+              const int row = (pid * p.Hkv + d.h) * P + kb * 16;
+              uint8_t* ks = sm + s * 2 * G_::TILE;
+              #pragma unroll
+              for (int bx = 0; bx < G_::NBOX; ++bx) {
+                tma_load_2d(ks + bx * G_::BOX_BYTES, &tmK, bx * G_::BOX_ELEMS, row, &full[s]);
+                tma_load_2d(ks + G_::TILE + bx * G_::BOX_BYTES, &tmV, bx * G_::BOX_ELEMS, row, &full[s]);
+              }
+            }
+            ++n_fill;
+            if (++s == STAGES) { s = 0; eph ^= 1; }
+          }
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      // a wait gave up: let the copies already issued land before the CTA exits. Fill n of
+      // ring stage n % STAGES completes phase (n / STAGES) & 1 of its barrier.
+      for (int64_t n = n_fill > STAGES ? n_fill - STAGES : 0; n < n_fill; ++n)
+        mbar_wait(&full[n % STAGES], (uint32_t)((n / STAGES) & 1), nullptr);
+      for (int64_t n = n_qfill > 2 ? n_qfill - 2 : 0; n < n_qfill; ++n)
+        mbar_wait(&qfull[n % 2], (uint32_t)((n / 2) & 1), nullptr);
+    }
+    return;
+  }
+
+  // ======================================================================= consumer
+  const int gid = lane >> 2, tig = lane & 3;
+  int s = 0; uint32_t fph = 0;
+  int qs = 0; uint32_t qfph = 0;
+  const float LN2 = 0.6931471805599453f;
+  for (int u = u0; u < u1; ++u) {
+    if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qs], qfph, p.status))) return;
+    const Unit d = qmeta[qs];
+    // ---- q fragments (B operand of S^T = K Q^T): column n = query row
+    uint32_t qf[NQ][D / 16][2];
+    {
+      const uint8_t* qsm = sm + S_::OFF_Q + qs * S_::QBYTES;
+      #pragma unroll
+      for (int nq = 0; nq < NQ; ++nq) {
+        const int r = qrow_of_col<DUP>(8 * nq + gid, p.GT);
+        const uint16_t* qr = reinterpret_cast<const uint16_t*>(qsm) + (r < 0 ? 0 : r) * D;
+        #pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          if (KVT == 0) {
+            const uint32_t x0 = *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * tig);
+            const uint32_t x1 = *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 8 + 2 * tig);
+            qf[nq][kk][0] = r < 0 ? 0u : x0;
+            qf[nq][kk][1] = r < 0 ? 0u : x1;
+          } else {
+            // FP8 K is read 4 consecutive codes per thread: logical k = 2*tig + {0,1} holds
+            // d = 16kk + 4tig + {0,1}, logical k = 8 + 2*tig + {0,1} holds d = 16kk + 4tig + {2,3}
+            const uint2 x = *reinterpret_cast<const uint2*>(qr + 16 * kk + 4 * tig);
+            qf[nq][kk][0] = r < 0 ? 0u : pack_f16(bf16_lo(x.x), bf16_hi(x.x));
+            qf[nq][kk][1] = r < 0 ? 0u : pack_f16(bf16_lo(x.y), bf16_hi(x.y));
+          }
+        }
+      }
+    }
+    __syncwarp();
+    mbar_arrive(&qempty[qs]);
+    qs ^= 1; if (qs == 0) qfph ^= 1;
+
+    // ---- per-column limits: key j is visible to query token t if j <= Lb - T + t
+    int lim[NQ][2];
+    #pragma unroll
+    for (int nq = 0; nq < NQ; ++nq)
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int r = qrow_of_col<DUP>(8 * nq + 2 * tig + e, p.GT);
+        lim[nq][e] = r < 0 ? 0x7fffffff : d.seq_len - p.T + r / p.G;
+      }
+    int lim_min = 0x7fffffff;
+    #pragma unroll
+    for (int nq = 0; nq < NQ; ++nq) lim_min = min(lim_min, min(lim[nq][0], lim[nq][1]));
+    lim_min = __reduce_min_sync(0xffffffffu, lim_min);
+    const int safe_end = min(d.tok_end, lim_min + 1);  // keys below this need no mask
+
+    float o[NPV][D / 16][4];
+    #pragma unroll
+    for (int j = 0; j < NPV; ++j)
+      #pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) o[j][mt][0] = o[j][mt][1] = o[j][mt][2] = o[j][mt][3] = 0.f;
+    float mrow[NQ][2], lrow[NQ][2];
+    #pragma unroll
+    for (int nq = 0; nq < NQ; ++nq) mrow[nq][0] = mrow[nq][1] = -INFINITY, lrow[nq][0] = lrow[nq][1] = 0.f;
+
+    const int nkb = (d.tok_end - d.tok_begin + 15) / 16;
+    for (int kbi = 0; kbi < nkb; ++kbi) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], fph, p.status))) return;
+      const int kbase = d.tok_begin + 16 * kbi;
+      const uint32_t ks = smem_u32(sm + s * 2 * G_::TILE);
+      const uint32_t vs = ks + G_::TILE;
+      float sc2 = p.qk_scale_log2, vsc = 1.f;
+      if (KVT == 1) {
+        sc2 *= meta_sc[s * 4 + 1] * 256.f;
+        vsc = meta_sc[s * 4 + 2] * 256.f;
+      }
+      // ---- S^T = K Q^T  (rows: 16 keys; columns: query rows)
+      float sacc[NQ][4];
+      #pragma unroll
+      for (int nq = 0; nq < NQ; ++nq) sacc[nq][0] = sacc[nq][1] = sacc[nq][2] = sacc[nq][3] = 0.f;
+      {
+        const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
+        if (KVT == 0) {
+          #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t a[4];
+            ldsm_x4(ks + G_::off(r, 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
+            #pragma unroll
+            for (int nq = 0; nq < NQ; ++nq) mma_bf16(sacc[nq], a, qf[nq][kk][0], qf[nq][kk][1]);
+          }
+        } else {
+          #pragma unroll
+          for (int k2 = 0; k2 < D / 32; ++k2) {
+            uint32_t R[4];
+            ldsm_x4(ks + G_::off(r, 2 * k2 + (lane >> 4)), R[0], R[1], R[2], R[3]);
+            #pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              uint32_t a[4];
+              a[0] = e4m3x2_hi_bytes_to_f16x2(prmt(R[2 * h2], 0, 0x1100));
+              a[2] = e4m3x2_hi_bytes_to_f16x2(prmt(R[2 * h2], 0, 0x3322));
+              a[1] = e4m3x2_hi_bytes_to_f16x2(prmt(R[2 * h2 + 1], 0, 0x1100));
+              a[3] = e4m3x2_hi_bytes_to_f16x2(prmt(R[2 * h2 + 1], 0, 0x3322));
+              #pragma unroll
+              for (int nq = 0; nq < NQ; ++nq) mma_f16(sacc[nq], a, qf[nq][2 * k2 + h2][0], qf[nq][2 * k2 + h2][1]);
+            }
+          }
+        }
+      }
+      // ---- scale, mask, online softmax (log2 domain, fp32 state)
+      const bool need_mask = kbase + 16 > safe_end;
+      bool grew = false;
+      float alpha[NQ][2];
+      float pv[NQ][4];
+      #pragma unroll
+      for (int nq = 0; nq < NQ; ++nq) {
+        float sv4[4];
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          sv4[i] = sacc[nq][i] * sc2;
+          if (need_mask) {
+            const int j = kbase + gid + (i >> 1) * 8;
+            if (j >= d.tok_end || j > lim[nq][i & 1]) sv4[i] = -INFINITY;
+          }
+        }
+        #pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float mx = fmaxf(sv4[e], sv4[e + 2]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float mnew = fmaxf(mrow[nq][e], mx);
+          grew |= mnew > mrow[nq][e];
+          const float muse = mnew == -INFINITY ? 0.f : mnew;
+          alpha[nq][e] = fast_exp2(mrow[nq][e] - muse);
+          pv[nq][e] = fast_exp2(sv4[e] - muse);
+          pv[nq][e + 2] = fast_exp2(sv4[e + 2] - muse);
+          lrow[nq][e] = lrow[nq][e] * alpha[nq][e] + pv[nq][e] + pv[nq][e + 2];
+          mrow[nq][e] = mnew;
+        }
+      }
+      if (__any_sync(0xffffffffu, grew)) {
+        #pragma unroll
+        for (int j = 0; j < NPV; ++j) {
+          const int nq = (KVT == 0 && !DUP) ? j / 2 : j;
+          #pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt) {
+            o[j][mt][0] *= alpha[nq][0]; o[j][mt][1] *= alpha[nq][1];
+            o[j][mt][2] *= alpha[nq][0]; o[j][mt][3] *= alpha[nq][1];
+          }
+        }
+      }
+      // ---- P^T as B fragments: C-fragment rows (keys) become the K index via movmatrix
+      uint32_t bp[NPV][2];
+      #pragma unroll
+      for (int nq = 0; nq < NQ; ++nq) {
+        if (KVT == 1) {
+          bp[nq][0] = movmatrix_t(pack_f16(pv[nq][0] * vsc, pv[nq][1] * vsc));
+          bp[nq][1] = movmatrix_t(pack_f16(pv[nq][2] * vsc, pv[nq][3] * vsc));
+        } else {
+          const uint32_t h01 = pack_bf16(pv[nq][0], pv[nq][1]);
+          const uint32_t h23 = pack_bf16(pv[nq][2], pv[nq][3]);
+          const uint32_t l01 = pack_bf16(pv[nq][0] - bf16_lo(h01), pv[nq][1] - bf16_hi(h01));
+          const uint32_t l23 = pack_bf16(pv[nq][2] - bf16_lo(h23), pv[nq][3] - bf16_hi(h23));
+          if (DUP) {
+            const bool lo_lane = tig >= 2;  // columns 4..7 carry the low halves
+            bp[0][0] = movmatrix_t(lo_lane ? l01 : h01);
+            bp[0][1] = movmatrix_t(lo_lane ? l23 : h23);
+          } else {
+            bp[2 * nq][0] = movmatrix_t(h01);
+            bp[2 * nq][1] = movmatrix_t(h23);
+            bp[2 * nq + 1][0] = movmatrix_t(l01);
+            bp[2 * nq + 1][1] = movmatrix_t(l23);
+          }
+        }
+      }
+      // ---- O^T += V^T P^T  (rows: head_dim; contraction: the 16 keys)
+      if (KVT == 0) {
+        const int q4 = lane >> 3;
+        const int r = (lane & 7) + (q4 >> 1) * 8;
+        #pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          uint32_t a[4];
+          ldsm_x4_t(vs + G_::off(r, 2 * mt + (q4 & 1)), a[0], a[1], a[2], a[3]);
+          #pragma unroll
+          for (int j = 0; j < NPV; ++j) mma_bf16(o[j][mt], a, bp[j][0], bp[j][1]);
+        }
+      } else {
+        // thread (gid, tig) reads 4 codes at d = 32pp + 4gid .. +3 of keys 2tig, 2tig+1,
+        // 2tig+8, 2tig+9 and pairs them by key: M-row gid of m-tile 2pp+sub is
+        // d = 32pp + 4gid + 2sub, M-row gid+8 is d + 1.
+        #pragma unroll
+        for (int pp = 0; pp < D / 32; ++pp) {
+          const int cg = 2 * pp + (gid >> 2), inb = (4 * gid) & 15;
+          const uint8_t* vb = sm + s * 2 * G_::TILE + G_::TILE;
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vb + G_::off(2 * tig, cg) + inb);
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(vb + G_::off(2 * tig + 1, cg) + inb);
+          const uint32_t w2 = *reinterpret_cast<const uint32_t*>(vb + G_::off(2 * tig + 8, cg) + inb);
+          const uint32_t w3 = *reinterpret_cast<const uint32_t*>(vb + G_::off(2 * tig + 9, cg) + inb);
+          #pragma unroll
+          for (int sub = 0; sub < 2; ++sub) {
+            const uint32_t sel0 = ((4 + 2 * sub) << 12) | ((4 + 2 * sub) << 8) | ((2 * sub) << 4) | (2 * sub);
+            const uint32_t sel1 = sel0 + 0x1111;
+            uint32_t a[4];
+            a[0] = e4m3x2_hi_bytes_to_f16x2(prmt(w0, w1, sel0));
+            a[1] = e4m3x2_hi_bytes_to_f16x2(prmt(w0, w1, sel1));
+            a[2] = e4m3x2_hi_bytes_to_f16x2(prmt(w2, w3, sel0));
+            a[3] = e4m3x2_hi_bytes_to_f16x2(prmt(w2, w3, sel1));
+            #pragma unroll
+            for (int j = 0; j < NPV; ++j) mma_f16(o[j][2 * pp + sub], a, bp[j][0], bp[j][1]);
+          }
+        }
+      }
+      __syncwarp();
+      mbar_arrive(&empty[s]);
+      if (++s == STAGES) { s = 0; fph ^= 1; }
+    }
+
+    // ---- epilogue: row sums, hi + lo, normalise, store
+    #pragma unroll
+    for (int nq = 0; nq < NQ; ++nq)
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float l = lrow[nq][e];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        lrow[nq][e] = l;
+      }
+    if (KVT == 0) {
+      if (DUP) {
+        #pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt)
+          #pragma unroll
+          for (int i = 0; i < 4; ++i) o[0][mt][i] += __shfl_xor_sync(0xffffffffu, o[0][mt][i], 2);
+      } else {
+        #pragma unroll
+        for (int nq = 0; nq < NQ; ++nq)
+          #pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt)
+            #pragma unroll
+            for (int i = 0; i < 4; ++i) o[2 * nq][mt][i] += o[2 * nq + 1][mt][i];
+      }
+    }
+    #pragma unroll
+    for (int nq = 0; nq < NQ; ++nq) {
+      const int j = (KVT == 0 && !DUP) ? 2 * nq : nq;
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int n = 8 * nq + 2 * tig + e;
+        if (DUP && n >= 4) continue;
+        const int r = n < p.GT ? n : -1;
+        if (r < 0) continue;
+        const float l = lrow[nq][e];
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float lse_v = l > 0.f ? (mrow[nq][e] + __log2f(l)) * LN2 : -INFINITY;
+        const int t = r / p.G, g = r % p.G;
+        float* dst;
+        float* dst_lse;
+        if (d.slot < 0) {
+          const int64_t row = ((int64_t)d.b * p.T + t) * p.Hq + (int64_t)d.h * p.G + g;
+          dst = p.out + row * D;
+          dst_lse = p.lse + row;
+        } else {
+          const int64_t row = (int64_t)d.slot * p.GT + r;
+          dst = p.part_o + row * D;
+          dst_lse = p.part_lse + row;
+        }
+        if (KVT == 0) {
+          #pragma unroll
+          for (int mt = 0; mt < D / 16; ++mt) {
+            dst[16 * mt + gid] = o[j][mt][e] * inv;
+            dst[16 * mt + gid + 8] = o[j][mt][2 + e] * inv;
+          }
+        } else {
+          #pragma unroll
+          for (int pp = 0; pp < D / 32; ++pp) {
+            float4 v;
+            v.x = o[j][2 * pp][e] * inv;
+            v.y = o[j][2 * pp][2 + e] * inv;
+            v.z = o[j][2 * pp + 1][e] * inv;
+            v.w = o[j][2 * pp + 1][2 + e] * inv;
+            *reinterpret_cast<float4*>(dst + 32 * pp + 4 * gid) = v;
+          }
+        }
+        if (gid == 0) *dst_lse = lse_v;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+template <int KVT, int D, int NQ, int NPV, bool DUP>
+static cudaError_t launch_variant(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                                  cudaStream_t st) {
+  auto fn = split_kernel<KVT, D, NQ, NPV, DUP>;
+  const int smem = Smem<KVT, D, NQ>::ALLOC;
+  if (!ensure_smem_attr((const void*)fn, smem)) return cudaErrorInvalidValue;
+  fn<<<p.n_bins, kSplitThreads, smem, st>>>(p, tmK, tmV);
+  return cudaGetLastError();
+}
+
+template <int KVT, int D>
+static cudaError_t launch_gt(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st) {
+  if constexpr (KVT == 0) {
+    if (p.GT <= 4) return launch_variant<KVT, D, 1, 1, true>(p, tmK, tmV, st);
+    if (p.GT <= 8) return launch_variant<KVT, D, 1, 2, false>(p, tmK, tmV, st);
+    return launch_variant<KVT, D, 2, 4, false>(p, tmK, tmV, st);
+  } else {
+    if (p.GT <= 8) return launch_variant<KVT, D, 1, 1, false>(p, tmK, tmV, st);
+    return launch_variant<KVT, D, 2, 2, false>(p, tmK, tmV, st);
+  }
+}
+
+bool split_supported(int kv_dtype, int D, int GT) {
+  return GT >= 1 && GT <= 16 && (D == 64 || D == 128) &&
+         (kv_dtype == DECATTN_KV_BF16 || kv_dtype == DECATTN_KV_FP8E4M3);
+}
+
+cudaError_t launch_split(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int kv_dtype, int D,
+                         cudaStream_t st) {
+  if (!split_supported(kv_dtype, D, p.GT)) return cudaErrorInvalidValue;
+  if (kv_dtype == DECATTN_KV_BF16) return D == 128 ? launch_gt<0, 128>(p, tmK, tmV, st) : launch_gt<0, 64>(p, tmK, tmV, st);
+  return D == 128 ? launch_gt<1, 128>(p, tmK, tmV, st) : launch_gt<1, 64>(p, tmK, tmV, st);
+}
+
+int split_ctas_per_sm() { return kCtasPerSm; }
+
+}  // namespace decattn

@@ -1,0 +1,123 @@
+"""The C ABI without a GPU: the library loads, exports exactly what include/decattn.h
+declares, and rejects bad arguments on the host before anything is enqueued."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+import paged_kv_decode_29_b200 as da
+from paged_kv_decode_29_b200 import build as dbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "decattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dbuild.build()
+    return da.load_library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"DECATTN_API\s+[\w\s\*]*?\b(dec_attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_api():
+    assert declared_symbols() == sorted(da.API)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", da.LIB_PATH]).decode()
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    for sym in declared_symbols():
+        assert sym in exported, sym
+        assert getattr(lib, sym) is not None
+    # nothing else leaks out of the library as a public function
+    assert {s for s in exported if s.startswith("dec_attn")} == set(declared_symbols())
+
+
+def test_status_strings(lib):
+    for code in (da.OK, da.EINVAL, da.ENOTSUP, da.ESMALL, da.ECUDA, da.ETIMEOUT, da.EDEVICE, da.EALIGN,
+                 da.ECAPACITY):
+        s = da.status_string(code)
+        assert s and s != "unknown status"
+    assert da.status_string(12345) == "unknown status"
+
+
+def test_plan_bytes_host_only(lib):
+    n = lib.dec_attn_plan_bytes(32, 8, 256, 32 * 4096, 592)
+    assert n > 32 * 4096 // 256 * 8 * 32  # holds the tile list
+    assert lib.dec_attn_plan_bytes(32, 8, 250, 1000, 592) == 0      # tile not a multiple of 16
+    assert lib.dec_attn_plan_bytes(-1, 8, 256, 1000, 592) == 0
+    assert lib.dec_attn_plan_bytes(4, 0, 256, 1000, 592) == 0
+    assert lib.dec_attn_plan_bytes(4, 8, 256, 1000, 100000) == 0     # too many bins
+
+
+def _shape(**kw):
+    base = dict(batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, q_tokens=1, page_size=16, num_pages=64,
+                max_pages_per_seq=8, kv_dtype=da.KV_BF16, sm_scale=0.0)
+    base.update(kw)
+    return da.ShapeT(*[base[f] for f, _ in da.ShapeT._fields_])
+
+
+def _plan(**kw):
+    base = dict(buf=0x10000, buf_bytes=1 << 20, batch=2, n_kv_heads=2, tile_len=64, n_bins=8, max_units=64)
+    base.update(kw)
+    return da.PlanT(*[base[f] for f, _ in da.PlanT._fields_])
+
+
+FAKE = 0x7f0000000000  # never dereferenced: every case below fails a host check first
+
+
+def _run(lib, shape, plan, q=FAKE, k=FAKE, v=FAKE, tab=FAKE, lens=FAKE, sc=None, ws=FAKE, ws_bytes=1 << 30,
+         out=FAKE, lse=FAKE):
+    return lib.dec_attn_run(C.byref(shape), q, k, v, tab, lens, sc, C.byref(plan), ws, ws_bytes, out, lse, None)
+
+
+@pytest.mark.parametrize("shape_kw,plan_kw,code", [
+    (dict(head_dim=96), {}, da.ENOTSUP),
+    (dict(head_dim=256), {}, da.ENOTSUP),
+    (dict(page_size=8), {}, da.ENOTSUP),
+    (dict(page_size=48), dict(tile_len=64), da.ENOTSUP),       # tile not a multiple of the page
+    (dict(n_q_heads=64, n_kv_heads=2, q_tokens=1), {}, da.ENOTSUP),   # G*T = 32
+    (dict(q_tokens=5, n_q_heads=8, n_kv_heads=2), {}, da.ENOTSUP),   # G*T = 20
+    (dict(kv_dtype=7), {}, da.ENOTSUP),
+    (dict(n_q_heads=6, n_kv_heads=4), dict(n_kv_heads=4), da.EINVAL),
+    (dict(batch=3), {}, da.EINVAL),                             # plan made for another batch
+    (dict(q_tokens=0), {}, da.EINVAL),
+])
+def test_run_rejects_bad_shapes(lib, shape_kw, plan_kw, code):
+    assert _run(lib, _shape(**shape_kw), _plan(**plan_kw)) == code
+
+
+def test_run_rejects_null_and_misaligned(lib):
+    s, p = _shape(), _plan()
+    assert _run(lib, s, p, q=None) == da.EINVAL
+    assert _run(lib, s, p, ws=None) == da.EINVAL
+    assert _run(lib, _shape(kv_dtype=da.KV_FP8E4M3), p, sc=None) == da.EINVAL
+    assert _run(lib, s, p, q=FAKE + 8) == da.EALIGN
+    assert _run(lib, s, p, k=FAKE + 4) == da.EALIGN
+    assert _run(lib, s, p, lse=FAKE + 2) == da.EALIGN
+
+
+def test_run_rejects_small_workspace(lib):
+    s, p = _shape(), _plan()
+    need = lib.dec_attn_workspace_bytes(C.byref(s), C.byref(p))
+    assert need > 0
+    assert _run(lib, s, p, ws_bytes=need - 1) == da.ESMALL
+
+
+def test_empty_batch_is_a_no_op(lib):
+    assert _run(lib, _shape(batch=0), _plan(batch=0), q=None, k=None, v=None) == da.OK
+
+
+def test_plan_rejects_bad_args(lib):
+    h = da.PlanT()
+    assert lib.dec_attn_plan(FAKE, 2, 2, 64, 1000, 8, None, 1 << 20, C.byref(h), None) == da.EINVAL
+    assert lib.dec_attn_plan(FAKE, 2, 2, 64, 1000, 8, FAKE + 8, 1 << 20, C.byref(h), None) == da.EALIGN
+    assert lib.dec_attn_plan(FAKE, 2, 2, 60, 1000, 8, FAKE, 1 << 20, C.byref(h), None) == da.ENOTSUP
+    need = lib.dec_attn_plan_bytes(2, 2, 64, 1000, 8)
+    assert lib.dec_attn_plan(FAKE, 2, 2, 64, 1000, 8, FAKE, need - 1, C.byref(h), None) == da.ESMALL

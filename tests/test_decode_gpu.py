@@ -1,0 +1,153 @@
+"""Split + combine on the GPU vs the fp64 oracle (out max-abs <= 2e-3, lse <= 1e-4).
+
+Small problems cover every kernel variant (bf16 / FP8 KV, head_dim 64 / 128, G*T from 1 to
+16, page sizes 16 / 32 / 64), ragged tails, one-key and empty requests, T > 1 causal rows
+that see no key, single-tile requests (final output written by the split kernel) and
+many-tile requests (combine). The five workloads run at full size with sampled rows
+checked against the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_decode_29_b200 as da
+import workloads as W
+from tests import _gpu as U
+from tests import _helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+def small(seq_lens, *, Hq=8, Hkv=2, d=128, P=16, T=1, kv="bf16", seed=7, tl=64, peaky=0.0, pool=None):
+    return W.make_problem(name="small", batch=len(seq_lens), n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d,
+                          seq_lens=seq_lens, page_size=P, q_tokens=T, kv_dtype=kv, seed=seed, tile_len=tl,
+                          pool_pages=pool, peaky_frac=peaky)
+
+
+def check_all(pr, **kw):
+    out, lse, pl, st = U.run_problem(pr, **kw)
+    assert st == da.OK, da.status_string(st)
+    ref_o, ref_l = oracle.decode(pr)
+    return U.check_rows(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, pr.name)
+
+
+def test_tiny_config_all_rows():
+    check_all(W.make_config("tiny"))
+
+
+LENS = [1, 15, 16, 17, 63, 64, 65, 200, 333]
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8e4m3"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("G,T", [(1, 1), (2, 1), (3, 1), (4, 1), (5, 1), (8, 1), (2, 4), (4, 3), (16, 1), (4, 4)])
+def test_variants(kv, d, G, T):
+    Hkv = 2
+    pr = small(LENS, Hq=G * Hkv, Hkv=Hkv, d=d, T=T, kv=kv, seed=G * 10 + T)
+    check_all(pr)
+
+
+@pytest.mark.parametrize("P,tl", [(16, 16), (16, 256), (32, 64), (64, 64), (64, 256)])
+@pytest.mark.parametrize("kv", ["bf16", "fp8e4m3"])
+def test_page_sizes_and_tiles(P, tl, kv):
+    pr = small([5, 64, 100, 777, 1024, 1500], Hq=8, Hkv=2, d=128, P=P, T=2, kv=kv, tl=tl, seed=P + tl)
+    check_all(pr)
+
+
+def test_empty_and_short_requests():
+    # L = 0 (no keys), L < T (early query tokens see nothing), L = T, one key
+    pr = small([0, 1, 2, 3, 4, 0, 50], Hq=8, Hkv=2, d=64, T=4, tl=16)
+    check_all(pr)
+
+
+def test_peaky_softmax_bf16():
+    pr = small([300, 2000, 4100], Hq=8, Hkv=2, d=128, T=1, tl=256, peaky=0.05)
+    check_all(pr)
+
+
+def test_small_bins_and_single_bin():
+    pr = small([100, 700, 1300], Hq=8, Hkv=2, d=128, T=1, tl=64)
+    check_all(pr, n_bins=1)
+    check_all(pr, n_bins=3)
+
+
+def test_page_renumbering_gives_identical_gpu_output():
+    pr = small([77, 500, 1000], Hq=8, Hkv=2, d=128, T=2, tl=128)
+    o1, l1, _, s1 = U.run_problem(pr)
+    o2, l2, _, s2 = U.run_problem(H.repage(pr, 4))
+    assert s1 == s2 == da.OK
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_bad_page_id_sets_status_without_fault():
+    pr = small([40, 90], Hq=8, Hkv=2, d=128, tl=64)
+    pr.page_table = pr.page_table.copy()
+    pr.page_table[1, 2] = pr.num_pages + 5        # outside the pool
+    out, lse, pl, st = U.run_problem(pr)
+    ws_status = st
+    assert ws_status == da.EDEVICE
+
+
+def test_capacity_overflow_propagates_to_run():
+    pr = small([400, 900], Hq=8, Hkv=2, d=128, tl=64)
+    dev = U.to_device(pr)
+    pl = da.plan(dev["lens"], 2, 64, max_total_kv_tokens=100)
+    out = torch.full((2, 1, 8, 128), 7.0, device="cuda")
+    lse = torch.full((2, 1, 8), 7.0, device="cuda")
+    da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl, out=out, lse=lse)
+    assert da.read_status(pl) == da.ECAPACITY
+    assert torch.all(out == 7.0) and torch.all(lse == 7.0)   # nothing written
+
+
+def test_cuda_graph_replay_matches_eager():
+    pr = small([100, 700, 1300, 5], Hq=8, Hkv=2, d=128, T=1, tl=64)
+    dev = U.to_device(pr)
+    total = int(pr.seq_lens.sum())
+    pl = da.plan(dev["lens"], 2, 64, max_total_kv_tokens=total)
+    out_e, lse_e = da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl)
+    torch.cuda.synchronize()
+    buf = torch.empty_like(pl.buf)
+    shape = da.make_shape(dev["q"], dev["k"], dev["tab"], da.KV_BF16)
+    ws = torch.empty(da.workspace_bytes(shape, pl), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(out_e)
+    lse = torch.empty_like(lse_e)
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        # warm-up outside capture sets the per-device kernel attributes
+        pl2 = da.plan(dev["lens"], 2, 64, max_total_kv_tokens=total, buf=buf, stream=s)
+        da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl2, workspace=ws, out=out, lse=lse, stream=s)
+        s.synchronize()
+        out.zero_(); lse.zero_()
+        with torch.cuda.graph(g, stream=s):
+            pl2 = da.plan(dev["lens"], 2, 64, max_total_kv_tokens=total, buf=buf, stream=s)
+            da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl2, workspace=ws, out=out, lse=lse,
+                   stream=s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, out_e) and torch.equal(lse, lse_e)
+
+
+def _sample_rows(pr, n, seed):
+    rng = np.random.default_rng(seed)
+    B, T, Hq = pr.batch, pr.q_tokens, pr.n_q_heads
+    rows = {(int(np.argmax(pr.seq_lens)), T - 1, Hq - 1), (int(np.argmin(pr.seq_lens)), 0, 0), (B - 1, T - 1, 0)}
+    while len(rows) < n:
+        rows.add((int(rng.integers(B)), int(rng.integers(T)), int(rng.integers(Hq))))
+    return np.array(sorted(rows), dtype=np.int32)
+
+
+@pytest.mark.parametrize("name", ["uniform", "mixed", "long_b1", "long_b4", "fp8_spec"])
+def test_full_size_configs_sampled_rows(name):
+    pr = W.make_config(name)
+    out, lse, pl, st = U.run_problem(pr)
+    assert st == da.OK, da.status_string(st)
+    out = out.cpu().numpy()
+    lse = lse.cpu().numpy()
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    rows = _sample_rows(pr, 48, seed=1)
+    ref_o, ref_l = oracle.decode_rows(pr, rows)
+    got_o = out[rows[:, 0], rows[:, 1], rows[:, 2]]
+    got_l = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
+    U.check_rows(got_o, got_l, ref_o, ref_l, name)
