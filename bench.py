@@ -1,0 +1,500 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark on B200: microseconds per decode step and achieved HBM
+bandwidth, for GQA decode attention over a paged KV cache with split-KV scheduling.
+
+A step is one pass of the whole path on one batch: the planner kernel, the split kernel
+and the combine kernel (plan + split + combine). Inputs are seeded synthetic data of the
+named workload (``--config``, default "uniform": batch 32, 32 query / 8 KV heads,
+head_dim 128, every KV length 4096, page size 16, bf16), resident in HBM before timing.
+
+Timing: W untimed warm-up steps, then K timed steps (events at step boundaries only, so the
+three kernels keep their programmatic-dependent-launch overlap), then the same K steps again
+with events between the kernels for the per-kernel breakdown used by the roofline. Before each step the L2 is flushed
+by reading a 256 MiB buffer (a read leaves no dirty lines for the timed kernels to write
+back; the KV of every full-size workload is larger than the 126 MB L2 as well) and the GPU is kept busy for a moment so that every launch of the step is queued
+before the step starts; CUDA events on the launching stream bracket the planner, the
+split kernel and the combine kernel of every step. ``value`` is the mean step time
+(max over ranks when run under torchrun: the path does not shard, so each rank runs a
+full replica). One JSON line is printed by rank 0.
+
+``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample of the same
+workload (rows chosen at random, time scaled to the whole step).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "decode-attention µs/step and achieved HBM GB/s as % of B200 peak, 1 GPU"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+FLUSH_BYTES = 256 << 20
+SLEEP_CYCLES = 1_000_000  # ~0.5 ms of GPU spin before each step: longer than the host needs to queue it
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="uniform", choices=sorted(W.CONFIGS))
+    ap.add_argument("--tile-len", type=int, default=0, help="override the workload's tile length")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="keep only the first BATCH requests of the workload (smaller profiling cases)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay figure")
+    ap.add_argument("--profile", action="store_true",
+                    help="only warm-up + timed steps (for ncu launch lists): no baseline, e2e, graph or clocks")
+    ap.add_argument("--json-out", default="", help="also append the JSON line to this file")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("split.cu", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "paged_kv_decode_29_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(config: str, tile_len: int):
+    """DRAM bytes per split-kernel launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "split_kernel_dram_traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    e = d.get("configs", {}).get(f"{config}/tl{tile_len}")
+    return None if e is None else float(e["bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = None
+        self.err = ""
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu_id:
+            cmd.insert(1, f"--id={self.gpu_id}")
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+        except Exception as e:
+            self.proc = None
+            self.err = str(e)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, self.err = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "error": self.err[-200:]}
+        rows = [r for r in csv.reader(io.StringIO(self.out)) if len(r) >= 9]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle timing (CPU)
+
+def oracle_timing(pr, budget_s: float, seed: int = 0):
+    """Times the fp64 oracle on a random sample of query rows sized to ~budget_s, and scales the
+    time to the whole step by the rows' key counts. Returns (us_per_step, threads, sample text)."""
+    import oracle
+    B, T, Hq = pr.batch, pr.q_tokens, pr.n_q_heads
+    rows = np.array([(b, t, qh) for b in range(B) for t in range(T) for qh in range(Hq)], dtype=np.int32)
+    keys = np.maximum(pr.seq_lens[rows[:, 0]].astype(np.int64) - T + 1 + rows[:, 1], 0)
+    total_keys = int(keys.sum())
+    rng = np.random.default_rng(seed)
+    order = rng.permutation(len(rows))
+    threads = oracle.max_threads()
+    # calibration on a few rows, then a sample sized to the budget
+    n0 = min(len(rows), max(threads, 8))
+    t0 = time.perf_counter()
+    oracle.decode_rows(pr, rows[order[:n0]], nthreads=threads)
+    dt0 = max(time.perf_counter() - t0, 1e-4)
+    per_key = dt0 / max(int(keys[order[:n0]].sum()), 1)
+    want_keys = budget_s / per_key
+    csum = np.cumsum(keys[order])
+    n = int(np.searchsorted(csum, want_keys)) + 1
+    n = max(min(n, len(rows)), 1)
+    sel = order[:n]
+    t0 = time.perf_counter()
+    oracle.decode_rows(pr, rows[sel], nthreads=threads)
+    dt = time.perf_counter() - t0
+    frac = int(keys[sel].sum()) / max(total_keys, 1)
+    us = dt / max(frac, 1e-12) * 1e6
+    sample = (f"{n} of {len(rows)} query rows ({100 * frac:.1f}% of the row x key work) of the {pr.name} "
+              f"workload, fp64 oracle, time scaled by key count")
+    return us, threads, sample
+
+
+# ---------------------------------------------------------------- reference arm
+
+def make_workload(args):
+    kw = dict(W.CONFIGS[args.config])
+    if args.tile_len:
+        kw["tile_len"] = args.tile_len
+    lens = W.config_seq_lens(args.config)
+    name = args.config
+    if args.batch:
+        lens = lens[: args.batch]
+        kw["batch"] = len(lens)
+        name = f"{args.config}[:{len(lens)}]"
+        if "pool_pages" in kw:
+            del kw["pool_pages"]
+    return W.make_problem(name=name, seq_lens=lens, **kw)
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return 0
+    pr = make_workload(args)
+    import oracle
+    oracle.build()
+    budget = max(0.5, 90.0 / max(args.steps + args.warmup, 1))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        us, threads, sample = oracle_timing(pr, budget, seed=i)
+        if i >= args.warmup:
+            vals.append(us)
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "us/step",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value / 1e3, 6),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": pr.name, **workload_desc(pr)},
+        "cpu_baseline": {"value": round(value, 3), "unit": "us/step", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: {sample}"},
+        "e2e": {"value": round(value, 3), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    emit(line, args)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+
+def workload_desc(pr):
+    return {"batch": pr.batch, "n_q_heads": pr.n_q_heads, "n_kv_heads": pr.n_kv_heads, "head_dim": pr.head_dim,
+            "q_tokens": pr.q_tokens, "page_size": pr.page_size, "kv_dtype": pr.kv_dtype, "tile_len": pr.tile_len,
+            "total_kv_tokens": int(pr.seq_lens.astype(np.int64).sum()),
+            "kv_bytes": int(pr.seq_lens.astype(np.int64).sum()) * pr.n_kv_heads * pr.head_dim * 2
+            * pr.kv_elem_bytes()}
+
+
+def emit(line, args):
+    s = json.dumps(line)
+    print(s, flush=True)
+    if args.json_out:
+        with open(args.json_out, "a") as f:
+            f.write(s + "\n")
+
+
+def run_ours(args, rank: int, world: int, local_rank: int, dist):
+    import torch
+
+    import paged_kv_decode_29_b200 as da
+    from paged_kv_decode_29_b200 import build as dbuild
+
+    if not os.path.exists(da.LIB_PATH):
+        dbuild.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pr = make_workload(args)
+    log(f"[rank {rank}] workload {pr.name}: B={pr.batch} Hq={pr.n_q_heads} Hkv={pr.n_kv_heads} d={pr.head_dim} "
+        f"T={pr.q_tokens} P={pr.page_size} kv={pr.kv_dtype} tl={pr.tile_len} tokens={int(pr.seq_lens.sum())}")
+
+    def to_dev(a, dt=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return t.to(dev) if dt is None else t.view(dt).to(dev)
+
+    q = torch.from_numpy(pr.q.view(np.int16)).view(torch.bfloat16).to(dev)
+    if pr.kv_dtype == "bf16":
+        k = torch.from_numpy(pr.k_pages.view(np.int16)).view(torch.bfloat16).to(dev)
+        v = torch.from_numpy(pr.v_pages.view(np.int16)).view(torch.bfloat16).to(dev)
+        sc = None
+    else:
+        k, v, sc = to_dev(pr.k_pages), to_dev(pr.v_pages), to_dev(pr.kv_scales)
+    tab, lens = to_dev(pr.page_table), to_dev(pr.seq_lens)
+    total = int(pr.seq_lens.astype(np.int64).sum())
+    stream = torch.cuda.current_stream()
+    pl = da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total)
+    shape = da.make_shape(q, k, tab, da.kv_dtype_of(k), pr.sm_scale)
+    ws = torch.empty(da.workspace_bytes(shape, pl), dtype=torch.uint8, device=dev)
+    out = torch.empty((pr.batch, pr.q_tokens, pr.n_q_heads, pr.head_dim), dtype=torch.float32, device=dev)
+    lse = torch.empty((pr.batch, pr.q_tokens, pr.n_q_heads), dtype=torch.float32, device=dev)
+    flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.int64, device=dev)
+
+    def flush_l2():
+        torch.sum(flush, dim=0, out=flush_sink)  # reads 256 MiB: evicts the KV, leaves clean lines
+    pbuf = pl.buf
+    kw = dict(kv_scales=sc, sm_scale=pr.sm_scale, workspace=ws, out=out, lse=lse)
+
+    def enqueue_step(evs):
+        """plan + split + combine; evs: 2 events (step boundaries) or 4 (also between kernels,
+        which stops the kernels' programmatic overlap -- used for the per-kernel breakdown)."""
+        evs[0].record(stream)
+        da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=pbuf)
+        if len(evs) == 4:
+            evs[1].record(stream)
+        da.run(q, k, v, tab, lens, pl, stage="split", **kw)
+        if len(evs) == 4:
+            evs[2].record(stream)
+        da.run(q, k, v, tab, lens, pl, stage="combine", **kw)
+        evs[-1].record(stream)
+
+    def one_step(evs):
+        flush_l2()
+        torch.cuda._sleep(SLEEP_CYCLES)  # keeps the GPU busy while the host queues the step
+        enqueue_step(evs)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def new_events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = ""
+    # clocks are sampled every 200 ms from before the warm-up to after the last measurement
+    # pass; short runs get extra untimed steps so that the samples cover GPU activity
+    sampler = ClockSampler(gpu_id) if not args.profile else None
+    if sampler:
+        sampler.__enter__()
+    t_window = time.perf_counter()
+    for _ in range(args.warmup):
+        one_step(new_events(4))
+    st = da.read_status(pl, ws)
+    if st != da.OK:
+        raise RuntimeError(f"device status after warm-up: {da.status_string(st)}")
+    mean = statistics.mean
+
+    # ---- the timed steps: events at step boundaries only
+    evs = [new_events(2) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        one_step(evs[i])
+    barrier()
+    step_us = [evs[i][0].elapsed_time(evs[i][1]) * 1e3 for i in range(args.steps)]
+
+    # ---- per-kernel breakdown: the same steps with events between the kernels
+    bevs = [new_events(4) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        one_step(bevs[i])
+    barrier()
+    plan_us = [bevs[i][0].elapsed_time(bevs[i][1]) * 1e3 for i in range(args.steps)]
+    split_us = [bevs[i][1].elapsed_time(bevs[i][2]) * 1e3 for i in range(args.steps)]
+    comb_us = [bevs[i][2].elapsed_time(bevs[i][3]) * 1e3 for i in range(args.steps)]
+    st = da.read_status(pl, ws)
+    if st != da.OK:
+        raise RuntimeError(f"device status after timing: {da.status_string(st)}")
+    local = [mean(step_us), mean(plan_us), mean(split_us), mean(comb_us)]
+    if dist is not None:
+        t = torch.tensor(local, dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        local = t.tolist()
+    step_m, plan_m, split_m, comb_m = local
+
+    # CUDA-graph replay of the same step (context figure)
+    graph_us = None
+    if not args.no_graph and not args.profile:
+        g = torch.cuda.CUDAGraph()
+        gs = torch.cuda.Stream()
+        gs.wait_stream(stream)
+        with torch.cuda.stream(gs):
+            with torch.cuda.graph(g, stream=gs):
+                da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=pbuf, stream=gs)
+                da.run(q, k, v, tab, lens, pl, stream=gs, **kw)
+        stream.wait_stream(gs)
+        gt = []
+        for i in range(args.warmup + args.steps):
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush_l2()
+            torch.cuda._sleep(SLEEP_CYCLES)
+            a.record(stream)
+            g.replay()
+            b_.record(stream)
+            b_.synchronize()
+            if i >= args.warmup:
+                gt.append(a.elapsed_time(b_) * 1e3)
+        graph_us = mean(gt)
+        del g
+
+    if sampler:
+        while time.perf_counter() - t_window < 1.5:
+            one_step(new_events(2))
+            torch.cuda.synchronize()
+        sampler.__exit__(None, None, None)
+
+    # end to end through the C ABI: inputs of the step from pinned host memory, result back
+    e2e = None
+    if not args.no_e2e and not args.profile:
+        hq = torch.from_numpy(pr.q.view(np.int16)).view(torch.bfloat16).pin_memory()
+        htab = torch.from_numpy(pr.page_table).pin_memory()
+        hlens = torch.from_numpy(pr.seq_lens).pin_memory()
+        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        h2d = hq.numel() * 2 + htab.numel() * 4 + hlens.numel() * 4
+        d2h = hout.numel() * 4 + hlse.numel() * 4
+        et = []
+        for i in range(args.warmup + args.steps):
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush_l2()
+            torch.cuda._sleep(SLEEP_CYCLES)
+            a.record(stream)
+            q.copy_(hq, non_blocking=True)
+            tab.copy_(htab, non_blocking=True)
+            lens.copy_(hlens, non_blocking=True)
+            da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=pbuf)
+            da.run(q, k, v, tab, lens, pl, **kw)
+            hout.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+            b_.record(stream)
+            b_.synchronize()
+            if i >= args.warmup:
+                et.append(a.elapsed_time(b_) * 1e3)
+        e2e_local = mean(et)
+        if dist is not None:
+            t = torch.tensor([e2e_local], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_local = t.item()
+        e2e = {"value": round(e2e_local, 3), "unit": "us/step", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h),
+               "note": "per step: q, page table and seq_lens from pinned host memory, plan + split + combine, "
+                       "out and lse back to pinned host memory; the KV cache stays resident in HBM"}
+
+    if rank != 0:
+        return 0
+    alg = pr.algorithmic_bytes()
+    peak, peak_kind = measured_peak()
+    split_gbs = alg / (split_m * 1e-6) / 1e9
+    step_gbs = alg / (step_m * 1e-6) / 1e9
+    traffic = ncu_traffic(args.config, pr.tile_len)
+    line = {
+        "metric": METRIC, "value": round(step_m, 3), "unit": "us/step", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_m / 1e3, 6), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3->f16" if pr.kv_dtype == "fp8e4m3" else "bf16",
+        "data": "synthetic",
+        "config": {"workload": pr.name, **workload_desc(pr), "n_bins": pl.n_bins,
+                   "l2": "flushed before every step (256 MiB memset); KV bytes exceed the 126 MB L2",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "breakdown_note": "plan/split/combine: a second pass of the same steps with events between the kernels",
+        "plan_us": round(plan_m, 3), "split_us": round(split_m, 3), "combine_us": round(comb_m, 3),
+        "graph_step_us": None if graph_us is None else round(graph_us, 3),
+        "algorithmic_bytes": int(alg),
+        "hbm_gbs_step": round(step_gbs, 1), "pct_of_8tbs_step": round(100 * step_gbs / NOMINAL_HBM_GBS, 2),
+        "hbm_gbs_split": round(split_gbs, 1), "pct_of_8tbs_split": round(100 * split_gbs / NOMINAL_HBM_GBS, 2),
+        "roofline": {"bound": "hbm", "kernel": "split_kernel", "achieved": round(split_gbs, 1),
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(split_gbs / peak, 4),
+                     "traffic": None if traffic is None else int(traffic)},
+        "gpu_launches": 3 * args.steps,  # planner, split and combine kernels per timed step
+    }
+    if sampler:
+        line["clocks"] = sampler.summary()
+    if e2e is not None:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline and not args.profile and world == 1:
+        import oracle
+        oracle.build()
+        us, threads, sample = oracle_timing(pr, budget_s=15.0)
+        line["cpu_baseline"] = {"value": round(us, 1), "unit": "us/step", "cores": threads, "kind": "oracle",
+                                "sample": sample}
+    emit(line, args)
+    return 0
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                 device_id=torch.device("cuda", local_rank))
+        dist = tdist
+    try:
+        return run_ours(args, rank, world, local_rank, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

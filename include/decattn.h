@@ -33,8 +33,11 @@
  *    shapes, buffers too small) return a negative decattn_status and enqueue
  *    nothing. Errors only the device can see (a page id outside the pool, more
  *    tiles than the plan can hold, a pipeline wait that gives up) never trap:
- *    they set a status word in the plan or workspace, which
+ *    they set a status word in the plan buffer's header, which
  *    dec_attn_read_status() returns.
+ *  - The planner, split and combine kernels are chained with programmatic
+ *    dependent launch: each later kernel may be scheduled while the earlier one
+ *    drains and waits on the device until it has finished.
  */
 #ifndef DECATTN_H
 #define DECATTN_H
@@ -123,8 +126,9 @@ DECATTN_API size_t dec_attn_plan_bytes(int batch, int n_kv_heads, int tile_len, 
 DECATTN_API int dec_attn_plan(const int32_t *seq_lens, int batch, int n_kv_heads, int tile_len, int64_t max_total_kv_tokens,
                   int n_bins, void *plan_buf, size_t plan_bytes, dec_attn_plan_t *plan, void *stream);
 
-/* Bytes of the device workspace dec_attn_run needs: a status word plus room for
- * the partial (o, lse) of every tile the plan can hold (fp32, [tiles][G*T][d+1]).
+/* Bytes of the device workspace dec_attn_run needs: room for the partial (o, lse)
+ * of every tile the plan can hold (fp32, [tiles][G*T][d+1]) after a 256-byte
+ * reserved header.
  * Returns 0 for invalid arguments. */
 DECATTN_API size_t dec_attn_workspace_bytes(const dec_attn_shape *shape, const dec_attn_plan_t *plan);
 
@@ -158,9 +162,24 @@ DECATTN_API int dec_attn_run(const dec_attn_shape *shape, const void *q, const v
                  const dec_attn_plan_t *plan, void *workspace, size_t workspace_bytes, float *out, float *lse,
                  void *stream);
 
-/* Synchronises `stream`, then returns the first device-detected status recorded in
- * the plan header and (if not NULL) the workspace, or DECATTN_OK. Either pointer
- * may be NULL. For tests and diagnostics, not for the hot path. */
+/* The two stages of dec_attn_run as separate calls (same arguments, same checks):
+ * dec_attn_split enqueues only the split kernel, dec_attn_combine only the combine
+ * kernel, which reads the partials the split kernel left in `workspace`. dec_attn_run(...) == dec_attn_split(...) followed by
+ * dec_attn_combine(...) on the same stream. Useful to time or overlap the stages. */
+DECATTN_API int dec_attn_split(const dec_attn_shape *shape, const void *q, const void *k_pages, const void *v_pages,
+                               const int32_t *page_table, const int32_t *seq_lens, const float *kv_scales,
+                               const dec_attn_plan_t *plan, void *workspace, size_t workspace_bytes, float *out,
+                               float *lse, void *stream);
+DECATTN_API int dec_attn_combine(const dec_attn_shape *shape, const void *q, const void *k_pages, const void *v_pages,
+                                 const int32_t *page_table, const int32_t *seq_lens, const float *kv_scales,
+                                 const dec_attn_plan_t *plan, void *workspace, size_t workspace_bytes, float *out,
+                                 float *lse, void *stream);
+
+/* Synchronises `stream`, then returns the planner's status if it failed, else the
+ * first device-detected error of any split kernel run on this plan since the plan
+ * was made (the planner clears it), else DECATTN_OK. `workspace` is accepted for
+ * symmetry with dec_attn_run and not read. For tests and diagnostics, not for the
+ * hot path. */
 DECATTN_API int dec_attn_read_status(const dec_attn_plan_t *plan, const void *workspace, void *stream);
 
 /* Static text for a decattn_status value. */

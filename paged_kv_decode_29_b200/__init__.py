@@ -27,7 +27,7 @@ LIB_PATH = os.path.join(_HERE, "libdecattn.so")
 OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1, -2, -3, -4, -5, -6, -7, -8
 KV_BF16, KV_FP8E4M3 = 0, 1
 API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_workspace_bytes",
-       "dec_attn_run", "dec_attn_read_status", "dec_attn_status_string")
+       "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_read_status", "dec_attn_status_string")
 
 
 class DecAttnError(RuntimeError):
@@ -70,8 +70,10 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_plan.restype = i32
         lib.dec_attn_workspace_bytes.argtypes = [C.POINTER(ShapeT), C.POINTER(PlanT)]
         lib.dec_attn_workspace_bytes.restype = sz
-        lib.dec_attn_run.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, C.POINTER(PlanT), vp, sz, vp, vp, vp]
-        lib.dec_attn_run.restype = i32
+        for name in ("dec_attn_run", "dec_attn_split", "dec_attn_combine"):
+            f = getattr(lib, name)
+            f.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, C.POINTER(PlanT), vp, sz, vp, vp, vp]
+            f.restype = i32
         lib.dec_attn_read_status.argtypes = [C.POINTER(PlanT), vp, vp]
         lib.dec_attn_read_status.restype = i32
         lib.dec_attn_status_string.argtypes = [i32]
@@ -172,12 +174,13 @@ def workspace_bytes(shape: ShapeT, pl: Plan) -> int:
 def run(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_table: torch.Tensor,
         seq_lens: torch.Tensor, pl: Plan, *, kv_scales: torch.Tensor | None = None, sm_scale: float = 0.0,
         workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
-        stream=None):
+        stream=None, stage: str = "run"):
     """Enqueues split + combine on ``stream``; returns (out fp32 [B][T][Hq][d], lse fp32 [B][T][Hq]).
 
     q: bf16 [B][T][Hq][d]; k_pages / v_pages: [num_pages][Hkv][P][d] bf16, or uint8 / float8_e4m3fn
     E4M3 codes with ``kv_scales`` fp32 [2][num_pages][Hkv]; page_table: int32 [B][max_pages_per_seq];
-    seq_lens: int32 [B] (the values the plan was made from)."""
+    seq_lens: int32 [B] (the values the plan was made from). ``stage``: "run" (split + combine), or
+    "split" / "combine" alone (the combine reads the partials the split left in ``workspace``)."""
     lib = load_library()
     kvt = kv_dtype_of(k_pages)
     shape = make_shape(q, k_pages, page_table, kvt, sm_scale)
@@ -188,11 +191,12 @@ def run(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_tabl
         lse = torch.empty((B, T, Hq), dtype=torch.float32, device=q.device)
     if workspace is None:
         workspace = torch.empty(workspace_bytes(shape, pl), dtype=torch.uint8, device=q.device)
-    rc = lib.dec_attn_run(C.byref(shape), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(seq_lens),
-                          _ptr(kv_scales), C.byref(pl.handle), _ptr(workspace), workspace.numel(), _ptr(out),
-                          _ptr(lse), _stream_handle(stream))
+    fn = {"run": lib.dec_attn_run, "split": lib.dec_attn_split, "combine": lib.dec_attn_combine}[stage]
+    rc = fn(C.byref(shape), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table), _ptr(seq_lens),
+            _ptr(kv_scales), C.byref(pl.handle), _ptr(workspace), workspace.numel(), _ptr(out), _ptr(lse),
+            _stream_handle(stream))
     if rc != OK:
-        raise DecAttnError(rc, "dec_attn_run")
+        raise DecAttnError(rc, f"dec_attn_{stage}")
     return out, lse
 
 

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI front end: argument checks, workspace layout, TMA tensor maps and
 // the launches of the split and combine kernels. See include/decattn.h for the contract.
 #include <math.h>
+#include <stddef.h>
 
 #include <map>
 #include <mutex>
@@ -77,24 +78,33 @@ static bool make_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int D,
 }
 
 struct WsLayout {
-  int64_t off_part_lse, off_part_o, total;
+  int64_t off_part_lse, off_part_o, off_row_cnt, off_chunk, total;
 };
 
-static WsLayout ws_layout(int64_t max_units, int GT, int D) {
+// Workspace: reserved header | partial lse [units][GT] | partial o [units][GT][D] |
+// combine row counters [B*T*Hq] | combine chunk states [items][D + 4].
+static WsLayout ws_layout(int64_t max_units, const dec_attn_shape& s) {
+  const int GT = s.n_q_heads / s.n_kv_heads * s.q_tokens;
+  const int D = s.head_dim;
+  const int64_t rows = (int64_t)s.batch * s.q_tokens * s.n_q_heads;
+  const int64_t items = (int64_t)GT * ((max_units + kCombineChunk - 1) / kCombineChunk) + rows;
   WsLayout w;
   int64_t o = sizeof(WorkspaceHeader);
   w.off_part_lse = o; o = align_up(o + 4 * max_units * GT, 256);
   w.off_part_o = o; o = align_up(o + 4 * max_units * GT * D, 256);
+  w.off_row_cnt = o; o = align_up(o + 4 * rows, 256);
+  w.off_chunk = o; o = align_up(o + 4 * items * (D + 4), 256);
   w.total = o;
   return w;
 }
 
 // Same layout arithmetic as dec_attn_plan (plan.cu).
-static void plan_offsets(const dec_attn_plan_t* pl, int64_t* off_bin_off, int64_t* off_pair_off,
+static void plan_offsets(const dec_attn_plan_t* pl, int64_t* off_bin_off, int64_t* off_pair_off, int64_t* off_cb,
                          int64_t* off_units) {
   int64_t o = sizeof(PlanHeader);
   *off_bin_off = o; o = align_up(o + 4 * (int64_t)(pl->n_bins + 1), 32);
   *off_pair_off = o; o = align_up(o + 4 * ((int64_t)pl->batch * pl->n_kv_heads + 1), 32);
+  *off_cb = o; o = align_up(o + 4 * ((int64_t)pl->batch + 1), 32);
   *off_units = o;
 }
 
@@ -120,22 +130,13 @@ static int check_shape(const dec_attn_shape* s, const dec_attn_plan_t* pl) {
   return DECATTN_OK;
 }
 
-}  // namespace decattn
+// Checks the arguments and enqueues the requested stages (kStageSplit, kStageCombine).
+enum { kStageSplit = 1, kStageCombine = 2 };
 
-using namespace decattn;
-
-extern "C" int dec_attn_default_bins(int device) { return default_bins(device); }
-
-extern "C" size_t dec_attn_workspace_bytes(const dec_attn_shape* shape, const dec_attn_plan_t* plan) {
-  if (check_shape(shape, plan) != DECATTN_OK) return 0;
-  const int GT = shape->n_q_heads / shape->n_kv_heads * shape->q_tokens;
-  return (size_t)ws_layout(plan->max_units, GT, shape->head_dim).total;
-}
-
-extern "C" int dec_attn_run(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
-                            const int32_t* page_table, const int32_t* seq_lens, const float* kv_scales,
-                            const dec_attn_plan_t* plan, void* workspace, size_t workspace_bytes, float* out,
-                            float* lse, void* stream) {
+static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
+                   const int32_t* page_table, const int32_t* seq_lens, const float* kv_scales,
+                   const dec_attn_plan_t* plan, void* workspace, size_t workspace_bytes, float* out, float* lse,
+                   void* stream) {
   int rc = check_shape(shape, plan);
   if (rc != DECATTN_OK) return rc;
   const dec_attn_shape& s = *shape;
@@ -153,65 +154,108 @@ extern "C" int dec_attn_run(const dec_attn_shape* shape, const void* q, const vo
   const int G = s.n_q_heads / s.n_kv_heads;
   const int GT = G * s.q_tokens;
   const int D = s.head_dim;
-  const WsLayout wl = ws_layout(plan->max_units, GT, D);
+  (void)GT;
+  const WsLayout wl = ws_layout(plan->max_units, s);
   if ((int64_t)workspace_bytes < wl.total) return DECATTN_ESMALL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DECATTN_ECUDA;
 
-  CUtensorMap tmK, tmV;
-  const int64_t rows = (int64_t)s.num_pages * s.n_kv_heads * s.page_size;
-  if (!make_kv_map(&tmK, k_pages, s.kv_dtype, D, rows) || !make_kv_map(&tmV, v_pages, s.kv_dtype, D, rows))
-    return DECATTN_ECUDA;
-
-  int64_t off_bin_off, off_pair_off, off_units;
-  plan_offsets(plan, &off_bin_off, &off_pair_off, &off_units);
+  int64_t off_bin_off, off_pair_off, off_cb, off_units;
+  plan_offsets(plan, &off_bin_off, &off_pair_off, &off_cb, &off_units);
   char* ws = static_cast<char*>(workspace);
+  int32_t* row_cnt = reinterpret_cast<int32_t*>(ws + wl.off_row_cnt);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), st) != cudaSuccess) return DECATTN_ECUDA;
+  float* part_o = reinterpret_cast<float*>(ws + wl.off_part_o);
+  float* part_lse = reinterpret_cast<float*>(ws + wl.off_part_lse);
 
-  const float scale = s.sm_scale > 0.f ? s.sm_scale : 1.0f / sqrtf((float)D);
-  SplitParams sp;
-  sp.q = static_cast<const uint16_t*>(q);
-  sp.page_table = page_table;
-  sp.kv_scales = kv_scales;
-  sp.plan = static_cast<const char*>(plan->buf);
-  sp.out = out;
-  sp.lse = lse;
-  sp.part_o = reinterpret_cast<float*>(ws + wl.off_part_o);
-  sp.part_lse = reinterpret_cast<float*>(ws + wl.off_part_lse);
-  sp.status = reinterpret_cast<int32_t*>(ws);
-  sp.B = s.batch; sp.T = s.q_tokens; sp.Hq = s.n_q_heads; sp.Hkv = s.n_kv_heads; sp.G = G; sp.GT = GT;
-  sp.P = s.page_size; sp.num_pages = s.num_pages; sp.mpps = s.max_pages_per_seq; sp.n_bins = plan->n_bins;
-  sp.off_bin_off = (int)off_bin_off;
-  sp.off_units = (int)off_units;
-  sp.qk_scale_log2 = scale * 1.4426950408889634f;
-  if (launch_split(sp, tmK, tmV, s.kv_dtype, D, st) != cudaSuccess) return DECATTN_ECUDA;
-
-  CombineParams cp;
-  cp.plan = sp.plan;
-  cp.seq_lens = seq_lens;
-  cp.part_o = sp.part_o;
-  cp.part_lse = sp.part_lse;
-  cp.out = out;
-  cp.lse = lse;
-  cp.T = s.q_tokens; cp.Hq = s.n_q_heads; cp.Hkv = s.n_kv_heads; cp.G = G; cp.GT = GT; cp.D = D;
-  cp.tl = plan->tile_len;
-  cp.off_pair_off = (int)off_pair_off;
-  if (launch_combine(cp, s.batch * s.q_tokens * s.n_q_heads, st) != cudaSuccess) return DECATTN_ECUDA;
+  if (stages & kStageSplit) {
+    CUtensorMap tmK, tmV;
+    const int64_t rows = (int64_t)s.num_pages * s.n_kv_heads * s.page_size;
+    if (!make_kv_map(&tmK, k_pages, s.kv_dtype, D, rows) || !make_kv_map(&tmV, v_pages, s.kv_dtype, D, rows))
+      return DECATTN_ECUDA;
+    const float scale = s.sm_scale > 0.f ? s.sm_scale : 1.0f / sqrtf((float)D);
+    SplitParams sp;
+    sp.q = static_cast<const uint16_t*>(q);
+    sp.page_table = page_table;
+    sp.kv_scales = kv_scales;
+    sp.plan = static_cast<const char*>(plan->buf);
+    sp.out = out;
+    sp.lse = lse;
+    sp.part_o = part_o;
+    sp.part_lse = part_lse;
+    sp.row_cnt = row_cnt;
+    sp.status = reinterpret_cast<int32_t*>(static_cast<char*>(plan->buf) + offsetof(PlanHeader, run_status));
+    sp.B = s.batch; sp.T = s.q_tokens; sp.Hq = s.n_q_heads; sp.Hkv = s.n_kv_heads; sp.G = G; sp.GT = GT;
+    sp.P = s.page_size; sp.num_pages = s.num_pages; sp.mpps = s.max_pages_per_seq; sp.n_bins = plan->n_bins;
+    sp.off_bin_off = (int)off_bin_off;
+    sp.off_units = (int)off_units;
+    sp.qk_scale_log2 = scale * 1.4426950408889634f;
+    if (launch_split(sp, tmK, tmV, s.kv_dtype, D, st) != cudaSuccess) return DECATTN_ECUDA;
+  }
+  if (stages & kStageCombine) {
+    CombineParams cp;
+    cp.plan = static_cast<const char*>(plan->buf);
+    cp.seq_lens = seq_lens;
+    cp.part_o = part_o;
+    cp.part_lse = part_lse;
+    cp.out = out;
+    cp.lse = lse;
+    cp.row_cnt = row_cnt;
+    cp.chunk_state = reinterpret_cast<float*>(ws + wl.off_chunk);
+    cp.B = s.batch; cp.T = s.q_tokens; cp.Hq = s.n_q_heads; cp.Hkv = s.n_kv_heads; cp.G = G; cp.GT = GT; cp.D = D;
+    cp.tl = plan->tile_len;
+    cp.off_pair_off = (int)off_pair_off;
+    cp.off_cb = (int)off_cb;
+    if (launch_combine(cp, dev, st) != cudaSuccess) return DECATTN_ECUDA;
+  }
   return DECATTN_OK;
+}
+
+}  // namespace decattn
+
+using namespace decattn;
+
+extern "C" int dec_attn_default_bins(int device) { return default_bins(device); }
+
+extern "C" size_t dec_attn_workspace_bytes(const dec_attn_shape* shape, const dec_attn_plan_t* plan) {
+  if (check_shape(shape, plan) != DECATTN_OK) return 0;
+  return (size_t)ws_layout(plan->max_units, *shape).total;
+}
+
+extern "C" int dec_attn_run(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
+                            const int32_t* page_table, const int32_t* seq_lens, const float* kv_scales,
+                            const dec_attn_plan_t* plan, void* workspace, size_t workspace_bytes, float* out,
+                            float* lse, void* stream) {
+  return enqueue(kStageSplit | kStageCombine, shape, q, k_pages, v_pages, page_table,
+                          seq_lens, kv_scales, plan, workspace, workspace_bytes, out, lse, stream);
+}
+
+extern "C" int dec_attn_split(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
+                              const int32_t* page_table, const int32_t* seq_lens, const float* kv_scales,
+                              const dec_attn_plan_t* plan, void* workspace, size_t workspace_bytes, float* out,
+                              float* lse, void* stream) {
+  return enqueue(kStageSplit, shape, q, k_pages, v_pages, page_table, seq_lens, kv_scales, plan,
+                          workspace, workspace_bytes, out, lse, stream);
+}
+
+extern "C" int dec_attn_combine(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* page_table, const int32_t* seq_lens, const float* kv_scales,
+                                const dec_attn_plan_t* plan, void* workspace, size_t workspace_bytes, float* out,
+                                float* lse, void* stream) {
+  return enqueue(kStageCombine, shape, q, k_pages, v_pages, page_table, seq_lens, kv_scales, plan,
+                          workspace, workspace_bytes, out, lse, stream);
 }
 
 extern "C" int dec_attn_read_status(const dec_attn_plan_t* plan, const void* workspace, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return DECATTN_ECUDA;
+  (void)workspace;  // device errors of a run are recorded in the plan buffer's header
   if (plan && plan->buf) {
     PlanHeader h;
     if (cudaMemcpy(&h, plan->buf, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return DECATTN_ECUDA;
     if (h.magic != kPlanMagic) return DECATTN_EINVAL;
     if (h.status != DECATTN_OK) return h.status;
-  }
-  if (workspace) {
-    int32_t w = 0;
-    if (cudaMemcpy(&w, workspace, sizeof w, cudaMemcpyDeviceToHost) != cudaSuccess) return DECATTN_ECUDA;
-    if (w != DECATTN_OK) return w;
+    if (h.run_status != DECATTN_OK) return h.run_status;
   }
   return DECATTN_OK;
 }

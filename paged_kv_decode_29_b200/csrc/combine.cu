@@ -7,91 +7,170 @@
 // lse = M + ln sum_i w_i. A tile that saw no key of the row has lse_i = -inf and weight
 // 0; a row with no visible key at all gets out = 0, lse = -inf.
 //
-// One CTA per query row; each group of D/4 threads reads one partial row as float4s, the
-// groups stride over the row's partials, and the CTA folds the group sums in shared
-// memory. Rows of requests held in a single tile were written by the split kernel and
-// are skipped here.
+// Work decomposition (computed by the planner): each query row of request b is cut into
+// cb_b chunks of up to kCombineChunk tiles; the items (b, row, chunk) are numbered request
+// by request. The kernel is persistent: every warp takes items w, w + #warps, ...
+//  * a warp loads the lse and the D floats of up to 16 partial rows at once (16 loads in
+//    flight per lane) and folds them into (max, weight, weighted sum);
+//  * a row made of one chunk is finished right there;
+//  * otherwise the warp publishes its chunk state and bumps the row's counter; the warp
+//    that brings the counter to cb_b merges the row's chunk states and writes the row.
+// Rows of requests held in a single tile were written by the split kernel (cb_b = 0).
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace decattn {
 
-
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 128;
+constexpr int kCombineWarps = kCombineThreads / 32;
+constexpr int kCombineCtasPerSm = 4;
 
 template <int D>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineParams p) {
-  constexpr int TPP = D / 4;                       // threads per partial row (float4 each)
-  constexpr int PPB = kCombineThreads / TPP;       // partial rows in flight per pass
-  const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
-  if (hdr->magic != kPlanMagic || hdr->status != DECATTN_OK) return;  // the split kernel reports it
-  const int row = blockIdx.x;
-  const int b = row / (p.T * p.Hq), t = (row / p.Hq) % p.T, qh = row % p.Hq;
-  const int L = p.seq_lens[b];
-  const int nb = L > 0 ? (L + p.tl - 1) / p.tl : 0;
-  if (nb == 1) return;
-  float* orow = p.out + (int64_t)row * D;
-  if (nb == 0) {
-    for (int i = threadIdx.x; i < D; i += kCombineThreads) orow[i] = 0.f;
-    if (threadIdx.x == 0) p.lse[row] = -INFINITY;
-    return;
-  }
-  const int h = qh / p.G, r = t * p.G + (qh % p.G);
-  const int32_t* pair_off = reinterpret_cast<const int32_t*>(p.plan + p.off_pair_off);
-  const int64_t slot0 = pair_off[(int64_t)b * p.Hkv + h];
-  __shared__ float red[kCombineThreads / 32];
-  __shared__ float accs[PPB][D];
-  __shared__ float ws[PPB];
+struct CombineVec {
+  static constexpr int VEC = D / 32;  // floats per lane
+  using T = typename std::conditional<VEC == 4, float4, float2>::type;
+};
 
-  // pass 1: M = max lse_i
-  float M = -INFINITY;
-  for (int i = threadIdx.x; i < nb; i += kCombineThreads) M = fmaxf(M, p.part_lse[(slot0 + i) * p.GT + r]);
+template <int D>
+__device__ __forceinline__ void write_row(float* orow, float* lse_out, int lane, float M, float W,
+                                          const float (&acc)[D / 32]) {
+  constexpr int VEC = D / 32;
+  using V = typename CombineVec<D>::T;
+  V v;
+  float* f = reinterpret_cast<float*>(&v);
+  const bool empty = M == -INFINITY || !(W > 0.f);
+  const float inv = empty ? 0.f : 1.f / W;
   #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = M;
-  __syncthreads();
-  M = red[0];
-  #pragma unroll
-  for (int w = 1; w < kCombineThreads / 32; ++w) M = fmaxf(M, red[w]);
-  if (M == -INFINITY) {
-    for (int i = threadIdx.x; i < D; i += kCombineThreads) orow[i] = 0.f;
-    if (threadIdx.x == 0) p.lse[row] = -INFINITY;
-    return;
-  }
-
-  // pass 2: weighted sum of the partial rows
-  const int sub = threadIdx.x / TPP, q4 = threadIdx.x % TPP;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float W = 0.f;
-  #pragma unroll 4
-  for (int i = sub; i < nb; i += PPB) {
-    const int64_t pr = (slot0 + i) * p.GT + r;
-    const float li = p.part_lse[pr];
-    const float4 v = reinterpret_cast<const float4*>(p.part_o + pr * D)[q4];
-    const float w = li == -INFINITY ? 0.f : expf(li - M);
-    acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
-    W += w;
-  }
-  reinterpret_cast<float4*>(&accs[sub][0])[q4] = acc;
-  if (q4 == 0) ws[sub] = W;
-  __syncthreads();
-  float Wt = 0.f;
-  #pragma unroll
-  for (int k = 0; k < PPB; ++k) Wt += ws[k];
-  for (int i = threadIdx.x; i < D; i += kCombineThreads) {
-    float s = 0.f;
-    #pragma unroll
-    for (int k = 0; k < PPB; ++k) s += accs[k][i];
-    orow[i] = s / Wt;
-  }
-  if (threadIdx.x == 0) p.lse[row] = M + logf(Wt);
+  for (int e = 0; e < VEC; ++e) f[e] = acc[e] * inv;
+  reinterpret_cast<V*>(orow)[lane] = v;
+  if (lane == 0) *lse_out = empty ? -INFINITY : M + logf(W);
 }
 
-cudaError_t launch_combine(const CombineParams& p, int rows, cudaStream_t st) {
-  if (rows <= 0) return cudaSuccess;
-  if (p.D == 128) combine_kernel<128><<<rows, kCombineThreads, 0, st>>>(p);
-  else if (p.D == 64) combine_kernel<64><<<rows, kCombineThreads, 0, st>>>(p);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+template <int D>
+__global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_kernel(const CombineParams p) {
+  constexpr int VEC = D / 32;
+  using V = typename CombineVec<D>::T;
+  extern __shared__ int32_t cb_sm[];  // [B + 1] chunk prefix per request
+  griddep_wait();  // the split kernel's partials are complete and visible
+  const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
+  if (hdr->magic != kPlanMagic || hdr->status != DECATTN_OK) return;  // the split kernel reports it
+  const int32_t* cb_g = reinterpret_cast<const int32_t*>(p.plan + p.off_cb);
+  for (int i = threadIdx.x; i <= p.B; i += kCombineThreads) cb_sm[i] = cb_g[i];
+  __syncthreads();
+  const int32_t* pair_off = reinterpret_cast<const int32_t*>(p.plan + p.off_pair_off);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t rows_per_b = (int64_t)p.T * p.Hq;
+  const int64_t total = rows_per_b * cb_sm[p.B];
+  const int64_t nwarps = (int64_t)gridDim.x * kCombineWarps;
+
+  for (int64_t w = (int64_t)blockIdx.x * kCombineWarps + warp; w < total; w += nwarps) {
+    int lo = 0, hi = p.B - 1;  // request: last b with rows_per_b * cb[b] <= w
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (rows_per_b * cb_sm[mid] <= w) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const int ncb = cb_sm[b + 1] - cb_sm[b];
+    const int64_t local = w - rows_per_b * cb_sm[b];
+    const int row_in_b = (int)(local / ncb), j = (int)(local - (int64_t)row_in_b * ncb);
+    const int t = row_in_b / p.Hq, qh = row_in_b - t * p.Hq;
+    const int64_t row = ((int64_t)b * p.T + t) * p.Hq + qh;
+    float* orow = p.out + row * D;
+    const int L = p.seq_lens[b];
+    const int nb = L > 0 ? (L + p.tl - 1) / p.tl : 0;
+    float acc[VEC];
+    #pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+    if (nb == 0) {  // no key at all
+      write_row<D>(orow, p.lse + row, lane, -INFINITY, 0.f, acc);
+      continue;
+    }
+    const int h = qh / p.G, r = t * p.G + (qh - h * p.G);
+    const int64_t slot0 = pair_off[(int64_t)b * p.Hkv + h] + (int64_t)j * kCombineChunk;
+    const int n = min(kCombineChunk, nb - j * kCombineChunk);
+    // ---- fold up to kCombineChunk partial rows
+    const float my_lse = lane < n ? p.part_lse[(slot0 + lane) * p.GT + r] : -INFINITY;
+    V v[kCombineChunk];
+    #pragma unroll
+    for (int i = 0; i < kCombineChunk; ++i)
+      if (i < n) v[i] = reinterpret_cast<const V*>(p.part_o + ((slot0 + i) * p.GT + r) * D)[lane];
+    float M = my_lse;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float my_w = (lane < n && M != -INFINITY) ? expf(my_lse - M) : 0.f;
+    float W = my_w;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+    #pragma unroll
+    for (int i = 0; i < kCombineChunk; ++i) {
+      const float wi = __shfl_sync(0xffffffffu, my_w, i);
+      if (i < n) {
+        const float* f = reinterpret_cast<const float*>(&v[i]);
+        #pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += wi * f[e];
+      }
+    }
+    if (ncb == 1) {
+      write_row<D>(orow, p.lse + row, lane, M, W, acc);
+      continue;
+    }
+    // ---- publish this chunk; the last chunk of the row merges them all
+    float* cs = p.chunk_state + w * (D + 4);
+    #pragma unroll
+    for (int e = 0; e < VEC; ++e) cs[4 + lane * VEC + e] = acc[e];
+    if (lane == 0) { cs[0] = M; cs[1] = W; }
+    __threadfence();
+    __syncwarp();
+    int prev = 0;
+    if (lane == 0) prev = atomicAdd(&p.row_cnt[row], 1);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev != ncb - 1) continue;
+    __threadfence();
+    const float* cs0 = p.chunk_state + (w - j) * (D + 4);
+    float Mt = -INFINITY;
+    for (int c = lane; c < ncb; c += 32) Mt = fmaxf(Mt, __ldcg(cs0 + (int64_t)c * (D + 4)));
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Mt = fmaxf(Mt, __shfl_xor_sync(0xffffffffu, Mt, o));
+    float Wt = 0.f;
+    #pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+    if (Mt != -INFINITY) {
+      #pragma unroll 8
+      for (int c = 0; c < ncb; ++c) {
+        const float* s = cs0 + (int64_t)c * (D + 4);
+        const float mc = __ldcg(s), wc = __ldcg(s + 1);
+        const float sc = mc == -INFINITY ? 0.f : expf(mc - Mt);
+        Wt += sc * wc;
+        #pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += sc * __ldcg(s + 4 + lane * VEC + e);
+      }
+    }
+    write_row<D>(orow, p.lse + row, lane, Mt, Wt, acc);
+    if (lane == 0) p.row_cnt[row] = 0;  // ready for the next combine on this workspace
+  }
+}
+
+cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st) {
+  if ((int64_t)p.B * p.T * p.Hq <= 0) return cudaSuccess;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return cudaErrorUnknown;
+  const void* fn = p.D == 128 ? (const void*)combine_kernel<128> : (const void*)combine_kernel<64>;
+  const int smem = 4 * (p.B + 1);
+  if (!ensure_smem_attr(fn, smem)) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sms * kCombineCtasPerSm);
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // scheduled while the split kernel drains
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (p.D == 128) return cudaLaunchKernelEx(&cfg, combine_kernel<128>, p);
+  if (p.D == 64) return cudaLaunchKernelEx(&cfg, combine_kernel<64>, p);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace decattn

@@ -30,7 +30,8 @@ struct PlanHeader {
   int32_t off_pair_off; // int32 [n_pairs + 1]: first partial slot of each (b, h)
   int32_t off_units;    // Unit [max_units]
   int32_t off_scratch;  // planner scratch
-  int32_t reserved[2];
+  int32_t run_status;   // first device-detected error of a split kernel run on this plan (0 = none)
+  int32_t off_cb;       // int32 [batch + 1]: prefix over requests of combine chunks per query row
 };
 static_assert(sizeof(PlanHeader) == 64, "plan header is 64 bytes");
 constexpr int32_t kPlanMagic = 0x31504144;  // "DAP1"
@@ -58,13 +59,23 @@ struct SplitParams {
   float* lse;               // [B][T][Hq]
   float* part_o;            // [max_units][GT][D]
   float* part_lse;          // [max_units][GT]
-  int32_t* status;          // workspace status word
+  int32_t* row_cnt;         // [B*T*Hq] combine counters, zeroed here for the combine that follows
+  int32_t* status;          // run status word (plan header)
   int B, T, Hq, Hkv, G, GT, P, num_pages, mpps, n_bins;
   int off_bin_off, off_units;
   float qk_scale_log2;      // sm_scale * log2(e)
 };
 
-// Arguments of the combine kernel (one CTA per query row).
+// The combine kernel folds the partials of one query row in chunks of this many tiles.
+// A request with n_b tiles gives each of its rows cb_b = ceil(n_b / kCombineChunk) chunks
+// (1 if n_b == 0: the row is zero-filled; 0 if n_b == 1: the split kernel wrote the row).
+constexpr int kCombineChunk = 16;
+
+__host__ __device__ inline int combine_chunks(int64_t n_b) {
+  return n_b == 0 ? 1 : n_b == 1 ? 0 : (int)((n_b + kCombineChunk - 1) / kCombineChunk);
+}
+
+// Arguments of the combine kernel (persistent; warps walk the (row, chunk) items).
 struct CombineParams {
   const char* plan;
   const int32_t* seq_lens;
@@ -72,8 +83,10 @@ struct CombineParams {
   const float* part_lse;
   float* out;
   float* lse;
-  int T, Hq, Hkv, G, GT, D, tl;
-  int off_pair_off;
+  int32_t* row_cnt;         // [B*T*Hq] chunks of the row folded so far (zeroed by the split kernel)
+  float* chunk_state;       // [items][D + 4]: max, weight, -, -, then the weighted sum
+  int B, T, Hq, Hkv, G, GT, D, tl;
+  int off_pair_off, off_cb;
 };
 
 __host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -82,6 +95,13 @@ __host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + 
 __device__ __forceinline__ void set_status(int32_t* st, int32_t code) {
   if (st) atomicCAS(st, 0, code);
 }
+
+// Programmatic dependent launch: let the next kernel of the stream start its prologue
+// early / wait until the previous kernel has completed and its writes are visible.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -260,6 +280,6 @@ bool split_supported(int kv_dtype, int D, int GT);                // split.cu
 cudaError_t launch_split(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int kv_dtype,
                          int D, cudaStream_t st);                 // split.cu
 int split_ctas_per_sm();                                          // split.cu
-cudaError_t launch_combine(const CombineParams& p, int rows, cudaStream_t st);  // combine.cu
+cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st);  // combine.cu
 
 }  // namespace decattn

@@ -20,40 +20,43 @@
 
 namespace decattn {
 
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 512;
 constexpr int kPlanMaxBins = 8192;
+constexpr int kPlanSmemRequests = 4096;  // per-request arrays sit in shared memory up to this batch
+constexpr int kPlanMaxSmem = 200 * 1024;
 
-struct PlanScratch {
-  int64_t* S;        // [B+1] exclusive prefix over requests of tiles per (b, h) pair
-  int64_t* SF;       // [B+1] same for full tiles
-  int32_t* SP;       // [B+1] same for "has a partial tile"
-  int32_t* plist;    // [B]   requests with a partial tile, in b order
-  int32_t* pcost;    // [B]   their partial-tile cost
-  int32_t* sorted_b; // [B]   same requests sorted by cost desc, b asc
-  int32_t* part_bin; // [B*Hkv] bin of the s-th partial tile in greedy order
-  int32_t* part_pos; // [B*Hkv] its position among that bin's partial tiles
+// Per-request arrays (index b): exclusive prefix sums over requests of the tiles of one
+// (b, h) pair (S), of its full tiles (SF) and of "has a partial tile" (SP); the requests
+// with a partial tile in b order (plist, with their partial-tile cost pcost) and sorted by
+// that cost, largest first (sorted_b).
+struct ReqArrays {
+  int32_t *S, *SF, *SP, *plist, *pcost, *sorted_b;
 };
 
+__host__ __device__ inline int64_t plan_bins_smem(int N) { return align_up(12 * (int64_t)N + 4, 16); }
+__host__ __device__ inline int64_t req_stride(int B) { return align_up(4 * (int64_t)(B + 1), 16); }
+__host__ __device__ inline int64_t req_arrays_bytes(int B) { return 6 * req_stride(B); }
+
+// Global scratch of the plan buffer: the per-request arrays when they do not fit in shared
+// memory, then the bin and in-bin position of every partial tile in greedy order.
 __host__ __device__ inline int64_t plan_scratch_bytes(int B, int Hkv) {
-  return align_up(8 * (int64_t)(B + 1), 32) * 2 + align_up(4 * (int64_t)(B + 1), 32) +
-         align_up(4 * (int64_t)B, 32) * 3 + align_up(4 * (int64_t)B * Hkv, 32) * 2;
+  return req_arrays_bytes(B) + 2 * align_up(4 * (int64_t)B * Hkv, 32);
 }
 
-__device__ inline PlanScratch carve_scratch(char* p, int B, int Hkv) {
-  PlanScratch s;
-  s.S = reinterpret_cast<int64_t*>(p); p += align_up(8 * (int64_t)(B + 1), 32);
-  s.SF = reinterpret_cast<int64_t*>(p); p += align_up(8 * (int64_t)(B + 1), 32);
-  s.SP = reinterpret_cast<int32_t*>(p); p += align_up(4 * (int64_t)(B + 1), 32);
-  s.plist = reinterpret_cast<int32_t*>(p); p += align_up(4 * (int64_t)B, 32);
-  s.pcost = reinterpret_cast<int32_t*>(p); p += align_up(4 * (int64_t)B, 32);
-  s.sorted_b = reinterpret_cast<int32_t*>(p); p += align_up(4 * (int64_t)B, 32);
-  s.part_bin = reinterpret_cast<int32_t*>(p); p += align_up(4 * (int64_t)B * Hkv, 32);
-  s.part_pos = reinterpret_cast<int32_t*>(p);
-  return s;
+__device__ inline ReqArrays carve_req(char* p, int B) {
+  const int64_t st = req_stride(B);
+  ReqArrays r;
+  r.S = reinterpret_cast<int32_t*>(p);
+  r.SF = reinterpret_cast<int32_t*>(p + st);
+  r.SP = reinterpret_cast<int32_t*>(p + 2 * st);
+  r.plist = reinterpret_cast<int32_t*>(p + 3 * st);
+  r.pcost = reinterpret_cast<int32_t*>(p + 4 * st);
+  r.sorted_b = reinterpret_cast<int32_t*>(p + 5 * st);
+  return r;
 }
 
 // Exclusive block-wide scan of (a, b, c) over kPlanThreads threads; returns the prefix and
-// adds the block totals into tot.
+// adds the block totals into tot. warp_tot holds one entry per warp (at most 32 warps).
 struct Tri { long long a, b; int c; };
 
 __device__ inline Tri block_exscan(Tri v, Tri& tot, Tri* warp_tot) {
@@ -69,7 +72,7 @@ __device__ inline Tri block_exscan(Tri v, Tri& tot, Tri* warp_tot) {
   if (lane == 31) warp_tot[w] = inc;
   __syncthreads();
   if (w == 0) {
-    Tri t = warp_tot[lane];
+    Tri t = lane < kPlanThreads / 32 ? warp_tot[lane] : Tri{0, 0, 0};
     #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       long long a = __shfl_up_sync(0xffffffffu, t.a, o);
@@ -81,34 +84,125 @@ __device__ inline Tri block_exscan(Tri v, Tri& tot, Tri* warp_tot) {
   }
   __syncthreads();
   Tri base = w ? warp_tot[w - 1] : Tri{0, 0, 0};
-  Tri all = warp_tot[31];
+  Tri all = warp_tot[kPlanThreads / 32 - 1];
   __syncthreads();
   Tri ex{base.a + inc.a - v.a, base.b + inc.b - v.b, base.c + inc.c - v.c};
   tot.a += all.a; tot.b += all.b; tot.c += all.c;
   return ex;
 }
 
+// Greedy placement of the partial tiles s in [first, m) by one warp. Lane l owns the bins
+// [l*K, (l+1)*K) and keeps their loads (relative to the common full-tile base) in
+// registers; a warp-wide min over the packed key (load << 5 | lane) finds the least-loaded
+// bin, the lowest bin index winning ties (lower lanes own lower bins, and each lane keeps
+// its lowest-index minimum). Needs every relative load below 2^27 (checked on the host).
+template <int KMAX>
+__device__ void greedy_partials(int lane, int N, int64_t first, int64_t m, int Hkv, int tl,
+                                const int32_t* __restrict__ seq_lens, const int32_t* sorted_b, uint32_t* load_sm,
+                                int32_t* pcount_sm, int32_t* part_bin, int32_t* part_pos) {
+  const int K = (N + 31) / 32;
+  const int k0 = lane * K;
+  uint32_t ld[KMAX];
+  int32_t pc[KMAX];
+  #pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    const int k = k0 + j;
+    const bool ok = j < K && k < N;
+    ld[j] = ok ? load_sm[k] : 0x07ffffffu;  // above any real load
+    pc[j] = ok ? pcount_sm[k] : 0;
+  }
+  uint32_t lmin = ld[0];
+  int lj = 0;
+  #pragma unroll
+  for (int j = 1; j < KMAX; ++j)
+    if (ld[j] < lmin) { lmin = ld[j]; lj = j; }
+  for (int64_t s0 = first; s0 < m; s0 += 32) {
+    const int64_t sl = s0 + lane;
+    const uint32_t cl = sl < m ? (uint32_t)(seq_lens[sorted_b[sl / Hkv]] % tl) : 0u;
+    const int n_here = (int)(m - s0 < 32 ? m - s0 : 32);
+    for (int i = 0; i < n_here; ++i) {
+      const uint32_t c = __shfl_sync(0xffffffffu, cl, i);
+      const uint32_t key = __reduce_min_sync(0xffffffffu, (lmin << 5) | (uint32_t)lane);
+      if ((int)(key & 31u) == lane) {
+        const int64_t s = s0 + i;
+        part_bin[s] = k0 + lj;
+        #pragma unroll
+        for (int j = 0; j < KMAX; ++j)
+          if (j == lj) { part_pos[s] = pc[j]; pc[j] += 1; ld[j] += c; }
+        lmin = ld[0];
+        lj = 0;
+        #pragma unroll
+        for (int j = 1; j < KMAX; ++j)
+          if (ld[j] < lmin) { lmin = ld[j]; lj = j; }
+      }
+    }
+  }
+  #pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    const int k = k0 + j;
+    if (j < K && k < N) pcount_sm[k] = pc[j];
+  }
+}
+
+// Same rule with the loads in shared memory (more bins than the register version holds).
+__device__ void greedy_partials_smem(int lane, int N, int64_t first, int64_t m, int Hkv, int tl,
+                                     const int32_t* __restrict__ seq_lens, const int32_t* sorted_b, uint32_t* load_sm,
+                                     int32_t* pcount_sm, int32_t* part_bin, int32_t* part_pos) {
+  const int K = (N + 31) / 32;
+  const int k0 = lane * K, k1 = min(N, k0 + K);
+  uint32_t lmin = 0x07ffffffu;
+  int lk = k0;
+  for (int k = k0; k < k1; ++k)
+    if (load_sm[k] < lmin) { lmin = load_sm[k]; lk = k; }
+  for (int64_t s0 = first; s0 < m; s0 += 32) {
+    const int64_t sl = s0 + lane;
+    const uint32_t cl = sl < m ? (uint32_t)(seq_lens[sorted_b[sl / Hkv]] % tl) : 0u;
+    const int n_here = (int)(m - s0 < 32 ? m - s0 : 32);
+    for (int i = 0; i < n_here; ++i) {
+      const uint32_t c = __shfl_sync(0xffffffffu, cl, i);
+      const uint32_t key = __reduce_min_sync(0xffffffffu, (lmin << 5) | (uint32_t)lane);
+      if ((int)(key & 31u) == lane) {
+        const int64_t s = s0 + i;
+        part_bin[s] = lk;
+        part_pos[s] = pcount_sm[lk]++;
+        load_sm[lk] += c;
+        lmin = 0x07ffffffu;
+        for (int k = k0; k < k1; ++k)
+          if (load_sm[k] < lmin) { lmin = load_sm[k]; lk = k; }
+      }
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kPlanThreads, 1)
 plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* __restrict__ plan) {
+  // the split kernel may start its prologue now; it waits for this grid before reading the plan
+  griddep_launch_dependents();
   const int B = init.batch, Hkv = init.n_kv_heads, tl = init.tile_len, N = init.n_bins;
   const int64_t max_units = init.max_units;
-  extern __shared__ uint32_t sm_dyn[];
-  uint32_t* load = sm_dyn;           // [N] bin load minus the common full-tile base
-  int32_t* pcount = reinterpret_cast<int32_t*>(sm_dyn + N);  // [N] partial tiles per bin
+  extern __shared__ __align__(16) uint8_t plan_smem[];
+  uint32_t* load = reinterpret_cast<uint32_t*>(plan_smem);                 // [N] load above the full-tile base
+  int32_t* pcount = reinterpret_cast<int32_t*>(plan_smem + 4 * (int64_t)N);  // [N] partial tiles per bin
+  int32_t* boff = reinterpret_cast<int32_t*>(plan_smem + 8 * (int64_t)N);    // [N + 1] CSR offsets
   __shared__ Tri warp_tot[32];
-  __shared__ int32_t sh_cost[kPlanThreads];
   __shared__ int32_t sh_status;
 
   PlanHeader* hdr = reinterpret_cast<PlanHeader*>(plan);
   int32_t* bin_off = reinterpret_cast<int32_t*>(plan + init.off_bin_off);
   int32_t* pair_off = reinterpret_cast<int32_t*>(plan + init.off_pair_off);
+  int32_t* cbuf = reinterpret_cast<int32_t*>(plan + init.off_cb);
   Unit* units = reinterpret_cast<Unit*>(plan + init.off_units);
-  PlanScratch sc = carve_scratch(plan + init.off_scratch, B, Hkv);
+  char* gscratch = plan + init.off_scratch;
+  const ReqArrays R = carve_req(B <= kPlanSmemRequests ? reinterpret_cast<char*>(plan_smem + plan_bins_smem(N))
+                                                       : gscratch, B);
+  int32_t* part_bin = reinterpret_cast<int32_t*>(gscratch + req_arrays_bytes(B));
+  int32_t* part_pos = part_bin + align_up((int64_t)B * Hkv, 8);
   const int tid = threadIdx.x;
   if (tid == 0) {
     sh_status = 0;
     PlanHeader h = init;
     h.magic = 0;  // published last, once the plan is complete
+    h.run_status = 0;
     *hdr = h;
   }
 
@@ -122,13 +216,13 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
     Tri before = carry;
     Tri ex = block_exscan(v, carry, warp_tot);
     if (b < B) {
-      sc.S[b] = before.a + ex.a;
-      sc.SF[b] = before.b + ex.b;
-      sc.SP[b] = before.c + ex.c;
-      if (v.c) { sc.plist[before.c + ex.c] = b; sc.pcost[before.c + ex.c] = (int32_t)(L % tl); }
+      R.S[b] = (int32_t)(before.a + ex.a);
+      R.SF[b] = (int32_t)(before.b + ex.b);
+      R.SP[b] = before.c + ex.c;
+      if (v.c) { R.plist[before.c + ex.c] = b; R.pcost[before.c + ex.c] = (int32_t)(L % tl); }
     }
   }
-  if (tid == 0) { sc.S[B] = carry.a; sc.SF[B] = carry.b; sc.SP[B] = carry.c; }
+  if (tid == 0) { R.S[B] = (int32_t)carry.a; R.SF[B] = (int32_t)carry.b; R.SP[B] = carry.c; }
   const int64_t U = (int64_t)Hkv * carry.a;
   const int64_t F = (int64_t)Hkv * carry.b;
   const int mB = carry.c;
@@ -147,29 +241,28 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
     return;
   }
 
-  // ---- 2. pair offsets (first partial slot of each (b, h))
-  for (int64_t p = tid; p < (int64_t)B * Hkv; p += kPlanThreads) {
-    const int b = (int)(p / Hkv), h = (int)(p % Hkv);
-    pair_off[p] = (int32_t)(Hkv * sc.S[b] + (int64_t)h * (sc.S[b + 1] - sc.S[b]));
+  // ---- 2. combine chunks per query row of each request, and their prefix over requests
+  {
+    Tri c3{0, 0, 0};
+    for (int base = 0; base < B; base += kPlanThreads) {
+      const int b = base + tid;
+      const long long cb = b < B ? combine_chunks(R.S[b + 1] - R.S[b]) : 0;
+      Tri before = c3;
+      Tri ex = block_exscan(Tri{cb, 0, 0}, c3, warp_tot);
+      if (b < B) cbuf[b] = (int32_t)(before.a + ex.a);
+    }
+    if (tid == 0) cbuf[B] = (int32_t)c3.a;
   }
-  if (tid == 0) pair_off[(int64_t)B * Hkv] = (int32_t)U;
 
   // ---- 3. requests with a partial tile, sorted by cost (desc), then b: rank by counting
-  for (int jb = 0; jb < mB; jb += kPlanThreads) {
-    const int j = jb + tid;
-    const int cj = j < mB ? sc.pcost[j] : 0;
+  for (int j = tid; j < mB; j += kPlanThreads) {
+    const int cj = R.pcost[j];
     int rank = 0;
-    for (int cb = 0; cb < mB; cb += kPlanThreads) {
-      __syncthreads();
-      sh_cost[tid] = cb + tid < mB ? sc.pcost[cb + tid] : -1;
-      __syncthreads();
-      const int lim = min(kPlanThreads, mB - cb);
-      for (int k = 0; k < lim; ++k) {
-        const int c = sh_cost[k];
-        rank += (c > cj) | ((c == cj) & (cb + k < j));
-      }
+    for (int k = 0; k < mB; ++k) {
+      const int c = R.pcost[k];
+      rank += (c > cj) | ((c == cj) & (k < j));
     }
-    if (j < mB) sc.sorted_b[rank] = sc.plist[j];
+    R.sorted_b[rank] = R.plist[j];
   }
   __syncthreads();
 
@@ -183,42 +276,28 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
     int32_t pc = 0;
     const int64_t s = k - rf;
     if (k >= rf && s < first) {
-      l += (uint32_t)(seq_lens[sc.sorted_b[s / Hkv]] % tl);
+      l += (uint32_t)(seq_lens[R.sorted_b[(int)s / Hkv]] % tl);
       pc = 1;
-      sc.part_bin[s] = k;
-      sc.part_pos[s] = 0;
+      part_bin[s] = k;
+      part_pos[s] = 0;
     }
     load[k] = l;
     pcount[k] = pc;
   }
   __syncthreads();
   if (tid < 32 && first < m) {
-    const int lane = tid;
-    // each lane watches bins lane, lane+32, ...; it caches the least (load, bin) among them
-    uint32_t lmin = 0xffffffffu, lidx = 0xffffffffu;
-    for (int k = lane; k < N; k += 32)
-      if (load[k] < lmin) { lmin = load[k]; lidx = (uint32_t)k; }
-    int32_t cost_next = 0;
-    for (int64_t s0 = first; s0 < m; s0 += 32) {
-      const int64_t s_l = s0 + lane;
-      cost_next = s_l < m ? (int32_t)(seq_lens[sc.sorted_b[s_l / Hkv]] % tl) : 0;
-      const int64_t n_here = m - s0 < 32 ? m - s0 : 32;
-      for (int i = 0; i < n_here; ++i) {
-        const uint32_t c = (uint32_t)__shfl_sync(0xffffffffu, cost_next, i);
-        const uint32_t gmin = __reduce_min_sync(0xffffffffu, lmin);
-        const uint32_t kbest = __reduce_min_sync(0xffffffffu, lmin == gmin ? lidx : 0xffffffffu);
-        if (lane == (int)(kbest & 31)) {
-          const int64_t s = s0 + i;
-          sc.part_bin[s] = (int32_t)kbest;
-          sc.part_pos[s] = pcount[kbest]++;
-          load[kbest] += c;
-          lmin = 0xffffffffu; lidx = 0xffffffffu;
-          for (int k = lane; k < N; k += 32)
-            if (load[k] < lmin) { lmin = load[k]; lidx = (uint32_t)k; }
-        }
-        __syncwarp();
-      }
-    }
+    const int K = (N + 31) / 32;
+    #define DECATTN_GREEDY(KM) greedy_partials<KM>(tid, N, first, m, Hkv, tl, seq_lens, R.sorted_b, load, pcount, \
+                                                    part_bin, part_pos)
+    if (K <= 4) DECATTN_GREEDY(4);
+    else if (K <= 8) DECATTN_GREEDY(8);
+    else if (K <= 12) DECATTN_GREEDY(12);
+    else if (K <= 16) DECATTN_GREEDY(16);
+    else if (K <= 20) DECATTN_GREEDY(20);
+    else if (K <= 24) DECATTN_GREEDY(24);
+    else if (K <= 32) DECATTN_GREEDY(32);
+    else greedy_partials_smem(tid, N, first, m, Hkv, tl, seq_lens, R.sorted_b, load, pcount, part_bin, part_pos);
+    #undef DECATTN_GREEDY
   }
   __syncthreads();
 
@@ -230,44 +309,51 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
       const long long cnt = k < N ? (long long)(qf + (k < rf)) + pcount[k] : 0;
       Tri before = c2;
       Tri ex = block_exscan(Tri{cnt, 0, 0}, c2, warp_tot);
-      if (k < N) bin_off[k] = (int32_t)(before.a + ex.a);
+      if (k < N) bin_off[k] = boff[k] = (int32_t)(before.a + ex.a);
     }
-    if (tid == 0) bin_off[N] = (int32_t)c2.a;
+    if (tid == 0) bin_off[N] = boff[N] = (int32_t)c2.a;
   }
   __syncthreads();
 
-  // ---- 6. the tiles
-  for (int64_t f = tid; f < F; f += kPlanThreads) {
-    int lo = 0, hi = B - 1;  // last b with Hkv * SF[b] <= f
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if ((int64_t)Hkv * sc.SF[mid] <= f) lo = mid; else hi = mid - 1;
+  // ---- 6. the tiles. Warp w takes pairs p = w, w + 32, ...; lane l writes the pair's full
+  //         tiles i = l, l + 32, ...; full tile f = Hkv*SF[b] + h*fb + i goes to bin f mod N at
+  //         position f div N (kept incrementally: all indices fit in 32 bits, U < 2^31).
+  {
+    const int warp = tid >> 5, lane = tid & 31;
+    const int n_pairs = B * Hkv;
+    for (int pr = warp; pr < n_pairs; pr += kPlanThreads / 32) {
+      const int b = pr / Hkv, h = pr - b * Hkv;
+      const int fb = R.SF[b + 1] - R.SF[b];
+      const int nb = R.S[b + 1] - R.S[b];
+      const int32_t L = seq_lens[b];
+      const int slot0 = Hkv * R.S[b] + h * nb;
+      if (lane == 0) pair_off[pr] = slot0;
+      const int f0 = Hkv * R.SF[b] + h * fb + lane;
+      int q = (int)((unsigned)f0 / (unsigned)N), r = f0 - q * N;
+      const int step_q = 32 / N, step_r = 32 - step_q * N;
+      for (int i = lane; i < fb; i += 32) {
+        Unit u;
+        u.b = b; u.h = h; u.tok_begin = i * tl; u.tok_end = (i + 1) * tl; u.seq_len = L;
+        u.slot = nb == 1 ? -1 : slot0 + i;
+        u.tile = i; u.zero = 0;
+        units[boff[r] + q] = u;
+        q += step_q; r += step_r;
+        if (r >= N) { r -= N; ++q; }
+      }
     }
-    const int b = lo;
-    const int64_t fb = sc.SF[b + 1] - sc.SF[b];
-    const int64_t r = f - (int64_t)Hkv * sc.SF[b];
-    const int h = (int)(r / fb);
-    const int64_t i = r % fb;
-    const int64_t nb = sc.S[b + 1] - sc.S[b];
-    const int32_t L = seq_lens[b];
-    Unit u;
-    u.b = b; u.h = h; u.tok_begin = (int32_t)(i * tl); u.tok_end = (int32_t)((i + 1) * tl); u.seq_len = L;
-    u.slot = nb == 1 ? -1 : (int32_t)(Hkv * sc.S[b] + h * nb + i);
-    u.tile = (int32_t)i; u.zero = 0;
-    const int k = (int)(f % N);
-    units[bin_off[k] + f / N] = u;
+    if (tid == 0) pair_off[n_pairs] = (int32_t)U;
   }
-  for (int64_t s = tid; s < m; s += kPlanThreads) {
-    const int b = sc.sorted_b[s / Hkv], h = (int)(s % Hkv);
-    const int64_t fb = sc.SF[b + 1] - sc.SF[b];
-    const int64_t nb = sc.S[b + 1] - sc.S[b];
+  for (int s = tid; s < (int)m; s += kPlanThreads) {
+    const int b = R.sorted_b[s / Hkv], h = s % Hkv;
+    const int fb = R.SF[b + 1] - R.SF[b];
+    const int nb = R.S[b + 1] - R.S[b];
     const int32_t L = seq_lens[b];
     Unit u;
-    u.b = b; u.h = h; u.tok_begin = (int32_t)(fb * tl); u.tok_end = L; u.seq_len = L;
-    u.slot = nb == 1 ? -1 : (int32_t)(Hkv * sc.S[b] + h * nb + fb);
-    u.tile = (int32_t)fb; u.zero = 0;
-    const int k = sc.part_bin[s];
-    units[bin_off[k] + (qf + (k < rf)) + sc.part_pos[s]] = u;
+    u.b = b; u.h = h; u.tok_begin = fb * tl; u.tok_end = L; u.seq_len = L;
+    u.slot = nb == 1 ? -1 : Hkv * R.S[b] + h * nb + fb;
+    u.tile = fb; u.zero = 0;
+    const int k = part_bin[s];
+    units[boff[k] + (int)(qf + (k < rf)) + part_pos[s]] = u;
   }
   __syncthreads();
   if (tid == 0) {
@@ -280,7 +366,7 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
 
 // ------------------------------------------------------------------ host side
 struct PlanLayout {
-  int64_t off_bin_off, off_pair_off, off_units, off_scratch, total;
+  int64_t off_bin_off, off_pair_off, off_cb, off_units, off_scratch, total;
 };
 
 static PlanLayout plan_layout(int B, int Hkv, int N, int64_t max_units) {
@@ -288,6 +374,7 @@ static PlanLayout plan_layout(int B, int Hkv, int N, int64_t max_units) {
   int64_t o = sizeof(PlanHeader);
   L.off_bin_off = o; o = align_up(o + 4 * (int64_t)(N + 1), 32);
   L.off_pair_off = o; o = align_up(o + 4 * ((int64_t)B * Hkv + 1), 32);
+  L.off_cb = o; o = align_up(o + 4 * ((int64_t)B + 1), 32);
   L.off_units = o; o = align_up(o + (int64_t)sizeof(Unit) * max_units, 32);
   L.off_scratch = o; o = align_up(o + plan_scratch_bytes(B, Hkv), 32);
   L.total = o;
@@ -303,8 +390,8 @@ static bool plan_args_ok(int B, int Hkv, int tl, int64_t max_total, int N) {
   if (B < 0 || Hkv <= 0 || tl <= 0 || (tl % 16) != 0 || max_total < 0 || N <= 0 || N > kPlanMaxBins) return false;
   const int64_t cap = plan_capacity(B, Hkv, tl, max_total);
   if (cap >= (1ll << 31) - 1 || max_total >= (1ll << 31)) return false;
-  // keeps every relative bin load of the greedy pass below 2^32
-  if ((double)B * Hkv * tl / N + 2.0 * tl >= 4294967295.0) return false;
+  // keeps every relative bin load of the greedy pass below 2^27 (its packed min key)
+  if ((double)B * Hkv * tl / N + 2.0 * tl >= 134217727.0) return false;
   return true;
 }
 
@@ -355,9 +442,10 @@ extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads,
   h.off_pair_off = (int32_t)L.off_pair_off;
   h.off_units = (int32_t)L.off_units;
   h.off_scratch = (int32_t)L.off_scratch;
+  h.off_cb = (int32_t)L.off_cb;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t smem = (size_t)n_bins * 8;
-  if (!ensure_smem_attr((const void*)plan_kernel, kPlanMaxBins * 8)) return DECATTN_ECUDA;
+  const size_t smem = (size_t)plan_bins_smem(n_bins) + (batch <= kPlanSmemRequests ? (size_t)req_arrays_bytes(batch) : 0);
+  if (!ensure_smem_attr((const void*)plan_kernel, kPlanMaxSmem)) return DECATTN_ECUDA;
   plan_kernel<<<1, kPlanThreads, smem, st>>>(seq_lens, h, static_cast<char*>(plan_buf));
   if (cudaGetLastError() != cudaSuccess) return DECATTN_ECUDA;
   plan->buf = plan_buf;

@@ -96,6 +96,12 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   Unit* qmeta = reinterpret_cast<Unit*>(sm + S_::OFF_QMETA);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_launch_dependents();  // the combine kernel may be scheduled; it waits for this grid
+  griddep_wait();               // the plan kernel has finished and its writes are visible
+  // the combine counters of this workspace start from zero on every run
+  for (int64_t i = (int64_t)blockIdx.x * kSplitThreads + threadIdx.x; i < (int64_t)p.B * p.T * p.Hq;
+       i += (int64_t)gridDim.x * kSplitThreads)
+    p.row_cnt[i] = 0;
   const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
   if (hdr->magic != kPlanMagic || hdr->status != DECATTN_OK || hdr->n_bins != (int)gridDim.x ||
       hdr->batch != p.B || hdr->n_kv_heads != p.Hkv) {
@@ -498,8 +504,17 @@ static cudaError_t launch_variant(const SplitParams& p, const CUtensorMap& tmK, 
   auto fn = split_kernel<KVT, D, NQ, NPV, DUP>;
   const int smem = Smem<KVT, D, NQ>::ALLOC;
   if (!ensure_smem_attr((const void*)fn, smem)) return cudaErrorInvalidValue;
-  fn<<<p.n_bins, kSplitThreads, smem, st>>>(p, tmK, tmV);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_bins);
+  cfg.blockDim = dim3(kSplitThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlaps our prologue with the planner
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, p, tmK, tmV);
 }
 
 template <int KVT, int D>

@@ -151,3 +151,27 @@ def test_full_size_configs_sampled_rows(name):
     got_o = out[rows[:, 0], rows[:, 1], rows[:, 2]]
     got_l = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
     U.check_rows(got_o, got_l, ref_o, ref_l, name)
+
+
+def test_repeated_runs_on_one_workspace_and_stage_calls():
+    # multi-chunk rows (tile 16, up to 94 tiles per row) exercise the combine's per-row counters
+    pr = small([5, 300, 1500, 1000], Hq=8, Hkv=2, d=128, T=2, tl=16, seed=3)
+    dev = U.to_device(pr)
+    total = int(pr.seq_lens.sum())
+    pl = da.plan(dev["lens"], 2, 16, max_total_kv_tokens=total)
+    shape = da.make_shape(dev["q"], dev["k"], dev["tab"], da.KV_BF16)
+    ws = torch.empty(da.workspace_bytes(shape, pl), dtype=torch.uint8, device="cuda")
+    o1, l1 = da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl, workspace=ws)
+    o1, l1 = o1.clone(), l1.clone()
+    for _ in range(3):
+        o2, l2 = da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl, workspace=ws)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    out = torch.empty_like(o1)
+    lse = torch.empty_like(l1)
+    da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl, workspace=ws, out=out, lse=lse, stage="split")
+    da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl, workspace=ws, out=out, lse=lse,
+           stage="combine")
+    assert da.read_status(pl, ws) == da.OK
+    assert torch.equal(out, o1) and torch.equal(lse, l1)
+    ref_o, ref_l = oracle.decode(pr)
+    U.check_rows(o1.cpu().numpy(), l1.cpu().numpy(), ref_o, ref_l, "repeated")
