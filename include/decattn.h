@@ -126,6 +126,15 @@ DECATTN_API size_t dec_attn_plan_bytes(int batch, int n_kv_heads, int tile_len, 
 DECATTN_API int dec_attn_plan(const int32_t *seq_lens, int batch, int n_kv_heads, int tile_len, int64_t max_total_kv_tokens,
                   int n_bins, void *plan_buf, size_t plan_bytes, dec_attn_plan_t *plan, void *stream);
 
+/* Writes the explicit work list of a finished plan (the device plan stores full tiles in
+ * closed form): bin_off device int32 [n_bins + 1] (CSR offsets), units device int32
+ * [max_units][8] with one record per tile {b, h, tok_begin, tok_end, seq_len, slot, i, 0}
+ * in bin order, and *n_units (device int32) = the tile count, or -1 if the plan failed or
+ * max_units is too small. seq_lens must be the values the plan was made from. One
+ * single-block kernel on `stream`; for tests and diagnostics. */
+DECATTN_API int dec_attn_plan_export(const dec_attn_plan_t *plan, const int32_t *seq_lens, int32_t *bin_off,
+                                     void *units, int64_t max_units, int32_t *n_units, void *stream);
+
 /* Bytes of the device workspace dec_attn_run needs: room for the partial (o, lse)
  * of every tile the plan can hold (fp32, [tiles][G*T][d+1]) after a 256-byte
  * reserved header.

@@ -26,8 +26,9 @@ LIB_PATH = os.path.join(_HERE, "libdecattn.so")
 
 OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1, -2, -3, -4, -5, -6, -7, -8
 KV_BF16, KV_FP8E4M3 = 0, 1
-API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_workspace_bytes",
-       "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_read_status", "dec_attn_status_string")
+API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
+       "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_read_status",
+       "dec_attn_status_string")
 
 
 class DecAttnError(RuntimeError):
@@ -68,6 +69,8 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_plan_bytes.restype = sz
         lib.dec_attn_plan.argtypes = [vp, i32, i32, i32, i64, i32, vp, sz, C.POINTER(PlanT), vp]
         lib.dec_attn_plan.restype = i32
+        lib.dec_attn_plan_export.argtypes = [C.POINTER(PlanT), vp, vp, vp, i64, vp, vp]
+        lib.dec_attn_plan_export.restype = i32
         lib.dec_attn_workspace_bytes.argtypes = [C.POINTER(ShapeT), C.POINTER(PlanT)]
         lib.dec_attn_workspace_bytes.restype = sz
         for name in ("dec_attn_run", "dec_attn_split", "dec_attn_combine"):
@@ -207,18 +210,25 @@ def read_status(pl: Plan | None = None, workspace: torch.Tensor | None = None, s
                                         _stream_handle(stream)))
 
 
-def plan_contents(pl: Plan) -> dict:
-    """Copies the work list back to the host (layout: the plan header of csrc/common.cuh)."""
+def plan_contents(pl: Plan, seq_lens: torch.Tensor, stream=None) -> dict:
+    """The plan's explicit work list (dec_attn_plan_export), copied to the host: status, n_units,
+    bin_off [n_bins + 1] and units [n_units][8] = (b, h, tok_begin, tok_end, seq_len, slot, tile, 0)."""
     import numpy as np
-    raw = pl.buf.cpu().numpy()
-    hdr = raw[:64].view(np.int32)
-    magic, status, n_bins, batch, hkv, tl, n_units, n_pairs = (int(x) for x in hdr[:8])
-    off_bin_off, off_pair_off, off_units = (int(x) for x in hdr[10:13])
-    bin_off = raw[off_bin_off:off_bin_off + 4 * (n_bins + 1)].view(np.int32).copy()
-    pair_off = raw[off_pair_off:off_pair_off + 4 * (n_pairs + 1)].view(np.int32).copy()
-    units = raw[off_units:off_units + 32 * n_units].view(np.int32).reshape(n_units, 8).copy()
-    return dict(magic=magic, status=status, n_bins=n_bins, n_units=n_units, tile_len=tl,
-                bin_off=bin_off, pair_off=pair_off, units=units)
+    lib = load_library()
+    dev = pl.buf.device
+    cap = int(pl.handle.max_units)
+    bin_off = torch.empty(pl.n_bins + 1, dtype=torch.int32, device=dev)
+    units = torch.empty((max(cap, 1), 8), dtype=torch.int32, device=dev)
+    n = torch.empty(1, dtype=torch.int32, device=dev)
+    rc = lib.dec_attn_plan_export(C.byref(pl.handle), _ptr(seq_lens), _ptr(bin_off), _ptr(units), cap, _ptr(n),
+                                  _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_plan_export")
+    hdr = pl.buf[:128].cpu().numpy().view(np.int32)
+    n_units = int(n.item())
+    return dict(magic=int(hdr[0]), status=int(hdr[1]), run_status=int(hdr[2]), n_bins=int(hdr[3]),
+                n_units=n_units, bin_off=bin_off.cpu().numpy(),
+                units=units[:max(n_units, 0)].cpu().numpy())
 
 
 def sm_scale_default(head_dim: int) -> float:

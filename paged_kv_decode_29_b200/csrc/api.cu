@@ -98,16 +98,6 @@ static WsLayout ws_layout(int64_t max_units, const dec_attn_shape& s) {
   return w;
 }
 
-// Same layout arithmetic as dec_attn_plan (plan.cu).
-static void plan_offsets(const dec_attn_plan_t* pl, int64_t* off_bin_off, int64_t* off_pair_off, int64_t* off_cb,
-                         int64_t* off_units) {
-  int64_t o = sizeof(PlanHeader);
-  *off_bin_off = o; o = align_up(o + 4 * (int64_t)(pl->n_bins + 1), 32);
-  *off_pair_off = o; o = align_up(o + 4 * ((int64_t)pl->batch * pl->n_kv_heads + 1), 32);
-  *off_cb = o; o = align_up(o + 4 * ((int64_t)pl->batch + 1), 32);
-  *off_units = o;
-}
-
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 static int check_shape(const dec_attn_shape* s, const dec_attn_plan_t* pl) {
@@ -160,8 +150,6 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DECATTN_ECUDA;
 
-  int64_t off_bin_off, off_pair_off, off_cb, off_units;
-  plan_offsets(plan, &off_bin_off, &off_pair_off, &off_cb, &off_units);
   char* ws = static_cast<char*>(workspace);
   int32_t* row_cnt = reinterpret_cast<int32_t*>(ws + wl.off_row_cnt);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -177,6 +165,7 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
     SplitParams sp;
     sp.q = static_cast<const uint16_t*>(q);
     sp.page_table = page_table;
+    sp.seq_lens = seq_lens;
     sp.kv_scales = kv_scales;
     sp.plan = static_cast<const char*>(plan->buf);
     sp.out = out;
@@ -187,8 +176,6 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
     sp.status = reinterpret_cast<int32_t*>(static_cast<char*>(plan->buf) + offsetof(PlanHeader, run_status));
     sp.B = s.batch; sp.T = s.q_tokens; sp.Hq = s.n_q_heads; sp.Hkv = s.n_kv_heads; sp.G = G; sp.GT = GT;
     sp.P = s.page_size; sp.num_pages = s.num_pages; sp.mpps = s.max_pages_per_seq; sp.n_bins = plan->n_bins;
-    sp.off_bin_off = (int)off_bin_off;
-    sp.off_units = (int)off_units;
     sp.qk_scale_log2 = scale * 1.4426950408889634f;
     if (launch_split(sp, tmK, tmV, s.kv_dtype, D, st) != cudaSuccess) return DECATTN_ECUDA;
   }
@@ -204,8 +191,6 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
     cp.chunk_state = reinterpret_cast<float*>(ws + wl.off_chunk);
     cp.B = s.batch; cp.T = s.q_tokens; cp.Hq = s.n_q_heads; cp.Hkv = s.n_kv_heads; cp.G = G; cp.GT = GT; cp.D = D;
     cp.tl = plan->tile_len;
-    cp.off_pair_off = (int)off_pair_off;
-    cp.off_cb = (int)off_cb;
     if (launch_combine(cp, dev, st) != cudaSuccess) return DECATTN_ECUDA;
   }
   return DECATTN_OK;

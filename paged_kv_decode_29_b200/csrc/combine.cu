@@ -55,10 +55,10 @@ __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_ke
   griddep_wait();  // the split kernel's partials are complete and visible
   const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
   if (hdr->magic != kPlanMagic || hdr->status != DECATTN_OK) return;  // the split kernel reports it
-  const int32_t* cb_g = reinterpret_cast<const int32_t*>(p.plan + p.off_cb);
+  const int32_t* cb_g = plan_arr(p.plan, hdr->off_cb);
+  const int32_t* S = plan_arr(p.plan, hdr->off_S);
   for (int i = threadIdx.x; i <= p.B; i += kCombineThreads) cb_sm[i] = cb_g[i];
   __syncthreads();
-  const int32_t* pair_off = reinterpret_cast<const int32_t*>(p.plan + p.off_pair_off);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t rows_per_b = (int64_t)p.T * p.Hq;
   const int64_t total = rows_per_b * cb_sm[p.B];
@@ -87,7 +87,8 @@ __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_ke
       continue;
     }
     const int h = qh / p.G, r = t * p.G + (qh - h * p.G);
-    const int64_t slot0 = pair_off[(int64_t)b * p.Hkv + h] + (int64_t)j * kCombineChunk;
+    const int nbs = S[b + 1] - S[b];  // == nb
+    const int64_t slot0 = (int64_t)p.Hkv * S[b] + (int64_t)h * nbs + (int64_t)j * kCombineChunk;
     const int n = min(kCombineChunk, nb - j * kCombineChunk);
     // ---- fold up to kCombineChunk partial rows
     const float my_lse = lane < n ? p.part_lse[(slot0 + lane) * p.GT + r] : -INFINITY;

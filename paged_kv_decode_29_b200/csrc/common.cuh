@@ -15,32 +15,92 @@ namespace decattn {
 
 // ------------------------------------------------------------------ plan layout
 // The plan buffer starts with this header; the arrays follow at the byte offsets it
-// records. All offsets are multiples of 32.
+// records (multiples of 32). The work list is stored compactly:
+//  * full tiles (cost tile_len) are dealt round-robin by the greedy rule, so bin k holds
+//    full tiles f = k + n_bins * j for j < full_q + (k < full_r), with f counting the full
+//    tiles in (b, h, i) order; (b, h, i) is recovered from the prefix array SF;
+//  * after them, bin k holds the partial tiles plist[pbin_off[k] .. pbin_off[k + 1]) in
+//    the order they were assigned; partial tile s is head s % Hkv of request
+//    sorted[s / Hkv].
+// plan_unit() decodes the j-th tile of bin k; it is the only reader of this encoding.
 struct PlanHeader {
   int32_t magic;        // kPlanMagic once the planner kernel has written the plan
-  int32_t status;       // DECATTN_OK or a negative device-detected status
-  int32_t n_bins;       // CTAs of the split kernel; bin k is run by CTA k
+  int32_t status;       // DECATTN_OK or a negative device-detected status of the planner
+  int32_t run_status;   // first device-detected error of a split kernel run on this plan (0 = none)
+  int32_t n_bins;       // N: CTAs of the split kernel; bin k is run by CTA k
   int32_t batch;
   int32_t n_kv_heads;
   int32_t tile_len;
-  int32_t n_units;      // tiles in the work list
-  int32_t n_pairs;      // batch * n_kv_heads
-  int64_t max_units;    // capacity of units[]
-  int32_t off_bin_off;  // int32 [n_bins + 1]: CSR offsets of each bin's tiles in units[]
-  int32_t off_pair_off; // int32 [n_pairs + 1]: first partial slot of each (b, h)
-  int32_t off_units;    // Unit [max_units]
-  int32_t off_scratch;  // planner scratch
-  int32_t run_status;   // first device-detected error of a split kernel run on this plan (0 = none)
+  int32_t n_units;      // U: tiles in the work list
+  int32_t n_full;       // F: full tiles
+  int32_t n_partial;    // m: partial tiles (at most one per (b, h))
+  int32_t full_q;       // F / N
+  int32_t full_r;       // F % N
+  int64_t max_units;    // capacity (sizes the workspace's partial slots)
+  int32_t off_S;        // int32 [batch + 1]: prefix over requests of n_b = ceil(L_b / tile_len)
+  int32_t off_SF;       // int32 [batch + 1]: prefix over requests of full tiles floor(L_b / tile_len)
   int32_t off_cb;       // int32 [batch + 1]: prefix over requests of combine chunks per query row
+  int32_t off_sorted;   // int32 [batch]: requests with a partial tile, by cost (desc), then b
+  int32_t off_pbin_off; // int32 [n_bins + 1]: CSR offsets of each bin's partial tiles in plist
+  int32_t off_plist;    // int32 [batch * n_kv_heads]: partial tiles, bin by bin
+  int32_t off_scratch;  // planner scratch
+  int32_t reserved[11];
 };
-static_assert(sizeof(PlanHeader) == 64, "plan header is 64 bytes");
-constexpr int32_t kPlanMagic = 0x31504144;  // "DAP1"
+static_assert(sizeof(PlanHeader) == 128, "plan header is 128 bytes");
+constexpr int32_t kPlanMagic = 0x32504144;  // "DAP2"
 
-// One tile of the work list (32 bytes).
+// One tile of the work list.
 struct Unit {
   int32_t b, h, tok_begin, tok_end, seq_len, slot, tile, zero;
 };
 static_assert(sizeof(Unit) == 32, "unit is 32 bytes");
+
+__device__ __forceinline__ const int32_t* plan_arr(const char* plan, int32_t off) {
+  return reinterpret_cast<const int32_t*>(plan + off);
+}
+
+// Number of tiles in bin k.
+__device__ __forceinline__ int plan_bin_size(const char* plan, const PlanHeader& h, int k) {
+  const int32_t* pbo = plan_arr(plan, h.off_pbin_off);
+  return h.full_q + (k < h.full_r) + pbo[k + 1] - pbo[k];
+}
+
+// The j-th tile of bin k (j < plan_bin_size). A tile of a pair with several tiles writes
+// partial slot S-prefix * Hkv + h * n_b + i; a pair held in one tile gets slot -1.
+__device__ __forceinline__ Unit plan_unit(const char* plan, const PlanHeader& h, const int32_t* seq_lens, int k,
+                                          int j) {
+  const int32_t* S = plan_arr(plan, h.off_S);
+  const int32_t* SF = plan_arr(plan, h.off_SF);
+  const int N = h.n_bins, Hkv = h.n_kv_heads, tl = h.tile_len;
+  const int fc = h.full_q + (k < h.full_r);
+  int b, hh, i, end;
+  if (j < fc) {
+    const int f = k + N * j;
+    int lo = 0, hi = h.batch - 1;  // last request b with Hkv * SF[b] <= f
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (Hkv * SF[mid] <= f) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    const int fb = SF[b + 1] - SF[b];
+    const int r = f - Hkv * SF[b];
+    hh = r / fb;
+    i = r - hh * fb;
+    end = (i + 1) * tl;
+  } else {
+    const int s = plan_arr(plan, h.off_plist)[plan_arr(plan, h.off_pbin_off)[k] + (j - fc)];
+    b = plan_arr(plan, h.off_sorted)[s / Hkv];
+    hh = s % Hkv;
+    i = SF[b + 1] - SF[b];
+    end = seq_lens[b];
+  }
+  const int nb = S[b + 1] - S[b];
+  Unit u;
+  u.b = b; u.h = hh; u.tok_begin = i * tl; u.tok_end = end; u.seq_len = seq_lens[b];
+  u.slot = nb == 1 ? -1 : Hkv * S[b] + hh * nb + i;
+  u.tile = i; u.zero = 0;
+  return u;
+}
 
 // Workspace: a status word, then partial outputs and their LSEs.
 struct WorkspaceHeader {
@@ -53,6 +113,7 @@ static_assert(sizeof(WorkspaceHeader) == 256, "workspace header is 256 bytes");
 struct SplitParams {
   const uint16_t* q;        // bf16 [B][T][Hq][D]
   const int32_t* page_table;
+  const int32_t* seq_lens;  // [B]
   const float* kv_scales;   // [2][num_pages][Hkv] or null
   const char* plan;
   float* out;               // [B][T][Hq][D]
@@ -62,7 +123,6 @@ struct SplitParams {
   int32_t* row_cnt;         // [B*T*Hq] combine counters, zeroed here for the combine that follows
   int32_t* status;          // run status word (plan header)
   int B, T, Hq, Hkv, G, GT, P, num_pages, mpps, n_bins;
-  int off_bin_off, off_units;
   float qk_scale_log2;      // sm_scale * log2(e)
 };
 
@@ -86,7 +146,6 @@ struct CombineParams {
   int32_t* row_cnt;         // [B*T*Hq] chunks of the row folded so far (zeroed by the split kernel)
   float* chunk_state;       // [items][D + 4]: max, weight, -, -, then the weighted sum
   int B, T, Hq, Hkv, G, GT, D, tl;
-  int off_pair_off, off_cb;
 };
 
 __host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }

@@ -11,16 +11,19 @@
 // How the block computes it without a sequential pass over every tile:
 //  * full tiles all cost tile_len and come first in the sorted order, so the greedy pass
 //    deals them round-robin: full tile f (in (b, h, i) order) goes to bin f mod N at
-//    position f div N;
+//    position f div N -- a closed form, so the plan stores only the prefix sums it is
+//    decoded from (plan_unit() in common.cuh);
 //  * after them, bins [F mod N, N) hold the least load; the next N - F mod N tiles (the
 //    largest partial tiles) each find an untouched least-loaded bin, in index order;
 //  * only the remaining partial tiles (at most one per (b, h)) need the sequential
 //    least-loaded search, done by one warp with warp-wide min reductions.
+// The plan's size is O(batch * n_kv_heads + n_bins), independent of the tile count.
 #include "common.cuh"
 
 namespace decattn {
 
 constexpr int kPlanThreads = 512;
+constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kPlanMaxBins = 8192;
 constexpr int kPlanSmemRequests = 4096;  // per-request arrays sit in shared memory up to this batch
 constexpr int kPlanMaxSmem = 200 * 1024;
@@ -33,9 +36,9 @@ struct ReqArrays {
   int32_t *S, *SF, *SP, *plist, *pcost, *sorted_b;
 };
 
-__host__ __device__ inline int64_t plan_bins_smem(int N) { return align_up(12 * (int64_t)N + 4, 16); }
 __host__ __device__ inline int64_t req_stride(int B) { return align_up(4 * (int64_t)(B + 1), 16); }
 __host__ __device__ inline int64_t req_arrays_bytes(int B) { return 6 * req_stride(B); }
+__host__ __device__ inline int64_t plan_bins_smem(int N) { return align_up(12 * (int64_t)N + 4, 16); }
 
 // Global scratch of the plan buffer: the per-request arrays when they do not fit in shared
 // memory, then the bin and in-bin position of every partial tile in greedy order.
@@ -56,7 +59,7 @@ __device__ inline ReqArrays carve_req(char* p, int B) {
 }
 
 // Exclusive block-wide scan of (a, b, c) over kPlanThreads threads; returns the prefix and
-// adds the block totals into tot. warp_tot holds one entry per warp (at most 32 warps).
+// adds the block totals into tot. warp_tot holds one entry per warp.
 struct Tri { long long a, b; int c; };
 
 __device__ inline Tri block_exscan(Tri v, Tri& tot, Tri* warp_tot) {
@@ -72,7 +75,7 @@ __device__ inline Tri block_exscan(Tri v, Tri& tot, Tri* warp_tot) {
   if (lane == 31) warp_tot[w] = inc;
   __syncthreads();
   if (w == 0) {
-    Tri t = lane < kPlanThreads / 32 ? warp_tot[lane] : Tri{0, 0, 0};
+    Tri t = lane < kPlanWarps ? warp_tot[lane] : Tri{0, 0, 0};
     #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       long long a = __shfl_up_sync(0xffffffffu, t.a, o);
@@ -80,11 +83,11 @@ __device__ inline Tri block_exscan(Tri v, Tri& tot, Tri* warp_tot) {
       int c = __shfl_up_sync(0xffffffffu, t.c, o);
       if (lane >= o) { t.a += a; t.b += b; t.c += c; }
     }
-    warp_tot[lane] = t;
+    if (lane < kPlanWarps) warp_tot[lane] = t;
   }
   __syncthreads();
   Tri base = w ? warp_tot[w - 1] : Tri{0, 0, 0};
-  Tri all = warp_tot[kPlanThreads / 32 - 1];
+  Tri all = warp_tot[kPlanWarps - 1];
   __syncthreads();
   Tri ex{base.a + inc.a - v.a, base.b + inc.b - v.b, base.c + inc.c - v.c};
   tot.a += all.a; tot.b += all.b; tot.c += all.c;
@@ -97,7 +100,7 @@ __device__ inline Tri block_exscan(Tri v, Tri& tot, Tri* warp_tot) {
 // bin, the lowest bin index winning ties (lower lanes own lower bins, and each lane keeps
 // its lowest-index minimum). Needs every relative load below 2^27 (checked on the host).
 template <int KMAX>
-__device__ void greedy_partials(int lane, int N, int64_t first, int64_t m, int Hkv, int tl,
+__device__ void greedy_partials(int lane, int N, int first, int m, int Hkv, int tl,
                                 const int32_t* __restrict__ seq_lens, const int32_t* sorted_b, uint32_t* load_sm,
                                 int32_t* pcount_sm, int32_t* part_bin, int32_t* part_pos) {
   const int K = (N + 31) / 32;
@@ -116,15 +119,15 @@ __device__ void greedy_partials(int lane, int N, int64_t first, int64_t m, int H
   #pragma unroll
   for (int j = 1; j < KMAX; ++j)
     if (ld[j] < lmin) { lmin = ld[j]; lj = j; }
-  for (int64_t s0 = first; s0 < m; s0 += 32) {
-    const int64_t sl = s0 + lane;
+  for (int s0 = first; s0 < m; s0 += 32) {
+    const int sl = s0 + lane;
     const uint32_t cl = sl < m ? (uint32_t)(seq_lens[sorted_b[sl / Hkv]] % tl) : 0u;
-    const int n_here = (int)(m - s0 < 32 ? m - s0 : 32);
+    const int n_here = min(32, m - s0);
     for (int i = 0; i < n_here; ++i) {
       const uint32_t c = __shfl_sync(0xffffffffu, cl, i);
       const uint32_t key = __reduce_min_sync(0xffffffffu, (lmin << 5) | (uint32_t)lane);
       if ((int)(key & 31u) == lane) {
-        const int64_t s = s0 + i;
+        const int s = s0 + i;
         part_bin[s] = k0 + lj;
         #pragma unroll
         for (int j = 0; j < KMAX; ++j)
@@ -145,7 +148,7 @@ __device__ void greedy_partials(int lane, int N, int64_t first, int64_t m, int H
 }
 
 // Same rule with the loads in shared memory (more bins than the register version holds).
-__device__ void greedy_partials_smem(int lane, int N, int64_t first, int64_t m, int Hkv, int tl,
+__device__ void greedy_partials_smem(int lane, int N, int first, int m, int Hkv, int tl,
                                      const int32_t* __restrict__ seq_lens, const int32_t* sorted_b, uint32_t* load_sm,
                                      int32_t* pcount_sm, int32_t* part_bin, int32_t* part_pos) {
   const int K = (N + 31) / 32;
@@ -154,15 +157,15 @@ __device__ void greedy_partials_smem(int lane, int N, int64_t first, int64_t m, 
   int lk = k0;
   for (int k = k0; k < k1; ++k)
     if (load_sm[k] < lmin) { lmin = load_sm[k]; lk = k; }
-  for (int64_t s0 = first; s0 < m; s0 += 32) {
-    const int64_t sl = s0 + lane;
+  for (int s0 = first; s0 < m; s0 += 32) {
+    const int sl = s0 + lane;
     const uint32_t cl = sl < m ? (uint32_t)(seq_lens[sorted_b[sl / Hkv]] % tl) : 0u;
-    const int n_here = (int)(m - s0 < 32 ? m - s0 : 32);
+    const int n_here = min(32, m - s0);
     for (int i = 0; i < n_here; ++i) {
       const uint32_t c = __shfl_sync(0xffffffffu, cl, i);
       const uint32_t key = __reduce_min_sync(0xffffffffu, (lmin << 5) | (uint32_t)lane);
       if ((int)(key & 31u) == lane) {
-        const int64_t s = s0 + i;
+        const int s = s0 + i;
         part_bin[s] = lk;
         part_pos[s] = pcount_sm[lk]++;
         load_sm[lk] += c;
@@ -179,22 +182,23 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
   // the split kernel may start its prologue now; it waits for this grid before reading the plan
   griddep_launch_dependents();
   const int B = init.batch, Hkv = init.n_kv_heads, tl = init.tile_len, N = init.n_bins;
-  const int64_t max_units = init.max_units;
   extern __shared__ __align__(16) uint8_t plan_smem[];
-  uint32_t* load = reinterpret_cast<uint32_t*>(plan_smem);                 // [N] load above the full-tile base
+  uint32_t* load = reinterpret_cast<uint32_t*>(plan_smem);                   // [N] load above the full-tile base
   int32_t* pcount = reinterpret_cast<int32_t*>(plan_smem + 4 * (int64_t)N);  // [N] partial tiles per bin
-  int32_t* boff = reinterpret_cast<int32_t*>(plan_smem + 8 * (int64_t)N);    // [N + 1] CSR offsets
-  __shared__ Tri warp_tot[32];
+  __shared__ Tri warp_tot[kPlanWarps];
   __shared__ int32_t sh_status;
 
   PlanHeader* hdr = reinterpret_cast<PlanHeader*>(plan);
-  int32_t* bin_off = reinterpret_cast<int32_t*>(plan + init.off_bin_off);
-  int32_t* pair_off = reinterpret_cast<int32_t*>(plan + init.off_pair_off);
-  int32_t* cbuf = reinterpret_cast<int32_t*>(plan + init.off_cb);
-  Unit* units = reinterpret_cast<Unit*>(plan + init.off_units);
+  int32_t* gS = reinterpret_cast<int32_t*>(plan + init.off_S);
+  int32_t* gSF = reinterpret_cast<int32_t*>(plan + init.off_SF);
+  int32_t* gcb = reinterpret_cast<int32_t*>(plan + init.off_cb);
+  int32_t* gsorted = reinterpret_cast<int32_t*>(plan + init.off_sorted);
+  int32_t* gpbo = reinterpret_cast<int32_t*>(plan + init.off_pbin_off);
+  int32_t* gplist = reinterpret_cast<int32_t*>(plan + init.off_plist);
   char* gscratch = plan + init.off_scratch;
-  const ReqArrays R = carve_req(B <= kPlanSmemRequests ? reinterpret_cast<char*>(plan_smem + plan_bins_smem(N))
-                                                       : gscratch, B);
+  const bool req_in_smem = B <= kPlanSmemRequests;
+  ReqArrays R = carve_req(req_in_smem ? reinterpret_cast<char*>(plan_smem + plan_bins_smem(N)) : gscratch, B);
+  if (!req_in_smem) { R.S = gS; R.SF = gSF; R.sorted_b = gsorted; }
   int32_t* part_bin = reinterpret_cast<int32_t*>(gscratch + req_arrays_bytes(B));
   int32_t* part_pos = part_bin + align_up((int64_t)B * Hkv, 8);
   const int tid = threadIdx.x;
@@ -223,15 +227,11 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
     }
   }
   if (tid == 0) { R.S[B] = (int32_t)carry.a; R.SF[B] = (int32_t)carry.b; R.SP[B] = carry.c; }
-  const int64_t U = (int64_t)Hkv * carry.a;
-  const int64_t F = (int64_t)Hkv * carry.b;
-  const int mB = carry.c;
-  const int64_t m = (int64_t)Hkv * mB;
+  const int64_t U64 = (int64_t)Hkv * carry.a;
   __syncthreads();
-  if (U > max_units) atomicCAS(&sh_status, 0, DECATTN_ECAPACITY);
+  if (U64 > init.max_units) atomicCAS(&sh_status, 0, DECATTN_ECAPACITY);
   __syncthreads();
   if (sh_status != 0) {
-    for (int k = tid; k <= N; k += kPlanThreads) bin_off[k] = 0;
     if (tid == 0) {
       hdr->n_units = 0;
       hdr->status = sh_status;
@@ -240,6 +240,10 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
     }
     return;
   }
+  const int U = (int)U64;  // < 2^31 from here on: the capacity is checked against that on the host
+  const int F = (int)((int64_t)Hkv * carry.b);
+  const int mB = carry.c;
+  const int m = Hkv * mB;
 
   // ---- 2. combine chunks per query row of each request, and their prefix over requests
   {
@@ -249,9 +253,9 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
       const long long cb = b < B ? combine_chunks(R.S[b + 1] - R.S[b]) : 0;
       Tri before = c3;
       Tri ex = block_exscan(Tri{cb, 0, 0}, c3, warp_tot);
-      if (b < B) cbuf[b] = (int32_t)(before.a + ex.a);
+      if (b < B) gcb[b] = (int32_t)(before.a + ex.a);
     }
-    if (tid == 0) cbuf[B] = (int32_t)c3.a;
+    if (tid == 0) gcb[B] = (int32_t)c3.a;
   }
 
   // ---- 3. requests with a partial tile, sorted by cost (desc), then b: rank by counting
@@ -268,15 +272,15 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
 
   // ---- 4. greedy placement of the partial tiles (s-th in sorted order: request
   //         sorted_b[s / Hkv], head s % Hkv)
-  const int64_t qf = F / N;
-  const int rf = (int)(F % N);
-  const int64_t first = m < (int64_t)(N - rf) ? m : (int64_t)(N - rf);
+  const int qf = F / N;
+  const int rf = F - qf * N;
+  const int first = min(m, N - rf);
   for (int k = tid; k < N; k += kPlanThreads) {
     uint32_t l = k < rf ? (uint32_t)tl : 0u;
     int32_t pc = 0;
-    const int64_t s = k - rf;
+    const int s = k - rf;
     if (k >= rf && s < first) {
-      l += (uint32_t)(seq_lens[R.sorted_b[(int)s / Hkv]] % tl);
+      l += (uint32_t)(seq_lens[R.sorted_b[s / Hkv]] % tl);
       pc = 1;
       part_bin[s] = k;
       part_pos[s] = 0;
@@ -287,8 +291,8 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
   __syncthreads();
   if (tid < 32 && first < m) {
     const int K = (N + 31) / 32;
-    #define DECATTN_GREEDY(KM) greedy_partials<KM>(tid, N, first, m, Hkv, tl, seq_lens, R.sorted_b, load, pcount, \
-                                                    part_bin, part_pos)
+#define DECATTN_GREEDY(KM) \
+  greedy_partials<KM>(tid, N, first, m, Hkv, tl, seq_lens, R.sorted_b, load, pcount, part_bin, part_pos)
     if (K <= 4) DECATTN_GREEDY(4);
     else if (K <= 8) DECATTN_GREEDY(8);
     else if (K <= 12) DECATTN_GREEDY(12);
@@ -297,85 +301,89 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
     else if (K <= 24) DECATTN_GREEDY(24);
     else if (K <= 32) DECATTN_GREEDY(32);
     else greedy_partials_smem(tid, N, first, m, Hkv, tl, seq_lens, R.sorted_b, load, pcount, part_bin, part_pos);
-    #undef DECATTN_GREEDY
+#undef DECATTN_GREEDY
   }
   __syncthreads();
 
-  // ---- 5. bin offsets (CSR): full tiles of bin k, then its partial tiles
+  // ---- 5. per-bin CSR offsets of the partial tiles, and the partial tiles bin by bin
   {
     Tri c2{0, 0, 0};
     for (int base = 0; base < N; base += kPlanThreads) {
       const int k = base + tid;
-      const long long cnt = k < N ? (long long)(qf + (k < rf)) + pcount[k] : 0;
       Tri before = c2;
-      Tri ex = block_exscan(Tri{cnt, 0, 0}, c2, warp_tot);
-      if (k < N) bin_off[k] = boff[k] = (int32_t)(before.a + ex.a);
+      Tri ex = block_exscan(Tri{k < N ? pcount[k] : 0, 0, 0}, c2, warp_tot);
+      if (k < N) gpbo[k] = (int32_t)(before.a + ex.a);
     }
-    if (tid == 0) bin_off[N] = boff[N] = (int32_t)c2.a;
+    if (tid == 0) gpbo[N] = (int32_t)c2.a;
   }
   __syncthreads();
+  for (int s = tid; s < m; s += kPlanThreads) gplist[gpbo[part_bin[s]] + part_pos[s]] = s;
 
-  // ---- 6. the tiles. Warp w takes pairs p = w, w + 32, ...; lane l writes the pair's full
-  //         tiles i = l, l + 32, ...; full tile f = Hkv*SF[b] + h*fb + i goes to bin f mod N at
-  //         position f div N (kept incrementally: all indices fit in 32 bits, U < 2^31).
-  {
-    const int warp = tid >> 5, lane = tid & 31;
-    const int n_pairs = B * Hkv;
-    for (int pr = warp; pr < n_pairs; pr += kPlanThreads / 32) {
-      const int b = pr / Hkv, h = pr - b * Hkv;
-      const int fb = R.SF[b + 1] - R.SF[b];
-      const int nb = R.S[b + 1] - R.S[b];
-      const int32_t L = seq_lens[b];
-      const int slot0 = Hkv * R.S[b] + h * nb;
-      if (lane == 0) pair_off[pr] = slot0;
-      const int f0 = Hkv * R.SF[b] + h * fb + lane;
-      int q = (int)((unsigned)f0 / (unsigned)N), r = f0 - q * N;
-      const int step_q = 32 / N, step_r = 32 - step_q * N;
-      for (int i = lane; i < fb; i += 32) {
-        Unit u;
-        u.b = b; u.h = h; u.tok_begin = i * tl; u.tok_end = (i + 1) * tl; u.seq_len = L;
-        u.slot = nb == 1 ? -1 : slot0 + i;
-        u.tile = i; u.zero = 0;
-        units[boff[r] + q] = u;
-        q += step_q; r += step_r;
-        if (r >= N) { r -= N; ++q; }
-      }
-    }
-    if (tid == 0) pair_off[n_pairs] = (int32_t)U;
-  }
-  for (int s = tid; s < (int)m; s += kPlanThreads) {
-    const int b = R.sorted_b[s / Hkv], h = s % Hkv;
-    const int fb = R.SF[b + 1] - R.SF[b];
-    const int nb = R.S[b + 1] - R.S[b];
-    const int32_t L = seq_lens[b];
-    Unit u;
-    u.b = b; u.h = h; u.tok_begin = fb * tl; u.tok_end = L; u.seq_len = L;
-    u.slot = nb == 1 ? -1 : Hkv * R.S[b] + h * nb + fb;
-    u.tile = fb; u.zero = 0;
-    const int k = part_bin[s];
-    units[boff[k] + (int)(qf + (k < rf)) + part_pos[s]] = u;
+  // ---- 6. publish the per-request arrays the decoder reads
+  if (req_in_smem) {
+    for (int b = tid; b <= B; b += kPlanThreads) { gS[b] = R.S[b]; gSF[b] = R.SF[b]; }
+    for (int j = tid; j < mB; j += kPlanThreads) gsorted[j] = R.sorted_b[j];
   }
   __syncthreads();
   if (tid == 0) {
-    hdr->n_units = (int32_t)U;
+    hdr->n_units = U;
+    hdr->n_full = F;
+    hdr->n_partial = m;
+    hdr->full_q = qf;
+    hdr->full_r = rf;
     hdr->status = DECATTN_OK;
     __threadfence();
     hdr->magic = kPlanMagic;
   }
 }
 
+// Writes the explicit work list of a finished plan: bin_off [N+1] and units [U] (CSR by
+// bin), decoded with the same plan_unit() the split kernel uses. One block; for tests and
+// diagnostics.
+__global__ void __launch_bounds__(1024)
+plan_export_kernel(const char* __restrict__ plan, const int32_t* __restrict__ seq_lens, int32_t* bin_off,
+                   Unit* units, int64_t max_units, int32_t* n_out) {
+  const PlanHeader h = *reinterpret_cast<const PlanHeader*>(plan);
+  __shared__ long long carry;
+  __shared__ long long part[1024];
+  const bool ok = h.magic == kPlanMagic && h.status == DECATTN_OK && h.n_units <= max_units;
+  if (threadIdx.x == 0) { carry = 0; *n_out = ok ? h.n_units : -1; }
+  __syncthreads();
+  if (!ok) return;
+  for (int base = 0; base < h.n_bins; base += 1024) {
+    const int k = base + threadIdx.x;
+    part[threadIdx.x] = k < h.n_bins ? plan_bin_size(plan, h, k) : 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      long long run = carry;
+      for (int i = 0; i < 1024; ++i) { const long long v = part[i]; part[i] = run; run += v; }
+      carry = run;
+    }
+    __syncthreads();
+    if (k < h.n_bins) {
+      bin_off[k] = (int32_t)part[threadIdx.x];
+      const int n = plan_bin_size(plan, h, k);
+      for (int j = 0; j < n; ++j) units[part[threadIdx.x] + j] = plan_unit(plan, h, seq_lens, k, j);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) bin_off[h.n_bins] = (int32_t)carry;
+}
+
 // ------------------------------------------------------------------ host side
 struct PlanLayout {
-  int64_t off_bin_off, off_pair_off, off_cb, off_units, off_scratch, total;
+  int64_t off_S, off_SF, off_cb, off_sorted, off_pbin_off, off_plist, off_scratch, total;
 };
 
-static PlanLayout plan_layout(int B, int Hkv, int N, int64_t max_units) {
+static PlanLayout plan_layout(int B, int Hkv, int N) {
   PlanLayout L;
   int64_t o = sizeof(PlanHeader);
-  L.off_bin_off = o; o = align_up(o + 4 * (int64_t)(N + 1), 32);
-  L.off_pair_off = o; o = align_up(o + 4 * ((int64_t)B * Hkv + 1), 32);
+  L.off_S = o; o = align_up(o + 4 * ((int64_t)B + 1), 32);
+  L.off_SF = o; o = align_up(o + 4 * ((int64_t)B + 1), 32);
   L.off_cb = o; o = align_up(o + 4 * ((int64_t)B + 1), 32);
-  L.off_units = o; o = align_up(o + (int64_t)sizeof(Unit) * max_units, 32);
+  L.off_sorted = o; o = align_up(o + 4 * ((int64_t)B + 1), 32);
+  L.off_pbin_off = o; o = align_up(o + 4 * ((int64_t)N + 1), 32);
+  L.off_plist = o; o = align_up(o + 4 * ((int64_t)B * Hkv + 1), 32);
   L.off_scratch = o; o = align_up(o + plan_scratch_bytes(B, Hkv), 32);
   L.total = o;
   return L;
@@ -385,11 +393,12 @@ static int64_t plan_capacity(int B, int Hkv, int tl, int64_t max_total) {
   return (int64_t)Hkv * ((max_total + tl - 1) / tl + B);
 }
 
-
 static bool plan_args_ok(int B, int Hkv, int tl, int64_t max_total, int N) {
   if (B < 0 || Hkv <= 0 || tl <= 0 || (tl % 16) != 0 || max_total < 0 || N <= 0 || N > kPlanMaxBins) return false;
   const int64_t cap = plan_capacity(B, Hkv, tl, max_total);
   if (cap >= (1ll << 31) - 1 || max_total >= (1ll << 31)) return false;
+  if ((int64_t)B * Hkv >= (1ll << 28)) return false;
+  if (plan_layout(B, Hkv, N).total >= (1ll << 31)) return false;
   // keeps every relative bin load of the greedy pass below 2^27 (its packed min key)
   if ((double)B * Hkv * tl / N + 2.0 * tl >= 134217727.0) return false;
   return true;
@@ -407,8 +416,7 @@ extern "C" size_t dec_attn_plan_bytes(int batch, int n_kv_heads, int tile_len, i
     n_bins = default_bins(dev);
   }
   if (!plan_args_ok(batch, n_kv_heads, tile_len, max_total_kv_tokens, n_bins)) return 0;
-  const int64_t cap = plan_capacity(batch, n_kv_heads, tile_len, max_total_kv_tokens);
-  return (size_t)plan_layout(batch, n_kv_heads, n_bins, cap).total;
+  return (size_t)plan_layout(batch, n_kv_heads, n_bins).total;
 }
 
 extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads, int tile_len,
@@ -425,26 +433,25 @@ extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads,
   if (!plan_args_ok(batch, n_kv_heads, tile_len, max_total_kv_tokens, n_bins)) return DECATTN_ENOTSUP;
   if ((reinterpret_cast<uintptr_t>(plan_buf) & 15) != 0) return DECATTN_EALIGN;
   const int64_t cap = plan_capacity(batch, n_kv_heads, tile_len, max_total_kv_tokens);
-  const PlanLayout L = plan_layout(batch, n_kv_heads, n_bins, cap);
+  const PlanLayout L = plan_layout(batch, n_kv_heads, n_bins);
   if ((int64_t)plan_bytes < L.total) return DECATTN_ESMALL;
 
   PlanHeader h{};
-  h.magic = 0;
-  h.status = DECATTN_OK;
   h.n_bins = n_bins;
   h.batch = batch;
   h.n_kv_heads = n_kv_heads;
   h.tile_len = tile_len;
-  h.n_units = 0;
-  h.n_pairs = batch * n_kv_heads;
   h.max_units = cap;
-  h.off_bin_off = (int32_t)L.off_bin_off;
-  h.off_pair_off = (int32_t)L.off_pair_off;
-  h.off_units = (int32_t)L.off_units;
-  h.off_scratch = (int32_t)L.off_scratch;
+  h.off_S = (int32_t)L.off_S;
+  h.off_SF = (int32_t)L.off_SF;
   h.off_cb = (int32_t)L.off_cb;
+  h.off_sorted = (int32_t)L.off_sorted;
+  h.off_pbin_off = (int32_t)L.off_pbin_off;
+  h.off_plist = (int32_t)L.off_plist;
+  h.off_scratch = (int32_t)L.off_scratch;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t smem = (size_t)plan_bins_smem(n_bins) + (batch <= kPlanSmemRequests ? (size_t)req_arrays_bytes(batch) : 0);
+  const size_t smem =
+      (size_t)plan_bins_smem(n_bins) + (batch <= kPlanSmemRequests ? (size_t)req_arrays_bytes(batch) : 0);
   if (!ensure_smem_attr((const void*)plan_kernel, kPlanMaxSmem)) return DECATTN_ECUDA;
   plan_kernel<<<1, kPlanThreads, smem, st>>>(seq_lens, h, static_cast<char*>(plan_buf));
   if (cudaGetLastError() != cudaSuccess) return DECATTN_ECUDA;
@@ -456,4 +463,13 @@ extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads,
   plan->n_bins = n_bins;
   plan->max_units = cap;
   return DECATTN_OK;
+}
+
+extern "C" int dec_attn_plan_export(const dec_attn_plan_t* plan, const int32_t* seq_lens, int32_t* bin_off,
+                                    void* units, int64_t max_units, int32_t* n_units, void* stream) {
+  if (!plan || !plan->buf || !bin_off || !units || !n_units || (plan->batch > 0 && !seq_lens) || max_units < 0)
+    return DECATTN_EINVAL;
+  plan_export_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const char*>(plan->buf), seq_lens, bin_off, static_cast<Unit*>(units), max_units, n_units);
+  return cudaGetLastError() == cudaSuccess ? DECATTN_OK : DECATTN_ECUDA;
 }

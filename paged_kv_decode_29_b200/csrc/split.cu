@@ -110,9 +110,8 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
                            : hdr->status != DECATTN_OK ? hdr->status : DECATTN_EINVAL);
     return;
   }
-  const int32_t* bin_off = reinterpret_cast<const int32_t*>(p.plan + p.off_bin_off);
-  const Unit* units = reinterpret_cast<const Unit*>(p.plan + p.off_units);
-  const int u0 = bin_off[blockIdx.x], u1 = bin_off[blockIdx.x + 1];
+  const PlanHeader hv = *hdr;
+  const int n_units = plan_bin_size(p.plan, hv, blockIdx.x);  // tiles of this CTA's bin
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 32); }
@@ -120,7 +119,7 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
     fence_mbar_init();
   }
   __syncthreads();
-  if (u0 >= u1) return;
+  if (n_units == 0) return;
 
   if (warp == 0) {
     // ===================================================================== producer
@@ -131,19 +130,19 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
     bool ok = true;
     int64_t n_fill = 0, n_qfill = 0;  // copies issued so far (ring stages, q slots)
     // tile descriptors run two tiles ahead and page ids one tile ahead of the copies
-    Unit dn = units[u0];
-    Unit dnn = u0 + 1 < u1 ? units[u0 + 1] : dn;
+    Unit dn = plan_unit(p.plan, hv, p.seq_lens, blockIdx.x, 0);
+    Unit dnn = n_units > 1 ? plan_unit(p.plan, hv, p.seq_lens, blockIdx.x, 1) : dn;
     int pid_next;
     {
       const int pg0 = dn.tok_begin / P, npg = (dn.tok_end - dn.tok_begin + P - 1) / P;
       pid_next = lane < npg ? p.page_table[(int64_t)dn.b * p.mpps + min(pg0 + lane, p.mpps - 1)] : 0;
     }
-    for (int u = u0; u < u1 && ok; ++u) {
+    for (int u = 0; u < n_units && ok; ++u) {
       const Unit d = dn;
       int pid_l = pid_next;
       dn = dnn;
-      if (u + 2 < u1) dnn = units[u + 2];
-      if (u + 1 < u1) {
+      if (u + 2 < n_units) dnn = plan_unit(p.plan, hv, p.seq_lens, blockIdx.x, u + 2);
+      if (u + 1 < n_units) {
         const int pg0 = dn.tok_begin / P, npg = (dn.tok_end - dn.tok_begin + P - 1) / P;
         pid_next = lane < npg ? p.page_table[(int64_t)dn.b * p.mpps + min(pg0 + lane, p.mpps - 1)] : 0;
       }
@@ -216,7 +215,7 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   int s = 0; uint32_t fph = 0;
   int qs = 0; uint32_t qfph = 0;
   const float LN2 = 0.6931471805599453f;
-  for (int u = u0; u < u1; ++u) {
+  for (int u = 0; u < n_units; ++u) {
     if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qs], qfph, p.status))) return;
     const Unit d = qmeta[qs];
     // ---- q fragments (B operand of S^T = K Q^T): column n = query row

@@ -49,7 +49,10 @@ def test_status_strings(lib):
 
 def test_plan_bytes_host_only(lib):
     n = lib.dec_attn_plan_bytes(32, 8, 256, 32 * 4096, 592)
-    assert n > 32 * 4096 // 256 * 8 * 32  # holds the tile list
+    assert 0 < n < 64 * 1024
+    # full tiles are stored in closed form: the plan does not grow with the KV length
+    assert lib.dec_attn_plan_bytes(32, 8, 256, 32 * 4096 * 100, 592) == n
+    assert lib.dec_attn_plan_bytes(64, 8, 256, 1000, 592) > n
     assert lib.dec_attn_plan_bytes(32, 8, 250, 1000, 592) == 0      # tile not a multiple of 16
     assert lib.dec_attn_plan_bytes(-1, 8, 256, 1000, 592) == 0
     assert lib.dec_attn_plan_bytes(4, 0, 256, 1000, 592) == 0
