@@ -171,6 +171,31 @@ DECATTN_API int dec_attn_run(const dec_attn_shape *shape, const void *q, const v
                  const dec_attn_plan_t *plan, void *workspace, size_t workspace_bytes, float *out, float *lse,
                  void *stream);
 
+/* Size of the fixed device scratch behind dec_attn_run_noalloc: 64 MiB per GPU. */
+#define DECATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* dec_attn_run without a caller-supplied workspace, for callers that cannot allocate device
+ * memory: a plugin hosted by an engine that owns all device memory through its own pool and
+ * offers no allocation hook, or a deployment that fixes its device memory budget up front and
+ * forbids allocation while decoding. It allocates nothing (no cudaMalloc / cudaFree, no
+ * allocating library call): the workspace is a file-scope device array of
+ * DECATTN_NOALLOC_SCRATCH_BYTES inside this library. The pages describe no such variant; it
+ * is a deployment convenience of this library.
+ *   Arguments, results and errors as dec_attn_run, minus workspace / workspace_bytes.
+ *   DECATTN_ESMALL if dec_attn_workspace_bytes(shape, plan) exceeds the scratch (nothing is
+ *   enqueued then); DECATTN_ECUDA if the scratch's device address cannot be looked up.
+ *   The first call on a device (with that device current) looks up the array's device address
+ *   and loads the module that holds it; make that first call before any stream capture. The
+ *   array then stays allocated on that GPU until the process exits.
+ *   All calls on one device share the array; its contents are left over from the last call and
+ *   need no clearing (the split kernel writes every partial the combine reads and resets the
+ *   combine counters). Calls whose work overlaps on the GPU (e.g. on two streams) race on it:
+ *   serialise them. */
+DECATTN_API int dec_attn_run_noalloc(const dec_attn_shape *shape, const void *q, const void *k_pages,
+                                     const void *v_pages, const int32_t *page_table, const int32_t *seq_lens,
+                                     const float *kv_scales, const dec_attn_plan_t *plan, float *out, float *lse,
+                                     void *stream);
+
 /* The two stages of dec_attn_run as separate calls (same arguments, same checks):
  * dec_attn_split enqueues only the split kernel, dec_attn_combine only the combine
  * kernel, which reads the partials the split kernel left in `workspace`. dec_attn_run(...) == dec_attn_split(...) followed by

@@ -27,8 +27,9 @@ LIB_PATH = os.path.join(_HERE, "libdecattn.so")
 OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1, -2, -3, -4, -5, -6, -7, -8
 KV_BF16, KV_FP8E4M3 = 0, 1
 API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
-       "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_read_status",
-       "dec_attn_status_string")
+       "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
+       "dec_attn_read_status", "dec_attn_status_string")
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class DecAttnError(RuntimeError):
@@ -77,6 +78,8 @@ def load_library(path: str = LIB_PATH):
             f = getattr(lib, name)
             f.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, C.POINTER(PlanT), vp, sz, vp, vp, vp]
             f.restype = i32
+        lib.dec_attn_run_noalloc.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, C.POINTER(PlanT), vp, vp, vp]
+        lib.dec_attn_run_noalloc.restype = i32
         lib.dec_attn_read_status.argtypes = [C.POINTER(PlanT), vp, vp]
         lib.dec_attn_read_status.restype = i32
         lib.dec_attn_status_string.argtypes = [i32]
@@ -200,6 +203,23 @@ def run(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_tabl
             _stream_handle(stream))
     if rc != OK:
         raise DecAttnError(rc, f"dec_attn_{stage}")
+    return out, lse
+
+
+def run_noalloc(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_table: torch.Tensor,
+                seq_lens: torch.Tensor, pl: Plan, out: torch.Tensor, lse: torch.Tensor, *,
+                kv_scales: torch.Tensor | None = None, sm_scale: float = 0.0, stream=None):
+    """dec_attn_run_noalloc: split + combine using the library's fixed 64 MiB device scratch instead
+    of a caller workspace, for callers that cannot allocate device memory. ``out`` and ``lse`` are
+    caller-provided (this wrapper allocates nothing either). Calls overlapping on the GPU race on the
+    shared scratch."""
+    lib = load_library()
+    shape = make_shape(q, k_pages, page_table, kv_dtype_of(k_pages), sm_scale)
+    rc = lib.dec_attn_run_noalloc(C.byref(shape), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
+                                  _ptr(seq_lens), _ptr(kv_scales), C.byref(pl.handle), _ptr(out), _ptr(lse),
+                                  _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_run_noalloc")
     return out, lse
 
 
