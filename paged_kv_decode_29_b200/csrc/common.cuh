@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -316,14 +317,11 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return d;
 }
 
-// Two OCP E4M3 codes sitting in bytes 1 and 3 of x -> f16x2 holding code * 2^-8 each
-// (low half from byte 1, high half from byte 3); bytes 0 and 2 are ignored.
-// An E4M3 code s.eeee.mmm and the f16 s.0eeee.mmm0000000 have the same sign, exponent
-// field and mantissa bits; the exponent biases (7 vs 15) differ by 8, so the f16 value
-// is exactly code * 2^-8, subnormals included (both formats read exponent field 0 as
-// 2^(1-bias) with no implicit bit). The 2^8 goes into the per-page scale.
-__device__ __forceinline__ uint32_t e4m3x2_hi_bytes_to_f16x2(uint32_t x) {
-  return (x & 0x80008000u) | ((x >> 1) & 0x3F803F80u);
+// Two OCP E4M3 codes (low byte -> low half) -> f16x2 with the same values (every finite
+// E4M3 value is exact in f16). CUDA's conversion, one hardware convert on sm_89 and later.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {

@@ -8,13 +8,14 @@
 // Library for LLM Inference Hot Paths", "How the kernels are organized around specific
 // workload shapes": uniform tiles balanced across CTAs, a combine merges the splits).
 //
-// CTA = 2 warps.
+// CTA = 1 producer warp + NCW consumer warps.
 //  * warp 0 (producer): reads the bin's tile list and page-table rows, and for every
 //    16-key block issues two 2-D TMA copies (K rows, V rows) of one (page, KV head) into
 //    the next ring stage; the tile's q rows go to a double-buffered q slot by bulk copy;
 //    FP8 page scales ride along as 4-byte cp.async copies folded into the stage's
 //    mbarrier. It waits only on "stage empty" barriers, so it runs ahead of the math.
-//  * warp 1 (consumer): per 16-key block, S^T = K Q^T on tensor cores with the keys on
+//  * warps 1..NCW (consumers; with NCW = 2 each takes one 8-row half of the G*T query rows
+//    and both read the same staged K/V): per 16-key block, S^T = K Q^T on tensor cores with the keys on
 //    the MMA's M side ("SwapAB", as in the pages' Attention SwapAB), so a G*T of 4..16
 //    query rows fills N = 8 or 16 instead of padding M to 16; then an online softmax in
 //    fp32 (log2 domain), then O^T += V^T P^T (again keys as the contraction, head_dim on
@@ -31,7 +32,9 @@
 namespace decattn {
 
 
-constexpr int kSplitThreads = 64;
+// FP8 KV: P is multiplied by (V page scale * kPScale) before its f16 rounding, so that small
+// probabilities stay normal f16 numbers; the epilogue divides kPScale back out.
+constexpr float kPScale = 256.f;
 constexpr int kCtasPerSm = 4;
 
 template <int KVT, int D>
@@ -78,13 +81,17 @@ __device__ __forceinline__ int qrow_of_col(int n, int GT) {
 }
 
 // KVT: 0 = bf16 KV, 1 = FP8 E4M3 KV.  NQ: 8-column tiles of S^T.  NPV: 8-column tiles of
-// O^T.  DUP: bf16 with G*T <= 4 (hi in columns 0..3, lo in 4..7 of one tile).
-template <int KVT, int D, int NQ, int NPV, bool DUP>
-__global__ void __launch_bounds__(kSplitThreads, kCtasPerSm)
+// O^T.  DUP: bf16 with G*T <= 4 (hi in columns 0..3, lo in 4..7 of one tile).  NCW: consumer
+// warps; consumer w owns S^T tiles [w*NQ/NCW, (w+1)*NQ/NCW) and the O^T tiles that go with them.
+template <int KVT, int D, int NQ, int NPV, bool DUP, int NCW>
+__global__ void __launch_bounds__(32 * (1 + NCW), kCtasPerSm)
 split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   using G_ = Geo<KVT, D>;
   using S_ = Smem<KVT, D, NQ>;
   constexpr int STAGES = G_::STAGES;
+  constexpr int NQW = NQ / NCW;    // S^T tiles per consumer warp
+  constexpr int NPVW = NPV / NCW;  // O^T tiles per consumer warp
+  static_assert(NQ % NCW == 0 && NPV % NCW == 0, "tiles split evenly over the consumer warps");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + S_::OFF_BAR);
@@ -99,8 +106,8 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   griddep_launch_dependents();  // the combine kernel may be scheduled; it waits for this grid
   griddep_wait();               // the plan kernel has finished and its writes are visible
   // the combine counters of this workspace start from zero on every run
-  for (int64_t i = (int64_t)blockIdx.x * kSplitThreads + threadIdx.x; i < (int64_t)p.B * p.T * p.Hq;
-       i += (int64_t)gridDim.x * kSplitThreads)
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)p.B * p.T * p.Hq;
+       i += (int64_t)gridDim.x * blockDim.x)
     p.row_cnt[i] = 0;
   const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
   if (hdr->magic != kPlanMagic || hdr->status != DECATTN_OK || hdr->n_bins != (int)gridDim.x ||
@@ -114,8 +121,8 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   const int n_units = plan_bin_size(p.plan, hv, blockIdx.x);  // tiles of this CTA's bin
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 32); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 32); }
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 32 * NCW); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 32 * NCW); }
     fence_mbar_init();
   }
   __syncthreads();
@@ -212,6 +219,7 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
 
   // ======================================================================= consumer
   const int gid = lane >> 2, tig = lane & 3;
+  const int nq0 = (warp - 1) * NQW;  // first S^T tile of this consumer warp
   int s = 0; uint32_t fph = 0;
   int qs = 0; uint32_t qfph = 0;
   const float LN2 = 0.6931471805599453f;
@@ -219,26 +227,26 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
     if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qs], qfph, p.status))) return;
     const Unit d = qmeta[qs];
     // ---- q fragments (B operand of S^T = K Q^T): column n = query row
-    uint32_t qf[NQ][D / 16][2];
+    uint32_t qf[NQW][D / 16][2];
     {
       const uint8_t* qsm = sm + S_::OFF_Q + qs * S_::QBYTES;
       #pragma unroll
-      for (int nq = 0; nq < NQ; ++nq) {
-        const int r = qrow_of_col<DUP>(8 * nq + gid, p.GT);
+      for (int nw = 0; nw < NQW; ++nw) {
+        const int r = qrow_of_col<DUP>(8 * (nq0 + nw) + gid, p.GT);
         const uint16_t* qr = reinterpret_cast<const uint16_t*>(qsm) + (r < 0 ? 0 : r) * D;
         #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           if (KVT == 0) {
             const uint32_t x0 = *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * tig);
             const uint32_t x1 = *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 8 + 2 * tig);
-            qf[nq][kk][0] = r < 0 ? 0u : x0;
-            qf[nq][kk][1] = r < 0 ? 0u : x1;
+            qf[nw][kk][0] = r < 0 ? 0u : x0;
+            qf[nw][kk][1] = r < 0 ? 0u : x1;
           } else {
             // FP8 K is read 4 consecutive codes per thread: logical k = 2*tig + {0,1} holds
             // d = 16kk + 4tig + {0,1}, logical k = 8 + 2*tig + {0,1} holds d = 16kk + 4tig + {2,3}
             const uint2 x = *reinterpret_cast<const uint2*>(qr + 16 * kk + 4 * tig);
-            qf[nq][kk][0] = r < 0 ? 0u : pack_f16(bf16_lo(x.x), bf16_hi(x.x));
-            qf[nq][kk][1] = r < 0 ? 0u : pack_f16(bf16_lo(x.y), bf16_hi(x.y));
+            qf[nw][kk][0] = r < 0 ? 0u : pack_f16(bf16_lo(x.x), bf16_hi(x.x));
+            qf[nw][kk][1] = r < 0 ? 0u : pack_f16(bf16_lo(x.y), bf16_hi(x.y));
           }
         }
       }
@@ -248,28 +256,28 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
     qs ^= 1; if (qs == 0) qfph ^= 1;
 
     // ---- per-column limits: key j is visible to query token t if j <= Lb - T + t
-    int lim[NQ][2];
+    int lim[NQW][2];
     #pragma unroll
-    for (int nq = 0; nq < NQ; ++nq)
+    for (int nw = 0; nw < NQW; ++nw)
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int r = qrow_of_col<DUP>(8 * nq + 2 * tig + e, p.GT);
-        lim[nq][e] = r < 0 ? 0x7fffffff : d.seq_len - p.T + r / p.G;
+        const int r = qrow_of_col<DUP>(8 * (nq0 + nw) + 2 * tig + e, p.GT);
+        lim[nw][e] = r < 0 ? 0x7fffffff : d.seq_len - p.T + r / p.G;
       }
     int lim_min = 0x7fffffff;
     #pragma unroll
-    for (int nq = 0; nq < NQ; ++nq) lim_min = min(lim_min, min(lim[nq][0], lim[nq][1]));
+    for (int nw = 0; nw < NQW; ++nw) lim_min = min(lim_min, min(lim[nw][0], lim[nw][1]));
     lim_min = __reduce_min_sync(0xffffffffu, lim_min);
     const int safe_end = min(d.tok_end, lim_min + 1);  // keys below this need no mask
 
-    float o[NPV][D / 16][4];
+    float o[NPVW][D / 16][4];
     #pragma unroll
-    for (int j = 0; j < NPV; ++j)
+    for (int j = 0; j < NPVW; ++j)
       #pragma unroll
       for (int mt = 0; mt < D / 16; ++mt) o[j][mt][0] = o[j][mt][1] = o[j][mt][2] = o[j][mt][3] = 0.f;
-    float mrow[NQ][2], lrow[NQ][2];
+    float mrow[NQW][2], lrow[NQW][2];
     #pragma unroll
-    for (int nq = 0; nq < NQ; ++nq) mrow[nq][0] = mrow[nq][1] = -INFINITY, lrow[nq][0] = lrow[nq][1] = 0.f;
+    for (int nw = 0; nw < NQW; ++nw) mrow[nw][0] = mrow[nw][1] = -INFINITY, lrow[nw][0] = lrow[nw][1] = 0.f;
 
     const int nkb = (d.tok_end - d.tok_begin + 15) / 16;
     for (int kbi = 0; kbi < nkb; ++kbi) {
@@ -279,13 +287,16 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
       const uint32_t vs = ks + G_::TILE;
       float sc2 = p.qk_scale_log2, vsc = 1.f;
       if (KVT == 1) {
-        sc2 *= meta_sc[s * 4 + 1] * 256.f;
-        vsc = meta_sc[s * 4 + 2] * 256.f;
+        sc2 *= meta_sc[s * 4 + 1];
+        vsc = meta_sc[s * 4 + 2] * kPScale;
       }
-      // ---- S^T = K Q^T  (rows: 16 keys; columns: query rows)
-      float sacc[NQ][4];
+      // ---- S^T = K Q^T  (rows: 16 keys; columns: query rows). Even and odd k-steps go to two
+      //      accumulators so that two MMA chains are in flight.
+      float sacc[2][NQW][4];
       #pragma unroll
-      for (int nq = 0; nq < NQ; ++nq) sacc[nq][0] = sacc[nq][1] = sacc[nq][2] = sacc[nq][3] = 0.f;
+      for (int c = 0; c < 2; ++c)
+        #pragma unroll
+        for (int nw = 0; nw < NQW; ++nw) sacc[c][nw][0] = sacc[c][nw][1] = sacc[c][nw][2] = sacc[c][nw][3] = 0.f;
       {
         const int r = (lane & 7) + ((lane >> 3) & 1) * 8;
         if (KVT == 0) {
@@ -294,7 +305,7 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
             uint32_t a[4];
             ldsm_x4(ks + G_::off(r, 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
             #pragma unroll
-            for (int nq = 0; nq < NQ; ++nq) mma_bf16(sacc[nq], a, qf[nq][kk][0], qf[nq][kk][1]);
+            for (int nw = 0; nw < NQW; ++nw) mma_bf16(sacc[kk & 1][nw], a, qf[nw][kk][0], qf[nw][kk][1]);
           }
         } else {
           #pragma unroll
@@ -304,12 +315,13 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
             #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               uint32_t a[4];
-              a[0] = e4m3x2_hi_bytes_to_f16x2(prmt(R[2 * h2], 0, 0x1100));
-              a[2] = e4m3x2_hi_bytes_to_f16x2(prmt(R[2 * h2], 0, 0x3322));
-              a[1] = e4m3x2_hi_bytes_to_f16x2(prmt(R[2 * h2 + 1], 0, 0x1100));
-              a[3] = e4m3x2_hi_bytes_to_f16x2(prmt(R[2 * h2 + 1], 0, 0x3322));
+              a[0] = e4m3x2_to_f16x2(R[2 * h2] & 0xffffu);
+              a[2] = e4m3x2_to_f16x2(R[2 * h2] >> 16);
+              a[1] = e4m3x2_to_f16x2(R[2 * h2 + 1] & 0xffffu);
+              a[3] = e4m3x2_to_f16x2(R[2 * h2 + 1] >> 16);
               #pragma unroll
-              for (int nq = 0; nq < NQ; ++nq) mma_f16(sacc[nq], a, qf[nq][2 * k2 + h2][0], qf[nq][2 * k2 + h2][1]);
+              for (int nw = 0; nw < NQW; ++nw)
+                mma_f16(sacc[h2][nw], a, qf[nw][2 * k2 + h2][0], qf[nw][2 * k2 + h2][1]);
             }
           }
         }
@@ -317,17 +329,17 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
       // ---- scale, mask, online softmax (log2 domain, fp32 state)
       const bool need_mask = kbase + 16 > safe_end;
       bool grew = false;
-      float alpha[NQ][2];
-      float pv[NQ][4];
+      float alpha[NQW][2];
+      float pv[NQW][4];
       #pragma unroll
-      for (int nq = 0; nq < NQ; ++nq) {
+      for (int nw = 0; nw < NQW; ++nw) {
         float sv4[4];
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          sv4[i] = sacc[nq][i] * sc2;
+          sv4[i] = (sacc[0][nw][i] + sacc[1][nw][i]) * sc2;
           if (need_mask) {
             const int j = kbase + gid + (i >> 1) * 8;
-            if (j >= d.tok_end || j > lim[nq][i & 1]) sv4[i] = -INFINITY;
+            if (j >= d.tok_end || j > lim[nw][i & 1]) sv4[i] = -INFINITY;
           }
         }
         #pragma unroll
@@ -336,48 +348,48 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          const float mnew = fmaxf(mrow[nq][e], mx);
-          grew |= mnew > mrow[nq][e];
+          const float mnew = fmaxf(mrow[nw][e], mx);
+          grew |= mnew > mrow[nw][e];
           const float muse = mnew == -INFINITY ? 0.f : mnew;
-          alpha[nq][e] = fast_exp2(mrow[nq][e] - muse);
-          pv[nq][e] = fast_exp2(sv4[e] - muse);
-          pv[nq][e + 2] = fast_exp2(sv4[e + 2] - muse);
-          lrow[nq][e] = lrow[nq][e] * alpha[nq][e] + pv[nq][e] + pv[nq][e + 2];
-          mrow[nq][e] = mnew;
+          alpha[nw][e] = fast_exp2(mrow[nw][e] - muse);
+          pv[nw][e] = fast_exp2(sv4[e] - muse);
+          pv[nw][e + 2] = fast_exp2(sv4[e + 2] - muse);
+          lrow[nw][e] = lrow[nw][e] * alpha[nw][e] + pv[nw][e] + pv[nw][e + 2];
+          mrow[nw][e] = mnew;
         }
       }
       if (__any_sync(0xffffffffu, grew)) {
         #pragma unroll
-        for (int j = 0; j < NPV; ++j) {
-          const int nq = (KVT == 0 && !DUP) ? j / 2 : j;
+        for (int j = 0; j < NPVW; ++j) {
+          const int nw = (KVT == 0 && !DUP) ? j / 2 : j;
           #pragma unroll
           for (int mt = 0; mt < D / 16; ++mt) {
-            o[j][mt][0] *= alpha[nq][0]; o[j][mt][1] *= alpha[nq][1];
-            o[j][mt][2] *= alpha[nq][0]; o[j][mt][3] *= alpha[nq][1];
+            o[j][mt][0] *= alpha[nw][0]; o[j][mt][1] *= alpha[nw][1];
+            o[j][mt][2] *= alpha[nw][0]; o[j][mt][3] *= alpha[nw][1];
           }
         }
       }
       // ---- P^T as B fragments: C-fragment rows (keys) become the K index via movmatrix
-      uint32_t bp[NPV][2];
+      uint32_t bp[NPVW][2];
       #pragma unroll
-      for (int nq = 0; nq < NQ; ++nq) {
+      for (int nw = 0; nw < NQW; ++nw) {
         if (KVT == 1) {
-          bp[nq][0] = movmatrix_t(pack_f16(pv[nq][0] * vsc, pv[nq][1] * vsc));
-          bp[nq][1] = movmatrix_t(pack_f16(pv[nq][2] * vsc, pv[nq][3] * vsc));
+          bp[nw][0] = movmatrix_t(pack_f16(pv[nw][0] * vsc, pv[nw][1] * vsc));
+          bp[nw][1] = movmatrix_t(pack_f16(pv[nw][2] * vsc, pv[nw][3] * vsc));
         } else {
-          const uint32_t h01 = pack_bf16(pv[nq][0], pv[nq][1]);
-          const uint32_t h23 = pack_bf16(pv[nq][2], pv[nq][3]);
-          const uint32_t l01 = pack_bf16(pv[nq][0] - bf16_lo(h01), pv[nq][1] - bf16_hi(h01));
-          const uint32_t l23 = pack_bf16(pv[nq][2] - bf16_lo(h23), pv[nq][3] - bf16_hi(h23));
+          const uint32_t h01 = pack_bf16(pv[nw][0], pv[nw][1]);
+          const uint32_t h23 = pack_bf16(pv[nw][2], pv[nw][3]);
+          const uint32_t l01 = pack_bf16(pv[nw][0] - bf16_lo(h01), pv[nw][1] - bf16_hi(h01));
+          const uint32_t l23 = pack_bf16(pv[nw][2] - bf16_lo(h23), pv[nw][3] - bf16_hi(h23));
           if (DUP) {
             const bool lo_lane = tig >= 2;  // columns 4..7 carry the low halves
             bp[0][0] = movmatrix_t(lo_lane ? l01 : h01);
             bp[0][1] = movmatrix_t(lo_lane ? l23 : h23);
           } else {
-            bp[2 * nq][0] = movmatrix_t(h01);
-            bp[2 * nq][1] = movmatrix_t(h23);
-            bp[2 * nq + 1][0] = movmatrix_t(l01);
-            bp[2 * nq + 1][1] = movmatrix_t(l23);
+            bp[2 * nw][0] = movmatrix_t(h01);
+            bp[2 * nw][1] = movmatrix_t(h23);
+            bp[2 * nw + 1][0] = movmatrix_t(l01);
+            bp[2 * nw + 1][1] = movmatrix_t(l23);
           }
         }
       }
@@ -390,7 +402,7 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
           uint32_t a[4];
           ldsm_x4_t(vs + G_::off(r, 2 * mt + (q4 & 1)), a[0], a[1], a[2], a[3]);
           #pragma unroll
-          for (int j = 0; j < NPV; ++j) mma_bf16(o[j][mt], a, bp[j][0], bp[j][1]);
+          for (int j = 0; j < NPVW; ++j) mma_bf16(o[j][mt], a, bp[j][0], bp[j][1]);
         }
       } else {
         // thread (gid, tig) reads 4 codes at d = 32pp + 4gid .. +3 of keys 2tig, 2tig+1,
@@ -406,15 +418,16 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
           const uint32_t w3 = *reinterpret_cast<const uint32_t*>(vb + G_::off(2 * tig + 9, cg) + inb);
           #pragma unroll
           for (int sub = 0; sub < 2; ++sub) {
-            const uint32_t sel0 = ((4 + 2 * sub) << 12) | ((4 + 2 * sub) << 8) | ((2 * sub) << 4) | (2 * sub);
-            const uint32_t sel1 = sel0 + 0x1111;
+            // bytes 0,1 <- (key 2tig, key 2tig+1) at d offset 2sub, bytes 2,3 <- the same at 2sub+1
+            const uint32_t sel = sub == 0 ? 0x5140u : 0x7362u;
+            const uint32_t x01 = prmt(w0, w1, sel), x23 = prmt(w2, w3, sel);
             uint32_t a[4];
-            a[0] = e4m3x2_hi_bytes_to_f16x2(prmt(w0, w1, sel0));
-            a[1] = e4m3x2_hi_bytes_to_f16x2(prmt(w0, w1, sel1));
-            a[2] = e4m3x2_hi_bytes_to_f16x2(prmt(w2, w3, sel0));
-            a[3] = e4m3x2_hi_bytes_to_f16x2(prmt(w2, w3, sel1));
+            a[0] = e4m3x2_to_f16x2(x01 & 0xffffu);
+            a[1] = e4m3x2_to_f16x2(x01 >> 16);
+            a[2] = e4m3x2_to_f16x2(x23 & 0xffffu);
+            a[3] = e4m3x2_to_f16x2(x23 >> 16);
             #pragma unroll
-            for (int j = 0; j < NPV; ++j) mma_f16(o[j][2 * pp + sub], a, bp[j][0], bp[j][1]);
+            for (int j = 0; j < NPVW; ++j) mma_f16(o[j][2 * pp + sub], a, bp[j][0], bp[j][1]);
           }
         }
       }
@@ -425,14 +438,14 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
 
     // ---- epilogue: row sums, hi + lo, normalise, store
     #pragma unroll
-    for (int nq = 0; nq < NQ; ++nq)
+    for (int nw = 0; nw < NQW; ++nw)
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        float l = lrow[nq][e];
+        float l = lrow[nw][e];
         l += __shfl_xor_sync(0xffffffffu, l, 4);
         l += __shfl_xor_sync(0xffffffffu, l, 8);
         l += __shfl_xor_sync(0xffffffffu, l, 16);
-        lrow[nq][e] = l;
+        lrow[nw][e] = l;
       }
     if (KVT == 0) {
       if (DUP) {
@@ -442,25 +455,26 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
           for (int i = 0; i < 4; ++i) o[0][mt][i] += __shfl_xor_sync(0xffffffffu, o[0][mt][i], 2);
       } else {
         #pragma unroll
-        for (int nq = 0; nq < NQ; ++nq)
+        for (int nw = 0; nw < NQW; ++nw)
           #pragma unroll
           for (int mt = 0; mt < D / 16; ++mt)
             #pragma unroll
-            for (int i = 0; i < 4; ++i) o[2 * nq][mt][i] += o[2 * nq + 1][mt][i];
+            for (int i = 0; i < 4; ++i) o[2 * nw][mt][i] += o[2 * nw + 1][mt][i];
       }
     }
     #pragma unroll
-    for (int nq = 0; nq < NQ; ++nq) {
-      const int j = (KVT == 0 && !DUP) ? 2 * nq : nq;
+    for (int nw = 0; nw < NQW; ++nw) {
+      const int j = (KVT == 0 && !DUP) ? 2 * nw : nw;
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int n = 8 * nq + 2 * tig + e;
+        const int n = 8 * (nq0 + nw) + 2 * tig + e;
         if (DUP && n >= 4) continue;
         const int r = n < p.GT ? n : -1;
         if (r < 0) continue;
-        const float l = lrow[nq][e];
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        const float lse_v = l > 0.f ? (mrow[nq][e] + __log2f(l)) * LN2 : -INFINITY;
+        const float l = lrow[nw][e];
+        // FP8: P entered the MMA multiplied by kPScale (keeps it in f16's normal range)
+        const float inv = l > 0.f ? (KVT == 1 ? 1.f / (kPScale * l) : 1.f / l) : 0.f;
+        const float lse_v = l > 0.f ? (mrow[nw][e] + __log2f(l)) * LN2 : -INFINITY;
         const int t = r / p.G, g = r % p.G;
         float* dst;
         float* dst_lse;
@@ -497,15 +511,15 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
 }
 
 // ------------------------------------------------------------------ host side
-template <int KVT, int D, int NQ, int NPV, bool DUP>
+template <int KVT, int D, int NQ, int NPV, bool DUP, int NCW>
 static cudaError_t launch_variant(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                   cudaStream_t st) {
-  auto fn = split_kernel<KVT, D, NQ, NPV, DUP>;
+  auto fn = split_kernel<KVT, D, NQ, NPV, DUP, NCW>;
   const int smem = Smem<KVT, D, NQ>::ALLOC;
   if (!ensure_smem_attr((const void*)fn, smem)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_bins);
-  cfg.blockDim = dim3(kSplitThreads);
+  cfg.blockDim = dim3(32 * (1 + NCW));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -519,12 +533,12 @@ static cudaError_t launch_variant(const SplitParams& p, const CUtensorMap& tmK, 
 template <int KVT, int D>
 static cudaError_t launch_gt(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st) {
   if constexpr (KVT == 0) {
-    if (p.GT <= 4) return launch_variant<KVT, D, 1, 1, true>(p, tmK, tmV, st);
-    if (p.GT <= 8) return launch_variant<KVT, D, 1, 2, false>(p, tmK, tmV, st);
-    return launch_variant<KVT, D, 2, 4, false>(p, tmK, tmV, st);
+    if (p.GT <= 4) return launch_variant<KVT, D, 1, 1, true, 1>(p, tmK, tmV, st);
+    if (p.GT <= 8) return launch_variant<KVT, D, 1, 2, false, 1>(p, tmK, tmV, st);
+    return launch_variant<KVT, D, 2, 4, false, 2>(p, tmK, tmV, st);
   } else {
-    if (p.GT <= 8) return launch_variant<KVT, D, 1, 1, false>(p, tmK, tmV, st);
-    return launch_variant<KVT, D, 2, 2, false>(p, tmK, tmV, st);
+    if (p.GT <= 8) return launch_variant<KVT, D, 1, 1, false, 1>(p, tmK, tmV, st);
+    return launch_variant<KVT, D, 2, 2, false, 2>(p, tmK, tmV, st);
   }
 }
 
