@@ -25,6 +25,7 @@ namespace decattn {
 constexpr int kCombineThreads = 128;
 constexpr int kCombineWarps = kCombineThreads / 32;
 constexpr int kCombineCtasPerSm = 4;
+constexpr int kCombineSmemRequests = 4096;  // per-request arrays are copied to shared memory up to this batch
 
 template <int D>
 struct CombineVec {
@@ -51,14 +52,27 @@ template <int D>
 __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_kernel(const CombineParams p) {
   constexpr int VEC = D / 32;
   using V = typename CombineVec<D>::T;
-  extern __shared__ int32_t cb_sm[];  // [B + 1] chunk prefix per request
-  griddep_wait();  // the split kernel's partials are complete and visible
+  extern __shared__ int32_t req_sm[];  // [3][B + 1]: chunk prefix, tile prefix S, seq_lens
+  // The plan is complete when this grid starts (the split kernel lets it launch only after its
+  // own wait on the planner), so everything but the partials is read before waiting.
   const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
   if (hdr->magic != kPlanMagic || hdr->status != DECATTN_OK) return;  // the split kernel reports it
-  const int32_t* cb_g = plan_arr(p.plan, hdr->off_cb);
+  const int32_t* cb_sm = plan_arr(p.plan, hdr->off_cb);
   const int32_t* S = plan_arr(p.plan, hdr->off_S);
-  for (int i = threadIdx.x; i <= p.B; i += kCombineThreads) cb_sm[i] = cb_g[i];
-  __syncthreads();
+  const int32_t* Ls = p.seq_lens;
+  if (p.B <= kCombineSmemRequests) {
+    int32_t* a = req_sm;
+    int32_t* b = req_sm + (p.B + 1);
+    int32_t* c = req_sm + 2 * (p.B + 1);
+    for (int i = threadIdx.x; i <= p.B; i += kCombineThreads) {
+      a[i] = cb_sm[i];
+      b[i] = S[i];
+      c[i] = i < p.B ? Ls[i] : 0;
+    }
+    __syncthreads();
+    cb_sm = a; S = b; Ls = c;
+  }
+  griddep_wait();  // the split kernel's partials are complete and visible
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t rows_per_b = (int64_t)p.T * p.Hq;
   const int64_t total = rows_per_b * cb_sm[p.B];
@@ -77,7 +91,7 @@ __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_ke
     const int t = row_in_b / p.Hq, qh = row_in_b - t * p.Hq;
     const int64_t row = ((int64_t)b * p.T + t) * p.Hq + qh;
     float* orow = p.out + row * D;
-    const int L = p.seq_lens[b];
+    const int L = Ls[b];
     const int nb = L > 0 ? (L + p.tl - 1) / p.tl : 0;
     float acc[VEC];
     #pragma unroll
@@ -157,7 +171,7 @@ cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st) 
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return cudaErrorUnknown;
   const void* fn = p.D == 128 ? (const void*)combine_kernel<128> : (const void*)combine_kernel<64>;
-  const int smem = 4 * (p.B + 1);
+  const int smem = p.B <= kCombineSmemRequests ? 12 * (p.B + 1) : 0;
   if (!ensure_smem_attr(fn, smem)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms * kCombineCtasPerSm);

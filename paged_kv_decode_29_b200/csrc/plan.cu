@@ -58,9 +58,9 @@ __device__ inline ReqArrays carve_req(char* p, int B) {
   return r;
 }
 
-// Exclusive block-wide scan of (a, b, c) over kPlanThreads threads; returns the prefix and
+// Exclusive block-wide scan of (a, b, c, d) over kPlanThreads threads; returns the prefix and
 // adds the block totals into tot. warp_tot holds one entry per warp.
-struct Tri { long long a, b; int c; };
+struct Tri { long long a, b; int c; long long d; };
 
 __device__ inline Tri block_exscan(Tri v, Tri& tot, Tri* warp_tot) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -70,27 +70,29 @@ __device__ inline Tri block_exscan(Tri v, Tri& tot, Tri* warp_tot) {
     long long a = __shfl_up_sync(0xffffffffu, inc.a, o);
     long long b = __shfl_up_sync(0xffffffffu, inc.b, o);
     int c = __shfl_up_sync(0xffffffffu, inc.c, o);
-    if (lane >= o) { inc.a += a; inc.b += b; inc.c += c; }
+    long long dd = __shfl_up_sync(0xffffffffu, inc.d, o);
+    if (lane >= o) { inc.a += a; inc.b += b; inc.c += c; inc.d += dd; }
   }
   if (lane == 31) warp_tot[w] = inc;
   __syncthreads();
   if (w == 0) {
-    Tri t = lane < kPlanWarps ? warp_tot[lane] : Tri{0, 0, 0};
+    Tri t = lane < kPlanWarps ? warp_tot[lane] : Tri{0, 0, 0, 0};
     #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       long long a = __shfl_up_sync(0xffffffffu, t.a, o);
       long long b = __shfl_up_sync(0xffffffffu, t.b, o);
       int c = __shfl_up_sync(0xffffffffu, t.c, o);
-      if (lane >= o) { t.a += a; t.b += b; t.c += c; }
+      long long dd = __shfl_up_sync(0xffffffffu, t.d, o);
+      if (lane >= o) { t.a += a; t.b += b; t.c += c; t.d += dd; }
     }
     if (lane < kPlanWarps) warp_tot[lane] = t;
   }
   __syncthreads();
-  Tri base = w ? warp_tot[w - 1] : Tri{0, 0, 0};
+  Tri base = w ? warp_tot[w - 1] : Tri{0, 0, 0, 0};
   Tri all = warp_tot[kPlanWarps - 1];
   __syncthreads();
-  Tri ex{base.a + inc.a - v.a, base.b + inc.b - v.b, base.c + inc.c - v.c};
-  tot.a += all.a; tot.b += all.b; tot.c += all.c;
+  Tri ex{base.a + inc.a - v.a, base.b + inc.b - v.b, base.c + inc.c - v.c, base.d + inc.d - v.d};
+  tot.a += all.a; tot.b += all.b; tot.c += all.c; tot.d += all.d;
   return ex;
 }
 
@@ -211,22 +213,25 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
   }
 
   // ---- 1. per-request tile counts and their prefix sums
-  Tri carry{0, 0, 0};
+  // (d: combine chunks per query row of the request, see combine_chunks())
+  Tri carry{0, 0, 0, 0};
   for (int base = 0; base < B; base += kPlanThreads) {
     const int b = base + tid;
     int64_t L = b < B ? seq_lens[b] : 0;
     if (L < 0) { atomicCAS(&sh_status, 0, DECATTN_EDEVICE); L = 0; }
-    Tri v{(L + tl - 1) / tl, L / tl, (L % tl) != 0};
+    const int64_t nb = (L + tl - 1) / tl;
+    Tri v{nb, L / tl, (L % tl) != 0, b < B ? combine_chunks(nb) : 0};
     Tri before = carry;
     Tri ex = block_exscan(v, carry, warp_tot);
     if (b < B) {
+      gcb[b] = (int32_t)(before.d + ex.d);
       R.S[b] = (int32_t)(before.a + ex.a);
       R.SF[b] = (int32_t)(before.b + ex.b);
       R.SP[b] = before.c + ex.c;
       if (v.c) { R.plist[before.c + ex.c] = b; R.pcost[before.c + ex.c] = (int32_t)(L % tl); }
     }
   }
-  if (tid == 0) { R.S[B] = (int32_t)carry.a; R.SF[B] = (int32_t)carry.b; R.SP[B] = carry.c; }
+  if (tid == 0) { R.S[B] = (int32_t)carry.a; R.SF[B] = (int32_t)carry.b; R.SP[B] = carry.c; gcb[B] = (int32_t)carry.d; }
   const int64_t U64 = (int64_t)Hkv * carry.a;
   __syncthreads();
   if (U64 > init.max_units) atomicCAS(&sh_status, 0, DECATTN_ECAPACITY);
@@ -244,19 +249,6 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
   const int F = (int)((int64_t)Hkv * carry.b);
   const int mB = carry.c;
   const int m = Hkv * mB;
-
-  // ---- 2. combine chunks per query row of each request, and their prefix over requests
-  {
-    Tri c3{0, 0, 0};
-    for (int base = 0; base < B; base += kPlanThreads) {
-      const int b = base + tid;
-      const long long cb = b < B ? combine_chunks(R.S[b + 1] - R.S[b]) : 0;
-      Tri before = c3;
-      Tri ex = block_exscan(Tri{cb, 0, 0}, c3, warp_tot);
-      if (b < B) gcb[b] = (int32_t)(before.a + ex.a);
-    }
-    if (tid == 0) gcb[B] = (int32_t)c3.a;
-  }
 
   // ---- 3. requests with a partial tile, sorted by cost (desc), then b: rank by counting
   for (int j = tid; j < mB; j += kPlanThreads) {
@@ -307,11 +299,11 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
 
   // ---- 5. per-bin CSR offsets of the partial tiles, and the partial tiles bin by bin
   {
-    Tri c2{0, 0, 0};
+    Tri c2{0, 0, 0, 0};
     for (int base = 0; base < N; base += kPlanThreads) {
       const int k = base + tid;
       Tri before = c2;
-      Tri ex = block_exscan(Tri{k < N ? pcount[k] : 0, 0, 0}, c2, warp_tot);
+      Tri ex = block_exscan(Tri{k < N ? pcount[k] : 0, 0, 0, 0}, c2, warp_tot);
       if (k < N) gpbo[k] = (int32_t)(before.a + ex.a);
     }
     if (tid == 0) gpbo[N] = (int32_t)c2.a;

@@ -103,8 +103,9 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   Unit* qmeta = reinterpret_cast<Unit*>(sm + S_::OFF_QMETA);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  griddep_launch_dependents();  // the combine kernel may be scheduled; it waits for this grid
   griddep_wait();               // the plan kernel has finished and its writes are visible
+  griddep_launch_dependents();  // the combine kernel may be scheduled now (it can read the finished
+                                // plan at once and waits for this grid before reading partials)
   // the combine counters of this workspace start from zero on every run
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)p.B * p.T * p.Hq;
        i += (int64_t)gridDim.x * blockDim.x)
@@ -227,27 +228,65 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
     if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qs], qfph, p.status))) return;
     const Unit d = qmeta[qs];
     // ---- q fragments (B operand of S^T = K Q^T): column n = query row
-    uint32_t qf[NQW][D / 16][2];
+    // BF16 KV: bf16 pairs along k. FP8 KV: S^T = K Q^T runs on E4M3 MMAs (m16n8k32) straight
+    // from the staged codes; q is scaled by a per-row power of two 2^E (largest |q| lands in
+    // [128, 256)) and split into two E4M3 parts, hi = E4M3(q 2^E) and lo = E4M3(q 2^E - hi),
+    // which together carry the 8 significant bits of a bf16 q. qcs = 2^-E undoes the scaling.
+    constexpr int QK_STEPS = KVT == 0 ? D / 16 : D / 32;
+    uint32_t qf[NQW][QK_STEPS][2];
+    uint32_t ql[NQW][KVT == 1 ? QK_STEPS : 1][2];
+    float qcs[NQW][2];
     {
       const uint8_t* qsm = sm + S_::OFF_Q + qs * S_::QBYTES;
       #pragma unroll
       for (int nw = 0; nw < NQW; ++nw) {
         const int r = qrow_of_col<DUP>(8 * (nq0 + nw) + gid, p.GT);
         const uint16_t* qr = reinterpret_cast<const uint16_t*>(qsm) + (r < 0 ? 0 : r) * D;
-        #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          if (KVT == 0) {
+        if (KVT == 0) {
+          #pragma unroll
+          for (int kk = 0; kk < QK_STEPS; ++kk) {
             const uint32_t x0 = *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 2 * tig);
             const uint32_t x1 = *reinterpret_cast<const uint32_t*>(qr + 16 * kk + 8 + 2 * tig);
             qf[nw][kk][0] = r < 0 ? 0u : x0;
             qf[nw][kk][1] = r < 0 ? 0u : x1;
-          } else {
-            // FP8 K is read 4 consecutive codes per thread: logical k = 2*tig + {0,1} holds
-            // d = 16kk + 4tig + {0,1}, logical k = 8 + 2*tig + {0,1} holds d = 16kk + 4tig + {2,3}
-            const uint2 x = *reinterpret_cast<const uint2*>(qr + 16 * kk + 4 * tig);
-            qf[nw][kk][0] = r < 0 ? 0u : pack_f16(bf16_lo(x.x), bf16_hi(x.x));
-            qf[nw][kk][1] = r < 0 ? 0u : pack_f16(bf16_lo(x.y), bf16_hi(x.y));
           }
+        } else {
+          // b0 holds k = 4tig..4tig+3, b1 holds k = 16+4tig..16+4tig+3 of each 32-wide k-step
+          uint2 xv[QK_STEPS][2];
+          float amax = 0.f;
+          #pragma unroll
+          for (int kk = 0; kk < QK_STEPS; ++kk)
+            #pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              xv[kk][h] = r < 0 ? make_uint2(0u, 0u)
+                                : *reinterpret_cast<const uint2*>(qr + 32 * kk + 16 * h + 4 * tig);
+              amax = fmaxf(amax, fmaxf(fmaxf(fabsf(bf16_lo(xv[kk][h].x)), fabsf(bf16_hi(xv[kk][h].x))),
+                                       fmaxf(fabsf(bf16_lo(xv[kk][h].y)), fabsf(bf16_hi(xv[kk][h].y)))));
+            }
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+          // 2^E with E = 7 - floor(log2 amax): exponent-field arithmetic, exact
+          const int ex = amax > 0.f ? ((__float_as_int(amax) >> 23) & 0xff) - 127 : 0;
+          const int E = min(max(7 - ex, -100), 100);
+          const float up = __int_as_float((127 + E) << 23);
+          const float down = __int_as_float((127 - E) << 23);
+          #pragma unroll
+          for (int kk = 0; kk < QK_STEPS; ++kk)
+            #pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float v0 = bf16_lo(xv[kk][h].x) * up, v1 = bf16_hi(xv[kk][h].x) * up;
+              const float v2 = bf16_lo(xv[kk][h].y) * up, v3 = bf16_hi(xv[kk][h].y) * up;
+              const uint32_t h01 = f32x2_to_e4m3x2(v0, v1), h23 = f32x2_to_e4m3x2(v2, v3);
+              const float2 b01 = f16x2_to_float2(e4m3x2_to_f16x2(h01));
+              const float2 b23 = f16x2_to_float2(e4m3x2_to_f16x2(h23));
+              const uint32_t l01 = f32x2_to_e4m3x2(v0 - b01.x, v1 - b01.y);
+              const uint32_t l23 = f32x2_to_e4m3x2(v2 - b23.x, v3 - b23.y);
+              qf[nw][kk][h] = h01 | (h23 << 16);
+              ql[nw][kk][h] = l01 | (l23 << 16);
+            }
+          // this lane holds row gid's factor; the softmax needs columns 2tig and 2tig+1
+          qcs[nw][0] = __shfl_sync(0xffffffffu, down, (2 * tig) * 4);
+          qcs[nw][1] = __shfl_sync(0xffffffffu, down, (2 * tig + 1) * 4);
         }
       }
     }
@@ -308,20 +347,16 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
             for (int nw = 0; nw < NQW; ++nw) mma_bf16(sacc[kk & 1][nw], a, qf[nw][kk][0], qf[nw][kk][1]);
           }
         } else {
+          // the staged codes are the A operand as they are: ldmatrix gives each lane 4 codes of
+          // one key row per register, which is the m16n8k32 E4M3 A fragment
           #pragma unroll
-          for (int k2 = 0; k2 < D / 32; ++k2) {
-            uint32_t R[4];
-            ldsm_x4(ks + G_::off(r, 2 * k2 + (lane >> 4)), R[0], R[1], R[2], R[3]);
+          for (int kk = 0; kk < QK_STEPS; ++kk) {
+            uint32_t a[4];
+            ldsm_x4(ks + G_::off(r, 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
             #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              uint32_t a[4];
-              a[0] = e4m3x2_to_f16x2(R[2 * h2] & 0xffffu);
-              a[2] = e4m3x2_to_f16x2(R[2 * h2] >> 16);
-              a[1] = e4m3x2_to_f16x2(R[2 * h2 + 1] & 0xffffu);
-              a[3] = e4m3x2_to_f16x2(R[2 * h2 + 1] >> 16);
-              #pragma unroll
-              for (int nw = 0; nw < NQW; ++nw)
-                mma_f16(sacc[h2][nw], a, qf[nw][2 * k2 + h2][0], qf[nw][2 * k2 + h2][1]);
+            for (int nw = 0; nw < NQW; ++nw) {
+              mma_e4m3(sacc[0][nw], a, qf[nw][kk][0], qf[nw][kk][1]);
+              mma_e4m3(sacc[1][nw], a, ql[nw][kk][0], ql[nw][kk][1]);
             }
           }
         }
@@ -336,7 +371,7 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
         float sv4[4];
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          sv4[i] = (sacc[0][nw][i] + sacc[1][nw][i]) * sc2;
+          sv4[i] = (sacc[0][nw][i] + sacc[1][nw][i]) * (KVT == 1 ? sc2 * qcs[nw][i & 1] : sc2);
           if (need_mask) {
             const int j = kbase + gid + (i >> 1) * 8;
             if (j >= d.tok_end || j > lim[nw][i & 1]) sv4[i] = -INFINITY;
