@@ -14,7 +14,8 @@
 //    flight per lane) and folds them into (max, weight, weighted sum);
 //  * a row made of one chunk is finished right there;
 //  * otherwise the warp publishes its chunk state and bumps the row's counter; the warp
-//    that brings the counter to cb_b merges the row's chunk states and writes the row.
+//    that brings the counter to cb_b merges the row's chunk states (8 at once, with an
+//    online rescale between groups) and writes the row.
 // Rows of requests held in a single tile were written by the split kernel (cb_b = 0).
 #include <type_traits>
 
@@ -26,6 +27,7 @@ constexpr int kCombineThreads = 128;
 constexpr int kCombineWarps = kCombineThreads / 32;
 constexpr int kCombineCtasPerSm = 4;
 constexpr int kCombineSmemRequests = 4096;  // per-request arrays are copied to shared memory up to this batch
+constexpr int kMergeGroup = 8;              // chunk states loaded at once by the merging warp
 
 template <int D>
 struct CombineVec {
@@ -142,24 +144,46 @@ __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_ke
     prev = __shfl_sync(0xffffffffu, prev, 0);
     if (prev != ncb - 1) continue;
     __threadfence();
+    // all chunk states of the row, in groups of kMergeGroup loaded at once (from L2: they were
+    // written by other warps of this grid)
     const float* cs0 = p.chunk_state + (w - j) * (D + 4);
-    float Mt = -INFINITY;
-    for (int c = lane; c < ncb; c += 32) Mt = fmaxf(Mt, __ldcg(cs0 + (int64_t)c * (D + 4)));
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) Mt = fmaxf(Mt, __shfl_xor_sync(0xffffffffu, Mt, o));
-    float Wt = 0.f;
+    float Mt = -INFINITY, Wt = 0.f;
     #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-    if (Mt != -INFINITY) {
-      #pragma unroll 8
-      for (int c = 0; c < ncb; ++c) {
-        const float* s = cs0 + (int64_t)c * (D + 4);
-        const float mc = __ldcg(s), wc = __ldcg(s + 1);
-        const float sc = mc == -INFINITY ? 0.f : expf(mc - Mt);
-        Wt += sc * wc;
-        #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[e] += sc * __ldcg(s + 4 + lane * VEC + e);
+    #pragma unroll 1
+    for (int c0 = 0; c0 < ncb; c0 += kMergeGroup) {
+      const int nc = min(kMergeGroup, ncb - c0);
+      const float* g = cs0 + (int64_t)c0 * (D + 4);
+      const float2 mw = lane < nc ? __ldcg(reinterpret_cast<const float2*>(g + (int64_t)lane * (D + 4)))
+                                  : make_float2(-INFINITY, 0.f);
+      const float mc = mw.x, wc = mw.y;
+      V cv[kMergeGroup];
+      #pragma unroll
+      for (int i = 0; i < kMergeGroup; ++i)
+        if (i < nc) cv[i] = __ldcg(reinterpret_cast<const V*>(g + (int64_t)i * (D + 4) + 4) + lane);
+      float Mg = mc;
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) Mg = fmaxf(Mg, __shfl_xor_sync(0xffffffffu, Mg, o));
+      const float Mn = fmaxf(Mt, Mg);
+      if (Mn == -INFINITY) continue;  // no visible key in any chunk so far
+      const float a = Mt == -INFINITY ? 0.f : expf(Mt - Mn);
+      const float wl = mc == -INFINITY ? 0.f : expf(mc - Mn);
+      float Wg = wl * wc;
+      #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) Wg += __shfl_xor_sync(0xffffffffu, Wg, o);
+      Wt = Wt * a + Wg;
+      #pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[e] *= a;
+      #pragma unroll
+      for (int i = 0; i < kMergeGroup; ++i) {
+        const float wi = __shfl_sync(0xffffffffu, wl, i);
+        if (i < nc) {
+          const float* f = reinterpret_cast<const float*>(&cv[i]);
+          #pragma unroll
+          for (int e = 0; e < VEC; ++e) acc[e] += wi * f[e];
+        }
       }
+      Mt = Mn;
     }
     write_row<D>(orow, p.lse + row, lane, Mt, Wt, acc);
     if (lane == 0) p.row_cnt[row] = 0;  // ready for the next combine on this workspace

@@ -124,6 +124,8 @@ struct SplitParams {
   int32_t* row_cnt;         // [B*T*Hq] combine counters, zeroed here for the combine that follows
   int32_t* status;          // run status word (plan header)
   int B, T, Hq, Hkv, G, GT, P, num_pages, mpps, n_bins;
+  int tile_len;             // the plan's tile length
+  int64_t max_units;        // the plan's capacity (partial slots of the workspace)
   float qk_scale_log2;      // sm_scale * log2(e)
 };
 

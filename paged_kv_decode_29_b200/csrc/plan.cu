@@ -181,7 +181,11 @@ __device__ void greedy_partials_smem(int lane, int N, int first, int m, int Hkv,
 
 __global__ void __launch_bounds__(kPlanThreads, 1)
 plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* __restrict__ plan) {
-  // the split kernel may start its prologue now; it waits for this grid before reading the plan
+  // Launched with programmatic serialisation: wait until the previous kernel of the stream has
+  // finished (seq_lens, and the inputs the split kernel reads before its own wait, are final),
+  // then let the split kernel start: it streams the full tiles, which need no plan, and waits
+  // for this grid before reading the plan.
+  griddep_wait();
   griddep_launch_dependents();
   const int B = init.batch, Hkv = init.n_kv_heads, tl = init.tile_len, N = init.n_bins;
   extern __shared__ __align__(16) uint8_t plan_smem[];
@@ -445,8 +449,18 @@ extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads,
   const size_t smem =
       (size_t)plan_bins_smem(n_bins) + (batch <= kPlanSmemRequests ? (size_t)req_arrays_bytes(batch) : 0);
   if (!ensure_smem_attr((const void*)plan_kernel, kPlanMaxSmem)) return DECATTN_ECUDA;
-  plan_kernel<<<1, kPlanThreads, smem, st>>>(seq_lens, h, static_cast<char*>(plan_buf));
-  if (cudaGetLastError() != cudaSuccess) return DECATTN_ECUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kPlanThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // launched while the previous kernel drains
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, plan_kernel, seq_lens, h, static_cast<char*>(plan_buf)) != cudaSuccess)
+    return DECATTN_ECUDA;
   plan->buf = plan_buf;
   plan->buf_bytes = plan_bytes;
   plan->batch = batch;

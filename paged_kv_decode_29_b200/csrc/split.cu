@@ -70,6 +70,104 @@ struct Smem {
   static constexpr int ALLOC = BYTES + 1024;                     // slack to align the base to 1024
 };
 
+// ------------------------------------------------------------------ full tiles without the plan
+// The greedy rule deals the full tiles round-robin: full tile f (counted in (b, h, i) order)
+// lands in bin f mod N at position f div N, ahead of every partial tile. A CTA can therefore
+// list its own full tiles from seq_lens alone and stream them while the planner is still
+// running; only its partial tiles wait for the plan. The walk runs in the producer warp
+// (every lane returns the same tile). It is used when the batch fits its 32 windows of 32
+// requests and the planner's device-side checks are known to pass (no negative length, tile
+// count within the capacity); otherwise every tile comes from the plan.
+constexpr int kWalkMaxReq = 32 * 32;
+
+struct FullTileWalk {
+  int fc;             // full tiles of this bin listed by the walk (0: all come from the plan)
+  int nwin;           // windows holding requests
+  long long wsf, ws;  // lane l: full tiles / tiles of one KV head in the requests before window l
+  int cur;            // window cached below (-1: none)
+  int L;              // lane i: length of request 32 cur + i
+  int nf_in, nb_in;   // lane i: inclusive prefix of full tiles / tiles over the cached window
+  long long csf, cs;  // wsf, ws of the cached window
+};
+
+__device__ __forceinline__ void walk_init(FullTileWalk& w, const SplitParams& p, int lane) {
+  w.fc = 0; w.nwin = 0; w.wsf = 0; w.ws = 0; w.cur = -1;
+  w.L = 0; w.nf_in = 0; w.nb_in = 0; w.csf = 0; w.cs = 0;
+  if (p.B > kWalkMaxReq || p.tile_len <= 0) return;
+  const uint32_t tl = (uint32_t)p.tile_len;  // 32-bit divisions: the 64-bit ones are software routines
+  const int nwin = (p.B + 31) / 32;
+  // window sums, one window per iteration (coalesced, the next window's load in flight); lane l
+  // keeps window l. A request with more than 2^26 tiles turns the walk off, so that a window
+  // sum fits 32 bits.
+  uint32_t my_sf = 0, my_sb = 0;
+  bool bad = false;
+  int Lnext = lane < p.B ? __ldg(p.seq_lens + lane) : 0;
+  #pragma unroll 1
+  for (int w0 = 0; w0 < nwin; ++w0) {
+    const int L = Lnext;
+    const int bn = 32 * (w0 + 1) + lane;
+    Lnext = bn < p.B ? __ldg(p.seq_lens + bn) : 0;
+    const uint32_t Lu = L < 0 ? 0u : (uint32_t)L, nf = Lu / tl, nb = nf + (Lu != nf * tl ? 1u : 0u);
+    bad |= L < 0 || nb > (1u << 26);
+    const uint32_t sf = __reduce_add_sync(0xffffffffu, nf), sb = __reduce_add_sync(0xffffffffu, nb);
+    if (lane == w0) { my_sf = sf; my_sb = sb; }
+  }
+  long long isf = my_sf, isb = my_sb;
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long a = __shfl_up_sync(0xffffffffu, isf, o), c = __shfl_up_sync(0xffffffffu, isb, o);
+    if (lane >= o) { isf += a; isb += c; }
+  }
+  const long long F = (long long)p.Hkv * __shfl_sync(0xffffffffu, isf, 31);
+  const long long U = (long long)p.Hkv * __shfl_sync(0xffffffffu, isb, 31);
+  // the planner reports a negative length or too many tiles; the tile and slot arithmetic
+  // below is 32-bit
+  if (__any_sync(0xffffffffu, bad) || U > p.max_units || U >= (1ll << 31)) return;
+  w.wsf = isf - my_sf;
+  w.ws = isb - my_sb;
+  w.nwin = nwin;
+  const uint32_t N = gridDim.x, Fu = (uint32_t)F;
+  w.fc = (int)(Fu / N + (blockIdx.x < Fu % N ? 1u : 0u));
+}
+
+// The j-th full tile of this CTA's bin (j < fc); the same tile plan_unit() decodes.
+__device__ __forceinline__ Unit walk_unit(FullTileWalk& w, const SplitParams& p, int lane, int j) {
+  const uint32_t tl = (uint32_t)p.tile_len;
+  const int Hkv = p.Hkv;
+  const long long f = (long long)blockIdx.x + (long long)gridDim.x * j;
+  // window: the last one whose first full tile is <= f
+  const int win = 31 - __clz(__ballot_sync(0xffffffffu, lane < w.nwin && (long long)Hkv * w.wsf <= f));
+  if (win != w.cur) {
+    const int b = 32 * win + lane;
+    w.L = b < p.B ? __ldg(p.seq_lens + b) : 0;
+    const uint32_t Lu = (uint32_t)w.L, q = Lu / tl;
+    int nf = (int)q, nb = (int)(q + (Lu != q * tl ? 1u : 0u));
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, nf, o), c = __shfl_up_sync(0xffffffffu, nb, o);
+      if (lane >= o) { nf += a; nb += c; }
+    }
+    w.nf_in = nf; w.nb_in = nb;
+    w.csf = __shfl_sync(0xffffffffu, w.wsf, win);
+    w.cs = __shfl_sync(0xffffffffu, w.ws, win);
+    w.cur = win;
+  }
+  // request: the first one of the window whose full tiles reach past f
+  const int i = __ffs(__ballot_sync(0xffffffffu, (long long)Hkv * (w.csf + w.nf_in) > f)) - 1;
+  const int L = __shfl_sync(0xffffffffu, w.L, i);
+  const int nfi = __shfl_sync(0xffffffffu, w.nf_in, i), nbi = __shfl_sync(0xffffffffu, w.nb_in, i);
+  const uint32_t Lu = (uint32_t)L, fb = Lu / tl, nb = fb + (Lu != fb * tl ? 1u : 0u);
+  const long long SFb = w.csf + nfi - (int)fb, Sb = w.cs + nbi - (int)nb;
+  const uint32_t r = (uint32_t)(f - (long long)Hkv * SFb);
+  const uint32_t hh = r / fb, it = r - hh * fb;
+  Unit u;
+  u.b = 32 * win + i; u.h = (int)hh; u.tok_begin = (int)(it * tl); u.tok_end = (int)((it + 1) * tl);
+  u.seq_len = L;
+  u.slot = nb == 1 ? -1 : (int)(Hkv * Sb + (long long)hh * nb + it);
+  u.tile = (int)it; u.zero = 0;
+  return u;
+}
+
 // Row of the staged q slot feeding MMA column n, or -1 for a zero column.
 template <bool DUP>
 __device__ __forceinline__ int qrow_of_col(int n, int GT) {
@@ -103,31 +201,17 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   Unit* qmeta = reinterpret_cast<Unit*>(sm + S_::OFF_QMETA);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  griddep_wait();               // the plan kernel has finished and its writes are visible
-  griddep_launch_dependents();  // the combine kernel may be scheduled now (it can read the finished
-                                // plan at once and waits for this grid before reading partials)
-  // the combine counters of this workspace start from zero on every run
+  // The combine counters of this workspace start from zero on every run. The combine of the
+  // previous run has finished: the planner, which this grid may overlap, started after it.
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)p.B * p.T * p.Hq;
        i += (int64_t)gridDim.x * blockDim.x)
     p.row_cnt[i] = 0;
-  const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
-  if (hdr->magic != kPlanMagic || hdr->status != DECATTN_OK || hdr->n_bins != (int)gridDim.x ||
-      hdr->batch != p.B || hdr->n_kv_heads != p.Hkv) {
-    if (threadIdx.x == 0 && blockIdx.x == 0)
-      set_status(p.status, hdr->magic != kPlanMagic ? DECATTN_EINVAL
-                           : hdr->status != DECATTN_OK ? hdr->status : DECATTN_EINVAL);
-    return;
-  }
-  const PlanHeader hv = *hdr;
-  const int n_units = plan_bin_size(p.plan, hv, blockIdx.x);  // tiles of this CTA's bin
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 32 * NCW); }
     for (int s = 0; s < 2; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 32 * NCW); }
     fence_mbar_init();
   }
   __syncthreads();
-  if (n_units == 0) return;
 
   if (warp == 0) {
     // ===================================================================== producer
@@ -137,23 +221,60 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
     int qs = 0; uint32_t qeph = 1;
     bool ok = true;
     int64_t n_fill = 0, n_qfill = 0;  // copies issued so far (ring stages, q slots)
-    // tile descriptors run two tiles ahead and page ids one tile ahead of the copies
-    Unit dn = plan_unit(p.plan, hv, p.seq_lens, blockIdx.x, 0);
-    Unit dnn = n_units > 1 ? plan_unit(p.plan, hv, p.seq_lens, blockIdx.x, 1) : dn;
-    int pid_next;
-    {
+    // Tiles: the bin's full tiles from the walk, then (after waiting for the planner) the rest
+    // from the plan. Errors found before the plan is complete are held back: the planner
+    // clears the status word when it starts.
+    FullTileWalk walk;
+    walk_init(walk, p, lane);
+    bool waited = false;
+    int n_units = walk.fc;
+    int32_t pending = 0;
+    PlanHeader hv = {};
+    auto note = [&](int32_t code) {
+      if (waited) set_status(p.status, code);
+      else if (pending == 0) pending = code;
+    };
+    auto await_plan = [&]() {
+      waited = true;
+      griddep_wait();               // the plan kernel has finished and its writes are visible
+      griddep_launch_dependents();  // the combine kernel may be scheduled now (it can read the
+                                    // finished plan at once and waits for this grid before
+                                    // reading partials)
+      const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
+      bool good = hdr->magic == kPlanMagic && hdr->status == DECATTN_OK && hdr->n_bins == (int)gridDim.x &&
+                  hdr->batch == p.B && hdr->n_kv_heads == p.Hkv && hdr->tile_len == p.tile_len;
+      if (good) {
+        hv = *hdr;
+        good = walk.fc == 0 || hv.full_q + ((int)blockIdx.x < hv.full_r ? 1 : 0) == walk.fc;
+      }
+      if (good) {
+        n_units = plan_bin_size(p.plan, hv, blockIdx.x);
+      } else if (lane == 0) {
+        set_status(p.status, hdr->magic != kPlanMagic ? DECATTN_EINVAL
+                             : hdr->status != DECATTN_OK ? hdr->status : DECATTN_EINVAL);
+      }
+      if (pending != 0) set_status(p.status, pending);
+    };
+    auto next_unit = [&](int j, Unit& u) -> bool {
+      if (j < walk.fc) { u = walk_unit(walk, p, lane, j); return true; }
+      if (!waited) await_plan();
+      if (j < n_units) { u = plan_unit(p.plan, hv, p.seq_lens, blockIdx.x, j); return true; }
+      return false;
+    };
+    // The next tile's descriptor and first 32 page ids are fetched right after the current
+    // tile's first stage is issued: they are ready long before its copies run out, and the
+    // kernel's first copy waits on one tile decode only.
+    Unit dn;
+    bool has_n = next_unit(0, dn);
+    int pid_next = 0;
+    if (has_n) {
       const int pg0 = dn.tok_begin / P, npg = (dn.tok_end - dn.tok_begin + P - 1) / P;
       pid_next = lane < npg ? p.page_table[(int64_t)dn.b * p.mpps + min(pg0 + lane, p.mpps - 1)] : 0;
     }
-    for (int u = 0; u < n_units && ok; ++u) {
+    for (int u = 0; has_n && ok; ++u) {
       const Unit d = dn;
       int pid_l = pid_next;
-      dn = dnn;
-      if (u + 2 < n_units) dnn = plan_unit(p.plan, hv, p.seq_lens, blockIdx.x, u + 2);
-      if (u + 1 < n_units) {
-        const int pg0 = dn.tok_begin / P, npg = (dn.tok_end - dn.tok_begin + P - 1) / P;
-        pid_next = lane < npg ? p.page_table[(int64_t)dn.b * p.mpps + min(pg0 + lane, p.mpps - 1)] : 0;
-      }
+      bool looked = false;  // every tile has at least one stage, so the look-ahead below runs
       // q rows of this tile: T bulk copies of G consecutive heads each
       if (!warp_wait_lane0(&qempty[qs], qeph, p.status)) { ok = false; break; }
       if (lane == 0) {
@@ -169,12 +290,12 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
       qs ^= 1; if (qs == 0) qeph ^= 1;
       const int pg0 = d.tok_begin / P;
       const int npg = (d.tok_end - d.tok_begin + P - 1) / P;
-      if (lane == 0 && pg0 + npg > p.mpps) set_status(p.status, DECATTN_EDEVICE);  // row too short
+      if (lane == 0 && pg0 + npg > p.mpps) note(DECATTN_EDEVICE);  // row too short
       for (int c0 = 0; c0 < npg && ok; c0 += 32) {
         if (c0 > 0)
           pid_l = c0 + lane < npg ? p.page_table[(int64_t)d.b * p.mpps + min(pg0 + c0 + lane, p.mpps - 1)] : 0;
         if (c0 + lane < npg && (pid_l < 0 || pid_l >= p.num_pages)) {
-          set_status(p.status, DECATTN_EDEVICE);
+          note(DECATTN_EDEVICE);
           pid_l = 0;  // keeps the copy inside the pool; the result is flagged invalid
         }
         const int n_here = min(32, npg - c0);
@@ -203,8 +324,28 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
             }
             ++n_fill;
             if (++s == STAGES) { s = 0; eph ^= 1; }
+            if (!looked) {
+              looked = true;
+              has_n = next_unit(u + 1, dn);
+              if (has_n) {
+                const int pg1 = dn.tok_begin / P, npg1 = (dn.tok_end - dn.tok_begin + P - 1) / P;
+                pid_next = lane < npg1 ? p.page_table[(int64_t)dn.b * p.mpps + min(pg1 + lane, p.mpps - 1)] : 0;
+              }
+            }
           }
         }
+      }
+    }
+    if (!waited) await_plan();
+    if (ok) {
+      // no more tiles: a unit with b = -1 tells the consumers to stop
+      if (warp_wait_lane0(&qempty[qs], qeph, p.status)) {
+        if (lane == 0) {
+          qmeta[qs].b = -1;
+          mbar_arrive(&qfull[qs]);
+        }
+      } else {
+        ok = false;
       }
     }
     if (!ok && lane == 0) {
@@ -224,9 +365,10 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   int s = 0; uint32_t fph = 0;
   int qs = 0; uint32_t qfph = 0;
   const float LN2 = 0.6931471805599453f;
-  for (int u = 0; u < n_units; ++u) {
+  for (;;) {
     if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qs], qfph, p.status))) return;
     const Unit d = qmeta[qs];
+    if (d.b < 0) return;  // the producer has no more tiles
     // ---- q fragments (B operand of S^T = K Q^T): column n = query row
     // BF16 KV: bf16 pairs along k. FP8 KV: S^T = K Q^T runs on E4M3 MMAs (m16n8k32) straight
     // from the staged codes; q is scaled by a per-row power of two 2^E (largest |q| lands in

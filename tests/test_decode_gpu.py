@@ -61,6 +61,19 @@ def test_empty_and_short_requests():
     check_all(pr)
 
 
+@pytest.mark.parametrize("B", [33, 1024, 1100])
+def test_many_requests(B):
+    # The split kernel lists a bin's full tiles itself, from seq_lens, in windows of 32
+    # requests (up to 1024 requests; beyond that every tile comes from the plan). Windows with
+    # no full tile, exact multiples of the tile and empty requests shift the round-robin.
+    rng = np.random.default_rng(B)
+    lens = rng.integers(0, 260, B)
+    lens[rng.random(B) < 0.2] = 0
+    lens[rng.random(B) < 0.2] = 64 * rng.integers(1, 4)
+    lens[: min(70, B // 2)] = rng.integers(0, 64, min(70, B // 2))  # leading windows: partial tiles only
+    check_all(small([int(x) for x in lens], Hq=4, Hkv=1, d=64, tl=64, seed=B))
+
+
 def test_peaky_softmax_bf16():
     pr = small([300, 2000, 4100], Hq=8, Hkv=2, d=128, T=1, tl=256, peaky=0.05)
     check_all(pr)
