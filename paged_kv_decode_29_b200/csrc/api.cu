@@ -79,6 +79,7 @@ static bool make_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int D,
 
 struct WsLayout {
   int64_t off_part_lse, off_part_o, off_row_cnt, off_chunk, total;
+  int64_t items;  // bound on the combine's (row, chunk) items
 };
 
 // Workspace: reserved header | partial lse [units][GT] | partial o [units][GT][D] |
@@ -95,6 +96,7 @@ static WsLayout ws_layout(int64_t max_units, const dec_attn_shape& s) {
   w.off_row_cnt = o; o = align_up(o + 4 * rows, 256);
   w.off_chunk = o; o = align_up(o + 4 * items * (D + 4), 256);
   w.total = o;
+  w.items = items;
   return w;
 }
 
@@ -147,6 +149,7 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
   (void)GT;
   const WsLayout wl = ws_layout(plan->max_units, s);
   if ((int64_t)workspace_bytes < wl.total) return DECATTN_ESMALL;
+  if (wl.items >= (1ll << 31)) return DECATTN_ENOTSUP;  // the combine numbers its items in 32 bits
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DECATTN_ECUDA;
 

@@ -10,8 +10,8 @@
 // Work decomposition (computed by the planner): each query row of request b is cut into
 // cb_b chunks of up to kCombineChunk tiles; the items (b, row, chunk) are numbered request
 // by request. The kernel is persistent: every warp takes items w, w + #warps, ...
-//  * a warp loads the lse and the D floats of up to 16 partial rows at once (16 loads in
-//    flight per lane) and folds them into (max, weight, weighted sum);
+//  * a warp loads the lse and the D floats of up to 16 partial rows (8 loads in flight per
+//    lane at a time) and folds them into (max, weight, weighted sum);
 //  * a row made of one chunk is finished right there;
 //  * otherwise the warp publishes its chunk state and bumps the row's counter; the warp
 //    that brings the counter to cb_b merges the row's chunk states (8 at once, with an
@@ -28,6 +28,7 @@ constexpr int kCombineWarps = kCombineThreads / 32;
 constexpr int kCombineCtasPerSm = 4;
 constexpr int kCombineSmemRequests = 4096;  // per-request arrays are copied to shared memory up to this batch
 constexpr int kMergeGroup = 8;              // chunk states loaded at once by the merging warp
+constexpr int kCombineGroup = 4;            // items a warp folds before one fence and its counter updates
 
 template <int D>
 struct CombineVec {
@@ -76,117 +77,156 @@ __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_ke
   }
   griddep_wait();  // the split kernel's partials are complete and visible
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t rows_per_b = (int64_t)p.T * p.Hq;
-  const int64_t total = rows_per_b * cb_sm[p.B];
-  const int64_t nwarps = (int64_t)gridDim.x * kCombineWarps;
+  // item numbers fit 32 bits (checked on the host), so does every product below
+  const int rows_per_b = p.T * p.Hq;
+  const int total = rows_per_b * cb_sm[p.B];
+  const int nwarps = gridDim.x * kCombineWarps;
 
-  for (int64_t w = (int64_t)blockIdx.x * kCombineWarps + warp; w < total; w += nwarps) {
-    int lo = 0, hi = p.B - 1;  // request: last b with rows_per_b * cb[b] <= w
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (rows_per_b * cb_sm[mid] <= w) lo = mid; else hi = mid - 1;
-    }
-    const int b = lo;
-    const int ncb = cb_sm[b + 1] - cb_sm[b];
-    const int64_t local = w - rows_per_b * cb_sm[b];
-    const int row_in_b = (int)(local / ncb), j = (int)(local - (int64_t)row_in_b * ncb);
-    const int t = row_in_b / p.Hq, qh = row_in_b - t * p.Hq;
-    const int64_t row = ((int64_t)b * p.T + t) * p.Hq + qh;
-    float* orow = p.out + row * D;
-    const int L = Ls[b];
-    const int nb = L > 0 ? (L + p.tl - 1) / p.tl : 0;
-    float acc[VEC];
-    #pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-    if (nb == 0) {  // no key at all
-      write_row<D>(orow, p.lse + row, lane, -INFINITY, 0.f, acc);
-      continue;
-    }
-    const int h = qh / p.G, r = t * p.G + (qh - h * p.G);
-    const int nbs = S[b + 1] - S[b];  // == nb
-    const int64_t slot0 = (int64_t)p.Hkv * S[b] + (int64_t)h * nbs + (int64_t)j * kCombineChunk;
-    const int n = min(kCombineChunk, nb - j * kCombineChunk);
-    // ---- fold up to kCombineChunk partial rows
-    const float my_lse = lane < n ? p.part_lse[(slot0 + lane) * p.GT + r] : -INFINITY;
-    V v[kCombineChunk];
-    #pragma unroll
-    for (int i = 0; i < kCombineChunk; ++i)
-      if (i < n) v[i] = reinterpret_cast<const V*>(p.part_o + ((slot0 + i) * p.GT + r) * D)[lane];
-    float M = my_lse;
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float my_w = (lane < n && M != -INFINITY) ? expf(my_lse - M) : 0.f;
-    float W = my_w;
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
-    #pragma unroll
-    for (int i = 0; i < kCombineChunk; ++i) {
-      const float wi = __shfl_sync(0xffffffffu, my_w, i);
-      if (i < n) {
-        const float* f = reinterpret_cast<const float*>(&v[i]);
-        #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[e] += wi * f[e];
-      }
-    }
-    if (ncb == 1) {
-      write_row<D>(orow, p.lse + row, lane, M, W, acc);
-      continue;
-    }
-    // ---- publish this chunk; the last chunk of the row merges them all
-    float* cs = p.chunk_state + w * (D + 4);
-    #pragma unroll
-    for (int e = 0; e < VEC; ++e) cs[4 + lane * VEC + e] = acc[e];
-    if (lane == 0) { cs[0] = M; cs[1] = W; }
-    __threadfence();
-    __syncwarp();
-    int prev = 0;
-    if (lane == 0) prev = atomicAdd(&p.row_cnt[row], 1);
-    prev = __shfl_sync(0xffffffffu, prev, 0);
-    if (prev != ncb - 1) continue;
-    __threadfence();
-    // all chunk states of the row, in groups of kMergeGroup loaded at once (from L2: they were
-    // written by other warps of this grid)
-    const float* cs0 = p.chunk_state + (w - j) * (D + 4);
-    float Mt = -INFINITY, Wt = 0.f;
-    #pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+  // The warp's items w0, w0 + nwarps, ... are taken kCombineGroup at a time: each is folded; a
+  // row made of one chunk is written at once, the others publish their chunk state. Then one
+  // fence for the group and the row counters of its items bumped together (one lane each);
+  // the warp merges the rows it completed.
+  for (int w0 = blockIdx.x * kCombineWarps + warp; w0 < total; w0 += nwarps * kCombineGroup) {
+    int64_t g_row = -1;  // lane k: row of the group's k-th item if that item published a chunk
+    int g_first = 0;     // lane k: item number of chunk 0 of that row
+    int g_ncb = 0;       // lane k: chunks of that row
     #pragma unroll 1
-    for (int c0 = 0; c0 < ncb; c0 += kMergeGroup) {
-      const int nc = min(kMergeGroup, ncb - c0);
-      const float* g = cs0 + (int64_t)c0 * (D + 4);
-      const float2 mw = lane < nc ? __ldcg(reinterpret_cast<const float2*>(g + (int64_t)lane * (D + 4)))
-                                  : make_float2(-INFINITY, 0.f);
-      const float mc = mw.x, wc = mw.y;
-      V cv[kMergeGroup];
+    for (int k = 0; k < kCombineGroup; ++k) {
+      const int64_t wl = (int64_t)w0 + (int64_t)k * nwarps;
+      if (wl >= total) break;
+      const int w = (int)wl;
+      int lo = 0, hi = p.B - 1;  // request: last b with rows_per_b * cb[b] <= w
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (rows_per_b * cb_sm[mid] <= w) lo = mid; else hi = mid - 1;
+      }
+      const int b = lo;
+      const int ncb = cb_sm[b + 1] - cb_sm[b];
+      const int local = w - rows_per_b * cb_sm[b];
+      const int row_in_b = local / ncb, j = local - row_in_b * ncb;
+      const int t = row_in_b / p.Hq, qh = row_in_b - t * p.Hq;
+      const int64_t row = ((int64_t)b * p.T + t) * p.Hq + qh;
+      float* orow = p.out + row * D;
+      const int L = Ls[b];
+      const int nb = L > 0 ? (L + p.tl - 1) / p.tl : 0;
+      float acc[VEC];
       #pragma unroll
-      for (int i = 0; i < kMergeGroup; ++i)
-        if (i < nc) cv[i] = __ldcg(reinterpret_cast<const V*>(g + (int64_t)i * (D + 4) + 4) + lane);
-      float Mg = mc;
+      for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+      if (nb == 0) {  // no key at all
+        write_row<D>(orow, p.lse + row, lane, -INFINITY, 0.f, acc);
+        continue;
+      }
+      const int h = qh / p.G, r = t * p.G + (qh - h * p.G);
+      const int nbs = S[b + 1] - S[b];  // == nb
+      const int64_t slot0 = (int64_t)p.Hkv * S[b] + (int64_t)h * nbs + (int64_t)j * kCombineChunk;
+      const int n = min(kCombineChunk, nb - j * kCombineChunk);
+      // ---- fold up to kCombineChunk partial rows, in two halves of loads in flight at once
+      //      (with every warp loading, the fold runs at DRAM bandwidth; halves keep the
+      //      registers below the occupancy limit)
+      const float my_lse = lane < n ? p.part_lse[(slot0 + lane) * p.GT + r] : -INFINITY;
+      const V* src = reinterpret_cast<const V*>(p.part_o + (slot0 * p.GT + r) * D) + lane;
+      const int64_t stride = (int64_t)p.GT * (D / VEC);  // V elements between consecutive tiles' rows
+      constexpr int kHalf = kCombineChunk / 2;
+      V v[kHalf];
       #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) Mg = fmaxf(Mg, __shfl_xor_sync(0xffffffffu, Mg, o));
-      const float Mn = fmaxf(Mt, Mg);
-      if (Mn == -INFINITY) continue;  // no visible key in any chunk so far
-      const float a = Mt == -INFINITY ? 0.f : expf(Mt - Mn);
-      const float wl = mc == -INFINITY ? 0.f : expf(mc - Mn);
-      float Wg = wl * wc;
+      for (int i = 0; i < kHalf; ++i)
+        if (i < n) v[i] = __ldcs(src + i * stride);
+      float M = my_lse;
       #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) Wg += __shfl_xor_sync(0xffffffffu, Wg, o);
-      Wt = Wt * a + Wg;
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      const float my_w = (lane < n && M != -INFINITY) ? expf(my_lse - M) : 0.f;
+      float W = my_w;
       #pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[e] *= a;
+      for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
       #pragma unroll
-      for (int i = 0; i < kMergeGroup; ++i) {
-        const float wi = __shfl_sync(0xffffffffu, wl, i);
-        if (i < nc) {
-          const float* f = reinterpret_cast<const float*>(&cv[i]);
+      for (int hf = 0; hf < 2; ++hf) {
+        if (hf == 1) {
+          if (n <= kHalf) break;
           #pragma unroll
-          for (int e = 0; e < VEC; ++e) acc[e] += wi * f[e];
+          for (int i = 0; i < kHalf; ++i)
+            if (kHalf + i < n) v[i] = __ldcs(src + (kHalf + i) * stride);
+        }
+        #pragma unroll
+        for (int i = 0; i < kHalf; ++i) {
+          const float wi = __shfl_sync(0xffffffffu, my_w, hf * kHalf + i);
+          if (hf * kHalf + i < n) {
+            const float* f = reinterpret_cast<const float*>(&v[i]);
+            #pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] += wi * f[e];
+          }
         }
       }
-      Mt = Mn;
+      if (ncb == 1) {
+        write_row<D>(orow, p.lse + row, lane, M, W, acc);
+        continue;
+      }
+      // ---- publish this chunk
+      float* cs = p.chunk_state + (int64_t)w * (D + 4);
+      V av;
+      #pragma unroll
+      for (int e = 0; e < VEC; ++e) reinterpret_cast<float*>(&av)[e] = acc[e];
+      reinterpret_cast<V*>(cs + 4)[lane] = av;
+      if (lane == 0) *reinterpret_cast<float2*>(cs) = make_float2(M, W);
+      if (lane == k) { g_row = row; g_first = w - j; g_ncb = ncb; }
     }
-    write_row<D>(orow, p.lse + row, lane, Mt, Wt, acc);
-    if (lane == 0) p.row_cnt[row] = 0;  // ready for the next combine on this workspace
+    if (__ballot_sync(0xffffffffu, g_row >= 0) == 0u) continue;
+    __threadfence();  // the group's chunk states are visible before its counters move
+    int prev = -1;
+    if (g_row >= 0) prev = atomicAdd(&p.row_cnt[g_row], 1);
+    unsigned last = __ballot_sync(0xffffffffu, g_row >= 0 && prev == g_ncb - 1);
+    if (last == 0u) continue;
+    __threadfence();  // and the other chunks' states are read after the counter
+    while (last != 0u) {
+      const int k = __ffs(last) - 1;
+      last &= last - 1u;
+      const int64_t row = __shfl_sync(0xffffffffu, g_row, k);
+      const int first = __shfl_sync(0xffffffffu, g_first, k);
+      const int ncb = __shfl_sync(0xffffffffu, g_ncb, k);
+      // ---- merge the row's chunk states, kMergeGroup loaded at once (from L2: they were written
+      //      by other warps of this grid), with an online rescale between groups
+      const float* cs0 = p.chunk_state + (int64_t)first * (D + 4);
+      float acc[VEC];
+      float Mt = -INFINITY, Wt = 0.f;
+      #pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+      #pragma unroll 1
+      for (int c0 = 0; c0 < ncb; c0 += kMergeGroup) {
+        const int nc = min(kMergeGroup, ncb - c0);
+        const float* g = cs0 + (int64_t)c0 * (D + 4);
+        const float2 mw = lane < nc ? __ldcg(reinterpret_cast<const float2*>(g + (int64_t)lane * (D + 4)))
+                                    : make_float2(-INFINITY, 0.f);
+        const float mc = mw.x, wc = mw.y;
+        V cv[kMergeGroup];
+        #pragma unroll
+        for (int i = 0; i < kMergeGroup; ++i)
+          if (i < nc) cv[i] = __ldcg(reinterpret_cast<const V*>(g + (int64_t)i * (D + 4) + 4) + lane);
+        float Mg = mc;
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Mg = fmaxf(Mg, __shfl_xor_sync(0xffffffffu, Mg, o));
+        const float Mn = fmaxf(Mt, Mg);
+        if (Mn == -INFINITY) continue;  // no visible key in any chunk so far
+        const float a = Mt == -INFINITY ? 0.f : expf(Mt - Mn);
+        const float wl = mc == -INFINITY ? 0.f : expf(mc - Mn);
+        float Wg = wl * wc;
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Wg += __shfl_xor_sync(0xffffffffu, Wg, o);
+        Wt = Wt * a + Wg;
+        #pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] *= a;
+        #pragma unroll
+        for (int i = 0; i < kMergeGroup; ++i) {
+          const float wi = __shfl_sync(0xffffffffu, wl, i);
+          if (i < nc) {
+            const float* f = reinterpret_cast<const float*>(&cv[i]);
+            #pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] += wi * f[e];
+          }
+        }
+        Mt = Mn;
+      }
+      write_row<D>(p.out + row * D, p.lse + row, lane, Mt, Wt, acc);
+      if (lane == 0) p.row_cnt[row] = 0;  // ready for the next combine on this workspace
+    }
   }
 }
 
