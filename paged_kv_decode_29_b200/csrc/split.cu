@@ -22,6 +22,11 @@
 //    M). Probabilities go to the MMA as bf16 hi + bf16 lo (BF16 KV: two columns of the
 //    same MMA when G*T <= 4, two N tiles otherwise), or as f16 scaled by the page's V
 //    scale (FP8 KV).
+//  * FP8 KV: S^T runs on E4M3 MMAs straight from the staged codes (K is never widened);
+//    V is widened to f16. With one consumer warp it is widened in registers; with two,
+//    each widens half of every V block into a shared f16 block (laid out like a bf16
+//    stage, two buffers) and both read V^T from it with ldmatrix, so no element is
+//    widened twice; the raw stage is released as soon as it is widened and used for S^T.
 //  * the tile ends with either the final output (the tile covers its whole request) or
 //    a normalised partial (o, lse) in the workspace for the combine kernel.
 //
@@ -47,7 +52,6 @@ struct Geo {
   static constexpr int BOX_ELEMS = RB / ESZ;
   static constexpr int BOX_BYTES = 16 * RB;
   static constexpr int TILE = 16 * ROW;                         // K (or V) bytes per stage
-  static constexpr int STAGES = (40 * 1024) / (2 * TILE);
   static_assert(RB == 128 || RB == 64, "box rows are 64 or 128 bytes");
   // byte offset of (row r, 16-byte chunk cg of the full row) in a stage buffer
   __device__ static __forceinline__ uint32_t off(int r, int cg) {
@@ -57,15 +61,21 @@ struct Geo {
   }
 };
 
-template <int KVT, int D, int NQ>
+// VSH: the consumer warps share the widening of each FP8 V block (two f16 blocks in the layout
+// of a bf16 stage, after the ring).
+template <int KVT, int D, int NQ, bool VSH>
 struct Smem {
   using G_ = Geo<KVT, D>;
+  using G16 = Geo<0, D>;                                         // layout of a widened V block
+  static constexpr int V16 = VSH ? 2 * G16::TILE : 0;
+  static constexpr int STAGES = (40 * 1024 - V16) / (2 * G_::TILE);
   static constexpr int QBYTES = 8 * NQ * D * 2;
-  static constexpr int OFF_Q = G_::STAGES * 2 * G_::TILE;
+  static constexpr int OFF_V16 = STAGES * 2 * G_::TILE;
+  static constexpr int OFF_Q = OFF_V16 + V16;
   static constexpr int OFF_BAR = OFF_Q + 2 * QBYTES;
-  static constexpr int NBAR = 2 * G_::STAGES + 4;
+  static constexpr int NBAR = 2 * STAGES + 4 + (VSH ? 2 : 0);   // full, empty, qfull, qempty, vready
   static constexpr int OFF_META = OFF_BAR + 8 * NBAR;            // per stage: pad, K scale, V scale, pad
-  static constexpr int OFF_QMETA = OFF_META + 16 * G_::STAGES;   // Unit x 2
+  static constexpr int OFF_QMETA = OFF_META + 16 * STAGES;       // Unit x 2
   static constexpr int BYTES = OFF_QMETA + 2 * (int)sizeof(Unit);
   static constexpr int ALLOC = BYTES + 1024;                     // slack to align the base to 1024
 };
@@ -185,8 +195,11 @@ template <int KVT, int D, int NQ, int NPV, bool DUP, int NCW>
 __global__ void __launch_bounds__(32 * (1 + NCW), kCtasPerSm)
 split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   using G_ = Geo<KVT, D>;
-  using S_ = Smem<KVT, D, NQ>;
-  constexpr int STAGES = G_::STAGES;
+  // FP8 with two consumer warps: each widens half of every V block into a shared f16 block
+  constexpr bool VSH = KVT == 1 && NCW == 2;
+  using S_ = Smem<KVT, D, NQ, VSH>;
+  using G16 = typename S_::G16;
+  constexpr int STAGES = S_::STAGES;
   constexpr int NQW = NQ / NCW;    // S^T tiles per consumer warp
   constexpr int NPVW = NPV / NCW;  // O^T tiles per consumer warp
   static_assert(NQ % NCW == 0 && NPV % NCW == 0, "tiles split evenly over the consumer warps");
@@ -197,6 +210,7 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   uint64_t* empty = bar + STAGES;
   uint64_t* qfull = bar + 2 * STAGES;
   uint64_t* qempty = bar + 2 * STAGES + 2;
+  uint64_t* vready = bar + 2 * STAGES + 4;  // VSH: both halves of widened V block b are written
   float* meta_sc = reinterpret_cast<float*>(sm + S_::OFF_META);      // [s*4 + 1] = K scale, [s*4 + 2] = V scale
   Unit* qmeta = reinterpret_cast<Unit*>(sm + S_::OFF_QMETA);
 
@@ -209,6 +223,8 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 32 * NCW); }
     for (int s = 0; s < 2; ++s) { mbar_init(&qfull[s], 1); mbar_init(&qempty[s], 32 * NCW); }
+    if (VSH)
+      for (int b = 0; b < 2; ++b) mbar_init(&vready[b], 32 * NCW);
     fence_mbar_init();
   }
   __syncthreads();
@@ -364,6 +380,8 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
   const int nq0 = (warp - 1) * NQW;  // first S^T tile of this consumer warp
   int s = 0; uint32_t fph = 0;
   int qs = 0; uint32_t qfph = 0;
+  int vblk = 0;       // VSH: V blocks widened so far (block vblk uses buffer vblk & 1)
+  uint32_t vph = 0;   // VSH: bit b = phase of vready[b] to wait for next
   const float LN2 = 0.6931471805599453f;
   for (;;) {
     if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qs], qfph, p.status))) return;
@@ -471,11 +489,34 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
         sc2 *= meta_sc[s * 4 + 1];
         vsc = meta_sc[s * 4 + 2] * kPScale;
       }
+      const int vb = vblk & 1;
+      if (VSH) {
+        // ---- widen this warp's half of the V block (d in [D/2 * (warp-1), D/2 * warp)) to f16
+        //      in the layout of a bf16 stage; two lanes per key, 16 codes per 16-byte chunk
+        constexpr int CH = D / 16 / NCW;  // raw 16-byte chunks of a key row per warp
+        const uint8_t* vraw = sm + s * 2 * G_::TILE + G_::TILE;
+        uint8_t* v16 = sm + S_::OFF_V16 + vb * G16::TILE;
+        const int key = lane >> 1, hh = lane & 1;
+        #pragma unroll
+        for (int c = 0; c < CH / 2; ++c) {
+          const int cg = (warp - 1) * CH + hh * (CH / 2) + c;  // codes d = 16 cg .. 16 cg + 15
+          const uint4 w = *reinterpret_cast<const uint4*>(vraw + G_::off(key, cg));
+          uint4 lo, hi;
+          lo.x = e4m3x2_to_f16x2(w.x & 0xffffu); lo.y = e4m3x2_to_f16x2(w.x >> 16);
+          lo.z = e4m3x2_to_f16x2(w.y & 0xffffu); lo.w = e4m3x2_to_f16x2(w.y >> 16);
+          hi.x = e4m3x2_to_f16x2(w.z & 0xffffu); hi.y = e4m3x2_to_f16x2(w.z >> 16);
+          hi.z = e4m3x2_to_f16x2(w.w & 0xffffu); hi.w = e4m3x2_to_f16x2(w.w >> 16);
+          *reinterpret_cast<uint4*>(v16 + G16::off(key, 2 * cg)) = lo;
+          *reinterpret_cast<uint4*>(v16 + G16::off(key, 2 * cg + 1)) = hi;
+        }
+        mbar_arrive(&vready[vb]);
+      }
       // ---- S^T = K Q^T  (rows: 16 keys; columns: query rows). Even and odd k-steps go to two
       //      accumulators so that two MMA chains are in flight.
-      float sacc[2][NQW][4];
+      constexpr int NCH = KVT == 1 ? 4 : 2;  // independent accumulation chains
+      float sacc[NCH][NQW][4];
       #pragma unroll
-      for (int c = 0; c < 2; ++c)
+      for (int c = 0; c < NCH; ++c)
         #pragma unroll
         for (int nw = 0; nw < NQW; ++nw) sacc[c][nw][0] = sacc[c][nw][1] = sacc[c][nw][2] = sacc[c][nw][3] = 0.f;
       {
@@ -497,11 +538,16 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
             ldsm_x4(ks + G_::off(r, 2 * kk + (lane >> 4)), a[0], a[1], a[2], a[3]);
             #pragma unroll
             for (int nw = 0; nw < NQW; ++nw) {
-              mma_e4m3(sacc[0][nw], a, qf[nw][kk][0], qf[nw][kk][1]);
-              mma_e4m3(sacc[1][nw], a, ql[nw][kk][0], ql[nw][kk][1]);
+              mma_e4m3(sacc[2 * (kk & 1)][nw], a, qf[nw][kk][0], qf[nw][kk][1]);
+              mma_e4m3(sacc[2 * (kk & 1) + 1][nw], a, ql[nw][kk][0], ql[nw][kk][1]);
             }
           }
         }
+      }
+      if (VSH) {
+        // the raw stage is no longer read: K went into S^T, this warp's half of V into the f16 block
+        __syncwarp();
+        mbar_arrive(&empty[s]);
       }
       // ---- scale, mask, online softmax (log2 domain, fp32 state)
       const bool need_mask = kbase + 16 > safe_end;
@@ -513,7 +559,9 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
         float sv4[4];
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          sv4[i] = (sacc[0][nw][i] + sacc[1][nw][i]) * (KVT == 1 ? sc2 * qcs[nw][i & 1] : sc2);
+          const float sum = KVT == 1 ? (sacc[0][nw][i] + sacc[1][nw][i]) + (sacc[NCH - 2][nw][i] + sacc[NCH - 1][nw][i])
+                                     : sacc[0][nw][i] + sacc[1][nw][i];
+          sv4[i] = sum * (KVT == 1 ? sc2 * qcs[nw][i & 1] : sc2);
           if (need_mask) {
             const int j = kbase + gid + (i >> 1) * 8;
             if (j >= d.tok_end || j > lim[nw][i & 1]) sv4[i] = -INFINITY;
@@ -581,6 +629,20 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
           #pragma unroll
           for (int j = 0; j < NPVW; ++j) mma_bf16(o[j][mt], a, bp[j][0], bp[j][1]);
         }
+      } else if (VSH) {
+        // both halves of the widened block are written: f16 V^T fragments as in the bf16 path
+        if (!__all_sync(0xffffffffu, mbar_wait(&vready[vb], (vph >> vb) & 1u, p.status))) return;
+        vph ^= 1u << vb;
+        const uint32_t v16 = smem_u32(sm + S_::OFF_V16 + vb * G16::TILE);
+        const int q4 = lane >> 3;
+        const int r = (lane & 7) + (q4 >> 1) * 8;
+        #pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          uint32_t a[4];
+          ldsm_x4_t(v16 + G16::off(r, 2 * mt + (q4 & 1)), a[0], a[1], a[2], a[3]);
+          #pragma unroll
+          for (int j = 0; j < NPVW; ++j) mma_f16(o[j][mt], a, bp[j][0], bp[j][1]);
+        }
       } else {
         // thread (gid, tig) reads 4 codes at d = 32pp + 4gid .. +3 of keys 2tig, 2tig+1,
         // 2tig+8, 2tig+9 and pairs them by key: M-row gid of m-tile 2pp+sub is
@@ -608,8 +670,11 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
           }
         }
       }
-      __syncwarp();
-      mbar_arrive(&empty[s]);
+      if (!VSH) {
+        __syncwarp();
+        mbar_arrive(&empty[s]);
+      }
+      ++vblk;
       if (++s == STAGES) { s = 0; fph ^= 1; }
     }
 
@@ -664,13 +729,13 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
           dst = p.part_o + row * D;
           dst_lse = p.part_lse + row;
         }
-        if (KVT == 0) {
+        if (KVT == 0 || VSH) {  // M-row gid of m-tile mt is d = 16 mt + gid
           #pragma unroll
           for (int mt = 0; mt < D / 16; ++mt) {
             dst[16 * mt + gid] = o[j][mt][e] * inv;
             dst[16 * mt + gid + 8] = o[j][mt][2 + e] * inv;
           }
-        } else {
+        } else {  // register-widened FP8 V: M-row gid of m-tile 2pp+sub is d = 32pp + 4gid + 2sub
           #pragma unroll
           for (int pp = 0; pp < D / 32; ++pp) {
             float4 v;
@@ -692,7 +757,7 @@ template <int KVT, int D, int NQ, int NPV, bool DUP, int NCW>
 static cudaError_t launch_variant(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                   cudaStream_t st) {
   auto fn = split_kernel<KVT, D, NQ, NPV, DUP, NCW>;
-  const int smem = Smem<KVT, D, NQ>::ALLOC;
+  const int smem = Smem<KVT, D, NQ, KVT == 1 && NCW == 2>::ALLOC;
   if (!ensure_smem_attr((const void*)fn, smem)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_bins);
