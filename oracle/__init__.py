@@ -74,6 +74,11 @@ def _load():
             lib.oracle_e4m3_value.argtypes = [C.c_uint8]
             lib.oracle_e4m3_value.restype = C.c_double
             lib.oracle_max_threads.restype = C.c_int
+            lib.oracle_rope_row.argtypes = [C.c_void_p, C.c_int, C.c_double, C.c_double, C.c_void_p]
+            lib.oracle_bf16_bits.argtypes = [C.c_double]
+            lib.oracle_bf16_bits.restype = C.c_uint16
+            lib.oracle_append_rope.argtypes = [C.c_void_p] * 5 + [C.c_int] * 8 + [C.c_double] + [C.c_void_p] * 3
+            lib.oracle_append_rope.restype = C.c_int64
             _lib = lib
     return _lib
 
@@ -174,3 +179,47 @@ def e4m3_value(code: int) -> float:
 
 def e4m3_table() -> np.ndarray:
     return np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+# ---- fused pre-processing of a decode step: rotary embedding + KV append (oracle.c)
+
+def rope_rows(x, positions, base: float = 10000.0):
+    """fp64 rotate-half rotary embedding of the rows x[n][d] at positions[n] (no rounding)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    n, d = x.shape
+    pos = np.asarray(positions, dtype=np.float64).reshape(n)
+    y = np.empty_like(x)
+    for i in range(n):
+        lib.oracle_rope_row(x[i].ctypes.data, int(d), float(pos[i]), float(base), y[i].ctypes.data)
+    return y
+
+
+def bf16_bits(values):
+    """bf16 bit patterns nearest to the fp64 values (ties to even)."""
+    lib = _load()
+    v = np.asarray(values, dtype=np.float64)
+    return np.array([lib.oracle_bf16_bits(float(x)) for x in v.reshape(-1)], dtype=np.uint16).reshape(v.shape)
+
+
+def append_rope(q_new, k_new, v_new, page_table, seq_lens, k_pages, v_pages, base: float = 10000.0):
+    """Rotary embedding of the T new q and k rows and their append to the paged cache.
+    q_new [B][T][Hq][d], k_new / v_new [B][T][Hkv][d], k_pages / v_pages [num_pages][Hkv][P][d]:
+    bf16 bit patterns (uint16). Returns (q_out, k_pages', v_pages', rows written), the pages
+    copied, or rows written = -1 for a page id out of range."""
+    lib = _load()
+    qn = np.ascontiguousarray(q_new, dtype=np.uint16)
+    kn = np.ascontiguousarray(k_new, dtype=np.uint16)
+    vn = np.ascontiguousarray(v_new, dtype=np.uint16)
+    tab = np.ascontiguousarray(page_table, dtype=np.int32)
+    L = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    kp = np.array(k_pages, dtype=np.uint16, copy=True, order="C")
+    vp = np.array(v_pages, dtype=np.uint16, copy=True, order="C")
+    B, T, Hq, d = qn.shape
+    Hkv = kn.shape[2]
+    num_pages, _, P, _ = kp.shape
+    q_out = np.empty_like(qn)
+    n = lib.oracle_append_rope(qn.ctypes.data, kn.ctypes.data, vn.ctypes.data, tab.ctypes.data, L.ctypes.data,
+                               B, T, Hq, Hkv, d, P, num_pages, int(tab.shape[1]), float(base), q_out.ctypes.data,
+                               kp.ctypes.data, vp.ctypes.data)
+    return q_out, kp, vp, int(n)

@@ -230,3 +230,94 @@ int64_t oracle_plan(const int32_t *seq_lens, int B, int Hkv, int tl, int n_bins,
     free(tb); free(key); free(load); free(count); free(bin_of); free(rank_in_bin);
     return U;
 }
+
+/* ------------------------------------------------------------------------------------------
+ * Fused pre-processing of a decode step: rotary position embedding of the new q and k, and
+ * the append of the new K/V rows into their pages ("PaddlePaddle/HALOps" README, Highlights,
+ * GQA attention item: fused pre/post-processing around paged-KV decode). The pages name this
+ * step without defining it; the reading written out here:
+ *  - rotate-half rotary embedding: for i < d/2, theta_i = base^(-2i/d), and the pair
+ *    (x_i, x_{i+d/2}) of a row at position pos becomes
+ *    (x_i cos(pos theta_i) - x_{i+d/2} sin(pos theta_i), x_{i+d/2} cos(pos theta_i) + x_i sin(pos theta_i));
+ *  - the T new tokens of request b sit at positions Lb - T + t, t < T (seq_lens already
+ *    counts them, as the decode does);
+ *  - rotated q goes to q_out; rotated k and unchanged v go to page page_table[b][pos / P],
+ *    slot pos % P, of their KV head; stored values are the bf16 nearest to the fp64 result;
+ *  - a token with pos < 0 has no slot: nothing is written for it and its q row is the
+ *    rotation at position 0 (the identity).
+ * ------------------------------------------------------------------------------------------ */
+
+/* The rotation of one row of d values at position pos, in fp64. */
+void oracle_rope_row(const double *x, int d, double pos, double base, double *y)
+{
+    int half = d / 2;
+    for (int i = 0; i < half; ++i) {
+        double theta = pow(base, -2.0 * i / d);
+        double c = cos(pos * theta), s = sin(pos * theta);
+        y[i] = x[i] * c - x[i + half] * s;
+        y[i + half] = x[i + half] * c + x[i] * s;
+    }
+}
+
+/* The bf16 (8 significant bits, binary32's exponent range) nearest to v, ties to even, as its
+ * bit pattern; rounded in one step from the double (no detour through binary32). */
+uint16_t oracle_bf16_bits(double v)
+{
+    if (isnan(v)) return 0x7fc0;
+    int sgn = signbit(v) ? 1 : 0;
+    double a = fabs(v), r;
+    if (a == 0.0) return (uint16_t)(sgn << 15);
+    int e;
+    frexp(a, &e);                     /* a = m 2^e, m in [0.5, 1) */
+    if (e < -125) e = -125;           /* below the normal range the spacing stays 2^-133 */
+    r = ldexp(rint(ldexp(a, 8 - e)), e - 8);
+    if (r >= 0x1p128) return (uint16_t)((sgn << 15) | 0x7f80);
+    float f = (float)r;               /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)((u >> 16) | (uint32_t)(sgn << 15));
+}
+
+/* Applies the pre-processing to bf16 inputs. q_new [B][T][Hq][d], k_new / v_new [B][T][Hkv][d]
+ * (bf16 bits); q_out [B][T][Hq][d]; k_pages / v_pages [num_pages][Hkv][P][d] (bf16 bits,
+ * updated in place). Returns the number of (token, KV head) rows written, or -1 if a page id
+ * read for a written row lies outside [0, num_pages) or past the page-table row. */
+int64_t oracle_append_rope(const uint16_t *q_new, const uint16_t *k_new, const uint16_t *v_new,
+                           const int32_t *page_table, const int32_t *seq_lens, int B, int T, int Hq,
+                           int Hkv, int d, int P, int num_pages, int mpps, double base, uint16_t *q_out,
+                           uint16_t *k_pages, uint16_t *v_pages)
+{
+    double *x = (double *)malloc(sizeof(double) * (size_t)d);
+    double *y = (double *)malloc(sizeof(double) * (size_t)d);
+    int64_t written = 0;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            int64_t pos = (int64_t)seq_lens[b] - T + t;
+            double rpos = pos < 0 ? 0.0 : (double)pos;
+            for (int qh = 0; qh < Hq; ++qh) {
+                size_t o = (((size_t)b * T + t) * Hq + qh) * d;
+                for (int c = 0; c < d; ++c) x[c] = bf16_value(q_new[o + c]);
+                oracle_rope_row(x, d, rpos, base, y);
+                for (int c = 0; c < d; ++c) q_out[o + c] = oracle_bf16_bits(y[c]);
+            }
+            if (pos < 0) continue;
+            if (pos / P >= mpps) { written = -1; goto done; }
+            int32_t pid = page_table[(int64_t)b * mpps + pos / P];
+            if (pid < 0 || pid >= num_pages) { written = -1; goto done; }
+            for (int h = 0; h < Hkv; ++h) {
+                size_t in = (((size_t)b * T + t) * Hkv + h) * d;
+                size_t dst = (((size_t)pid * Hkv + h) * P + (size_t)(pos % P)) * d;
+                for (int c = 0; c < d; ++c) x[c] = bf16_value(k_new[in + c]);
+                oracle_rope_row(x, d, (double)pos, base, y);
+                for (int c = 0; c < d; ++c) {
+                    k_pages[dst + c] = oracle_bf16_bits(y[c]);
+                    v_pages[dst + c] = v_new[in + c];
+                }
+                ++written;
+            }
+        }
+done:
+    free(x);
+    free(y);
+    return written;
+}
