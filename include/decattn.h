@@ -219,6 +219,41 @@ DECATTN_API int dec_attn_read_status(const dec_attn_plan_t *plan, const void *wo
 /* Static text for a decattn_status value. */
 DECATTN_API const char *dec_attn_status_string(int status);
 
+/* Fused pre-processing of a decode step ("PaddlePaddle/HALOps" README, Highlights, GQA
+ * attention item: fused pre/post-processing around paged-KV decode). The pages name the step
+ * without defining it; the reading implemented, in one kernel on `stream`:
+ *   - rotary position embedding, rotate-half form: for i < d/2, theta_i = rope_base^(-2i/d),
+ *     and the pair (x_i, x_{i+d/2}) of a row at position pos becomes
+ *     (x_i cos(pos theta_i) - x_{i+d/2} sin(pos theta_i), x_{i+d/2} cos(pos theta_i) + x_i sin(pos theta_i)),
+ *     computed in fp32 from an fp64 angle and rounded to bf16 (nearest, ties to even);
+ *   - the T = shape->q_tokens new tokens of request b sit at positions Lb - T + t, t < T:
+ *     seq_lens must already count them, exactly as dec_attn_run expects;
+ *   - q_out[b][t][qh] = rotated q_new[b][t][qh]; the rotated k_new[b][t][h] and the unchanged
+ *     v_new[b][t][h] are written to page page_table[b][pos / P], slot pos % P, of KV head h;
+ *   - a token with pos < 0 (Lb < T) has no slot: nothing is written for it and its q row is
+ *     copied unrotated (the rotation at position 0).
+ * Run it before dec_attn_plan / dec_attn_run of the same step, on the same stream, passing
+ * q_out as their q. It is launched with programmatic stream serialisation and waits for the
+ * previous kernel of the stream before reading anything.
+ * Arguments (device pointers; 4-byte aligned for head_dim 128, 2-byte for 64):
+ *   shape       batch, n_q_heads, n_kv_heads, head_dim (64 or 128), q_tokens, page_size,
+ *               num_pages, max_pages_per_seq, kv_dtype (DECATTN_KV_BF16 only; sm_scale unused)
+ *   q_new       bf16 [B][T][Hq][d];  k_new, v_new  bf16 [B][T][Hkv][d]
+ *   page_table  int32 [B][max_pages_per_seq];  seq_lens  int32 [B]
+ *   rope_base   > 0 (10000 in the usual configuration)
+ *   q_out       bf16 [B][T][Hq][d], may be q_new (rotated in place)
+ *   k_pages, v_pages  bf16 [num_pages][Hkv][P][d], updated in place
+ *   status      optional device int32: a page id outside [0, num_pages), or a page past the
+ *               row's max_pages_per_seq entries, skips that token's K/V write and sets
+ *               DECATTN_EDEVICE here (first error wins; the caller zeroes it). May be NULL.
+ * Returns DECATTN_ENOTSUP for FP8 KV (appending to an FP8 page would need its scale, which
+ * covers the whole page) or another head_dim, DECATTN_EINVAL / DECATTN_EALIGN for bad
+ * arguments (nothing enqueued), DECATTN_ECUDA if the launch fails. */
+DECATTN_API int dec_attn_append_rope(const dec_attn_shape *shape, const void *q_new, const void *k_new,
+                                     const void *v_new, const int32_t *page_table, const int32_t *seq_lens,
+                                     float rope_base, void *q_out, void *k_pages, void *v_pages, int32_t *status,
+                                     void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,7 @@ OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1
 KV_BF16, KV_FP8E4M3 = 0, 1
 API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
-       "dec_attn_read_status", "dec_attn_status_string")
+       "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -84,6 +84,8 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_read_status.restype = i32
         lib.dec_attn_status_string.argtypes = [i32]
         lib.dec_attn_status_string.restype = C.c_char_p
+        lib.dec_attn_append_rope.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, C.c_float, vp, vp, vp, vp, vp]
+        lib.dec_attn_append_rope.restype = i32
         _lib = lib
         return lib
 
@@ -221,6 +223,28 @@ def run_noalloc(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, p
     if rc != OK:
         raise DecAttnError(rc, "dec_attn_run_noalloc")
     return out, lse
+
+
+def append_rope(q_new: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, page_table: torch.Tensor,
+                seq_lens: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, *,
+                q_out: torch.Tensor | None = None, rope_base: float = 10000.0,
+                status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """dec_attn_append_rope: rotary embedding of the step's new q / k rows and the append of the
+    new K/V rows into their pages (bf16 pools, updated in place); returns the rotated q.
+
+    q_new: bf16 [B][T][Hq][d]; k_new / v_new: bf16 [B][T][Hkv][d]; seq_lens: int32 [B], counting the
+    T new tokens (token t of request b sits at position Lb - T + t); ``status``: optional int32
+    device scalar that receives DECATTN_EDEVICE for a bad page id."""
+    lib = load_library()
+    shape = make_shape(q_new, k_pages, page_table, kv_dtype_of(k_pages))
+    if q_out is None:
+        q_out = torch.empty_like(q_new)
+    rc = lib.dec_attn_append_rope(C.byref(shape), _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(page_table),
+                                  _ptr(seq_lens), float(rope_base), _ptr(q_out), _ptr(k_pages), _ptr(v_pages),
+                                  _ptr(status), _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_append_rope")
+    return q_out
 
 
 def read_status(pl: Plan | None = None, workspace: torch.Tensor | None = None, stream=None) -> int:

@@ -1,0 +1,178 @@
+// append.cu -- the fused pre-processing of a decode step: rotary position embedding of the
+// step's new q and k rows, and the append of the new K/V rows into their pages, in one kernel
+// ("PaddlePaddle/HALOps" README, Highlights, GQA attention item: fused pre/post-processing
+// around paged-KV decode). The pages name the step without defining it; this kernel computes:
+//  * rotate-half rotary embedding: for i < d/2, theta_i = base^(-2i/d); the pair
+//    (x_i, x_{i+d/2}) at position pos becomes
+//    (x_i cos(pos theta_i) - x_{i+d/2} sin(pos theta_i), x_{i+d/2} cos(pos theta_i) + x_i sin(pos theta_i));
+//  * token t of request b sits at position Lb - T + t (seq_lens already counts the new tokens,
+//    as the decode does);
+//  * rotated q goes to q_out; rotated k and unchanged v go to page page_table[b][pos / P], slot
+//    pos % P, of their KV head; a token with pos < 0 has no slot (its q is left unrotated).
+//
+// One block per new token: the block computes (cos, sin) of its position once (the angle in
+// fp64: pos * theta in fp32 would be off by up to ~0.016 rad at pos = 131072), then its warps
+// take the token's Hq + 2 Hkv rows; lane l holds elements [E l, E l + E) of both halves, so
+// each rotation pair sits in one lane. Values are rotated in fp32 and rounded to bf16 (RNE).
+#include <cmath>
+
+#include "common.cuh"
+
+namespace decattn {
+
+constexpr int kAppendThreads = 128;
+
+struct AppendParams {
+  const uint16_t* q_new;   // bf16 [B][T][Hq][D]
+  const uint16_t* k_new;   // bf16 [B][T][Hkv][D]
+  const uint16_t* v_new;   // bf16 [B][T][Hkv][D]
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  uint16_t* q_out;         // bf16 [B][T][Hq][D] (may be q_new)
+  uint16_t* k_pages;       // bf16 [num_pages][Hkv][P][D]
+  uint16_t* v_pages;
+  int32_t* status;         // optional device word: DECATTN_EDEVICE for a bad page id
+  int B, T, Hq, Hkv, P, num_pages, mpps;
+  double base;
+};
+
+template <int E>
+struct AppendVec;
+template <>
+struct AppendVec<1> { using T = uint16_t; };
+template <>
+struct AppendVec<2> { using T = uint32_t; };
+
+template <int D>
+__global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const AppendParams p) {
+  constexpr int HALF = D / 2;
+  constexpr int E = D / 64;  // elements of each half per lane
+  using V = typename AppendVec<E>::T;
+  __shared__ float2 cs[HALF];  // (cos, sin) of pos * theta_i
+  // the inputs are written by the previous kernel of the stream
+  griddep_wait();
+  const int bt = blockIdx.x;
+  const int b = bt / p.T, t = bt - b * p.T;
+  const int64_t pos = (int64_t)p.seq_lens[b] - p.T + t;
+  const double rpos = pos < 0 ? 0.0 : (double)pos;
+  for (int i = threadIdx.x; i < HALF; i += kAppendThreads) {
+    const double theta = pow(p.base, -2.0 * i / D);
+    double s, c;
+    sincos(rpos * theta, &s, &c);
+    cs[i] = make_float2((float)c, (float)s);
+  }
+  // the page slot of this token (none for pos < 0, or for a bad page id, which is reported)
+  int64_t slot_row = -1;  // (page * Hkv) * P + slot, before adding the head
+  if (pos >= 0) {
+    const int64_t pg = pos / p.P;
+    int pid = -1;
+    if (pg < p.mpps) pid = p.page_table[(int64_t)b * p.mpps + pg];
+    if (pid >= 0 && pid < p.num_pages) {
+      slot_row = (int64_t)pid * p.Hkv * p.P + pos % p.P;
+    } else if (threadIdx.x == 0) {
+      set_status(p.status, DECATTN_EDEVICE);
+    }
+  }
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rows = p.Hq + 2 * p.Hkv;
+  for (int r = warp; r < rows; r += kAppendThreads / 32) {
+    const uint16_t* src;
+    uint16_t* dst;
+    bool rotate = true;
+    if (r < p.Hq) {
+      src = p.q_new + ((int64_t)bt * p.Hq + r) * D;
+      dst = p.q_out + ((int64_t)bt * p.Hq + r) * D;
+    } else {
+      const bool is_k = r < p.Hq + p.Hkv;
+      const int h = is_k ? r - p.Hq : r - p.Hq - p.Hkv;
+      if (slot_row < 0) continue;
+      src = (is_k ? p.k_new : p.v_new) + ((int64_t)bt * p.Hkv + h) * D;
+      dst = (is_k ? p.k_pages : p.v_pages) + (slot_row + (int64_t)h * p.P) * D;
+      rotate = is_k;
+    }
+    const V lo = reinterpret_cast<const V*>(src)[lane];
+    const V hi = reinterpret_cast<const V*>(src + HALF)[lane];
+    if (!rotate) {
+      reinterpret_cast<V*>(dst)[lane] = lo;
+      reinterpret_cast<V*>(dst + HALF)[lane] = hi;
+      continue;
+    }
+    float x1[E], x2[E];
+    #pragma unroll
+    for (int e = 0; e < E; ++e) {
+      x1[e] = __uint_as_float((uint32_t)((lo >> (16 * e)) & 0xffffu) << 16);
+      x2[e] = __uint_as_float((uint32_t)((hi >> (16 * e)) & 0xffffu) << 16);
+    }
+    V olo = 0, ohi = 0;
+    #pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float2 c = cs[E * lane + e];
+      const float y1 = x1[e] * c.x - x2[e] * c.y;
+      const float y2 = x2[e] * c.x + x1[e] * c.y;
+      olo |= (V)((V)__bfloat16_as_ushort(__float2bfloat16_rn(y1)) << (16 * e));
+      ohi |= (V)((V)__bfloat16_as_ushort(__float2bfloat16_rn(y2)) << (16 * e));
+    }
+    reinterpret_cast<V*>(dst)[lane] = olo;
+    reinterpret_cast<V*>(dst + HALF)[lane] = ohi;
+  }
+}
+
+cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t st) {
+  const int64_t blocks = (int64_t)p.B * p.T;
+  if (blocks <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(kAppendThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // launched while the previous kernel drains
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (D == 128) return cudaLaunchKernelEx(&cfg, append_rope_kernel<128>, p);
+  if (D == 64) return cudaLaunchKernelEx(&cfg, append_rope_kernel<64>, p);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace decattn
+
+using namespace decattn;
+
+extern "C" int dec_attn_append_rope(const dec_attn_shape* shape, const void* q_new, const void* k_new,
+                                    const void* v_new, const int32_t* page_table, const int32_t* seq_lens,
+                                    float rope_base, void* q_out, void* k_pages, void* v_pages, int32_t* status,
+                                    void* stream) {
+  if (!shape) return DECATTN_EINVAL;
+  const dec_attn_shape& s = *shape;
+  if (s.batch < 0 || s.q_tokens <= 0 || s.n_q_heads <= 0 || s.n_kv_heads <= 0 || s.page_size <= 0 ||
+      s.num_pages < 0 || s.max_pages_per_seq < 0 || s.n_q_heads % s.n_kv_heads != 0)
+    return DECATTN_EINVAL;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return DECATTN_EINVAL;
+  if (s.kv_dtype != DECATTN_KV_BF16) return DECATTN_ENOTSUP;  // an FP8 page's scale would need the whole page
+  if (s.head_dim != 64 && s.head_dim != 128) return DECATTN_ENOTSUP;
+  if (s.batch == 0) return DECATTN_OK;
+  if (!q_new || !k_new || !v_new || !page_table || !seq_lens || !q_out || !k_pages || !v_pages)
+    return DECATTN_EINVAL;
+  const uintptr_t need = s.head_dim == 128 ? 3 : 1;  // 4-byte (d = 128) or 2-byte lane accesses
+  for (const void* ptr : {q_new, k_new, v_new, (const void*)q_out, (const void*)k_pages, (const void*)v_pages})
+    if (reinterpret_cast<uintptr_t>(ptr) & need) return DECATTN_EALIGN;
+  AppendParams p;
+  p.q_new = static_cast<const uint16_t*>(q_new);
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.v_new = static_cast<const uint16_t*>(v_new);
+  p.page_table = page_table;
+  p.seq_lens = seq_lens;
+  p.q_out = static_cast<uint16_t*>(q_out);
+  p.k_pages = static_cast<uint16_t*>(k_pages);
+  p.v_pages = static_cast<uint16_t*>(v_pages);
+  p.status = status;
+  p.B = s.batch; p.T = s.q_tokens; p.Hq = s.n_q_heads; p.Hkv = s.n_kv_heads; p.P = s.page_size;
+  p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
+  p.base = (double)rope_base;
+  if ((int64_t)s.batch * s.q_tokens > 0x7fffffff) return DECATTN_ENOTSUP;
+  const cudaError_t e = launch_append(p, s.head_dim, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DECATTN_OK : DECATTN_ECUDA;
+}

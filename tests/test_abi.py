@@ -124,3 +124,28 @@ def test_plan_rejects_bad_args(lib):
     assert lib.dec_attn_plan(FAKE, 2, 2, 60, 1000, 8, FAKE, 1 << 20, C.byref(h), None) == da.ENOTSUP
     need = lib.dec_attn_plan_bytes(2, 2, 64, 1000, 8)
     assert lib.dec_attn_plan(FAKE, 2, 2, 64, 1000, 8, FAKE, need - 1, C.byref(h), None) == da.ESMALL
+
+
+def _append(lib, s, base=10000.0, **ptrs):
+    a = dict(qn=FAKE, kn=FAKE, vn=FAKE, tab=FAKE, lens=FAKE, qo=FAKE, kp=FAKE, vp=FAKE, st=None)
+    a.update(ptrs)
+    return lib.dec_attn_append_rope(C.byref(s), a["qn"], a["kn"], a["vn"], a["tab"], a["lens"], base, a["qo"],
+                                    a["kp"], a["vp"], a["st"], None)
+
+
+def test_append_rope_rejects_bad_args(lib):
+    # every case fails a host check before a launch: the pointers are never dereferenced
+    s = _shape()
+    assert lib.dec_attn_append_rope(None, FAKE, FAKE, FAKE, FAKE, FAKE, 10000.0, FAKE, FAKE, FAKE, None,
+                                    None) == da.EINVAL
+    assert _append(lib, _shape(kv_dtype=da.KV_FP8E4M3)) == da.ENOTSUP  # FP8 pages: scale covers the page
+    assert _append(lib, _shape(head_dim=96)) == da.ENOTSUP
+    assert _append(lib, s, base=0.0) == da.EINVAL
+    assert _append(lib, s, base=float("inf")) == da.EINVAL
+    assert _append(lib, _shape(n_q_heads=6, n_kv_heads=4)) == da.EINVAL
+    for name in ("qn", "kn", "vn", "tab", "lens", "qo", "kp", "vp"):
+        assert _append(lib, s, **{name: None}) == da.EINVAL
+    assert _append(lib, s, qo=FAKE + 2) == da.EALIGN       # d = 128: 4-byte lane accesses
+    assert _append(lib, s, kp=FAKE + 2) == da.EALIGN
+    assert _append(lib, _shape(batch=0), qn=None, kn=None, vn=None, tab=None, lens=None, qo=None, kp=None,
+                   vp=None) == da.OK

@@ -35,6 +35,7 @@ import numpy as np
 
 _CHUNK = 1 << 22  # values per independent random chunk
 _STREAM_LENS, _STREAM_PERM, _STREAM_Q, _STREAM_K, _STREAM_V, _STREAM_PEAKY = range(6)
+_STREAM_NEW_Q, _STREAM_NEW_K, _STREAM_NEW_V = range(6, 9)
 
 E4M3_MAX = 448.0
 
@@ -275,3 +276,15 @@ def make_config(name: str, **overrides) -> Problem:
     kw = dict(CONFIGS[name])
     kw.update(overrides)
     return make_problem(name=name, seq_lens=config_seq_lens(name), **kw)
+
+
+def make_step_inputs(pr: Problem, seed: int | None = None):
+    """The new rows of one decode step before the fused pre-processing: q_new bf16 bits
+    [B][T][Hq][d], k_new and v_new bf16 bits [B][T][Hkv][d], all ~N(0,1) rounded to bf16.
+    Seeded by (seed or the problem's seed) on streams of their own; no method arithmetic."""
+    s = pr.meta["seed"] if seed is None else seed
+    B, T, hq, hkv, d = pr.batch, pr.q_tokens, pr.n_q_heads, pr.n_kv_heads, pr.head_dim
+    q = _fill_normal_bf16(s, _STREAM_NEW_Q, B * T * hq * d).reshape(B, T, hq, d)
+    k = _fill_normal_bf16(s, _STREAM_NEW_K, B * T * hkv * d).reshape(B, T, hkv, d)
+    v = _fill_normal_bf16(s, _STREAM_NEW_V, B * T * hkv * d).reshape(B, T, hkv, d)
+    return q, k, v
