@@ -70,6 +70,9 @@ def parse():
     ap.add_argument("--profile", action="store_true",
                     help="only warm-up + timed steps (for ncu launch lists): no baseline, e2e, graph or clocks")
     ap.add_argument("--json-out", default="", help="also append the JSON line to this file")
+    ap.add_argument("--append", action="store_true",
+                    help="each step starts with the fused pre-processing kernel (rotary embedding of the "
+                         "step's new q / k rows and their KV append), and the decode reads the rotated q")
     return ap.parse_args()
 
 
@@ -294,18 +297,38 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
         torch.sum(flush, dim=0, out=flush_sink)
     pbuf = pl.buf
     kw = dict(kv_scales=sc, sm_scale=pr.sm_scale, workspace=ws, out=out, lse=lse)
+    q_dec = q
+    if args.append:
+        # the step's new rows; every step rewrites the same slots with the same values
+        if pr.kv_dtype != "bf16":
+            raise SystemExit("--append needs a bf16 KV cache")
+        qn_h, kn_h, vn_h = W.make_step_inputs(pr)
+        q_new, k_new, v_new = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+                               for a in (qn_h, kn_h, vn_h))
+        q_dec = torch.empty_like(q_new)
+    n_kernels = 4 if args.append else 3
 
     def enqueue_step(evs):
-        """plan + split + combine; evs: 2 events (step boundaries) or 4 (also between kernels,
-        which stops the kernels' programmatic overlap -- used for the per-kernel breakdown)."""
-        evs[0].record(stream)
+        """[append +] plan + split + combine; evs: 2 events (step boundaries) or one per kernel
+        boundary (which stops the kernels' programmatic overlap -- used for the per-kernel
+        breakdown)."""
+        brk = len(evs) > 2
+        i = 0
+        evs[i].record(stream)
+        if args.append:
+            da.append_rope(q_new, k_new, v_new, tab, lens, k, v, q_out=q_dec)
+            if brk:
+                i += 1
+                evs[i].record(stream)
         da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=pbuf)
-        if len(evs) == 4:
-            evs[1].record(stream)
-        da.run(q, k, v, tab, lens, pl, stage="split", **kw)
-        if len(evs) == 4:
-            evs[2].record(stream)
-        da.run(q, k, v, tab, lens, pl, stage="combine", **kw)
+        if brk:
+            i += 1
+            evs[i].record(stream)
+        da.run(q_dec, k, v, tab, lens, pl, stage="split", **kw)
+        if brk:
+            i += 1
+            evs[i].record(stream)
+        da.run(q_dec, k, v, tab, lens, pl, stage="combine", **kw)
         evs[-1].record(stream)
 
     def one_step(evs):
@@ -332,7 +355,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
         sampler.__enter__()
     t_window = time.perf_counter()
     for _ in range(args.warmup):
-        one_step(new_events(4))
+        one_step(new_events(n_kernels + 1))
     st = da.read_status(pl, ws)
     if st != da.OK:
         raise RuntimeError(f"device status after warm-up: {da.status_string(st)}")
@@ -347,23 +370,25 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
     step_us = [evs[i][0].elapsed_time(evs[i][1]) * 1e3 for i in range(args.steps)]
 
     # ---- per-kernel breakdown: the same steps with events between the kernels
-    bevs = [new_events(4) for _ in range(args.steps)]
+    bevs = [new_events(n_kernels + 1) for _ in range(args.steps)]
     barrier()
     for i in range(args.steps):
         one_step(bevs[i])
     barrier()
-    plan_us = [bevs[i][0].elapsed_time(bevs[i][1]) * 1e3 for i in range(args.steps)]
-    split_us = [bevs[i][1].elapsed_time(bevs[i][2]) * 1e3 for i in range(args.steps)]
-    comb_us = [bevs[i][2].elapsed_time(bevs[i][3]) * 1e3 for i in range(args.steps)]
+    o = 1 if args.append else 0
+    app_us = [bevs[i][0].elapsed_time(bevs[i][1]) * 1e3 for i in range(args.steps)] if args.append else [0.0]
+    plan_us = [bevs[i][o].elapsed_time(bevs[i][o + 1]) * 1e3 for i in range(args.steps)]
+    split_us = [bevs[i][o + 1].elapsed_time(bevs[i][o + 2]) * 1e3 for i in range(args.steps)]
+    comb_us = [bevs[i][o + 2].elapsed_time(bevs[i][o + 3]) * 1e3 for i in range(args.steps)]
     st = da.read_status(pl, ws)
     if st != da.OK:
         raise RuntimeError(f"device status after timing: {da.status_string(st)}")
-    local = [mean(step_us), mean(plan_us), mean(split_us), mean(comb_us)]
+    local = [mean(step_us), mean(plan_us), mean(split_us), mean(comb_us), mean(app_us)]
     if dist is not None:
         t = torch.tensor(local, dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         local = t.tolist()
-    step_m, plan_m, split_m, comb_m = local
+    step_m, plan_m, split_m, comb_m, app_m = local
 
     # CUDA-graph replay of the same step (context figure)
     graph_us = None
@@ -373,8 +398,10 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
         gs.wait_stream(stream)
         with torch.cuda.stream(gs):
             with torch.cuda.graph(g, stream=gs):
+                if args.append:
+                    da.append_rope(q_new, k_new, v_new, tab, lens, k, v, q_out=q_dec, stream=gs)
                 da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=pbuf, stream=gs)
-                da.run(q, k, v, tab, lens, pl, stream=gs, **kw)
+                da.run(q_dec, k, v, tab, lens, pl, stream=gs, **kw)
         stream.wait_stream(gs)
         gt = []
         for i in range(args.warmup + args.steps):
@@ -399,12 +426,14 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
     # end to end through the C ABI: inputs of the step from pinned host memory, result back
     e2e = None
     if not args.no_e2e and not args.profile:
-        hq = torch.from_numpy(pr.q.view(np.int16)).view(torch.bfloat16).pin_memory()
+        # the step's inputs: q (or, with --append, the new q / k / v rows), page table, seq_lens
+        dq = [q_new, k_new, v_new] if args.append else [q]
+        hq = [torch.empty(t.shape, dtype=t.dtype).copy_(t.cpu()).pin_memory() for t in dq]
         htab = torch.from_numpy(pr.page_table).pin_memory()
         hlens = torch.from_numpy(pr.seq_lens).pin_memory()
         hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
         hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-        h2d = hq.numel() * 2 + htab.numel() * 4 + hlens.numel() * 4
+        h2d = sum(t.numel() * 2 for t in hq) + htab.numel() * 4 + hlens.numel() * 4
         d2h = hout.numel() * 4 + hlse.numel() * 4
         et = []
         for i in range(args.warmup + args.steps):
@@ -412,11 +441,14 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
             flush_l2()
             torch.cuda._sleep(SLEEP_CYCLES)
             a.record(stream)
-            q.copy_(hq, non_blocking=True)
+            for dt, ht in zip(dq, hq):
+                dt.copy_(ht, non_blocking=True)
             tab.copy_(htab, non_blocking=True)
             lens.copy_(hlens, non_blocking=True)
+            if args.append:
+                da.append_rope(q_new, k_new, v_new, tab, lens, k, v, q_out=q_dec)
             da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=pbuf)
-            da.run(q, k, v, tab, lens, pl, **kw)
+            da.run(q_dec, k, v, tab, lens, pl, **kw)
             hout.copy_(out, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
             b_.record(stream)
@@ -430,7 +462,9 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
             e2e_local = t.item()
         e2e = {"value": round(e2e_local, 3), "unit": "us/step", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h),
-               "note": "per step: q, page table and seq_lens from pinned host memory, plan + split + combine, "
+               "note": ("per step: the new q/k/v rows" if args.append else "per step: q") +
+                       ", page table and seq_lens from pinned host memory, " +
+                       ("append + " if args.append else "") + "plan + split + combine, "
                        "out and lse back to pinned host memory; the KV cache stays resident in HBM"}
 
     if rank != 0:
@@ -460,8 +494,19 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(split_gbs / peak, 4),
                      "traffic": None if traffic is None else int(traffic)},
-        "gpu_launches": 3 * args.steps,  # planner, split and combine kernels per timed step
+        "gpu_launches": n_kernels * args.steps,  # [append,] planner, split, combine kernels per timed step
     }
+    if args.append:
+        # the fused pre-processing kernel: bytes it must move once (new q/k/v rows in, rotated q
+        # and the k/v rows out, seq_lens and one page-table entry per new token)
+        rows = pr.batch * pr.q_tokens
+        app_bytes = rows * (2 * pr.n_q_heads + 4 * pr.n_kv_heads) * pr.head_dim * 2 + pr.batch * 4 + rows * 4
+        line["config"]["fused_append_rope"] = True
+        line["append_us"] = round(app_m, 3)
+        line["append_roofline"] = {"bound": "latency", "bytes": int(app_bytes),
+                                   "achieved_gbs": round(app_bytes / (app_m * 1e-6) / 1e9, 1),
+                                   "note": "one block per new token; a few hundred KB per launch, so the "
+                                           "launch and one dependent memory round trip set its time"}
     if sampler:
         line["clocks"] = sampler.summary()
     if e2e is not None:

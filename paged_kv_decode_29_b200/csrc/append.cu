@@ -10,17 +10,21 @@
 //  * rotated q goes to q_out; rotated k and unchanged v go to page page_table[b][pos / P], slot
 //    pos % P, of their KV head; a token with pos < 0 has no slot (its q is left unrotated).
 //
-// One block per new token: the block computes (cos, sin) of its position once (the angle in
-// fp64: pos * theta in fp32 would be off by up to ~0.016 rad at pos = 131072), then its warps
-// take the token's Hq + 2 Hkv rows; lane l holds elements [E l, E l + E) of both halves, so
-// each rotation pair sits in one lane. Values are rotated in fp32 and rounded to bf16 (RNE).
+// Block (token, g) takes rows 8g .. 8g+7 of the token's Hq + 2 Hkv rows (q heads, then k,
+// then v), one warp per row, so that every row's load is in flight at once. The block first
+// forms (cos, sin) of pos * theta_i in fp64 (theta_i comes from the host in fp64; pos * theta
+// in fp32 would be off by up to ~0.016 rad at pos = 131072). Lane l holds elements
+// [E l, E l + E) of both halves of its row, so each rotation pair sits in one lane; values are
+// rotated in fp32 and rounded to bf16 (RNE).
 #include <cmath>
 
 #include "common.cuh"
 
 namespace decattn {
 
-constexpr int kAppendThreads = 128;
+constexpr int kAppendWarps = 8;  // rows per block
+constexpr int kAppendThreads = 32 * kAppendWarps;
+constexpr int kAppendMaxHalf = 64;  // head_dim <= 128
 
 struct AppendParams {
   const uint16_t* q_new;   // bf16 [B][T][Hq][D]
@@ -33,7 +37,8 @@ struct AppendParams {
   uint16_t* v_pages;
   int32_t* status;         // optional device word: DECATTN_EDEVICE for a bad page id
   int B, T, Hq, Hkv, P, num_pages, mpps;
-  double base;
+  int groups;                     // row groups of kAppendWarps rows per token
+  double theta[kAppendMaxHalf];   // base^(-2i/d), i < d/2
 };
 
 template <int E>
@@ -51,14 +56,26 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
   __shared__ float2 cs[HALF];  // (cos, sin) of pos * theta_i
   // the inputs are written by the previous kernel of the stream
   griddep_wait();
-  const int bt = blockIdx.x;
+  const int bt = blockIdx.x / p.groups, grp = blockIdx.x - bt * p.groups;
   const int b = bt / p.T, t = bt - b * p.T;
   const int64_t pos = (int64_t)p.seq_lens[b] - p.T + t;
   const double rpos = pos < 0 ? 0.0 : (double)pos;
+  // this warp's row (q heads, then k, then v): its loads go out before the shared work below
+  const int lane = threadIdx.x & 31;
+  const int r = grp * kAppendWarps + (threadIdx.x >> 5);
+  const bool has_row = r < p.Hq + 2 * p.Hkv;
+  const bool is_q = r < p.Hq, is_k = !is_q && r < p.Hq + p.Hkv;
+  const int h = is_q ? 0 : is_k ? r - p.Hq : r - p.Hq - p.Hkv;
+  const uint16_t* src = is_q ? p.q_new + ((int64_t)bt * p.Hq + r) * D
+                             : (is_k ? p.k_new : p.v_new) + ((int64_t)bt * p.Hkv + h) * D;
+  V lo = 0, hi = 0;
+  if (has_row) {
+    lo = reinterpret_cast<const V*>(src)[lane];
+    hi = reinterpret_cast<const V*>(src + HALF)[lane];
+  }
   for (int i = threadIdx.x; i < HALF; i += kAppendThreads) {
-    const double theta = pow(p.base, -2.0 * i / D);
     double s, c;
-    sincos(rpos * theta, &s, &c);
+    sincos(rpos * p.theta[i], &s, &c);
     cs[i] = make_float2((float)c, (float)s);
   }
   // the page slot of this token (none for pos < 0, or for a bad page id, which is reported)
@@ -69,36 +86,26 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
     if (pg < p.mpps) pid = p.page_table[(int64_t)b * p.mpps + pg];
     if (pid >= 0 && pid < p.num_pages) {
       slot_row = (int64_t)pid * p.Hkv * p.P + pos % p.P;
-    } else if (threadIdx.x == 0) {
+    } else if (threadIdx.x == 0 && grp == 0) {
       set_status(p.status, DECATTN_EDEVICE);
     }
   }
   __syncthreads();
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rows = p.Hq + 2 * p.Hkv;
-  for (int r = warp; r < rows; r += kAppendThreads / 32) {
-    const uint16_t* src;
-    uint16_t* dst;
-    bool rotate = true;
-    if (r < p.Hq) {
-      src = p.q_new + ((int64_t)bt * p.Hq + r) * D;
-      dst = p.q_out + ((int64_t)bt * p.Hq + r) * D;
-    } else {
-      const bool is_k = r < p.Hq + p.Hkv;
-      const int h = is_k ? r - p.Hq : r - p.Hq - p.Hkv;
-      if (slot_row < 0) continue;
-      src = (is_k ? p.k_new : p.v_new) + ((int64_t)bt * p.Hkv + h) * D;
-      dst = (is_k ? p.k_pages : p.v_pages) + (slot_row + (int64_t)h * p.P) * D;
-      rotate = is_k;
-    }
-    const V lo = reinterpret_cast<const V*>(src)[lane];
-    const V hi = reinterpret_cast<const V*>(src + HALF)[lane];
-    if (!rotate) {
-      reinterpret_cast<V*>(dst)[lane] = lo;
-      reinterpret_cast<V*>(dst + HALF)[lane] = hi;
-      continue;
-    }
+  if (!has_row) return;
+  uint16_t* dst;
+  if (is_q) {
+    dst = p.q_out + ((int64_t)bt * p.Hq + r) * D;
+  } else {
+    if (slot_row < 0) return;
+    dst = (is_k ? p.k_pages : p.v_pages) + (slot_row + (int64_t)h * p.P) * D;
+  }
+  if (!is_q && !is_k) {
+    reinterpret_cast<V*>(dst)[lane] = lo;
+    reinterpret_cast<V*>(dst + HALF)[lane] = hi;
+    return;
+  }
+  {
     float x1[E], x2[E];
     #pragma unroll
     for (int e = 0; e < E; ++e) {
@@ -120,7 +127,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
 }
 
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t st) {
-  const int64_t blocks = (int64_t)p.B * p.T;
+  const int64_t blocks = (int64_t)p.B * p.T * p.groups;
   if (blocks <= 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)blocks);
@@ -171,8 +178,9 @@ extern "C" int dec_attn_append_rope(const dec_attn_shape* shape, const void* q_n
   p.status = status;
   p.B = s.batch; p.T = s.q_tokens; p.Hq = s.n_q_heads; p.Hkv = s.n_kv_heads; p.P = s.page_size;
   p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
-  p.base = (double)rope_base;
-  if ((int64_t)s.batch * s.q_tokens > 0x7fffffff) return DECATTN_ENOTSUP;
+  p.groups = (s.n_q_heads + 2 * s.n_kv_heads + kAppendWarps - 1) / kAppendWarps;
+  for (int i = 0; i < s.head_dim / 2; ++i) p.theta[i] = std::pow((double)rope_base, -2.0 * i / s.head_dim);
+  if ((int64_t)s.batch * s.q_tokens * p.groups > 0x7fffffff) return DECATTN_ENOTSUP;
   const cudaError_t e = launch_append(p, s.head_dim, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DECATTN_OK : DECATTN_ECUDA;
 }
