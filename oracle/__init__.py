@@ -54,6 +54,7 @@ class _Problem(C.Structure):
         ("sm_scale", C.c_double),
         ("q", C.c_void_p), ("k_pages", C.c_void_p), ("v_pages", C.c_void_p), ("kv_scales", C.c_void_p),
         ("page_table", C.c_void_p), ("seq_lens", C.c_void_p),
+        ("tile_mask", C.c_void_p), ("mask_words", C.c_int32), ("tile_len", C.c_int32),
     ]
 
 
@@ -71,6 +72,9 @@ def _load():
             lib.oracle_plan.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int64,
                                         C.c_void_p, C.c_void_p, C.c_void_p]
             lib.oracle_plan.restype = C.c_int64
+            lib.oracle_plan_masked.argtypes = [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_int, C.c_int,
+                                               C.c_int64, C.c_void_p, C.c_void_p, C.c_void_p]
+            lib.oracle_plan_masked.restype = C.c_int64
             lib.oracle_e4m3_value.argtypes = [C.c_uint8]
             lib.oracle_e4m3_value.restype = C.c_double
             lib.oracle_max_threads.restype = C.c_int
@@ -98,6 +102,7 @@ class _Bound:
             s=None if pr.kv_scales is None else np.ascontiguousarray(pr.kv_scales, dtype=np.float32),
             t=np.ascontiguousarray(pr.page_table, dtype=np.int32),
             L=np.ascontiguousarray(pr.seq_lens, dtype=np.int32),
+            m=None if getattr(pr, "tile_mask", None) is None else np.ascontiguousarray(pr.tile_mask, dtype=np.uint32),
         )
         a = self.arrs
         fp8 = pr.kv_dtype == "fp8e4m3"
@@ -105,7 +110,8 @@ class _Bound:
             raise ValueError("FP8 KV needs kv_scales")
         self.s = _Problem(pr.batch, pr.q_tokens, pr.n_q_heads, pr.n_kv_heads, pr.head_dim, pr.page_size,
                           int(a["k"].shape[0]), int(a["t"].shape[1]), int(fp8), 0, float(pr.sm_scale),
-                          _ptr(a["q"]), _ptr(a["k"]), _ptr(a["v"]), _ptr(a["s"]), _ptr(a["t"]), _ptr(a["L"]))
+                          _ptr(a["q"]), _ptr(a["k"]), _ptr(a["v"]), _ptr(a["s"]), _ptr(a["t"]), _ptr(a["L"]),
+                          _ptr(a["m"]), 0 if a["m"] is None else int(a["m"].shape[-1]), int(pr.tile_len))
 
 
 def max_threads() -> int:
@@ -155,9 +161,10 @@ def attend(pr, b, t, qh, j_lo=0, j_hi=None, weights=False):
 UNIT_FIELDS = ("b", "h", "tok_begin", "tok_end", "seq_len", "slot", "tile", "zero")
 
 
-def plan(seq_lens, n_kv_heads: int, tile_len: int, n_bins: int, capacity: int | None = None):
+def plan(seq_lens, n_kv_heads: int, tile_len: int, n_bins: int, capacity: int | None = None, tile_mask=None):
     """Greedy bin-packing of uniform KV tiles. Returns dict(n_units, bin_off, units[U][8], pair_off)
-    or None when the tile count exceeds ``capacity``."""
+    or None when the tile count exceeds ``capacity``. ``tile_mask`` (uint32 [B][Hkv][words]): only
+    the tiles whose bit is set enter the work list (block-sparse decode)."""
     lib = _load()
     L = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
     B = L.shape[0]
@@ -166,8 +173,14 @@ def plan(seq_lens, n_kv_heads: int, tile_len: int, n_bins: int, capacity: int | 
     bin_off = np.zeros(n_bins + 1, dtype=np.int32)
     units = np.zeros((max(U_max, 1), 8), dtype=np.int32)
     pair_off = np.zeros(B * n_kv_heads + 1, dtype=np.int32)
-    U = lib.oracle_plan(L.ctypes.data, B, int(n_kv_heads), int(tile_len), int(n_bins), cap,
-                        bin_off.ctypes.data, units.ctypes.data, pair_off.ctypes.data)
+    if tile_mask is None:
+        U = lib.oracle_plan(L.ctypes.data, B, int(n_kv_heads), int(tile_len), int(n_bins), cap,
+                            bin_off.ctypes.data, units.ctypes.data, pair_off.ctypes.data)
+    else:
+        m = np.ascontiguousarray(tile_mask, dtype=np.uint32)
+        assert m.shape[:2] == (B, n_kv_heads)
+        U = lib.oracle_plan_masked(L.ctypes.data, m.ctypes.data, int(m.shape[2]), B, int(n_kv_heads), int(tile_len),
+                                   int(n_bins), cap, bin_off.ctypes.data, units.ctypes.data, pair_off.ctypes.data)
     if U < 0:
         return None
     return dict(n_units=int(U), bin_off=bin_off, units=units[:U], pair_off=pair_off)

@@ -36,7 +36,22 @@ typedef struct {
     const float *kv_scales;      /* [2][num_pages][Hkv]: K scales, then V scales (FP8 only) */
     const int32_t *page_table;   /* [B][max_pages_per_seq] */
     const int32_t *seq_lens;     /* [B] */
+    /* block-sparse decode (NULL: every key may be seen): bit i % 32 of word i / 32 of row
+     * (b * Hkv + h) keeps tile i = keys [i * tile_len, (i + 1) * tile_len) of (b, h) */
+    const uint32_t *tile_mask;
+    int32_t mask_words, tile_len;
 } oracle_problem;
+
+/* Whether key j of (b, h) lies in a kept tile ("HPC-Ops ...", "How the kernels are organized
+ * around specific workload shapes": sparse attention skips the KV tiles its precomputed block
+ * mask masks out). */
+static int key_kept(const oracle_problem *pr, int b, int h, int64_t j)
+{
+    if (!pr->tile_mask) return 1;
+    int64_t i = j / pr->tile_len;
+    uint32_t w = pr->tile_mask[((int64_t)b * pr->n_kv_heads + h) * pr->mask_words + i / 32];
+    return (int)((w >> (i % 32)) & 1u);
+}
 
 /* bf16 -> double: the bf16 bit pattern is the top half of an IEEE binary32. */
 static double bf16_value(uint16_t h)
@@ -89,18 +104,23 @@ int64_t oracle_attend(const oracle_problem *pr, int b, int t, int qh, int64_t j_
     int64_t last = Lb - T + t;                              /* last visible key */
     int64_t lo = j_lo < 0 ? 0 : j_lo;
     int64_t hi = j_hi < last + 1 ? j_hi : last + 1;
-    int64_t n = hi > lo ? hi - lo : 0;
+    int64_t n = 0;
     const uint16_t *qrow = pr->q + (((int64_t)b * T + t) * pr->n_q_heads + qh) * d;
     double *s;
+    int64_t *key;
     int c;
     for (c = 0; c < d; ++c) out_row[c] = 0.0;
-    if (n == 0) { *lse = -INFINITY; return 0; }
+    if (hi <= lo) { *lse = -INFINITY; return 0; }
+    key = (int64_t *)malloc((size_t)(hi - lo) * sizeof(int64_t));  /* the visible keys, in order */
+    for (int64_t j = lo; j < hi; ++j)
+        if (key_kept(pr, b, h, j)) key[n++] = j;
+    if (n == 0) { *lse = -INFINITY; free(key); return 0; }
     s = (double *)malloc((size_t)n * sizeof(double));
     /* scores s_j = sm_scale * <q, k_j> */
-    for (int64_t j = lo; j < hi; ++j) {
+    for (int64_t i = 0; i < n; ++i) {
         double acc = 0.0;
-        for (c = 0; c < d; ++c) acc += bf16_value(qrow[c]) * kv_elem(pr, 0, b, h, j, c);
-        s[j - lo] = pr->sm_scale * acc;
+        for (c = 0; c < d; ++c) acc += bf16_value(qrow[c]) * kv_elem(pr, 0, b, h, key[i], c);
+        s[i] = pr->sm_scale * acc;
     }
     /* explicit full softmax */
     double m = s[0];
@@ -110,10 +130,11 @@ int64_t oracle_attend(const oracle_problem *pr, int b, int t, int qh, int64_t j_
     for (int64_t i = 0; i < n; ++i) {
         double w = exp(s[i] - m) / Z;
         if (weights) weights[i] = w;
-        for (c = 0; c < d; ++c) out_row[c] += w * kv_elem(pr, 1, b, h, lo + i, c);
+        for (c = 0; c < d; ++c) out_row[c] += w * kv_elem(pr, 1, b, h, key[i], c);
     }
     *lse = m + log(Z);
     free(s);
+    free(key);
     return n;
 }
 
@@ -184,13 +205,32 @@ static int cmp_tile(const void *a, const void *b)
     return x->idx < y->idx ? -1 : (x->idx > y->idx);             /* stable */
 }
 
+int64_t oracle_plan_masked(const int32_t *seq_lens, const uint32_t *mask, int mask_words, int B, int Hkv,
+                           int tl, int n_bins, int64_t capacity, int32_t *bin_off, int32_t *units,
+                           int32_t *pair_off);
+
 int64_t oracle_plan(const int32_t *seq_lens, int B, int Hkv, int tl, int n_bins, int64_t capacity,
                     int32_t *bin_off, int32_t *units, int32_t *pair_off)
 {
+    return oracle_plan_masked(seq_lens, NULL, 0, B, Hkv, tl, n_bins, capacity, bin_off, units, pair_off);
+}
+
+/* Block-sparse variant: only the tiles whose mask bit is set (row b * Hkv + h of mask, words
+ * of 32 tiles) enter the work list; a pair's kept tiles are numbered j = 0, 1, ... in tile
+ * order, its partial slots are pair_off[pair] + j (a pair with one kept tile writes the final
+ * output: slot -1), and unit field 6 is the tile's index i among all tiles of the pair. */
+int64_t oracle_plan_masked(const int32_t *seq_lens, const uint32_t *mask, int mask_words, int B, int Hkv,
+                           int tl, int n_bins, int64_t capacity, int32_t *bin_off, int32_t *units,
+                           int32_t *pair_off)
+{
     int64_t U = 0, p, k;
+#define KEPT(b, h, i) (!mask || ((mask[((int64_t)(b) * Hkv + (h)) * mask_words + (i) / 32] >> ((i) % 32)) & 1u))
     for (int b = 0; b < B; ++b) {
         int64_t nb = ((int64_t)seq_lens[b] + tl - 1) / tl;
-        for (int h = 0; h < Hkv; ++h) { pair_off[(int64_t)b * Hkv + h] = (int32_t)U; U += nb; }
+        for (int h = 0; h < Hkv; ++h) {
+            pair_off[(int64_t)b * Hkv + h] = (int32_t)U;
+            for (int64_t i = 0; i < nb; ++i) U += KEPT(b, h, i) ? 1 : 0;
+        }
     }
     pair_off[(int64_t)B * Hkv] = (int32_t)U;
     if (U > capacity) return -1;
@@ -200,16 +240,21 @@ int64_t oracle_plan(const int32_t *seq_lens, int B, int Hkv, int tl, int n_bins,
     int64_t u = 0;
     for (int b = 0; b < B; ++b) {
         int64_t Lb = seq_lens[b], nb = (Lb + tl - 1) / tl;
-        for (int h = 0; h < Hkv; ++h)
-            for (int64_t i = 0; i < nb; ++i, ++u) {
+        for (int h = 0; h < Hkv; ++h) {
+            int64_t p0 = pair_off[(int64_t)b * Hkv + h], m = pair_off[(int64_t)b * Hkv + h + 1] - p0, j = 0;
+            for (int64_t i = 0; i < nb; ++i) {
+                if (!KEPT(b, h, i)) continue;
                 int64_t beg = i * tl, end = (i + 1) * tl < Lb ? (i + 1) * tl : Lb;
                 int32_t *r = tb + 8 * u;
                 r[0] = b; r[1] = h; r[2] = (int32_t)beg; r[3] = (int32_t)end; r[4] = (int32_t)Lb;
-                r[5] = nb == 1 ? -1 : (int32_t)(pair_off[(int64_t)b * Hkv + h] + i);
+                r[5] = m == 1 ? -1 : (int32_t)(p0 + j);
                 r[6] = (int32_t)i; r[7] = 0;
                 key[u].cost = end - beg; key[u].idx = u;
+                ++u; ++j;
             }
+        }
     }
+#undef KEPT
     qsort(key, (size_t)U, sizeof(tile_key), cmp_tile);
 
     int64_t *load = (int64_t *)calloc((size_t)n_bins, sizeof(int64_t));

@@ -35,7 +35,7 @@ import numpy as np
 
 _CHUNK = 1 << 22  # values per independent random chunk
 _STREAM_LENS, _STREAM_PERM, _STREAM_Q, _STREAM_K, _STREAM_V, _STREAM_PEAKY = range(6)
-_STREAM_NEW_Q, _STREAM_NEW_K, _STREAM_NEW_V = range(6, 9)
+_STREAM_NEW_Q, _STREAM_NEW_K, _STREAM_NEW_V, _STREAM_MASK = range(6, 10)
 
 E4M3_MAX = 448.0
 
@@ -104,6 +104,7 @@ class Problem:
     v_pages: np.ndarray
     kv_scales: np.ndarray | None = None  # float32 [2][num_pages][Hkv] (K then V), FP8 only
     sm_scale: float = 0.0
+    tile_mask: np.ndarray | None = None  # uint32 [B][Hkv][words]: block-sparse decode, bit i keeps tile i
     meta: dict = field(default_factory=dict)
 
     @property
@@ -288,3 +289,24 @@ def make_step_inputs(pr: Problem, seed: int | None = None):
     k = _fill_normal_bf16(s, _STREAM_NEW_K, B * T * hkv * d).reshape(B, T, hkv, d)
     v = _fill_normal_bf16(s, _STREAM_NEW_V, B * T * hkv * d).reshape(B, T, hkv, d)
     return q, k, v
+
+
+def make_tile_mask(pr: Problem, density: float, seed: int | None = None, keep_last: bool = True) -> np.ndarray:
+    """A block-sparse decode mask: uint32 [B][Hkv][words] with bit i of (b, h) set (tile i of the
+    pair's tile_len-token tiles kept) independently with probability ``density``; with
+    ``keep_last`` the tile holding each request's newest token is always kept (a local window).
+    Bits past a request's last tile are 0. Seeded; no method arithmetic."""
+    s = pr.meta["seed"] if seed is None else seed
+    L = pr.seq_lens.astype(np.int64)
+    nb = (L + pr.tile_len - 1) // pr.tile_len
+    n_max = int(nb.max()) if pr.batch else 0
+    words = max(1, (n_max + 31) // 32)
+    keep = _gen(s, _STREAM_MASK, 0).random((pr.batch, pr.n_kv_heads, words * 32)) < density
+    idx = np.arange(words * 32)
+    keep &= idx[None, None, :] < nb[:, None, None]
+    if keep_last:
+        for b in range(pr.batch):
+            if nb[b] > 0:
+                keep[b, :, nb[b] - 1] = True
+    bits = (keep.reshape(pr.batch, pr.n_kv_heads, words, 32).astype(np.uint64) << np.arange(32, dtype=np.uint64))
+    return bits.sum(axis=-1).astype(np.uint32)
