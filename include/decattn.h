@@ -80,6 +80,8 @@ typedef struct {
   int32_t tile_len;   /* tokens per uniform KV tile */
   int32_t n_bins;     /* CTAs of the split kernel; one bin of tiles per CTA */
   int64_t max_units;  /* capacity of the tile list */
+  int32_t sparse;     /* 1 for a plan made by dec_attn_plan_sparse */
+  int32_t reserved_;
 } dec_attn_plan_t;
 
 /* Problem shape shared by dec_attn_workspace_bytes and dec_attn_run. */
@@ -125,6 +127,27 @@ DECATTN_API size_t dec_attn_plan_bytes(int batch, int n_kv_heads, int tile_len, 
  * writes nothing and reports the same status. */
 DECATTN_API int dec_attn_plan(const int32_t *seq_lens, int batch, int n_kv_heads, int tile_len, int64_t max_total_kv_tokens,
                   int n_bins, void *plan_buf, size_t plan_bytes, dec_attn_plan_t *plan, void *stream);
+
+/* Block-sparse decode planner ("HPC-Ops ...", "How the kernels are organized around specific
+ * workload shapes": sparse attention takes a precomputed block mask and skips the masked-out KV
+ * tiles). Same greedy rule as dec_attn_plan, over the kept tiles only:
+ *   tile_mask  device uint32 [batch][n_kv_heads][mask_words]: bit i % 32 of word i / 32 of row
+ *              (b, h) keeps tile i = keys [i*tl, min((i+1)*tl, Lb)) of request b, KV head h;
+ *              bits of tiles past a request's last tile are ignored, tiles past the row's
+ *              mask_words words count as masked; 4-byte aligned.
+ * Every query row of (b, h) then attends to the keys of the kept tiles only (with the causal
+ * rule for T > 1); a pair with no kept tile gets out = 0, lse = -inf. A pair's kept tiles are
+ * numbered j = 0, 1, ... in tile order; their partial slots are the prefix over pairs of kept
+ * tiles plus j, and a pair with one kept tile writes the final output. The plan is used with
+ * dec_attn_run / dec_attn_split / dec_attn_combine / dec_attn_plan_export unchanged; its
+ * buffer needs dec_attn_plan_sparse_bytes (4 bytes per tile of capacity more than a dense plan).
+ * Per-tile FP8 scales are the case of per-(page, head) scales equal across a tile's pages.
+ * Other arguments, errors and the launch as dec_attn_plan. */
+DECATTN_API size_t dec_attn_plan_sparse_bytes(int batch, int n_kv_heads, int tile_len, int64_t max_total_kv_tokens,
+                                              int n_bins);
+DECATTN_API int dec_attn_plan_sparse(const int32_t *seq_lens, const uint32_t *tile_mask, int mask_words, int batch,
+                                     int n_kv_heads, int tile_len, int64_t max_total_kv_tokens, int n_bins,
+                                     void *plan_buf, size_t plan_bytes, dec_attn_plan_t *plan, void *stream);
 
 /* Writes the explicit work list of a finished plan (the device plan stores full tiles in
  * closed form): bin_off device int32 [n_bins + 1] (CSR offsets), units device int32

@@ -28,7 +28,8 @@ OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1
 KV_BF16, KV_FP8E4M3 = 0, 1
 API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
-       "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope")
+       "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_plan_sparse_bytes",
+       "dec_attn_plan_sparse")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -40,7 +41,8 @@ class DecAttnError(RuntimeError):
 
 class PlanT(C.Structure):
     _fields_ = [("buf", C.c_void_p), ("buf_bytes", C.c_size_t), ("batch", C.c_int32), ("n_kv_heads", C.c_int32),
-                ("tile_len", C.c_int32), ("n_bins", C.c_int32), ("max_units", C.c_int64)]
+                ("tile_len", C.c_int32), ("n_bins", C.c_int32), ("max_units", C.c_int64),
+                ("sparse", C.c_int32), ("reserved_", C.c_int32)]
 
 
 class ShapeT(C.Structure):
@@ -85,6 +87,10 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_status_string.argtypes = [i32]
         lib.dec_attn_status_string.restype = C.c_char_p
         lib.dec_attn_append_rope.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, C.c_float, vp, vp, vp, vp, vp]
+        lib.dec_attn_plan_sparse_bytes.argtypes = [i32, i32, i32, i64, i32]
+        lib.dec_attn_plan_sparse_bytes.restype = sz
+        lib.dec_attn_plan_sparse.argtypes = [vp, vp, i32, i32, i32, i32, i64, i32, vp, sz, C.POINTER(PlanT), vp]
+        lib.dec_attn_plan_sparse.restype = i32
         lib.dec_attn_append_rope.restype = i32
         _lib = lib
         return lib
@@ -153,6 +159,33 @@ def plan(seq_lens: torch.Tensor, n_kv_heads: int, tile_len: int, max_total_kv_to
                            buf.data_ptr(), buf.numel(), C.byref(h), _stream_handle(stream))
     if rc != OK:
         raise DecAttnError(rc, "dec_attn_plan")
+    return Plan(buf=buf, handle=h)
+
+
+def plan_sparse(seq_lens: torch.Tensor, tile_mask: torch.Tensor, n_kv_heads: int, tile_len: int,
+                max_total_kv_tokens: int | None = None, n_bins: int = 0, buf: torch.Tensor | None = None,
+                stream=None) -> Plan:
+    """Enqueues the block-sparse planner: only the tiles whose bit is set in ``tile_mask`` (int32 or
+    uint32-valued CUDA tensor [B][n_kv_heads][words], bit i of (b, h) keeps tile i) enter the work
+    list. The plan is then used with ``run`` like a dense one."""
+    lib = load_library()
+    assert seq_lens.is_cuda and seq_lens.dtype == torch.int32 and seq_lens.is_contiguous()
+    assert tile_mask.is_cuda and tile_mask.dtype == torch.int32 and tile_mask.is_contiguous()
+    B = int(seq_lens.numel())
+    assert tile_mask.dim() == 3 and tile_mask.shape[0] == B and tile_mask.shape[1] == n_kv_heads
+    if max_total_kv_tokens is None:
+        max_total_kv_tokens = int(seq_lens.sum().item()) if B else 0
+    nbytes = lib.dec_attn_plan_sparse_bytes(B, n_kv_heads, tile_len, int(max_total_kv_tokens), n_bins)
+    if nbytes == 0:
+        raise DecAttnError(ENOTSUP, "dec_attn_plan_sparse_bytes")
+    if buf is None:
+        buf = torch.empty(nbytes, dtype=torch.uint8, device=seq_lens.device)
+    h = PlanT()
+    rc = lib.dec_attn_plan_sparse(_ptr(seq_lens), _ptr(tile_mask), int(tile_mask.shape[2]), B, n_kv_heads, tile_len,
+                                  int(max_total_kv_tokens), n_bins, buf.data_ptr(), buf.numel(), C.byref(h),
+                                  _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_plan_sparse")
     return Plan(buf=buf, handle=h)
 
 

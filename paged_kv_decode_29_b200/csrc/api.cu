@@ -179,7 +179,7 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
     sp.status = reinterpret_cast<int32_t*>(static_cast<char*>(plan->buf) + offsetof(PlanHeader, run_status));
     sp.B = s.batch; sp.T = s.q_tokens; sp.Hq = s.n_q_heads; sp.Hkv = s.n_kv_heads; sp.G = G; sp.GT = GT;
     sp.P = s.page_size; sp.num_pages = s.num_pages; sp.mpps = s.max_pages_per_seq; sp.n_bins = plan->n_bins;
-    sp.tile_len = plan->tile_len; sp.max_units = plan->max_units;
+    sp.tile_len = plan->tile_len; sp.max_units = plan->max_units; sp.sparse = plan->sparse;
     sp.qk_scale_log2 = scale * 1.4426950408889634f;
     if (launch_split(sp, tmK, tmV, s.kv_dtype, D, st) != cudaSuccess) return DECATTN_ECUDA;
   }
@@ -195,6 +195,7 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
     cp.chunk_state = reinterpret_cast<float*>(ws + wl.off_chunk);
     cp.B = s.batch; cp.T = s.q_tokens; cp.Hq = s.n_q_heads; cp.Hkv = s.n_kv_heads; cp.G = G; cp.GT = GT; cp.D = D;
     cp.tl = plan->tile_len;
+    cp.sparse = plan->sparse;
     if (launch_combine(cp, dev, st) != cudaSuccess) return DECATTN_ECUDA;
   }
   return DECATTN_OK;

@@ -9,7 +9,8 @@
 //
 // Work decomposition (computed by the planner): each query row of request b is cut into
 // cb_b chunks of up to kCombineChunk tiles; the items (b, row, chunk) are numbered request
-// by request. The kernel is persistent: every warp takes items w, w + #warps, ...
+// by request (block-sparse plans: (request, KV head) pair by pair, since pairs keep their
+// own tiles). The kernel is persistent: every warp takes items w, w + #warps, ...
 //  * a warp loads the lse and the D floats of up to 16 partial rows (8 loads in flight per
 //    lane at a time) and folds them into (max, weight, weighted sum);
 //  * a row made of one chunk is finished right there;
@@ -51,35 +52,38 @@ __device__ __forceinline__ void write_row(float* orow, float* lse_out, int lane,
   if (lane == 0) *lse_out = empty ? -INFINITY : M + logf(W);
 }
 
-template <int D>
+// Items are numbered unit by unit: per request (dense plans: every KV head of a request has the
+// same tiles) or per (request, KV head) pair (block-sparse plans); NU units of RPU query rows.
+template <int D, bool SPARSE>
 __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_kernel(const CombineParams p) {
   constexpr int VEC = D / 32;
   using V = typename CombineVec<D>::T;
-  extern __shared__ int32_t req_sm[];  // [3][B + 1]: chunk prefix, tile prefix S, seq_lens
+  extern __shared__ int32_t req_sm[];  // chunk prefix [NU + 1], tile prefix [NU + 1], seq_lens [B + 1]
   // The plan is complete when this grid starts (the split kernel lets it launch only after its
   // own wait on the planner), so everything but the partials is read before waiting.
   const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
   if (hdr->magic != kPlanMagic || hdr->status != DECATTN_OK) return;  // the split kernel reports it
+  const int NU = SPARSE ? p.B * p.Hkv : p.B;
   const int32_t* cb_sm = plan_arr(p.plan, hdr->off_cb);
   const int32_t* S = plan_arr(p.plan, hdr->off_S);
   const int32_t* Ls = p.seq_lens;
-  if (p.B <= kCombineSmemRequests) {
+  if (NU <= kCombineSmemRequests) {
     int32_t* a = req_sm;
-    int32_t* b = req_sm + (p.B + 1);
-    int32_t* c = req_sm + 2 * (p.B + 1);
-    for (int i = threadIdx.x; i <= p.B; i += kCombineThreads) {
+    int32_t* b = req_sm + (NU + 1);
+    int32_t* c = req_sm + 2 * (NU + 1);
+    for (int i = threadIdx.x; i <= NU; i += kCombineThreads) {
       a[i] = cb_sm[i];
       b[i] = S[i];
-      c[i] = i < p.B ? Ls[i] : 0;
     }
+    for (int i = threadIdx.x; i <= p.B; i += kCombineThreads) c[i] = i < p.B ? Ls[i] : 0;
     __syncthreads();
     cb_sm = a; S = b; Ls = c;
   }
   griddep_wait();  // the split kernel's partials are complete and visible
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // item numbers fit 32 bits (checked on the host), so does every product below
-  const int rows_per_b = p.T * p.Hq;
-  const int total = rows_per_b * cb_sm[p.B];
+  const int rows_per_b = SPARSE ? p.GT : p.T * p.Hq;  // query rows per unit
+  const int total = rows_per_b * cb_sm[NU];
   const int nwarps = gridDim.x * kCombineWarps;
 
   // The warp's items w0, w0 + nwarps, ... are taken kCombineGroup at a time: each is folded; a
@@ -95,31 +99,44 @@ __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_ke
       const int64_t wl = (int64_t)w0 + (int64_t)k * nwarps;
       if (wl >= total) break;
       const int w = (int)wl;
-      int lo = 0, hi = p.B - 1;  // request: last b with rows_per_b * cb[b] <= w
+      int lo = 0, hi = NU - 1;  // unit: last u with rows_per_b * cb[u] <= w
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (rows_per_b * cb_sm[mid] <= w) lo = mid; else hi = mid - 1;
       }
-      const int b = lo;
-      const int ncb = cb_sm[b + 1] - cb_sm[b];
-      const int local = w - rows_per_b * cb_sm[b];
-      const int row_in_b = local / ncb, j = local - row_in_b * ncb;
-      const int t = row_in_b / p.Hq, qh = row_in_b - t * p.Hq;
-      const int64_t row = ((int64_t)b * p.T + t) * p.Hq + qh;
+      const int u = lo;
+      const int ncb = cb_sm[u + 1] - cb_sm[u];
+      const int local = w - rows_per_b * cb_sm[u];
+      const int row_in_u = local / ncb, j = local - row_in_u * ncb;
+      int64_t row, slot_base;
+      int r, nt;  // query row within the tile's partial block; tiles of the row's (request, head)
+      if (SPARSE) {
+        const int b = u / p.Hkv, h = u - b * p.Hkv;
+        const int t = row_in_u / p.G, g = row_in_u - t * p.G;
+        row = ((int64_t)b * p.T + t) * p.Hq + h * p.G + g;
+        r = row_in_u;
+        nt = S[u + 1] - S[u];  // kept tiles of the pair
+        slot_base = S[u];
+      } else {
+        const int b = u;
+        const int t = row_in_u / p.Hq, qh = row_in_u - t * p.Hq;
+        row = ((int64_t)b * p.T + t) * p.Hq + qh;
+        const int h = qh / p.G;
+        r = t * p.G + (qh - h * p.G);
+        const int L = Ls[b];
+        nt = L > 0 ? (L + p.tl - 1) / p.tl : 0;  // == S[b + 1] - S[b]
+        slot_base = (int64_t)p.Hkv * S[b] + (int64_t)h * nt;
+      }
       float* orow = p.out + row * D;
-      const int L = Ls[b];
-      const int nb = L > 0 ? (L + p.tl - 1) / p.tl : 0;
       float acc[VEC];
       #pragma unroll
       for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-      if (nb == 0) {  // no key at all
+      if (nt == 0) {  // no key at all
         write_row<D>(orow, p.lse + row, lane, -INFINITY, 0.f, acc);
         continue;
       }
-      const int h = qh / p.G, r = t * p.G + (qh - h * p.G);
-      const int nbs = S[b + 1] - S[b];  // == nb
-      const int64_t slot0 = (int64_t)p.Hkv * S[b] + (int64_t)h * nbs + (int64_t)j * kCombineChunk;
-      const int n = min(kCombineChunk, nb - j * kCombineChunk);
+      const int64_t slot0 = slot_base + (int64_t)j * kCombineChunk;
+      const int n = min(kCombineChunk, nt - j * kCombineChunk);
       // ---- fold up to kCombineChunk partial rows, in two halves of loads in flight at once
       //      (with every warp loading, the fold runs at DRAM bandwidth; halves keep the
       //      registers below the occupancy limit)
@@ -234,8 +251,11 @@ cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st) 
   if ((int64_t)p.B * p.T * p.Hq <= 0) return cudaSuccess;
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return cudaErrorUnknown;
-  const void* fn = p.D == 128 ? (const void*)combine_kernel<128> : (const void*)combine_kernel<64>;
-  const int smem = p.B <= kCombineSmemRequests ? 12 * (p.B + 1) : 0;
+  if (p.D != 128 && p.D != 64) return cudaErrorInvalidValue;
+  const void* fn = p.sparse ? (p.D == 128 ? (const void*)combine_kernel<128, true> : (const void*)combine_kernel<64, true>)
+                            : (p.D == 128 ? (const void*)combine_kernel<128, false> : (const void*)combine_kernel<64, false>);
+  const int64_t nu = p.sparse ? (int64_t)p.B * p.Hkv : p.B;
+  const int smem = nu <= kCombineSmemRequests ? (int)(4 * (2 * (nu + 1) + p.B + 1)) : 0;
   if (!ensure_smem_attr(fn, smem)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms * kCombineCtasPerSm);
@@ -247,9 +267,8 @@ cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st) 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (p.D == 128) return cudaLaunchKernelEx(&cfg, combine_kernel<128>, p);
-  if (p.D == 64) return cudaLaunchKernelEx(&cfg, combine_kernel<64>, p);
-  return cudaErrorInvalidValue;
+  void* args[] = {const_cast<CombineParams*>(&p)};
+  return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
 }  // namespace decattn

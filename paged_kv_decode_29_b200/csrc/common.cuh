@@ -45,7 +45,9 @@ struct PlanHeader {
   int32_t off_pbin_off; // int32 [n_bins + 1]: CSR offsets of each bin's partial tiles in plist
   int32_t off_plist;    // int32 [batch * n_kv_heads]: partial tiles, bin by bin
   int32_t off_scratch;  // planner scratch
-  int32_t reserved[11];
+  int32_t sparse;       // 1: block-sparse plan (per-pair arrays below, see plan_unit_sparse)
+  int32_t off_kl;       // sparse: int32 [max_units]: tile index of kept tile j of pair p at PS[p] + j
+  int32_t reserved[9];
 };
 static_assert(sizeof(PlanHeader) == 128, "plan header is 128 bytes");
 constexpr int32_t kPlanMagic = 0x32504144;  // "DAP2"
@@ -103,6 +105,50 @@ __device__ __forceinline__ Unit plan_unit(const char* plan, const PlanHeader& h,
   return u;
 }
 
+// Block-sparse plans ("HPC-Ops ...", "How the kernels are organized around specific workload
+// shapes": sparse attention skips the KV tiles a precomputed block mask masks out) index per
+// (request, KV head) pair p = b * Hkv + h instead of per request, because each pair keeps its
+// own tiles; the header offsets then mean:
+//   off_S      PS  [P+1]: prefix over pairs of kept tiles (a pair's partial slots start at PS[p])
+//   off_SF     PF  [P+1]: prefix over pairs of kept full tiles
+//   off_cb     CBP [P+1]: prefix over pairs of combine chunks per query row
+//   off_sorted      [P] : pairs whose partial tile is kept, by cost (desc), then pair index
+//   off_kl     KL  [U]  : tile index of the pair's j-th kept tile at KL[PS[p] + j]
+// Kept full tiles precede a pair's kept partial tile in tile order, so under the greedy rule
+// kept full tile f (in (p, j) order) again sits in bin f mod N at position f div N.
+__device__ __forceinline__ Unit plan_unit_sparse(const char* plan, const PlanHeader& h, const int32_t* seq_lens,
+                                                 int k, int j) {
+  const int32_t* PS = plan_arr(plan, h.off_S);
+  const int32_t* PF = plan_arr(plan, h.off_SF);
+  const int32_t* KL = plan_arr(plan, h.off_kl);
+  const int N = h.n_bins, Hkv = h.n_kv_heads, tl = h.tile_len;
+  const int fc = h.full_q + (k < h.full_r);
+  int pr, kj;
+  if (j < fc) {
+    const int f = k + N * j;
+    int lo = 0, hi = h.batch * Hkv - 1;  // last pair p with PF[p] <= f
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (PF[mid] <= f) lo = mid; else hi = mid - 1;
+    }
+    pr = lo;
+    kj = f - PF[pr];
+  } else {
+    const int s = plan_arr(plan, h.off_plist)[plan_arr(plan, h.off_pbin_off)[k] + (j - fc)];
+    pr = plan_arr(plan, h.off_sorted)[s];
+    kj = PS[pr + 1] - PS[pr] - 1;  // the partial tile is the pair's last kept tile
+  }
+  const int b = pr / Hkv;
+  const int m = PS[pr + 1] - PS[pr];
+  const int i = KL[PS[pr] + kj];
+  const int L = seq_lens[b];
+  Unit u;
+  u.b = b; u.h = pr - b * Hkv; u.tok_begin = i * tl; u.tok_end = min((i + 1) * tl, L); u.seq_len = L;
+  u.slot = m == 1 ? -1 : PS[pr] + kj;
+  u.tile = i; u.zero = 0;
+  return u;
+}
+
 // Workspace: a status word, then partial outputs and their LSEs.
 struct WorkspaceHeader {
   int32_t status;
@@ -125,6 +171,7 @@ struct SplitParams {
   int32_t* status;          // run status word (plan header)
   int B, T, Hq, Hkv, G, GT, P, num_pages, mpps, n_bins;
   int tile_len;             // the plan's tile length
+  int sparse;               // the plan is block-sparse (its tiles come from the plan only)
   int64_t max_units;        // the plan's capacity (partial slots of the workspace)
   float qk_scale_log2;      // sm_scale * log2(e)
 };
@@ -149,6 +196,7 @@ struct CombineParams {
   int32_t* row_cnt;         // [B*T*Hq] chunks of the row folded so far (zeroed by the split kernel)
   float* chunk_state;       // [items][D + 4]: max, weight, -, -, then the weighted sum
   int B, T, Hq, Hkv, G, GT, D, tl;
+  int sparse;               // block-sparse plan: chunks are counted per (request, KV head) pair
 };
 
 __host__ __device__ inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }

@@ -333,6 +333,230 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
   }
 }
 
+// ------------------------------------------------------------------ block-sparse planner
+// "HPC-Ops ...", "How the kernels are organized around specific workload shapes": sparse
+// attention takes a precomputed block mask and skips the masked-out KV tiles. The same greedy
+// rule runs over the kept tiles only; each (request, KV head) pair p = b * Hkv + h keeps its
+// own tiles (bit i % 32 of word i / 32 of mask row p keeps tile i; tiles past the row's
+// mask_words words count as masked), so the plan's per-request arrays become per-pair ones
+// (see plan_unit_sparse() in common.cuh).
+__host__ __device__ inline int64_t plan_sparse_scratch_bytes(int B, int Hkv) {
+  return 4 * align_up(4 * ((int64_t)B + 1), 32) + 3 * align_up(4 * ((int64_t)B * Hkv + 1), 32);
+}
+
+__device__ __forceinline__ uint32_t bits_below(int64_t n) {  // tiles [0, n) of a 32-tile word
+  return n >= 32 ? 0xffffffffu : n <= 0 ? 0u : (1u << n) - 1u;
+}
+
+__global__ void __launch_bounds__(kPlanThreads, 1)
+plan_sparse_kernel(const int32_t* __restrict__ seq_lens, const uint32_t* __restrict__ mask, int W,
+                   const PlanHeader init, char* __restrict__ plan) {
+  griddep_wait();  // as the dense planner: inputs from the previous kernel are final
+  griddep_launch_dependents();
+  const int B = init.batch, Hkv = init.n_kv_heads, tl = init.tile_len, N = init.n_bins;
+  const int P = B * Hkv;
+  extern __shared__ __align__(16) uint8_t plan_smem[];
+  uint32_t* load = reinterpret_cast<uint32_t*>(plan_smem);                   // [N] load above the full-tile base
+  int32_t* pcount = reinterpret_cast<int32_t*>(plan_smem + 4 * (int64_t)N);  // [N] partial tiles per bin
+  __shared__ Tri warp_tot[kPlanWarps];
+  __shared__ int32_t sh_status;
+
+  PlanHeader* hdr = reinterpret_cast<PlanHeader*>(plan);
+  int32_t* PS = reinterpret_cast<int32_t*>(plan + init.off_S);
+  int32_t* PF = reinterpret_cast<int32_t*>(plan + init.off_SF);
+  int32_t* CBP = reinterpret_cast<int32_t*>(plan + init.off_cb);
+  int32_t* spairs = reinterpret_cast<int32_t*>(plan + init.off_sorted);
+  int32_t* gpbo = reinterpret_cast<int32_t*>(plan + init.off_pbin_off);
+  int32_t* gplist = reinterpret_cast<int32_t*>(plan + init.off_plist);
+  int32_t* KL = reinterpret_cast<int32_t*>(plan + init.off_kl);
+  char* scr = plan + init.off_scratch;
+  const int64_t rs = align_up(4 * ((int64_t)B + 1), 32), ps = align_up(4 * ((int64_t)P + 1), 32);
+  int32_t* rq_list = reinterpret_cast<int32_t*>(scr);           // requests with a partial tile, b order
+  int32_t* rq_cost = reinterpret_cast<int32_t*>(scr + rs);      // their partial-tile cost
+  int32_t* rq_sorted = reinterpret_cast<int32_t*>(scr + 2 * rs);  // by cost (desc), then b
+  int32_t* sb = reinterpret_cast<int32_t*>(scr + 4 * rs);       // [m] request of sorted partial pair s
+  int32_t* part_bin = reinterpret_cast<int32_t*>(scr + 4 * rs + ps);
+  int32_t* part_pos = reinterpret_cast<int32_t*>(scr + 4 * rs + 2 * ps);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    sh_status = 0;
+    PlanHeader h = init;
+    h.magic = 0;  // published last, once the plan is complete
+    h.run_status = 0;
+    *hdr = h;
+  }
+
+  // ---- 1. per pair: kept tiles (a), kept full tiles (b), kept partial tile (c), combine chunks (d)
+  Tri carry{0, 0, 0, 0};
+  for (int base = 0; base < P; base += kPlanThreads) {
+    const int p = base + tid;
+    Tri v{0, 0, 0, 0};
+    if (p < P) {
+      int64_t L = seq_lens[p / Hkv];
+      if (L < 0) { atomicCAS(&sh_status, 0, DECATTN_EDEVICE); L = 0; }
+      const int64_t nb = (L + tl - 1) / tl, nf = L / tl;
+      const uint32_t* row = mask + (int64_t)p * W;
+      const int64_t nw = min((nb + 31) / 32, (int64_t)W);
+      long long kept = 0, keptf = 0;
+      for (int64_t w = 0; w < nw; ++w) {
+        const uint32_t word = row[w];
+        kept += __popc(word & bits_below(nb - 32 * w));
+        keptf += __popc(word & bits_below(nf - 32 * w));
+      }
+      v = Tri{kept, keptf, (int)(kept - keptf), combine_chunks(kept)};  // the partial tile is the only non-full one
+    }
+    Tri before = carry;
+    Tri ex = block_exscan(v, carry, warp_tot);
+    if (p < P) {
+      PS[p] = (int32_t)(before.a + ex.a);
+      PF[p] = (int32_t)(before.b + ex.b);
+      CBP[p] = (int32_t)(before.d + ex.d);
+    }
+  }
+  if (tid == 0) { PS[P] = (int32_t)carry.a; PF[P] = (int32_t)carry.b; CBP[P] = (int32_t)carry.d; }
+  const int64_t U64 = carry.a;
+  __syncthreads();
+  if (U64 > init.max_units) atomicCAS(&sh_status, 0, DECATTN_ECAPACITY);
+  __syncthreads();
+  if (sh_status != 0) {
+    if (tid == 0) {
+      hdr->n_units = 0;
+      hdr->status = sh_status;
+      __threadfence();
+      hdr->magic = kPlanMagic;
+    }
+    return;
+  }
+  const int U = (int)U64;
+  const int F = (int)carry.b;
+  const int m = carry.c;
+
+  // ---- 2. kept-tile lists: KL[PS[p] + j] = index of the pair's j-th kept tile
+  for (int p = tid; p < P; p += kPlanThreads) {
+    const int64_t L = seq_lens[p / Hkv];
+    const int64_t nb = (L + tl - 1) / tl;
+    const uint32_t* row = mask + (int64_t)p * W;
+    const int64_t nw = min((nb + 31) / 32, (int64_t)W);
+    int o = PS[p];
+    for (int64_t w = 0; w < nw; ++w) {
+      uint32_t word = row[w] & bits_below(nb - 32 * w);
+      while (word) {
+        KL[o++] = (int32_t)(32 * w + __ffs(word) - 1);
+        word &= word - 1u;
+      }
+    }
+  }
+
+  // ---- 3. requests with a partial tile by cost (desc), then b; then, in that order, their
+  //         pairs whose partial tile is kept (pair order within a request)
+  Tri c2{0, 0, 0, 0};
+  for (int base = 0; base < B; base += kPlanThreads) {
+    const int b = base + tid;
+    const int64_t L = b < B ? seq_lens[b] : 0;
+    const int has = b < B && L > 0 && (L % tl) != 0;
+    Tri before = c2;
+    Tri ex = block_exscan(Tri{has, 0, 0, 0}, c2, warp_tot);
+    if (has) {
+      rq_list[before.a + ex.a] = b;
+      rq_cost[before.a + ex.a] = (int32_t)(L % tl);
+    }
+  }
+  const int mB = (int)c2.a;
+  __syncthreads();
+  for (int j = tid; j < mB; j += kPlanThreads) {
+    const int cj = rq_cost[j];
+    int rank = 0;
+    for (int k = 0; k < mB; ++k) {
+      const int c = rq_cost[k];
+      rank += (c > cj) | ((c == cj) & (k < j));
+    }
+    rq_sorted[rank] = rq_list[j];
+  }
+  __syncthreads();
+  Tri c3{0, 0, 0, 0};
+  for (int base = 0; base < mB; base += kPlanThreads) {
+    const int i = base + tid;
+    int b = 0, last = 0;
+    long long cnt = 0;
+    if (i < mB) {
+      b = rq_sorted[i];
+      last = (int)((seq_lens[b] + tl - 1) / tl) - 1;  // the partial tile
+      for (int h = 0; h < Hkv; ++h)
+        if (last / 32 < W) cnt += (mask[((int64_t)b * Hkv + h) * W + last / 32] >> (last % 32)) & 1u;
+    }
+    Tri before = c3;
+    Tri ex = block_exscan(Tri{cnt, 0, 0, 0}, c3, warp_tot);
+    if (i < mB) {
+      int o = (int)(before.a + ex.a);
+      for (int h = 0; h < Hkv; ++h)
+        if (last / 32 < W && ((mask[((int64_t)b * Hkv + h) * W + last / 32] >> (last % 32)) & 1u)) {
+          spairs[o] = b * Hkv + h;
+          sb[o] = b;
+          ++o;
+        }
+    }
+  }
+  __syncthreads();
+
+  // ---- 4. greedy placement of the kept partial tiles (s-th in sorted order: pair spairs[s])
+  const int qf = F / N;
+  const int rf = F - qf * N;
+  const int first = min(m, N - rf);
+  for (int k = tid; k < N; k += kPlanThreads) {
+    uint32_t l = k < rf ? (uint32_t)tl : 0u;
+    int32_t pc = 0;
+    const int s = k - rf;
+    if (k >= rf && s < first) {
+      l += (uint32_t)(seq_lens[sb[s]] % tl);
+      pc = 1;
+      part_bin[s] = k;
+      part_pos[s] = 0;
+    }
+    load[k] = l;
+    pcount[k] = pc;
+  }
+  __syncthreads();
+  if (tid < 32 && first < m) {
+    const int K = (N + 31) / 32;
+#define DECATTN_GREEDY(KM) greedy_partials<KM>(tid, N, first, m, 1, tl, seq_lens, sb, load, pcount, part_bin, part_pos)
+    if (K <= 4) DECATTN_GREEDY(4);
+    else if (K <= 8) DECATTN_GREEDY(8);
+    else if (K <= 12) DECATTN_GREEDY(12);
+    else if (K <= 16) DECATTN_GREEDY(16);
+    else if (K <= 20) DECATTN_GREEDY(20);
+    else if (K <= 24) DECATTN_GREEDY(24);
+    else if (K <= 32) DECATTN_GREEDY(32);
+    else greedy_partials_smem(tid, N, first, m, 1, tl, seq_lens, sb, load, pcount, part_bin, part_pos);
+#undef DECATTN_GREEDY
+  }
+  __syncthreads();
+
+  // ---- 5. per-bin CSR offsets of the partial tiles, and the partial tiles bin by bin
+  {
+    Tri c4{0, 0, 0, 0};
+    for (int base = 0; base < N; base += kPlanThreads) {
+      const int k = base + tid;
+      Tri before = c4;
+      Tri ex = block_exscan(Tri{k < N ? pcount[k] : 0, 0, 0, 0}, c4, warp_tot);
+      if (k < N) gpbo[k] = (int32_t)(before.a + ex.a);
+    }
+    if (tid == 0) gpbo[N] = (int32_t)c4.a;
+  }
+  __syncthreads();
+  for (int s = tid; s < m; s += kPlanThreads) gplist[gpbo[part_bin[s]] + part_pos[s]] = s;
+  __syncthreads();
+  if (tid == 0) {
+    hdr->n_units = U;
+    hdr->n_full = F;
+    hdr->n_partial = m;
+    hdr->full_q = qf;
+    hdr->full_r = rf;
+    hdr->status = DECATTN_OK;
+    __threadfence();
+    hdr->magic = kPlanMagic;
+  }
+}
+
 // Writes the explicit work list of a finished plan: bin_off [N+1] and units [U] (CSR by
 // bin), decoded with the same plan_unit() the split kernel uses. One block; for tests and
 // diagnostics.
@@ -359,7 +583,9 @@ plan_export_kernel(const char* __restrict__ plan, const int32_t* __restrict__ se
     if (k < h.n_bins) {
       bin_off[k] = (int32_t)part[threadIdx.x];
       const int n = plan_bin_size(plan, h, k);
-      for (int j = 0; j < n; ++j) units[part[threadIdx.x] + j] = plan_unit(plan, h, seq_lens, k, j);
+      for (int j = 0; j < n; ++j)
+        units[part[threadIdx.x] + j] = h.sparse ? plan_unit_sparse(plan, h, seq_lens, k, j)
+                                                : plan_unit(plan, h, seq_lens, k, j);
     }
     __syncthreads();
   }
@@ -468,6 +694,7 @@ extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads,
   plan->tile_len = tile_len;
   plan->n_bins = n_bins;
   plan->max_units = cap;
+  plan->sparse = 0;
   return DECATTN_OK;
 }
 
@@ -478,4 +705,104 @@ extern "C" int dec_attn_plan_export(const dec_attn_plan_t* plan, const int32_t* 
   plan_export_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const char*>(plan->buf), seq_lens, bin_off, static_cast<Unit*>(units), max_units, n_units);
   return cudaGetLastError() == cudaSuccess ? DECATTN_OK : DECATTN_ECUDA;
+}
+
+// ------------------------------------------------------------------ block-sparse plan (host)
+namespace decattn {
+
+struct SparseLayout {
+  int64_t off_PS, off_PF, off_CBP, off_sp, off_pbo, off_pl, off_kl, off_scratch, total;
+};
+
+static SparseLayout plan_sparse_layout(int B, int Hkv, int N, int64_t cap) {
+  const int64_t P = (int64_t)B * Hkv;
+  SparseLayout L;
+  int64_t o = sizeof(PlanHeader);
+  L.off_PS = o; o = align_up(o + 4 * (P + 1), 32);
+  L.off_PF = o; o = align_up(o + 4 * (P + 1), 32);
+  L.off_CBP = o; o = align_up(o + 4 * (P + 1), 32);
+  L.off_sp = o; o = align_up(o + 4 * (P + 1), 32);
+  L.off_pbo = o; o = align_up(o + 4 * ((int64_t)N + 1), 32);
+  L.off_pl = o; o = align_up(o + 4 * (P + 1), 32);
+  L.off_kl = o; o = align_up(o + 4 * (cap + 1), 32);
+  L.off_scratch = o; o = align_up(o + plan_sparse_scratch_bytes(B, Hkv), 32);
+  L.total = o;
+  return L;
+}
+
+}  // namespace decattn
+
+extern "C" size_t dec_attn_plan_sparse_bytes(int batch, int n_kv_heads, int tile_len, int64_t max_total_kv_tokens,
+                                              int n_bins) {
+  if (n_bins == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    n_bins = default_bins(dev);
+  }
+  if (!plan_args_ok(batch, n_kv_heads, tile_len, max_total_kv_tokens, n_bins)) return 0;
+  const SparseLayout L = plan_sparse_layout(batch, n_kv_heads, n_bins,
+                                            plan_capacity(batch, n_kv_heads, tile_len, max_total_kv_tokens));
+  return L.total >= (1ll << 31) ? 0 : (size_t)L.total;
+}
+
+extern "C" int dec_attn_plan_sparse(const int32_t* seq_lens, const uint32_t* tile_mask, int mask_words, int batch,
+                                    int n_kv_heads, int tile_len, int64_t max_total_kv_tokens, int n_bins,
+                                    void* plan_buf, size_t plan_bytes, dec_attn_plan_t* plan, void* stream) {
+  if (!plan || !plan_buf || (batch > 0 && (!seq_lens || !tile_mask)) || mask_words <= 0) return DECATTN_EINVAL;
+  if (n_bins == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DECATTN_ECUDA;
+    n_bins = default_bins(dev);
+    if (n_bins <= 0) return DECATTN_ECUDA;
+  }
+  if (batch < 0 || n_kv_heads <= 0 || tile_len <= 0 || max_total_kv_tokens < 0 || n_bins < 0) return DECATTN_EINVAL;
+  if (!plan_args_ok(batch, n_kv_heads, tile_len, max_total_kv_tokens, n_bins)) return DECATTN_ENOTSUP;
+  if ((int64_t)batch * n_kv_heads * mask_words >= (1ll << 31)) return DECATTN_ENOTSUP;
+  if ((reinterpret_cast<uintptr_t>(plan_buf) & 15) != 0 || (reinterpret_cast<uintptr_t>(tile_mask) & 3) != 0)
+    return DECATTN_EALIGN;
+  const int64_t cap = plan_capacity(batch, n_kv_heads, tile_len, max_total_kv_tokens);
+  const SparseLayout L = plan_sparse_layout(batch, n_kv_heads, n_bins, cap);
+  if (L.total >= (1ll << 31)) return DECATTN_ENOTSUP;
+  if ((int64_t)plan_bytes < L.total) return DECATTN_ESMALL;
+
+  PlanHeader h{};
+  h.n_bins = n_bins;
+  h.batch = batch;
+  h.n_kv_heads = n_kv_heads;
+  h.tile_len = tile_len;
+  h.max_units = cap;
+  h.off_S = (int32_t)L.off_PS;
+  h.off_SF = (int32_t)L.off_PF;
+  h.off_cb = (int32_t)L.off_CBP;
+  h.off_sorted = (int32_t)L.off_sp;
+  h.off_pbin_off = (int32_t)L.off_pbo;
+  h.off_plist = (int32_t)L.off_pl;
+  h.off_kl = (int32_t)L.off_kl;
+  h.off_scratch = (int32_t)L.off_scratch;
+  h.sparse = 1;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t smem = (size_t)plan_bins_smem(n_bins);
+  if (!ensure_smem_attr((const void*)plan_sparse_kernel, kPlanMaxSmem)) return DECATTN_ECUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kPlanThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // launched while the previous kernel drains
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, plan_sparse_kernel, seq_lens, tile_mask, mask_words, h,
+                         static_cast<char*>(plan_buf)) != cudaSuccess)
+    return DECATTN_ECUDA;
+  plan->buf = plan_buf;
+  plan->buf_bytes = plan_bytes;
+  plan->batch = batch;
+  plan->n_kv_heads = n_kv_heads;
+  plan->tile_len = tile_len;
+  plan->n_bins = n_bins;
+  plan->max_units = cap;
+  plan->sparse = 1;
+  return DECATTN_OK;
 }

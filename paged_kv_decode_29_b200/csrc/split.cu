@@ -103,7 +103,7 @@ struct FullTileWalk {
 __device__ __forceinline__ void walk_init(FullTileWalk& w, const SplitParams& p, int lane) {
   w.fc = 0; w.nwin = 0; w.wsf = 0; w.ws = 0; w.cur = -1;
   w.L = 0; w.nf_in = 0; w.nb_in = 0; w.csf = 0; w.cs = 0;
-  if (p.B > kWalkMaxReq || p.tile_len <= 0) return;
+  if (p.sparse || p.B > kWalkMaxReq || p.tile_len <= 0) return;  // a sparse plan lists every tile
   const uint32_t tl = (uint32_t)p.tile_len;  // 32-bit divisions: the 64-bit ones are software routines
   const int nwin = (p.B + 31) / 32;
   // window sums, one window per iteration (coalesced, the next window's load in flight); lane l
@@ -258,7 +258,8 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
                                     // reading partials)
       const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
       bool good = hdr->magic == kPlanMagic && hdr->status == DECATTN_OK && hdr->n_bins == (int)gridDim.x &&
-                  hdr->batch == p.B && hdr->n_kv_heads == p.Hkv && hdr->tile_len == p.tile_len;
+                  hdr->batch == p.B && hdr->n_kv_heads == p.Hkv && hdr->tile_len == p.tile_len &&
+                  hdr->sparse == p.sparse;
       if (good) {
         hv = *hdr;
         good = walk.fc == 0 || hv.full_q + ((int)blockIdx.x < hv.full_r ? 1 : 0) == walk.fc;
@@ -274,7 +275,11 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
     auto next_unit = [&](int j, Unit& u) -> bool {
       if (j < walk.fc) { u = walk_unit(walk, p, lane, j); return true; }
       if (!waited) await_plan();
-      if (j < n_units) { u = plan_unit(p.plan, hv, p.seq_lens, blockIdx.x, j); return true; }
+      if (j < n_units) {
+        u = hv.sparse ? plan_unit_sparse(p.plan, hv, p.seq_lens, blockIdx.x, j)
+                      : plan_unit(p.plan, hv, p.seq_lens, blockIdx.x, j);
+        return true;
+      }
       return false;
     };
     // The next tile's descriptor and first 32 page ids are fetched right after the current

@@ -67,7 +67,8 @@ def _shape(**kw):
 
 
 def _plan(**kw):
-    base = dict(buf=0x10000, buf_bytes=1 << 20, batch=2, n_kv_heads=2, tile_len=64, n_bins=8, max_units=64)
+    base = dict(buf=0x10000, buf_bytes=1 << 20, batch=2, n_kv_heads=2, tile_len=64, n_bins=8, max_units=64,
+                sparse=0, reserved_=0)
     base.update(kw)
     return da.PlanT(*[base[f] for f, _ in da.PlanT._fields_])
 
