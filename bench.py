@@ -70,6 +70,9 @@ def parse():
     ap.add_argument("--profile", action="store_true",
                     help="only warm-up + timed steps (for ncu launch lists): no baseline, e2e, graph or clocks")
     ap.add_argument("--json-out", default="", help="also append the JSON line to this file")
+    ap.add_argument("--sparse", type=float, default=0.0,
+                    help="block-sparse decode: keep each (request, KV head, tile) with this probability "
+                         "(the tile with each request's newest token always kept); 0 = dense")
     ap.add_argument("--append", action="store_true",
                     help="each step starts with the fused pre-processing kernel (rotary embedding of the "
                          "step's new q / k rows and their KV append), and the decode reads the rotated q")
@@ -283,7 +286,18 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
     tab, lens = to_dev(pr.page_table), to_dev(pr.seq_lens)
     total = int(pr.seq_lens.astype(np.int64).sum())
     stream = torch.cuda.current_stream()
-    pl = da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total)
+    mask_dev = None
+    if args.sparse > 0:
+        pr.tile_mask = W.make_tile_mask(pr, args.sparse)
+        mask_dev = torch.from_numpy(pr.tile_mask.view(np.int32)).to(dev)
+
+    def make_plan(buf=None, stream=None):
+        if mask_dev is not None:
+            return da.plan_sparse(lens, mask_dev, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=buf,
+                                  stream=stream)
+        return da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=buf, stream=stream)
+
+    pl = make_plan()
     shape = da.make_shape(q, k, tab, da.kv_dtype_of(k), pr.sm_scale)
     ws = torch.empty(da.workspace_bytes(shape, pl), dtype=torch.uint8, device=dev)
     out = torch.empty((pr.batch, pr.q_tokens, pr.n_q_heads, pr.head_dim), dtype=torch.float32, device=dev)
@@ -320,7 +334,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
             if brk:
                 i += 1
                 evs[i].record(stream)
-        da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=pbuf)
+        make_plan(buf=pbuf)
         if brk:
             i += 1
             evs[i].record(stream)
@@ -400,7 +414,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
             with torch.cuda.graph(g, stream=gs):
                 if args.append:
                     da.append_rope(q_new, k_new, v_new, tab, lens, k, v, q_out=q_dec, stream=gs)
-                da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=pbuf, stream=gs)
+                make_plan(buf=pbuf, stream=gs)
                 da.run(q_dec, k, v, tab, lens, pl, stream=gs, **kw)
         stream.wait_stream(gs)
         gt = []
@@ -447,7 +461,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
             lens.copy_(hlens, non_blocking=True)
             if args.append:
                 da.append_rope(q_new, k_new, v_new, tab, lens, k, v, q_out=q_dec)
-            da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=pbuf)
+            make_plan(buf=pbuf)
             da.run(q_dec, k, v, tab, lens, pl, **kw)
             hout.copy_(out, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
@@ -474,7 +488,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
     split_gbs = alg / (split_m * 1e-6) / 1e9
     step_gbs = alg / (step_m * 1e-6) / 1e9
     sc_gbs = alg / ((split_m + comb_m) * 1e-6) / 1e9  # split + combine, each timed between events
-    traffic = ncu_traffic(args.config, pr.tile_len)
+    traffic = None if mask_dev is not None else ncu_traffic(args.config, pr.tile_len)
     line = {
         "metric": METRIC, "value": round(step_m, 3), "unit": "us/step", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_m / 1e3, 6), "higher_is_better": False,
@@ -496,6 +510,13 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
                      "traffic": None if traffic is None else int(traffic)},
         "gpu_launches": n_kernels * args.steps,  # [append,] planner, split, combine kernels per timed step
     }
+    if mask_dev is not None:
+        nb = (pr.seq_lens.astype(np.int64) + pr.tile_len - 1) // pr.tile_len
+        i = np.arange(int(nb.max()) if pr.batch else 0)
+        kept = ((pr.tile_mask[:, :, i // 32] >> (i % 32).astype(np.uint32)) & 1).astype(bool) & (i[None, None, :] < nb[:, None, None])
+        line["config"]["sparse"] = {"density": args.sparse, "kept_tiles": int(kept.sum()),
+                                    "tiles": int(nb.sum()) * pr.n_kv_heads,
+                                    "note": "algorithmic bytes count the kept tiles' KV only"}
     if args.append:
         # the fused pre-processing kernel: bytes it must move once (new q/k/v rows in, rotated q
         # and the k/v rows out, seq_lens and one page-table entry per new token)

@@ -130,10 +130,16 @@ __device__ void greedy_partials(int lane, int N, int first, int m, int Hkv, int 
       const uint32_t key = __reduce_min_sync(0xffffffffu, (lmin << 5) | (uint32_t)lane);
       if ((int)(key & 31u) == lane) {
         const int s = s0 + i;
-        part_bin[s] = k0 + lj;
+        int pos = 0;
         #pragma unroll
-        for (int j = 0; j < KMAX; ++j)
-          if (j == lj) { part_pos[s] = pc[j]; pc[j] += 1; ld[j] += c; }
+        for (int j = 0; j < KMAX; ++j) {  // selects only: no store or branch per register
+          const bool sel = j == lj;
+          pos = sel ? pc[j] : pos;
+          pc[j] += sel ? 1 : 0;
+          ld[j] += sel ? c : 0u;
+        }
+        part_bin[s] = k0 + lj;
+        part_pos[s] = pos;
         lmin = ld[0];
         lj = 0;
         #pragma unroll

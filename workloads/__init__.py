@@ -123,15 +123,31 @@ class Problem:
         return 1 if self.kv_dtype == "fp8e4m3" else 2
 
     def algorithmic_bytes(self) -> int:
-        """Bytes the method must move once: visible KV rows, q, out+lse, page-table rows, scales."""
+        """Bytes the method must move once: visible KV rows, q, out+lse, page-table rows, scales.
+        With a block-sparse tile mask, only the kept tiles' KV rows (per KV head), and the pages
+        some head keeps."""
         d, P, hkv = self.head_dim, self.page_size, self.n_kv_heads
         L = self.seq_lens.astype(np.int64)
-        kv = int(L.sum()) * hkv * d * self.kv_elem_bytes() * 2
         q = self.q.nbytes
         out = self.batch * self.q_tokens * self.n_q_heads * (d + 1) * 4
-        pages = int(((L + P - 1) // P).sum())
+        if self.tile_mask is None:
+            kv = int(L.sum()) * hkv * d * self.kv_elem_bytes() * 2
+            pages = int(((L + P - 1) // P).sum())
+            kv_pages = pages * hkv
+        else:
+            tl = self.tile_len
+            kv = pages = kv_pages = 0
+            for b in range(self.batch):
+                nb = int((L[b] + tl - 1) // tl)
+                i = np.arange(nb)
+                kept = ((self.tile_mask[b][:, i // 32] >> (i % 32).astype(np.uint32)) & 1).astype(bool)  # [Hkv][nb]
+                toks = np.minimum((i + 1) * tl, L[b]) - i * tl
+                kv += int((kept * toks[None, :]).sum()) * d * self.kv_elem_bytes() * 2
+                pg = -(-toks // P)  # pages per tile
+                pages += int((kept.any(axis=0) * pg).sum())
+                kv_pages += int((kept * pg[None, :]).sum())
         table = pages * 4 + self.batch * 4
-        scales = pages * hkv * 2 * 4 if self.kv_scales is not None else 0
+        scales = kv_pages * 2 * 4 if self.kv_scales is not None else 0
         return kv + q + out + table + scales
 
 
