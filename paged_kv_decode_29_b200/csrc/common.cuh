@@ -47,7 +47,8 @@ struct PlanHeader {
   int32_t off_scratch;  // planner scratch
   int32_t sparse;       // 1: block-sparse plan (per-pair arrays below, see plan_unit_sparse)
   int32_t off_kl;       // sparse: int32 [max_units]: tile index of kept tile j of pair p at PS[p] + j
-  int32_t reserved[9];
+  int32_t gsm_off;      // planner launch: offset of the batched greedy's shared-memory area (0: none)
+  int32_t reserved[8];
 };
 static_assert(sizeof(PlanHeader) == 128, "plan header is 128 bytes");
 constexpr int32_t kPlanMagic = 0x32504144;  // "DAP2"

@@ -155,6 +155,116 @@ __device__ void greedy_partials(int lane, int N, int first, int m, int Hkv, int 
   }
 }
 
+// The same greedy pass over the partial tiles s in [first, m), batched: the bins are kept
+// sorted by (load, bin) in shared memory, and each round one warp tries the next up-to-32
+// tiles (largest first) on the least-loaded bins in order. Tile t of the round goes to the
+// t-th sorted bin exactly when that bin's key is below every bin the round has touched
+// (their keys plus the tiles they got), so the round assigns its longest prefix of such tiles
+// (at least one), merges the touched bins back into the sorted list and repeats. Same
+// assignment as one tile at a time, ties included (the bin index is the key's low word).
+// Called by every thread of the block (the first sort is block-wide). Shared area: the sorted
+// keys [P2] and a merge buffer [N] (uint64), the round's new keys [32], the tiles' costs [m].
+__host__ __device__ inline int pow2_ceil(int n) {
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
+__host__ __device__ inline int64_t greedy_batched_bytes(int N, int64_t max_partials) {
+  return align_up(8 * (int64_t)pow2_ceil(N) + 8 * (int64_t)N + 8 * 32 + 4 * max_partials, 16);
+}
+
+__device__ void greedy_batched(int N, int first, int m, int Hkv, int tl, const int32_t* __restrict__ seq_lens,
+                               const int32_t* sorted_b, const uint32_t* load_sm, int32_t* pcount_sm, uint8_t* area,
+                               int32_t* part_bin, int32_t* part_pos) {
+  const int tid = threadIdx.x;
+  const int P2 = pow2_ceil(N);
+  uint64_t* A = reinterpret_cast<uint64_t*>(area);
+  uint64_t* A2 = A + P2;
+  uint64_t* Bn = A2 + N;
+  uint32_t* cost = reinterpret_cast<uint32_t*>(Bn + 32);
+  for (int s = first + tid; s < m; s += kPlanThreads) cost[s - first] = (uint32_t)(seq_lens[sorted_b[s / Hkv]] % tl);
+  for (int i = tid; i < P2; i += kPlanThreads) A[i] = i < N ? ((uint64_t)load_sm[i] << 32) | (uint32_t)i : ~0ull;
+  __syncthreads();
+  for (int k = 2; k <= P2; k <<= 1)  // bitonic sort, ascending
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < P2; i += kPlanThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint64_t x = A[i], y = A[ixj];
+          if ((x > y) == ((i & k) == 0)) { A[i] = y; A[ixj] = x; }
+        }
+      }
+      __syncthreads();
+    }
+  if (tid < 32) {
+    const int lane = tid;
+    uint64_t* cur = A;
+    uint64_t* nxt = A2;
+    for (int s = first; s < m;) {
+      const int W = min(min(32, m - s), N);  // a round tries at most one tile per bin
+      const uint64_t a = lane < W ? cur[lane] : ~0ull;
+      const uint64_t nw = lane < W ? a + ((uint64_t)cost[s - first + lane] << 32) : ~0ull;
+      uint64_t x = nw;  // inclusive prefix minimum of the round's new keys
+      #pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x = min(x, y);
+      }
+      uint64_t pm = __shfl_up_sync(0xffffffffu, x, 1);
+      if (lane == 0) pm = ~0ull;
+      const unsigned bad = __ballot_sync(0xffffffffu, !(lane < W && a < pm));
+      const int J = bad ? __ffs(bad) - 1 : 32;  // >= 1: lane 0 always qualifies
+      if (lane < J) {
+        const int bin = (int)(uint32_t)a;
+        part_bin[s + lane] = bin;
+        part_pos[s + lane] = pcount_sm[bin];
+        pcount_sm[bin] += 1;
+      }
+      uint64_t key = lane < J ? nw : ~0ull;  // sort the touched bins' keys across the warp
+      #pragma unroll
+      for (int k = 2; k <= 32; k <<= 1)
+        #pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+          const uint64_t other = __shfl_xor_sync(0xffffffffu, key, j);
+          key = (((lane & j) == 0) == ((lane & k) == 0)) ? min(key, other) : max(key, other);
+        }
+      Bn[lane] = key;
+      __syncwarp();
+      if (lane < J) {  // a touched bin lands after the untouched keys below it
+        int lo = J, hi = N;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (cur[mid] < key) lo = mid + 1; else hi = mid;
+        }
+        nxt[lane + (lo - J)] = key;
+      }
+      const int n_old = N - J;  // the untouched keys, one contiguous run per lane
+      const int ch = (n_old + 31) >> 5;
+      const int i0 = lane * ch, i1 = min(n_old, i0 + ch);
+      if (i0 < i1) {
+        int lo = 0, hi = J;
+        const uint64_t x0 = cur[J + i0];
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (Bn[mid] < x0) lo = mid + 1; else hi = mid;
+        }
+        int r = lo;
+        for (int i = i0; i < i1; ++i) {
+          const uint64_t xo = cur[J + i];
+          while (r < J && Bn[r] < xo) ++r;
+          nxt[i + r] = xo;
+        }
+      }
+      __syncwarp();
+      uint64_t* t = cur;
+      cur = nxt;
+      nxt = t;
+      s += J;
+    }
+  }
+}
+
 // Same rule with the loads in shared memory (more bins than the register version holds).
 __device__ void greedy_partials_smem(int lane, int N, int first, int m, int Hkv, int tl,
                                      const int32_t* __restrict__ seq_lens, const int32_t* sorted_b, uint32_t* load_sm,
@@ -291,7 +401,10 @@ plan_kernel(const int32_t* __restrict__ seq_lens, const PlanHeader init, char* _
     pcount[k] = pc;
   }
   __syncthreads();
-  if (tid < 32 && first < m) {
+  if (first < m && init.gsm_off > 0) {
+    greedy_batched(N, first, m, Hkv, tl, seq_lens, R.sorted_b, load, pcount, plan_smem + init.gsm_off, part_bin,
+                   part_pos);
+  } else if (tid < 32 && first < m) {
     const int K = (N + 31) / 32;
 #define DECATTN_GREEDY(KM) \
   greedy_partials<KM>(tid, N, first, m, Hkv, tl, seq_lens, R.sorted_b, load, pcount, part_bin, part_pos)
@@ -522,7 +635,9 @@ plan_sparse_kernel(const int32_t* __restrict__ seq_lens, const uint32_t* __restr
     pcount[k] = pc;
   }
   __syncthreads();
-  if (tid < 32 && first < m) {
+  if (first < m && init.gsm_off > 0) {
+    greedy_batched(N, first, m, 1, tl, seq_lens, sb, load, pcount, plan_smem + init.gsm_off, part_bin, part_pos);
+  } else if (tid < 32 && first < m) {
     const int K = (N + 31) / 32;
 #define DECATTN_GREEDY(KM) greedy_partials<KM>(tid, N, first, m, 1, tl, seq_lens, sb, load, pcount, part_bin, part_pos)
     if (K <= 4) DECATTN_GREEDY(4);
@@ -678,8 +793,14 @@ extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads,
   h.off_plist = (int32_t)L.off_plist;
   h.off_scratch = (int32_t)L.off_scratch;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t smem =
+  size_t smem =
       (size_t)plan_bins_smem(n_bins) + (batch <= kPlanSmemRequests ? (size_t)req_arrays_bytes(batch) : 0);
+  smem = (size_t)align_up((int64_t)smem, 16);
+  const int64_t gsm = greedy_batched_bytes(n_bins, (int64_t)batch * n_kv_heads);
+  if ((int64_t)smem + gsm <= kPlanMaxSmem) {  // room for the batched greedy pass
+    h.gsm_off = (int32_t)smem;
+    smem += (size_t)gsm;
+  }
   if (!ensure_smem_attr((const void*)plan_kernel, kPlanMaxSmem)) return DECATTN_ECUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
@@ -787,7 +908,12 @@ extern "C" int dec_attn_plan_sparse(const int32_t* seq_lens, const uint32_t* til
   h.off_scratch = (int32_t)L.off_scratch;
   h.sparse = 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t smem = (size_t)plan_bins_smem(n_bins);
+  size_t smem = (size_t)align_up(plan_bins_smem(n_bins), 16);
+  const int64_t gsm = greedy_batched_bytes(n_bins, (int64_t)batch * n_kv_heads);
+  if ((int64_t)smem + gsm <= kPlanMaxSmem) {  // room for the batched greedy pass
+    h.gsm_off = (int32_t)smem;
+    smem += (size_t)gsm;
+  }
   if (!ensure_smem_attr((const void*)plan_sparse_kernel, kPlanMaxSmem)) return DECATTN_ECUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
