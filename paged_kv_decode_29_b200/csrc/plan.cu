@@ -27,6 +27,7 @@ constexpr int kPlanWarps = kPlanThreads / 32;
 constexpr int kPlanMaxBins = 8192;
 constexpr int kPlanSmemRequests = 4096;  // per-request arrays sit in shared memory up to this batch
 constexpr int kPlanMaxSmem = 200 * 1024;
+constexpr int kPlanRegWords = 8;  // sparse planner: mask words of a pair held in registers
 
 // Per-request arrays (index b): exclusive prefix sums over requests of the tiles of one
 // (b, h) pair (S), of its full tiles (SF) and of "has a partial tile" (SP); the requests
@@ -155,113 +156,138 @@ __device__ void greedy_partials(int lane, int N, int first, int m, int Hkv, int 
   }
 }
 
-// The same greedy pass over the partial tiles s in [first, m), batched: the bins are kept
-// sorted by (load, bin) in shared memory, and each round one warp tries the next up-to-32
-// tiles (largest first) on the least-loaded bins in order. Tile t of the round goes to the
-// t-th sorted bin exactly when that bin's key is below every bin the round has touched
-// (their keys plus the tiles they got), so the round assigns its longest prefix of such tiles
-// (at least one), merges the touched bins back into the sorted list and repeats. Same
-// assignment as one tile at a time, ties included (the bin index is the key's low word).
-// Called by every thread of the block (the first sort is block-wide). Shared area: the sorted
-// keys [P2] and a merge buffer [N] (uint64), the round's new keys [32], the tiles' costs [m].
-__host__ __device__ inline int pow2_ceil(int n) {
-  int p = 1;
-  while (p < n) p <<= 1;
-  return p;
+// The same greedy pass over the partial tiles s in [first, m), batched across the block: the
+// bins are kept sorted by key (load << 32 | bin) in shared memory, and each round tries the
+// next up-to-kPlanThreads tiles (largest first) on the least-loaded bins in order. Tile t of
+// the round goes to the t-th sorted bin exactly when that bin's key is below every key the
+// round has made so far (a touched bin's key plus its tile), so the round assigns the longest
+// prefix of such tiles (at least one), merges the touched bins back into the sorted list and
+// repeats. Same assignment as one tile at a time, ties included (the bin index is the key's
+// low word).
+//
+// Called only when the closed-form first batch left tiles over (first < m), so the first batch
+// filled bins rf .. N-1 (rf = N - first), one tile each, with non-increasing loads, and bins
+// 0 .. rf-1 hold one more full tile (load tl, above every partial tile's cost). The sorted list
+// therefore starts without a sort: the first batch's bins by (load, bin), each placed with two
+// binary searches, then bins 0 .. rf-1 in order. The merge of a round places every key by its
+// rank: the round's new keys are sorted within each warp (32-key chunks), and a key's rank is
+// its count of smaller keys in every chunk and in the untouched run.
+// Called by every thread of the block. Shared area: two key lists [N], the round's new keys
+// [kPlanThreads], warp minima [kPlanWarps], the round's prefix length, the costs of tiles
+// [first, m).
+__host__ __device__ inline int64_t greedy_batched_bytes(int N, int64_t max_partials) {
+  return align_up(16 * (int64_t)N + 8 * (int64_t)(kPlanThreads + kPlanWarps) + 16 + 4 * max_partials, 16);
 }
 
-__host__ __device__ inline int64_t greedy_batched_bytes(int N, int64_t max_partials) {
-  return align_up(8 * (int64_t)pow2_ceil(N) + 8 * (int64_t)N + 8 * 32 + 4 * max_partials, 16);
+__device__ __forceinline__ int count_below32(const uint64_t* c, uint64_t k) {  // sorted c[0, 32)
+  int pos = 0;
+  #pragma unroll
+  for (int step = 16; step > 0; step >>= 1)
+    if (c[pos + step - 1] < k) pos += step;
+  return pos + (c[pos] < k ? 1 : 0);  // pos = min(count, 31) here
+}
+
+__device__ __forceinline__ int count_below(const uint64_t* c, int n, uint64_t k) {  // sorted c[0, n)
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (c[mid] < k) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
 }
 
 __device__ void greedy_batched(int N, int first, int m, int Hkv, int tl, const int32_t* __restrict__ seq_lens,
                                const int32_t* sorted_b, const uint32_t* load_sm, int32_t* pcount_sm, uint8_t* area,
                                int32_t* part_bin, int32_t* part_pos) {
-  const int tid = threadIdx.x;
-  const int P2 = pow2_ceil(N);
-  uint64_t* A = reinterpret_cast<uint64_t*>(area);
-  uint64_t* A2 = A + P2;
-  uint64_t* Bn = A2 + N;
-  uint32_t* cost = reinterpret_cast<uint32_t*>(Bn + 32);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint64_t* cur = reinterpret_cast<uint64_t*>(area);
+  uint64_t* nxt = cur + N;
+  uint64_t* Bn = nxt + N;
+  uint64_t* wmin = Bn + kPlanThreads;
+  int* sJ = reinterpret_cast<int*>(wmin + kPlanWarps);
+  uint32_t* cost = reinterpret_cast<uint32_t*>(sJ + 4);
+  const int rf = N - first;
   for (int s = first + tid; s < m; s += kPlanThreads) cost[s - first] = (uint32_t)(seq_lens[sorted_b[s / Hkv]] % tl);
-  for (int i = tid; i < P2; i += kPlanThreads) A[i] = i < N ? ((uint64_t)load_sm[i] << 32) | (uint32_t)i : ~0ull;
+  const uint32_t* c0 = load_sm + rf;  // the first batch's loads, non-increasing in s
+  for (int s = tid; s < first; s += kPlanThreads) {
+    const uint32_t c = c0[s];
+    int lo = 0, hi = s;  // first index holding c
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (c0[mid] > c) lo = mid + 1;
+      else hi = mid;
+    }
+    const int eq0 = lo;
+    lo = s + 1;
+    hi = first;  // first index below c
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (c0[mid] >= c) lo = mid + 1;
+      else hi = mid;
+    }
+    cur[(first - lo) + (s - eq0)] = ((uint64_t)c << 32) | (uint32_t)(rf + s);
+  }
+  for (int k = tid; k < rf; k += kPlanThreads) cur[first + k] = ((uint64_t)load_sm[k] << 32) | (uint32_t)k;
   __syncthreads();
-  for (int k = 2; k <= P2; k <<= 1)  // bitonic sort, ascending
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P2; i += kPlanThreads) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint64_t x = A[i], y = A[ixj];
-          if ((x > y) == ((i & k) == 0)) { A[i] = y; A[ixj] = x; }
-        }
-      }
-      __syncthreads();
+  for (int s = first; s < m;) {
+    const int W = min(min(kPlanThreads, m - s), N);  // a round tries at most one tile per bin
+    if (tid == 0) *sJ = W;
+    const uint64_t a = tid < W ? cur[tid] : ~0ull;
+    const uint64_t nw = tid < W ? a + ((uint64_t)cost[s - first + tid] << 32) : ~0ull;
+    uint64_t x = nw;  // inclusive prefix minimum of the round's new keys
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x = min(x, y);
     }
-  if (tid < 32) {
-    const int lane = tid;
-    uint64_t* cur = A;
-    uint64_t* nxt = A2;
-    for (int s = first; s < m;) {
-      const int W = min(min(32, m - s), N);  // a round tries at most one tile per bin
-      const uint64_t a = lane < W ? cur[lane] : ~0ull;
-      const uint64_t nw = lane < W ? a + ((uint64_t)cost[s - first + lane] << 32) : ~0ull;
-      uint64_t x = nw;  // inclusive prefix minimum of the round's new keys
-      #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x = min(x, y);
-      }
-      uint64_t pm = __shfl_up_sync(0xffffffffu, x, 1);
-      if (lane == 0) pm = ~0ull;
-      const unsigned bad = __ballot_sync(0xffffffffu, !(lane < W && a < pm));
-      const int J = bad ? __ffs(bad) - 1 : 32;  // >= 1: lane 0 always qualifies
-      if (lane < J) {
-        const int bin = (int)(uint32_t)a;
-        part_bin[s + lane] = bin;
-        part_pos[s + lane] = pcount_sm[bin];
-        pcount_sm[bin] += 1;
-      }
-      uint64_t key = lane < J ? nw : ~0ull;  // sort the touched bins' keys across the warp
-      #pragma unroll
-      for (int k = 2; k <= 32; k <<= 1)
-        #pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-          const uint64_t other = __shfl_xor_sync(0xffffffffu, key, j);
-          key = (((lane & j) == 0) == ((lane & k) == 0)) ? min(key, other) : max(key, other);
-        }
-      Bn[lane] = key;
-      __syncwarp();
-      if (lane < J) {  // a touched bin lands after the untouched keys below it
-        int lo = J, hi = N;
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (cur[mid] < key) lo = mid + 1; else hi = mid;
-        }
-        nxt[lane + (lo - J)] = key;
-      }
-      const int n_old = N - J;  // the untouched keys, one contiguous run per lane
-      const int ch = (n_old + 31) >> 5;
-      const int i0 = lane * ch, i1 = min(n_old, i0 + ch);
-      if (i0 < i1) {
-        int lo = 0, hi = J;
-        const uint64_t x0 = cur[J + i0];
-        while (lo < hi) {
-          const int mid = (lo + hi) >> 1;
-          if (Bn[mid] < x0) lo = mid + 1; else hi = mid;
-        }
-        int r = lo;
-        for (int i = i0; i < i1; ++i) {
-          const uint64_t xo = cur[J + i];
-          while (r < J && Bn[r] < xo) ++r;
-          nxt[i + r] = xo;
-        }
-      }
-      __syncwarp();
-      uint64_t* t = cur;
-      cur = nxt;
-      nxt = t;
-      s += J;
+    if (lane == 31) wmin[warp] = x;
+    __syncthreads();
+    uint64_t pm = ~0ull;
+    for (int w = 0; w < warp; ++w) pm = min(pm, wmin[w]);
+    const uint64_t up = __shfl_up_sync(0xffffffffu, x, 1);
+    if (lane > 0) pm = min(pm, up);  // exclusive: the keys of tiles 0 .. tid-1
+    if (tid < W && !(a < pm)) atomicMin(sJ, tid);
+    __syncthreads();
+    const int J = *sJ;  // >= 1: tile 0 always qualifies
+    uint64_t key = ~0ull;
+    if (tid < J) {
+      const int bin = (int)(uint32_t)a;
+      part_bin[s + tid] = bin;
+      part_pos[s + tid] = pcount_sm[bin];
+      pcount_sm[bin] += 1;  // the round's bins are distinct
+      key = nw;
     }
+    #pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)  // sort the warp's chunk, ascending (~0 pads last)
+      #pragma unroll
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        const uint64_t other = __shfl_xor_sync(0xffffffffu, key, j);
+        key = (((lane & j) == 0) == ((lane & k) == 0)) ? min(key, other) : max(key, other);
+      }
+    Bn[tid] = key;
+    __syncthreads();
+    const int nc = (J + 31) >> 5;
+    if (key != ~0ull) {
+      int r = lane + count_below(cur + J, N - J, key);
+      #pragma unroll
+      for (int c = 0; c < kPlanWarps; ++c)
+        if (c < nc && c != warp) r += count_below32(Bn + 32 * c, key);
+      nxt[r] = key;
+    }
+    for (int i = J + tid; i < N; i += kPlanThreads) {
+      const uint64_t xo = cur[i];
+      int r = i - J;
+      #pragma unroll
+      for (int c = 0; c < kPlanWarps; ++c)
+        if (c < nc) r += count_below32(Bn + 32 * c, xo);
+      nxt[r] = xo;
+    }
+    __syncthreads();
+    uint64_t* t = cur;
+    cur = nxt;
+    nxt = t;
+    s += J;
   }
 }
 
@@ -505,20 +531,33 @@ plan_sparse_kernel(const int32_t* __restrict__ seq_lens, const uint32_t* __restr
     *hdr = h;
   }
 
-  // ---- 1. per pair: kept tiles (a), kept full tiles (b), kept partial tile (c), combine chunks (d)
+  // ---- 1. per pair: kept tiles (a), kept full tiles (b), kept partial tile (c), combine chunks (d);
+  //         then the pair's kept-tile list KL[PS[p] + j] = index of its j-th kept tile. The
+  //         first kPlanRegWords mask words stay in registers between the two (loads in flight
+  //         together); a pair whose list would pass max_units is not listed (the plan fails).
   Tri carry{0, 0, 0, 0};
   for (int base = 0; base < P; base += kPlanThreads) {
     const int p = base + tid;
     Tri v{0, 0, 0, 0};
+    uint32_t wr[kPlanRegWords];
+    int64_t nb = 0, nw = 0;
+    const uint32_t* row = mask + (int64_t)p * W;
     if (p < P) {
       int64_t L = seq_lens[p / Hkv];
       if (L < 0) { atomicCAS(&sh_status, 0, DECATTN_EDEVICE); L = 0; }
-      const int64_t nb = (L + tl - 1) / tl, nf = L / tl;
-      const uint32_t* row = mask + (int64_t)p * W;
-      const int64_t nw = min((nb + 31) / 32, (int64_t)W);
+      nb = (L + tl - 1) / tl;
+      const int64_t nf = L / tl;
+      nw = min((nb + 31) / 32, (int64_t)W);
+      #pragma unroll
+      for (int w = 0; w < kPlanRegWords; ++w) wr[w] = w < nw ? __ldg(row + w) & bits_below(nb - 32 * w) : 0u;
       long long kept = 0, keptf = 0;
-      for (int64_t w = 0; w < nw; ++w) {
-        const uint32_t word = row[w];
+      #pragma unroll
+      for (int w = 0; w < kPlanRegWords; ++w) {
+        kept += __popc(wr[w]);
+        keptf += __popc(wr[w] & bits_below(nf - 32 * w));
+      }
+      for (int64_t w = kPlanRegWords; w < nw; ++w) {
+        const uint32_t word = __ldg(row + w);
         kept += __popc(word & bits_below(nb - 32 * w));
         keptf += __popc(word & bits_below(nf - 32 * w));
       }
@@ -527,9 +566,28 @@ plan_sparse_kernel(const int32_t* __restrict__ seq_lens, const uint32_t* __restr
     Tri before = carry;
     Tri ex = block_exscan(v, carry, warp_tot);
     if (p < P) {
-      PS[p] = (int32_t)(before.a + ex.a);
+      const long long o0 = before.a + ex.a;
+      PS[p] = (int32_t)o0;
       PF[p] = (int32_t)(before.b + ex.b);
       CBP[p] = (int32_t)(before.d + ex.d);
+      if (o0 + v.a <= init.max_units) {
+        int o = (int)o0;
+        #pragma unroll
+        for (int w = 0; w < kPlanRegWords; ++w) {
+          uint32_t word = wr[w];
+          while (word) {
+            KL[o++] = (int32_t)(32 * w + __ffs(word) - 1);
+            word &= word - 1u;
+          }
+        }
+        for (int64_t w = kPlanRegWords; w < nw; ++w) {
+          uint32_t word = __ldg(row + w) & bits_below(nb - 32 * w);
+          while (word) {
+            KL[o++] = (int32_t)(32 * w + __ffs(word) - 1);
+            word &= word - 1u;
+          }
+        }
+      }
     }
   }
   if (tid == 0) { PS[P] = (int32_t)carry.a; PF[P] = (int32_t)carry.b; CBP[P] = (int32_t)carry.d; }
@@ -549,22 +607,6 @@ plan_sparse_kernel(const int32_t* __restrict__ seq_lens, const uint32_t* __restr
   const int U = (int)U64;
   const int F = (int)carry.b;
   const int m = carry.c;
-
-  // ---- 2. kept-tile lists: KL[PS[p] + j] = index of the pair's j-th kept tile
-  for (int p = tid; p < P; p += kPlanThreads) {
-    const int64_t L = seq_lens[p / Hkv];
-    const int64_t nb = (L + tl - 1) / tl;
-    const uint32_t* row = mask + (int64_t)p * W;
-    const int64_t nw = min((nb + 31) / 32, (int64_t)W);
-    int o = PS[p];
-    for (int64_t w = 0; w < nw; ++w) {
-      uint32_t word = row[w] & bits_below(nb - 32 * w);
-      while (word) {
-        KL[o++] = (int32_t)(32 * w + __ffs(word) - 1);
-        word &= word - 1u;
-      }
-    }
-  }
 
   // ---- 3. requests with a partial tile by cost (desc), then b; then, in that order, their
   //         pairs whose partial tile is kept (pair order within a request)

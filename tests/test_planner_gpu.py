@@ -57,6 +57,9 @@ def test_plan_random(seed):
     ([4096] * 32, 8, 256, 592),           # full tiles only: round-robin
     (list(range(1, 1200)), 8, 1024, 592), # ~9.6k partial tiles through the sequential pass
     ([65536] * 3 + [17] * 5, 4, 128, 7),
+    ([300] * 500, 8, 256, 592),           # 4000 partial tiles of one cost: ties in every round
+    (list(range(1, 3000, 7)), 2, 64, 37), # few bins, many rounds of the batched pass
+    ([4000 + 37 * i for i in range(80)], 8, 256, 592),  # the first batch leaves a few tiles over
 ])
 def test_plan_edges(lens, hkv, tl, n_bins):
     assert_same(lens, hkv, tl, n_bins)

@@ -43,6 +43,8 @@ def gpu_plan_sparse(lens, mask, hkv, tl, n_bins, max_total=None):
     ([131072], 8, 256, 592, 0.1),
     ([700, 1, 33, 2000, 64, 65] * 20, 4, 64, 148, 0.5),
     ([40] * 3, 2, 16, 5, 0.0),
+    ([300] * 200, 8, 256, 592, 0.5),      # many kept partial tiles of one cost
+    ([5000 + 41 * i for i in range(64)], 8, 256, 592, 0.3),
 ])
 def test_sparse_plan_matches_oracle(lens, hkv, tl, n_bins, density):
     mask = _random_mask(lens, hkv, tl, density, seed=len(lens) + hkv)
