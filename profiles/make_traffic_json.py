@@ -17,10 +17,10 @@ import workloads as W  # noqa: E402
 
 # workload -> (requests captured, dram read bytes, dram write bytes) of the captured launch
 CAPTURED = {
-    "uniform": (8, 134357504, 3178752),
-    "mixed": (16, 1039154432, 17398016),
-    "fp8_spec": (4, 167197184, 8819968),
-    "long_b4": (1, 536966144, 6233856),
+    "uniform": (8, 134361088, 3281408),
+    "mixed": (16, 1039147264, 17551104),
+    "fp8_spec": (4, 167213568, 5203200),
+    "long_b4": (1, 536967936, 5665536),
 }
 
 
