@@ -1,0 +1,808 @@
+// split_tc.cu -- the split kernel for FP8 E4M3 KV on the fifth-generation tensor cores
+// (tcgen05, accumulators in tensor memory). Same method, plan, workspace and outputs as
+// split.cu ("PaddlePaddle/HALOps" README, Highlights, GQA attention item: paged-KV decode with
+// FP8 KV and speculative decoding; "HPC-Ops: Tencent's CUDA Kernel Library for LLM Inference
+// Hot Paths", "How the kernels are organized around specific workload shapes": uniform tiles,
+// greedy bins, a combine), for head_dim 128 and G*T <= 16.
+//
+// The legacy warp-level MMA path spends most of its instructions moving fragments: with G*T = 16
+// and FP8 K/V it is bound by instruction issue, not by memory. Here a tile is processed in
+// chunks of 128 keys and each product is one tensor-core instruction stream:
+//  * S^T (128 keys x 16 query rows, fp32 in tensor memory) = K Q^T on kind::f8f6f4, A = the
+//    staged K codes as TMA left them (K-major, 128-byte swizzle), B = q split into two E4M3
+//    parts hi + lo (written K-major by the softmax warps), accumulated into one result;
+//  * O^T (128 head dims x 16 query rows, fp32 in tensor memory) += V^T P^T on kind::f16, A = V
+//    widened to f16 once per element (MN-major), B = P^T in f16 (MN-major).
+// Thread j of the 128-thread softmax group owns key j of the chunk (tensor-memory lane j) and
+// reads its 16 scores with one tcgen05.ld, so the per-key work has no fragment shuffles.
+//
+// Online softmax with a reference maximum: P = 2^(s - m_ref) for every key of a tile, where
+// m_ref is the exact maximum of the tile's first chunk and moves (to the running maximum) only
+// when a later chunk holds a score above m_ref + kTcTau; then O^T and the running sums are
+// rescaled in place. P is thus at most 2^kTcTau, which keeps P * (V page scale) * kTcPScale
+// inside f16, and most chunks need only a one-flag-per-warp check instead of an exact maximum.
+//
+// CTA: 6 warps, 2 CTAs per SM, and one wave of CTAs: CTA i takes bins i, i + grid, ... .
+//  * warps 0-3 (softmax group; warp w reads tensor-memory lanes 32w..32w+31): per chunk, V
+//    widening first (it frees the ring stage early), then scores -> P and the O^T rescale; per
+//    tile, the next tile's q (loaded from global memory during the last chunk and published
+//    before the epilogue, so the MMA warp starts that tile meanwhile) and the epilogue;
+//  * warp 4 (producer): the bins' tiles (walk, then plan) and their K/V pages by TMA, 128-key
+//    chunks in a two-stage ring, FP8 page scales by cp.async;
+//  * warp 5 (MMA): allocates tensor memory and issues every tcgen05.mma from one thread.
+// Every wait is bounded; a wait that gives up sets DECATTN_ETIMEOUT and a CTA-wide abort flag,
+// after which every role leaves its loop and the CTA frees its tensor memory and exits.
+#include "common.cuh"
+#include "walk.cuh"
+
+namespace decattn {
+
+constexpr int kTcD = 128;          // head_dim
+constexpr int kTcN = 16;           // MMA N: query rows of the KV group, zero-padded
+constexpr int kTcChunk = 128;      // keys per chunk: the M of S^T and the contraction of O^T
+constexpr int kTcBlk = kTcChunk / 16;  // 16-key blocks (one TMA box each) per chunk
+constexpr int kTcStages = 2;       // chunk stages of the K/V ring
+constexpr int kTcThreads = 192;
+constexpr int kTcTau = 6;          // P <= 2^kTcTau
+constexpr float kTcPScale = 64.f;  // P enters the MMA as P * (V page scale) * kTcPScale
+constexpr int kTcTmemCols = 64;    // S^T double buffer (2 x 16 columns), O^T (16), spare (power of 2)
+
+// Shared-memory layout (offsets from a 1024-byte aligned base).
+struct TcSmem {
+  static constexpr int KCH = kTcChunk * kTcD;                // bytes of one K (or V) chunk: 16 KB
+  static constexpr int QB = 2 * kTcN * kTcD;                 // q hi [16][128] then lo, E4M3
+  static constexpr int OFF_K = 0;                            // [stage][128 keys][128 B], 128-B swizzle
+  static constexpr int OFF_V = OFF_K + kTcStages * KCH;
+  static constexpr int OFF_V16 = OFF_V + kTcStages * KCH;    // f16 V^T, MN-major interleaved core matrices
+  static constexpr int OFF_P16 = OFF_V16 + 2 * KCH;          // f16 P^T, MN-major interleaved
+  static constexpr int OFF_QB = OFF_P16 + kTcChunk * kTcN * 2;  // [tile parity] q hi / lo, 128-B swizzle
+  static constexpr int OFF_SC = OFF_QB + 2 * QB;             // per stage: 8 K scales, 8 V scales
+  static constexpr int OFF_QCS = OFF_SC + kTcStages * 2 * kTcBlk * 4;  // [tile parity][16]: 2^-E of q rows
+  static constexpr int OFF_FLG = OFF_QCS + 2 * kTcN * 4;     // [2][4] per-warp "passes the reference" flags
+  static constexpr int OFF_RED = OFF_FLG + 2 * 4 * 4;        // [2][4][16] chunk maxima per warp
+  static constexpr int OFF_ERED = OFF_RED + 2 * 4 * kTcN * 4;  // [4][16] row-sum partials
+  static constexpr int OFF_UNIT = OFF_ERED + 4 * kTcN * 4;   // Unit x 2
+  static constexpr int OFF_BAR = OFF_UNIT + 2 * (int)sizeof(Unit);
+  static constexpr int NBAR = 17;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;        // tensor-memory base, abort flag
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;                 // slack to align the base to 1024
+};
+static_assert(TcSmem::OFF_QB % 1024 == 0 && TcSmem::QB % 1024 == 0, "swizzled q operands need 1024-byte bases");
+static_assert(TcSmem::OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
+static_assert(2 * (TcSmem::ALLOC + 1024) <= 228 * 1024, "two CTAs per SM");
+
+// Barrier slots.
+enum TcBar {
+  kKvFull = 0,   // [2] producer -> MMA, softmax: K, V and scales of a chunk landed
+  kKvEmpty = 2,  // [2] MMA commit (K read) + 4 softmax warps (V widened) -> producer
+  kSFull = 4,    // [2] MMA commit -> softmax: S^T of a chunk is in tensor memory
+  kSFree = 6,    // [2] 4 softmax warps -> MMA: that S^T buffer has been read
+  kPReady = 8,   // 4 softmax warps -> MMA: P^T and V^T (f16) written, O^T rescaled if needed
+  kPvDone = 9,   // MMA commit -> softmax: O^T += V^T P^T of a chunk complete
+  kUFull = 10,   // [2] producer -> MMA, softmax: tile descriptor written
+  kUEmpty = 12,  // [2] MMA + 4 softmax warps -> producer: tile descriptor read
+  kQReady = 14,  // 4 softmax warps -> MMA: q hi / lo of the next tile written
+  kGroup = 15,   // 4 softmax warps: the group's own barrier (bounded, unlike bar.sync)
+  kFin = 16,     // MMA commit -> MMA: every tensor-core operation of the CTA complete
+};
+// ------------------------------------------------------------------ tcgen05 helpers
+// Shared-memory matrix descriptor: start address, leading / stride byte offsets (16-byte
+// units), version 1, layout type (0: no swizzle, 2: 128-byte swizzle).
+__device__ __forceinline__ uint64_t umma_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  return (uint64_t)((addr >> 4) & 0x3fffu) | ((uint64_t)((lbo >> 4) & 0x3fffu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3fffu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+
+// Instruction descriptor: fp32 accumulator, A / B formats (kind::f8f6f4: 0 = E4M3;
+// kind::f16: 0 = f16), A / B major-ness (0 = K, 1 = MN), N and M.
+__host__ __device__ constexpr uint32_t umma_idesc(uint32_t afmt, uint32_t bfmt, uint32_t amaj, uint32_t bmaj, int M,
+                                                  int N) {
+  return (1u << 4) | (afmt << 7) | (bfmt << 10) | (amaj << 15) | (bmaj << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// The mbarrier gets one arrival once every tensor-core operation issued so far by this thread
+// has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Generic-proxy shared-memory writes become visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 16 consecutive 32-bit columns of this warp's 32 tensor-memory lanes (lane i -> thread i).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  #pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Non-blocking test of a phase (no suspend: the pipeline hand-offs here are short and a
+// suspended waiter wakes late).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// A bounded wait that also gives up at once when another role has aborted the CTA.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    #pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_test(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_status(status, DECATTN_ETIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+// Float -> integer with the same order (for warp max reductions with redux.sync).
+__device__ __forceinline__ int ordered_int(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float ordered_float(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
+
+}  // namespace decattn
+
+namespace decattn {
+
+// q rows of a tile, bf16: thread (r = tid / 8, seg = tid % 8) loads elements 16 seg .. 16 seg + 15
+// of query row r (rows >= G*T are zero).
+__device__ __forceinline__ void tc_load_q(const SplitParams& p, const Unit& d, uint4 (&x)[2]) {
+  const int r = threadIdx.x >> 3, seg = threadIdx.x & 7;
+  x[0] = x[1] = make_uint4(0, 0, 0, 0);
+  if (r < p.GT) {
+    const int t = r / p.G, gg = r - t * p.G;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        p.q + (((int64_t)d.b * p.T + t) * p.Hq + (int64_t)d.h * p.G + gg) * kTcD + 16 * seg);
+    x[0] = __ldg(src);
+    x[1] = __ldg(src + 1);
+  }
+}
+
+// q hi / lo of a tile into its operand buffer (E4M3, K-major, 128-byte swizzle) and the
+// per-row factor 2^-E into qcs. q is scaled by a per-row power of two 2^E (largest |q| lands in
+// [128, 256)) and split into two E4M3 parts, hi = E4M3(q 2^E) and lo = E4M3(q 2^E - hi), which
+// together carry the 8 significant bits of a bf16 q.
+__device__ __forceinline__ void tc_store_q(const uint4 (&x)[2], uint8_t* qb, float* qcs) {
+  const int r = threadIdx.x >> 3, seg = threadIdx.x & 7;
+  float v[16];
+  #pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t w4[4] = {x[h].x, x[h].y, x[h].z, x[h].w};
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) { v[8 * h + 2 * i] = bf16_lo(w4[i]); v[8 * h + 2 * i + 1] = bf16_hi(w4[i]); }
+  }
+  float amax = 0.f;
+  #pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+  // 2^E with E = 7 - floor(log2 amax): exponent-field arithmetic, exact
+  const int ex = amax > 0.f ? ((__float_as_int(amax) >> 23) & 0xff) - 127 : 0;
+  const int E = min(max(7 - ex, -100), 100);
+  const float up = __int_as_float((127 + E) << 23);
+  uint32_t hw[4], lw[4];
+  #pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t hh[2], ll[2];
+    #pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float a0 = v[4 * i + 2 * k] * up, a1 = v[4 * i + 2 * k + 1] * up;
+      hh[k] = f32x2_to_e4m3x2(a0, a1);
+      const float2 b = f16x2_to_float2(e4m3x2_to_f16x2(hh[k]));
+      ll[k] = f32x2_to_e4m3x2(a0 - b.x, a1 - b.y);
+    }
+    hw[i] = hh[0] | (hh[1] << 16);
+    lw[i] = ll[0] | (ll[1] << 16);
+  }
+  const int off = r * kTcD + ((seg ^ (r & 7)) << 4);
+  *reinterpret_cast<uint4*>(qb + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  *reinterpret_cast<uint4*>(qb + kTcN * kTcD + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  if (seg == 0) qcs[r] = __int_as_float((127 - E) << 23);
+}
+
+__global__ void __launch_bounds__(kTcThreads, 2)
+split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+  using L = TcSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  float* sc = reinterpret_cast<float*>(sm + L::OFF_SC);  // [stage][16]: K scales of the 8 blocks, then V scales
+  Unit* umeta = reinterpret_cast<Unit*>(sm + L::OFF_UNIT);
+  uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(sm + L::OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(sm + L::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // The combine counters of this workspace start from zero on every run (as in split.cu).
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)p.B * p.T * p.Hq;
+       i += (int64_t)gridDim.x * blockDim.x)
+    p.row_cnt[i] = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&bar[kKvFull + s], 1);
+      mbar_init(&bar[kKvEmpty + s], 1 + 4);
+      mbar_init(&bar[kSFull + s], 1);
+      mbar_init(&bar[kSFree + s], 4);
+      mbar_init(&bar[kUFull + s], 1);
+      mbar_init(&bar[kUEmpty + s], 1 + 4);
+    }
+    mbar_init(&bar[kPReady], 4);
+    mbar_init(&bar[kPvDone], 1);
+    mbar_init(&bar[kQReady], 4);
+    mbar_init(&bar[kGroup], 4);
+    mbar_init(&bar[kFin], 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {  // tensor memory: S^T (two buffers), O^T
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_base_sm)),
+                 "n"(kTcTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_sm;
+
+  if (warp == 4) {
+    // ===================================================================== producer
+    if (lane == 0) { prefetch_tensormap(&tmK); prefetch_tensormap(&tmV); }
+    const int P = p.P;
+    int st = 0; uint32_t eph = 1;  // K/V ring stage and the parity of its "empty" wait
+    int us = 0; uint32_t ueph = 1; // tile descriptor slot
+    int64_t n_fill = 0;            // chunks issued
+    bool ok = true;
+    // Tiles of this CTA's bins (bin = blockIdx.x, blockIdx.x + gridDim.x, ...: the grid holds
+    // only as many CTAs as are resident at once): each bin's full tiles from the walk, then
+    // (after waiting for the planner, once) the rest from the plan, as in split.cu.
+    int bin = blockIdx.x;
+    FullTileWalk walk;
+    walk_init(walk, p, lane, bin, p.n_bins);
+    int jb = 0;              // next tile of the current bin
+    int bin_units = -1;      // tiles of the current bin, once the plan is read
+    bool plan_loaded = false, plan_good = false;
+    int32_t pending = 0;
+    PlanHeader hv = {};
+    auto note = [&](int32_t code) {
+      if (plan_loaded) set_status(p.status, code);
+      else if (pending == 0) pending = code;
+    };
+    auto load_plan = [&]() {
+      plan_loaded = true;
+      griddep_wait();               // the plan kernel has finished and its writes are visible
+      griddep_launch_dependents();  // the combine kernel may be scheduled now
+      const PlanHeader* hdr = reinterpret_cast<const PlanHeader*>(p.plan);
+      plan_good = hdr->magic == kPlanMagic && hdr->status == DECATTN_OK && hdr->n_bins == p.n_bins &&
+                  hdr->batch == p.B && hdr->n_kv_heads == p.Hkv && hdr->tile_len == p.tile_len &&
+                  hdr->sparse == p.sparse;
+      if (plan_good) hv = *hdr;
+      else if (lane == 0)
+        set_status(p.status, hdr->magic != kPlanMagic ? DECATTN_EINVAL
+                             : hdr->status != DECATTN_OK ? hdr->status : DECATTN_EINVAL);
+      if (pending != 0) set_status(p.status, pending);
+    };
+    auto next_unit = [&](Unit& u) -> bool {
+      while (bin < p.n_bins) {
+        if (jb < walk.fc) { u = walk_unit(walk, p, lane, jb++, bin, p.n_bins); return true; }
+        if (!plan_loaded) load_plan();
+        if (plan_good && bin_units < 0) {
+          if (walk.fc != 0 && hv.full_q + (bin < hv.full_r ? 1 : 0) != walk.fc) {  // walk and plan disagree
+            if (lane == 0) set_status(p.status, DECATTN_EINVAL);
+            plan_good = false;
+          } else {
+            bin_units = plan_bin_size(p.plan, hv, bin);
+          }
+        }
+        if (plan_good && jb < bin_units) {
+          u = hv.sparse ? plan_unit_sparse(p.plan, hv, p.seq_lens, bin, jb)
+                        : plan_unit(p.plan, hv, p.seq_lens, bin, jb);
+          ++jb;
+          return true;
+        }
+        bin += gridDim.x;  // the next bin of this CTA
+        jb = 0;
+        bin_units = -1;
+        walk_rebin(walk, bin, p.n_bins);
+      }
+      return false;
+    };
+    auto wait0 = [&](uint64_t* b, uint32_t par) -> bool {  // lane 0 waits, the warp follows
+      int r = 1;
+      if (lane == 0) r = tc_wait(b, par, p.status, abort) ? 1 : 0;
+      return __shfl_sync(0xffffffffu, r, 0) != 0;
+    };
+    Unit dn;
+    bool has_n = next_unit(dn);
+    for (int u = 0; has_n && ok; ++u) {
+      const Unit d = dn;
+      if (!wait0(&bar[kUEmpty + us], ueph)) { ok = false; break; }
+      if (lane == 0) {
+        umeta[us] = d;
+        mbar_arrive(&bar[kUFull + us]);
+      }
+      us ^= 1; if (us == 0) ueph ^= 1;
+      const int pg0 = d.tok_begin / P;
+      const int npg = (d.tok_end - d.tok_begin + P - 1) / P;
+      if (lane == 0 && pg0 + npg > p.mpps) note(DECATTN_EDEVICE);  // row too short
+      const int nblk = (d.tok_end - d.tok_begin + 15) / 16;
+      int win = -1, pid_w = 0;  // page ids of pages [32 win, 32 win + 32) of the tile, one per lane
+      bool looked = false;
+      for (int b0 = 0; b0 < nblk && ok; b0 += kTcBlk) {
+        const int nb = min(kTcBlk, nblk - b0);
+        const int blk = b0 + lane;        // this lane's block (lane < nb)
+        const int ip = (blk * 16) / P;    // its page, relative to the tile
+        // a chunk starts page-aligned (tiles are multiples of the page size) and spans <= 8
+        // pages, so all of its pages sit in one window of 32
+        const int w_need = (b0 * 16) / P / 32;
+        if (w_need != win) {
+          win = w_need;
+          const int pg = win * 32 + lane;
+          pid_w = pg < npg ? p.page_table[(int64_t)d.b * p.mpps + min(pg0 + pg, p.mpps - 1)] : 0;
+          if (pg < npg && (pid_w < 0 || pid_w >= p.num_pages)) {
+            note(DECATTN_EDEVICE);
+            pid_w = 0;  // keeps the copy inside the pool; the result is flagged invalid
+          }
+        }
+        const int pid = __shfl_sync(0xffffffffu, pid_w, (ip - win * 32) & 31);
+        if (!wait0(&bar[kKvEmpty + st], eph)) { ok = false; break; }
+        if (lane < nb) {  // FP8 page scales of the block (K, V), folded into the chunk's barrier
+          const int64_t si = (int64_t)pid * p.Hkv + d.h;
+          cp_async_4(&sc[st * 16 + lane], p.kv_scales + si);
+          cp_async_4(&sc[st * 16 + 8 + lane], p.kv_scales + (int64_t)p.num_pages * p.Hkv + si);
+          cp_async_mbar_arrive(&bar[kKvFull + st]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(&bar[kKvFull + st], (uint32_t)(nb * 2 * 16 * kTcD));
+        __syncwarp();
+        if (lane < nb) {
+          const int row = (pid * p.Hkv + d.h) * P + (blk * 16) % P;
+          tma_load_2d(sm + L::OFF_K + st * L::KCH + lane * 16 * kTcD, &tmK, 0, row, &bar[kKvFull + st]);
+          tma_load_2d(sm + L::OFF_V + st * L::KCH + lane * 16 * kTcD, &tmV, 0, row, &bar[kKvFull + st]);
+        }
+        ++n_fill;
+        if (++st == kTcStages) { st = 0; eph ^= 1; }
+        if (!looked) {  // the next tile's descriptor, fetched while this tile's first copies fly
+          looked = true;
+          has_n = next_unit(dn);
+        }
+      }
+      if (!looked && ok) has_n = next_unit(dn);
+    }
+    if (!plan_loaded) load_plan();
+    if (ok) {
+      // no more tiles: a descriptor with b = -1 tells the MMA warp and the softmax group to stop
+      if (wait0(&bar[kUEmpty + us], ueph)) {
+        if (lane == 0) {
+          umeta[us].b = -1;
+          mbar_arrive(&bar[kUFull + us]);
+        }
+      } else {
+        ok = false;
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort = 1;
+      // let the copies already issued land before the CTA exits
+      for (int64_t n = n_fill > kTcStages ? n_fill - kTcStages : 0; n < n_fill; ++n)
+        mbar_wait(&bar[kKvFull + n % kTcStages], (uint32_t)((n / kTcStages) & 1), nullptr);
+    }
+  } else if (warp == 5) {
+    // ===================================================================== MMA issue
+    if (lane == 0) {
+      const uint32_t base = smem_u32(sm);
+      constexpr uint32_t idS = umma_idesc(0, 0, 0, 0, kTcChunk, kTcN);  // E4M3 x E4M3, both K-major
+      constexpr uint32_t idO = umma_idesc(0, 0, 1, 1, kTcD, kTcN);      // f16 x f16, both MN-major
+      int us = 0; uint32_t uph = 0;
+      int64_t g = 0;  // chunks issued so far
+      int ut = 0;     // tiles started so far
+      bool ok = true;
+      // O^T (+)= V^T P^T over the chunk's 128 keys, 16 per instruction. A tile's first chunk
+      // overwrites O^T: the softmax group signals that chunk's P only after it has read the
+      // previous tile's O^T in its epilogue.
+      // descriptors, built once: the start address is the low 14 bits (16-byte units), so a
+      // k-step adds to the base descriptor
+      const uint64_t dV = umma_desc(base + L::OFF_V16, 128, 2048, 0), dP = umma_desc(base + L::OFF_P16, 128, 2048, 0);
+      const uint64_t dK0 = umma_desc(base + L::OFF_K, 16, 1024, 2), dQ0 = umma_desc(base + L::OFF_QB, 16, 1024, 2);
+      auto pv = [&](int64_t gg, bool first_of_tile, uint32_t tO) -> bool {
+        if (!tc_wait(&bar[kPReady], (uint32_t)(gg & 1), p.status, abort)) return false;
+        tc_fence_after();
+        #pragma unroll
+        for (int k = 0; k < kTcChunk / 16; ++k)
+          umma_f16(tO, dV + (uint64_t)(16 * k), dP + (uint64_t)(16 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
+        umma_commit(&bar[kPvDone]);
+        return true;
+      };
+      for (;;) {
+        if (!tc_wait(&bar[kUFull + us], uph, p.status, abort)) { ok = false; break; }
+        const Unit d = umeta[us];
+        mbar_arrive(&bar[kUEmpty + us]);
+        us ^= 1; if (us == 0) uph ^= 1;
+        if (d.b < 0) break;
+        const int nc = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
+        if (!tc_wait(&bar[kQReady], (uint32_t)(ut & 1), p.status, abort)) { ok = false; break; }
+        const uint64_t dQ = dQ0 + (uint64_t)(((ut & 1) * L::QB) >> 4);
+        const uint32_t tO = tmem + 2 * kTcN;
+        for (int c = 0; c < nc; ++c, ++g) {
+          const int st = (int)(g % kTcStages), sb = (int)(g & 1);
+          if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort) ||
+              !tc_wait(&bar[kSFree + sb], (uint32_t)(((g >> 1) & 1) ^ 1), p.status, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // S^T = K (q hi)^T + K (q lo)^T: four 32-byte k-steps of the 128-byte swizzled rows
+          const uint64_t dK = dK0 + (uint64_t)((st * L::KCH) >> 4);
+          #pragma unroll
+          for (int kk = 0; kk < kTcD / 32; ++kk) {
+            const uint64_t a = dK + (uint64_t)(2 * kk);
+            umma_f8(tmem + kTcN * sb, a, dQ + (uint64_t)(2 * kk), idS, kk > 0 ? 1u : 0u);
+            umma_f8(tmem + kTcN * sb, a, dQ + (uint64_t)((kTcN * kTcD) >> 4) + (uint64_t)(2 * kk), idS, 1u);
+          }
+          umma_commit(&bar[kSFull + sb]);
+          umma_commit(&bar[kKvEmpty + st]);  // the K half of the stage has been read
+          if (c > 0 && !pv(g - 1, c == 1, tO)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (!pv(g - 1, nc == 1, tO)) { ok = false; break; }
+        ++ut;
+      }
+      if (!ok) *abort = 1;
+      // every tensor-core operation of the CTA completes before the memory is freed
+      umma_commit(&bar[kFin]);
+      mbar_wait(&bar[kFin], 0, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ===================================================================== softmax group
+    const int key = threadIdx.x;  // key of the chunk / head dim of O^T = tensor-memory lane
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const float LN2 = 0.6931471805599453f;
+    float* qcs_sm = reinterpret_cast<float*>(sm + L::OFF_QCS);   // [tile parity][16]
+    int* red = reinterpret_cast<int*>(sm + L::OFF_RED);          // [2][4][16] chunk maxima (ordered ints)
+    int* flg = reinterpret_cast<int*>(sm + L::OFF_FLG);          // [2][4]
+    float* ered = reinterpret_cast<float*>(sm + L::OFF_ERED);    // [4][16] row-sum partials
+    int us = 0; uint32_t uph = 0;
+    int64_t g = 0;    // chunks processed so far
+    int ut = 0;       // tiles processed so far
+    uint32_t gn = 0;  // group-barrier uses so far
+    bool ok = true;
+    auto gsync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[kGroup]);
+      return tc_wait(&bar[kGroup], (gn++) & 1u, p.status, abort);
+    };
+    auto next_desc = [&](Unit& dd) -> bool {
+      if (!tc_wait(&bar[kUFull + us], uph, p.status, abort)) return false;
+      dd = umeta[us];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[kUEmpty + us]);
+      us ^= 1; if (us == 0) uph ^= 1;
+      return true;
+    };
+    // q of a tile into operand buffer `par`; the MMA warp may start the tile afterwards
+    auto publish_q = [&](const uint4 (&x)[2], int par) -> bool {
+      tc_store_q(x, sm + L::OFF_QB + par * L::QB, qcs_sm + kTcN * par);
+      fence_async_smem();
+      if (!gsync()) return false;
+      if (lane == 0) mbar_arrive(&bar[kQReady]);
+      return true;
+    };
+    Unit d;
+    d.b = -1;
+    if (!next_desc(d)) ok = false;
+    if (ok && d.b >= 0) {
+      uint4 x[2];
+      tc_load_q(p, d, x);
+      ok = publish_q(x, 0);
+    }
+    while (ok && d.b >= 0) {
+      const int qp = ut & 1;
+      const uint32_t tO = tmem + lane_off + 2 * kTcN;
+      const float4* qcs4 = reinterpret_cast<const float4*>(qcs_sm + kTcN * qp);
+      // lane n < G*T: the output row of query row n (final out, or the tile's partial slot)
+      int64_t row_n = 0;
+      if (lane < p.GT) {
+        const int t = lane / p.G, gg = lane - (lane / p.G) * p.G;
+        row_n = d.slot < 0 ? ((int64_t)d.b * p.T + t) * p.Hq + (int64_t)d.h * p.G + gg
+                           : (int64_t)d.slot * p.GT + lane;
+      }
+      const int causal_base = d.seq_len - p.T;  // query row n sees key j iff j - base <= n / G
+      float mref[kTcN], lacc[kTcN];
+      #pragma unroll
+      for (int n = 0; n < kTcN; ++n) {
+        mref[n] = -INFINITY;
+        lacc[n] = 0.f;
+      }
+      Unit dnext;
+      dnext.b = -1;
+      uint4 qx[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+      const int nc = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
+      for (int c = 0; c < nc; ++c, ++g) {
+        const int st = (int)(g % kTcStages), sb = (int)(g & 1);
+        if (c == nc - 1) {  // the next tile: its descriptor now, its q rows in flight meanwhile
+          if (!next_desc(dnext)) { ok = false; break; }
+          if (dnext.b >= 0) tc_load_q(p, dnext, qx);
+        }
+        // ---- V first: it frees the ring stage for the producer as early as possible. The
+        //      previous chunk's P V must have read the f16 buffers.
+        if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort) ||
+            (c > 0 && !tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort))) {
+          ok = false;
+          break;
+        }
+        const int j = d.tok_begin + c * kTcChunk + key;
+        const bool valid = j < d.tok_end;
+        // ---- V row of this key widened to f16 (exact), 8 head dims per 16-byte core-matrix row
+        {
+          const uint8_t* vr = sm + L::OFF_V + st * L::KCH + key * kTcD;
+          uint8_t* vd = sm + L::OFF_V16 + (key >> 3) * 128 + (key & 7) * 16;
+          #pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (valid) w = *reinterpret_cast<const uint4*>(vr + ((cc ^ (key & 7)) << 4));  // codes d = 16cc ..
+            const uint4 lo = make_uint4(e4m3x2_to_f16x2(w.x & 0xffffu), e4m3x2_to_f16x2(w.x >> 16),
+                                        e4m3x2_to_f16x2(w.y & 0xffffu), e4m3x2_to_f16x2(w.y >> 16));
+            const uint4 hi = make_uint4(e4m3x2_to_f16x2(w.z & 0xffffu), e4m3x2_to_f16x2(w.z >> 16),
+                                        e4m3x2_to_f16x2(w.w & 0xffffu), e4m3x2_to_f16x2(w.w >> 16));
+            *reinterpret_cast<uint4*>(vd + (2 * cc) * 2048) = lo;
+            *reinterpret_cast<uint4*>(vd + (2 * cc + 1) * 2048) = hi;
+          }
+        }
+        // this key's page scales, read before the stage (scales included) goes back to the producer
+        const int blk = key >> 4;
+        const float f = p.qk_scale_log2 * sc[st * 16 + blk];
+        const float vsc = sc[st * 16 + 8 + blk] * kTcPScale;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[kKvEmpty + st]);  // the V half of the stage has been read
+        if (!tc_wait(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort)) { ok = false; break; }
+        tc_fence_after();
+        float s[kTcN];
+        tmem_ld16(tmem + lane_off + kTcN * sb, s);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[kSFree + sb]);
+
+        // ---- scale, mask; per-column maxima of the chunk
+        int* rw = red + ((sb * 4 + warp) * kTcN);
+        #pragma unroll
+        for (int q4 = 0; q4 < kTcN / 4; ++q4) {
+          const float4 qc = qcs4[q4];
+          s[4 * q4] *= f * qc.x; s[4 * q4 + 1] *= f * qc.y; s[4 * q4 + 2] *= f * qc.z; s[4 * q4 + 3] *= f * qc.w;
+        }
+        const int over = j - causal_base;  // > 0 only for the last T - 1 keys of the request
+        if (!valid) {
+          #pragma unroll
+          for (int n = 0; n < kTcN; ++n) s[n] = -INFINITY;
+        } else if (over > 0) {
+          #pragma unroll
+          for (int n = 0; n < kTcN; ++n)
+            if (n < p.GT && over > n / p.G) s[n] = -INFINITY;
+        }
+        // does any score of the chunk pass the reference by more than kTcTau? (one flag per warp)
+        // (a tile's first chunk goes straight to the exact maxima: its reference is unset)
+        bool upd = c == 0;
+        if (!upd) {
+          bool over_ref = false;
+          #pragma unroll
+          for (int n = 0; n < kTcN; ++n) over_ref |= s[n] > mref[n] + (float)kTcTau;
+          const int wflag = __any_sync(0xffffffffu, over_ref) ? 1 : 0;
+          if (lane == 0) flg[sb * 4 + warp] = wflag;
+          if (!gsync()) { ok = false; break; }
+          const int4 f4 = *reinterpret_cast<const int4*>(flg + sb * 4);
+          upd = (f4.x | f4.y | f4.z | f4.w) != 0;  // the same in every thread
+        }
+        float cm[kTcN];
+        if (upd) {
+          // exact maxima of the chunk: the reference moves to the running maximum
+          #pragma unroll
+          for (int n = 0; n < kTcN; ++n) {
+            const int m = __reduce_max_sync(0xffffffffu, ordered_int(s[n]));
+            if (lane == 0) rw[n] = m;
+          }
+          if (!gsync()) { ok = false; break; }
+          const int4* r4 = reinterpret_cast<const int4*>(red + sb * 4 * kTcN);
+          #pragma unroll
+          for (int q4 = 0; q4 < kTcN / 4; ++q4) {
+            int4 m = r4[q4];
+            #pragma unroll
+            for (int w = 1; w < 4; ++w) {
+              const int4 o = r4[w * (kTcN / 4) + q4];
+              m.x = max(m.x, o.x); m.y = max(m.y, o.y); m.z = max(m.z, o.z); m.w = max(m.w, o.w);
+            }
+            cm[4 * q4] = ordered_float(m.x); cm[4 * q4 + 1] = ordered_float(m.y);
+            cm[4 * q4 + 2] = ordered_float(m.z); cm[4 * q4 + 3] = ordered_float(m.w);
+          }
+        }
+        if (upd) {
+          float alpha[kTcN];
+          bool resc = false;
+          #pragma unroll
+          for (int n = 0; n < kTcN; ++n) {
+            const float mn = fmaxf(mref[n], cm[n]);
+            alpha[n] = mn == -INFINITY ? 1.f : fast_exp2(mref[n] - mn);
+            resc |= alpha[n] != 1.f;
+            mref[n] = mn;
+            lacc[n] *= alpha[n];
+          }
+          if (c > 0 && resc) {
+            // O^T holds chunks 0 .. c-1 of this tile (their P V is done): rescale it in place
+            tc_fence_after();
+            float o[kTcN];
+            tmem_ld16(tO, o);
+            #pragma unroll
+            for (int n = 0; n < kTcN; ++n) o[n] *= alpha[n];
+            tmem_st16(tO, o);
+          }
+        }
+        // ---- P = 2^(s - m_ref) (at most 2^kTcTau); row sums in fp32
+        float (&pr)[kTcN] = s;  // in place
+        #pragma unroll
+        for (int n = 0; n < kTcN; ++n) {
+          pr[n] = fast_exp2(s[n] - (mref[n] == -INFINITY ? 0.f : mref[n]));
+          lacc[n] += pr[n];
+        }
+        // ---- P^T row of this key: f16 P * (V page scale) * kTcPScale, 16 query rows
+        {
+          uint32_t h[8];
+          #pragma unroll
+          for (int i = 0; i < 8; ++i) h[i] = valid ? pack_f16(pr[2 * i] * vsc, pr[2 * i + 1] * vsc) : 0u;
+          uint8_t* pp = sm + L::OFF_P16 + (key >> 3) * 128 + (key & 7) * 16;
+          *reinterpret_cast<uint4*>(pp) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(pp + 2048) = make_uint4(h[4], h[5], h[6], h[7]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[kPReady]);
+      }
+      if (!ok) break;
+      // ---- the next tile's q: the MMA warp starts that tile while this one's epilogue runs
+      if (dnext.b >= 0 && !publish_q(qx, qp ^ 1)) { ok = false; break; }
+
+      // ---- epilogue: row sums over the tile, O^T / l, out or partial
+      if (!tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
+      tc_fence_after();
+      // row sums over the warp's 32 keys by a butterfly reduce-scatter: after the five levels,
+      // lanes 2c and 2c + 1 hold column c's sum
+      {
+        float v[kTcN];
+        #pragma unroll
+        for (int n = 0; n < kTcN; ++n) v[n] = lacc[n];
+        #pragma unroll
+        for (int h = kTcN / 2, bit = 16; h >= 1; h >>= 1, bit >>= 1) {
+          const bool up = (lane & bit) != 0;
+          #pragma unroll
+          for (int i = 0; i < h; ++i) {
+            const float send = up ? v[i] : v[i + h];
+            const float keep = up ? v[i + h] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+          }
+        }
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+        const int col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+        if ((lane & 1) == 0) ered[warp * kTcN + col] = v[0];
+      }
+      float o[kTcN];
+      tmem_ld16(tO, o);
+      tc_fence_before();
+      if (!gsync()) { ok = false; break; }
+      // lane n: row n's sum, its reciprocal and (one warp) its lse
+      float l_n = 0.f;
+      if (lane < kTcN) l_n = ered[lane] + ered[kTcN + lane] + ered[2 * kTcN + lane] + ered[3 * kTcN + lane];
+      const float inv_n = l_n > 0.f ? __fdividef(1.f, kTcPScale * l_n) : 0.f;
+      if (warp == 0 && lane < p.GT) {
+        float mr = mref[0];
+        #pragma unroll
+        for (int n = 1; n < kTcN; ++n) mr = lane == n ? mref[n] : mr;
+        float* dst_lse = (d.slot < 0 ? p.lse : p.part_lse) + row_n;
+        *dst_lse = l_n > 0.f ? (mr + __log2f(l_n)) * LN2 : -INFINITY;
+      }
+      const int dd = key;  // head dim
+      float* base_out = d.slot < 0 ? p.out : p.part_o;
+      #pragma unroll
+      for (int n = 0; n < kTcN; ++n) {
+        if (n >= p.GT) break;
+        const int64_t row = __shfl_sync(0xffffffffu, row_n, n);
+        const float inv = __shfl_sync(0xffffffffu, inv_n, n);
+        base_out[row * kTcD + dd] = o[n] * inv;
+      }
+      ++ut;
+      d = dnext;
+    }
+    if (!ok) *abort = 1;
+  }
+
+  // ---- teardown: every role has left its loop; the MMA warp has seen its last MMA complete
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kTcTmemCols) : "memory");
+}
+
+}  // namespace decattn
+
+namespace decattn {
+
+bool split_tc_supported(int kv_dtype, int D, int GT) {
+  return kv_dtype == DECATTN_KV_FP8E4M3 && D == kTcD && GT >= 1 && GT <= kTcN;
+}
+
+cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st) {
+  const int smem = TcSmem::ALLOC;
+  if (!ensure_smem_attr((const void*)split_tc_kernel, smem)) return cudaErrorInvalidValue;
+  // one wave: as many CTAs as are resident at once (2 per SM: the layout is sized for it),
+  // each taking every grid-th bin
+  static int sm_count[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidValue;
+  if (sm_count[dev] == 0 && cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  const int resident = 2 * sm_count[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(min(p.n_bins, resident));
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlaps our prologue with the planner
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, split_tc_kernel, p, tmK, tmV);
+}
+
+}  // namespace decattn
