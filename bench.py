@@ -73,6 +73,8 @@ def parse():
     ap.add_argument("--sparse", type=float, default=0.0,
                     help="block-sparse decode: keep each (request, KV head, tile) with this probability "
                          "(the tile with each request's newest token always kept); 0 = dense")
+    ap.add_argument("--bins", type=int, default=0,
+                    help="bins of the plan (0: the library's default, SM count x 4)")
     ap.add_argument("--append", action="store_true",
                     help="each step starts with the fused pre-processing kernel (rotary embedding of the "
                          "step's new q / k rows and their KV append), and the decode reads the rotated q")
@@ -95,6 +97,14 @@ def kernel_source_hash() -> str:
     for f in ("split.cu", "split_tc.cu", "walk.cuh", "common.cuh"):
         h.update(open(os.path.join(ROOT, "paged_kv_decode_29_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
+
+
+def split_kernel_name(pr) -> str:
+    """The split kernel the library runs for this workload: FP8 KV with head_dim 128 and
+    G*T <= 16 runs on the tcgen05 kernel, everything else on the warp-MMA kernel."""
+    if pr.kv_dtype == "fp8e4m3" and pr.head_dim == 128 and pr.group * pr.q_tokens <= 16:
+        return "split_tc_kernel"
+    return "split_kernel"
 
 
 def ncu_traffic(config: str, tile_len: int):
@@ -294,8 +304,9 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
     def make_plan(buf=None, stream=None):
         if mask_dev is not None:
             return da.plan_sparse(lens, mask_dev, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=buf,
-                                  stream=stream)
-        return da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=buf, stream=stream)
+                                  stream=stream, n_bins=args.bins)
+        return da.plan(lens, pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total, buf=buf, stream=stream,
+                       n_bins=args.bins)
 
     pl = make_plan()
     shape = da.make_shape(q, k, tab, da.kv_dtype_of(k), pr.sm_scale)
@@ -504,7 +515,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
         "hbm_gbs_step": round(step_gbs, 1), "pct_of_8tbs_step": round(100 * step_gbs / NOMINAL_HBM_GBS, 2),
         "hbm_gbs_split": round(split_gbs, 1), "pct_of_8tbs_split": round(100 * split_gbs / NOMINAL_HBM_GBS, 2),
         "hbm_gbs_split_combine": round(sc_gbs, 1), "frac_split_combine": round(sc_gbs / peak, 4),
-        "roofline": {"bound": "hbm", "kernel": "split_kernel", "achieved": round(split_gbs, 1),
+        "roofline": {"bound": "hbm", "kernel": split_kernel_name(pr), "achieved": round(split_gbs, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(split_gbs / peak, 4),
                      "traffic": None if traffic is None else int(traffic)},
