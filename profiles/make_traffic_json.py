@@ -2,7 +2,8 @@
 workload, scaled from an ncu capture of a smaller case of the same workload (its first requests)
 by the ratio of algorithmic bytes. Reads measured within 0.05% of the algorithmic bytes on every
 captured case, so traffic grows in proportion. The figures below are the captured ncu values
-(`dram__bytes_read.sum`, `dram__bytes_write.sum`) of one split-kernel launch of each smaller case.
+(`dram__bytes_read.sum`, `dram__bytes_write.sum`) of one split-kernel launch of each smaller case (the split kernel that runs for the workload: split_tc_kernel for fp8_spec,
+split_kernel for the others).
 Run from the repository root after the capture: python profiles/make_traffic_json.py"""
 import hashlib
 import json
@@ -17,10 +18,10 @@ import workloads as W  # noqa: E402
 
 # workload -> (requests captured, dram read bytes, dram write bytes) of the captured launch
 CAPTURED = {
-    "uniform": (8, 134361088, 3281408),
-    "mixed": (16, 1039147264, 17551104),
-    "fp8_spec": (4, 167213568, 5203200),
-    "long_b4": (1, 536967936, 5665536),
+    "uniform": (8, 134361600, 3171584),
+    "mixed": (16, 1039219968, 18049280),
+    "fp8_spec": (4, 167430400, 7366912),
+    "long_b4": (1, 536984832, 6270976),
 }
 
 
