@@ -73,6 +73,9 @@ def parse():
     ap.add_argument("--sparse", type=float, default=0.0,
                     help="block-sparse decode: keep each (request, KV head, tile) with this probability "
                          "(the tile with each request's newest token always kept); 0 = dense")
+    ap.add_argument("--mma8", action="store_true",
+                    help="FP8 workloads: both products on E4M3 tensor cores (q and P rounded to E4M3; "
+                         "its own tolerance)")
     ap.add_argument("--bins", type=int, default=0,
                     help="bins of the plan (0: the library's default, SM count x 4)")
     ap.add_argument("--append", action="store_true",
@@ -321,7 +324,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
         # evicts the KV and leaves only clean lines in L2
         torch.sum(flush, dim=0, out=flush_sink)
     pbuf = pl.buf
-    kw = dict(kv_scales=sc, sm_scale=pr.sm_scale, workspace=ws, out=out, lse=lse)
+    kw = dict(kv_scales=sc, sm_scale=pr.sm_scale, workspace=ws, out=out, lse=lse, mma8=args.mma8)
     q_dec = q
     if args.append:
         # the step's new rows; every step rewrites the same slots with the same values
@@ -503,9 +506,10 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
     line = {
         "metric": METRIC, "value": round(step_m, 3), "unit": "us/step", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_m / 1e3, 6), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3->f16" if pr.kv_dtype == "fp8e4m3" else "bf16",
+        "scaling": "weak", "vs_baseline": None, "dtype": ("fp8e4m3 (q, P in e4m3)" if args.mma8 else "fp8e4m3->f16") if pr.kv_dtype == "fp8e4m3" else "bf16",
         "data": "synthetic",
         "config": {"workload": pr.name, **workload_desc(pr), "n_bins": pl.n_bins,
+                   **({"products": "e4m3 tensor cores (q and P rounded to e4m3)"} if args.mma8 else {}),
                    "l2": "flushed before every step (a reduction reading 256 MiB); KV bytes exceed the 126 MB L2",
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "breakdown_note": "plan/split/combine: a second pass of the same steps with events between the kernels",

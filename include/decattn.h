@@ -68,7 +68,22 @@ typedef enum {
   DECATTN_ECAPACITY = -8 /* device: the tiles of seq_lens exceed the plan's capacity */
 } decattn_status;
 
-typedef enum { DECATTN_KV_BF16 = 0, DECATTN_KV_FP8E4M3 = 1 } decattn_kv_dtype;
+/* KV element type of the pools, and how the products are formed:
+ *   DECATTN_KV_BF16          bf16 pages;
+ *   DECATTN_KV_FP8E4M3       OCP E4M3 pages with fp32 per-(page, KV head) scales; q keeps bf16
+ *                            precision (two E4M3 parts) and P enters P V as f16: the result is
+ *                            checked against the fp64 oracle on the dequantised pages (out 2e-3,
+ *                            lse 1e-4);
+ *   DECATTN_KV_FP8E4M3_MMA8  the same pages and scales, with both products on E4M3 tensor cores
+ *                            ("HPC-Ops ...", "How the kernels are organized around specific
+ *                            workload shapes": FP8 attention with per-tile scaling): q rounded to
+ *                            one E4M3 part per row (power-of-two row scale 2^E, E = 7 -
+ *                            floor(log2 max|q_row|)), and P rounded to E4M3 after scaling by
+ *                            (V page scale) * C, C a power of two per 128-key chunk. Its own
+ *                            tolerance: the oracle runs on the rounded q, and P's rounding is
+ *                            bounded per row (see the tests). head_dim 128 and G*T <= 16 only
+ *                            (DECATTN_ENOTSUP otherwise). */
+typedef enum { DECATTN_KV_BF16 = 0, DECATTN_KV_FP8E4M3 = 1, DECATTN_KV_FP8E4M3_MMA8 = 2 } decattn_kv_dtype;
 
 /* Host-side handle of a plan. dec_attn_plan fills it; dec_attn_run reads it. The
  * work list itself lives in the caller's device buffer `buf`. */

@@ -15,7 +15,8 @@ Everything is computed in fp64 by ``oracle.c``:
   Tencent's CUDA Kernel Library for LLM Inference Hot Paths", "How the kernels
   are organized around specific workload shapes"), as a literal sequential
   greedy over the tiles sorted by cost.
-* ``e4m3_value``: the OCP E4M3 "fn" code table.
+* ``e4m3_value``: the OCP E4M3 "fn" code table; ``e4m3_round`` / ``round_q_e4m3_rows``: the q
+  rounding of the FP8-products mode, from the format's definition (nearest value, ties to even).
 
 Parity pins for each function live in ``tests/test_oracle_pins.py``.
 """
@@ -192,6 +193,40 @@ def e4m3_value(code: int) -> float:
 
 def e4m3_table() -> np.ndarray:
     return np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+# ---- FP8 products mode: q rounded to one E4M3 part per row
+
+def e4m3_round(x) -> np.ndarray:
+    """The E4M3 value nearest to each x (fp64 array), ties to the even code, saturating at +-448:
+    round-to-nearest-even onto the finite set of the OCP E4M3 "fn" format."""
+    x = np.asarray(x, dtype=np.float64)
+    tab = e4m3_table()
+    codes = np.arange(128)  # non-negative codes 0x00 .. 0x7F (0x7F is NaN)
+    vals = tab[:127]        # 0 .. 448, increasing with the code
+    a = np.minimum(np.abs(x), 448.0)
+    hi = np.clip(np.searchsorted(vals, a, side="left"), 0, 126)
+    lo = np.clip(hi - 1, 0, 126)
+    dlo, dhi = a - vals[lo], vals[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (codes[hi] % 2 == 0))
+    r = np.where(pick_hi, vals[hi], vals[lo])
+    return np.copysign(r, x)
+
+
+def round_q_e4m3_rows(q_bits) -> np.ndarray:
+    """q of the FP8-products mode (KV_FP8E4M3_MMA8): each query row (the last axis) is scaled by
+    2^E, E = 7 - floor(log2 max|q_row|) (E = 7 for a zero row, clamped to [-100, 100]), rounded to
+    the nearest E4M3 value (ties to even) and scaled back. Input and output: bf16 bit patterns
+    (every such value is a bf16 number). The oracle then runs on these rows."""
+    qb = np.asarray(q_bits, dtype=np.uint16)
+    v = (qb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    amax = np.max(np.abs(v), axis=-1, keepdims=True)
+    _, e = np.frexp(np.where(amax > 0, amax, 1.0))  # amax = m 2^e, m in [0.5, 1)
+    E = np.where(amax > 0, 7 - (e - 1), 7)
+    E = np.clip(E, -100, 100)
+    r = e4m3_round(np.ldexp(v, E))
+    out = np.ldexp(r, -E)
+    return bf16_bits(out)
 
 
 # ---- fused pre-processing of a decode step: rotary embedding + KV append (oracle.c)

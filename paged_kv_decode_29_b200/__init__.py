@@ -25,7 +25,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdecattn.so")
 
 OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1, -2, -3, -4, -5, -6, -7, -8
-KV_BF16, KV_FP8E4M3 = 0, 1
+KV_BF16, KV_FP8E4M3, KV_FP8E4M3_MMA8 = 0, 1, 2
 API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
        "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_plan_sparse_bytes",
@@ -215,15 +215,21 @@ def workspace_bytes(shape: ShapeT, pl: Plan) -> int:
 def run(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_table: torch.Tensor,
         seq_lens: torch.Tensor, pl: Plan, *, kv_scales: torch.Tensor | None = None, sm_scale: float = 0.0,
         workspace: torch.Tensor | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
-        stream=None, stage: str = "run"):
+        stream=None, stage: str = "run", mma8: bool = False):
     """Enqueues split + combine on ``stream``; returns (out fp32 [B][T][Hq][d], lse fp32 [B][T][Hq]).
 
     q: bf16 [B][T][Hq][d]; k_pages / v_pages: [num_pages][Hkv][P][d] bf16, or uint8 / float8_e4m3fn
     E4M3 codes with ``kv_scales`` fp32 [2][num_pages][Hkv]; page_table: int32 [B][max_pages_per_seq];
     seq_lens: int32 [B] (the values the plan was made from). ``stage``: "run" (split + combine), or
-    "split" / "combine" alone (the combine reads the partials the split left in ``workspace``)."""
+    "split" / "combine" alone (the combine reads the partials the split left in ``workspace``).
+    ``mma8``: E4M3 pages with both products on E4M3 tensor cores (KV_FP8E4M3_MMA8: q and P rounded
+    to E4M3; head_dim 128, G*T <= 16)."""
     lib = load_library()
     kvt = kv_dtype_of(k_pages)
+    if mma8:
+        if kvt != KV_FP8E4M3:
+            raise ValueError("mma8 needs E4M3 pages")
+        kvt = KV_FP8E4M3_MMA8
     shape = make_shape(q, k_pages, page_table, kvt, sm_scale)
     B, T, Hq, d = q.shape
     if out is None:

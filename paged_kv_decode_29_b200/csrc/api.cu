@@ -135,7 +135,7 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
   if (!workspace) return DECATTN_EINVAL;
   if (s.batch == 0) return DECATTN_OK;
   if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !out || !lse) return DECATTN_EINVAL;
-  if (s.kv_dtype == DECATTN_KV_FP8E4M3 && !kv_scales) return DECATTN_EINVAL;
+  if (s.kv_dtype != DECATTN_KV_BF16 && !kv_scales) return DECATTN_EINVAL;
   if (s.num_pages <= 0 || s.max_pages_per_seq <= 0) return DECATTN_EINVAL;
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out) || !aligned16(workspace) ||
       !aligned16(plan->buf))

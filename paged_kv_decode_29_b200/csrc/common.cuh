@@ -409,7 +409,7 @@ cudaError_t launch_split(const SplitParams& p, const CUtensorMap& tmK, const CUt
                          int D, cudaStream_t st);                 // split.cu
 int split_ctas_per_sm();                                          // split.cu
 bool split_tc_supported(int kv_dtype, int D, int GT);             // split_tc.cu
-cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int kv_dtype,
                             cudaStream_t st);                     // split_tc.cu
 cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st);  // combine.cu
 

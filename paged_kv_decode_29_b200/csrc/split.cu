@@ -695,6 +695,7 @@ static cudaError_t launch_gt(const SplitParams& p, const CUtensorMap& tmK, const
 }
 
 bool split_supported(int kv_dtype, int D, int GT) {
+  if (kv_dtype == DECATTN_KV_FP8E4M3_MMA8) return split_tc_supported(kv_dtype, D, GT);  // tcgen05 kernel only
   return GT >= 1 && GT <= 16 && (D == 64 || D == 128) &&
          (kv_dtype == DECATTN_KV_BF16 || kv_dtype == DECATTN_KV_FP8E4M3);
 }
@@ -703,7 +704,8 @@ cudaError_t launch_split(const SplitParams& p, const CUtensorMap& tmK, const CUt
                          cudaStream_t st) {
   if (!split_supported(kv_dtype, D, p.GT)) return cudaErrorInvalidValue;
   if (kv_dtype == DECATTN_KV_BF16) return D == 128 ? launch_gt<0, 128>(p, tmK, tmV, st) : launch_gt<0, 64>(p, tmK, tmV, st);
-  if (split_tc_supported(kv_dtype, D, p.GT)) return launch_split_tc(p, tmK, tmV, st);  // tcgen05 path
+  if (split_tc_supported(kv_dtype, D, p.GT)) return launch_split_tc(p, tmK, tmV, kv_dtype, st);  // tcgen05 path
+  if (kv_dtype == DECATTN_KV_FP8E4M3_MMA8) return cudaErrorInvalidValue;  // the tcgen05 kernel only
   return D == 128 ? launch_gt<1, 128>(p, tmK, tmV, st) : launch_gt<1, 64>(p, tmK, tmV, st);
 }
 

@@ -41,50 +41,54 @@ constexpr int kTcD = 128;          // head_dim
 constexpr int kTcN = 16;           // MMA N: query rows of the KV group, zero-padded
 constexpr int kTcChunk = 128;      // keys per chunk: the M of S^T and the contraction of O^T
 constexpr int kTcBlk = kTcChunk / 16;  // 16-key blocks (one TMA box each) per chunk
-constexpr int kTcStages = 2;       // chunk stages of the K/V ring
 constexpr int kTcThreads = 192;
 constexpr int kTcTau = 6;          // P <= 2^kTcTau
-constexpr float kTcPScale = 64.f;  // P enters the MMA as P * (V page scale) * kTcPScale
+constexpr float kTcPScale = 64.f;  // f16 P^T: P * (V page scale) * kTcPScale
 constexpr int kTcTmemCols = 64;    // S^T double buffer (2 x 16 columns), O^T (16), spare (power of 2)
 
-// Shared-memory layout (offsets from a 1024-byte aligned base).
+// Shared-memory layout (offsets from a 1024-byte aligned base). Q8: both products on E4M3 (no
+// f16 V^T buffer, which pays for a third ring stage; P^T in E4M3).
+template <bool Q8>
 struct TcSmem {
+  static constexpr int STAGES = Q8 ? 3 : 2;                  // chunk stages of the K/V ring
   static constexpr int KCH = kTcChunk * kTcD;                // bytes of one K (or V) chunk: 16 KB
   static constexpr int QB = 2 * kTcN * kTcD;                 // q hi [16][128] then lo, E4M3
+  static constexpr int PB = kTcChunk * kTcN * (Q8 ? 1 : 2);  // P^T: E4M3 or f16
   static constexpr int OFF_K = 0;                            // [stage][128 keys][128 B], 128-B swizzle
-  static constexpr int OFF_V = OFF_K + kTcStages * KCH;
-  static constexpr int OFF_V16 = OFF_V + kTcStages * KCH;    // f16 V^T, MN-major interleaved core matrices
-  static constexpr int OFF_P16 = OFF_V16 + 2 * KCH;          // f16 P^T, MN-major interleaved
-  static constexpr int OFF_QB = OFF_P16 + kTcChunk * kTcN * 2;  // [tile parity] q hi / lo, 128-B swizzle
+  static constexpr int OFF_V = OFF_K + STAGES * KCH;
+  static constexpr int OFF_V16 = OFF_V + STAGES * KCH;       // f16 V^T, MN-major interleaved core matrices
+  static constexpr int OFF_P = OFF_V16 + (Q8 ? 0 : 2 * KCH); // P^T, MN-major interleaved
+  static constexpr int OFF_QB = OFF_P + PB;                  // [tile parity] q hi / lo, 128-B swizzle
   static constexpr int OFF_SC = OFF_QB + 2 * QB;             // per stage: 8 K scales, 8 V scales
-  static constexpr int OFF_QCS = OFF_SC + kTcStages * 2 * kTcBlk * 4;  // [tile parity][16]: 2^-E of q rows
+  static constexpr int OFF_QCS = OFF_SC + STAGES * 2 * kTcBlk * 4;  // [tile parity][16]: 2^-E of q rows
   static constexpr int OFF_FLG = OFF_QCS + 2 * kTcN * 4;     // [2][4] per-warp "passes the reference" flags
   static constexpr int OFF_RED = OFF_FLG + 2 * 4 * 4;        // [2][4][16] chunk maxima per warp
-  static constexpr int OFF_ERED = OFF_RED + 2 * 4 * kTcN * 4;  // [4][16] row-sum partials
-  static constexpr int OFF_UNIT = OFF_ERED + 4 * kTcN * 4;   // Unit x 2
+  static constexpr int OFF_ERED = OFF_RED + 2 * 4 * kTcN * 4;  // [2][4][16] row-sum partials (Q8: exact, rounded)
+  static constexpr int OFF_UNIT = OFF_ERED + 2 * 4 * kTcN * 4;  // Unit x 2
   static constexpr int OFF_BAR = OFF_UNIT + 2 * (int)sizeof(Unit);
-  static constexpr int NBAR = 17;
+  static constexpr int NBAR = 19;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;        // tensor-memory base, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;                 // slack to align the base to 1024
+  static_assert(OFF_QB % 1024 == 0 && QB % 1024 == 0, "swizzled q operands need 1024-byte bases");
+  static_assert(OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
+  static_assert(2 * (ALLOC + 1024) <= 228 * 1024, "two CTAs per SM");
 };
-static_assert(TcSmem::OFF_QB % 1024 == 0 && TcSmem::QB % 1024 == 0, "swizzled q operands need 1024-byte bases");
-static_assert(TcSmem::OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
-static_assert(2 * (TcSmem::ALLOC + 1024) <= 228 * 1024, "two CTAs per SM");
 
 // Barrier slots.
 enum TcBar {
-  kKvFull = 0,   // [2] producer -> MMA, softmax: K, V and scales of a chunk landed
-  kKvEmpty = 2,  // [2] MMA commit (K read) + 4 softmax warps (V widened) -> producer
-  kSFull = 4,    // [2] MMA commit -> softmax: S^T of a chunk is in tensor memory
-  kSFree = 6,    // [2] 4 softmax warps -> MMA: that S^T buffer has been read
-  kPReady = 8,   // 4 softmax warps -> MMA: P^T and V^T (f16) written, O^T rescaled if needed
-  kPvDone = 9,   // MMA commit -> softmax: O^T += V^T P^T of a chunk complete
-  kUFull = 10,   // [2] producer -> MMA, softmax: tile descriptor written
-  kUEmpty = 12,  // [2] MMA + 4 softmax warps -> producer: tile descriptor read
-  kQReady = 14,  // 4 softmax warps -> MMA: q hi / lo of the next tile written
-  kGroup = 15,   // 4 softmax warps: the group's own barrier (bounded, unlike bar.sync)
-  kFin = 16,     // MMA commit -> MMA: every tensor-core operation of the CTA complete
+  kKvFull = 0,   // [stages] producer -> MMA, softmax: K, V and scales of a chunk landed
+  kKvEmpty = 3,  // [stages] the stage may be refilled: MMA commit (K read) + 4 softmax warps (V
+                 //          widened); Q8: the MMA commit after the chunk's P V (V read in place)
+  kSFull = 6,    // [2] MMA commit -> softmax: S^T of a chunk is in tensor memory
+  kSFree = 8,    // [2] 4 softmax warps -> MMA: that S^T buffer has been read
+  kPReady = 10,  // 4 softmax warps -> MMA: P^T (and the f16 V^T) written, O^T rescaled if needed
+  kPvDone = 11,  // MMA commit -> softmax: O^T += V^T P^T of a chunk complete
+  kUFull = 12,   // [2] producer -> MMA, softmax: tile descriptor written
+  kUEmpty = 14,  // [2] MMA + 4 softmax warps -> producer: tile descriptor read
+  kQReady = 16,  // 4 softmax warps -> MMA: q hi / lo of the next tile written
+  kGroup = 17,   // 4 softmax warps: the group's own barrier (bounded, unlike bar.sync)
+  kFin = 18,     // MMA commit -> MMA: every tensor-core operation of the CTA complete
 };
 // ------------------------------------------------------------------ tcgen05 helpers
 // Shared-memory matrix descriptor: start address, leading / stride byte offsets (16-byte
@@ -253,9 +257,11 @@ __device__ __forceinline__ void tc_store_q(const uint4 (&x)[2], uint8_t* qb, flo
   if (seg == 0) qcs[r] = __int_as_float((127 - E) << 23);
 }
 
+template <bool Q8>
 __global__ void __launch_bounds__(kTcThreads, 2)
 split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
-  using L = TcSmem;
+  using L = TcSmem<Q8>;
+  constexpr int kTcStages = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
@@ -272,7 +278,9 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       mbar_init(&bar[kKvFull + s], 1);
-      mbar_init(&bar[kKvEmpty + s], 1 + 4);
+      mbar_init(&bar[kKvEmpty + s], Q8 ? 1 : 1 + 4);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[kSFull + s], 1);
       mbar_init(&bar[kSFree + s], 4);
       mbar_init(&bar[kUFull + s], 1);
@@ -449,20 +457,34 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       int64_t g = 0;  // chunks issued so far
       int ut = 0;     // tiles started so far
       bool ok = true;
-      // O^T (+)= V^T P^T over the chunk's 128 keys, 16 per instruction. A tile's first chunk
-      // overwrites O^T: the softmax group signals that chunk's P only after it has read the
-      // previous tile's O^T in its epilogue.
       // descriptors, built once: the start address is the low 14 bits (16-byte units), so a
-      // k-step adds to the base descriptor
-      const uint64_t dV = umma_desc(base + L::OFF_V16, 128, 2048, 0), dP = umma_desc(base + L::OFF_P16, 128, 2048, 0);
+      // stage or a k-step adds to the base descriptor
+      const uint64_t dV = umma_desc(base + L::OFF_V16, 128, 2048, 0), dP = umma_desc(base + L::OFF_P, 128, 2048, 0);
       const uint64_t dK0 = umma_desc(base + L::OFF_K, 16, 1024, 2), dQ0 = umma_desc(base + L::OFF_QB, 16, 1024, 2);
+      // Q8: A = V^T as staged (E4M3, MN-major: head dims contiguous, 128-byte swizzle; 8-key groups
+      // 1024 B apart), B = P^T (E4M3, MN-major interleaved: key j at 16 j, 8-key groups 128 B
+      // apart). Both leading offsets equal the stride offsets, so either reading stays in bounds.
+      const uint64_t dV8 = umma_desc(base + L::OFF_V, 1024, 1024, 2), dP8 = umma_desc(base + L::OFF_P, 128, 128, 0);
+      constexpr uint32_t idO8 = umma_idesc(0, 0, 1, 1, kTcD, kTcN);     // E4M3 x E4M3, both MN-major
+      // O^T (+)= V^T P^T over chunk gg's 128 keys. A tile's first chunk overwrites O^T: the
+      // softmax group signals that chunk's P only after it has read the previous tile's O^T.
       auto pv = [&](int64_t gg, bool first_of_tile, uint32_t tO) -> bool {
         if (!tc_wait(&bar[kPReady], (uint32_t)(gg & 1), p.status, abort)) return false;
         tc_fence_after();
-        #pragma unroll
-        for (int k = 0; k < kTcChunk / 16; ++k)
-          umma_f16(tO, dV + (uint64_t)(16 * k), dP + (uint64_t)(16 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
-        umma_commit(&bar[kPvDone]);
+        if constexpr (Q8) {
+          const int sg = (int)(gg % kTcStages);
+          const uint64_t a0 = dV8 + (uint64_t)((sg * L::KCH) >> 4);
+          #pragma unroll
+          for (int k = 0; k < kTcChunk / 32; ++k)  // 32 keys per instruction: 4 KB of V, 512 B of P
+            umma_f8(tO, a0 + (uint64_t)(256 * k), dP8 + (uint64_t)(32 * k), idO8, (first_of_tile && k == 0) ? 0u : 1u);
+          umma_commit(&bar[kPvDone]);
+          umma_commit(&bar[kKvEmpty + sg]);  // K and V of the stage have both been read
+        } else {
+          #pragma unroll
+          for (int k = 0; k < kTcChunk / 16; ++k)
+            umma_f16(tO, dV + (uint64_t)(16 * k), dP + (uint64_t)(16 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
+          umma_commit(&bar[kPvDone]);
+        }
         return true;
       };
       for (;;) {
@@ -483,16 +505,18 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
             break;
           }
           tc_fence_after();
-          // S^T = K (q hi)^T + K (q lo)^T: four 32-byte k-steps of the 128-byte swizzled rows
+          // S^T = K (q hi)^T + K (q lo)^T (Q8: q hi only): four 32-byte k-steps of the 128-byte
+          // swizzled rows
           const uint64_t dK = dK0 + (uint64_t)((st * L::KCH) >> 4);
           #pragma unroll
           for (int kk = 0; kk < kTcD / 32; ++kk) {
             const uint64_t a = dK + (uint64_t)(2 * kk);
             umma_f8(tmem + kTcN * sb, a, dQ + (uint64_t)(2 * kk), idS, kk > 0 ? 1u : 0u);
-            umma_f8(tmem + kTcN * sb, a, dQ + (uint64_t)((kTcN * kTcD) >> 4) + (uint64_t)(2 * kk), idS, 1u);
+            if constexpr (!Q8)
+              umma_f8(tmem + kTcN * sb, a, dQ + (uint64_t)((kTcN * kTcD) >> 4) + (uint64_t)(2 * kk), idS, 1u);
           }
           umma_commit(&bar[kSFull + sb]);
-          umma_commit(&bar[kKvEmpty + st]);  // the K half of the stage has been read
+          if constexpr (!Q8) umma_commit(&bar[kKvEmpty + st]);  // the K half of the stage has been read
           if (c > 0 && !pv(g - 1, c == 1, tO)) { ok = false; break; }
         }
         if (!ok) break;
@@ -560,12 +584,15 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
                            : (int64_t)d.slot * p.GT + lane;
       }
       const int causal_base = d.seq_len - p.T;  // query row n sees key j iff j - base <= n / G
-      float mref[kTcN], lacc[kTcN];
+      // row sums of P: lacc (exact), and Q8: lrnd of the weights as rounded for P V
+      float mref[kTcN], lacc[kTcN], lrnd[Q8 ? kTcN : 1];
       #pragma unroll
       for (int n = 0; n < kTcN; ++n) {
         mref[n] = -INFINITY;
         lacc[n] = 0.f;
+        if constexpr (Q8) lrnd[n] = 0.f;
       }
+      float c_ref = 1.f;  // Q8: the power of two that O^T carries
       Unit dnext;
       dnext.b = -1;
       uint4 qx[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
@@ -576,17 +603,18 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           if (!next_desc(dnext)) { ok = false; break; }
           if (dnext.b >= 0) tc_load_q(p, dnext, qx);
         }
-        // ---- V first: it frees the ring stage for the producer as early as possible. The
-        //      previous chunk's P V must have read the f16 buffers.
+        // ---- the chunk's K, V and scales have landed. f16 V^T: widened first (it frees the ring
+        //      stage early; the previous chunk's P V must have read the f16 buffers). Q8: V stays
+        //      in the stage as the E4M3 operand and the MMA warp frees the stage after P V.
         if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort) ||
-            (c > 0 && !tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort))) {
+            (!Q8 && c > 0 && !tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort))) {
           ok = false;
           break;
         }
         const int j = d.tok_begin + c * kTcChunk + key;
         const bool valid = j < d.tok_end;
-        // ---- V row of this key widened to f16 (exact), 8 head dims per 16-byte core-matrix row
-        {
+        if constexpr (!Q8) {
+          // V row of this key widened to f16 (exact), 8 head dims per 16-byte core-matrix row
           const uint8_t* vr = sm + L::OFF_V + st * L::KCH + key * kTcD;
           uint8_t* vd = sm + L::OFF_V16 + (key >> 3) * 128 + (key & 7) * 16;
           #pragma unroll
@@ -604,9 +632,22 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         // this key's page scales, read before the stage (scales included) goes back to the producer
         const int blk = key >> 4;
         const float f = p.qk_scale_log2 * sc[st * 16 + blk];
-        const float vsc = sc[st * 16 + 8 + blk] * kTcPScale;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[kKvEmpty + st]);  // the V half of the stage has been read
+        const float vsc = sc[st * 16 + 8 + blk] * (Q8 ? 1.f : kTcPScale);
+        // Q8: E4M3 P^T = P * (V page scale) * C with C a power of two such that the largest P
+        // (2^kTcTau) times the chunk's largest V scale lands in (224, 448]; the same in every thread
+        float c_chunk = 1.f;
+        if constexpr (Q8) {
+          const float4 a4 = *reinterpret_cast<const float4*>(sc + st * 16 + 8);
+          const float4 b4 = *reinterpret_cast<const float4*>(sc + st * 16 + 12);
+          const float svmax = fmaxf(fmaxf(fmaxf(a4.x, a4.y), fmaxf(a4.z, a4.w)), fmaxf(fmaxf(b4.x, b4.y), fmaxf(b4.z, b4.w)));
+          const float r = 448.f / ((float)(1 << kTcTau) * svmax);
+          // the largest power of two <= r (exponent field only); 1 when no scale is usable
+          c_chunk = (svmax > 0.f && r < 1e30f) ? __int_as_float(__float_as_int(r) & 0x7f800000) : 1.f;
+        }
+        if constexpr (!Q8) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[kKvEmpty + st]);  // the V half of the stage has been read
+        }
         if (!tc_wait(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort)) { ok = false; break; }
         tc_fence_after();
         float s[kTcN];
@@ -666,19 +707,38 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
             cm[4 * q4 + 2] = ordered_float(m.z); cm[4 * q4 + 3] = ordered_float(m.w);
           }
         }
-        if (upd) {
+        // Q8: C may only shrink within a tile (the accumulated O^T carries the tile's C)
+        float c_factor = 1.f;
+        if constexpr (Q8) {
+          if (c == 0) {
+            c_ref = c_chunk;
+          } else if (c_chunk < c_ref) {
+            c_factor = c_chunk / c_ref;  // a power of two: exact
+            c_ref = c_chunk;
+          }
+        }
+        bool pv_waited = false;
+        if (upd || c_factor != 1.f) {
           float alpha[kTcN];
-          bool resc = false;
+          bool resc = c_factor != 1.f;
           #pragma unroll
           for (int n = 0; n < kTcN; ++n) {
-            const float mn = fmaxf(mref[n], cm[n]);
-            alpha[n] = mn == -INFINITY ? 1.f : fast_exp2(mref[n] - mn);
+            float a = 1.f;
+            if (upd) {
+              const float mn = fmaxf(mref[n], cm[n]);
+              a = mn == -INFINITY ? 1.f : fast_exp2(mref[n] - mn);
+              mref[n] = mn;
+              lacc[n] *= a;
+              if constexpr (Q8) lrnd[n] *= a;
+            }
+            alpha[n] = a * c_factor;
             resc |= alpha[n] != 1.f;
-            mref[n] = mn;
-            lacc[n] *= alpha[n];
           }
           if (c > 0 && resc) {
-            // O^T holds chunks 0 .. c-1 of this tile (their P V is done): rescale it in place
+            // O^T holds chunks 0 .. c-1 of this tile (their P V is done; Q8 waits for it here):
+            // rescale it in place
+            if (Q8 && !tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
+            pv_waited = true;
             tc_fence_after();
             float o[kTcN];
             tmem_ld16(tO, o);
@@ -694,12 +754,34 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           pr[n] = fast_exp2(s[n] - (mref[n] == -INFINITY ? 0.f : mref[n]));
           lacc[n] += pr[n];
         }
-        // ---- P^T row of this key: f16 P * (V page scale) * kTcPScale, 16 query rows
-        {
+        // ---- P^T row of this key, 16 query rows: f16 P * (V page scale) * kTcPScale, or Q8:
+        //      E4M3 P * (V page scale) * C once the previous chunk's P V has read the buffer
+        if (Q8 && c > 0 && !pv_waited && !tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) {
+          ok = false;
+          break;
+        }
+        if constexpr (Q8) {
+          // the output is normalised by the weights as rounded, so it stays a convex combination of
+          // V rows (a single visible key reproduces its V row); lse keeps the exact sums
+          const float xs = vsc * c_ref, rxs = 1.f / xs;
+          uint32_t w8[4];
+          #pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = f32x2_to_e4m3x2(pr[4 * i] * xs, pr[4 * i + 1] * xs);
+            const uint32_t hi = f32x2_to_e4m3x2(pr[4 * i + 2] * xs, pr[4 * i + 3] * xs);
+            w8[i] = valid ? (lo | (hi << 16)) : 0u;
+            if (valid) {
+              const float2 a = f16x2_to_float2(e4m3x2_to_f16x2(lo)), b = f16x2_to_float2(e4m3x2_to_f16x2(hi));
+              lrnd[4 * i] += a.x * rxs; lrnd[4 * i + 1] += a.y * rxs;
+              lrnd[4 * i + 2] += b.x * rxs; lrnd[4 * i + 3] += b.y * rxs;
+            }
+          }
+          *reinterpret_cast<uint4*>(sm + L::OFF_P + key * kTcN) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+        } else {
           uint32_t h[8];
           #pragma unroll
           for (int i = 0; i < 8; ++i) h[i] = valid ? pack_f16(pr[2 * i] * vsc, pr[2 * i + 1] * vsc) : 0u;
-          uint8_t* pp = sm + L::OFF_P16 + (key >> 3) * 128 + (key & 7) * 16;
+          uint8_t* pp = sm + L::OFF_P + (key >> 3) * 128 + (key & 7) * 16;
           *reinterpret_cast<uint4*>(pp) = make_uint4(h[0], h[1], h[2], h[3]);
           *reinterpret_cast<uint4*>(pp + 2048) = make_uint4(h[4], h[5], h[6], h[7]);
         }
@@ -716,11 +798,11 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       if (!tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
       tc_fence_after();
       // row sums over the warp's 32 keys by a butterfly reduce-scatter: after the five levels,
-      // lanes 2c and 2c + 1 hold column c's sum
-      {
+      // lanes 2c and 2c + 1 hold column c's sum (Q8: the exact sums, then the rounded ones)
+      auto warp_colsum = [&](const float (&in)[kTcN], float* dst) {
         float v[kTcN];
         #pragma unroll
-        for (int n = 0; n < kTcN; ++n) v[n] = lacc[n];
+        for (int n = 0; n < kTcN; ++n) v[n] = in[n];
         #pragma unroll
         for (int h = kTcN / 2, bit = 16; h >= 1; h >>= 1, bit >>= 1) {
           const bool up = (lane & bit) != 0;
@@ -733,16 +815,22 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         }
         v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
         const int col = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
-        if ((lane & 1) == 0) ered[warp * kTcN + col] = v[0];
-      }
+        if ((lane & 1) == 0) dst[warp * kTcN + col] = v[0];
+      };
+      warp_colsum(lacc, ered);
+      if constexpr (Q8) warp_colsum(lrnd, ered + 4 * kTcN);
       float o[kTcN];
       tmem_ld16(tO, o);
       tc_fence_before();
       if (!gsync()) { ok = false; break; }
-      // lane n: row n's sum, its reciprocal and (one warp) its lse
-      float l_n = 0.f;
-      if (lane < kTcN) l_n = ered[lane] + ered[kTcN + lane] + ered[2 * kTcN + lane] + ered[3 * kTcN + lane];
-      const float inv_n = l_n > 0.f ? __fdividef(1.f, kTcPScale * l_n) : 0.f;
+      // lane n: row n's sums, the reciprocal that normalises O^T and (one warp) its lse
+      float l_n = 0.f, lr_n = 0.f;
+      if (lane < kTcN) {
+        l_n = ered[lane] + ered[kTcN + lane] + ered[2 * kTcN + lane] + ered[3 * kTcN + lane];
+        const float* er = ered + (Q8 ? 4 * kTcN : 0);
+        lr_n = er[lane] + er[kTcN + lane] + er[2 * kTcN + lane] + er[3 * kTcN + lane];
+      }
+      const float inv_n = lr_n > 0.f ? __fdividef(1.f, (Q8 ? c_ref : kTcPScale) * lr_n) : 0.f;
       if (warp == 0 && lane < p.GT) {
         float mr = mref[0];
         #pragma unroll
@@ -778,12 +866,15 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
 namespace decattn {
 
 bool split_tc_supported(int kv_dtype, int D, int GT) {
-  return kv_dtype == DECATTN_KV_FP8E4M3 && D == kTcD && GT >= 1 && GT <= kTcN;
+  return (kv_dtype == DECATTN_KV_FP8E4M3 || kv_dtype == DECATTN_KV_FP8E4M3_MMA8) && D == kTcD && GT >= 1 &&
+         GT <= kTcN;
 }
 
-cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st) {
-  const int smem = TcSmem::ALLOC;
-  if (!ensure_smem_attr((const void*)split_tc_kernel, smem)) return cudaErrorInvalidValue;
+template <bool Q8>
+static cudaError_t launch_tc(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st) {
+  const int smem = TcSmem<Q8>::ALLOC;
+  auto fn = split_tc_kernel<Q8>;
+  if (!ensure_smem_attr((const void*)fn, smem)) return cudaErrorInvalidValue;
   // one wave: as many CTAs as are resident at once (2 per SM: the layout is sized for it),
   // each taking every grid-th bin
   static int sm_count[64] = {};
@@ -791,9 +882,8 @@ cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const 
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidValue;
   if (sm_count[dev] == 0 && cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return cudaErrorInvalidValue;
-  const int resident = 2 * sm_count[dev];
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(min(p.n_bins, resident));
+  cfg.gridDim = dim3(min(p.n_bins, 2 * sm_count[dev]));
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -802,7 +892,12 @@ cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, split_tc_kernel, p, tmK, tmV);
+  return cudaLaunchKernelEx(&cfg, fn, p, tmK, tmV);
+}
+
+cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int kv_dtype,
+                            cudaStream_t st) {
+  return kv_dtype == DECATTN_KV_FP8E4M3_MMA8 ? launch_tc<true>(p, tmK, tmV, st) : launch_tc<false>(p, tmK, tmV, st);
 }
 
 }  // namespace decattn

@@ -1,0 +1,99 @@
+"""FP8-products mode (KV_FP8E4M3_MMA8) on the GPU: E4M3 pages with both products on E4M3 tensor
+cores, q rounded to one E4M3 part per row and P rounded to E4M3 ("HPC-Ops: Tencent's CUDA Kernel
+Library for LLM Inference Hot Paths", "How the kernels are organized around specific workload
+shapes": FP8 attention with per-tile scaling). Judged against the fp64 oracle run on the rounded q
+(oracle.round_q_e4m3_rows), with its own tolerance:
+  * lse within 1e-4 (the scores use the rounded q exactly; P's rounding does not enter lse);
+  * out, per element: P = p * (V page scale) * C is rounded to E4M3, a relative error d_j of at
+    most 2^-4 on each weight in E4M3's normal range; the row sums take the rounded weights, so the
+    output is sum_j w_j (1 + d_j) v_j / sum_j w_j (1 + d_j) and
+    |out - ref| <= (2^-3 / (1 - 2^-4)) * max_j |v_j - ref| over the row's visible keys, plus 1e-3
+    for weights in E4M3's subnormal range (below 2^-6 after scaling);
+  * out, over all elements: RMS error below 4e-3 (independent rounding errors average out; a
+    wrong operand layout gives errors of order |v|).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_decode_29_b200 as da
+import workloads as W
+from tests import _gpu as U
+from tests import _helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+def _problem(lens, *, Hq, Hkv=2, T=1, seed=13, tl=512):
+    return W.make_problem(name="mma8", batch=len(lens), n_q_heads=Hq, n_kv_heads=Hkv, head_dim=128,
+                          seq_lens=lens, page_size=16, q_tokens=T, kv_dtype="fp8e4m3", seed=seed, tile_len=tl)
+
+
+def _run(pr):
+    dev = U.to_device(pr)
+    total = int(pr.seq_lens.astype(np.int64).sum())
+    pl = da.plan(dev["lens"], pr.n_kv_heads, pr.tile_len, max_total_kv_tokens=total)
+    out, lse = da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl, kv_scales=dev["sc"],
+                      sm_scale=pr.sm_scale, mma8=True)
+    return out.cpu().numpy(), lse.cpu().numpy(), da.read_status(pl)
+
+
+def _vdev_rows(pr, rows, ref_o):
+    """max_j |v_j - ref| over the visible keys j of each (b, t, qh) row (and all head dims)."""
+    res = []
+    cache = {}
+    for (b, t, qh), ref in zip(rows, ref_o):
+        if b not in cache:
+            cache[b] = H.dense_kv(pr, b, "v")
+        h = qh // pr.group
+        vis = int(pr.seq_lens[b]) - pr.q_tokens + t + 1
+        res.append(np.abs(cache[b][h][:vis] - ref[None, :]).max() if vis > 0 else 0.0)
+    return np.array(res)
+
+
+def _check(pr, out, lse, ref_o, ref_l, rows, what):
+    both_empty = np.isneginf(lse) & np.isneginf(ref_l)
+    assert np.all(both_empty | (np.abs(lse - ref_l) <= 1e-4)), what
+    bound = 2.0 ** -3 / (1 - 2.0 ** -4) * _vdev_rows(pr, rows, ref_o)[:, None] + 1e-3
+    err = np.abs(out - ref_o)
+    rms = float(np.sqrt(np.mean(err ** 2)))
+    print(f"{what}: max err {err.max():.2e}, rms {rms:.2e}, max err / bound {np.max(err / bound):.3f}")
+    assert np.all(err <= bound), what
+    assert rms < 4e-3, what
+
+
+@pytest.mark.parametrize("G,T", [(1, 1), (4, 1), (8, 1), (16, 1), (4, 4), (2, 3)])
+def test_mma8_matches_oracle_on_rounded_q(G, T):
+    pr = _problem([1, 40, 300, 1000, 2049, 4100], Hq=2 * G, T=T)
+    out, lse, st = _run(pr)
+    assert st == da.OK, da.status_string(st)
+    pr_q = W.Problem(**{**pr.__dict__, "q": oracle.round_q_e4m3_rows(pr.q)})
+    ref_o, ref_l = oracle.decode(pr_q)
+    B, Tn, Hq = lse.shape
+    rows = [(b, t, qh) for b in range(B) for t in range(Tn) for qh in range(Hq)]
+    _check(pr, out.reshape(-1, 128), lse.reshape(-1), ref_o.reshape(-1, 128), ref_l.reshape(-1), rows,
+           f"mma8 G{G} T{T}")
+
+
+def test_mma8_full_size_fp8_spec_sampled_rows():
+    pr = W.make_config("fp8_spec")
+    out, lse, st = _run(pr)
+    assert st == da.OK, da.status_string(st)
+    rng = np.random.default_rng(5)
+    rows = sorted({(int(rng.integers(pr.batch)), int(rng.integers(pr.q_tokens)), int(rng.integers(pr.n_q_heads)))
+                   for _ in range(48)})
+    pr_q = W.Problem(**{**pr.__dict__, "q": oracle.round_q_e4m3_rows(pr.q)})
+    ref_o, ref_l = oracle.decode_rows(pr_q, np.array(rows, dtype=np.int32))
+    r = np.array(rows)
+    _check(pr, out[r[:, 0], r[:, 1], r[:, 2]], lse[r[:, 0], r[:, 1], r[:, 2]], ref_o, ref_l, rows,
+           "mma8 fp8_spec sampled")
+
+
+def test_mma8_needs_head_dim_128():
+    pr = W.make_problem(name="mma8", batch=2, n_q_heads=4, n_kv_heads=2, head_dim=64, seq_lens=[100, 30],
+                        page_size=16, q_tokens=1, kv_dtype="fp8e4m3", seed=3, tile_len=64)
+    dev = U.to_device(pr)
+    pl = da.plan(dev["lens"], 2, 64, max_total_kv_tokens=130)
+    with pytest.raises(da.DecAttnError):
+        da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl, kv_scales=dev["sc"], mma8=True)
