@@ -75,8 +75,8 @@ typedef enum {
  *                            checked against the fp64 oracle on the dequantised pages (out 2e-3,
  *                            lse 1e-4);
  *   DECATTN_KV_FP8E4M3_MMA8  the same pages and scales, with both products on E4M3 tensor cores
- *                            ("HPC-Ops ...", "How the kernels are organized around specific
- *                            workload shapes": FP8 attention with per-tile scaling): q rounded to
+ *                            (the HPC-Ops article at sdftguanye.com, section on fine-grained task
+ *                            scheduling and data rearrangement: an FP8 attention kernel): q rounded to
  *                            one E4M3 part per row (power-of-two row scale 2^E, E = 7 -
  *                            floor(log2 max|q_row|)), and P rounded to E4M3 after scaling by
  *                            (V page scale) * C, C a power of two per 128-key chunk. Its own

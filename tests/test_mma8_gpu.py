@@ -1,7 +1,7 @@
 """FP8-products mode (KV_FP8E4M3_MMA8) on the GPU: E4M3 pages with both products on E4M3 tensor
-cores, q rounded to one E4M3 part per row and P rounded to E4M3 ("HPC-Ops: Tencent's CUDA Kernel
-Library for LLM Inference Hot Paths", "How the kernels are organized around specific workload
-shapes": FP8 attention with per-tile scaling). Judged against the fp64 oracle run on the rounded q
+cores, q rounded to one E4M3 part per row and P rounded to E4M3 (the HPC-Ops article at
+sdftguanye.com, section on fine-grained task scheduling and data rearrangement: an FP8 attention
+kernel). Judged against the fp64 oracle run on the rounded q
 (oracle.round_q_e4m3_rows), with its own tolerance:
   * lse within 1e-4 (the scores use the rounded q exactly; P's rounding does not enter lse);
   * out, per element: P = p * (V page scale) * C is rounded to E4M3, a relative error d_j of at

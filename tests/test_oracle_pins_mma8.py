@@ -1,6 +1,6 @@
-"""CPU pins of the oracle's q rounding for the FP8-products mode (KV_FP8E4M3_MMA8; "HPC-Ops:
-Tencent's CUDA Kernel Library for LLM Inference Hot Paths", "How the kernels are organized around
-specific workload shapes": FP8 attention). Each against something other than the function itself:
+"""CPU pins of the oracle's q rounding for the FP8-products mode (KV_FP8E4M3_MMA8; the HPC-Ops
+article at sdftguanye.com, section on fine-grained task scheduling and data rearrangement: an FP8
+attention kernel). Each against something other than the function itself:
   * e4m3_round against a brute-force nearest search over all finite codes, ties to the even code;
   * the row scaling lands every row's largest magnitude in [128, 256) before rounding, so each
     row keeps E4M3's 4 significant bits on its largest entries;
