@@ -292,6 +292,28 @@ DECATTN_API int dec_attn_append_rope(const dec_attn_shape *shape, const void *q_
                                      float rope_base, void *q_out, void *k_pages, void *v_pages, int32_t *status,
                                      void *stream);
 
+/* Prefill: causal attention of many query rows per request over the paged KV cache (the
+ * prefill side of "PaddlePaddle/HALOps" README, Highlights, GQA attention item: variable-length
+ * prefill and paged-KV decode over a BF16 KV cache, GQA). The shape's q_tokens = T query rows of
+ * request b are its last T positions, already in the pages: row t attends to keys
+ * 0 .. seq_lens[b] - T + t (the decode's bottom-right causal rule; rows before position 0 see
+ * nothing and get out = 0, lse = -inf). Output as dec_attn_run (out fp32 [B][T][Hq][128], lse
+ * natural log [B][T][Hq]); no plan and no workspace. Runs on tcgen05 tensor cores: one CTA per
+ * (request, q head, 128 query rows), 128-key blocks of K and V by TMA.
+ *   shape       batch, n_q_heads, n_kv_heads, head_dim (128), q_tokens (T >= 1), page_size (a
+ *               multiple of 16), num_pages, max_pages_per_seq, kv_dtype (DECATTN_KV_BF16),
+ *               sm_scale (0: 1/sqrt(head_dim));
+ *   q           device bf16 [B][T][Hq][128], 16-byte aligned;
+ *   k_pages, v_pages, page_table, seq_lens   as dec_attn_run;
+ *   out, lse    device fp32 outputs (out 16-byte aligned);
+ *   status      optional device int32 (may be NULL): DECATTN_EDEVICE for a page id outside the
+ *               pool or a negative length, DECATTN_ETIMEOUT if a pipeline wait gave up.
+ * Returns DECATTN_ENOTSUP for other dtypes, head dims or page sizes, DECATTN_EINVAL /
+ * DECATTN_EALIGN for bad arguments (nothing is launched), DECATTN_ECUDA if the launch fails. */
+DECATTN_API int dec_attn_prefill(const dec_attn_shape *shape, const void *q, const void *k_pages, const void *v_pages,
+                                 const int32_t *page_table, const int32_t *seq_lens, float *out, float *lse,
+                                 int32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

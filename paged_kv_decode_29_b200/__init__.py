@@ -28,7 +28,7 @@ OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1
 KV_BF16, KV_FP8E4M3, KV_FP8E4M3_MMA8 = 0, 1, 2
 API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
-       "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_plan_sparse_bytes",
+       "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_prefill", "dec_attn_plan_sparse_bytes",
        "dec_attn_plan_sparse")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -92,6 +92,8 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_plan_sparse.argtypes = [vp, vp, i32, i32, i32, i32, i64, i32, vp, sz, C.POINTER(PlanT), vp]
         lib.dec_attn_plan_sparse.restype = i32
         lib.dec_attn_append_rope.restype = i32
+        lib.dec_attn_prefill.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.dec_attn_prefill.restype = i32
         _lib = lib
         return lib
 
@@ -284,6 +286,27 @@ def append_rope(q_new: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, p
     if rc != OK:
         raise DecAttnError(rc, "dec_attn_append_rope")
     return q_out
+
+
+def prefill(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_table: torch.Tensor,
+            seq_lens: torch.Tensor, *, sm_scale: float = 0.0, out: torch.Tensor | None = None,
+            lse: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None):
+    """dec_attn_prefill: causal attention of the T query rows of each request (its last T
+    positions, already in the bf16 pages) over its paged KV; returns (out fp32 [B][T][Hq][128],
+    lse fp32 [B][T][Hq]). ``status``: optional int32 device scalar (DECATTN_EDEVICE /
+    DECATTN_ETIMEOUT)."""
+    lib = load_library()
+    shape = make_shape(q, k_pages, page_table, kv_dtype_of(k_pages), sm_scale)
+    B, T, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, T, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, T, Hq), dtype=torch.float32, device=q.device)
+    rc = lib.dec_attn_prefill(C.byref(shape), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
+                              _ptr(seq_lens), _ptr(out), _ptr(lse), _ptr(status), _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_prefill")
+    return out, lse
 
 
 def read_status(pl: Plan | None = None, workspace: torch.Tensor | None = None, stream=None) -> int:

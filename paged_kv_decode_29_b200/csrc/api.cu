@@ -205,6 +205,45 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
 
 using namespace decattn;
 
+extern "C" int dec_attn_prefill(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* page_table, const int32_t* seq_lens, float* out, float* lse,
+                                int32_t* status, void* stream) {
+  if (!shape) return DECATTN_EINVAL;
+  const dec_attn_shape& s = *shape;
+  if (s.batch < 0 || s.q_tokens <= 0 || s.n_q_heads <= 0 || s.n_kv_heads <= 0 || s.page_size <= 0 ||
+      s.num_pages < 0 || s.max_pages_per_seq < 0 || s.n_q_heads % s.n_kv_heads != 0)
+    return DECATTN_EINVAL;
+  if (s.kv_dtype != DECATTN_KV_BF16 || s.head_dim != 128 || s.page_size % 16 != 0) return DECATTN_ENOTSUP;
+  if (s.batch > 65535 || s.n_q_heads > 65535) return DECATTN_ENOTSUP;
+  if ((int64_t)s.batch * s.q_tokens * s.n_q_heads >= (1ll << 31) ||
+      (int64_t)s.num_pages * s.n_kv_heads * s.page_size >= (1ll << 31))
+    return DECATTN_ENOTSUP;
+  if (s.batch == 0) return DECATTN_OK;
+  if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !out || !lse) return DECATTN_EINVAL;
+  if (s.num_pages <= 0 || s.max_pages_per_seq <= 0) return DECATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out)) return DECATTN_EALIGN;
+  if (((reinterpret_cast<uintptr_t>(page_table) | reinterpret_cast<uintptr_t>(seq_lens) |
+        reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(status)) & 3) != 0)
+    return DECATTN_EALIGN;
+  CUtensorMap tmK, tmV;
+  const int64_t rows = (int64_t)s.num_pages * s.n_kv_heads * s.page_size;
+  if (!make_kv_map(&tmK, k_pages, s.kv_dtype, s.head_dim, rows) ||
+      !make_kv_map(&tmV, v_pages, s.kv_dtype, s.head_dim, rows))
+    return DECATTN_ECUDA;
+  const float scale = s.sm_scale > 0.f ? s.sm_scale : 1.0f / sqrtf((float)s.head_dim);
+  PrefillParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.page_table = page_table;
+  p.seq_lens = seq_lens;
+  p.out = out;
+  p.lse = lse;
+  p.status = status;
+  p.B = s.batch; p.T = s.q_tokens; p.Hq = s.n_q_heads; p.Hkv = s.n_kv_heads; p.G = s.n_q_heads / s.n_kv_heads;
+  p.P = s.page_size; p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
+  p.qk_scale_log2 = scale * 1.4426950408889634f;
+  return launch_prefill(p, tmK, tmV, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DECATTN_OK : DECATTN_ECUDA;
+}
+
 extern "C" int dec_attn_default_bins(int device) { return default_bins(device); }
 
 extern "C" size_t dec_attn_workspace_bytes(const dec_attn_shape* shape, const dec_attn_plan_t* plan) {

@@ -177,6 +177,18 @@ struct SplitParams {
   float qk_scale_log2;      // sm_scale * log2(e)
 };
 
+// Arguments of the prefill kernel (prefill.cu).
+struct PrefillParams {
+  const uint16_t* q;          // bf16 [B][T][Hq][D]
+  const int32_t* page_table;  // [B][mpps]
+  const int32_t* seq_lens;    // [B]
+  float* out;                 // [B][T][Hq][D]
+  float* lse;                 // [B][T][Hq]
+  int32_t* status;            // optional device word
+  int B, T, Hq, Hkv, G, P, num_pages, mpps;
+  float qk_scale_log2;        // sm_scale * log2(e)
+};
+
 // The combine kernel folds the partials of one query row in chunks of this many tiles.
 // A request with n_b tiles gives each of its rows cb_b = ceil(n_b / kCombineChunk) chunks
 // (1 if n_b == 0: the row is zero-filled; 0 if n_b == 1: the split kernel wrote the row).
@@ -412,5 +424,7 @@ bool split_tc_supported(int kv_dtype, int D, int GT);             // split_tc.cu
 cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int kv_dtype,
                             cudaStream_t st);                     // split_tc.cu
 cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st);  // combine.cu
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                           cudaStream_t st);                      // prefill.cu
 
 }  // namespace decattn

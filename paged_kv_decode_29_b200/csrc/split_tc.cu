@@ -33,6 +33,7 @@
 // Every wait is bounded; a wait that gives up sets DECATTN_ETIMEOUT and a CTA-wide abort flag,
 // after which every role leaves its loop and the CTA frees its tensor memory and exits.
 #include "common.cuh"
+#include "tc.cuh"
 #include "walk.cuh"
 
 namespace decattn {
@@ -90,111 +91,6 @@ enum TcBar {
   kGroup = 17,   // 4 softmax warps: the group's own barrier (bounded, unlike bar.sync)
   kFin = 18,     // MMA commit -> MMA: every tensor-core operation of the CTA complete
 };
-// ------------------------------------------------------------------ tcgen05 helpers
-// Shared-memory matrix descriptor: start address, leading / stride byte offsets (16-byte
-// units), version 1, layout type (0: no swizzle, 2: 128-byte swizzle).
-__device__ __forceinline__ uint64_t umma_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
-  return (uint64_t)((addr >> 4) & 0x3fffu) | ((uint64_t)((lbo >> 4) & 0x3fffu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3fffu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
-}
-
-// Instruction descriptor: fp32 accumulator, A / B formats (kind::f8f6f4: 0 = E4M3;
-// kind::f16: 0 = f16), A / B major-ness (0 = K, 1 = MN), N and M.
-__host__ __device__ constexpr uint32_t umma_idesc(uint32_t afmt, uint32_t bfmt, uint32_t amaj, uint32_t bmaj, int M,
-                                                  int N) {
-  return (1u << 4) | (afmt << 7) | (bfmt << 10) | (amaj << 15) | (bmaj << 16) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-// The mbarrier gets one arrival once every tensor-core operation issued so far by this thread
-// has completed.
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-// Generic-proxy shared-memory writes become visible to the tensor core (async proxy).
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// 16 consecutive 32-bit columns of this warp's 32 tensor-memory lanes (lane i -> thread i).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-  #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
-      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
-      : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// Non-blocking test of a phase (no suspend: the pipeline hand-offs here are short and a
-// suspended waiter wakes late).
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// A bounded wait that also gives up at once when another role has aborted the CTA.
-__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort) {
-  if (mbar_test(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    #pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_test(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      set_status(status, DECATTN_ETIMEOUT);
-      *abort = 1;
-      return false;
-    }
-  }
-}
-
-// Float -> integer with the same order (for warp max reductions with redux.sync).
-__device__ __forceinline__ int ordered_int(float f) {
-  const int i = __float_as_int(f);
-  return i >= 0 ? i : i ^ 0x7fffffff;
-}
-__device__ __forceinline__ float ordered_float(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
 
 }  // namespace decattn
 
@@ -275,6 +171,14 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)p.B * p.T * p.Hq;
        i += (int64_t)gridDim.x * blockDim.x)
     p.row_cnt[i] = 0;
+  if constexpr (Q8) {
+    // V is read in place by the MMA, including the rows of a tile's last chunk that no page
+    // fills: they meet P = 0 and must be finite, so the ring starts zeroed (afterwards it only
+    // ever holds codes from the pool). Ordered before the first TMA write and MMA read.
+    for (int i = threadIdx.x; i < 2 * kTcStages * L::KCH / 16; i += kTcThreads)
+      reinterpret_cast<uint4*>(sm + L::OFF_K)[i] = make_uint4(0, 0, 0, 0);
+    fence_async_smem();
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       mbar_init(&bar[kKvFull + s], 1);
@@ -546,10 +450,10 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     auto gsync = [&]() -> bool {
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[kGroup]);
-      return tc_wait(&bar[kGroup], (gn++) & 1u, p.status, abort);
+      return tc_wait_warp(&bar[kGroup], (gn++) & 1u, p.status, abort);
     };
     auto next_desc = [&](Unit& dd) -> bool {
-      if (!tc_wait(&bar[kUFull + us], uph, p.status, abort)) return false;
+      if (!tc_wait_warp(&bar[kUFull + us], uph, p.status, abort)) return false;
       dd = umeta[us];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[kUEmpty + us]);
@@ -606,8 +510,8 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         // ---- the chunk's K, V and scales have landed. f16 V^T: widened first (it frees the ring
         //      stage early; the previous chunk's P V must have read the f16 buffers). Q8: V stays
         //      in the stage as the E4M3 operand and the MMA warp frees the stage after P V.
-        if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort) ||
-            (!Q8 && c > 0 && !tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort))) {
+        if (!tc_wait_warp(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort) ||
+            (!Q8 && c > 0 && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort))) {
           ok = false;
           break;
         }
@@ -637,9 +541,12 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         // (2^kTcTau) times the chunk's largest V scale lands in (224, 448]; the same in every thread
         float c_chunk = 1.f;
         if constexpr (Q8) {
-          const float4 a4 = *reinterpret_cast<const float4*>(sc + st * 16 + 8);
-          const float4 b4 = *reinterpret_cast<const float4*>(sc + st * 16 + 12);
-          const float svmax = fmaxf(fmaxf(fmaxf(a4.x, a4.y), fmaxf(a4.z, a4.w)), fmaxf(fmaxf(b4.x, b4.y), fmaxf(b4.z, b4.w)));
+          // only the blocks the producer filled for this chunk (the other slots hold stale values)
+          const int nblk = min(kTcBlk, (d.tok_end - d.tok_begin - c * kTcChunk + 15) / 16);
+          float svmax = 0.f;
+          #pragma unroll
+          for (int i = 0; i < kTcBlk; ++i)
+            if (i < nblk) svmax = fmaxf(svmax, sc[st * 16 + 8 + i]);
           const float r = 448.f / ((float)(1 << kTcTau) * svmax);
           // the largest power of two <= r (exponent field only); 1 when no scale is usable
           c_chunk = (svmax > 0.f && r < 1e30f) ? __int_as_float(__float_as_int(r) & 0x7f800000) : 1.f;
@@ -648,7 +555,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar[kKvEmpty + st]);  // the V half of the stage has been read
         }
-        if (!tc_wait(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort)) { ok = false; break; }
+        if (!tc_wait_warp(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort)) { ok = false; break; }
         tc_fence_after();
         float s[kTcN];
         tmem_ld16(tmem + lane_off + kTcN * sb, s);
@@ -737,7 +644,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           if (c > 0 && resc) {
             // O^T holds chunks 0 .. c-1 of this tile (their P V is done; Q8 waits for it here):
             // rescale it in place
-            if (Q8 && !tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
+            if (Q8 && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
             pv_waited = true;
             tc_fence_after();
             float o[kTcN];
@@ -756,7 +663,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         }
         // ---- P^T row of this key, 16 query rows: f16 P * (V page scale) * kTcPScale, or Q8:
         //      E4M3 P * (V page scale) * C once the previous chunk's P V has read the buffer
-        if (Q8 && c > 0 && !pv_waited && !tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) {
+        if (Q8 && c > 0 && !pv_waited && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) {
           ok = false;
           break;
         }
@@ -795,7 +702,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       if (dnext.b >= 0 && !publish_q(qx, qp ^ 1)) { ok = false; break; }
 
       // ---- epilogue: row sums over the tile, O^T / l, out or partial
-      if (!tc_wait(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
+      if (!tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
       tc_fence_after();
       // row sums over the warp's 32 keys by a butterfly reduce-scatter: after the five levels,
       // lanes 2c and 2c + 1 hold column c's sum (Q8: the exact sums, then the rounded ones)

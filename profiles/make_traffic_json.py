@@ -45,7 +45,7 @@ def alg_bytes(name, batch=None):
 
 def source_hash():
     h = hashlib.sha256()
-    for f in ("split.cu", "split_tc.cu", "walk.cuh", "common.cuh"):
+    for f in ("split.cu", "split_tc.cu", "walk.cuh", "tc.cuh", "common.cuh"):
         h.update(open(os.path.join(ROOT, "paged_kv_decode_29_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 

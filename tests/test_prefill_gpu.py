@@ -1,0 +1,101 @@
+"""Prefill on the GPU (dec_attn_prefill: the T query rows of each request, its last T positions,
+over its paged bf16 KV with the bottom-right causal rule; "PaddlePaddle/HALOps" README,
+Highlights, GQA attention item: variable-length prefill) against the fp64 oracle, which computes
+the same attention for any number of query rows.
+
+Tolerance, derived from the kernel's arithmetic: scores are exact products of bf16 q and K summed
+in fp32 (lse within 1e-4); P is rounded once to bf16 for P V (relative error at most 2^-9 per
+weight) while the row sums stay in fp32, so out = sum_j w_j (1 + d_j) v_j with |d_j| <= 2^-9 and
+|out - ref| <= 2^-9 * max_j |v_j| over the row's visible keys (plus 1e-5 for fp32 accumulation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_decode_29_b200 as da
+import workloads as W
+from tests import _gpu as U
+from tests import _helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+def _problem(lens, *, T, Hq=4, Hkv=2, P=16, seed=17):
+    return W.make_problem(name="prefill", batch=len(lens), n_q_heads=Hq, n_kv_heads=Hkv, head_dim=128,
+                          seq_lens=lens, page_size=P, q_tokens=T, kv_dtype="bf16", seed=seed, tile_len=max(P, 64))
+
+
+def _run(pr):
+    dev = U.to_device(pr)
+    st = torch.zeros((), dtype=torch.int32, device="cuda")
+    out, lse = da.prefill(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], sm_scale=pr.sm_scale, status=st)
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), lse.cpu().numpy(), int(st.item())
+
+
+def _vmax(pr, rows):
+    cache, res = {}, []
+    for b, t, qh in rows:
+        if b not in cache:
+            cache[b] = H.dense_kv(pr, b, "v")
+        vis = int(pr.seq_lens[b]) - pr.q_tokens + t + 1
+        res.append(np.abs(cache[b][qh // pr.group][:vis]).max() if vis > 0 else 0.0)
+    return np.array(res)
+
+
+def _check(pr, out, lse, ref_o, ref_l, rows, what):
+    both_empty = np.isneginf(lse) & np.isneginf(ref_l)
+    assert np.all(both_empty | (np.abs(lse - ref_l) <= 1e-4)), what
+    err = np.abs(out - ref_o)
+    bound = 2.0 ** -9 * _vmax(pr, rows)[:, None] + 1e-5
+    print(f"{what}: max err {err.max():.2e}, max err / bound {np.max(err / bound):.3f}")
+    assert np.all(err <= bound), what
+
+
+@pytest.mark.parametrize("lens,T,Hq,Hkv,P", [
+    ([300, 700], 200, 4, 2, 16),     # two query blocks, partial last one
+    ([129, 1000], 1, 8, 2, 16),      # one query row (a decode through the prefill path)
+    ([256, 256], 256, 2, 2, 64),     # pure prefill: T = L, two whole blocks
+    ([90, 400, 131], 130, 8, 1, 16), # T > L for one request (its first rows see nothing), G = 8
+    ([513], 385, 4, 4, 32),          # keys and rows not multiples of the block
+])
+def test_prefill_matches_oracle(lens, T, Hq, Hkv, P):
+    pr = _problem(lens, T=T, Hq=Hq, Hkv=Hkv, P=P)
+    out, lse, st = _run(pr)
+    assert st == da.OK, da.status_string(st)
+    ref_o, ref_l = oracle.decode(pr)
+    B = len(lens)
+    rows = [(b, t, qh) for b in range(B) for t in range(T) for qh in range(Hq)]
+    _check(pr, out.reshape(-1, 128), lse.reshape(-1), ref_o.reshape(-1, 128), ref_l.reshape(-1), rows,
+           f"prefill L{lens} T{T} G{Hq // Hkv} P{P}")
+
+
+def test_prefill_full_size_sampled_rows():
+    pr = W.make_config("prefill")
+    out, lse, st = _run(pr)
+    assert st == da.OK, da.status_string(st)
+    rng = np.random.default_rng(9)
+    rows = sorted({(int(rng.integers(pr.batch)), int(rng.integers(pr.q_tokens)), int(rng.integers(pr.n_q_heads)))
+                   for _ in range(40)})
+    ref_o, ref_l = oracle.decode_rows(pr, np.array(rows, dtype=np.int32))
+    r = np.array(rows)
+    _check(pr, out[r[:, 0], r[:, 1], r[:, 2]], lse[r[:, 0], r[:, 1], r[:, 2]], ref_o, ref_l, rows,
+           "prefill full size, sampled rows")
+
+
+def test_prefill_bad_page_id_is_reported():
+    pr = _problem([300, 200], T=100)
+    tab = pr.page_table.copy()
+    tab[1, 3] = pr.num_pages + 5
+    pr2 = W.Problem(**{**pr.__dict__, "page_table": tab})
+    _, _, st = _run(pr2)
+    assert st == da.EDEVICE
+
+
+def test_prefill_rejects_unsupported_shapes():
+    pr = W.make_problem(name="p", batch=1, n_q_heads=2, n_kv_heads=1, head_dim=64, seq_lens=[100], page_size=16,
+                        q_tokens=10, kv_dtype="bf16", seed=1, tile_len=64)
+    dev = U.to_device(pr)
+    with pytest.raises(da.DecAttnError):
+        da.prefill(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"])

@@ -268,6 +268,8 @@ def config_seq_lens(name: str) -> list[int]:
         return [131072] * 4
     if name == "fp8_spec":
         return [int(x) for x in _gen(4, _STREAM_LENS, 0).integers(1024, 32768, size=16, endpoint=True)]
+    if name == "prefill":
+        return [2048] * 4
     raise KeyError(name)
 
 
@@ -286,6 +288,9 @@ CONFIGS = {
                     kv_dtype="bf16", tile_len=1024, seed=3),
     "fp8_spec": dict(batch=16, n_q_heads=32, n_kv_heads=8, head_dim=128, page_size=16, q_tokens=4,
                      kv_dtype="fp8e4m3", tile_len=512, seed=4),
+    # prefill (dec_attn_prefill): 4 prompts of 2048 tokens, every position a query row
+    "prefill": dict(batch=4, n_q_heads=32, n_kv_heads=8, head_dim=128, page_size=16, q_tokens=2048,
+                    kv_dtype="bf16", tile_len=256, seed=6),
 }
 
 
