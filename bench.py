@@ -17,6 +17,9 @@ split kernel and the combine kernel of every step. ``value`` is the mean step ti
 (max over ranks when run under torchrun: the path does not shard, so each rank runs a
 full replica). One JSON line is printed by rank 0.
 
+``--config prefill`` times the causal prefill kernel instead (4 prompts of 2048 tokens; one
+kernel per step, reported against the measured bf16 tensor peak).
+
 ``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample of the same
 workload (rows chosen at random, time scaled to the whole step).
 """
@@ -44,8 +47,10 @@ if ROOT not in sys.path:
 import workloads as W  # noqa: E402
 
 METRIC = "decode-attention µs/step and achieved HBM GB/s as % of B200 peak, 1 GPU"
+PREFILL_METRIC = "prefill-attention µs/step and achieved bf16 TFLOP/s as a fraction of B200 peak, 1 GPU"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 FLUSH_BYTES = 256 << 20
 SLEEP_CYCLES = 1_000_000  # ~0.5 ms of GPU spin before each step: longer than the host needs to queue it
 
@@ -241,7 +246,7 @@ def run_reference(args, rank: int):
             vals.append(us)
     value = statistics.mean(vals)
     line = {
-        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "us/step",
+        "impl": "reference", "metric": PREFILL_METRIC if args.config == "prefill" else METRIC, "value": round(value, 3), "unit": "us/step",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value / 1e3, 6),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": pr.name, **workload_desc(pr)},
@@ -557,6 +562,157 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
     return 0
 
 
+# ---------------------------------------------------------------- prefill (tensor-bound)
+
+def measured_tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return float(json.load(open(p))["bf16_tflops"]), "measured (cuBLAS bf16, burst)"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def prefill_flops(pr) -> int:
+    """Algorithmic FLOPs of causal prefill: row t of request b sees L_b - T + t + 1 keys (none
+    when that is <= 0), and each key costs 2 d for q.k and 2 d for p v."""
+    T, d = pr.q_tokens, pr.head_dim
+    t = np.arange(T, dtype=np.int64)
+    vis = np.clip(pr.seq_lens.astype(np.int64)[:, None] - T + 1 + t[None, :], 0, None)
+    return int(vis.sum()) * pr.n_q_heads * 4 * d
+
+
+def run_prefill(args, rank: int, world: int, local_rank: int, dist):
+    import torch
+
+    import paged_kv_decode_29_b200 as da
+    from paged_kv_decode_29_b200 import build as dbuild
+
+    if not os.path.exists(da.LIB_PATH):
+        dbuild.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pr = make_workload(args)
+    log(f"[rank {rank}] prefill workload {pr.name}: B={pr.batch} Hq={pr.n_q_heads} Hkv={pr.n_kv_heads} "
+        f"d={pr.head_dim} T={pr.q_tokens} P={pr.page_size} tokens={int(pr.seq_lens.sum())}")
+    bf = torch.bfloat16
+    q = torch.from_numpy(pr.q.view(np.int16)).view(bf).to(dev)
+    k = torch.from_numpy(pr.k_pages.view(np.int16)).view(bf).to(dev)
+    v = torch.from_numpy(pr.v_pages.view(np.int16)).view(bf).to(dev)
+    tab, lens = (torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in (pr.page_table, pr.seq_lens))
+    out = torch.empty((pr.batch, pr.q_tokens, pr.n_q_heads, pr.head_dim), dtype=torch.float32, device=dev)
+    lse = torch.empty((pr.batch, pr.q_tokens, pr.n_q_heads), dtype=torch.float32, device=dev)
+    status = torch.zeros((), dtype=torch.int32, device=dev)
+    flush = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def one_step(a, b_):
+        torch.sum(flush, dim=0, out=flush_sink)
+        torch.cuda._sleep(SLEEP_CYCLES)
+        a.record(stream)
+        da.prefill(q, k, v, tab, lens, sm_scale=pr.sm_scale, out=out, lse=lse, status=status)
+        b_.record(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = ""
+    sampler = ClockSampler(gpu_id) if not args.profile else None
+    if sampler:
+        sampler.__enter__()
+    t_window = time.perf_counter()
+    for _ in range(args.warmup):
+        one_step(ev(), ev())
+    barrier()
+    if int(status.item()) != da.OK:
+        raise RuntimeError(f"device status after warm-up: {da.status_string(int(status.item()))}")
+    evs = [(ev(), ev()) for _ in range(args.steps)]
+    barrier()
+    for a, b_ in evs:
+        one_step(a, b_)
+    barrier()
+    if int(status.item()) != da.OK:
+        raise RuntimeError(f"device status after timing: {da.status_string(int(status.item()))}")
+    step_m = statistics.mean(a.elapsed_time(b_) * 1e3 for a, b_ in evs)
+    if sampler:
+        while time.perf_counter() - t_window < 1.5:
+            one_step(ev(), ev())
+            torch.cuda.synchronize()
+        sampler.__exit__(None, None, None)
+
+    e2e = None
+    if not args.no_e2e and not args.profile:
+        hq = torch.empty(q.shape, dtype=bf).copy_(q.cpu()).pin_memory()
+        htab = torch.from_numpy(pr.page_table).pin_memory()
+        hlens = torch.from_numpy(pr.seq_lens).pin_memory()
+        hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        h2d = hq.numel() * 2 + htab.numel() * 4 + hlens.numel() * 4
+        d2h = hout.numel() * 4 + hlse.numel() * 4
+        et = []
+        for i in range(args.warmup + args.steps):
+            a, b_ = ev(), ev()
+            torch.sum(flush, dim=0, out=flush_sink)
+            torch.cuda._sleep(SLEEP_CYCLES)
+            a.record(stream)
+            q.copy_(hq, non_blocking=True)
+            tab.copy_(htab, non_blocking=True)
+            lens.copy_(hlens, non_blocking=True)
+            da.prefill(q, k, v, tab, lens, sm_scale=pr.sm_scale, out=out, lse=lse, status=status)
+            hout.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+            b_.record(stream)
+            b_.synchronize()
+            if i >= args.warmup:
+                et.append(a.elapsed_time(b_) * 1e3)
+        e2e = {"value": round(statistics.mean(et), 3), "unit": "us/step", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h),
+               "note": "per step: q, page table and seq_lens from pinned host memory, prefill, out and lse back "
+                       "to pinned host memory; the KV cache stays resident in HBM"}
+    if dist is not None:
+        t = torch.tensor([step_m], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_m = t.item()
+    if rank != 0:
+        return 0
+    flops = prefill_flops(pr)
+    peak, peak_kind = measured_tensor_peak()
+    tflops = flops / (step_m * 1e-6) / 1e12
+    line = {
+        "metric": PREFILL_METRIC,
+        "value": round(step_m, 3), "unit": "us/step", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_m / 1e3, 6), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": pr.name, **workload_desc(pr),
+                   "l2": "flushed before every step (a reduction reading 256 MiB)",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "algorithmic_flops": flops,
+        "roofline": {"bound": "tensor", "kernel": "prefill_kernel", "achieved": round(tflops, 1), "peak": peak,
+                     "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None},
+        "gpu_launches": args.steps,  # one prefill kernel per timed step
+    }
+    if sampler:
+        line["clocks"] = sampler.summary()
+    if e2e is not None:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline and not args.profile and world == 1:
+        import oracle
+        oracle.build()
+        us, threads, sample = oracle_timing(pr, budget_s=15.0)
+        line["cpu_baseline"] = {"value": round(us, 1), "unit": "us/step", "cores": threads, "kind": "oracle",
+                                "sample": sample}
+    emit(line, args)
+    return 0
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -575,6 +731,8 @@ def main():
                                  device_id=torch.device("cuda", local_rank))
         dist = tdist
     try:
+        if args.config == "prefill":
+            return run_prefill(args, rank, world, local_rank, dist)
         return run_ours(args, rank, world, local_rank, dist)
     finally:
         if dist is not None:

@@ -18,10 +18,10 @@ import workloads as W  # noqa: E402
 
 # workload -> (requests captured, dram read bytes, dram write bytes) of the captured launch
 CAPTURED = {
-    "uniform": (8, 134361600, 3171584),
-    "mixed": (16, 1039219968, 18049280),
-    "fp8_spec": (4, 167430400, 7366912),
-    "long_b4": (1, 536984832, 6270976),
+    "uniform": (8, 134364672, 3204352),
+    "mixed": (16, 1039151360, 17712384),
+    "fp8_spec": (4, 167202048, 7321088),
+    "long_b4": (1, 536968704, 5867520),
 }
 
 
