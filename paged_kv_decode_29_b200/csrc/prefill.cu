@@ -3,58 +3,122 @@
 // prefill and paged-KV decode over a BF16 KV cache, GQA). The T query rows of request b are its
 // last T positions: row t sees keys 0 .. Lb - T + t (the decode's bottom-right causal rule,
 // with T large). A dense contraction, on the fifth-generation tensor cores:
-//  * CTA = (request, q head, block of 128 query rows), heaviest blocks first. Q (128 rows x 128
-//    bf16) sits in shared memory as the A operand of S = Q K^T (K-major, 128-byte swizzle).
-//  * per block of 128 keys: S (128 x 128 fp32) in tensor memory on kind::f16 (B = the K tile as
-//    TMA staged it, K-major); thread r of the 128-thread softmax group owns query row r (tensor-
-//    memory lane r), so a row's maximum and sum need no exchange between threads; P (bf16) goes to
-//    shared memory as the A operand of O += P V, B = the V tile as staged (head dims contiguous:
-//    MN-major); O (128 x 128 fp32) stays in tensor memory.
+//  * CTA = two tiles of 128 query rows that read the same keys: two q heads of one KV head with
+//    the same rows when G is even, else two adjacent row blocks of one q head. Every K/V block
+//    brought in by TMA serves both tiles. CTAs are numbered heaviest first.
+//  * per block of 128 keys and tile u: S_u = Q_u K^T (128 x 128 fp32) in tensor memory on
+//    kind::f16 (Q and K K-major, 128-byte swizzle); softmax warpgroup u (thread r owns query row
+//    r = tensor-memory lane r) turns S_u into P_u, bf16 packed two to a column over S_u's first
+//    64 columns; O_u += P_u V reads P_u from tensor memory and V as TMA staged it (head dims
+//    contiguous: MN-major). O_0 and O_1 (128 x 128 fp32 each) stay in tensor memory.
+//  * the MMA warp alternates the tiles: while warpgroup 0 works on S_0, the tensor core runs
+//    tile 1's P V and next S, and the other way round.
 //  * online softmax with a per-row reference maximum that moves only when a score passes it by
-//    more than 2^kPfTau (then the row of O is rescaled in place), so most blocks skip the rescale.
-// CTA: 6 warps: warps 0-3 softmax group, warp 4 TMA producer (two K/V stages of 128 keys), warp 5
-// MMA issue (one thread). Every wait is bounded (DECATTN_ETIMEOUT, then an orderly exit).
+//    more than 2^kPfTau: P is computed in one pass against the current reference, and the pass
+//    is redone (after rescaling the row of O) only in the rare block that moves it.
+// CTA: 10 warps: 0-3 softmax of tile 0, 4-7 softmax of tile 1, 8 TMA producer (separate K and V
+// rings of two 128-key stages), 9 MMA issue (one thread). Every wait is bounded (DECATTN_ETIMEOUT,
+// then an orderly exit).
 #include "common.cuh"
 #include "tc.cuh"
 
 namespace decattn {
 
-constexpr int kPfD = 128;        // head_dim
-constexpr int kPfM = 128;        // query rows per CTA: the M of both products
-constexpr int kPfN = 128;        // keys per block: the N of S and the contraction of P V
-constexpr int kPfStages = 2;     // K/V stages
-constexpr int kPfThreads = 192;
-constexpr int kPfTau = 8;        // P <= 2^kPfTau
-constexpr int kPfTmemCols = 512; // S double buffer (2 x 128 columns), O (128)
-
+constexpr int kPfD = 128;         // head_dim
+constexpr int kPfM = 128;         // query rows per tile: the M of both products
+constexpr int kPfN = 128;         // keys per block: the N of S and the contraction of P V
+constexpr int kPfStages = 2;      // K stages and V stages
+constexpr int kPfWarps = 10;
+constexpr int kPfThreads = 32 * kPfWarps;
+constexpr int kPfTau = 8;         // P <= 2^kPfTau
+constexpr int kPfTmemCols = 512;  // S_0, S_1, O_0, O_1: 128 columns each
 
 // Shared-memory layout (offsets from a 1024-byte aligned base). A 128 x 128 bf16 tile is two
 // "atoms" of 64 elements (128 bytes) per row: atom a holds elements 64a .. 64a + 63 of all 128
 // rows, row r at 128 r, 16-byte chunk c at (c ^ (r % 8)) * 16 (the TMA 128-byte swizzle).
 struct PfSmem {
-  static constexpr int ATOM = 128 * 128;                 // 16 KB
-  static constexpr int TILE = 2 * ATOM;                  // 32 KB
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_STAGE = OFF_Q + TILE;         // [stage]: K tile, then V tile
-  static constexpr int OFF_P = OFF_STAGE + kPfStages * 2 * TILE;
-  static constexpr int OFF_BAR = OFF_P + TILE;
-  static constexpr int NBAR = 12;
-  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;    // tensor-memory base, abort flag
+  static constexpr int ATOM = 128 * 128;                  // 16 KB
+  static constexpr int TILE = 2 * ATOM;                   // 32 KB
+  static constexpr int OFF_Q = 0;                         // [tile]
+  static constexpr int OFF_K = OFF_Q + 2 * TILE;          // [stage]
+  static constexpr int OFF_V = OFF_K + kPfStages * TILE;  // [stage]
+  static constexpr int OFF_BAR = OFF_V + kPfStages * TILE;
+  static constexpr int NBAR = 16;
+  static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;     // tensor-memory base, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
   static_assert(ALLOC <= 227 * 1024, "one CTA per SM");
 };
 
 enum PfBar {
-  kPfKvFull = 0,   // [2] producer -> MMA: K and V tiles of a key block landed
-  kPfKvEmpty = 2,  // [2] MMA commit after the block's P V -> producer
-  kPfSFull = 4,    // [2] MMA commit -> softmax: S of a key block in tensor memory
-  kPfSFree = 6,    // [2] 4 softmax warps -> MMA: that S buffer has been read
-  kPfPReady = 8,   // 4 softmax warps -> MMA: P written (and rows of O rescaled)
-  kPfPvDone = 9,   // MMA commit -> softmax: O += P V of a block complete
-  kPfQReady = 10,  // 4 softmax warps -> MMA: Q written
-  kPfFin = 11,     // MMA commit -> MMA: every tensor-core operation complete
+  kPfKFull = 0,    // [stage] producer -> MMA: K tile landed
+  kPfKEmpty = 2,   // [stage] MMA commit after the block's last S -> producer
+  kPfVFull = 4,    // [stage] producer -> MMA: V tile landed
+  kPfVEmpty = 6,   // [stage] MMA commit after the block's last P V -> producer
+  kPfSFull = 8,    // [tile] MMA commit -> softmax: S_u of the next block in tensor memory
+  kPfPReady = 10,  // [tile] 4 softmax warps -> MMA: P_u written (and rows of O_u rescaled)
+  kPfOFin = 12,    // [tile] MMA commit after tile u's last P V -> softmax epilogue
+  kPfQReady = 14,  // 8 softmax warps -> MMA: Q of both tiles written
+  kPfDrain = 15,   // MMA commit -> MMA: every tensor-core operation complete
 };
+
+// The two tiles of CTA `cta` (numbered heaviest first); the host sizes the grid the same way.
+struct PfTile {
+  int qh, t0, nkb;  // q head, first query row, key blocks its rows see
+};
+
+__host__ __device__ inline int pf_tiles_per_head(int T) { return (T + kPfM - 1) / kPfM; }
+__host__ __device__ inline int pf_grid(int B, int T, int Hq, int G) {
+  const int nqb = pf_tiles_per_head(T);
+  return (G % 2 == 0) ? nqb * B * (Hq / 2) : ((nqb + 1) / 2) * B * Hq;
+}
+
+// P_u = 2^(s * scale - m) over this warp's 32 rows of S_u (128 keys each), written as bf16
+// pairs (the lower key in the low half) over S_u's first 64 columns as the chunks are read:
+// chunk c lands on columns 16c .. 16c + 15, which hold scores already read. Returns the row
+// sum of P in fp32. Keys from nvis on are invisible to the row when `masked`.
+__device__ __forceinline__ float pf_exp(uint32_t tS, float sc, float m, bool masked, int nvis) {
+  const float nmu = m == -INFINITY ? 0.f : -m;
+  float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+  #pragma unroll
+  for (int c = 0; c < kPfN / 32; ++c) {
+    float v[32];
+    tmem_ld32(tS + 32 * c, v);
+    if (masked) {
+      #pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (32 * c + i >= nvis) v[i] = -INFINITY;
+    }
+    uint32_t w[16];
+    #pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+      const float p0 = fast_exp2(fmaf(v[i], sc, nmu)), p1 = fast_exp2(fmaf(v[i + 1], sc, nmu));
+      const float p2 = fast_exp2(fmaf(v[i + 2], sc, nmu)), p3 = fast_exp2(fmaf(v[i + 3], sc, nmu));
+      l0 += p0; l1 += p1; l2 += p2; l3 += p3;
+      w[i / 2] = pack_bf16(p0, p1);
+      w[i / 2 + 1] = pack_bf16(p2, p3);
+    }
+    tmem_st16u(tS + 16 * c, w);
+  }
+  return (l0 + l1) + (l2 + l3);
+}
+
+// The row maximum of the raw scores of this warp's 32 rows of S_u (the scale is positive).
+__device__ __forceinline__ float pf_max(uint32_t tS, bool masked, int nvis) {
+  float m0 = -INFINITY, m1 = -INFINITY;
+  #pragma unroll
+  for (int c = 0; c < kPfN / 32; ++c) {
+    float v[32];
+    tmem_ld32(tS + 32 * c, v);
+    #pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+      const bool vis0 = !masked || 32 * c + i < nvis, vis1 = !masked || 32 * c + i + 1 < nvis;
+      m0 = fmaxf(m0, vis0 ? v[i] : -INFINITY);
+      m1 = fmaxf(m1, vis1 ? v[i + 1] : -INFINITY);
+    }
+  }
+  return fmaxf(m0, m1);
+}
 
 __global__ void __launch_bounds__(kPfThreads, 1)
 prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
@@ -66,36 +130,55 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int qb = (int)gridDim.x - 1 - (int)blockIdx.x;  // the longest query blocks start first
-  const int qh = blockIdx.y, b = blockIdx.z, h = qh / p.G;
+  // ---- request, KV head and the two tiles of this CTA. The row-block step is the slowest
+  //      index of the grid, counted down, so the CTAs with the most keys start first.
+  const bool head_pair = (p.G % 2) == 0;
+  const int ny = head_pair ? p.Hq / 2 : p.Hq;
+  const int nsteps = head_pair ? pf_tiles_per_head(p.T) : (pf_tiles_per_head(p.T) + 1) / 2;
+  const int step = nsteps - 1 - (int)blockIdx.x / (p.B * ny);
+  const int rem = (int)blockIdx.x % (p.B * ny);
+  const int b = rem / ny, y = rem % ny;
   const int Lb = p.seq_lens[b];
-  const int t0 = qb * kPfM;
-  const int t_last = min(t0 + kPfM, p.T) - 1;
-  // keys the block's last row sees: [0, min(Lb, Lb - T + t_last + 1))
-  const int kmax = Lb < 0 ? 0 : max(0, min(Lb, Lb - p.T + t_last + 1));
-  const int nkb = (kmax + kPfN - 1) / kPfN;
+  PfTile tl0, tl1;
+  {
+    tl0.qh = head_pair ? 2 * y : y;
+    tl1.qh = head_pair ? 2 * y + 1 : y;
+    tl0.t0 = head_pair ? step * kPfM : 2 * step * kPfM;
+    tl1.t0 = head_pair ? step * kPfM : (2 * step + 1) * kPfM;
+    // keys the tile's last row sees: [0, min(Lb, Lb - T + t_last + 1))
+    const int tlast0 = min(tl0.t0 + kPfM, p.T) - 1, tlast1 = min(tl1.t0 + kPfM, p.T) - 1;
+    const int kmax0 = (Lb < 0 || tl0.t0 >= p.T) ? 0 : max(0, min(Lb, Lb - p.T + tlast0 + 1));
+    const int kmax1 = (Lb < 0 || tl1.t0 >= p.T) ? 0 : max(0, min(Lb, Lb - p.T + tlast1 + 1));
+    tl0.nkb = (kmax0 + kPfN - 1) / kPfN;
+    tl1.nkb = (kmax1 + kPfN - 1) / kPfN;
+  }
+  const int h = tl0.qh / p.G;
+  const int nkb_max = max(tl0.nkb, tl1.nkb);
 
   // The K/V stages start zeroed: rows past a request's last page are never loaded, and their
   // contents meet P = 0 in the MMA, so they must be finite.
-  for (int i = threadIdx.x; i < kPfStages * 2 * L::TILE / 16; i += kPfThreads)
-    reinterpret_cast<uint4*>(sm + L::OFF_STAGE)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = threadIdx.x; i < 2 * kPfStages * L::TILE / 16; i += kPfThreads)
+    reinterpret_cast<uint4*>(sm + L::OFF_K)[i] = make_uint4(0, 0, 0, 0);
   fence_async_smem();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPfStages; ++s) {
-      mbar_init(&bar[kPfKvFull + s], 1);
-      mbar_init(&bar[kPfKvEmpty + s], 1);
-      mbar_init(&bar[kPfSFull + s], 1);
-      mbar_init(&bar[kPfSFree + s], 4);
+      mbar_init(&bar[kPfKFull + s], 1);
+      mbar_init(&bar[kPfKEmpty + s], 1);
+      mbar_init(&bar[kPfVFull + s], 1);
+      mbar_init(&bar[kPfVEmpty + s], 1);
     }
-    mbar_init(&bar[kPfPReady], 4);
-    mbar_init(&bar[kPfPvDone], 1);
-    mbar_init(&bar[kPfQReady], 4);
-    mbar_init(&bar[kPfFin], 1);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bar[kPfSFull + u], 1);
+      mbar_init(&bar[kPfPReady + u], 4);
+      mbar_init(&bar[kPfOFin + u], 1);
+    }
+    mbar_init(&bar[kPfQReady], 8);
+    mbar_init(&bar[kPfDrain], 1);
     *abort = 0;
     if (Lb < 0) set_status(p.status, DECATTN_EDEVICE);
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_base_sm)),
                  "n"(kPfTmemCols)
                  : "memory");
@@ -106,17 +189,15 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
   tc_fence_after();
   const uint32_t tmem = *tmem_base_sm;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ===================================================================== producer
     if (lane == 0) { prefetch_tensormap(&tmK); prefetch_tensormap(&tmV); }
-    int st = 0; uint32_t eph = 1;
-    int64_t n_fill = 0;
-    for (int kb = 0; kb < nkb; ++kb) {
-      int r = 1;
-      if (lane == 0) r = tc_wait(&bar[kPfKvEmpty + st], eph, p.status, abort) ? 1 : 0;
-      if (!__shfl_sync(0xffffffffu, r, 0)) break;
-      // lane g < 8: the 16-key group g of the block (its page id and row in the pool)
-      const int key16 = kb * kPfN + 16 * lane;
+    int nk = 0, nv = 0;  // K / V blocks whose copies were issued
+    for (int g = 0; g < nkb_max; ++g) {
+      const int st = g % kPfStages;
+      const uint32_t eph = (uint32_t)((g / kPfStages) & 1) ^ 1u;
+      // lane i < 8: the 16-key group i of the block (its page id and row in the pool)
+      const int key16 = g * kPfN + 16 * lane;
       const bool has = lane < kPfN / 16 && key16 < Lb;
       int row = 0;
       if (has) {
@@ -128,140 +209,163 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
         }
         row = (pid * p.Hkv + h) * p.P + key16 % p.P;
       }
-      const int ngroups = __popc(__ballot_sync(0xffffffffu, has));
-      if (lane == 0) mbar_arrive_expect_tx(&bar[kPfKvFull + st], (uint32_t)(ngroups * 4 * 16 * 128));
+      const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, has)) * 2u * 16u * 128u;
+      int r = 1;
+      if (lane == 0) r = tc_wait(&bar[kPfKEmpty + st], eph, p.status, abort) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, r, 0)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&bar[kPfKFull + st], bytes);
       __syncwarp();
       if (has) {
-        uint8_t* kt = sm + L::OFF_STAGE + st * 2 * L::TILE;
-        uint8_t* vt = kt + L::TILE;
         #pragma unroll
-        for (int a = 0; a < 2; ++a) {  // head dims 64a .. 64a + 63: one 128-byte swizzled atom
-          tma_load_2d(kt + a * L::ATOM + lane * 16 * 128, &tmK, 64 * a, row, &bar[kPfKvFull + st]);
-          tma_load_2d(vt + a * L::ATOM + lane * 16 * 128, &tmV, 64 * a, row, &bar[kPfKvFull + st]);
-        }
+        for (int a = 0; a < 2; ++a)  // head dims 64a .. 64a + 63: one 128-byte swizzled atom
+          tma_load_2d(sm + L::OFF_K + st * L::TILE + a * L::ATOM + lane * 16 * 128, &tmK, 64 * a, row,
+                      &bar[kPfKFull + st]);
       }
-      ++n_fill;
-      if (++st == kPfStages) { st = 0; eph ^= 1; }
+      ++nk;
+      if (lane == 0) r = tc_wait(&bar[kPfVEmpty + st], eph, p.status, abort) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, r, 0)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&bar[kPfVFull + st], bytes);
+      __syncwarp();
+      if (has) {
+        #pragma unroll
+        for (int a = 0; a < 2; ++a)
+          tma_load_2d(sm + L::OFF_V + st * L::TILE + a * L::ATOM + lane * 16 * 128, &tmV, 64 * a, row,
+                      &bar[kPfVFull + st]);
+      }
+      ++nv;
     }
     if (*abort && lane == 0) {
       // let the copies already issued land before the CTA exits
-      for (int64_t n = n_fill > kPfStages ? n_fill - kPfStages : 0; n < n_fill; ++n)
-        mbar_wait(&bar[kPfKvFull + n % kPfStages], (uint32_t)((n / kPfStages) & 1), nullptr);
+      for (int n = max(nk - kPfStages, 0); n < nk; ++n)
+        mbar_wait(&bar[kPfKFull + n % kPfStages], (uint32_t)((n / kPfStages) & 1), nullptr);
+      for (int n = max(nv - kPfStages, 0); n < nv; ++n)
+        mbar_wait(&bar[kPfVFull + n % kPfStages], (uint32_t)((n / kPfStages) & 1), nullptr);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ===================================================================== MMA issue
     if (lane == 0) {
       const uint32_t base = smem_u32(sm);
       constexpr uint32_t idS = umma_idesc(1, 1, 0, 0, kPfM, kPfN);  // bf16 x bf16, both K-major
       constexpr uint32_t idO = umma_idesc(1, 1, 0, 1, kPfM, kPfD);  // bf16 x bf16, B (V) MN-major
       // descriptors (start address in 16-byte units in the low bits, so offsets add on):
-      // Q, K, P K-major with 128-byte swizzle (8-row groups 1024 B apart; a 16-element k-step is
+      // Q and K K-major with 128-byte swizzle (8-row groups 1024 B apart; a 16-element k-step is
       // 32 bytes inside an atom, the next atom 16 KB on); V MN-major with 128-byte swizzle (the
       // two 64-element atoms of the head dims 16 KB apart, 8-key groups 1024 B apart).
-      const uint64_t dQ = umma_desc(base + L::OFF_Q, 16, 1024, 2);
-      const uint64_t dK0 = umma_desc(base + L::OFF_STAGE, 16, 1024, 2);
-      const uint64_t dP = umma_desc(base + L::OFF_P, 16, 1024, 2);
-      const uint64_t dV0 = umma_desc(base + L::OFF_STAGE + L::TILE, L::ATOM, 1024, 2);
-      const uint32_t tO = tmem + 2 * kPfN;
-      bool ok = tc_wait(&bar[kPfQReady], 0, p.status, abort);
+      const uint64_t dQ0 = umma_desc(base + L::OFF_Q, 16, 1024, 2);
+      const uint64_t dK0 = umma_desc(base + L::OFF_K, 16, 1024, 2);
+      const uint64_t dV0 = umma_desc(base + L::OFF_V, L::ATOM, 1024, 2);
+      const int nkb[2] = {tl0.nkb, tl1.nkb};
       auto kstep = [](int k) -> uint64_t {  // 16-element step k of a K-major 128-element operand
         return (uint64_t)(((k >> 2) * L::ATOM + (k & 3) * 32) >> 4);
       };
-      auto pv = [&](int g) -> bool {
-        if (!tc_wait(&bar[kPfPReady], (uint32_t)(g & 1), p.status, abort)) return false;
-        tc_fence_after();
-        const int sg = g % kPfStages;
-        const uint64_t dV = dV0 + (uint64_t)((sg * 2 * L::TILE) >> 4);
+      auto issue_s = [&](int u, int g) {  // S_u = Q_u K(g)^T
+        const uint64_t dQ = dQ0 + (uint64_t)((u * L::TILE) >> 4);
+        const uint64_t dK = dK0 + (uint64_t)(((g % kPfStages) * L::TILE) >> 4);
         #pragma unroll
-        for (int k = 0; k < kPfN / 16; ++k)  // 16 keys per instruction: V advances 2 KB
-          umma_f16(tO, dP + kstep(k), dV + (uint64_t)((k * 2048) >> 4), idO, (g > 0 || k > 0) ? 1u : 0u);
-        umma_commit(&bar[kPfPvDone]);
-        umma_commit(&bar[kPfKvEmpty + sg]);  // K and V of the stage have both been read
-        return true;
+        for (int k = 0; k < kPfD / 16; ++k) umma_f16(tmem + kPfN * u, dQ + kstep(k), dK + kstep(k), idS, k > 0 ? 1u : 0u);
+        umma_commit(&bar[kPfSFull + u]);
       };
-      for (int g = 0; ok && g < nkb; ++g) {
-        const int st = g % kPfStages, sb = g & 1;
-        if (!tc_wait(&bar[kPfKvFull + st], (uint32_t)((g / kPfStages) & 1), p.status, abort) ||
-            !tc_wait(&bar[kPfSFree + sb], (uint32_t)(((g >> 1) & 1) ^ 1), p.status, abort)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint64_t dK = dK0 + (uint64_t)((st * 2 * L::TILE) >> 4);
+      auto issue_pv = [&](int u, int g) {  // O_u += P_u V(g); P_u: 16 keys = 8 columns per step
+        const uint64_t dV = dV0 + (uint64_t)(((g % kPfStages) * L::TILE) >> 4);
+        const uint32_t tP = tmem + kPfN * u, tO = tmem + 2 * kPfN + kPfD * u;
         #pragma unroll
-        for (int k = 0; k < kPfD / 16; ++k)
-          umma_f16(tmem + kPfN * sb, dQ + kstep(k), dK + kstep(k), idS, k > 0 ? 1u : 0u);
-        umma_commit(&bar[kPfSFull + sb]);
-        if (g > 0 && !pv(g - 1)) { ok = false; break; }
+        for (int k = 0; k < kPfN / 16; ++k)  // V advances 16 keys = 2 KB
+          umma_f16_tmem_a(tO, tP + 8 * k, dV + (uint64_t)((k * 2048) >> 4), idO, (g > 0 || k > 0) ? 1u : 0u);
+      };
+      bool ok = tc_wait(&bar[kPfQReady], 0, p.status, abort);
+      if (ok && nkb_max > 0) {
+        ok = tc_wait(&bar[kPfKFull], 0, p.status, abort);
+        if (ok) {
+          tc_fence_after();
+          if (nkb[0] > 0) issue_s(0, 0);
+          if (nkb[1] > 0) issue_s(1, 0);
+          umma_commit(&bar[kPfKEmpty]);
+        }
       }
-      if (ok && nkb > 0 && !pv(nkb - 1)) ok = false;
+      for (int g = 0; ok && g < nkb_max; ++g) {
+        const int st = g % kPfStages;
+        bool v_ready = false, k_ready = false;
+        #pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (g >= nkb[u]) continue;
+          if (!v_ready) {
+            if (!tc_wait(&bar[kPfVFull + st], (uint32_t)((g / kPfStages) & 1), p.status, abort)) { ok = false; break; }
+            v_ready = true;
+          }
+          if (!tc_wait(&bar[kPfPReady + u], (uint32_t)(g & 1), p.status, abort)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(u, g);
+          if (u == 1 || g >= nkb[1]) umma_commit(&bar[kPfVEmpty + st]);  // the block's last P V
+          if (g == nkb[u] - 1) umma_commit(&bar[kPfOFin + u]);
+          if (g + 1 < nkb[u]) {
+            const int sn = (g + 1) % kPfStages;
+            if (!k_ready) {
+              if (!tc_wait(&bar[kPfKFull + sn], (uint32_t)(((g + 1) / kPfStages) & 1), p.status, abort)) {
+                ok = false;
+                break;
+              }
+              k_ready = true;
+              tc_fence_after();
+            }
+            issue_s(u, g + 1);
+            if (u == 1 || g + 1 >= nkb[1]) umma_commit(&bar[kPfKEmpty + sn]);  // the next block's last S
+          }
+        }
+      }
       if (!ok) *abort = 1;
-      umma_commit(&bar[kPfFin]);
-      mbar_wait(&bar[kPfFin], 0, nullptr);
+      umma_commit(&bar[kPfDrain]);
+      mbar_wait(&bar[kPfDrain], 0, nullptr);
     }
     __syncwarp();
   } else {
-    // ===================================================================== softmax group
-    const int r = threadIdx.x;  // query row of the block = tensor-memory lane
-    const int t = t0 + r;
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    const uint32_t tO = tmem + lane_off + 2 * kPfN;
+    // ===================================================================== softmax warpgroups
+    const int u = warp >> 2, wq = warp & 3;
+    const int r = 32 * wq + lane;  // query row of the tile = tensor-memory lane
+    const int qh = u ? tl1.qh : tl0.qh;
+    const int t = (u ? tl1.t0 : tl0.t0) + r;
+    const int nkb = u ? tl1.nkb : tl0.nkb;
+    const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+    const uint32_t tS = tmem + lane_off + kPfN * u;
+    const uint32_t tO = tmem + lane_off + 2 * kPfN + kPfD * u;
     // ---- Q row t into its K-major swizzled place (zero past T)
     {
       uint4 x[16];
       const bool has = t < p.T;
-      const uint4* src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * p.T + t) * p.Hq + qh) * kPfD);
+      const uint4* src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * p.T + (has ? t : 0)) * p.Hq + qh) * kPfD);
       #pragma unroll
       for (int c = 0; c < 16; ++c) x[c] = has ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+      uint8_t* q_sm = sm + L::OFF_Q + u * L::TILE;
       #pragma unroll
       for (int c = 0; c < 16; ++c)  // chunk c: head dims 8c .. 8c + 7
-        *reinterpret_cast<uint4*>(sm + L::OFF_Q + (c >> 3) * L::ATOM + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = x[c];
+        *reinterpret_cast<uint4*>(q_sm + (c >> 3) * L::ATOM + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = x[c];
     }
     fence_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bar[kPfQReady]);
 
-    const int lim = t < p.T ? Lb - p.T + t : -1;  // the last key this row sees
-    float mref = -INFINITY, l = 0.f;
+    const int lim = t < p.T ? Lb - p.T + t : -1;  // the last key this row sees (< 0: none)
+    const int lim_min = __reduce_min_sync(0xffffffffu, lim);
+    const float sc = p.qk_scale_log2;
+    float mref = -INFINITY, l = 0.f;  // reference maximum (log2 units) and row sum
     bool ok = true;
     for (int g = 0; g < nkb; ++g) {
-      const int sb = g & 1;
-      if (!tc_wait_warp(&bar[kPfSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort)) { ok = false; break; }
+      if (!tc_wait_warp(&bar[kPfSFull + u], (uint32_t)(g & 1), p.status, abort)) { ok = false; break; }
       tc_fence_after();
-      float s[kPfN];
-      #pragma unroll
-      for (int q4 = 0; q4 < kPfN / 32; ++q4) {
-        float v[32];
-        tmem_ld32(tmem + lane_off + kPfN * sb + 32 * q4, v);
-        #pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * q4 + i] = v[i];
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[kPfSFree + sb]);
-      // ---- scale, mask (keys past the row's limit or the request), block maximum
       const int j0 = g * kPfN;
-      const int nvis = min(kPfN, min(lim, Lb - 1) - j0 + 1);  // keys j0 .. j0 + nvis - 1 are visible
-      float bm = -INFINITY;
-      #pragma unroll
-      for (int i = 0; i < kPfN; ++i) {
-        s[i] = i < nvis ? s[i] * p.qk_scale_log2 : -INFINITY;
-        bm = fmaxf(bm, s[i]);
-      }
-      bool pv_waited = false;
+      const bool masked = j0 + kPfN - 1 > lim_min;  // warp-uniform: some row does not see every key
+      const int nvis = lim - j0 + 1;                // keys j0 .. j0 + nvis - 1 are visible to the row
+      // the row maximum first; the reference moves when it is passed by more than 2^kPfTau
+      const float xmax = pf_max(tS, masked, nvis) * sc;
       float alpha = 1.f;
-      if (bm > mref + (float)kPfTau) {
-        // the row's reference moves to this block's maximum; O's row is rescaled in place
-        alpha = mref == -INFINITY ? 0.f : fast_exp2(mref - bm);
+      if (xmax > mref + (float)kPfTau) {  // false when the row sees nothing here (xmax = -inf)
+        alpha = mref == -INFINITY ? 0.f : fast_exp2(mref - xmax);
         l *= alpha;
-        mref = bm;
+        mref = xmax;
       }
-      // tensor-memory loads and stores are warp-wide: the warp rescales when any of its rows
-      // needs it (alpha = 1 for the others)
+      // O_u's rows hold every block before this one: S_u of this block was committed after the
+      // previous P V, so that product is complete. Tensor-memory accesses are warp-wide: the warp
+      // rescales when any of its rows moved (alpha = 1 for the others).
       if (g > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if (!tc_wait_warp(&bar[kPfPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
-        pv_waited = true;
-        tc_fence_after();
         #pragma unroll
         for (int q4 = 0; q4 < kPfD / 32; ++q4) {
           float o[32];
@@ -271,31 +375,14 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
           tmem_st32(tO + 32 * q4, o);
         }
       }
-      // ---- P = 2^(s - m_ref) (at most 2^kPfTau), row sum, bf16 into the P tile (after the
-      //      previous block's P V has read it)
-      const float mu = mref == -INFINITY ? 0.f : mref;
-      #pragma unroll
-      for (int i = 0; i < kPfN; ++i) {
-        s[i] = fast_exp2(s[i] - mu);
-        l += s[i];
-      }
-      if (g > 0 && !pv_waited && !tc_wait_warp(&bar[kPfPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) {
-        ok = false;
-        break;
-      }
-      #pragma unroll
-      for (int c = 0; c < 16; ++c) {  // keys 8c .. 8c + 7
-        const uint4 w = make_uint4(pack_bf16(s[8 * c], s[8 * c + 1]), pack_bf16(s[8 * c + 2], s[8 * c + 3]),
-                                   pack_bf16(s[8 * c + 4], s[8 * c + 5]), pack_bf16(s[8 * c + 6], s[8 * c + 7]));
-        *reinterpret_cast<uint4*>(sm + L::OFF_P + (c >> 3) * L::ATOM + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = w;
-      }
-      fence_async_smem();
+      l += pf_exp(tS, sc, mref, masked, nvis);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[kPfPReady]);
+      if (lane == 0) mbar_arrive(&bar[kPfPReady + u]);
     }
     // ---- epilogue: O / l and lse of row t
-    if (ok && nkb > 0 && !tc_wait_warp(&bar[kPfPvDone], (uint32_t)((nkb - 1) & 1), p.status, abort)) ok = false;
+    if (ok && nkb > 0 && !tc_wait_warp(&bar[kPfOFin + u], 0, p.status, abort)) ok = false;
     if (!ok) *abort = 1;
     if (ok) {  // warp-uniform: every lane takes part in the tensor-memory loads
       tc_fence_after();
@@ -325,17 +412,18 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5)
+  if (warp == 9)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kPfTmemCols) : "memory");
 }
 
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st) {
   const int smem = PfSmem::ALLOC;
   if (!ensure_smem_attr((const void*)prefill_kernel, smem)) return cudaErrorInvalidValue;
-  const int nqb = (p.T + kPfM - 1) / kPfM;
-  if (p.B == 0 || nqb == 0) return cudaSuccess;
+  if (p.B == 0 || p.T == 0 || p.Hq == 0) return cudaSuccess;
+  const int64_t grid = (int64_t)pf_grid(p.B, p.T, p.Hq, p.G);
+  if (grid <= 0 || grid > 0x7fffffff) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(nqb, p.Hq, p.B);
+  cfg.gridDim = dim3((unsigned)grid);
   cfg.blockDim = dim3(kPfThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
