@@ -413,6 +413,29 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Two fp32 lanes in one instruction (fma.rn.f32x2 / add.rn.f32x2, sm_100): (d0, d1) = (a0 b0 + c0,
+// a1 b1 + c1), each rounded once as fmaf would; and (a0 + b0, a1 + b1).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n .reg .b64 ra, rb, rc, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n mov.b64 rc, {%6, %7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n .reg .b64 ra, rb, rd;\n mov.b64 ra, {%2, %3};\n mov.b64 rb, {%4, %5};\n"
+      " add.rn.f32x2 rd, ra, rb;\n mov.b64 {%0, %1}, rd;\n}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // ------------------------------------------------------------------ host-side launchers
 int default_bins(int device);                                     // api.cu
 bool ensure_smem_attr(const void* kernel, int bytes);             // api.cu
@@ -425,6 +448,6 @@ cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const 
                             cudaStream_t st);                     // split_tc.cu
 cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st);  // combine.cu
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                           cudaStream_t st);                      // prefill.cu
+                           const CUtensorMap& tmO, cudaStream_t st);  // prefill.cu
 
 }  // namespace decattn

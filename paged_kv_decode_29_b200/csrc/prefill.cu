@@ -73,55 +73,81 @@ __host__ __device__ inline int pf_grid(int B, int T, int Hq, int G) {
   return (G % 2 == 0) ? nqb * B * (Hq / 2) : ((nqb + 1) / 2) * B * Hq;
 }
 
-// P_u = 2^(s * scale - m) over this warp's 32 rows of S_u (128 keys each), written as bf16
-// pairs (the lower key in the low half) over S_u's first 64 columns as the chunks are read:
-// chunk c lands on columns 16c .. 16c + 15, which hold scores already read. Returns the row
-// sum of P in fp32. Keys from nvis on are invisible to the row when `masked`.
-__device__ __forceinline__ float pf_exp(uint32_t tS, float sc, float m, bool masked, int nvis) {
+// All 128 columns of this warp's 32 lanes of S_u in one round trip (four loads, one wait).
+__device__ __forceinline__ void pf_ld128(uint32_t taddr, float (&v)[128]) {
+  uint32_t r[128];
+  asm volatile(
+      "{\n"
+      " tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%128];\n"
+      " tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%129];\n"
+      " tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95}, [%130];\n"
+      " tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%131];\n"
+      " tcgen05.wait::ld.sync.aligned;\n}"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]),
+        "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]),
+        "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]),
+        "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]),
+        "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]),
+        "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]),
+        "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]),
+        "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]),
+        "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
+      : "memory");
+  #pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// P_u = 2^(s * scale - m) from the row's 128 scores, written as bf16 pairs (the lower key in
+// the low half) over S_u's first 64 columns, chunk c of 32 keys on columns 16c .. 16c + 15.
+// Returns the row sum of P in fp32.
+__device__ __forceinline__ float pf_exp(uint32_t tS, const float (&v)[128], float sc, float m) {
   const float nmu = m == -INFINITY ? 0.f : -m;
-  float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+  float la0 = 0.f, la1 = 0.f, lb0 = 0.f, lb1 = 0.f;
   #pragma unroll
   for (int c = 0; c < kPfN / 32; ++c) {
-    float v[32];
-    tmem_ld32(tS + 32 * c, v);
-    if (masked) {
-      #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (32 * c + i >= nvis) v[i] = -INFINITY;
-    }
     uint32_t w[16];
     #pragma unroll
-    for (int i = 0; i < 32; i += 4) {
-      const float p0 = fast_exp2(fmaf(v[i], sc, nmu)), p1 = fast_exp2(fmaf(v[i + 1], sc, nmu));
-      const float p2 = fast_exp2(fmaf(v[i + 2], sc, nmu)), p3 = fast_exp2(fmaf(v[i + 3], sc, nmu));
-      l0 += p0; l1 += p1; l2 += p2; l3 += p3;
-      w[i / 2] = pack_bf16(p0, p1);
-      w[i / 2 + 1] = pack_bf16(p2, p3);
+    for (int i = 32 * c; i < 32 * c + 32; i += 4) {
+      float x0, x1, x2, x3;
+      ffma2(x0, x1, v[i], v[i + 1], sc, sc, nmu, nmu);
+      ffma2(x2, x3, v[i + 2], v[i + 3], sc, sc, nmu, nmu);
+      const float p0 = fast_exp2(x0), p1 = fast_exp2(x1), p2 = fast_exp2(x2), p3 = fast_exp2(x3);
+      fadd2(la0, la1, la0, la1, p0, p1);
+      fadd2(lb0, lb1, lb0, lb1, p2, p3);
+      w[(i - 32 * c) / 2] = pack_bf16(p0, p1);
+      w[(i - 32 * c) / 2 + 1] = pack_bf16(p2, p3);
     }
     tmem_st16u(tS + 16 * c, w);
   }
-  return (l0 + l1) + (l2 + l3);
+  return (la0 + la1) + (lb0 + lb1);
 }
 
-// The row maximum of the raw scores of this warp's 32 rows of S_u (the scale is positive).
-__device__ __forceinline__ float pf_max(uint32_t tS, bool masked, int nvis) {
-  float m0 = -INFINITY, m1 = -INFINITY;
-  #pragma unroll
-  for (int c = 0; c < kPfN / 32; ++c) {
-    float v[32];
-    tmem_ld32(tS + 32 * c, v);
-    #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-      const bool vis0 = !masked || 32 * c + i < nvis, vis1 = !masked || 32 * c + i + 1 < nvis;
-      m0 = fmaxf(m0, vis0 ? v[i] : -INFINITY);
-      m1 = fmaxf(m1, vis1 ? v[i + 1] : -INFINITY);
-    }
-  }
-  return fmaxf(m0, m1);
+// 4-D tiled TMA store of a shared-memory box, tracked by this thread's bulk async-groups.
+__device__ __forceinline__ void pf_tma_store_4d(const CUtensorMap* map, const void* src, int x, int y, int z, int w) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(map),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "r"(w)
+               : "memory");
 }
+__device__ __forceinline__ void pf_bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's bulk groups are still reading shared memory.
+template <int N>
+__device__ __forceinline__ void pf_bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Waits until every bulk group of this thread has completed (its global writes performed).
+__device__ __forceinline__ void pf_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kPfThreads, 1)
-prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+               const __grid_constant__ CUtensorMap tmO) {
   using L = PfSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -211,7 +237,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
       }
       const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, has)) * 2u * 16u * 128u;
       int r = 1;
-      if (lane == 0) r = tc_wait(&bar[kPfKEmpty + st], eph, p.status, abort) ? 1 : 0;
+      if (lane == 0) r = tc_wait_suspend(&bar[kPfKEmpty + st], eph, p.status, abort) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, r, 0)) break;
       if (lane == 0) mbar_arrive_expect_tx(&bar[kPfKFull + st], bytes);
       __syncwarp();
@@ -222,7 +248,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
                       &bar[kPfKFull + st]);
       }
       ++nk;
-      if (lane == 0) r = tc_wait(&bar[kPfVEmpty + st], eph, p.status, abort) ? 1 : 0;
+      if (lane == 0) r = tc_wait_suspend(&bar[kPfVEmpty + st], eph, p.status, abort) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, r, 0)) break;
       if (lane == 0) mbar_arrive_expect_tx(&bar[kPfVFull + st], bytes);
       __syncwarp();
@@ -272,9 +298,9 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
         for (int k = 0; k < kPfN / 16; ++k)  // V advances 16 keys = 2 KB
           umma_f16_tmem_a(tO, tP + 8 * k, dV + (uint64_t)((k * 2048) >> 4), idO, (g > 0 || k > 0) ? 1u : 0u);
       };
-      bool ok = tc_wait(&bar[kPfQReady], 0, p.status, abort);
+      bool ok = tc_wait_suspend(&bar[kPfQReady], 0, p.status, abort);
       if (ok && nkb_max > 0) {
-        ok = tc_wait(&bar[kPfKFull], 0, p.status, abort);
+        ok = tc_wait_suspend(&bar[kPfKFull], 0, p.status, abort);
         if (ok) {
           tc_fence_after();
           if (nkb[0] > 0) issue_s(0, 0);
@@ -289,10 +315,10 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
         for (int u = 0; u < 2; ++u) {
           if (g >= nkb[u]) continue;
           if (!v_ready) {
-            if (!tc_wait(&bar[kPfVFull + st], (uint32_t)((g / kPfStages) & 1), p.status, abort)) { ok = false; break; }
+            if (!tc_wait_suspend(&bar[kPfVFull + st], (uint32_t)((g / kPfStages) & 1), p.status, abort)) { ok = false; break; }
             v_ready = true;
           }
-          if (!tc_wait(&bar[kPfPReady + u], (uint32_t)(g & 1), p.status, abort)) { ok = false; break; }
+          if (!tc_wait_suspend(&bar[kPfPReady + u], (uint32_t)(g & 1), p.status, abort)) { ok = false; break; }
           tc_fence_after();
           issue_pv(u, g);
           if (u == 1 || g >= nkb[1]) umma_commit(&bar[kPfVEmpty + st]);  // the block's last P V
@@ -300,7 +326,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
           if (g + 1 < nkb[u]) {
             const int sn = (g + 1) % kPfStages;
             if (!k_ready) {
-              if (!tc_wait(&bar[kPfKFull + sn], (uint32_t)(((g + 1) / kPfStages) & 1), p.status, abort)) {
+              if (!tc_wait_suspend(&bar[kPfKFull + sn], (uint32_t)(((g + 1) / kPfStages) & 1), p.status, abort)) {
                 ok = false;
                 break;
               }
@@ -349,19 +375,35 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
     float mref = -INFINITY, l = 0.f;  // reference maximum (log2 units) and row sum
     bool ok = true;
     for (int g = 0; g < nkb; ++g) {
-      if (!tc_wait_warp(&bar[kPfSFull + u], (uint32_t)(g & 1), p.status, abort)) { ok = false; break; }
+      if (!tc_wait_suspend_warp(&bar[kPfSFull + u], (uint32_t)(g & 1), p.status, abort)) { ok = false; break; }
       tc_fence_after();
       const int j0 = g * kPfN;
       const bool masked = j0 + kPfN - 1 > lim_min;  // warp-uniform: some row does not see every key
       const int nvis = lim - j0 + 1;                // keys j0 .. j0 + nvis - 1 are visible to the row
-      // the row maximum first; the reference moves when it is passed by more than 2^kPfTau
-      const float xmax = pf_max(tS, masked, nvis) * sc;
+      // the row's 128 scores in registers; keys past the row's limit are invisible
+      float v[128];
+      pf_ld128(tS, v);
+      if (masked) {
+        #pragma unroll
+        for (int i = 0; i < kPfN; ++i)
+          if (i >= nvis) v[i] = -INFINITY;
+      }
+      // the row maximum (the scale is positive); the reference moves when it is passed by more
+      // than 2^kPfTau
+      float m0 = -INFINITY, m1 = -INFINITY;
+      #pragma unroll
+      for (int i = 0; i < kPfN; i += 4) {
+        m0 = fmax3(m0, v[i], v[i + 1]);
+        m1 = fmax3(m1, v[i + 2], v[i + 3]);
+      }
+      const float xmax = fmaxf(m0, m1) * sc;
       float alpha = 1.f;
       if (xmax > mref + (float)kPfTau) {  // false when the row sees nothing here (xmax = -inf)
         alpha = mref == -INFINITY ? 0.f : fast_exp2(mref - xmax);
         l *= alpha;
         mref = xmax;
       }
+      l += pf_exp(tS, v, sc, mref);
       // O_u's rows hold every block before this one: S_u of this block was committed after the
       // previous P V, so that product is complete. Tensor-memory accesses are warp-wide: the warp
       // rescales when any of its rows moved (alpha = 1 for the others).
@@ -375,21 +417,25 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
           tmem_st32(tO + 32 * q4, o);
         }
       }
-      l += pf_exp(tS, sc, mref, masked, nvis);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[kPfPReady + u]);
     }
     // ---- epilogue: O / l and lse of row t
-    if (ok && nkb > 0 && !tc_wait_warp(&bar[kPfOFin + u], 0, p.status, abort)) ok = false;
+    if (ok && nkb > 0 && !tc_wait_suspend_warp(&bar[kPfOFin + u], 0, p.status, abort)) ok = false;
     if (!ok) *abort = 1;
     if (ok) {  // warp-uniform: every lane takes part in the tensor-memory loads
+      // O / l through shared memory: this warp's 32 rows, 32 columns at a time, into one of two
+      // 4 KB boxes in its tile's Q area (no tensor-core operation reads Q_u any more: they all
+      // completed before the tile's last P V), swizzled as the store's tensor map expects (row i
+      // at 128 i, 16-byte chunk c at (c ^ (i % 8)) * 16), then a TMA store of the box to
+      // out[b][t0w .. t0w + 31][qh][32 q4 ..]. Rows past T fall outside the map and are not written.
       tc_fence_after();
-      const bool has = t < p.T;
-      const int64_t row = ((int64_t)b * p.T + (has ? t : 0)) * p.Hq + qh;
-      float4* dst = reinterpret_cast<float4*>(p.out + row * kPfD);
+      const int t0w = t - lane;  // the warp's first row
+      const bool any_row = t0w < p.T;
       const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint8_t* stage = sm + L::OFF_Q + warp * 8192;
       #pragma unroll
       for (int q4 = 0; q4 < kPfD / 32; ++q4) {
         float o[32];
@@ -399,13 +445,25 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
           #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
         }
-        if (has) {
-          #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[8 * q4 + i] = make_float4(o[4 * i] * inv, o[4 * i + 1] * inv, o[4 * i + 2] * inv, o[4 * i + 3] * inv);
+        uint8_t* box = stage + (q4 & 1) * 4096;
+        if (q4 >= 2) {  // the store that read this box two chunks ago
+          if (lane == 0) pf_bulk_wait_read<1>();
+          __syncwarp();
+        }
+        #pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<float4*>(box + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+              make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv, o[4 * c + 3] * inv);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0 && any_row) {
+          pf_tma_store_4d(&tmO, box, 32 * q4, qh, t0w, b);
+          pf_bulk_commit();
         }
       }
-      if (has) p.lse[row] = l > 0.f ? (mref + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      if (lane == 0) pf_bulk_wait_all();
+      __syncwarp();
+      if (t < p.T) p.lse[((int64_t)b * p.T + t) * p.Hq + qh] = l > 0.f ? (mref + __log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
   }
 
@@ -416,7 +474,8 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kPfTmemCols) : "memory");
 }
 
-cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, cudaStream_t st) {
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                           const CUtensorMap& tmO, cudaStream_t st) {
   const int smem = PfSmem::ALLOC;
   if (!ensure_smem_attr((const void*)prefill_kernel, smem)) return cudaErrorInvalidValue;
   if (p.B == 0 || p.T == 0 || p.Hq == 0) return cudaSuccess;
@@ -427,7 +486,7 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const
   cfg.blockDim = dim3(kPfThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  return cudaLaunchKernelEx(&cfg, prefill_kernel, p, tmK, tmV);
+  return cudaLaunchKernelEx(&cfg, prefill_kernel, p, tmK, tmV, tmO);
 }
 
 }  // namespace decattn

@@ -169,6 +169,29 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, int
   return __all_sync(0xffffffffu, tc_wait(bar, parity, status, abort));
 }
 
+// A bounded wait that lets the hardware suspend the thread between checks
+// (mbarrier.try_wait: the thread resumes when the phase completes), for long waits in kernels
+// where a polling warp would take issue slots from the warps doing the work on its
+// sub-partition. Gives up like tc_wait.
+__device__ __forceinline__ bool tc_wait_suspend(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_status(status, DECATTN_ETIMEOUT);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ bool tc_wait_suspend_warp(uint64_t* bar, uint32_t parity, int32_t* status,
+                                                     volatile int* abort) {
+  return __all_sync(0xffffffffu, tc_wait_suspend(bar, parity, status, abort));
+}
+
 // Float -> integer with the same order (for warp max reductions with redux.sync).
 __device__ __forceinline__ int ordered_int(float f) {
   const int i = __float_as_int(f);
