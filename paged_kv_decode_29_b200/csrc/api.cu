@@ -77,6 +77,21 @@ static bool make_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int D,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Prefill queries as a 4-D bf16 tensor {head dim, q head, query row, request} (q is
+// [B][T][Hq][D]); the kernel loads boxes of 64 head dims x 128 rows with 128-byte swizzle, the
+// K-major layout of the MMA's A operand. Rows past T read as zeros.
+static bool make_prefill_q_map(CUtensorMap* map, const void* q, int B, int T, int Hq, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2, (cuuint64_t)T * Hq * D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Prefill output as a 4-D fp32 tensor {head dim, q head, query row, request} (out is
 // [B][T][Hq][D]); the kernel stores boxes of 32 rows x 32 head dims with 128-byte swizzle.
 // Rows past T are outside the map, so a partial tile's store writes only its own rows.
@@ -240,9 +255,10 @@ extern "C" int dec_attn_prefill(const dec_attn_shape* shape, const void* q, cons
   if (((reinterpret_cast<uintptr_t>(page_table) | reinterpret_cast<uintptr_t>(seq_lens) |
         reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(status)) & 3) != 0)
     return DECATTN_EALIGN;
-  CUtensorMap tmK, tmV, tmO;
+  CUtensorMap tmQ, tmK, tmV, tmO;
   const int64_t rows = (int64_t)s.num_pages * s.n_kv_heads * s.page_size;
-  if (!make_kv_map(&tmK, k_pages, s.kv_dtype, s.head_dim, rows) ||
+  if (!make_prefill_q_map(&tmQ, q, s.batch, s.q_tokens, s.n_q_heads, s.head_dim) ||
+      !make_kv_map(&tmK, k_pages, s.kv_dtype, s.head_dim, rows) ||
       !make_kv_map(&tmV, v_pages, s.kv_dtype, s.head_dim, rows) ||
       !make_prefill_out_map(&tmO, out, s.batch, s.q_tokens, s.n_q_heads, s.head_dim))
     return DECATTN_ECUDA;
@@ -257,7 +273,7 @@ extern "C" int dec_attn_prefill(const dec_attn_shape* shape, const void* q, cons
   p.B = s.batch; p.T = s.q_tokens; p.Hq = s.n_q_heads; p.Hkv = s.n_kv_heads; p.G = s.n_q_heads / s.n_kv_heads;
   p.P = s.page_size; p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
   p.qk_scale_log2 = scale * 1.4426950408889634f;
-  return launch_prefill(p, tmK, tmV, tmO, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DECATTN_OK
+  return launch_prefill(p, tmQ, tmK, tmV, tmO, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DECATTN_OK
                                                                                                : DECATTN_ECUDA;
 }
 

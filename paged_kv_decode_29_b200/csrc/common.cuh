@@ -447,7 +447,7 @@ bool split_tc_supported(int kv_dtype, int D, int GT);             // split_tc.cu
 cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int kv_dtype,
                             cudaStream_t st);                     // split_tc.cu
 cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st);  // combine.cu
-cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                           const CUtensorMap& tmO, cudaStream_t st);  // prefill.cu
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t st);  // prefill.cu
 
 }  // namespace decattn

@@ -16,9 +16,10 @@
 //  * online softmax with a per-row reference maximum that moves only when a score passes it by
 //    more than 2^kPfTau: P is computed in one pass against the current reference, and the pass
 //    is redone (after rescaling the row of O) only in the rare block that moves it.
-// CTA: 10 warps: 0-3 softmax of tile 0, 4-7 softmax of tile 1, 8 TMA producer (separate K and V
-// rings of two 128-key stages), 9 MMA issue (one thread). Every wait is bounded (DECATTN_ETIMEOUT,
-// then an orderly exit).
+// CTA: 10 warps: 0-3 softmax of tile 0, 4-7 softmax of tile 1, 8 TMA producer (Q of both tiles
+// first, then separate K and V rings of two 128-key stages), 9 MMA issue (one thread). The
+// epilogue stages O through the Q area and writes it with TMA stores. Every wait is bounded
+// (DECATTN_ETIMEOUT, then an orderly exit).
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -58,7 +59,7 @@ enum PfBar {
   kPfSFull = 8,    // [tile] MMA commit -> softmax: S_u of the next block in tensor memory
   kPfPReady = 10,  // [tile] 4 softmax warps -> MMA: P_u written (and rows of O_u rescaled)
   kPfOFin = 12,    // [tile] MMA commit after tile u's last P V -> softmax epilogue
-  kPfQReady = 14,  // 8 softmax warps -> MMA: Q of both tiles written
+  kPfQFull = 14,   // producer -> MMA: Q of both tiles landed (TMA)
   kPfDrain = 15,   // MMA commit -> MMA: every tensor-core operation complete
 };
 
@@ -130,6 +131,16 @@ __device__ __forceinline__ float pf_exp(uint32_t tS, const float (&v)[128], floa
   return (la0 + la1) + (lb0 + lb1);
 }
 
+// 4-D tiled TMA load into shared memory, completion signalled on an mbarrier.
+__device__ __forceinline__ void pf_tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                               uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 4-D tiled TMA store of a shared-memory box, tracked by this thread's bulk async-groups.
 __device__ __forceinline__ void pf_tma_store_4d(const CUtensorMap* map, const void* src, int x, int y, int z, int w) {
   asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(map),
@@ -146,8 +157,8 @@ __device__ __forceinline__ void pf_bulk_wait_read() {
 __device__ __forceinline__ void pf_bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kPfThreads, 1)
-prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const __grid_constant__ CUtensorMap tmO) {
+prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO) {
   using L = PfSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -181,11 +192,6 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
   const int h = tl0.qh / p.G;
   const int nkb_max = max(tl0.nkb, tl1.nkb);
 
-  // The K/V stages start zeroed: rows past a request's last page are never loaded, and their
-  // contents meet P = 0 in the MMA, so they must be finite.
-  for (int i = threadIdx.x; i < 2 * kPfStages * L::TILE / 16; i += kPfThreads)
-    reinterpret_cast<uint4*>(sm + L::OFF_K)[i] = make_uint4(0, 0, 0, 0);
-  fence_async_smem();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPfStages; ++s) {
       mbar_init(&bar[kPfKFull + s], 1);
@@ -198,7 +204,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
       mbar_init(&bar[kPfPReady + u], 4);
       mbar_init(&bar[kPfOFin + u], 1);
     }
-    mbar_init(&bar[kPfQReady], 8);
+    mbar_init(&bar[kPfQFull], 1);
     mbar_init(&bar[kPfDrain], 1);
     *abort = 0;
     if (Lb < 0) set_status(p.status, DECATTN_EDEVICE);
@@ -217,7 +223,19 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
 
   if (warp == 8) {
     // ===================================================================== producer
-    if (lane == 0) { prefetch_tensormap(&tmK); prefetch_tensormap(&tmV); }
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      // Q of both tiles: per tile two boxes of 64 head dims x 128 rows, which land as the two
+      // K-major 128-byte-swizzled atoms the MMA reads; rows past T read as zeros
+      mbar_arrive_expect_tx(&bar[kPfQFull], 4u * (uint32_t)L::ATOM);
+      #pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        pf_tma_load_4d(sm + L::OFF_Q + a * L::ATOM, &tmQ, 64 * a, tl0.qh, tl0.t0, b, &bar[kPfQFull]);
+        pf_tma_load_4d(sm + L::OFF_Q + L::TILE + a * L::ATOM, &tmQ, 64 * a, tl1.qh, tl1.t0, b, &bar[kPfQFull]);
+      }
+    }
     int nk = 0, nv = 0;  // K / V blocks whose copies were issued
     for (int g = 0; g < nkb_max; ++g) {
       const int st = g % kPfStages;
@@ -250,6 +268,15 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
       ++nk;
       if (lane == 0) r = tc_wait_suspend(&bar[kPfVEmpty + st], eph, p.status, abort) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, r, 0)) break;
+      if (lane < kPfN / 16 && !has) {
+        // keys past the request's end: no copy; their P is 0, so their V rows must be finite
+        uint8_t* vt = sm + L::OFF_V + st * L::TILE + lane * 16 * 128;
+        #pragma unroll 4
+        for (int i = 0; i < 2 * 16 * 128 / 16; ++i)
+          reinterpret_cast<uint4*>(vt + (i >> 7) * L::ATOM)[i & 127] = make_uint4(0, 0, 0, 0);
+        fence_async_smem();
+      }
+      __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(&bar[kPfVFull + st], bytes);
       __syncwarp();
       if (has) {
@@ -298,7 +325,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
         for (int k = 0; k < kPfN / 16; ++k)  // V advances 16 keys = 2 KB
           umma_f16_tmem_a(tO, tP + 8 * k, dV + (uint64_t)((k * 2048) >> 4), idO, (g > 0 || k > 0) ? 1u : 0u);
       };
-      bool ok = tc_wait_suspend(&bar[kPfQReady], 0, p.status, abort);
+      bool ok = tc_wait_suspend(&bar[kPfQFull], 0, p.status, abort);
       if (ok && nkb_max > 0) {
         ok = tc_wait_suspend(&bar[kPfKFull], 0, p.status, abort);
         if (ok) {
@@ -353,22 +380,6 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
     const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
     const uint32_t tS = tmem + lane_off + kPfN * u;
     const uint32_t tO = tmem + lane_off + 2 * kPfN + kPfD * u;
-    // ---- Q row t into its K-major swizzled place (zero past T)
-    {
-      uint4 x[16];
-      const bool has = t < p.T;
-      const uint4* src = reinterpret_cast<const uint4*>(p.q + (((int64_t)b * p.T + (has ? t : 0)) * p.Hq + qh) * kPfD);
-      #pragma unroll
-      for (int c = 0; c < 16; ++c) x[c] = has ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-      uint8_t* q_sm = sm + L::OFF_Q + u * L::TILE;
-      #pragma unroll
-      for (int c = 0; c < 16; ++c)  // chunk c: head dims 8c .. 8c + 7
-        *reinterpret_cast<uint4*>(q_sm + (c >> 3) * L::ATOM + r * 128 + (((c & 7) ^ (r & 7)) << 4)) = x[c];
-    }
-    fence_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bar[kPfQReady]);
-
     const int lim = t < p.T ? Lb - p.T + t : -1;  // the last key this row sees (< 0: none)
     const int lim_min = __reduce_min_sync(0xffffffffu, lim);
     const float sc = p.qk_scale_log2;
@@ -474,8 +485,8 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK, c
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kPfTmemCols) : "memory");
 }
 
-cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                           const CUtensorMap& tmO, cudaStream_t st) {
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t st) {
   const int smem = PfSmem::ALLOC;
   if (!ensure_smem_attr((const void*)prefill_kernel, smem)) return cudaErrorInvalidValue;
   if (p.B == 0 || p.T == 0 || p.Hq == 0) return cudaSuccess;
@@ -486,7 +497,7 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmK, const
   cfg.blockDim = dim3(kPfThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  return cudaLaunchKernelEx(&cfg, prefill_kernel, p, tmK, tmV, tmO);
+  return cudaLaunchKernelEx(&cfg, prefill_kernel, p, tmQ, tmK, tmV, tmO);
 }
 
 }  // namespace decattn
