@@ -18,10 +18,10 @@ import workloads as W  # noqa: E402
 
 # workload -> (requests captured, dram read bytes, dram write bytes) of the captured launch
 CAPTURED = {
-    "uniform": (8, 134364672, 3204352),
-    "mixed": (16, 1039151360, 17712384),
-    "fp8_spec": (4, 167202048, 7321088),
-    "long_b4": (1, 536968704, 5867520),
+    "uniform": (8, 134362368, 3598080),
+    "mixed": (16, 1039144960, 17676288),
+    "fp8_spec": (4, 167250432, 6338304),
+    "long_b4": (1, 536982272, 5664256),
 }
 
 
