@@ -299,7 +299,11 @@ DECATTN_API int dec_attn_append_rope(const dec_attn_shape *shape, const void *q_
  * 0 .. seq_lens[b] - T + t (the decode's bottom-right causal rule; rows before position 0 see
  * nothing and get out = 0, lse = -inf). Output as dec_attn_run (out fp32 [B][T][Hq][128], lse
  * natural log [B][T][Hq]); no plan and no workspace. Runs on tcgen05 tensor cores: one CTA per
- * (request, q head, 128 query rows), 128-key blocks of K and V by TMA.
+ * two tiles of 128 query rows that read the same keys (two q heads of one KV head when
+ * n_q_heads / n_kv_heads is even, else two adjacent row blocks of one head); q, K and V arrive by
+ * TMA in 128-key blocks, and out is written by TMA stores (so q and out need the 16-byte
+ * alignment below; their rows are 256 and 512 bytes). Rows of a request are independent of the
+ * other requests: no cross-request state.
  *   shape       batch, n_q_heads, n_kv_heads, head_dim (128), q_tokens (T >= 1), page_size (a
  *               multiple of 16), num_pages, max_pages_per_seq, kv_dtype (DECATTN_KV_BF16),
  *               sm_scale (0: 1/sqrt(head_dim));

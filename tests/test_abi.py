@@ -150,3 +150,30 @@ def test_append_rope_rejects_bad_args(lib):
     assert _append(lib, s, kp=FAKE + 2) == da.EALIGN
     assert _append(lib, _shape(batch=0), qn=None, kn=None, vn=None, tab=None, lens=None, qo=None, kp=None,
                    vp=None) == da.OK
+
+
+def _prefill(lib, s, **ptrs):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, tab=FAKE, lens=FAKE, out=FAKE, lse=FAKE, st=None)
+    a.update(ptrs)
+    return lib.dec_attn_prefill(C.byref(s), a["q"], a["k"], a["v"], a["tab"], a["lens"], a["out"], a["lse"], a["st"],
+                                None)
+
+
+def test_prefill_rejects_bad_args(lib):
+    # every case fails a host check before any tensor map is built or a kernel launched
+    s = _shape(q_tokens=300)
+    assert lib.dec_attn_prefill(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == da.EINVAL
+    assert _prefill(lib, _shape(q_tokens=0)) == da.EINVAL
+    assert _prefill(lib, _shape(batch=-1)) == da.EINVAL
+    assert _prefill(lib, _shape(n_q_heads=6, n_kv_heads=4)) == da.EINVAL
+    assert _prefill(lib, _shape(kv_dtype=da.KV_FP8E4M3)) == da.ENOTSUP   # bf16 pages only
+    assert _prefill(lib, _shape(head_dim=64)) == da.ENOTSUP
+    assert _prefill(lib, _shape(page_size=8)) == da.ENOTSUP
+    for name in ("q", "k", "v", "tab", "lens", "out", "lse"):
+        assert _prefill(lib, s, **{name: None}) == da.EINVAL
+    assert _prefill(lib, s, q=FAKE + 8) == da.EALIGN
+    assert _prefill(lib, s, out=FAKE + 4) == da.EALIGN
+    assert _prefill(lib, s, lse=FAKE + 2) == da.EALIGN
+    assert _prefill(lib, s, st=FAKE + 1) == da.EALIGN
+    assert _prefill(lib, _shape(batch=0, q_tokens=300), q=None, k=None, v=None, tab=None, lens=None, out=None,
+                    lse=None) == da.OK
