@@ -572,6 +572,21 @@ def measured_tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def prefill_traffic():
+    """DRAM bytes per prefill-kernel launch from the committed ncu capture, if it was taken on the
+    current kernel source (else None)."""
+    try:
+        d = json.load(open(os.path.join(ROOT, "profiles", "prefill_kernel_dram_traffic.json")))
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for f in ("prefill.cu", "tc.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "paged_kv_decode_29_b200", "csrc", f), "rb").read())
+    if d.get("source_hash") != h.hexdigest()[:16]:
+        return None
+    return int(d["configs"]["prefill"]["bytes_per_launch"])
+
+
 def prefill_flops(pr) -> int:
     """Algorithmic FLOPs of causal prefill: row t of request b sees L_b - T + t + 1 keys (none
     when that is <= 0), and each key costs 2 d for q.k and 2 d for p v."""
@@ -696,7 +711,8 @@ def run_prefill(args, rank: int, world: int, local_rank: int, dist):
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "algorithmic_flops": flops,
         "roofline": {"bound": "tensor", "kernel": "prefill_kernel", "achieved": round(tflops, 1), "peak": peak,
-                     "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None},
+                     "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                     "traffic": prefill_traffic() if pr.name == "prefill" else None},
         "gpu_launches": args.steps,  # one prefill kernel per timed step
     }
     if sampler:

@@ -4,6 +4,8 @@ by the ratio of algorithmic bytes. Reads measured within 0.05% of the algorithmi
 captured case, so traffic grows in proportion. The figures below are the captured ncu values
 (`dram__bytes_read.sum`, `dram__bytes_write.sum`) of one split-kernel launch of each smaller case (the split kernel that runs for the workload: split_tc_kernel for fp8_spec,
 split_kernel for the others).
+It also writes prefill_kernel_dram_traffic.json: the prefill kernel's DRAM bytes per launch on
+the full prefill workload, captured directly (the workload holds a few hundred MB on the device).
 Run from the repository root after the capture: python profiles/make_traffic_json.py"""
 import hashlib
 import json
@@ -23,6 +25,11 @@ CAPTURED = {
     "fp8_spec": (4, 167250432, 6338304),
     "long_b4": (1, 536982272, 5664256),
 }
+
+
+# prefill_kernel on the full prefill workload (dram read bytes, dram write bytes) of the launch
+# captured by `ncu --set full` (profiles/prefill_kernel_prefill_b4.md)
+PREFILL_CAPTURED = (108316928, 87724800)
 
 
 def alg_bytes(name, batch=None):
@@ -50,6 +57,13 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
+def prefill_source_hash():
+    h = hashlib.sha256()
+    for f in ("prefill.cu", "tc.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "paged_kv_decode_29_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def main():
     out = {"source_hash": source_hash(), "configs": {}}
     for name, (nb, rd, wr) in CAPTURED.items():
@@ -65,6 +79,11 @@ def main():
     with open(p, "w") as f:
         json.dump(out, f, indent=1)
     print(json.dumps(out, indent=1))
+    rd, wr = PREFILL_CAPTURED
+    pf = {"source_hash": prefill_source_hash(),
+          "configs": {"prefill": {"bytes_per_launch": rd + wr, "captured_read": rd, "captured_write": wr}}}
+    with open(os.path.join(ROOT, "profiles", "prefill_kernel_dram_traffic.json"), "w") as f:
+        json.dump(pf, f, indent=1)
 
 
 if __name__ == "__main__":
