@@ -60,6 +60,7 @@ def _check(pr, out, lse, ref_o, ref_l, rows, what):
     ([90, 400, 131], 130, 8, 1, 16), # T > L for one request (its first rows see nothing), G = 8
     ([513], 385, 4, 4, 32),          # keys and rows not multiples of the block
     ([700, 333], 300, 6, 2, 16),     # G = 3: adjacent row blocks paired, the last pair's second past T
+    ([900, 640], 640, 64, 8, 16),    # 320 tile pairs: more than one per CTA on any current GPU
 ])
 def test_prefill_matches_oracle(lens, T, Hq, Hkv, P):
     pr = _problem(lens, T=T, Hq=Hq, Hkv=Hkv, P=P)
