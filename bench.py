@@ -91,6 +91,17 @@ def parse():
 
 # ---------------------------------------------------------------- helpers
 
+def max_over_ranks(vals, dist, device):
+    """Element-wise maximum of a list of floats over all ranks (the list itself without a process
+    group). Every rank must call it at the same point: it is one collective."""
+    if dist is None:
+        return [float(x) for x in vals]
+    import torch
+    t = torch.tensor([float(x) for x in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def measured_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -417,11 +428,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
     if st != da.OK:
         raise RuntimeError(f"device status after timing: {da.status_string(st)}")
     local = [mean(step_us), mean(plan_us), mean(split_us), mean(comb_us), mean(app_us)]
-    if dist is not None:
-        t = torch.tensor(local, dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        local = t.tolist()
-    step_m, plan_m, split_m, comb_m, app_m = local
+    step_m, plan_m, split_m, comb_m, app_m = max_over_ranks(local, dist, dev)
 
     # CUDA-graph replay of the same step (context figure)
     graph_us = None
@@ -488,11 +495,7 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
             b_.synchronize()
             if i >= args.warmup:
                 et.append(a.elapsed_time(b_) * 1e3)
-        e2e_local = mean(et)
-        if dist is not None:
-            t = torch.tensor([e2e_local], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_local = t.item()
+        e2e_local = max_over_ranks([mean(et)], dist, dev)[0]
         e2e = {"value": round(e2e_local, 3), "unit": "us/step", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h),
                "note": ("per step: the new q/k/v rows" if args.append else "per step: q") +
@@ -688,14 +691,12 @@ def run_prefill(args, rank: int, world: int, local_rank: int, dist):
             b_.synchronize()
             if i >= args.warmup:
                 et.append(a.elapsed_time(b_) * 1e3)
-        e2e = {"value": round(statistics.mean(et), 3), "unit": "us/step", "h2d_bytes_per_step": int(h2d),
+        e2e = {"value": round(max_over_ranks([statistics.mean(et)], dist, dev)[0], 3), "unit": "us/step",
+               "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h),
                "note": "per step: q, page table and seq_lens from pinned host memory, prefill, out and lse back "
                        "to pinned host memory; the KV cache stays resident in HBM"}
-    if dist is not None:
-        t = torch.tensor([step_m], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_m = t.item()
+    step_m = max_over_ranks([step_m], dist, dev)[0]
     if rank != 0:
         return 0
     flops = prefill_flops(pr)
