@@ -1,0 +1,67 @@
+"""bench.py's host-side arithmetic on CPU: the algorithmic FLOPs behind the prefill roofline, which
+split kernel a workload runs on, and the rule that an ncu traffic figure is reported only while
+the kernel sources hash as they did at the capture."""
+import json
+import os
+import shutil
+
+import numpy as np
+
+import bench
+import workloads as W
+
+
+class _Pr:
+    def __init__(self, lens, T, Hq, d=128):
+        self.seq_lens = np.asarray(lens, dtype=np.int32)
+        self.q_tokens, self.n_q_heads, self.head_dim = T, Hq, d
+
+
+def test_prefill_flops_closed_forms():
+    # T = L: row t sees t + 1 keys, sum = T (T + 1) / 2; each (row, key) costs 4 d per head
+    assert bench.prefill_flops(_Pr([2048] * 4, 2048, 32)) == 4 * 32 * 4 * 128 * 2048 * 2049 // 2
+    # L > T: row t sees L - T + t + 1 keys
+    L, T = 1000, 10
+    assert bench.prefill_flops(_Pr([L], T, 1)) == 4 * 128 * sum(L - T + t + 1 for t in range(T))
+    # L < T: the first T - L rows see nothing
+    assert bench.prefill_flops(_Pr([3], 5, 2)) == 4 * 2 * 128 * (0 + 0 + 1 + 2 + 3)
+    # the full prefill workload: 137.5 GFLOP
+    pr = _Pr(W.config_seq_lens("prefill"), W.CONFIGS["prefill"]["q_tokens"], W.CONFIGS["prefill"]["n_q_heads"])
+    assert abs(bench.prefill_flops(pr) / 1e9 - 137.506062336) < 1e-6
+
+
+def test_split_kernel_name():
+    class P:
+        pass
+
+    p = P()
+    p.kv_dtype, p.head_dim, p.group, p.q_tokens = "fp8e4m3", 128, 4, 4
+    assert bench.split_kernel_name(p) == "split_tc_kernel"
+    p.q_tokens = 5  # G*T = 20 > 16
+    assert bench.split_kernel_name(p) == "split_kernel"
+    p.kv_dtype, p.q_tokens = "bf16", 1
+    assert bench.split_kernel_name(p) == "split_kernel"
+    p.kv_dtype, p.head_dim = "fp8e4m3", 64
+    assert bench.split_kernel_name(p) == "split_kernel"
+
+
+def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
+    # the committed captures match the committed sources
+    assert bench.ncu_traffic("uniform", 256) is not None
+    assert bench.prefill_traffic() is not None
+    # a copy of the tree whose kernel sources differ by one byte reports none
+    root = tmp_path / "repo"
+    shutil.copytree(os.path.join(bench.ROOT, "profiles"), root / "profiles")
+    shutil.copytree(os.path.join(bench.ROOT, "paged_kv_decode_29_b200", "csrc"),
+                    root / "paged_kv_decode_29_b200" / "csrc")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.ncu_traffic("uniform", 256) is not None
+    assert bench.prefill_traffic() is not None
+    for f in ("split.cu", "prefill.cu"):
+        path = root / "paged_kv_decode_29_b200" / "csrc" / f
+        path.write_bytes(path.read_bytes() + b"\n")
+    assert bench.ncu_traffic("uniform", 256) is None
+    assert bench.prefill_traffic() is None
+    # a tile length that was not captured has no figure
+    d = json.load(open(root / "profiles" / "split_kernel_dram_traffic.json"))
+    assert "uniform/tl128" not in d["configs"]
