@@ -254,6 +254,12 @@ DECATTN_API int dec_attn_combine(const dec_attn_shape *shape, const void *q, con
  * hot path. */
 DECATTN_API int dec_attn_read_status(const dec_attn_plan_t *plan, const void *workspace, void *stream);
 
+/* The CUDA error behind the last DECATTN_ECUDA returned on the calling host thread: the failing
+ * step and CUDA's error string, e.g. "prefill kernel launch: too many resources requested for
+ * launch". Writes at most len - 1 characters and a terminating zero into buf (NULL: nothing
+ * written); returns the full message length (0: no DECATTN_ECUDA on this thread yet). Host only. */
+DECATTN_API size_t dec_attn_last_error(char *buf, size_t len);
+
 /* Static text for a decattn_status value. */
 DECATTN_API const char *dec_attn_status_string(int status);
 

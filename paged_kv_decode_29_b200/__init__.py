@@ -29,14 +29,19 @@ KV_BF16, KV_FP8E4M3, KV_FP8E4M3_MMA8 = 0, 1, 2
 API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
        "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_prefill", "dec_attn_plan_sparse_bytes",
-       "dec_attn_plan_sparse")
+       "dec_attn_plan_sparse", "dec_attn_last_error")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class DecAttnError(RuntimeError):
     def __init__(self, code: int, what: str = ""):
         self.code = code
-        super().__init__(f"{what}: {status_string(code)} ({code})" if what else f"{status_string(code)} ({code})")
+        msg = f"{what}: {status_string(code)} ({code})" if what else f"{status_string(code)} ({code})"
+        if code == ECUDA:
+            detail = last_error()
+            if detail:
+                msg += f" [{detail}]"
+        super().__init__(msg)
 
 
 class PlanT(C.Structure):
@@ -86,6 +91,8 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_read_status.restype = i32
         lib.dec_attn_status_string.argtypes = [i32]
         lib.dec_attn_status_string.restype = C.c_char_p
+        lib.dec_attn_last_error.argtypes = [C.c_char_p, sz]
+        lib.dec_attn_last_error.restype = sz
         lib.dec_attn_append_rope.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, C.c_float, vp, vp, vp, vp, vp]
         lib.dec_attn_plan_sparse_bytes.argtypes = [i32, i32, i32, i64, i32]
         lib.dec_attn_plan_sparse_bytes.restype = sz
@@ -100,6 +107,17 @@ def load_library(path: str = LIB_PATH):
 
 def status_string(code: int) -> str:
     return load_library().dec_attn_status_string(int(code)).decode()
+
+
+def last_error() -> str:
+    """dec_attn_last_error: the failing step and CUDA error behind this thread's last ECUDA ('' if none)."""
+    lib = load_library()
+    n = int(lib.dec_attn_last_error(None, 0))
+    if n == 0:
+        return ""
+    buf = C.create_string_buffer(n + 1)
+    lib.dec_attn_last_error(buf, n + 1)
+    return buf.value.decode(errors="replace")
 
 
 def _stream_handle(stream) -> int | None:

@@ -3,6 +3,8 @@
 #include <math.h>
 #include <stddef.h>
 
+#include <cstdio>
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -12,6 +14,16 @@
 namespace decattn {
 
 static std::mutex g_mu;
+
+// The CUDA error behind the last DECATTN_ECUDA of this host thread (dec_attn_last_error).
+static thread_local char g_last_error[256] = "";
+
+int cuda_fail(const char* what, cudaError_t e) {
+  if (e == cudaSuccess) e = cudaPeekAtLastError();
+  snprintf(g_last_error, sizeof g_last_error, "%s: %s", what,
+           e == cudaSuccess ? "failed without a CUDA runtime error (a driver-API call)" : cudaGetErrorString(e));
+  return DECATTN_ECUDA;
+}
 
 int default_bins(int device) {
   static std::map<int, int> cache;
@@ -181,7 +193,7 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
   if ((int64_t)workspace_bytes < wl.total) return DECATTN_ESMALL;
   if (wl.items >= (1ll << 31)) return DECATTN_ENOTSUP;  // the combine numbers its items in 32 bits
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return DECATTN_ECUDA;
+  if (const cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
 
   char* ws = static_cast<char*>(workspace);
   int32_t* row_cnt = reinterpret_cast<int32_t*>(ws + wl.off_row_cnt);
@@ -193,7 +205,7 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
     CUtensorMap tmK, tmV;
     const int64_t rows = (int64_t)s.num_pages * s.n_kv_heads * s.page_size;
     if (!make_kv_map(&tmK, k_pages, s.kv_dtype, D, rows) || !make_kv_map(&tmV, v_pages, s.kv_dtype, D, rows))
-      return DECATTN_ECUDA;
+      return cuda_fail("K/V tensor map (cuTensorMapEncodeTiled)");
     const float scale = s.sm_scale > 0.f ? s.sm_scale : 1.0f / sqrtf((float)D);
     SplitParams sp;
     sp.q = static_cast<const uint16_t*>(q);
@@ -211,7 +223,8 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
     sp.P = s.page_size; sp.num_pages = s.num_pages; sp.mpps = s.max_pages_per_seq; sp.n_bins = plan->n_bins;
     sp.tile_len = plan->tile_len; sp.max_units = plan->max_units; sp.sparse = plan->sparse;
     sp.qk_scale_log2 = scale * 1.4426950408889634f;
-    if (launch_split(sp, tmK, tmV, s.kv_dtype, D, st) != cudaSuccess) return DECATTN_ECUDA;
+    if (const cudaError_t e = launch_split(sp, tmK, tmV, s.kv_dtype, D, st); e != cudaSuccess)
+      return cuda_fail("split kernel launch", e);
   }
   if (stages & kStageCombine) {
     CombineParams cp;
@@ -226,7 +239,7 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
     cp.B = s.batch; cp.T = s.q_tokens; cp.Hq = s.n_q_heads; cp.Hkv = s.n_kv_heads; cp.G = G; cp.GT = GT; cp.D = D;
     cp.tl = plan->tile_len;
     cp.sparse = plan->sparse;
-    if (launch_combine(cp, dev, st) != cudaSuccess) return DECATTN_ECUDA;
+    if (const cudaError_t e = launch_combine(cp, dev, st); e != cudaSuccess) return cuda_fail("combine kernel launch", e);
   }
   return DECATTN_OK;
 }
@@ -261,7 +274,7 @@ extern "C" int dec_attn_prefill(const dec_attn_shape* shape, const void* q, cons
       !make_kv_map(&tmK, k_pages, s.kv_dtype, s.head_dim, rows) ||
       !make_kv_map(&tmV, v_pages, s.kv_dtype, s.head_dim, rows) ||
       !make_prefill_out_map(&tmO, out, s.batch, s.q_tokens, s.n_q_heads, s.head_dim))
-    return DECATTN_ECUDA;
+    return cuda_fail("prefill tensor maps (cuTensorMapEncodeTiled)");
   const float scale = s.sm_scale > 0.f ? s.sm_scale : 1.0f / sqrtf((float)s.head_dim);
   PrefillParams p;
   p.q = static_cast<const uint16_t*>(q);
@@ -273,8 +286,8 @@ extern "C" int dec_attn_prefill(const dec_attn_shape* shape, const void* q, cons
   p.B = s.batch; p.T = s.q_tokens; p.Hq = s.n_q_heads; p.Hkv = s.n_kv_heads; p.G = s.n_q_heads / s.n_kv_heads;
   p.P = s.page_size; p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
   p.qk_scale_log2 = scale * 1.4426950408889634f;
-  return launch_prefill(p, tmQ, tmK, tmV, tmO, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DECATTN_OK
-                                                                                               : DECATTN_ECUDA;
+  const cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, tmO, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DECATTN_OK : cuda_fail("prefill kernel launch", e);
 }
 
 extern "C" int dec_attn_default_bins(int device) { return default_bins(device); }
@@ -310,16 +323,27 @@ extern "C" int dec_attn_combine(const dec_attn_shape* shape, const void* q, cons
 
 extern "C" int dec_attn_read_status(const dec_attn_plan_t* plan, const void* workspace, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(st) != cudaSuccess) return DECATTN_ECUDA;
+  if (const cudaError_t e = cudaStreamSynchronize(st); e != cudaSuccess) return cuda_fail("cudaStreamSynchronize", e);
   (void)workspace;  // device errors of a run are recorded in the plan buffer's header
   if (plan && plan->buf) {
     PlanHeader h;
-    if (cudaMemcpy(&h, plan->buf, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return DECATTN_ECUDA;
+    if (const cudaError_t e = cudaMemcpy(&h, plan->buf, sizeof h, cudaMemcpyDeviceToHost); e != cudaSuccess)
+      return cuda_fail("plan header copy", e);
     if (h.magic != kPlanMagic) return DECATTN_EINVAL;
     if (h.status != DECATTN_OK) return h.status;
     if (h.run_status != DECATTN_OK) return h.run_status;
   }
   return DECATTN_OK;
+}
+
+extern "C" size_t dec_attn_last_error(char* buf, size_t len) {
+  const size_t n = strlen(g_last_error);
+  if (buf && len > 0) {
+    const size_t k = n < len - 1 ? n : len - 1;
+    memcpy(buf, g_last_error, k);
+    buf[k] = 0;
+  }
+  return n;
 }
 
 extern "C" const char* dec_attn_status_string(int status) {

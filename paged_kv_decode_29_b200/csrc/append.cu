@@ -182,5 +182,5 @@ extern "C" int dec_attn_append_rope(const dec_attn_shape* shape, const void* q_n
   for (int i = 0; i < s.head_dim / 2; ++i) p.theta[i] = std::pow((double)rope_base, -2.0 * i / s.head_dim);
   if ((int64_t)s.batch * s.q_tokens * p.groups > 0x7fffffff) return DECATTN_ENOTSUP;
   const cudaError_t e = launch_append(p, s.head_dim, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? DECATTN_OK : DECATTN_ECUDA;
+  return e == cudaSuccess ? DECATTN_OK : cuda_fail("append kernel launch", e);
 }

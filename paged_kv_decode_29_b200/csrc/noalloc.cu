@@ -36,11 +36,13 @@ void* g_noalloc_ptr[kMaxDevices] = {};
 // Device address of g_noalloc_scratch on the current device (looked up once per device).
 int noalloc_scratch(void** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DECATTN_ECUDA;
+  if (const cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  if (dev < 0 || dev >= kMaxDevices) return cuda_fail("device ordinal beyond the scratch table", cudaErrorInvalidDevice);
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
   if (!g_noalloc_ptr[dev]) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return DECATTN_ECUDA;
+    if (const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch); e != cudaSuccess || !ptr)
+      return cuda_fail("scratch address (cudaGetSymbolAddress)", e == cudaSuccess ? cudaErrorInvalidSymbol : e);
     g_noalloc_ptr[dev] = ptr;
   }
   *out = g_noalloc_ptr[dev];

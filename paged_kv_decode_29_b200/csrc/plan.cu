@@ -810,9 +810,9 @@ extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads,
   if (!plan || !plan_buf || (batch > 0 && !seq_lens)) return DECATTN_EINVAL;
   if (n_bins == 0) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return DECATTN_ECUDA;
+    if (const cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
     n_bins = default_bins(dev);
-    if (n_bins <= 0) return DECATTN_ECUDA;
+    if (n_bins <= 0) return cuda_fail("SM count (cudaDeviceGetAttribute)");
   }
   if (batch < 0 || n_kv_heads <= 0 || tile_len <= 0 || max_total_kv_tokens < 0 || n_bins < 0) return DECATTN_EINVAL;
   if (!plan_args_ok(batch, n_kv_heads, tile_len, max_total_kv_tokens, n_bins)) return DECATTN_ENOTSUP;
@@ -843,7 +843,7 @@ extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads,
     h.gsm_off = (int32_t)smem;
     smem += (size_t)gsm;
   }
-  if (!ensure_smem_attr((const void*)plan_kernel, kPlanMaxSmem)) return DECATTN_ECUDA;
+  if (!ensure_smem_attr((const void*)plan_kernel, kPlanMaxSmem)) return cuda_fail("planner shared-memory attribute");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(kPlanThreads);
@@ -854,8 +854,9 @@ extern "C" int dec_attn_plan(const int32_t* seq_lens, int batch, int n_kv_heads,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, plan_kernel, seq_lens, h, static_cast<char*>(plan_buf)) != cudaSuccess)
-    return DECATTN_ECUDA;
+  if (const cudaError_t e = cudaLaunchKernelEx(&cfg, plan_kernel, seq_lens, h, static_cast<char*>(plan_buf));
+      e != cudaSuccess)
+    return cuda_fail("planner launch", e);
   plan->buf = plan_buf;
   plan->buf_bytes = plan_bytes;
   plan->batch = batch;
@@ -873,7 +874,8 @@ extern "C" int dec_attn_plan_export(const dec_attn_plan_t* plan, const int32_t* 
     return DECATTN_EINVAL;
   plan_export_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const char*>(plan->buf), seq_lens, bin_off, static_cast<Unit*>(units), max_units, n_units);
-  return cudaGetLastError() == cudaSuccess ? DECATTN_OK : DECATTN_ECUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? DECATTN_OK : cuda_fail("plan export launch", e);
 }
 
 // ------------------------------------------------------------------ block-sparse plan (host)
@@ -920,9 +922,9 @@ extern "C" int dec_attn_plan_sparse(const int32_t* seq_lens, const uint32_t* til
   if (!plan || !plan_buf || (batch > 0 && (!seq_lens || !tile_mask)) || mask_words <= 0) return DECATTN_EINVAL;
   if (n_bins == 0) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return DECATTN_ECUDA;
+    if (const cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
     n_bins = default_bins(dev);
-    if (n_bins <= 0) return DECATTN_ECUDA;
+    if (n_bins <= 0) return cuda_fail("SM count (cudaDeviceGetAttribute)");
   }
   if (batch < 0 || n_kv_heads <= 0 || tile_len <= 0 || max_total_kv_tokens < 0 || n_bins < 0) return DECATTN_EINVAL;
   if (!plan_args_ok(batch, n_kv_heads, tile_len, max_total_kv_tokens, n_bins)) return DECATTN_ENOTSUP;
@@ -956,7 +958,7 @@ extern "C" int dec_attn_plan_sparse(const int32_t* seq_lens, const uint32_t* til
     h.gsm_off = (int32_t)smem;
     smem += (size_t)gsm;
   }
-  if (!ensure_smem_attr((const void*)plan_sparse_kernel, kPlanMaxSmem)) return DECATTN_ECUDA;
+  if (!ensure_smem_attr((const void*)plan_sparse_kernel, kPlanMaxSmem)) return cuda_fail("sparse planner shared-memory attribute");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(1);
   cfg.blockDim = dim3(kPlanThreads);
@@ -967,9 +969,10 @@ extern "C" int dec_attn_plan_sparse(const int32_t* seq_lens, const uint32_t* til
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, plan_sparse_kernel, seq_lens, tile_mask, mask_words, h,
-                         static_cast<char*>(plan_buf)) != cudaSuccess)
-    return DECATTN_ECUDA;
+  if (const cudaError_t e = cudaLaunchKernelEx(&cfg, plan_sparse_kernel, seq_lens, tile_mask, mask_words, h,
+                                               static_cast<char*>(plan_buf));
+      e != cudaSuccess)
+    return cuda_fail("sparse planner launch", e);
   plan->buf = plan_buf;
   plan->buf_bytes = plan_bytes;
   plan->batch = batch;

@@ -177,3 +177,32 @@ def test_prefill_rejects_bad_args(lib):
     assert _prefill(lib, s, st=FAKE + 1) == da.EALIGN
     assert _prefill(lib, _shape(batch=0, q_tokens=300), q=None, k=None, v=None, tab=None, lens=None, out=None,
                     lse=None) == da.OK
+
+
+def _no_usable_gpu():
+    import torch
+
+    return not torch.cuda.is_available()
+
+
+@pytest.mark.skipif(not _no_usable_gpu(), reason="makes a CUDA call fail, which needs a host without a usable GPU")
+def test_last_error_names_the_failing_step(lib):
+    import threading
+
+    # no device: the stream synchronisation fails and the step is recorded with CUDA's message
+    assert lib.dec_attn_read_status(None, None, None) == da.ECUDA
+    msg = da.last_error()
+    assert msg.startswith("cudaStreamSynchronize: ") and len(msg) > len("cudaStreamSynchronize: ")
+    # truncation: len counts the terminating zero; the full length is returned
+    buf = C.create_string_buffer(8)
+    assert lib.dec_attn_last_error(buf, 8) == len(msg)
+    assert buf.value.decode() == msg[:7]
+    assert lib.dec_attn_last_error(None, 0) == len(msg)
+    # the binding's exception carries the detail
+    assert "[cudaStreamSynchronize: " in str(da.DecAttnError(da.ECUDA, "dec_attn_read_status"))
+    # per host thread: a fresh thread has no error recorded
+    seen = []
+    t = threading.Thread(target=lambda: seen.append(da.last_error()))
+    t.start()
+    t.join()
+    assert seen == [""]
