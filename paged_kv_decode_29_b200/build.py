@@ -9,7 +9,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB = os.path.join(HERE, "libdecattn.so")
 SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
-DEPS = SOURCES + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh"))) + [
+DEPS = SOURCES + sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh"))) + sorted(
+    glob.glob(os.path.join(HERE, "csrc", "*.h"))) + [
     os.path.join(os.path.dirname(HERE), "include", "decattn.h")]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -10,6 +10,7 @@
 #include <utility>
 
 #include "common.cuh"
+#include "host_errors.h"
 
 namespace decattn {
 

@@ -19,6 +19,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "host_errors.h"
 
 namespace decattn {
 

@@ -438,10 +438,6 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
 
 // ------------------------------------------------------------------ host-side launchers
 int default_bins(int device);                                     // api.cu
-// Records the CUDA error behind a DECATTN_ECUDA result for dec_attn_last_error (per host thread) and
-// returns DECATTN_ECUDA. e == cudaSuccess takes the runtime's last error (a helper that returned
-// false right after the failing call); `what` names the failing step.
-int cuda_fail(const char* what, cudaError_t e = cudaSuccess);     // api.cu
 bool ensure_smem_attr(const void* kernel, int bytes);             // api.cu
 bool split_supported(int kv_dtype, int D, int GT);                // split.cu
 cudaError_t launch_split(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV, int kv_dtype,

@@ -19,6 +19,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "host_errors.h"
 
 namespace decattn {
 

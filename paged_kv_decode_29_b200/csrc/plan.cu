@@ -19,6 +19,7 @@
 //    least-loaded search, done by one warp with warp-wide min reductions.
 // The plan's size is O(batch * n_kv_heads + n_bins), independent of the tile count.
 #include "common.cuh"
+#include "host_errors.h"
 
 namespace decattn {
 
