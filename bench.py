@@ -75,6 +75,8 @@ def parse():
     ap.add_argument("--profile", action="store_true",
                     help="only warm-up + timed steps (for ncu launch lists): no baseline, e2e, graph or clocks")
     ap.add_argument("--json-out", default="", help="also append the JSON line to this file")
+    ap.add_argument("--write-traffic", action="store_true",
+                    help="write the DRAM-traffic JSON files under profiles/ from the capture tables and exit")
     ap.add_argument("--sparse", type=float, default=0.0,
                     help="block-sparse decode: keep each (request, KV head, tile) with this probability "
                          "(the tile with each request's newest token always kept); 0 = dense")
@@ -124,6 +126,67 @@ def split_kernel_name(pr) -> str:
     if pr.kv_dtype == "fp8e4m3" and pr.head_dim == 128 and pr.group * pr.q_tokens <= 16:
         return "split_tc_kernel"
     return "split_kernel"
+
+
+# ---------------------------------------------------------------- DRAM traffic captures
+# DRAM bytes (dram__bytes_read.sum, dram__bytes_write.sum) of one launch, from the ncu captures that
+# profiles/split_kernel_dram_traffic.md and profiles/prefill_kernel_prefill_b4.md describe.
+# `python bench.py --write-traffic` turns them into the JSON files that roofline.traffic reads.
+# Split kernels: a smaller case of each workload (its first requests), scaled to a full launch by
+# the ratio of algorithmic bytes (reads measured within 0.05% of the algorithmic bytes on every
+# captured case, so traffic grows in proportion): workload -> (requests captured, read, write).
+SPLIT_TRAFFIC_CAPTURED = {
+    "uniform": (8, 134362368, 3598080),
+    "mixed": (16, 1039144960, 17676288),
+    "fp8_spec": (4, 167250432, 6338304),
+    "long_b4": (1, 536982272, 5664256),
+}
+# prefill_kernel on the full prefill workload (read, write): a few hundred MB on the device.
+PREFILL_TRAFFIC_CAPTURED = (108316928, 87724800)
+
+
+def config_algorithmic_bytes(name: str, batch: int | None = None) -> int:
+    """Problem.algorithmic_bytes() of a workload (or its first `batch` requests) without generating
+    its data."""
+    c = W.CONFIGS[name]
+    L = np.asarray(W.config_seq_lens(name), dtype=np.int64)
+    if batch is not None:
+        L = L[:batch]
+    B, d, P, hkv, hq, T = len(L), c["head_dim"], c["page_size"], c["n_kv_heads"], c["n_q_heads"], c["q_tokens"]
+    eb = 1 if c["kv_dtype"] == "fp8e4m3" else 2
+    pages = int(((L + P - 1) // P).sum())
+    return (int(L.sum()) * hkv * d * eb * 2 + B * T * hq * d * 2 + B * T * hq * (d + 1) * 4 + pages * 4 + B * 4
+            + (pages * hkv * 2 * 4 if c["kv_dtype"] == "fp8e4m3" else 0))
+
+
+def prefill_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("prefill.cu", "tc.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "paged_kv_decode_29_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def write_traffic_json():
+    """Writes profiles/split_kernel_dram_traffic.json and profiles/prefill_kernel_dram_traffic.json
+    from the capture tables above, stamped with the current source hashes (run it right after a
+    capture of the current sources)."""
+    out = {"source_hash": kernel_source_hash(), "configs": {}}
+    for name, (nb, rd, wr) in SPLIT_TRAFFIC_CAPTURED.items():
+        small, full = config_algorithmic_bytes(name, nb), config_algorithmic_bytes(name)
+        scale = full / small
+        out["configs"][f"{name}/tl{W.CONFIGS[name]['tile_len']}"] = {
+            "bytes_per_launch": int(round((rd + wr) * scale)),
+            "captured_requests": nb, "captured_read": rd, "captured_write": wr,
+            "captured_algorithmic": small, "scale": round(scale, 6),
+            "read_over_algorithmic": round(rd / small, 5),
+        }
+    with open(os.path.join(ROOT, "profiles", "split_kernel_dram_traffic.json"), "w") as f:
+        json.dump(out, f, indent=1)
+    rd, wr = PREFILL_TRAFFIC_CAPTURED
+    pf = {"source_hash": prefill_source_hash(),
+          "configs": {"prefill": {"bytes_per_launch": rd + wr, "captured_read": rd, "captured_write": wr}}}
+    with open(os.path.join(ROOT, "profiles", "prefill_kernel_dram_traffic.json"), "w") as f:
+        json.dump(pf, f, indent=1)
 
 
 def ncu_traffic(config: str, tile_len: int):
@@ -582,10 +645,7 @@ def prefill_traffic():
         d = json.load(open(os.path.join(ROOT, "profiles", "prefill_kernel_dram_traffic.json")))
     except Exception:
         return None
-    h = hashlib.sha256()
-    for f in ("prefill.cu", "tc.cuh", "common.cuh"):
-        h.update(open(os.path.join(ROOT, "paged_kv_decode_29_b200", "csrc", f), "rb").read())
-    if d.get("source_hash") != h.hexdigest()[:16]:
+    if d.get("source_hash") != prefill_source_hash():
         return None
     return int(d["configs"]["prefill"]["bytes_per_launch"])
 
@@ -732,6 +792,9 @@ def run_prefill(args, rank: int, world: int, local_rank: int, dist):
 
 def main():
     args = parse()
+    if args.write_traffic:
+        write_traffic_json()
+        return 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

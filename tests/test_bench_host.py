@@ -73,3 +73,12 @@ def test_traffic_is_reported_only_for_the_captured_sources(tmp_path, monkeypatch
         path.write_bytes(path.read_bytes() + b"\n")
     assert bench.ncu_traffic("uniform", 256) is None
     assert bench.prefill_traffic() is None
+
+
+def test_config_algorithmic_bytes_matches_the_generated_workload():
+    # the traffic scaling counts a workload's bytes without generating it: same figure as the problem's
+    for name, batch in (("tiny", None), ("fp8_spec", 2), ("uniform", 3)):
+        pr = W.make_problem(name=name, seq_lens=W.config_seq_lens(name)[:batch] if batch else W.config_seq_lens(name),
+                            **{k: v for k, v in W.CONFIGS[name].items() if k not in ("batch", "pool_pages")},
+                            batch=batch or W.CONFIGS[name]["batch"])
+        assert bench.config_algorithmic_bytes(name, batch) == pr.algorithmic_bytes(), name
