@@ -4,8 +4,9 @@ bandwidth, for GQA decode attention over a paged KV cache with split-KV scheduli
 
 A step is one pass of the whole path on one batch: the planner kernel, the split kernel
 and the combine kernel (plan + split + combine). Inputs are seeded synthetic data of the
-named workload (``--config``, default "uniform": batch 32, 32 query / 8 KV heads,
-head_dim 128, every KV length 4096, page size 16, bf16), resident in HBM before timing.
+named workload (``--config``, default "mixed": batch 64, 32 query / 8 KV heads, head_dim 128,
+KV lengths log-uniform in [128, 65536], 1% of K rows x8, page size 16, bf16; the largest
+single-GPU workload), resident in HBM before timing.
 
 Timing: W untimed warm-up steps, then K timed steps (events at step boundaries only, so the
 three kernels keep their programmatic-dependent-launch overlap), then the same K steps again
@@ -65,7 +66,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="uniform", choices=sorted(W.CONFIGS))
+    ap.add_argument("--config", default="mixed", choices=sorted(W.CONFIGS))
     ap.add_argument("--tile-len", type=int, default=0, help="override the workload's tile length")
     ap.add_argument("--batch", type=int, default=0,
                     help="keep only the first BATCH requests of the workload (smaller profiling cases)")
@@ -136,13 +137,16 @@ def split_kernel_name(pr) -> str:
 # the ratio of algorithmic bytes (reads measured within 0.05% of the algorithmic bytes on every
 # captured case, so traffic grows in proportion): workload -> (requests captured, read, write).
 SPLIT_TRAFFIC_CAPTURED = {
-    "uniform": (8, 134362368, 3598080),
-    "mixed": (16, 1039144960, 17676288),
-    "fp8_spec": (4, 167250432, 6338304),
-    "long_b4": (1, 536982272, 5664256),
+    "source_hash": "2cd4dd2d54b1c127",  # kernel_source_hash() of the sources these were captured on
+    "configs": {
+        "uniform": (8, 134362368, 3598080),
+        "mixed": (16, 1039144960, 17676288),
+        "fp8_spec": (4, 167250432, 6338304),
+        "long_b4": (1, 536982272, 5664256),
+    },
 }
 # prefill_kernel on the full prefill workload (read, write): a few hundred MB on the device.
-PREFILL_TRAFFIC_CAPTURED = (108316928, 87724800)
+PREFILL_TRAFFIC_CAPTURED = {"source_hash": "22fe69057deeaf7e", "read": 108316928, "write": 87724800}
 
 
 def config_algorithmic_bytes(name: str, batch: int | None = None) -> int:
@@ -168,25 +172,35 @@ def prefill_source_hash() -> str:
 
 def write_traffic_json():
     """Writes profiles/split_kernel_dram_traffic.json and profiles/prefill_kernel_dram_traffic.json
-    from the capture tables above, stamped with the current source hashes (run it right after a
-    capture of the current sources)."""
-    out = {"source_hash": kernel_source_hash(), "configs": {}}
-    for name, (nb, rd, wr) in SPLIT_TRAFFIC_CAPTURED.items():
-        small, full = config_algorithmic_bytes(name, nb), config_algorithmic_bytes(name)
-        scale = full / small
-        out["configs"][f"{name}/tl{W.CONFIGS[name]['tile_len']}"] = {
-            "bytes_per_launch": int(round((rd + wr) * scale)),
-            "captured_requests": nb, "captured_read": rd, "captured_write": wr,
-            "captured_algorithmic": small, "scale": round(scale, 6),
-            "read_over_algorithmic": round(rd / small, 5),
-        }
-    with open(os.path.join(ROOT, "profiles", "split_kernel_dram_traffic.json"), "w") as f:
-        json.dump(out, f, indent=1)
-    rd, wr = PREFILL_TRAFFIC_CAPTURED
-    pf = {"source_hash": prefill_source_hash(),
-          "configs": {"prefill": {"bytes_per_launch": rd + wr, "captured_read": rd, "captured_write": wr}}}
-    with open(os.path.join(ROOT, "profiles", "prefill_kernel_dram_traffic.json"), "w") as f:
-        json.dump(pf, f, indent=1)
+    from the capture tables above. Each table records the source hash it was captured on; a table
+    whose hash is not the current sources' is not written (its figures would describe other code)."""
+    wrote = []
+    if SPLIT_TRAFFIC_CAPTURED["source_hash"] == kernel_source_hash():
+        out = {"source_hash": SPLIT_TRAFFIC_CAPTURED["source_hash"], "configs": {}}
+        for name, (nb, rd, wr) in SPLIT_TRAFFIC_CAPTURED["configs"].items():
+            small, full = config_algorithmic_bytes(name, nb), config_algorithmic_bytes(name)
+            scale = full / small
+            out["configs"][f"{name}/tl{W.CONFIGS[name]['tile_len']}"] = {
+                "bytes_per_launch": int(round((rd + wr) * scale)),
+                "captured_requests": nb, "captured_read": rd, "captured_write": wr,
+                "captured_algorithmic": small, "scale": round(scale, 6),
+                "read_over_algorithmic": round(rd / small, 5),
+            }
+        with open(os.path.join(ROOT, "profiles", "split_kernel_dram_traffic.json"), "w") as f:
+            json.dump(out, f, indent=1)
+        wrote.append("split")
+    else:
+        log("split-kernel traffic table was captured on other sources: not written")
+    if PREFILL_TRAFFIC_CAPTURED["source_hash"] == prefill_source_hash():
+        rd, wr = PREFILL_TRAFFIC_CAPTURED["read"], PREFILL_TRAFFIC_CAPTURED["write"]
+        pf = {"source_hash": PREFILL_TRAFFIC_CAPTURED["source_hash"],
+              "configs": {"prefill": {"bytes_per_launch": rd + wr, "captured_read": rd, "captured_write": wr}}}
+        with open(os.path.join(ROOT, "profiles", "prefill_kernel_dram_traffic.json"), "w") as f:
+            json.dump(pf, f, indent=1)
+        wrote.append("prefill")
+    else:
+        log("prefill-kernel traffic table was captured on other sources: not written")
+    return wrote
 
 
 def ncu_traffic(config: str, tile_len: int):
@@ -323,7 +337,7 @@ def run_reference(args, rank: int):
         "impl": "reference", "metric": PREFILL_METRIC if args.config == "prefill" else METRIC, "value": round(value, 3), "unit": "us/step",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(value / 1e3, 6),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": pr.name, **workload_desc(pr)},
+        "config": bench_config(pr, args.gpus, prefill=args.config == "prefill"),
         "cpu_baseline": {"value": round(value, 3), "unit": "us/step", "cores": threads, "kind": "oracle",
                          "sample": f"each step: {sample}"},
         "e2e": {"value": round(value, 3), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -333,6 +347,15 @@ def run_reference(args, rank: int):
 
 
 # ---------------------------------------------------------------- our arm
+
+def bench_config(pr, world: int, prefill: bool = False):
+    """The `config` object of the JSON line, identical on both arms: the workload, its shapes, how
+    the L2 is kept from serving the inputs, and the multi-GPU layout."""
+    l2 = ("flushed before every step (a reduction reading 256 MiB)" if prefill else
+          "flushed before every step (a reduction reading 256 MiB); KV bytes exceed the 126 MB L2")
+    return {"workload": pr.name, **workload_desc(pr), "l2": l2,
+            "parallelism": "replicas" if world > 1 else "single GPU"}
+
 
 def workload_desc(pr):
     return {"batch": pr.batch, "n_q_heads": pr.n_q_heads, "n_kv_heads": pr.n_kv_heads, "head_dim": pr.head_dim,
@@ -579,10 +602,9 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
         "warmup": args.warmup, "ms_per_step": round(step_m / 1e3, 6), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": ("fp8e4m3 (q, P in e4m3)" if args.mma8 else "fp8e4m3->f16") if pr.kv_dtype == "fp8e4m3" else "bf16",
         "data": "synthetic",
-        "config": {"workload": pr.name, **workload_desc(pr), "n_bins": pl.n_bins,
-                   **({"products": "e4m3 tensor cores (q and P rounded to e4m3)"} if args.mma8 else {}),
-                   "l2": "flushed before every step (a reduction reading 256 MiB); KV bytes exceed the 126 MB L2",
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "config": {**bench_config(pr, world),
+                   **({"products": "e4m3 tensor cores (q and P rounded to e4m3)"} if args.mma8 else {})},
+        "n_bins": pl.n_bins,
         "breakdown_note": "plan/split/combine: a second pass of the same steps with events between the kernels",
         "plan_us": round(plan_m, 3), "split_us": round(split_m, 3), "combine_us": round(comb_m, 3),
         "graph_step_us": None if graph_us is None else round(graph_us, 3),
@@ -767,9 +789,7 @@ def run_prefill(args, rank: int, world: int, local_rank: int, dist):
         "value": round(step_m, 3), "unit": "us/step", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_m / 1e3, 6), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": pr.name, **workload_desc(pr),
-                   "l2": "flushed before every step (a reduction reading 256 MiB)",
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "config": bench_config(pr, world, prefill=True),
         "algorithmic_flops": flops,
         "roofline": {"bound": "tensor", "kernel": "prefill_kernel", "achieved": round(tflops, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),

@@ -224,7 +224,10 @@ DECATTN_API int dec_attn_run(const dec_attn_shape *shape, const void *q, const v
  *   enqueued then); DECATTN_ECUDA if the scratch's device address cannot be looked up.
  *   The first call on a device (with that device current) looks up the array's device address
  *   and loads the module that holds it; make that first call before any stream capture. The
- *   array then stays allocated on that GPU until the process exits.
+ *   array then stays allocated on that GPU until the process exits. The address is cached per
+ *   device together with the CUDA context it was looked up in, and is valid in that context
+ *   only: after cudaDeviceReset the next call finds a new context and looks it up again (so
+ *   that call, too, should come before any capture).
  *   All calls on one device share the array; its contents are left over from the last call and
  *   need no clearing (the split kernel writes every partial the combine reads and resets the
  *   combine counters). Calls whose work overlaps on the GPU (e.g. on two streams) race on it:
@@ -236,8 +239,11 @@ DECATTN_API int dec_attn_run_noalloc(const dec_attn_shape *shape, const void *q,
 
 /* The two stages of dec_attn_run as separate calls (same arguments, same checks):
  * dec_attn_split enqueues only the split kernel, dec_attn_combine only the combine
- * kernel, which reads the partials the split kernel left in `workspace`. dec_attn_run(...) == dec_attn_split(...) followed by
- * dec_attn_combine(...) on the same stream. Useful to time or overlap the stages. */
+ * kernel, which reads the partials the split kernel left in `workspace`. dec_attn_run(...) ==
+ * dec_attn_split(...) followed by dec_attn_combine(...) on the same stream. Useful to time or
+ * overlap the stages. The split kernel zeroes the combine's per-row counters, and the combine
+ * returns every counter it used to zero after merging its row, so dec_attn_combine may also be
+ * repeated on the partials of one dec_attn_split (e.g. to time the combine alone). */
 DECATTN_API int dec_attn_split(const dec_attn_shape *shape, const void *q, const void *k_pages, const void *v_pages,
                                const int32_t *page_table, const int32_t *seq_lens, const float *kv_scales,
                                const dec_attn_plan_t *plan, void *workspace, size_t workspace_bytes, float *out,

@@ -9,11 +9,15 @@
 //
 // How: the workspace lives in g_noalloc_scratch below, kDecattnNoallocBytes (64 MiB) per GPU.
 // Host code cannot use the array's name as a device address, so the first call on each device
-// (with that device current) looks the address up with cudaGetSymbolAddress and caches it;
-// that first call also makes the CUDA runtime load the module holding the array, so it should
-// come before any stream capture. The array stays allocated on every GPU where it was set up
-// until the process exits. Nothing in it has to start at zero: the split kernel writes every
-// partial the combine reads and zeroes the combine's per-row counters at the start of each run.
+// (with that device current) looks the address up with cudaGetSymbolAddress and caches it,
+// together with the identity of the CUDA context it belongs to; that first call also makes the
+// CUDA runtime load the module holding the array, so it should come before any stream capture.
+// A cached address is only valid in its own context: after cudaDeviceReset the device gets a new
+// primary context (and a new copy of the module), so a call that finds another context current
+// looks the address up again instead of handing the kernels a dangling pointer. The array stays
+// allocated on every GPU where it was set up until the process (or a device reset) ends it.
+// Nothing in it has to start at zero: the split kernel writes every partial the combine reads
+// and zeroes the combine's per-row counters at the start of each run.
 // All calls on a device share the one array, so calls whose work overlaps on the GPU (e.g. on
 // two streams) race and corrupt each other's results; serialise them.
 #include <mutex>
@@ -32,21 +36,57 @@ static_assert(kDecattnNoallocBytes == (size_t)DECATTN_NOALLOC_SCRATCH_BYTES, "sc
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct ScratchEntry {
+  void* ptr;             // device address of g_noalloc_scratch in context `ctx_id`
+  unsigned long long ctx_id;
+};
+ScratchEntry g_noalloc[kMaxDevices] = {};
 
-// Device address of g_noalloc_scratch on the current device (looked up once per device).
+// Identity of the current CUDA context (cuCtxGetCurrent + cuCtxGetId, fetched through the
+// runtime so that the library needs no libcuda link). 0 when the driver cannot say, in which
+// case the address is looked up on every call.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool tried = false;
+  if (!tried) {  // called with g_noalloc_mu held
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  }
+  if (!get_cur || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch on the current device, looked up once per (device,
+// context) and again whenever the current context is not the one it was looked up in.
 int noalloc_scratch(void** out) {
   int dev = 0;
   if (const cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
   if (dev < 0 || dev >= kMaxDevices) return cuda_fail("device ordinal beyond the scratch table", cudaErrorInvalidDevice);
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  const unsigned long long ctx = current_ctx_id();  // 0 also before the runtime's first call made one
+  ScratchEntry& ent = g_noalloc[dev];
+  if (!ent.ptr || ctx == 0 || ent.ctx_id != ctx) {
     void* ptr = nullptr;
     if (const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch); e != cudaSuccess || !ptr)
       return cuda_fail("scratch address (cudaGetSymbolAddress)", e == cudaSuccess ? cudaErrorInvalidSymbol : e);
-    g_noalloc_ptr[dev] = ptr;
+    ent.ptr = ptr;
+    ent.ctx_id = current_ctx_id();  // the lookup has made the device's primary context current
   }
-  *out = g_noalloc_ptr[dev];
+  *out = ent.ptr;
   return DECATTN_OK;
 }
 }  // namespace

@@ -24,12 +24,20 @@ def kv_values(pr, which: str) -> np.ndarray:
 
 
 def dense_kv(pr, b: int, which: str) -> np.ndarray:
-    """Logical K or V of request b as float64 [Hkv][Lb][d], gathered through the page table."""
-    vals = kv_values(pr, which)
+    """Logical K or V of request b as float64 [Hkv][Lb][d], gathered through the page table (only
+    the request's pages are converted)."""
     Lb, P = int(pr.seq_lens[b]), pr.page_size
     npg = (Lb + P - 1) // P
     pages = pr.page_table[b, :npg]
-    x = vals[pages]                      # [npg][Hkv][P][d]
+    pool = pr.k_pages if which == "k" else pr.v_pages
+    raw = pool[pages]                    # [npg][Hkv][P][d]
+    if pr.kv_dtype == "bf16":
+        x = W.bf16_bits_to_f32(raw).astype(np.float64)
+    else:
+        import torch
+        x = torch.from_numpy(np.ascontiguousarray(raw)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        sc = pr.kv_scales[0 if which == "k" else 1].astype(np.float64)[pages]   # [npg][Hkv]
+        x = x * sc[:, :, None, None]
     x = x.transpose(1, 0, 2, 3).reshape(pr.n_kv_heads, npg * P, pr.head_dim)
     return x[:, :Lb]
 

@@ -82,3 +82,33 @@ def test_config_algorithmic_bytes_matches_the_generated_workload():
                             **{k: v for k, v in W.CONFIGS[name].items() if k not in ("batch", "pool_pages")},
                             batch=batch or W.CONFIGS[name]["batch"])
         assert bench.config_algorithmic_bytes(name, batch) == pr.algorithmic_bytes(), name
+
+
+def test_write_traffic_refuses_tables_captured_on_other_sources(tmp_path, monkeypatch):
+    # the capture tables carry the hash of the sources they were taken on; after a kernel edit
+    # --write-traffic must not stamp them with the new hash
+    root = tmp_path / "repo"
+    (root / "profiles").mkdir(parents=True)
+    shutil.copytree(os.path.join(bench.ROOT, "paged_kv_decode_29_b200", "csrc"),
+                    root / "paged_kv_decode_29_b200" / "csrc")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    monkeypatch.setitem(bench.SPLIT_TRAFFIC_CAPTURED, "source_hash", "0" * 16)
+    monkeypatch.setitem(bench.PREFILL_TRAFFIC_CAPTURED, "source_hash", "0" * 16)
+    assert bench.write_traffic_json() == []
+    assert not (root / "profiles" / "split_kernel_dram_traffic.json").exists()
+    assert not (root / "profiles" / "prefill_kernel_dram_traffic.json").exists()
+    # with the current hashes both tables are written, stamped with the hash they were taken on
+    monkeypatch.setitem(bench.SPLIT_TRAFFIC_CAPTURED, "source_hash", bench.kernel_source_hash())
+    monkeypatch.setitem(bench.PREFILL_TRAFFIC_CAPTURED, "source_hash", bench.prefill_source_hash())
+    assert bench.write_traffic_json() == ["split", "prefill"]
+    d = json.load(open(root / "profiles" / "split_kernel_dram_traffic.json"))
+    assert d["source_hash"] == bench.kernel_source_hash()
+    assert set(d["configs"]) == {f"{n}/tl{W.CONFIGS[n]['tile_len']}" for n in bench.SPLIT_TRAFFIC_CAPTURED["configs"]}
+
+
+def test_both_arms_report_the_same_config():
+    pr = W.make_config("tiny")
+    assert bench.bench_config(pr, 1) == bench.bench_config(pr, 1)
+    c = bench.bench_config(pr, 1)
+    assert c["workload"] == "tiny" and "l2" in c and c["parallelism"] == "single GPU"
+    assert "n_bins" not in c
