@@ -202,8 +202,9 @@ DECATTN_API size_t dec_attn_workspace_bytes(const dec_attn_shape *shape, const d
  *   workspace  device, workspace_bytes >= dec_attn_workspace_bytes(shape, plan)
  *   out        fp32 [B][T][Hq][d];  lse  fp32 [B][T][Hq] (natural log)
  * Supported: head_dim 64 or 128; page_size a multiple of 16 up to 256;
- * tile_len a multiple of page_size; G*T <= 16. Anything else returns
- * DECATTN_ENOTSUP before any launch. */
+ * tile_len a multiple of page_size; q_tokens T <= 8 and G*T <= 64 query rows per KV head
+ * (G = n_q_heads / n_kv_heads: grouped-query heads and speculative tokens together). Anything
+ * else returns DECATTN_ENOTSUP before any launch. */
 DECATTN_API int dec_attn_run(const dec_attn_shape *shape, const void *q, const void *k_pages, const void *v_pages,
                  const int32_t *page_table, const int32_t *seq_lens, const float *kv_scales,
                  const dec_attn_plan_t *plan, void *workspace, size_t workspace_bytes, float *out, float *lse,

@@ -159,7 +159,8 @@ static int check_shape(const dec_attn_shape* s, const dec_attn_plan_t* pl) {
   if (s->head_dim != 64 && s->head_dim != 128) return DECATTN_ENOTSUP;
   if (s->page_size % 16 != 0 || s->page_size > 256) return DECATTN_ENOTSUP;
   if (pl->tile_len % s->page_size != 0) return DECATTN_ENOTSUP;
-  if (GT > 16 || !split_supported(s->kv_dtype, s->head_dim, (int)GT)) return DECATTN_ENOTSUP;
+  if (s->q_tokens > kMaxT || GT > kMaxGT || !split_supported(s->kv_dtype, s->head_dim, (int)GT))
+    return DECATTN_ENOTSUP;
   if ((int64_t)s->num_pages * s->n_kv_heads * s->page_size >= (1ll << 31)) return DECATTN_ENOTSUP;
   if ((int64_t)s->batch * s->q_tokens * s->n_q_heads >= (1ll << 31)) return DECATTN_ENOTSUP;
   return DECATTN_OK;

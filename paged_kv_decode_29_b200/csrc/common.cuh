@@ -189,6 +189,11 @@ struct PrefillParams {
   float qk_scale_log2;        // sm_scale * log2(e)
 };
 
+// Query rows of one KV head that a decode tile computes at once (G * T), and query tokens per
+// request (T), that dec_attn_run supports.
+constexpr int kMaxGT = 64;
+constexpr int kMaxT = 8;
+
 // The combine kernel folds the partials of one query row in chunks of this many tiles.
 // A request with n_b tiles gives each of its rows cb_b = ceil(n_b / kCombineChunk) chunks
 // (1 if n_b == 0: the row is zero-filled; 0 if n_b == 1: the split kernel wrote the row).

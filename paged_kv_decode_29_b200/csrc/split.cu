@@ -14,19 +14,25 @@
 //    the next ring stage; the tile's q rows go to a double-buffered q slot by bulk copy;
 //    FP8 page scales ride along as 4-byte cp.async copies folded into the stage's
 //    mbarrier. It waits only on "stage empty" barriers, so it runs ahead of the math.
-//  * warps 1..NCW (consumers; with NCW = 2 each takes one 8-row half of the G*T query rows
-//    and both read the same staged K/V): per 16-key block, S^T = K Q^T on tensor cores with the keys on
-//    the MMA's M side ("SwapAB", as in the pages' Attention SwapAB), so a G*T of 4..16
-//    query rows fills N = 8 or 16 instead of padding M to 16; then an online softmax in
+//  * warps 1..NCW (consumers; with NCW = 2, 4 or 8 each takes one 8-row slice of the G*T
+//    query rows, up to 64, and all read the same staged K/V): per 16-key block, S^T = K Q^T
+//    on tensor cores with the keys on the MMA's M side ("SwapAB", as in the pages' Attention
+//    SwapAB), so a G*T of 4..64 query rows fills N = 8 per warp instead of padding M to 16;
+//    then an online softmax in
 //    fp32 (log2 domain), then O^T += V^T P^T (again keys as the contraction, head_dim on
 //    M). Probabilities go to the MMA as bf16 hi + bf16 lo (BF16 KV: two columns of the
 //    same MMA when G*T <= 4, two N tiles otherwise), or as f16 scaled by the page's V
 //    scale (FP8 KV).
 //  * FP8 KV: S^T runs on E4M3 MMAs straight from the staged codes (K is never widened);
-//    V is widened to f16. With one consumer warp it is widened in registers; with two,
-//    each widens half of every V block into a shared f16 block (laid out like a bf16
-//    stage, two buffers) and both read V^T from it with ldmatrix, so no element is
+//    V is widened to f16. With one consumer warp it is widened in registers; with several,
+//    each widens its share of every V block into a shared f16 block (laid out like a bf16
+//    stage, two buffers) and all read V^T from it with ldmatrix, so no element is
 //    widened twice; the raw stage is released as soon as it is widened and used for S^T.
+//  * occupancy: 4 CTAs per SM with one or two consumer warps (G*T <= 16); the wide variants
+//    (G*T up to 32 / 64: 4 / 8 consumer warps) hold more registers and q rows per CTA and run
+//    2 / 1 CTAs per SM, each with a deeper ring (80 / 144 KB) to keep as many bytes in flight.
+//    The grid is one CTA per bin either way; with fewer CTAs resident than bins they run in
+//    waves of equal load (the bins are balanced by the planner).
 //  * the tile ends with either the final output (the tile covers its whole request) or
 //    a normalised partial (o, lse) in the workspace for the combine kernel.
 // FP8 KV with head_dim 128 and G*T <= 16 runs in split_tc.cu instead (tcgen05 tensor cores with
@@ -43,7 +49,16 @@ namespace decattn {
 // FP8 KV: P is multiplied by (V page scale * kPScale) before its f16 rounding, so that small
 // probabilities stay normal f16 numbers; the epilogue divides kPScale back out.
 constexpr float kPScale = 256.f;
-constexpr int kCtasPerSm = 4;
+constexpr int kCtasPerSm = 4;  // CTAs per SM of the variants with up to 2 consumer warps (G*T <= 16)
+
+// Resident CTAs per SM a variant is built for: 4 with one or two consumer warps; the wide
+// variants (G*T > 16: 4 or 8 consumer warps, one 8-row slice of the query rows each) hold more
+// registers and q rows per CTA and run 2 (4 warps) or 1 (8 warps) per SM with a deeper ring.
+template <int NCW>
+struct Occ {
+  static constexpr int CPS = NCW <= 2 ? kCtasPerSm : NCW == 4 ? 2 : 1;
+  static constexpr int RING = CPS == kCtasPerSm ? 40 * 1024 : CPS == 2 ? 80 * 1024 : 144 * 1024;
+};
 
 template <int KVT, int D>
 struct Geo {
@@ -66,12 +81,12 @@ struct Geo {
 
 // VSH: the consumer warps share the widening of each FP8 V block (two f16 blocks in the layout
 // of a bf16 stage, after the ring).
-template <int KVT, int D, int NQ, bool VSH>
+template <int KVT, int D, int NQ, bool VSH, int RING>
 struct Smem {
   using G_ = Geo<KVT, D>;
   using G16 = Geo<0, D>;                                         // layout of a widened V block
   static constexpr int V16 = VSH ? 2 * G16::TILE : 0;
-  static constexpr int STAGES = (40 * 1024 - V16) / (2 * G_::TILE);
+  static constexpr int STAGES = (RING - V16) / (2 * G_::TILE);
   static constexpr int QBYTES = 8 * NQ * D * 2;
   static constexpr int OFF_V16 = STAGES * 2 * G_::TILE;
   static constexpr int OFF_Q = OFF_V16 + V16;
@@ -97,12 +112,13 @@ __device__ __forceinline__ int qrow_of_col(int n, int GT) {
 // O^T.  DUP: bf16 with G*T <= 4 (hi in columns 0..3, lo in 4..7 of one tile).  NCW: consumer
 // warps; consumer w owns S^T tiles [w*NQ/NCW, (w+1)*NQ/NCW) and the O^T tiles that go with them.
 template <int KVT, int D, int NQ, int NPV, bool DUP, int NCW>
-__global__ void __launch_bounds__(32 * (1 + NCW), kCtasPerSm)
+__global__ void __launch_bounds__(32 * (1 + NCW), Occ<NCW>::CPS)
 split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   using G_ = Geo<KVT, D>;
-  // FP8 with two consumer warps: each widens half of every V block into a shared f16 block
-  constexpr bool VSH = KVT == 1 && NCW == 2;
-  using S_ = Smem<KVT, D, NQ, VSH>;
+  // FP8 with several consumer warps: they share the widening of every V block into a shared
+  // f16 block, so that no element is widened twice
+  constexpr bool VSH = KVT == 1 && NCW >= 2;
+  using S_ = Smem<KVT, D, NQ, VSH, Occ<NCW>::RING>;
   using G16 = typename S_::G16;
   constexpr int STAGES = S_::STAGES;
   constexpr int NQW = NQ / NCW;    // S^T tiles per consumer warp
@@ -401,15 +417,18 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
       }
       const int vb = vblk & 1;
       if (VSH) {
-        // ---- widen this warp's half of the V block (d in [D/2 * (warp-1), D/2 * warp)) to f16
-        //      in the layout of a bf16 stage; two lanes per key, 16 codes per 16-byte chunk
-        constexpr int CH = D / 16 / NCW;  // raw 16-byte chunks of a key row per warp
+        // ---- widen this warp's share of the V block to f16 in the layout of a bf16 stage: the
+        //      block's 16 keys x D/16 raw 16-byte chunks (16 codes each) are dealt to the
+        //      consumer warps' lanes, item i = (chunk i / 16, key i % 16)
+        constexpr int ITEMS = 16 * (D / 16);
+        constexpr int PER_LANE = (ITEMS + 32 * NCW - 1) / (32 * NCW);
         const uint8_t* vraw = sm + s * 2 * G_::TILE + G_::TILE;
         uint8_t* v16 = sm + S_::OFF_V16 + vb * G16::TILE;
-        const int key = lane >> 1, hh = lane & 1;
         #pragma unroll
-        for (int c = 0; c < CH / 2; ++c) {
-          const int cg = (warp - 1) * CH + hh * (CH / 2) + c;  // codes d = 16 cg .. 16 cg + 15
+        for (int c = 0; c < PER_LANE; ++c) {
+          const int item = (warp - 1) * 32 + lane + c * 32 * NCW;
+          if (ITEMS % (32 * NCW) != 0 && item >= ITEMS) break;
+          const int key = item & 15, cg = item >> 4;  // codes d = 16 cg .. 16 cg + 15 of this key
           const uint4 w = *reinterpret_cast<const uint4*>(vraw + G_::off(key, cg));
           uint4 lo, hi;
           lo.x = e4m3x2_to_f16x2(w.x & 0xffffu); lo.y = e4m3x2_to_f16x2(w.x >> 16);
@@ -667,7 +686,9 @@ template <int KVT, int D, int NQ, int NPV, bool DUP, int NCW>
 static cudaError_t launch_variant(const SplitParams& p, const CUtensorMap& tmK, const CUtensorMap& tmV,
                                   cudaStream_t st) {
   auto fn = split_kernel<KVT, D, NQ, NPV, DUP, NCW>;
-  const int smem = Smem<KVT, D, NQ, KVT == 1 && NCW == 2>::ALLOC;
+  const int smem = Smem<KVT, D, NQ, KVT == 1 && NCW >= 2, Occ<NCW>::RING>::ALLOC;
+  static_assert(Occ<NCW>::CPS * (Smem<KVT, D, NQ, KVT == 1 && NCW >= 2, Occ<NCW>::RING>::ALLOC + 1024) <=
+                    228 * 1024, "the variant's CTAs fit an SM's shared memory");
   if (!ensure_smem_attr((const void*)fn, smem)) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_bins);
@@ -687,16 +708,20 @@ static cudaError_t launch_gt(const SplitParams& p, const CUtensorMap& tmK, const
   if constexpr (KVT == 0) {
     if (p.GT <= 4) return launch_variant<KVT, D, 1, 1, true, 1>(p, tmK, tmV, st);
     if (p.GT <= 8) return launch_variant<KVT, D, 1, 2, false, 1>(p, tmK, tmV, st);
-    return launch_variant<KVT, D, 2, 4, false, 2>(p, tmK, tmV, st);
+    if (p.GT <= 16) return launch_variant<KVT, D, 2, 4, false, 2>(p, tmK, tmV, st);
+    if (p.GT <= 32) return launch_variant<KVT, D, 4, 8, false, 4>(p, tmK, tmV, st);
+    return launch_variant<KVT, D, 8, 16, false, 8>(p, tmK, tmV, st);
   } else {
     if (p.GT <= 8) return launch_variant<KVT, D, 1, 1, false, 1>(p, tmK, tmV, st);
-    return launch_variant<KVT, D, 2, 2, false, 2>(p, tmK, tmV, st);
+    if (p.GT <= 16) return launch_variant<KVT, D, 2, 2, false, 2>(p, tmK, tmV, st);
+    if (p.GT <= 32) return launch_variant<KVT, D, 4, 4, false, 4>(p, tmK, tmV, st);
+    return launch_variant<KVT, D, 8, 8, false, 8>(p, tmK, tmV, st);
   }
 }
 
 bool split_supported(int kv_dtype, int D, int GT) {
   if (kv_dtype == DECATTN_KV_FP8E4M3_MMA8) return split_tc_supported(kv_dtype, D, GT);  // tcgen05 kernel only
-  return GT >= 1 && GT <= 16 && (D == 64 || D == 128) &&
+  return GT >= 1 && GT <= kMaxGT && (D == 64 || D == 128) &&
          (kv_dtype == DECATTN_KV_BF16 || kv_dtype == DECATTN_KV_FP8E4M3);
 }
 

@@ -86,8 +86,10 @@ def _run(lib, shape, plan, q=FAKE, k=FAKE, v=FAKE, tab=FAKE, lens=FAKE, sc=None,
     (dict(head_dim=256), {}, da.ENOTSUP),
     (dict(page_size=8), {}, da.ENOTSUP),
     (dict(page_size=48), dict(tile_len=64), da.ENOTSUP),       # tile not a multiple of the page
-    (dict(n_q_heads=64, n_kv_heads=2, q_tokens=1), {}, da.ENOTSUP),   # G*T = 32
-    (dict(q_tokens=5, n_q_heads=8, n_kv_heads=2), {}, da.ENOTSUP),   # G*T = 20
+    (dict(n_q_heads=130, n_kv_heads=2, q_tokens=1), {}, da.ENOTSUP),  # G*T = 65
+    (dict(q_tokens=9, n_q_heads=2, n_kv_heads=2), {}, da.ENOTSUP),    # T = 9
+    (dict(q_tokens=5, n_q_heads=26, n_kv_heads=2), {}, da.ENOTSUP),   # G*T = 65
+    (dict(q_tokens=5, n_q_heads=8, n_kv_heads=2, kv_dtype=da.KV_FP8E4M3_MMA8), {}, da.ENOTSUP),  # 20 > 16
     (dict(kv_dtype=7), {}, da.ENOTSUP),
     (dict(n_q_heads=6, n_kv_heads=4), dict(n_kv_heads=4), da.EINVAL),
     (dict(batch=3), {}, da.EINVAL),                             # plan made for another batch
@@ -95,6 +97,20 @@ def _run(lib, shape, plan, q=FAKE, k=FAKE, v=FAKE, tab=FAKE, lens=FAKE, sc=None,
 ])
 def test_run_rejects_bad_shapes(lib, shape_kw, plan_kw, code):
     assert _run(lib, _shape(**shape_kw), _plan(**plan_kw)) == code
+
+
+@pytest.mark.parametrize("Hq,T,kv,ok", [
+    (128, 1, da.KV_BF16, True), (16, 8, da.KV_BF16, True), (16, 8, da.KV_FP8E4M3, True),   # G*T = 64
+    (130, 1, da.KV_BF16, False), (18, 8, da.KV_FP8E4M3, False), (2, 9, da.KV_BF16, False),
+    (8, 4, da.KV_FP8E4M3_MMA8, True), (8, 5, da.KV_FP8E4M3_MMA8, False),                  # MMA8: G*T <= 16
+])
+def test_supported_query_rows_per_kv_head(lib, Hq, T, kv, ok):
+    # host only: the workspace size is 0 exactly for the shapes dec_attn_run refuses
+    s = _shape(n_q_heads=Hq, n_kv_heads=2, q_tokens=T, kv_dtype=kv)
+    n = lib.dec_attn_workspace_bytes(C.byref(s), C.byref(_plan()))
+    assert (n > 0) == ok
+    if ok:  # partials [tiles][G*T][d + 1] fp32 among the rest
+        assert n >= 64 * (Hq // 2) * T * 129 * 4
 
 
 def test_run_rejects_null_and_misaligned(lib):

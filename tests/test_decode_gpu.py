@@ -1,7 +1,7 @@
 """Split + combine on the GPU vs the fp64 oracle (out max-abs <= 2e-3, lse <= 1e-4).
 
 Small problems cover every kernel variant (bf16 / FP8 KV, head_dim 64 / 128, G*T from 1 to
-16, page sizes 16 / 32 / 64), ragged tails, one-key and empty requests, T > 1 causal rows
+64 with T up to 8, page sizes 16 / 32 / 64), ragged tails, one-key and empty requests, T > 1 causal rows
 that see no key, single-tile requests (final output written by the split kernel) and
 many-tile requests (combine). The five workloads run at full size with every row checked
 against the oracle.
@@ -41,7 +41,9 @@ LENS = [1, 15, 16, 17, 63, 64, 65, 200, 333]
 
 @pytest.mark.parametrize("kv", ["bf16", "fp8e4m3"])
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("G,T", [(1, 1), (2, 1), (3, 1), (4, 1), (5, 1), (8, 1), (2, 4), (4, 3), (16, 1), (4, 4)])
+@pytest.mark.parametrize("G,T", [(1, 1), (2, 1), (3, 1), (4, 1), (5, 1), (8, 1), (2, 4), (4, 3), (16, 1), (4, 4),
+                                 # G*T from 17 to 64: 4 or 8 consumer warps (GQA x speculative decode)
+                                 (8, 4), (16, 2), (32, 1), (6, 3), (3, 7), (8, 8), (64, 1), (5, 8)])
 def test_variants(kv, d, G, T):
     Hkv = 2
     pr = small(LENS, Hq=G * Hkv, Hkv=Hkv, d=d, T=T, kv=kv, seed=G * 10 + T)
@@ -154,6 +156,17 @@ def test_full_size_configs_all_rows(name):
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
     ref_o, ref_l = oracle.decode(pr)
     U.check_rows(out, lse, ref_o, ref_l, name)
+
+
+@pytest.mark.parametrize("T", [4, 8])
+def test_long_context_speculative_decode_all_rows(T):
+    # the long-context head layout (64 query / 8 KV heads) with T speculative tokens: G*T = 32 or 64
+    # query rows per KV head over 131072 keys, every row against the oracle
+    pr = W.make_config("long_b1", q_tokens=T)
+    out, lse, pl, st = U.run_problem(pr)
+    assert st == da.OK, da.status_string(st)
+    ref_o, ref_l = oracle.decode(pr)
+    U.check_rows(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, f"long_b1 T={T}")
 
 
 def test_repeated_runs_on_one_workspace_and_stage_calls():
