@@ -10,7 +10,8 @@ Everything is computed in fp64 by ``oracle.c``:
 * ``decode`` / ``decode_rows`` / ``attend``: scaled-dot-product attention of
   each query row over the paged KV cache, with an explicit full softmax and the
   bottom-right causal mask of speculative multi-token queries ("PaddlePaddle/
-  HALOps" README, Highlights, GQA attention item).
+  HALOps" README, Highlights, GQA attention item); ``decode_varlen``: the same
+  with a different number of query rows per request (each request on its own).
 * ``plan``: the greedy bin-packing of uniform KV tiles onto CTAs ("HPC-Ops:
   Tencent's CUDA Kernel Library for LLM Inference Hot Paths", "How the kernels
   are organized around specific workload shapes"), as a literal sequential
@@ -138,6 +139,32 @@ def decode_rows(pr, rows, nthreads: int = 0):
     out = np.zeros((n, pr.head_dim), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
     lib.oracle_decode_rows(C.byref(bd.s), rows.ctypes.data, n, out.ctypes.data, lse.ctypes.data, int(nthreads))
+    return out, lse
+
+
+def decode_varlen(pr):
+    """Variable-length query rows (``pr.cu_q`` set, q packed [total][Hq][d]): request b's
+    Tb = cu_q[b+1] - cu_q[b] rows are its last Tb positions, with the bottom-right causal rule
+    ("PaddlePaddle/HALOps" README, Highlights, GQA attention item: variable-length prefill). By
+    definition each request is computed alone, as a decode of that one request with T = Tb.
+    Returns out float64 [total][Hq][d] and lse float64 [total][Hq]."""
+    import copy
+    cu = np.asarray(pr.cu_q, dtype=np.int64)
+    total = int(cu[-1])
+    out = np.zeros((total, pr.n_q_heads, pr.head_dim), dtype=np.float64)
+    lse = np.zeros((total, pr.n_q_heads), dtype=np.float64)
+    for b in range(pr.batch):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        if hi == lo:
+            continue
+        one = copy.copy(pr)
+        one.batch, one.q_tokens, one.cu_q, one.tile_mask = 1, hi - lo, None, None
+        one.q = np.ascontiguousarray(pr.q[lo:hi][None])
+        one.seq_lens = np.ascontiguousarray(pr.seq_lens[b:b + 1])
+        one.page_table = np.ascontiguousarray(pr.page_table[b:b + 1])
+        o, l = decode(one)
+        out[lo:hi] = o[0]
+        lse[lo:hi] = l[0]
     return out, lse
 
 

@@ -105,6 +105,9 @@ class Problem:
     kv_scales: np.ndarray | None = None  # float32 [2][num_pages][Hkv] (K then V), FP8 only
     sm_scale: float = 0.0
     tile_mask: np.ndarray | None = None  # uint32 [B][Hkv][words]: block-sparse decode, bit i keeps tile i
+    # variable-length query rows (prefill): request b's rows are rows cu_q[b] .. cu_q[b+1]-1 of a
+    # packed q [total][Hq][d]; q_tokens is then the largest per-request count
+    cu_q: np.ndarray | None = None       # int32 [B+1]
     meta: dict = field(default_factory=dict)
 
     @property
@@ -292,6 +295,24 @@ CONFIGS = {
     "prefill": dict(batch=4, n_q_heads=32, n_kv_heads=8, head_dim=128, page_size=16, q_tokens=2048,
                     kv_dtype="bf16", tile_len=256, seed=6),
 }
+
+
+def make_varlen_problem(*, name="varlen", q_lens, **kw) -> Problem:
+    """A problem with a different number of query rows per request: ``q_lens[b]`` rows for request
+    b (its last q_lens[b] positions), packed into q [sum q_lens][Hq][d] with offsets cu_q [B+1].
+    The rows of request b are the first q_lens[b] rows of the same seeded draw that a problem with
+    max(q_lens) query tokens would use. Other arguments as make_problem (q_tokens is set)."""
+    ql = np.asarray(q_lens, dtype=np.int64)
+    assert ql.ndim == 1 and np.all(ql >= 0)
+    T = max(int(ql.max()) if ql.size else 0, 1)
+    pr = make_problem(name=name, q_tokens=T, **kw)
+    cu = np.zeros(ql.size + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(ql)
+    assert cu[-1] < 2 ** 31
+    pr.q = np.ascontiguousarray(np.concatenate([pr.q[b, : ql[b]] for b in range(ql.size)], axis=0)
+                                if ql.size else np.zeros((0, pr.n_q_heads, pr.head_dim), dtype=np.uint16))
+    pr.cu_q = cu.astype(np.int32)
+    return pr
 
 
 def make_config(name: str, **overrides) -> Problem:
