@@ -331,6 +331,28 @@ DECATTN_API int dec_attn_prefill(const dec_attn_shape *shape, const void *q, con
                                  const int32_t *page_table, const int32_t *seq_lens, float *out, float *lse,
                                  int32_t *status, void *stream);
 
+/* Variable-length prefill (the same passage: "variable-length prefill"): request b has its own
+ * number of query rows Tb = cu_q_lens[b + 1] - cu_q_lens[b] >= 0, its last Tb positions, and the
+ * rows of all requests are packed back to back. Row t < Tb of request b is packed row
+ * cu_q_lens[b] + t and attends to keys 0 .. seq_lens[b] - Tb + t (rows before position 0 see
+ * nothing: out = 0, lse = -inf). By definition each request is computed as dec_attn_prefill of
+ * that request alone with T = Tb. Same kernel and tolerances as dec_attn_prefill.
+ *   shape        as dec_attn_prefill, with q_tokens = the largest Tb of the batch (>= 1): it sizes
+ *                the grid; a request with more rows is reported as below and left unwritten;
+ *   q            device bf16 [total_q_rows][Hq][128], 16-byte aligned;
+ *   cu_q_lens    device int32 [batch + 1]: non-decreasing row offsets, cu_q_lens[0] = 0 and
+ *                cu_q_lens[batch] = total_q_rows (4-byte aligned);
+ *   total_q_rows host: the number of packed rows;
+ *   out, lse     device fp32 [total_q_rows][Hq][128] and [total_q_rows][Hq] (out 16-byte aligned);
+ *   status       optional device int32: DECATTN_EDEVICE also when a request's offsets fall outside
+ *                [0, total_q_rows] or its Tb exceeds q_tokens (that request is not written).
+ * The ragged last 32-row group of each request is written with plain stores, the rest by TMA
+ * stores, so rows of one request never overwrite another's. Returns as dec_attn_prefill. */
+DECATTN_API int dec_attn_prefill_varlen(const dec_attn_shape *shape, const void *q, const void *k_pages,
+                                        const void *v_pages, const int32_t *page_table, const int32_t *seq_lens,
+                                        const int32_t *cu_q_lens, int64_t total_q_rows, float *out, float *lse,
+                                        int32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,8 @@ OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1
 KV_BF16, KV_FP8E4M3, KV_FP8E4M3_MMA8 = 0, 1, 2
 API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
-       "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_prefill", "dec_attn_plan_sparse_bytes",
+       "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_prefill",
+       "dec_attn_prefill_varlen", "dec_attn_plan_sparse_bytes",
        "dec_attn_plan_sparse", "dec_attn_last_error")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -101,6 +102,8 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_append_rope.restype = i32
         lib.dec_attn_prefill.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.dec_attn_prefill.restype = i32
+        lib.dec_attn_prefill_varlen.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp]
+        lib.dec_attn_prefill_varlen.restype = i32
         _lib = lib
         return lib
 
@@ -324,6 +327,30 @@ def prefill(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_
                               _ptr(seq_lens), _ptr(out), _ptr(lse), _ptr(status), _stream_handle(stream))
     if rc != OK:
         raise DecAttnError(rc, "dec_attn_prefill")
+    return out, lse
+
+
+def prefill_varlen(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, page_table: torch.Tensor,
+                   seq_lens: torch.Tensor, cu_q_lens: torch.Tensor, max_q_rows: int, *, sm_scale: float = 0.0,
+                   out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                   status: torch.Tensor | None = None, stream=None):
+    """dec_attn_prefill_varlen: request b's rows are the packed rows cu_q_lens[b] .. cu_q_lens[b+1]-1
+    of q [total][Hq][128] (its last Tb positions); ``max_q_rows`` bounds every Tb. Returns (out fp32
+    [total][Hq][128], lse fp32 [total][Hq])."""
+    lib = load_library()
+    total, Hq, d = q.shape
+    B = page_table.shape[0]
+    shape = ShapeT(B, Hq, k_pages.shape[1], d, int(max_q_rows), k_pages.shape[2], k_pages.shape[0],
+                   page_table.shape[1], kv_dtype_of(k_pages), float(sm_scale))
+    if out is None:
+        out = torch.empty((total, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((total, Hq), dtype=torch.float32, device=q.device)
+    rc = lib.dec_attn_prefill_varlen(C.byref(shape), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
+                                     _ptr(seq_lens), _ptr(cu_q_lens), int(total), _ptr(out), _ptr(lse), _ptr(status),
+                                     _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_prefill_varlen")
     return out, lse
 
 

@@ -90,32 +90,32 @@ static bool make_kv_map(CUtensorMap* map, const void* base, int kv_dtype, int D,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Prefill queries as a 4-D bf16 tensor {head dim, q head, query row, request} (q is
-// [B][T][Hq][D]); the kernel loads boxes of 64 head dims x 128 rows with 128-byte swizzle, the
-// K-major layout of the MMA's A operand. Rows past T read as zeros.
-static bool make_prefill_q_map(CUtensorMap* map, const void* q, int B, int T, int Hq, int D) {
+// Prefill queries as a 3-D bf16 tensor {head dim, q head, packed row} (q is [rows][Hq][D]); the
+// kernel loads boxes of 64 head dims x 128 rows with 128-byte swizzle, the K-major layout of the
+// MMA's A operand. Rows past the last one read as zeros.
+static bool make_prefill_q_map(CUtensorMap* map, const void* q, int64_t rows, int Hq, int D) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2, (cuuint64_t)T * Hq * D * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box, estr,
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Prefill output as a 4-D fp32 tensor {head dim, q head, query row, request} (out is
-// [B][T][Hq][D]); the kernel stores boxes of 32 rows x 32 head dims with 128-byte swizzle.
-// Rows past T are outside the map, so a partial tile's store writes only its own rows.
-static bool make_prefill_out_map(CUtensorMap* map, float* out, int B, int T, int Hq, int D) {
+// Prefill output as a 3-D fp32 tensor {head dim, q head, packed row} (out is [rows][Hq][D]); the
+// kernel stores boxes of 32 rows x 32 head dims with 128-byte swizzle, only boxes whose rows all
+// belong to one request (the ragged last box of a request is written with plain stores).
+static bool make_prefill_out_map(CUtensorMap* map, float* out, int64_t rows, int Hq, int D) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)Hq * D * 4, (cuuint64_t)T * Hq * D * 4};
-  cuuint32_t box[4] = {32, 1, 32, 1};
-  cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)Hq * D * 4};
+  cuuint32_t box[3] = {32, 1, 32};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
@@ -246,6 +246,52 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
   return DECATTN_OK;
 }
 
+// Shared by dec_attn_prefill (cu_q null: T rows per request) and dec_attn_prefill_varlen.
+static int prefill_enqueue(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
+                           const int32_t* page_table, const int32_t* seq_lens, const int32_t* cu_q,
+                           int64_t total_rows, float* out, float* lse, int32_t* status, void* stream) {
+  if (!shape) return DECATTN_EINVAL;
+  const dec_attn_shape& s = *shape;
+  if (s.batch < 0 || s.q_tokens <= 0 || s.n_q_heads <= 0 || s.n_kv_heads <= 0 || s.page_size <= 0 ||
+      s.num_pages < 0 || s.max_pages_per_seq < 0 || s.n_q_heads % s.n_kv_heads != 0 || total_rows < 0)
+    return DECATTN_EINVAL;
+  if (s.kv_dtype != DECATTN_KV_BF16 || s.head_dim != 128 || s.page_size % 16 != 0) return DECATTN_ENOTSUP;
+  if (s.batch > 65535 || s.n_q_heads > 65535) return DECATTN_ENOTSUP;
+  if (total_rows * s.n_q_heads >= (1ll << 31) || (int64_t)s.batch * s.q_tokens >= (1ll << 31) ||
+      (int64_t)s.num_pages * s.n_kv_heads * s.page_size >= (1ll << 31))
+    return DECATTN_ENOTSUP;
+  if (s.batch == 0 || total_rows == 0) return DECATTN_OK;
+  if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !out || !lse) return DECATTN_EINVAL;
+  if (s.num_pages <= 0 || s.max_pages_per_seq <= 0) return DECATTN_EINVAL;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out)) return DECATTN_EALIGN;
+  if (((reinterpret_cast<uintptr_t>(page_table) | reinterpret_cast<uintptr_t>(seq_lens) |
+        reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(status) | reinterpret_cast<uintptr_t>(cu_q)) &
+       3) != 0)
+    return DECATTN_EALIGN;
+  CUtensorMap tmQ, tmK, tmV, tmO;
+  const int64_t rows = (int64_t)s.num_pages * s.n_kv_heads * s.page_size;
+  if (!make_prefill_q_map(&tmQ, q, total_rows, s.n_q_heads, s.head_dim) ||
+      !make_kv_map(&tmK, k_pages, s.kv_dtype, s.head_dim, rows) ||
+      !make_kv_map(&tmV, v_pages, s.kv_dtype, s.head_dim, rows) ||
+      !make_prefill_out_map(&tmO, out, total_rows, s.n_q_heads, s.head_dim))
+    return cuda_fail("prefill tensor maps (cuTensorMapEncodeTiled)");
+  const float scale = s.sm_scale > 0.f ? s.sm_scale : 1.0f / sqrtf((float)s.head_dim);
+  PrefillParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.page_table = page_table;
+  p.seq_lens = seq_lens;
+  p.cu_q = cu_q;
+  p.out = out;
+  p.lse = lse;
+  p.status = status;
+  p.B = s.batch; p.T = s.q_tokens; p.Hq = s.n_q_heads; p.Hkv = s.n_kv_heads; p.G = s.n_q_heads / s.n_kv_heads;
+  p.P = s.page_size; p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
+  p.total_rows = total_rows;
+  p.qk_scale_log2 = scale * 1.4426950408889634f;
+  const cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, tmO, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DECATTN_OK : cuda_fail("prefill kernel launch", e);
+}
+
 }  // namespace decattn
 
 using namespace decattn;
@@ -254,42 +300,19 @@ extern "C" int dec_attn_prefill(const dec_attn_shape* shape, const void* q, cons
                                 const int32_t* page_table, const int32_t* seq_lens, float* out, float* lse,
                                 int32_t* status, void* stream) {
   if (!shape) return DECATTN_EINVAL;
-  const dec_attn_shape& s = *shape;
-  if (s.batch < 0 || s.q_tokens <= 0 || s.n_q_heads <= 0 || s.n_kv_heads <= 0 || s.page_size <= 0 ||
-      s.num_pages < 0 || s.max_pages_per_seq < 0 || s.n_q_heads % s.n_kv_heads != 0)
-    return DECATTN_EINVAL;
-  if (s.kv_dtype != DECATTN_KV_BF16 || s.head_dim != 128 || s.page_size % 16 != 0) return DECATTN_ENOTSUP;
-  if (s.batch > 65535 || s.n_q_heads > 65535) return DECATTN_ENOTSUP;
-  if ((int64_t)s.batch * s.q_tokens * s.n_q_heads >= (1ll << 31) ||
-      (int64_t)s.num_pages * s.n_kv_heads * s.page_size >= (1ll << 31))
-    return DECATTN_ENOTSUP;
-  if (s.batch == 0) return DECATTN_OK;
-  if (!q || !k_pages || !v_pages || !page_table || !seq_lens || !out || !lse) return DECATTN_EINVAL;
-  if (s.num_pages <= 0 || s.max_pages_per_seq <= 0) return DECATTN_EINVAL;
-  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out)) return DECATTN_EALIGN;
-  if (((reinterpret_cast<uintptr_t>(page_table) | reinterpret_cast<uintptr_t>(seq_lens) |
-        reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(status)) & 3) != 0)
-    return DECATTN_EALIGN;
-  CUtensorMap tmQ, tmK, tmV, tmO;
-  const int64_t rows = (int64_t)s.num_pages * s.n_kv_heads * s.page_size;
-  if (!make_prefill_q_map(&tmQ, q, s.batch, s.q_tokens, s.n_q_heads, s.head_dim) ||
-      !make_kv_map(&tmK, k_pages, s.kv_dtype, s.head_dim, rows) ||
-      !make_kv_map(&tmV, v_pages, s.kv_dtype, s.head_dim, rows) ||
-      !make_prefill_out_map(&tmO, out, s.batch, s.q_tokens, s.n_q_heads, s.head_dim))
-    return cuda_fail("prefill tensor maps (cuTensorMapEncodeTiled)");
-  const float scale = s.sm_scale > 0.f ? s.sm_scale : 1.0f / sqrtf((float)s.head_dim);
-  PrefillParams p;
-  p.q = static_cast<const uint16_t*>(q);
-  p.page_table = page_table;
-  p.seq_lens = seq_lens;
-  p.out = out;
-  p.lse = lse;
-  p.status = status;
-  p.B = s.batch; p.T = s.q_tokens; p.Hq = s.n_q_heads; p.Hkv = s.n_kv_heads; p.G = s.n_q_heads / s.n_kv_heads;
-  p.P = s.page_size; p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
-  p.qk_scale_log2 = scale * 1.4426950408889634f;
-  const cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, tmO, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? DECATTN_OK : cuda_fail("prefill kernel launch", e);
+  if (shape->batch < 0 || shape->q_tokens <= 0) return DECATTN_EINVAL;
+  return prefill_enqueue(shape, q, k_pages, v_pages, page_table, seq_lens, nullptr,
+                         (int64_t)shape->batch * shape->q_tokens, out, lse, status, stream);
+}
+
+extern "C" int dec_attn_prefill_varlen(const dec_attn_shape* shape, const void* q, const void* k_pages,
+                                       const void* v_pages, const int32_t* page_table, const int32_t* seq_lens,
+                                       const int32_t* cu_q_lens, int64_t total_q_rows, float* out, float* lse,
+                                       int32_t* status, void* stream) {
+  if (!shape) return DECATTN_EINVAL;
+  if (shape->batch > 0 && total_q_rows > 0 && !cu_q_lens) return DECATTN_EINVAL;
+  return prefill_enqueue(shape, q, k_pages, v_pages, page_table, seq_lens, cu_q_lens, total_q_rows, out, lse, status,
+                         stream);
 }
 
 extern "C" int dec_attn_default_bins(int device) { return default_bins(device); }

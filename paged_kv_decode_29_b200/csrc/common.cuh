@@ -177,15 +177,20 @@ struct SplitParams {
   float qk_scale_log2;      // sm_scale * log2(e)
 };
 
-// Arguments of the prefill kernel (prefill.cu).
+// Arguments of the prefill kernel (prefill.cu). Query rows are packed: request b's Tb rows are
+// rows qoff_b .. qoff_b + Tb - 1 of q [total_rows][Hq][D] (and of out / lse), with qoff_b = b T and
+// Tb = T when cu_q is null (every request has T rows), else qoff_b = cu_q[b], Tb = cu_q[b+1] -
+// cu_q[b] <= T (variable-length rows).
 struct PrefillParams {
-  const uint16_t* q;          // bf16 [B][T][Hq][D]
+  const uint16_t* q;          // bf16 [total_rows][Hq][D]
   const int32_t* page_table;  // [B][mpps]
   const int32_t* seq_lens;    // [B]
-  float* out;                 // [B][T][Hq][D]
-  float* lse;                 // [B][T][Hq]
+  const int32_t* cu_q;        // [B + 1] row offsets, or null
+  float* out;                 // [total_rows][Hq][D]
+  float* lse;                 // [total_rows][Hq]
   int32_t* status;            // optional device word
   int B, T, Hq, Hkv, G, P, num_pages, mpps;
+  int64_t total_rows;
   float qk_scale_log2;        // sm_scale * log2(e)
 };
 

@@ -131,20 +131,19 @@ __device__ __forceinline__ float pf_exp(uint32_t tS, const float (&v)[128], floa
   return (la0 + la1) + (lb0 + lb1);
 }
 
-// 4-D tiled TMA load into shared memory, completion signalled on an mbarrier.
-__device__ __forceinline__ void pf_tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
-                                               uint64_t* bar) {
+// 3-D tiled TMA load into shared memory, completion signalled on an mbarrier.
+__device__ __forceinline__ void pf_tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(
+      "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
           smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
 
-// 4-D tiled TMA store of a shared-memory box, tracked by this thread's bulk async-groups.
-__device__ __forceinline__ void pf_tma_store_4d(const CUtensorMap* map, const void* src, int x, int y, int z, int w) {
-  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(map),
-               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "r"(w)
+// 3-D tiled TMA store of a shared-memory box, tracked by this thread's bulk async-groups.
+__device__ __forceinline__ void pf_tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
                : "memory");
 }
 __device__ __forceinline__ void pf_bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -176,18 +175,36 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
   const int rem = (int)blockIdx.x % (p.B * ny);
   const int b = rem / ny, y = rem % ny;
   const int Lb = p.seq_lens[b];
+  // the request's query rows: Tb of them from packed row qoff on
+  int Tb = p.T;
+  int qoff = b * p.T;  // packed rows times Hq stay below 2^31 (checked on the host)
+  if (p.cu_q) {
+    const int c0 = p.cu_q[b], c1 = p.cu_q[b + 1];
+    Tb = c1 - c0;
+    qoff = c0;
+    if (c0 < 0 || Tb < 0 || Tb > p.T || (int64_t)c1 > p.total_rows) {  // offsets outside the packed rows
+      if (threadIdx.x == 0) set_status(p.status, DECATTN_EDEVICE);
+      return;
+    }
+  }
   PfTile tl0, tl1;
   {
     tl0.qh = head_pair ? 2 * y : y;
     tl1.qh = head_pair ? 2 * y + 1 : y;
     tl0.t0 = head_pair ? step * kPfM : 2 * step * kPfM;
     tl1.t0 = head_pair ? step * kPfM : (2 * step + 1) * kPfM;
-    // keys the tile's last row sees: [0, min(Lb, Lb - T + t_last + 1))
-    const int tlast0 = min(tl0.t0 + kPfM, p.T) - 1, tlast1 = min(tl1.t0 + kPfM, p.T) - 1;
-    const int kmax0 = (Lb < 0 || tl0.t0 >= p.T) ? 0 : max(0, min(Lb, Lb - p.T + tlast0 + 1));
-    const int kmax1 = (Lb < 0 || tl1.t0 >= p.T) ? 0 : max(0, min(Lb, Lb - p.T + tlast1 + 1));
+    // keys the tile's last row sees: [0, min(Lb, Lb - Tb + t_last + 1))
+    const int tlast0 = min(tl0.t0 + kPfM, Tb) - 1, tlast1 = min(tl1.t0 + kPfM, Tb) - 1;
+    const int kmax0 = (Lb < 0 || tl0.t0 >= Tb) ? 0 : max(0, min(Lb, Lb - Tb + tlast0 + 1));
+    const int kmax1 = (Lb < 0 || tl1.t0 >= Tb) ? 0 : max(0, min(Lb, Lb - Tb + tlast1 + 1));
     tl0.nkb = (kmax0 + kPfN - 1) / kPfN;
     tl1.nkb = (kmax1 + kPfN - 1) / kPfN;
+  }
+  // a row block past the request's rows (variable-length rows, or T not a multiple of two
+  // blocks): nothing to compute or write; the whole CTA leaves before it sets anything up
+  if (tl0.t0 >= Tb && tl1.t0 >= Tb) {
+    if (threadIdx.x == 0 && Lb < 0) set_status(p.status, DECATTN_EDEVICE);
+    return;
   }
   const int h = tl0.qh / p.G;
   const int nkb_max = max(tl0.nkb, tl1.nkb);
@@ -227,13 +244,15 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      // Q of both tiles: per tile two boxes of 64 head dims x 128 rows, which land as the two
-      // K-major 128-byte-swizzled atoms the MMA reads; rows past T read as zeros
+      // Q of both tiles: per tile two boxes of 64 head dims x 128 packed rows, which land as the
+      // two K-major 128-byte-swizzled atoms the MMA reads. Rows past the request's Tb belong to
+      // the next request (or read as zeros past the last row): they are computed and never written.
       mbar_arrive_expect_tx(&bar[kPfQFull], 4u * (uint32_t)L::ATOM);
       #pragma unroll
       for (int a = 0; a < 2; ++a) {
-        pf_tma_load_4d(sm + L::OFF_Q + a * L::ATOM, &tmQ, 64 * a, tl0.qh, tl0.t0, b, &bar[kPfQFull]);
-        pf_tma_load_4d(sm + L::OFF_Q + L::TILE + a * L::ATOM, &tmQ, 64 * a, tl1.qh, tl1.t0, b, &bar[kPfQFull]);
+        pf_tma_load_3d(sm + L::OFF_Q + a * L::ATOM, &tmQ, 64 * a, tl0.qh, qoff + tl0.t0, &bar[kPfQFull]);
+        pf_tma_load_3d(sm + L::OFF_Q + L::TILE + a * L::ATOM, &tmQ, 64 * a, tl1.qh, qoff + tl1.t0,
+                       &bar[kPfQFull]);
       }
     }
     int nk = 0, nv = 0;  // K / V blocks whose copies were issued
@@ -380,7 +399,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
     const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
     const uint32_t tS = tmem + lane_off + kPfN * u;
     const uint32_t tO = tmem + lane_off + 2 * kPfN + kPfD * u;
-    const int lim = t < p.T ? Lb - p.T + t : -1;  // the last key this row sees (< 0: none)
+    const int lim = t < Tb ? Lb - Tb + t : -1;  // the last key this row sees (< 0: none)
     const int lim_min = __reduce_min_sync(0xffffffffu, lim);
     const float sc = p.qk_scale_log2;
     float mref = -INFINITY, l = 0.f;  // reference maximum (log2 units) and row sum
@@ -440,11 +459,13 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
       // O / l through shared memory: this warp's 32 rows, 32 columns at a time, into one of two
       // 4 KB boxes in its tile's Q area (no tensor-core operation reads Q_u any more: they all
       // completed before the tile's last P V), swizzled as the store's tensor map expects (row i
-      // at 128 i, 16-byte chunk c at (c ^ (i % 8)) * 16), then a TMA store of the box to
-      // out[b][t0w .. t0w + 31][qh][32 q4 ..]. Rows past T fall outside the map and are not written.
+      // at 128 i, 16-byte chunk c at (c ^ (i % 8)) * 16), then a TMA store of the box to packed
+      // rows qoff + t0w .. qoff + t0w + 31, head qh, head dims 32 q4 ... A warp whose 32 rows run
+      // past the request's last row (the next rows are another request's) stores its valid rows
+      // with plain stores instead.
       tc_fence_after();
       const int t0w = t - lane;  // the warp's first row
-      const bool any_row = t0w < p.T;
+      const bool whole_box = t0w + 32 <= Tb;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint8_t* stage = sm + L::OFF_Q + warp * 8192;
       #pragma unroll
@@ -455,6 +476,15 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
         } else {
           #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+        if (!whole_box) {
+          if (t < Tb) {
+            float4* dst = reinterpret_cast<float4*>(p.out + ((int64_t)(qoff + t) * p.Hq + qh) * kPfD + 32 * q4);
+            #pragma unroll
+            for (int c = 0; c < 8; ++c)
+              dst[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv, o[4 * c + 3] * inv);
+          }
+          continue;
         }
         uint8_t* box = stage + (q4 & 1) * 4096;
         if (q4 >= 2) {  // the store that read this box two chunks ago
@@ -467,14 +497,14 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
               make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv, o[4 * c + 3] * inv);
         fence_async_smem();
         __syncwarp();
-        if (lane == 0 && any_row) {
-          pf_tma_store_4d(&tmO, box, 32 * q4, qh, t0w, b);
+        if (lane == 0) {
+          pf_tma_store_3d(&tmO, box, 32 * q4, qh, qoff + t0w);
           pf_bulk_commit();
         }
       }
       if (lane == 0) pf_bulk_wait_all();
       __syncwarp();
-      if (t < p.T) p.lse[((int64_t)b * p.T + t) * p.Hq + qh] = l > 0.f ? (mref + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      if (t < Tb) p.lse[(int64_t)(qoff + t) * p.Hq + qh] = l > 0.f ? (mref + __log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
   }
 

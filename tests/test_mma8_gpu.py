@@ -48,8 +48,12 @@ def _row_stats(pr, rows, ref_o):
     """Per (b, t, qh) row: max_j |v_j - ref| over the row's visible keys j and all head dims, and
     sqrt(sum_j a_j^2 m_j) with a_j the oracle's softmax weights and m_j = mean_c (v_jc - ref_c)^2.
     The maximum uses running maxima / minima of V over the keys (one pass per (request, KV head))."""
+    from concurrent.futures import ThreadPoolExecutor
     vdev = np.zeros(len(rows))
     wdev = np.zeros(len(rows))
+    # the oracle's weights of every row, on all cores (the C oracle runs without the GIL)
+    with ThreadPoolExecutor(max(1, oracle.max_threads())) as ex:
+        weights = list(ex.map(lambda r: oracle.attend(pr, int(r[0]), int(r[1]), int(r[2]), weights=True)[3], rows))
     by_pair = {}
     for i, (b, t, qh) in enumerate(rows):
         by_pair.setdefault((int(b), int(qh) // pr.group), []).append(i)
@@ -70,7 +74,8 @@ def _row_stats(pr, rows, ref_o):
                 continue
             ref = ref_o[i]
             vdev[i] = max(float(np.max(vmax[vis - 1] - ref)), float(np.max(ref - vmin[vis - 1])))
-            _, _, n, w = oracle.attend(pr, b, int(t), int(qh), weights=True)
+            w = weights[i]
+            n = w.shape[0]
             a2 = w * w
             d = pr.head_dim
             # sum_j a_j^2 mean_c (v_jc - ref_c)^2 = sum_j a_j^2 (|v_j|^2 - 2 v_j.ref + |ref|^2) / d
