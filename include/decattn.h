@@ -267,6 +267,19 @@ DECATTN_API int dec_attn_read_status(const dec_attn_plan_t *plan, const void *wo
  * written); returns the full message length (0: no DECATTN_ECUDA on this thread yet). Host only. */
 DECATTN_API size_t dec_attn_last_error(char *buf, size_t len);
 
+/* For tests of the bounded pipeline waits; the pages have no counterpart (it exists so that the
+ * failure path of every wait can be exercised without a GPU fault). Every mbarrier wait of the
+ * split and prefill kernels gives up after a limit (2 s by default), sets DECATTN_ETIMEOUT and
+ * lets the CTA leave in order (copies already issued land first, tensor memory is freed). This
+ * call sets, for the launches that follow it in this process:
+ *   limit_ns   the wait limit in ns, 1e5 .. 2e9 (0: back to the default);
+ *   skip_fill  >= 0: CTA 0's producer leaves that one pipeline fill out (ring fill of the split
+ *              kernels, K block of the prefill kernel), so that the waits on it run out and the
+ *              run ends with DECATTN_ETIMEOUT; -1: none (the default).
+ * Returns DECATTN_EINVAL for values outside those ranges. Not thread-safe against launches on
+ * other threads; not for production use. */
+DECATTN_API int dec_attn_test_set_waits(uint64_t limit_ns, int32_t skip_fill);
+
 /* Static text for a decattn_status value. */
 DECATTN_API const char *dec_attn_status_string(int status);
 

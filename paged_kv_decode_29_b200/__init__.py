@@ -30,7 +30,7 @@ API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_att
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
        "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_prefill",
        "dec_attn_prefill_varlen", "dec_attn_plan_sparse_bytes",
-       "dec_attn_plan_sparse", "dec_attn_last_error")
+       "dec_attn_plan_sparse", "dec_attn_last_error", "dec_attn_test_set_waits")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -104,6 +104,8 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_prefill.restype = i32
         lib.dec_attn_prefill_varlen.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp]
         lib.dec_attn_prefill_varlen.restype = i32
+        lib.dec_attn_test_set_waits.argtypes = [C.c_uint64, C.c_int32]
+        lib.dec_attn_test_set_waits.restype = i32
         _lib = lib
         return lib
 
@@ -352,6 +354,14 @@ def prefill_varlen(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor
     if rc != OK:
         raise DecAttnError(rc, "dec_attn_prefill_varlen")
     return out, lse
+
+
+def test_set_waits(limit_ns: int = 0, skip_fill: int = -1) -> None:
+    """dec_attn_test_set_waits: the wait limit (0: the default 2 s) and a pipeline fill of CTA 0 to
+    leave out (-1: none) for the launches that follow; for tests of the bounded waits only."""
+    rc = load_library().dec_attn_test_set_waits(int(limit_ns), int(skip_fill))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_test_set_waits")
 
 
 def read_status(pl: Plan | None = None, workspace: torch.Tensor | None = None, stream=None) -> int:

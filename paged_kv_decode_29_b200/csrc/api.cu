@@ -26,6 +26,17 @@ int cuda_fail(const char* what, cudaError_t e) {
   return DECATTN_ECUDA;
 }
 
+// Wait limit and left-out fill of the next launches (dec_attn_test_set_waits): the library's
+// default unless a test of the bounded waits lowers them.
+static uint64_t g_test_wait_ns = kWaitLimitNs;
+static int32_t g_test_skip_fill = -1;
+
+void test_waits(uint64_t* wait_ns, int32_t* skip_fill) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  *wait_ns = g_test_wait_ns;
+  *skip_fill = g_test_skip_fill;
+}
+
 int default_bins(int device) {
   static std::map<int, int> cache;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -225,6 +236,7 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
     sp.P = s.page_size; sp.num_pages = s.num_pages; sp.mpps = s.max_pages_per_seq; sp.n_bins = plan->n_bins;
     sp.tile_len = plan->tile_len; sp.max_units = plan->max_units; sp.sparse = plan->sparse;
     sp.qk_scale_log2 = scale * 1.4426950408889634f;
+    test_waits(&sp.wait_ns, &sp.skip_fill);
     if (const cudaError_t e = launch_split(sp, tmK, tmV, s.kv_dtype, D, st); e != cudaSuccess)
       return cuda_fail("split kernel launch", e);
   }
@@ -288,6 +300,7 @@ static int prefill_enqueue(const dec_attn_shape* shape, const void* q, const voi
   p.P = s.page_size; p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
   p.total_rows = total_rows;
   p.qk_scale_log2 = scale * 1.4426950408889634f;
+  test_waits(&p.wait_ns, &p.skip_fill);
   const cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, tmO, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DECATTN_OK : cuda_fail("prefill kernel launch", e);
 }
@@ -358,6 +371,15 @@ extern "C" int dec_attn_read_status(const dec_attn_plan_t* plan, const void* wor
     if (h.status != DECATTN_OK) return h.status;
     if (h.run_status != DECATTN_OK) return h.run_status;
   }
+  return DECATTN_OK;
+}
+
+extern "C" int dec_attn_test_set_waits(uint64_t limit_ns, int32_t skip_fill) {
+  if (limit_ns != 0 && (limit_ns < 100000ull || limit_ns > kWaitLimitNs)) return DECATTN_EINVAL;
+  if (skip_fill < -1) return DECATTN_EINVAL;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_test_wait_ns = limit_ns == 0 ? kWaitLimitNs : limit_ns;
+  g_test_skip_fill = skip_fill;
   return DECATTN_OK;
 }
 

@@ -175,6 +175,8 @@ struct SplitParams {
   int sparse;               // the plan is block-sparse (its tiles come from the plan only)
   int64_t max_units;        // the plan's capacity (partial slots of the workspace)
   float qk_scale_log2;      // sm_scale * log2(e)
+  uint64_t wait_ns;         // a pipeline wait gives up after this long (kWaitLimitNs unless a test lowers it)
+  int32_t skip_fill;        // tests only: CTA 0's producer leaves this ring fill out (-1: none)
 };
 
 // Arguments of the prefill kernel (prefill.cu). Query rows are packed: request b's Tb rows are
@@ -192,6 +194,8 @@ struct PrefillParams {
   int B, T, Hq, Hkv, G, P, num_pages, mpps;
   int64_t total_rows;
   float qk_scale_log2;        // sm_scale * log2(e)
+  uint64_t wait_ns;           // a pipeline wait gives up after this long
+  int32_t skip_fill;          // tests only: CTA 0's producer leaves this K block out (-1: none)
 };
 
 // Query rows of one KV head that a decode tile computes at once (G * T), and query tokens per
@@ -280,15 +284,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Returns false (after setting
-// DECATTN_ETIMEOUT) if it has not completed within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+// DECATTN_ETIMEOUT) if it has not completed within limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     #pragma unroll 1
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_status(status, DECATTN_ETIMEOUT);
       return false;
     }
@@ -297,9 +302,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
 
 // Lane 0 waits and tells the rest of the warp (used where only lane 0 touches the staged
 // data afterwards, e.g. the thread that issues the next copy into a freed stage).
-__device__ __forceinline__ bool warp_wait_lane0(uint64_t* bar, uint32_t parity, int32_t* status) {
+__device__ __forceinline__ bool warp_wait_lane0(uint64_t* bar, uint32_t parity, int32_t* status,
+                                                uint64_t limit_ns = kWaitLimitNs) {
   int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, status, limit_ns) ? 1 : 0;
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -447,6 +453,8 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
 }
 
 // ------------------------------------------------------------------ host-side launchers
+// Wait limit and left-out fill for the next launches (api.cu; tests of the bounded waits).
+void test_waits(uint64_t* wait_ns, int32_t* skip_fill);
 int default_bins(int device);                                     // api.cu
 bool ensure_smem_attr(const void* kernel, int bytes);             // api.cu
 bool split_supported(int kv_dtype, int D, int GT);                // split.cu

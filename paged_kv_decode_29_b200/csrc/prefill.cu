@@ -165,6 +165,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
   uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(sm + L::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t wl = p.wait_ns;  // every pipeline wait gives up after this long
 
   // ---- request, KV head and the two tiles of this CTA. The row-block step is the slowest
   //      index of the grid, counted down, so the CTAs with the most keys start first.
@@ -274,18 +275,20 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
       }
       const uint32_t bytes = (uint32_t)__popc(__ballot_sync(0xffffffffu, has)) * 2u * 16u * 128u;
       int r = 1;
-      if (lane == 0) r = tc_wait_suspend(&bar[kPfKEmpty + st], eph, p.status, abort) ? 1 : 0;
+      if (lane == 0) r = tc_wait_suspend(&bar[kPfKEmpty + st], eph, p.status, abort, wl) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, r, 0)) break;
-      if (lane == 0) mbar_arrive_expect_tx(&bar[kPfKFull + st], bytes);
+      // tests of the bounded waits leave one K block of CTA 0 out: nothing completes that stage
+      const bool fill = !(blockIdx.x == 0 && g == p.skip_fill);
+      if (fill && lane == 0) mbar_arrive_expect_tx(&bar[kPfKFull + st], bytes);
       __syncwarp();
-      if (has) {
+      if (fill && has) {
         #pragma unroll
         for (int a = 0; a < 2; ++a)  // head dims 64a .. 64a + 63: one 128-byte swizzled atom
           tma_load_2d(sm + L::OFF_K + st * L::TILE + a * L::ATOM + lane * 16 * 128, &tmK, 64 * a, row,
                       &bar[kPfKFull + st]);
       }
       ++nk;
-      if (lane == 0) r = tc_wait_suspend(&bar[kPfVEmpty + st], eph, p.status, abort) ? 1 : 0;
+      if (lane == 0) r = tc_wait_suspend(&bar[kPfVEmpty + st], eph, p.status, abort, wl) ? 1 : 0;
       if (!__shfl_sync(0xffffffffu, r, 0)) break;
       if (lane < kPfN / 16 && !has) {
         // keys past the request's end: no copy; their P is 0, so their V rows must be finite
@@ -309,9 +312,9 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
     if (*abort && lane == 0) {
       // let the copies already issued land before the CTA exits
       for (int n = max(nk - kPfStages, 0); n < nk; ++n)
-        mbar_wait(&bar[kPfKFull + n % kPfStages], (uint32_t)((n / kPfStages) & 1), nullptr);
+        mbar_wait(&bar[kPfKFull + n % kPfStages], (uint32_t)((n / kPfStages) & 1), nullptr, wl);
       for (int n = max(nv - kPfStages, 0); n < nv; ++n)
-        mbar_wait(&bar[kPfVFull + n % kPfStages], (uint32_t)((n / kPfStages) & 1), nullptr);
+        mbar_wait(&bar[kPfVFull + n % kPfStages], (uint32_t)((n / kPfStages) & 1), nullptr, wl);
     }
   } else if (warp == 9) {
     // ===================================================================== MMA issue
@@ -344,9 +347,9 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
         for (int k = 0; k < kPfN / 16; ++k)  // V advances 16 keys = 2 KB
           umma_f16_tmem_a(tO, tP + 8 * k, dV + (uint64_t)((k * 2048) >> 4), idO, (g > 0 || k > 0) ? 1u : 0u);
       };
-      bool ok = tc_wait_suspend(&bar[kPfQFull], 0, p.status, abort);
+      bool ok = tc_wait_suspend(&bar[kPfQFull], 0, p.status, abort, wl);
       if (ok && nkb_max > 0) {
-        ok = tc_wait_suspend(&bar[kPfKFull], 0, p.status, abort);
+        ok = tc_wait_suspend(&bar[kPfKFull], 0, p.status, abort, wl);
         if (ok) {
           tc_fence_after();
           if (nkb[0] > 0) issue_s(0, 0);
@@ -361,10 +364,10 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
         for (int u = 0; u < 2; ++u) {
           if (g >= nkb[u]) continue;
           if (!v_ready) {
-            if (!tc_wait_suspend(&bar[kPfVFull + st], (uint32_t)((g / kPfStages) & 1), p.status, abort)) { ok = false; break; }
+            if (!tc_wait_suspend(&bar[kPfVFull + st], (uint32_t)((g / kPfStages) & 1), p.status, abort, wl)) { ok = false; break; }
             v_ready = true;
           }
-          if (!tc_wait_suspend(&bar[kPfPReady + u], (uint32_t)(g & 1), p.status, abort)) { ok = false; break; }
+          if (!tc_wait_suspend(&bar[kPfPReady + u], (uint32_t)(g & 1), p.status, abort, wl)) { ok = false; break; }
           tc_fence_after();
           issue_pv(u, g);
           if (u == 1 || g >= nkb[1]) umma_commit(&bar[kPfVEmpty + st]);  // the block's last P V
@@ -372,7 +375,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
           if (g + 1 < nkb[u]) {
             const int sn = (g + 1) % kPfStages;
             if (!k_ready) {
-              if (!tc_wait_suspend(&bar[kPfKFull + sn], (uint32_t)(((g + 1) / kPfStages) & 1), p.status, abort)) {
+              if (!tc_wait_suspend(&bar[kPfKFull + sn], (uint32_t)(((g + 1) / kPfStages) & 1), p.status, abort, wl)) {
                 ok = false;
                 break;
               }
@@ -405,7 +408,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
     float mref = -INFINITY, l = 0.f;  // reference maximum (log2 units) and row sum
     bool ok = true;
     for (int g = 0; g < nkb; ++g) {
-      if (!tc_wait_suspend_warp(&bar[kPfSFull + u], (uint32_t)(g & 1), p.status, abort)) { ok = false; break; }
+      if (!tc_wait_suspend_warp(&bar[kPfSFull + u], (uint32_t)(g & 1), p.status, abort, wl)) { ok = false; break; }
       tc_fence_after();
       const int j0 = g * kPfN;
       const bool masked = j0 + kPfN - 1 > lim_min;  // warp-uniform: some row does not see every key
@@ -453,7 +456,7 @@ prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ, c
       if (lane == 0) mbar_arrive(&bar[kPfPReady + u]);
     }
     // ---- epilogue: O / l and lse of row t
-    if (ok && nkb > 0 && !tc_wait_suspend_warp(&bar[kPfOFin + u], 0, p.status, abort)) ok = false;
+    if (ok && nkb > 0 && !tc_wait_suspend_warp(&bar[kPfOFin + u], 0, p.status, abort, wl)) ok = false;
     if (!ok) *abort = 1;
     if (ok) {  // warp-uniform: every lane takes part in the tensor-memory loads
       // O / l through shared memory: this warp's 32 rows, 32 columns at a time, into one of two

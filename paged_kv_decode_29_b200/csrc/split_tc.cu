@@ -166,6 +166,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
   uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(sm + L::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(sm + L::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t wl = p.wait_ns;  // every pipeline wait gives up after this long
 
   // The combine counters of this workspace start from zero on every run (as in split.cu).
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)p.B * p.T * p.Hq;
@@ -273,7 +274,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     };
     auto wait0 = [&](uint64_t* b, uint32_t par) -> bool {  // lane 0 waits, the warp follows
       int r = 1;
-      if (lane == 0) r = tc_wait(b, par, p.status, abort) ? 1 : 0;
+      if (lane == 0) r = tc_wait(b, par, p.status, abort, wl) ? 1 : 0;
       return __shfl_sync(0xffffffffu, r, 0) != 0;
     };
     Unit dn;
@@ -310,16 +311,18 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         }
         const int pid = __shfl_sync(0xffffffffu, pid_w, (ip - win * 32) & 31);
         if (!wait0(&bar[kKvEmpty + st], eph)) { ok = false; break; }
-        if (lane < nb) {  // FP8 page scales of the block (K, V), folded into the chunk's barrier
+        // tests of the bounded waits leave one chunk of CTA 0 out: nothing completes that stage
+        const bool fill = !(blockIdx.x == 0 && n_fill == p.skip_fill);
+        if (fill && lane < nb) {  // FP8 page scales of the block (K, V), folded into the chunk's barrier
           const int64_t si = (int64_t)pid * p.Hkv + d.h;
           cp_async_4(&sc[st * 16 + lane], p.kv_scales + si);
           cp_async_4(&sc[st * 16 + 8 + lane], p.kv_scales + (int64_t)p.num_pages * p.Hkv + si);
           cp_async_mbar_arrive(&bar[kKvFull + st]);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_expect_tx(&bar[kKvFull + st], (uint32_t)(nb * 2 * 16 * kTcD));
+        if (fill && lane == 0) mbar_arrive_expect_tx(&bar[kKvFull + st], (uint32_t)(nb * 2 * 16 * kTcD));
         __syncwarp();
-        if (lane < nb) {
+        if (fill && lane < nb) {
           const int row = (pid * p.Hkv + d.h) * P + (blk * 16) % P;
           tma_load_2d(sm + L::OFF_K + st * L::KCH + lane * 16 * kTcD, &tmK, 0, row, &bar[kKvFull + st]);
           tma_load_2d(sm + L::OFF_V + st * L::KCH + lane * 16 * kTcD, &tmV, 0, row, &bar[kKvFull + st]);
@@ -349,7 +352,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       *abort = 1;
       // let the copies already issued land before the CTA exits
       for (int64_t n = n_fill > kTcStages ? n_fill - kTcStages : 0; n < n_fill; ++n)
-        mbar_wait(&bar[kKvFull + n % kTcStages], (uint32_t)((n / kTcStages) & 1), nullptr);
+        mbar_wait(&bar[kKvFull + n % kTcStages], (uint32_t)((n / kTcStages) & 1), nullptr, wl);
     }
   } else if (warp == 5) {
     // ===================================================================== MMA issue
@@ -373,7 +376,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       // O^T (+)= V^T P^T over chunk gg's 128 keys. A tile's first chunk overwrites O^T: the
       // softmax group signals that chunk's P only after it has read the previous tile's O^T.
       auto pv = [&](int64_t gg, bool first_of_tile, uint32_t tO) -> bool {
-        if (!tc_wait(&bar[kPReady], (uint32_t)(gg & 1), p.status, abort)) return false;
+        if (!tc_wait(&bar[kPReady], (uint32_t)(gg & 1), p.status, abort, wl)) return false;
         tc_fence_after();
         if constexpr (Q8) {
           const int sg = (int)(gg % kTcStages);
@@ -392,19 +395,19 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         return true;
       };
       for (;;) {
-        if (!tc_wait(&bar[kUFull + us], uph, p.status, abort)) { ok = false; break; }
+        if (!tc_wait(&bar[kUFull + us], uph, p.status, abort, wl)) { ok = false; break; }
         const Unit d = umeta[us];
         mbar_arrive(&bar[kUEmpty + us]);
         us ^= 1; if (us == 0) uph ^= 1;
         if (d.b < 0) break;
         const int nc = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
-        if (!tc_wait(&bar[kQReady], (uint32_t)(ut & 1), p.status, abort)) { ok = false; break; }
+        if (!tc_wait(&bar[kQReady], (uint32_t)(ut & 1), p.status, abort, wl)) { ok = false; break; }
         const uint64_t dQ = dQ0 + (uint64_t)(((ut & 1) * L::QB) >> 4);
         const uint32_t tO = tmem + 2 * kTcN;
         for (int c = 0; c < nc; ++c, ++g) {
           const int st = (int)(g % kTcStages), sb = (int)(g & 1);
-          if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort) ||
-              !tc_wait(&bar[kSFree + sb], (uint32_t)(((g >> 1) & 1) ^ 1), p.status, abort)) {
+          if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl) ||
+              !tc_wait(&bar[kSFree + sb], (uint32_t)(((g >> 1) & 1) ^ 1), p.status, abort, wl)) {
             ok = false;
             break;
           }
@@ -450,10 +453,10 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     auto gsync = [&]() -> bool {
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[kGroup]);
-      return tc_wait_warp(&bar[kGroup], (gn++) & 1u, p.status, abort);
+      return tc_wait_warp(&bar[kGroup], (gn++) & 1u, p.status, abort, wl);
     };
     auto next_desc = [&](Unit& dd) -> bool {
-      if (!tc_wait_warp(&bar[kUFull + us], uph, p.status, abort)) return false;
+      if (!tc_wait_warp(&bar[kUFull + us], uph, p.status, abort, wl)) return false;
       dd = umeta[us];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar[kUEmpty + us]);
@@ -510,8 +513,8 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         // ---- the chunk's K, V and scales have landed. f16 V^T: widened first (it frees the ring
         //      stage early; the previous chunk's P V must have read the f16 buffers). Q8: V stays
         //      in the stage as the E4M3 operand and the MMA warp frees the stage after P V.
-        if (!tc_wait_warp(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort) ||
-            (!Q8 && c > 0 && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort))) {
+        if (!tc_wait_warp(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl) ||
+            (!Q8 && c > 0 && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort, wl))) {
           ok = false;
           break;
         }
@@ -555,7 +558,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           __syncwarp();
           if (lane == 0) mbar_arrive(&bar[kKvEmpty + st]);  // the V half of the stage has been read
         }
-        if (!tc_wait_warp(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort)) { ok = false; break; }
+        if (!tc_wait_warp(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort, wl)) { ok = false; break; }
         tc_fence_after();
         float s[kTcN];
         tmem_ld16(tmem + lane_off + kTcN * sb, s);
@@ -644,7 +647,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           if (c > 0 && resc) {
             // O^T holds chunks 0 .. c-1 of this tile (their P V is done; Q8 waits for it here):
             // rescale it in place
-            if (Q8 && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
+            if (Q8 && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort, wl)) { ok = false; break; }
             pv_waited = true;
             tc_fence_after();
             float o[kTcN];
@@ -663,7 +666,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         }
         // ---- P^T row of this key, 16 query rows: f16 P * (V page scale) * kTcPScale, or Q8:
         //      E4M3 P * (V page scale) * C once the previous chunk's P V has read the buffer
-        if (Q8 && c > 0 && !pv_waited && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) {
+        if (Q8 && c > 0 && !pv_waited && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort, wl)) {
           ok = false;
           break;
         }
@@ -702,7 +705,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       if (dnext.b >= 0 && !publish_q(qx, qp ^ 1)) { ok = false; break; }
 
       // ---- epilogue: row sums over the tile, O^T / l, out or partial
-      if (!tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort)) { ok = false; break; }
+      if (!tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort, wl)) { ok = false; break; }
       tc_fence_after();
       // row sums over the warp's 32 keys by a butterfly reduce-scatter: after the five levels,
       // lanes 2c and 2c + 1 hold column c's sum (Q8: the exact sums, then the rounded ones)

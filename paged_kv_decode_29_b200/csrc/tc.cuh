@@ -147,7 +147,8 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // A bounded wait that also gives up at once when another role has aborted the CTA.
-__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort) {
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort,
+                                        uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -155,7 +156,7 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int32_t*
     for (int i = 0; i < 64; ++i)
       if (mbar_test(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_status(status, DECATTN_ETIMEOUT);
       *abort = 1;
       return false;
@@ -165,21 +166,23 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, int32_t*
 
 // The same wait for a whole warp: every lane gets the same answer, so a warp never splits in
 // front of its warp-wide tensor-memory loads and stores (all lanes must execute those).
-__device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort) {
-  return __all_sync(0xffffffffu, tc_wait(bar, parity, status, abort));
+__device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort,
+                                             uint64_t limit_ns = kWaitLimitNs) {
+  return __all_sync(0xffffffffu, tc_wait(bar, parity, status, abort, limit_ns));
 }
 
 // A bounded wait that lets the hardware suspend the thread between checks
 // (mbarrier.try_wait: the thread resumes when the phase completes), for long waits in kernels
 // where a polling warp would take issue slots from the warps doing the work on its
 // sub-partition. Gives up like tc_wait.
-__device__ __forceinline__ bool tc_wait_suspend(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort) {
+__device__ __forceinline__ bool tc_wait_suspend(uint64_t* bar, uint32_t parity, int32_t* status, volatile int* abort,
+                                                uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_status(status, DECATTN_ETIMEOUT);
       *abort = 1;
       return false;
@@ -188,8 +191,8 @@ __device__ __forceinline__ bool tc_wait_suspend(uint64_t* bar, uint32_t parity, 
 }
 
 __device__ __forceinline__ bool tc_wait_suspend_warp(uint64_t* bar, uint32_t parity, int32_t* status,
-                                                     volatile int* abort) {
-  return __all_sync(0xffffffffu, tc_wait_suspend(bar, parity, status, abort));
+                                                     volatile int* abort, uint64_t limit_ns = kWaitLimitNs) {
+  return __all_sync(0xffffffffu, tc_wait_suspend(bar, parity, status, abort, limit_ns));
 }
 
 // Float -> integer with the same order (for warp max reductions with redux.sync).

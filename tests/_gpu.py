@@ -25,16 +25,43 @@ def to_device(pr, device="cuda"):
     return dict(q=q, k=k, v=v, tab=tab, lens=lens, sc=sc)
 
 
+GUARD = 256          # canary bytes after the plan buffer, the workspace, out and lse
+CANARY = 0xA5
+
+
+def _guarded(nbytes, device):
+    """A device byte buffer of nbytes followed by GUARD canary bytes; returns (whole, head view)."""
+    whole = torch.full((nbytes + GUARD,), CANARY, dtype=torch.uint8, device=device)
+    return whole, whole[:nbytes]
+
+
+def check_canaries(*wholes):
+    for w in wholes:
+        tail = w[-GUARD:]
+        assert bool(torch.all(tail == CANARY)), "a kernel wrote past the end of its buffer"
+
+
 def run_problem(pr, dev=None, tile_len=None, n_bins=0, sync=True):
+    """Plan + split + combine through the C ABI. The plan buffer, the workspace, out and lse each
+    end in GUARD canary bytes, checked unchanged after the run."""
     dev = dev or to_device(pr)
     tl = tile_len or pr.tile_len
     total = int(pr.seq_lens.astype(np.int64).sum())
-    pl = da.plan(dev["lens"], pr.n_kv_heads, tl, max_total_kv_tokens=total, n_bins=n_bins)
+    d = dev["q"].device
+    pb_whole, pbuf = _guarded(da.plan_bytes(pr.batch, pr.n_kv_heads, tl, total, n_bins), d)
+    pl = da.plan(dev["lens"], pr.n_kv_heads, tl, max_total_kv_tokens=total, n_bins=n_bins, buf=pbuf)
     shape = da.make_shape(dev["q"], dev["k"], dev["tab"], da.kv_dtype_of(dev["k"]), pr.sm_scale)
-    ws = torch.empty(da.workspace_bytes(shape, pl), dtype=torch.uint8, device=dev["q"].device)
+    ws_whole, ws = _guarded(da.workspace_bytes(shape, pl), d)
+    B, T, Hq, D = dev["q"].shape
+    o_whole, o_bytes = _guarded(B * T * Hq * D * 4, d)
+    l_whole, l_bytes = _guarded(B * T * Hq * 4, d)
+    out = o_bytes.view(torch.float32).view(B, T, Hq, D)
+    lse = l_bytes.view(torch.float32).view(B, T, Hq)
     out, lse = da.run(dev["q"], dev["k"], dev["v"], dev["tab"], dev["lens"], pl, kv_scales=dev["sc"],
-                      sm_scale=pr.sm_scale, workspace=ws)
+                      sm_scale=pr.sm_scale, workspace=ws, out=out, lse=lse)
     status = da.read_status(pl, ws) if sync else None
+    if sync:
+        check_canaries(pb_whole, ws_whole, o_whole, l_whole)
     return out, lse, pl, status
 
 

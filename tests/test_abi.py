@@ -222,3 +222,11 @@ def test_last_error_names_the_failing_step(lib):
     t.start()
     t.join()
     assert seen == [""]
+
+
+def test_test_set_waits_checks_its_range(lib):
+    assert lib.dec_attn_test_set_waits(10, -1) == da.EINVAL             # below 0.1 ms
+    assert lib.dec_attn_test_set_waits(3_000_000_000, -1) == da.EINVAL  # above the default 2 s
+    assert lib.dec_attn_test_set_waits(1_000_000, -2) == da.EINVAL
+    assert lib.dec_attn_test_set_waits(1_000_000, 3) == da.OK
+    assert lib.dec_attn_test_set_waits(0, -1) == da.OK                  # back to the defaults
