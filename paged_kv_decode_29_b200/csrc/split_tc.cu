@@ -54,12 +54,13 @@ struct TcSmem {
   static constexpr int STAGES = Q8 ? 3 : 2;                  // chunk stages of the K/V ring
   static constexpr int KCH = kTcChunk * kTcD;                // bytes of one K (or V) chunk: 16 KB
   static constexpr int QB = 2 * kTcN * kTcD;                 // q hi [16][128] then lo, E4M3
-  static constexpr int PB = kTcChunk * kTcN * (Q8 ? 1 : 2);  // P^T: E4M3 or f16
+  static constexpr int PB = kTcChunk * kTcN * (Q8 ? 1 : 2);  // P^T of one chunk: E4M3 or f16
   static constexpr int OFF_K = 0;                            // [stage][128 keys][128 B], 128-B swizzle
   static constexpr int OFF_V = OFF_K + STAGES * KCH;
   static constexpr int OFF_V16 = OFF_V + STAGES * KCH;       // f16 V^T, MN-major interleaved core matrices
-  static constexpr int OFF_P = OFF_V16 + (Q8 ? 0 : 2 * KCH); // P^T, MN-major interleaved
-  static constexpr int OFF_QB = OFF_P + PB;                  // [tile parity] q hi / lo, 128-B swizzle
+  static constexpr int NPB = Q8 ? 2 : 1;                     // P^T buffers (Q8: one per chunk parity)
+  static constexpr int OFF_P = OFF_V16 + (Q8 ? 0 : 2 * KCH); // [NPB] P^T, MN-major interleaved
+  static constexpr int OFF_QB = OFF_P + NPB * PB;            // [tile parity] q hi / lo, 128-B swizzle
   static constexpr int OFF_SC = OFF_QB + 2 * QB;             // per stage: 8 K scales, 8 V scales
   static constexpr int OFF_QCS = OFF_SC + STAGES * 2 * kTcBlk * 4;  // [tile parity][16]: 2^-E of q rows
   static constexpr int OFF_FLG = OFF_QCS + 2 * kTcN * 4;     // [2][4] per-warp "passes the reference" flags
@@ -67,29 +68,33 @@ struct TcSmem {
   static constexpr int OFF_ERED = OFF_RED + 2 * 4 * kTcN * 4;  // [2][4][16] row-sum partials (Q8: exact, rounded)
   static constexpr int OFF_UNIT = OFF_ERED + 2 * 4 * kTcN * 4;  // Unit x 2
   static constexpr int OFF_BAR = OFF_UNIT + 2 * (int)sizeof(Unit);
-  static constexpr int NBAR = 19;
+  static constexpr int NBAR = 21;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;        // tensor-memory base, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;                 // slack to align the base to 1024
   static_assert(OFF_QB % 1024 == 0 && QB % 1024 == 0, "swizzled q operands need 1024-byte bases");
   static_assert(OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
+  static_assert(OFF_QB % 1024 == 0, "swizzled q operands need 1024-byte bases");
   static_assert(2 * (ALLOC + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
-// Barrier slots.
+// Barrier slots. The P / P V hand-off has one barrier per chunk parity: chunk g (counted over all
+// tiles of the CTA) signals kPReady + (g & 1) and its P V completes kPvDone + (g & 1), phase
+// (g >> 1) & 1, so that the softmax group can compute chunk g + 1's P while chunk g's P V runs
+// (Q8: and write it, into the other P^T buffer) without ever running two phases ahead of a waiter.
 enum TcBar {
   kKvFull = 0,   // [stages] producer -> MMA, softmax: K, V and scales of a chunk landed
   kKvEmpty = 3,  // [stages] the stage may be refilled: MMA commit (K read) + 4 softmax warps (V
                  //          widened); Q8: the MMA commit after the chunk's P V (V read in place)
   kSFull = 6,    // [2] MMA commit -> softmax: S^T of a chunk is in tensor memory
   kSFree = 8,    // [2] 4 softmax warps -> MMA: that S^T buffer has been read
-  kPReady = 10,  // 4 softmax warps -> MMA: P^T (and the f16 V^T) written, O^T rescaled if needed
-  kPvDone = 11,  // MMA commit -> softmax: O^T += V^T P^T of a chunk complete
-  kUFull = 12,   // [2] producer -> MMA, softmax: tile descriptor written
-  kUEmpty = 14,  // [2] MMA + 4 softmax warps -> producer: tile descriptor read
-  kQReady = 16,  // 4 softmax warps -> MMA: q hi / lo of the next tile written
-  kGroup = 17,   // 4 softmax warps: the group's own barrier (bounded, unlike bar.sync)
-  kFin = 18,     // MMA commit -> MMA: every tensor-core operation of the CTA complete
+  kPReady = 10,  // [chunk parity] 4 softmax warps -> MMA: P^T (and the f16 V^T) written, O^T rescaled
+  kPvDone = 12,  // [chunk parity] MMA commit -> softmax: O^T += V^T P^T of a chunk complete
+  kUFull = 14,   // [2] producer -> MMA, softmax: tile descriptor written
+  kUEmpty = 16,  // [2] MMA + 4 softmax warps -> producer: tile descriptor read
+  kQReady = 18,  // 4 softmax warps -> MMA: q hi / lo of the next tile written
+  kGroup = 19,   // 4 softmax warps: the group's own barrier (bounded, unlike bar.sync)
+  kFin = 20,     // MMA commit -> MMA: every tensor-core operation of the CTA complete
 };
 
 }  // namespace decattn
@@ -191,8 +196,10 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       mbar_init(&bar[kUFull + s], 1);
       mbar_init(&bar[kUEmpty + s], 1 + 4);
     }
-    mbar_init(&bar[kPReady], 4);
-    mbar_init(&bar[kPvDone], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[kPReady + s], 4);
+      mbar_init(&bar[kPvDone + s], 1);
+    }
     mbar_init(&bar[kQReady], 4);
     mbar_init(&bar[kGroup], 4);
     mbar_init(&bar[kFin], 1);
@@ -376,21 +383,24 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       // O^T (+)= V^T P^T over chunk gg's 128 keys. A tile's first chunk overwrites O^T: the
       // softmax group signals that chunk's P only after it has read the previous tile's O^T.
       auto pv = [&](int64_t gg, bool first_of_tile, uint32_t tO) -> bool {
-        if (!tc_wait(&bar[kPReady], (uint32_t)(gg & 1), p.status, abort, wl)) return false;
+        if (!tc_wait(&bar[kPReady + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl)) return false;
         tc_fence_after();
+        const uint64_t pofs = (uint64_t)(((gg & (L::NPB - 1)) * L::PB) >> 4);  // this chunk's P^T buffer
         if constexpr (Q8) {
           const int sg = (int)(gg % kTcStages);
           const uint64_t a0 = dV8 + (uint64_t)((sg * L::KCH) >> 4);
           #pragma unroll
           for (int k = 0; k < kTcChunk / 32; ++k)  // 32 keys per instruction: 4 KB of V, 512 B of P
-            umma_f8(tO, a0 + (uint64_t)(256 * k), dP8 + (uint64_t)(32 * k), idO8, (first_of_tile && k == 0) ? 0u : 1u);
-          umma_commit(&bar[kPvDone]);
+            umma_f8(tO, a0 + (uint64_t)(256 * k), dP8 + pofs + (uint64_t)(32 * k), idO8,
+                    (first_of_tile && k == 0) ? 0u : 1u);
+          umma_commit(&bar[kPvDone + (gg & 1)]);
           umma_commit(&bar[kKvEmpty + sg]);  // K and V of the stage have both been read
         } else {
           #pragma unroll
           for (int k = 0; k < kTcChunk / 16; ++k)
-            umma_f16(tO, dV + (uint64_t)(16 * k), dP + (uint64_t)(16 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
-          umma_commit(&bar[kPvDone]);
+            umma_f16(tO, dV + (uint64_t)(16 * k), dP + pofs + (uint64_t)(16 * k), idO,
+                     (first_of_tile && k == 0) ? 0u : 1u);
+          umma_commit(&bar[kPvDone + (gg & 1)]);
         }
         return true;
       };
@@ -510,33 +520,21 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           if (!next_desc(dnext)) { ok = false; break; }
           if (dnext.b >= 0) tc_load_q(p, dnext, qx);
         }
-        // ---- the chunk's K, V and scales have landed. f16 V^T: widened first (it frees the ring
-        //      stage early; the previous chunk's P V must have read the f16 buffers). Q8: V stays
-        //      in the stage as the E4M3 operand and the MMA warp frees the stage after P V.
-        if (!tc_wait_warp(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl) ||
-            (!Q8 && c > 0 && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort, wl))) {
+        // ---- the chunk's K, V and scales have landed. Order within the chunk: scores -> P first
+        //      (while the previous chunk's P V runs), then, once that P V has released the single
+        //      f16 V^T buffer, this chunk's V widened into it; the P V of the chunk follows.
+        //      Q8: V stays in the stage as the E4M3 operand and the MMA warp frees the stage after P V.
+        // waits on the previous chunks' P V: chunk gg's completes kPvDone + (gg & 1), phase (gg >> 1) & 1
+        auto wait_pv = [&](int64_t gg) -> bool {
+          return tc_wait_warp(&bar[kPvDone + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl);
+        };
+        if (!tc_wait_warp(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl)) {
           ok = false;
           break;
         }
         const int j = d.tok_begin + c * kTcChunk + key;
         const bool valid = j < d.tok_end;
-        if constexpr (!Q8) {
-          // V row of this key widened to f16 (exact), 8 head dims per 16-byte core-matrix row
-          const uint8_t* vr = sm + L::OFF_V + st * L::KCH + key * kTcD;
-          uint8_t* vd = sm + L::OFF_V16 + (key >> 3) * 128 + (key & 7) * 16;
-          #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (valid) w = *reinterpret_cast<const uint4*>(vr + ((cc ^ (key & 7)) << 4));  // codes d = 16cc ..
-            const uint4 lo = make_uint4(e4m3x2_to_f16x2(w.x & 0xffffu), e4m3x2_to_f16x2(w.x >> 16),
-                                        e4m3x2_to_f16x2(w.y & 0xffffu), e4m3x2_to_f16x2(w.y >> 16));
-            const uint4 hi = make_uint4(e4m3x2_to_f16x2(w.z & 0xffffu), e4m3x2_to_f16x2(w.z >> 16),
-                                        e4m3x2_to_f16x2(w.w & 0xffffu), e4m3x2_to_f16x2(w.w >> 16));
-            *reinterpret_cast<uint4*>(vd + (2 * cc) * 2048) = lo;
-            *reinterpret_cast<uint4*>(vd + (2 * cc + 1) * 2048) = hi;
-          }
-        }
-        // this key's page scales, read before the stage (scales included) goes back to the producer
+        // this key's page scales
         const int blk = key >> 4;
         const float f = p.qk_scale_log2 * sc[st * 16 + blk];
         const float vsc = sc[st * 16 + 8 + blk] * (Q8 ? 1.f : kTcPScale);
@@ -553,10 +551,6 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           const float r = 448.f / ((float)(1 << kTcTau) * svmax);
           // the largest power of two <= r (exponent field only); 1 when no scale is usable
           c_chunk = (svmax > 0.f && r < 1e30f) ? __int_as_float(__float_as_int(r) & 0x7f800000) : 1.f;
-        }
-        if constexpr (!Q8) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar[kKvEmpty + st]);  // the V half of the stage has been read
         }
         if (!tc_wait_warp(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort, wl)) { ok = false; break; }
         tc_fence_after();
@@ -627,7 +621,6 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
             c_ref = c_chunk;
           }
         }
-        bool pv_waited = false;
         if (upd || c_factor != 1.f) {
           float alpha[kTcN];
           bool resc = c_factor != 1.f;
@@ -645,10 +638,9 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
             resc |= alpha[n] != 1.f;
           }
           if (c > 0 && resc) {
-            // O^T holds chunks 0 .. c-1 of this tile (their P V is done; Q8 waits for it here):
-            // rescale it in place
-            if (Q8 && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort, wl)) { ok = false; break; }
-            pv_waited = true;
+            // O^T holds chunks 0 .. c-1 of this tile once the previous chunk's P V is done: rescale
+            // it in place
+            if (!wait_pv(g - 1)) { ok = false; break; }
             tc_fence_after();
             float o[kTcN];
             tmem_ld16(tO, o);
@@ -664,12 +656,12 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           pr[n] = fast_exp2(s[n] - (mref[n] == -INFINITY ? 0.f : mref[n]));
           lacc[n] += pr[n];
         }
-        // ---- P^T row of this key, 16 query rows: f16 P * (V page scale) * kTcPScale, or Q8:
-        //      E4M3 P * (V page scale) * C once the previous chunk's P V has read the buffer
-        if (Q8 && c > 0 && !pv_waited && !tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort, wl)) {
-          ok = false;
-          break;
-        }
+        // ---- P^T row of this key, 16 query rows: Q8: E4M3 P * (V page scale) * C into buffer g & 1,
+        //      which chunk g - 2's P V read; f16 P * (V page scale) * kTcPScale into the single P^T
+        //      buffer once the previous chunk's P V has read it and the f16 V^T buffer (a tile's first
+        //      chunk: the previous tile's epilogue waited for its last P V)
+        if (Q8 ? (g >= 2 && !wait_pv(g - 2)) : (c > 0 && !wait_pv(g - 1))) { ok = false; break; }
+        uint8_t* pbuf = sm + L::OFF_P + (int)(g & (L::NPB - 1)) * L::PB;
         if constexpr (Q8) {
           // the output is normalised by the weights as rounded, so it stays a convex combination of
           // V rows (a single visible key reproduces its V row); lse keeps the exact sums
@@ -686,26 +678,45 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
               lrnd[4 * i + 2] += b.x * rxs; lrnd[4 * i + 3] += b.y * rxs;
             }
           }
-          *reinterpret_cast<uint4*>(sm + L::OFF_P + key * kTcN) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+          *reinterpret_cast<uint4*>(pbuf + key * kTcN) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
         } else {
           uint32_t h[8];
           #pragma unroll
           for (int i = 0; i < 8; ++i) h[i] = valid ? pack_f16(pr[2 * i] * vsc, pr[2 * i + 1] * vsc) : 0u;
-          uint8_t* pp = sm + L::OFF_P + (key >> 3) * 128 + (key & 7) * 16;
+          uint8_t* pp = pbuf + (key >> 3) * 128 + (key & 7) * 16;
           *reinterpret_cast<uint4*>(pp) = make_uint4(h[0], h[1], h[2], h[3]);
           *reinterpret_cast<uint4*>(pp + 2048) = make_uint4(h[4], h[5], h[6], h[7]);
+          // ---- V row of this key widened to f16 (exact), 8 head dims per 16-byte core-matrix row
+          const uint8_t* vr = sm + L::OFF_V + st * L::KCH + key * kTcD;
+          uint8_t* vd = sm + L::OFF_V16 + (key >> 3) * 128 + (key & 7) * 16;
+          #pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (valid) w = *reinterpret_cast<const uint4*>(vr + ((cc ^ (key & 7)) << 4));  // codes d = 16cc ..
+            const uint4 lo = make_uint4(e4m3x2_to_f16x2(w.x & 0xffffu), e4m3x2_to_f16x2(w.x >> 16),
+                                        e4m3x2_to_f16x2(w.y & 0xffffu), e4m3x2_to_f16x2(w.y >> 16));
+            const uint4 hi = make_uint4(e4m3x2_to_f16x2(w.z & 0xffffu), e4m3x2_to_f16x2(w.z >> 16),
+                                        e4m3x2_to_f16x2(w.w & 0xffffu), e4m3x2_to_f16x2(w.w >> 16));
+            *reinterpret_cast<uint4*>(vd + (2 * cc) * 2048) = lo;
+            *reinterpret_cast<uint4*>(vd + (2 * cc + 1) * 2048) = hi;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[kKvEmpty + st]);  // the V half of the stage has been read
         }
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[kPReady]);
+        if (lane == 0) mbar_arrive(&bar[kPReady + (g & 1)]);
       }
       if (!ok) break;
       // ---- the next tile's q: the MMA warp starts that tile while this one's epilogue runs
       if (dnext.b >= 0 && !publish_q(qx, qp ^ 1)) { ok = false; break; }
 
-      // ---- epilogue: row sums over the tile, O^T / l, out or partial
-      if (!tc_wait_warp(&bar[kPvDone], (uint32_t)((g - 1) & 1), p.status, abort, wl)) { ok = false; break; }
+      // ---- epilogue: row sums over the tile, O^T / l, out or partial (after the tile's last P V)
+      if (!tc_wait_warp(&bar[kPvDone + ((g - 1) & 1)], (uint32_t)(((g - 1) >> 1) & 1), p.status, abort, wl)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       // row sums over the warp's 32 keys by a butterfly reduce-scatter: after the five levels,
       // lanes 2c and 2c + 1 hold column c's sum (Q8: the exact sums, then the rounded ones)
