@@ -117,6 +117,22 @@ typedef struct {
  * made with n_bins = 0: SM count x CTAs resident per SM. Returns < 0 on error. */
 DECATTN_API int dec_attn_default_bins(int device);
 
+/* A tile length for dec_attn_plan, from sizes the host knows. The pages fix uniform KV tiles
+ * ("HPC-Ops ...", "How the kernels are organized around specific workload shapes") but give no
+ * rule for their length; this one weighs the two costs the length trades: long tiles leave the
+ * busiest CTA more tokens than the average (the greedy bins differ by up to one tile), short
+ * tiles write and re-read more partial results and pay a fixed cost per tile more often.
+ * Candidates are page_size * 2^k up to 8192; with U = n_kv_heads * total_kv_tokens / tl tiles
+ * over n_bins bins, the estimate is
+ *   ceil(U / n_bins) * (tl * 2 * head_dim * elem + 8192) + U * rows * (head_dim + 1) * 8 / n_bins
+ * (elem = 2 for bf16, 1 for E4M3; rows = G * T query rows per KV head; 8192 = the fixed cost of a
+ * tile in KV bytes). A candidate with U >= n_bins is preferred, then the smallest estimate, then
+ * the shorter tile. Host only (no CUDA call): n_bins > 0 must be given, e.g.
+ * dec_attn_default_bins(device). Returns the tile length (a multiple of page_size and of 16), or
+ * DECATTN_EINVAL for invalid arguments. */
+DECATTN_API int dec_attn_default_tile_len(int batch, int n_kv_heads, int64_t total_kv_tokens, int page_size,
+                                          int head_dim, int rows_per_kv_head, int kv_dtype, int n_bins);
+
 /* Bytes of the device plan buffer for a plan of `batch` requests whose KV lengths
  * sum to at most max_total_kv_tokens. n_bins = 0 selects dec_attn_default_bins of
  * the current device. Returns 0 for invalid arguments. */

@@ -26,7 +26,7 @@ LIB_PATH = os.path.join(_HERE, "libdecattn.so")
 
 OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1, -2, -3, -4, -5, -6, -7, -8
 KV_BF16, KV_FP8E4M3, KV_FP8E4M3_MMA8 = 0, 1, 2
-API = ("dec_attn_default_bins", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
+API = ("dec_attn_default_bins", "dec_attn_default_tile_len", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
        "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_prefill",
        "dec_attn_prefill_varlen", "dec_attn_plan_sparse_bytes",
@@ -74,6 +74,8 @@ def load_library(path: str = LIB_PATH):
         vp, i32, i64, sz = C.c_void_p, C.c_int, C.c_int64, C.c_size_t
         lib.dec_attn_default_bins.argtypes = [i32]
         lib.dec_attn_default_bins.restype = i32
+        lib.dec_attn_default_tile_len.argtypes = [i32, i32, i64, i32, i32, i32, i32, i32]
+        lib.dec_attn_default_tile_len.restype = i32
         lib.dec_attn_plan_bytes.argtypes = [i32, i32, i32, i64, i32]
         lib.dec_attn_plan_bytes.restype = sz
         lib.dec_attn_plan.argtypes = [vp, i32, i32, i32, i64, i32, vp, sz, C.POINTER(PlanT), vp]
@@ -157,6 +159,18 @@ def default_bins(device: int | None = None) -> int:
     if n <= 0:
         raise DecAttnError(ECUDA, "dec_attn_default_bins")
     return n
+
+
+def default_tile_len(batch: int, n_kv_heads: int, total_kv_tokens: int, page_size: int, head_dim: int,
+                     rows_per_kv_head: int, kv_dtype: int = KV_BF16, n_bins: int | None = None) -> int:
+    """dec_attn_default_tile_len: the tile length that minimises the library's estimate of the
+    busiest CTA's bytes (host only when ``n_bins`` is given; else the current device's bins)."""
+    nb = default_bins() if n_bins is None else int(n_bins)
+    tl = load_library().dec_attn_default_tile_len(batch, n_kv_heads, int(total_kv_tokens), page_size, head_dim,
+                                                  rows_per_kv_head, kv_dtype, nb)
+    if tl <= 0:
+        raise DecAttnError(tl, "dec_attn_default_tile_len")
+    return int(tl)
 
 
 def plan_bytes(batch: int, n_kv_heads: int, tile_len: int, max_total_kv_tokens: int, n_bins: int = 0) -> int:

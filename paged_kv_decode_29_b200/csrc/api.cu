@@ -330,6 +330,37 @@ extern "C" int dec_attn_prefill_varlen(const dec_attn_shape* shape, const void* 
 
 extern "C" int dec_attn_default_bins(int device) { return default_bins(device); }
 
+extern "C" int dec_attn_default_tile_len(int batch, int n_kv_heads, int64_t total_kv_tokens, int page_size,
+                                         int head_dim, int rows_per_kv_head, int kv_dtype, int n_bins) {
+  if (batch <= 0 || n_kv_heads <= 0 || total_kv_tokens < 0 || page_size <= 0 || page_size % 16 != 0 ||
+      head_dim <= 0 || rows_per_kv_head <= 0 || n_bins <= 0)
+    return DECATTN_EINVAL;
+  const double elem = kv_dtype == DECATTN_KV_BF16 ? 2.0 : 1.0;
+  const double N = (double)n_bins;
+  const double W = (double)n_kv_heads * (double)total_kv_tokens;  // token-heads of the step
+  const double tile_cost = 8192.0;  // fixed cost of a tile (q, epilogue, pipeline start) in KV-byte terms
+  int best = 0;
+  double best_est = 0.0;
+  bool best_fills = false;  // the candidate gives every bin a tile
+  for (int tl = page_size; tl <= 8192; tl *= 2) {
+    const double U = W / tl;  // tiles, as if every tile were full
+    const bool fills = U >= N;
+    const double per_bin = U > 0 ? ceil(U / N) : 0.0;
+    // the busiest bin's KV bytes and tile overheads, plus the partials every tile writes and the
+    // combine reads back (fp32 o and lse per query row), spread over the bins
+    const double est = per_bin * (tl * 2.0 * head_dim * elem + tile_cost) +
+                       U * rows_per_kv_head * (head_dim + 1.0) * 8.0 / N;
+    // a candidate that fills every bin beats one that does not; then the smaller estimate, then
+    // the shorter tile
+    if (best == 0 || (fills && !best_fills) || (fills == best_fills && est < best_est)) {
+      best = tl;
+      best_est = est;
+      best_fills = fills;
+    }
+  }
+  return best;
+}
+
 extern "C" size_t dec_attn_workspace_bytes(const dec_attn_shape* shape, const dec_attn_plan_t* plan) {
   if (check_shape(shape, plan) != DECATTN_OK) return 0;
   return (size_t)ws_layout(plan->max_units, *shape).total;

@@ -230,3 +230,23 @@ def test_test_set_waits_checks_its_range(lib):
     assert lib.dec_attn_test_set_waits(1_000_000, -2) == da.EINVAL
     assert lib.dec_attn_test_set_waits(1_000_000, 3) == da.OK
     assert lib.dec_attn_test_set_waits(0, -1) == da.OK                  # back to the defaults
+
+
+def test_default_tile_len_rule(lib):
+    # host only; the rule's estimate (include/decattn.h) reproduces the hand-made choices where the
+    # trade-off is clear, and never returns a length that is not a multiple of the page
+    f = lib.dec_attn_default_tile_len
+    assert f(32, 8, 32 * 4096, 16, 128, 4, da.KV_BF16, 592) == 256         # uniform
+    assert f(1, 8, 131072, 64, 128, 8, da.KV_BF16, 592) == 256             # long context, one request
+    assert f(4, 8, 4 * 131072, 64, 128, 8, da.KV_BF16, 592) == 1024        # long context, four requests
+    assert f(2, 1, 317, 16, 64, 4, da.KV_BF16, 592) == 16                  # too small to fill the bins
+    for P in (16, 32, 48, 64, 256):
+        tl = f(8, 8, 100000, P, 128, 8, da.KV_BF16, 592)
+        assert tl > 0 and tl % P == 0 and tl % 16 == 0
+    # more query rows per KV head -> more partial bytes per tile -> tiles no shorter
+    a = f(16, 8, 270000, 16, 128, 4, da.KV_FP8E4M3, 592)
+    b = f(16, 8, 270000, 16, 128, 64, da.KV_FP8E4M3, 592)
+    assert b >= a
+    assert f(0, 8, 100, 16, 128, 4, da.KV_BF16, 592) == da.EINVAL
+    assert f(4, 8, 100, 24, 128, 4, da.KV_BF16, 592) == da.EINVAL           # page not a multiple of 16
+    assert f(4, 8, 100, 16, 128, 4, da.KV_BF16, 0) == da.EINVAL
