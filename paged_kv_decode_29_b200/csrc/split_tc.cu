@@ -5,30 +5,36 @@
 // Hot Paths", "How the kernels are organized around specific workload shapes": uniform tiles,
 // greedy bins, a combine), for head_dim 128 and G*T <= 16.
 //
-// The legacy warp-level MMA path spends most of its instructions moving fragments: with G*T = 16
-// and FP8 K/V it is bound by instruction issue, not by memory. Here a tile is processed in
-// chunks of 128 keys and each product is one tensor-core instruction stream:
-//  * S^T (128 keys x 16 query rows, fp32 in tensor memory) = K Q^T on kind::f8f6f4, A = the
-//    staged K codes as TMA left them (K-major, 128-byte swizzle), B = q split into two E4M3
-//    parts hi + lo (written K-major by the softmax warps), accumulated into one result;
-//  * O^T (128 head dims x 16 query rows, fp32 in tensor memory) += V^T P^T on kind::f16, A = V
-//    widened to f16 once per element (MN-major), B = P^T in f16 (MN-major).
+// Both products run on E4M3 tensor cores (kind::f8f6f4) straight from the staged pages, so no
+// element of K or V is ever converted. A tile is processed in chunks of 128 keys:
+//  * S^T (128 keys x 16 query rows, fp32 in tensor memory) = K Q^T, A = the staged K codes as TMA
+//    left them (K-major, 128-byte swizzle). B = q scaled by a power of two per row and split into
+//    E4M3 parts written K-major by the softmax warps: hi and lo side by side (N = 32; their two
+//    16-column halves are added when read), which carry a bf16 q exactly; Q8: hi only (N = 16).
+//  * O^T (128 head dims x 16 query rows, fp32 in tensor memory) += V^T P^T, A = the staged V codes
+//    (MN-major: head dims contiguous, 128-byte swizzle). B = P^T with P scaled by (V page scale) *
+//    C (C a power of two per chunk that keeps P within E4M3's range) and split into three E4M3
+//    parts hi, mid, lo side by side (N = 48; the three 16-column groups of O^T are added in the
+//    epilogue): about 12 significant bits, as close to P as an f16 P would be, so the result
+//    meets the same tolerance as the bf16 path. Q8: one part (N = 16) and its own tolerance.
 // Thread j of the 128-thread softmax group owns key j of the chunk (tensor-memory lane j) and
-// reads its 16 scores with one tcgen05.ld, so the per-key work has no fragment shuffles.
+// reads its scores with one tcgen05.ld, so the per-key work has no fragment shuffles.
 //
 // Online softmax with a reference maximum: P = 2^(s - m_ref) for every key of a tile, where
 // m_ref is the exact maximum of the tile's first chunk and moves (to the running maximum) only
 // when a later chunk holds a score above m_ref + kTcTau; then O^T and the running sums are
-// rescaled in place. P is thus at most 2^kTcTau, which keeps P * (V page scale) * kTcPScale
-// inside f16, and most chunks need only a one-flag-per-warp check instead of an exact maximum.
+// rescaled in place. P is thus at most 2^kTcTau, and most chunks need only a one-flag-per-warp
+// check instead of an exact maximum.
 //
 // CTA: 6 warps, 2 CTAs per SM, and one wave of CTAs: CTA i takes bins i, i + grid, ... .
-//  * warps 0-3 (softmax group; warp w reads tensor-memory lanes 32w..32w+31): per chunk, V
-//    widening first (it frees the ring stage early), then scores -> P and the O^T rescale; per
-//    tile, the next tile's q (loaded from global memory during the last chunk and published
-//    before the epilogue, so the MMA warp starts that tile meanwhile) and the epilogue;
+//  * warps 0-3 (softmax group; warp w reads tensor-memory lanes 32w..32w+31): per chunk, scores ->
+//    P and its E4M3 parts (while the previous chunk's P V runs), the O^T rescale when the
+//    reference moves; per tile, the next tile's q (loaded from global memory during the last
+//    chunk and published before the epilogue, so the MMA warp starts that tile meanwhile) and the
+//    epilogue;
 //  * warp 4 (producer): the bins' tiles (walk, then plan) and their K/V pages by TMA, 128-key
-//    chunks in a two-stage ring, FP8 page scales by cp.async;
+//    chunks in a three-stage ring, FP8 page scales by cp.async; the next tile's first page ids are
+//    read while the current tile's first chunk is in flight;
 //  * warp 5 (MMA): allocates tensor memory and issues every tcgen05.mma from one thread.
 // Every wait is bounded; a wait that gives up sets DECATTN_ETIMEOUT and a CTA-wide abort flag,
 // after which every role leaves its loop and the CTA frees its tensor memory and exits.
@@ -39,29 +45,40 @@
 namespace decattn {
 
 constexpr int kTcD = 128;          // head_dim
-constexpr int kTcN = 16;           // MMA N: query rows of the KV group, zero-padded
+constexpr int kTcN = 16;           // query rows of the KV group (zero-padded): one 16-column group
 constexpr int kTcChunk = 128;      // keys per chunk: the M of S^T and the contraction of O^T
 constexpr int kTcBlk = kTcChunk / 16;  // 16-key blocks (one TMA box each) per chunk
 constexpr int kTcThreads = 192;
 constexpr int kTcTau = 6;          // P <= 2^kTcTau
-constexpr float kTcPScale = 64.f;  // f16 P^T: P * (V page scale) * kTcPScale
-constexpr int kTcTmemCols = 64;    // S^T double buffer (2 x 16 columns), O^T (16), spare (power of 2)
+constexpr int kTcStages = 3;       // chunk stages of the K/V ring
 
-// Shared-memory layout (offsets from a 1024-byte aligned base). Q8: both products on E4M3 (no
-// f16 V^T buffer, which pays for a third ring stage; P^T in E4M3).
+// Per mode: Q8 = one E4M3 part for q and for P (its own tolerance); otherwise two parts of q and
+// three of P (the standard tolerance).
+template <bool Q8>
+struct TcMode {
+  static constexpr int QP = Q8 ? 1 : 2;            // E4M3 parts of q
+  static constexpr int PP = Q8 ? 1 : 3;            // E4M3 parts of P
+  static constexpr int NS = QP * kTcN;             // S^T columns (per q part, 16 query rows)
+  static constexpr int NO = PP * kTcN;             // O^T columns (per P part, 16 query rows)
+  static constexpr int NPB = Q8 ? 2 : 1;           // P^T buffers (Q8: one per chunk parity)
+  static constexpr int TMEM = Q8 ? 64 : 128;       // columns: S^T double buffer + O^T, a power of 2
+  static_assert(2 * NS + NO <= TMEM, "tensor-memory columns");
+};
+
+// Shared-memory layout (offsets from a 1024-byte aligned base).
 template <bool Q8>
 struct TcSmem {
-  static constexpr int STAGES = Q8 ? 3 : 2;                  // chunk stages of the K/V ring
+  using M = TcMode<Q8>;
+  static constexpr int STAGES = kTcStages;
   static constexpr int KCH = kTcChunk * kTcD;                // bytes of one K (or V) chunk: 16 KB
-  static constexpr int QB = 2 * kTcN * kTcD;                 // q hi [16][128] then lo, E4M3
-  static constexpr int PB = kTcChunk * kTcN * (Q8 ? 1 : 2);  // P^T of one chunk: E4M3 or f16
+  static constexpr int QB = M::QP * kTcN * kTcD;             // q parts [part][16][128], E4M3
+  static constexpr int PPLANE = kTcChunk * kTcN;             // one E4M3 part of P^T: 2 KB
+  static constexpr int PB = M::PP * PPLANE;                  // P^T of one chunk: [part][128 keys][16]
   static constexpr int OFF_K = 0;                            // [stage][128 keys][128 B], 128-B swizzle
   static constexpr int OFF_V = OFF_K + STAGES * KCH;
-  static constexpr int OFF_V16 = OFF_V + STAGES * KCH;       // f16 V^T, MN-major interleaved core matrices
-  static constexpr int NPB = Q8 ? 2 : 1;                     // P^T buffers (Q8: one per chunk parity)
-  static constexpr int OFF_P = OFF_V16 + (Q8 ? 0 : 2 * KCH); // [NPB] P^T, MN-major interleaved
-  static constexpr int OFF_QB = OFF_P + NPB * PB;            // [tile parity] q hi / lo, 128-B swizzle
-  static constexpr int OFF_SC = OFF_QB + 2 * QB;             // per stage: 8 K scales, 8 V scales
+  static constexpr int OFF_QB = OFF_V + STAGES * KCH;        // [tile parity] q parts, 128-B swizzle
+  static constexpr int OFF_P = OFF_QB + 2 * QB;              // [NPB] P^T, MN-major interleaved
+  static constexpr int OFF_SC = OFF_P + M::NPB * PB;         // per stage: 8 K scales, 8 V scales
   static constexpr int OFF_QCS = OFF_SC + STAGES * 2 * kTcBlk * 4;  // [tile parity][16]: 2^-E of q rows
   static constexpr int OFF_FLG = OFF_QCS + 2 * kTcN * 4;     // [2][4] per-warp "passes the reference" flags
   static constexpr int OFF_RED = OFF_FLG + 2 * 4 * 4;        // [2][4][16] chunk maxima per warp
@@ -74,7 +91,6 @@ struct TcSmem {
   static constexpr int ALLOC = BYTES + 1024;                 // slack to align the base to 1024
   static_assert(OFF_QB % 1024 == 0 && QB % 1024 == 0, "swizzled q operands need 1024-byte bases");
   static_assert(OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
-  static_assert(OFF_QB % 1024 == 0, "swizzled q operands need 1024-byte bases");
   static_assert(2 * (ALLOC + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
@@ -84,11 +100,10 @@ struct TcSmem {
 // (Q8: and write it, into the other P^T buffer) without ever running two phases ahead of a waiter.
 enum TcBar {
   kKvFull = 0,   // [stages] producer -> MMA, softmax: K, V and scales of a chunk landed
-  kKvEmpty = 3,  // [stages] the stage may be refilled: MMA commit (K read) + 4 softmax warps (V
-                 //          widened); Q8: the MMA commit after the chunk's P V (V read in place)
+  kKvEmpty = 3,  // [stages] the stage may be refilled: the MMA commit after the chunk's P V
   kSFull = 6,    // [2] MMA commit -> softmax: S^T of a chunk is in tensor memory
   kSFree = 8,    // [2] 4 softmax warps -> MMA: that S^T buffer has been read
-  kPReady = 10,  // [chunk parity] 4 softmax warps -> MMA: P^T (and the f16 V^T) written, O^T rescaled
+  kPReady = 10,  // [chunk parity] 4 softmax warps -> MMA: P^T written, O^T rescaled
   kPvDone = 12,  // [chunk parity] MMA commit -> softmax: O^T += V^T P^T of a chunk complete
   kUFull = 14,   // [2] producer -> MMA, softmax: tile descriptor written
   kUEmpty = 16,  // [2] MMA + 4 softmax warps -> producer: tile descriptor read
@@ -115,10 +130,11 @@ __device__ __forceinline__ void tc_load_q(const SplitParams& p, const Unit& d, u
   }
 }
 
-// q hi / lo of a tile into its operand buffer (E4M3, K-major, 128-byte swizzle) and the
-// per-row factor 2^-E into qcs. q is scaled by a per-row power of two 2^E (largest |q| lands in
-// [128, 256)) and split into two E4M3 parts, hi = E4M3(q 2^E) and lo = E4M3(q 2^E - hi), which
-// together carry the 8 significant bits of a bf16 q.
+// q parts of a tile into its operand buffer (E4M3, K-major, 128-byte swizzle) and the per-row
+// factor 2^-E into qcs. q is scaled by a per-row power of two 2^E (largest |q| lands in
+// [128, 256)) and rounded to E4M3: hi = E4M3(q 2^E); with two parts also lo = E4M3(q 2^E - hi)
+// in the rows after hi's 16, which together carry the 8 significant bits of a bf16 q.
+template <int QP>
 __device__ __forceinline__ void tc_store_q(const uint4 (&x)[2], uint8_t* qb, float* qcs) {
   const int r = threadIdx.x >> 3, seg = threadIdx.x & 7;
   float v[16];
@@ -146,15 +162,17 @@ __device__ __forceinline__ void tc_store_q(const uint4 (&x)[2], uint8_t* qb, flo
     for (int k = 0; k < 2; ++k) {
       const float a0 = v[4 * i + 2 * k] * up, a1 = v[4 * i + 2 * k + 1] * up;
       hh[k] = f32x2_to_e4m3x2(a0, a1);
-      const float2 b = f16x2_to_float2(e4m3x2_to_f16x2(hh[k]));
-      ll[k] = f32x2_to_e4m3x2(a0 - b.x, a1 - b.y);
+      if (QP == 2) {
+        const float2 b = f16x2_to_float2(e4m3x2_to_f16x2(hh[k]));
+        ll[k] = f32x2_to_e4m3x2(a0 - b.x, a1 - b.y);
+      }
     }
     hw[i] = hh[0] | (hh[1] << 16);
-    lw[i] = ll[0] | (ll[1] << 16);
+    if (QP == 2) lw[i] = ll[0] | (ll[1] << 16);
   }
   const int off = r * kTcD + ((seg ^ (r & 7)) << 4);
   *reinterpret_cast<uint4*>(qb + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-  *reinterpret_cast<uint4*>(qb + kTcN * kTcD + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  if (QP == 2) *reinterpret_cast<uint4*>(qb + kTcN * kTcD + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
   if (seg == 0) qcs[r] = __int_as_float((127 - E) << 23);
 }
 
@@ -162,7 +180,7 @@ template <bool Q8>
 __global__ void __launch_bounds__(kTcThreads, 2)
 split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   using L = TcSmem<Q8>;
-  constexpr int kTcStages = L::STAGES;
+  using M = TcMode<Q8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
@@ -177,26 +195,22 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)p.B * p.T * p.Hq;
        i += (int64_t)gridDim.x * blockDim.x)
     p.row_cnt[i] = 0;
-  if constexpr (Q8) {
-    // V is read in place by the MMA, including the rows of a tile's last chunk that no page
-    // fills: they meet P = 0 and must be finite, so the ring starts zeroed (afterwards it only
-    // ever holds codes from the pool). Ordered before the first TMA write and MMA read.
-    for (int i = threadIdx.x; i < 2 * kTcStages * L::KCH / 16; i += kTcThreads)
-      reinterpret_cast<uint4*>(sm + L::OFF_K)[i] = make_uint4(0, 0, 0, 0);
-    fence_async_smem();
-  }
+  // V is read in place by the MMA, including the rows of a tile's last chunk that no page fills:
+  // they meet P = 0 and must be finite, so the ring starts zeroed (afterwards it only ever holds
+  // codes from the pool). Ordered before the first TMA write and MMA read.
+  for (int i = threadIdx.x; i < 2 * kTcStages * L::KCH / 16; i += kTcThreads)
+    reinterpret_cast<uint4*>(sm + L::OFF_K)[i] = make_uint4(0, 0, 0, 0);
+  fence_async_smem();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
       mbar_init(&bar[kKvFull + s], 1);
-      mbar_init(&bar[kKvEmpty + s], Q8 ? 1 : 1 + 4);
+      mbar_init(&bar[kKvEmpty + s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[kSFull + s], 1);
       mbar_init(&bar[kSFree + s], 4);
       mbar_init(&bar[kUFull + s], 1);
       mbar_init(&bar[kUEmpty + s], 1 + 4);
-    }
-    for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[kPReady + s], 4);
       mbar_init(&bar[kPvDone + s], 1);
     }
@@ -208,7 +222,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
   }
   if (warp == 5) {  // tensor memory: S^T (two buffers), O^T
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_base_sm)),
-                 "n"(kTcTmemCols)
+                 "n"(M::TMEM)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -284,8 +298,14 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       if (lane == 0) r = tc_wait(b, par, p.status, abort, wl) ? 1 : 0;
       return __shfl_sync(0xffffffffu, r, 0) != 0;
     };
+    // lane l: page id of page l of a tile's first window of 32 pages (0 past the tile's pages)
+    auto first_window = [&](const Unit& u) -> int {
+      const int pg0 = u.tok_begin / P, npg = (u.tok_end - u.tok_begin + P - 1) / P;
+      return lane < npg ? p.page_table[(int64_t)u.b * p.mpps + min(pg0 + lane, p.mpps - 1)] : 0;
+    };
     Unit dn;
     bool has_n = next_unit(dn);
+    int pid_next = has_n ? first_window(dn) : 0;
     for (int u = 0; has_n && ok; ++u) {
       const Unit d = dn;
       if (!wait0(&bar[kUEmpty + us], ueph)) { ok = false; break; }
@@ -298,7 +318,8 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       const int npg = (d.tok_end - d.tok_begin + P - 1) / P;
       if (lane == 0 && pg0 + npg > p.mpps) note(DECATTN_EDEVICE);  // row too short
       const int nblk = (d.tok_end - d.tok_begin + 15) / 16;
-      int win = -1, pid_w = 0;  // page ids of pages [32 win, 32 win + 32) of the tile, one per lane
+      int win = 0, pid_w = pid_next;  // page ids of pages [32 win, 32 win + 32) of the tile, one per lane
+      bool checked = false;           // the window's ids have been range-checked
       bool looked = false;
       for (int b0 = 0; b0 < nblk && ok; b0 += kTcBlk) {
         const int nb = min(kTcBlk, nblk - b0);
@@ -311,6 +332,11 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           win = w_need;
           const int pg = win * 32 + lane;
           pid_w = pg < npg ? p.page_table[(int64_t)d.b * p.mpps + min(pg0 + pg, p.mpps - 1)] : 0;
+          checked = false;
+        }
+        if (!checked) {
+          checked = true;
+          const int pg = win * 32 + lane;
           if (pg < npg && (pid_w < 0 || pid_w >= p.num_pages)) {
             note(DECATTN_EDEVICE);
             pid_w = 0;  // keeps the copy inside the pool; the result is flagged invalid
@@ -336,12 +362,16 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         }
         ++n_fill;
         if (++st == kTcStages) { st = 0; eph ^= 1; }
-        if (!looked) {  // the next tile's descriptor, fetched while this tile's first copies fly
+        if (!looked) {  // the next tile's descriptor and first page ids, read while this tile's first copies fly
           looked = true;
           has_n = next_unit(dn);
+          if (has_n) pid_next = first_window(dn);
         }
       }
-      if (!looked && ok) has_n = next_unit(dn);
+      if (!looked && ok) {
+        has_n = next_unit(dn);
+        if (has_n) pid_next = first_window(dn);
+      }
     }
     if (!plan_loaded) load_plan();
     if (ok) {
@@ -365,43 +395,39 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     // ===================================================================== MMA issue
     if (lane == 0) {
       const uint32_t base = smem_u32(sm);
-      constexpr uint32_t idS = umma_idesc(0, 0, 0, 0, kTcChunk, kTcN);  // E4M3 x E4M3, both K-major
-      constexpr uint32_t idO = umma_idesc(0, 0, 1, 1, kTcD, kTcN);      // f16 x f16, both MN-major
+      // S^T: E4M3 x E4M3, both K-major, N = the q parts' columns; O^T: E4M3 x E4M3, both MN-major,
+      // N = the P parts' columns
+      constexpr uint32_t idS = umma_idesc(0, 0, 0, 0, kTcChunk, M::NS);
+      constexpr uint32_t idO = umma_idesc(0, 0, 1, 1, kTcD, M::NO);
       int us = 0; uint32_t uph = 0;
       int64_t g = 0;  // chunks issued so far
       int ut = 0;     // tiles started so far
       bool ok = true;
       // descriptors, built once: the start address is the low 14 bits (16-byte units), so a
-      // stage or a k-step adds to the base descriptor
-      const uint64_t dV = umma_desc(base + L::OFF_V16, 128, 2048, 0), dP = umma_desc(base + L::OFF_P, 128, 2048, 0);
+      // stage or a k-step adds to the base descriptor.
+      //  K and q: K-major, 128-byte swizzle (8-row groups 1024 B apart; a 32-byte k-step); the q
+      //    parts are consecutive 16-row blocks, so N = 32 spans hi then lo.
+      //  V^T: the staged V (E4M3, MN-major: head dims contiguous, 128-byte swizzle; 8-key groups
+      //    1024 B apart, a 32-key k-step is 4 KB).
+      //  P^T: MN-major interleaved, key j of part q at q * 2 KB + 16 j: 8-key groups 128 B apart
+      //    (leading offset), the next 16 columns (the next part) 2 KB on (stride offset).
       const uint64_t dK0 = umma_desc(base + L::OFF_K, 16, 1024, 2), dQ0 = umma_desc(base + L::OFF_QB, 16, 1024, 2);
-      // Q8: A = V^T as staged (E4M3, MN-major: head dims contiguous, 128-byte swizzle; 8-key groups
-      // 1024 B apart), B = P^T (E4M3, MN-major interleaved: key j at 16 j, 8-key groups 128 B
-      // apart). Both leading offsets equal the stride offsets, so either reading stays in bounds.
-      const uint64_t dV8 = umma_desc(base + L::OFF_V, 1024, 1024, 2), dP8 = umma_desc(base + L::OFF_P, 128, 128, 0);
-      constexpr uint32_t idO8 = umma_idesc(0, 0, 1, 1, kTcD, kTcN);     // E4M3 x E4M3, both MN-major
+      const uint64_t dV = umma_desc(base + L::OFF_V, 1024, 1024, 2);
+      const uint64_t dP = umma_desc(base + L::OFF_P, 128, L::PPLANE, 0);
+      const uint32_t tO = tmem + 2 * M::NS;
       // O^T (+)= V^T P^T over chunk gg's 128 keys. A tile's first chunk overwrites O^T: the
       // softmax group signals that chunk's P only after it has read the previous tile's O^T.
-      auto pv = [&](int64_t gg, bool first_of_tile, uint32_t tO) -> bool {
+      auto pv = [&](int64_t gg, bool first_of_tile) -> bool {
         if (!tc_wait(&bar[kPReady + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl)) return false;
         tc_fence_after();
-        const uint64_t pofs = (uint64_t)(((gg & (L::NPB - 1)) * L::PB) >> 4);  // this chunk's P^T buffer
-        if constexpr (Q8) {
-          const int sg = (int)(gg % kTcStages);
-          const uint64_t a0 = dV8 + (uint64_t)((sg * L::KCH) >> 4);
-          #pragma unroll
-          for (int k = 0; k < kTcChunk / 32; ++k)  // 32 keys per instruction: 4 KB of V, 512 B of P
-            umma_f8(tO, a0 + (uint64_t)(256 * k), dP8 + pofs + (uint64_t)(32 * k), idO8,
-                    (first_of_tile && k == 0) ? 0u : 1u);
-          umma_commit(&bar[kPvDone + (gg & 1)]);
-          umma_commit(&bar[kKvEmpty + sg]);  // K and V of the stage have both been read
-        } else {
-          #pragma unroll
-          for (int k = 0; k < kTcChunk / 16; ++k)
-            umma_f16(tO, dV + (uint64_t)(16 * k), dP + pofs + (uint64_t)(16 * k), idO,
-                     (first_of_tile && k == 0) ? 0u : 1u);
-          umma_commit(&bar[kPvDone + (gg & 1)]);
-        }
+        const int sg = (int)(gg % kTcStages);
+        const uint64_t a0 = dV + (uint64_t)((sg * L::KCH) >> 4);
+        const uint64_t b0 = dP + (uint64_t)((((int)(gg & (M::NPB - 1))) * L::PB) >> 4);
+        #pragma unroll
+        for (int k = 0; k < kTcChunk / 32; ++k)  // 32 keys per instruction: 4 KB of V, 512 B per P part
+          umma_f8(tO, a0 + (uint64_t)(256 * k), b0 + (uint64_t)(32 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
+        umma_commit(&bar[kPvDone + (gg & 1)]);
+        umma_commit(&bar[kKvEmpty + sg]);  // K and V of the stage have both been read
         return true;
       };
       for (;;) {
@@ -413,7 +439,6 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         const int nc = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
         if (!tc_wait(&bar[kQReady], (uint32_t)(ut & 1), p.status, abort, wl)) { ok = false; break; }
         const uint64_t dQ = dQ0 + (uint64_t)(((ut & 1) * L::QB) >> 4);
-        const uint32_t tO = tmem + 2 * kTcN;
         for (int c = 0; c < nc; ++c, ++g) {
           const int st = (int)(g % kTcStages), sb = (int)(g & 1);
           if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl) ||
@@ -422,22 +447,16 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
             break;
           }
           tc_fence_after();
-          // S^T = K (q hi)^T + K (q lo)^T (Q8: q hi only): four 32-byte k-steps of the 128-byte
-          // swizzled rows
+          // S^T = K (q parts)^T: four 32-byte k-steps of the 128-byte swizzled rows
           const uint64_t dK = dK0 + (uint64_t)((st * L::KCH) >> 4);
           #pragma unroll
-          for (int kk = 0; kk < kTcD / 32; ++kk) {
-            const uint64_t a = dK + (uint64_t)(2 * kk);
-            umma_f8(tmem + kTcN * sb, a, dQ + (uint64_t)(2 * kk), idS, kk > 0 ? 1u : 0u);
-            if constexpr (!Q8)
-              umma_f8(tmem + kTcN * sb, a, dQ + (uint64_t)((kTcN * kTcD) >> 4) + (uint64_t)(2 * kk), idS, 1u);
-          }
+          for (int kk = 0; kk < kTcD / 32; ++kk)
+            umma_f8(tmem + M::NS * sb, dK + (uint64_t)(2 * kk), dQ + (uint64_t)(2 * kk), idS, kk > 0 ? 1u : 0u);
           umma_commit(&bar[kSFull + sb]);
-          if constexpr (!Q8) umma_commit(&bar[kKvEmpty + st]);  // the K half of the stage has been read
-          if (c > 0 && !pv(g - 1, c == 1, tO)) { ok = false; break; }
+          if (c > 0 && !pv(g - 1, c == 1)) { ok = false; break; }
         }
         if (!ok) break;
-        if (!pv(g - 1, nc == 1, tO)) { ok = false; break; }
+        if (!pv(g - 1, nc == 1)) { ok = false; break; }
         ++ut;
       }
       if (!ok) *abort = 1;
@@ -475,11 +494,26 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     };
     // q of a tile into operand buffer `par`; the MMA warp may start the tile afterwards
     auto publish_q = [&](const uint4 (&x)[2], int par) -> bool {
-      tc_store_q(x, sm + L::OFF_QB + par * L::QB, qcs_sm + kTcN * par);
+      tc_store_q<M::QP>(x, sm + L::OFF_QB + par * L::QB, qcs_sm + kTcN * par);
       fence_async_smem();
       if (!gsync()) return false;
       if (lane == 0) mbar_arrive(&bar[kQReady]);
       return true;
+    };
+    // waits on a chunk's P V: chunk gg's completes kPvDone + (gg & 1), phase (gg >> 1) & 1
+    auto wait_pv = [&](int64_t gg) -> bool {
+      return tc_wait_warp(&bar[kPvDone + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl);
+    };
+    // this thread's row of O^T (its head dim), the P parts' 16-column groups added
+    auto o_sum = [&](uint32_t tO, float (&o)[kTcN]) {
+      tmem_ld16(tO, o);
+      #pragma unroll
+      for (int q = 1; q < M::PP; ++q) {
+        float t[kTcN];
+        tmem_ld16(tO + kTcN * q, t);
+        #pragma unroll
+        for (int n = 0; n < kTcN; ++n) o[n] += t[n];
+      }
     };
     Unit d;
     d.b = -1;
@@ -491,7 +525,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     }
     while (ok && d.b >= 0) {
       const int qp = ut & 1;
-      const uint32_t tO = tmem + lane_off + 2 * kTcN;
+      const uint32_t tO = tmem + lane_off + 2 * M::NS;
       const float4* qcs4 = reinterpret_cast<const float4*>(qcs_sm + kTcN * qp);
       // lane n < G*T: the output row of query row n (final out, or the tile's partial slot)
       int64_t row_n = 0;
@@ -509,7 +543,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         lacc[n] = 0.f;
         if constexpr (Q8) lrnd[n] = 0.f;
       }
-      float c_ref = 1.f;  // Q8: the power of two that O^T carries
+      float c_ref = 1.f;  // the power of two that O^T carries (P scaled by (V page scale) * C)
       Unit dnext;
       dnext.b = -1;
       uint4 qx[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
@@ -520,14 +554,8 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           if (!next_desc(dnext)) { ok = false; break; }
           if (dnext.b >= 0) tc_load_q(p, dnext, qx);
         }
-        // ---- the chunk's K, V and scales have landed. Order within the chunk: scores -> P first
-        //      (while the previous chunk's P V runs), then, once that P V has released the single
-        //      f16 V^T buffer, this chunk's V widened into it; the P V of the chunk follows.
-        //      Q8: V stays in the stage as the E4M3 operand and the MMA warp frees the stage after P V.
-        // waits on the previous chunks' P V: chunk gg's completes kPvDone + (gg & 1), phase (gg >> 1) & 1
-        auto wait_pv = [&](int64_t gg) -> bool {
-          return tc_wait_warp(&bar[kPvDone + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl);
-        };
+        // ---- the chunk's K, V and scales have landed; V stays in the stage as the E4M3 operand
+        //      and the MMA warp frees the stage after the chunk's P V
         if (!tc_wait_warp(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl)) {
           ok = false;
           break;
@@ -537,12 +565,12 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         // this key's page scales
         const int blk = key >> 4;
         const float f = p.qk_scale_log2 * sc[st * 16 + blk];
-        const float vsc = sc[st * 16 + 8 + blk] * (Q8 ? 1.f : kTcPScale);
-        // Q8: E4M3 P^T = P * (V page scale) * C with C a power of two such that the largest P
-        // (2^kTcTau) times the chunk's largest V scale lands in (224, 448]; the same in every thread
-        float c_chunk = 1.f;
-        if constexpr (Q8) {
-          // only the blocks the producer filled for this chunk (the other slots hold stale values)
+        const float vsc = sc[st * 16 + 8 + blk];
+        // P^T = P * (V page scale) * C with C a power of two such that the largest P (2^kTcTau)
+        // times the chunk's largest V scale lands in (224, 448]; the same in every thread. Only the
+        // blocks the producer filled for this chunk count (the other slots hold stale values).
+        float c_chunk;
+        {
           const int nblk = min(kTcBlk, (d.tok_end - d.tok_begin - c * kTcChunk + 15) / 16);
           float svmax = 0.f;
           #pragma unroll
@@ -555,7 +583,14 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         if (!tc_wait_warp(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort, wl)) { ok = false; break; }
         tc_fence_after();
         float s[kTcN];
-        tmem_ld16(tmem + lane_off + kTcN * sb, s);
+        if constexpr (M::QP == 2) {  // the q hi and lo halves of S^T, added
+          float s2[2 * kTcN];
+          tmem_ld32(tmem + lane_off + M::NS * sb, s2);
+          #pragma unroll
+          for (int n = 0; n < kTcN; ++n) s[n] = s2[n] + s2[kTcN + n];
+        } else {
+          tmem_ld16(tmem + lane_off + M::NS * sb, s);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kSFree + sb]);
@@ -611,15 +646,13 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
             cm[4 * q4 + 2] = ordered_float(m.z); cm[4 * q4 + 3] = ordered_float(m.w);
           }
         }
-        // Q8: C may only shrink within a tile (the accumulated O^T carries the tile's C)
+        // C may only shrink within a tile (the accumulated O^T carries the tile's C)
         float c_factor = 1.f;
-        if constexpr (Q8) {
-          if (c == 0) {
-            c_ref = c_chunk;
-          } else if (c_chunk < c_ref) {
-            c_factor = c_chunk / c_ref;  // a power of two: exact
-            c_ref = c_chunk;
-          }
+        if (c == 0) {
+          c_ref = c_chunk;
+        } else if (c_chunk < c_ref) {
+          c_factor = c_chunk / c_ref;  // a power of two: exact
+          c_ref = c_chunk;
         }
         if (upd || c_factor != 1.f) {
           float alpha[kTcN];
@@ -639,14 +672,17 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           }
           if (c > 0 && resc) {
             // O^T holds chunks 0 .. c-1 of this tile once the previous chunk's P V is done: rescale
-            // it in place
+            // every part's columns in place
             if (!wait_pv(g - 1)) { ok = false; break; }
             tc_fence_after();
-            float o[kTcN];
-            tmem_ld16(tO, o);
             #pragma unroll
-            for (int n = 0; n < kTcN; ++n) o[n] *= alpha[n];
-            tmem_st16(tO, o);
+            for (int q = 0; q < M::PP; ++q) {
+              float o[kTcN];
+              tmem_ld16(tO + kTcN * q, o);
+              #pragma unroll
+              for (int n = 0; n < kTcN; ++n) o[n] *= alpha[n];
+              tmem_st16(tO + kTcN * q, o);
+            }
           }
         }
         // ---- P = 2^(s - m_ref) (at most 2^kTcTau); row sums in fp32
@@ -656,53 +692,44 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           pr[n] = fast_exp2(s[n] - (mref[n] == -INFINITY ? 0.f : mref[n]));
           lacc[n] += pr[n];
         }
-        // ---- P^T row of this key, 16 query rows: Q8: E4M3 P * (V page scale) * C into buffer g & 1,
-        //      which chunk g - 2's P V read; f16 P * (V page scale) * kTcPScale into the single P^T
-        //      buffer once the previous chunk's P V has read it and the f16 V^T buffer (a tile's first
-        //      chunk: the previous tile's epilogue waited for its last P V)
-        if (Q8 ? (g >= 2 && !wait_pv(g - 2)) : (c > 0 && !wait_pv(g - 1))) { ok = false; break; }
-        uint8_t* pbuf = sm + L::OFF_P + (int)(g & (L::NPB - 1)) * L::PB;
-        if constexpr (Q8) {
-          // the output is normalised by the weights as rounded, so it stays a convex combination of
-          // V rows (a single visible key reproduces its V row); lse keeps the exact sums
-          const float xs = vsc * c_ref, rxs = 1.f / xs;
-          uint32_t w8[4];
+        // ---- P^T row of this key, 16 query rows: x = P * (V page scale) * C rounded to E4M3 parts,
+        //      x = hi + mid + lo (Q8: hi alone), computed before the wait for the buffer
+        const float xs = vsc * c_ref;
+        uint32_t w8[M::PP][4];
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float x[4] = {pr[4 * i] * xs, pr[4 * i + 1] * xs, pr[4 * i + 2] * xs, pr[4 * i + 3] * xs};
           #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = f32x2_to_e4m3x2(pr[4 * i] * xs, pr[4 * i + 1] * xs);
-            const uint32_t hi = f32x2_to_e4m3x2(pr[4 * i + 2] * xs, pr[4 * i + 3] * xs);
-            w8[i] = valid ? (lo | (hi << 16)) : 0u;
-            if (valid) {
+          for (int q = 0; q < M::PP; ++q) {
+            const uint32_t lo = f32x2_to_e4m3x2(x[0], x[1]);
+            const uint32_t hi = f32x2_to_e4m3x2(x[2], x[3]);
+            w8[q][i] = valid ? (lo | (hi << 16)) : 0u;
+            if (Q8 || q + 1 < M::PP) {
               const float2 a = f16x2_to_float2(e4m3x2_to_f16x2(lo)), b = f16x2_to_float2(e4m3x2_to_f16x2(hi));
-              lrnd[4 * i] += a.x * rxs; lrnd[4 * i + 1] += a.y * rxs;
-              lrnd[4 * i + 2] += b.x * rxs; lrnd[4 * i + 3] += b.y * rxs;
+              if constexpr (Q8) {
+                // the output is normalised by the weights as rounded, so it stays a convex
+                // combination of V rows (a single visible key reproduces its V row); lse keeps the
+                // exact sums
+                if (valid) {
+                  const float rxs = 1.f / xs;
+                  lrnd[4 * i] += a.x * rxs; lrnd[4 * i + 1] += a.y * rxs;
+                  lrnd[4 * i + 2] += b.x * rxs; lrnd[4 * i + 3] += b.y * rxs;
+                }
+              } else {
+                x[0] -= a.x; x[1] -= a.y; x[2] -= b.x; x[3] -= b.y;  // exact: the next part rounds the rest
+              }
             }
           }
-          *reinterpret_cast<uint4*>(pbuf + key * kTcN) = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-        } else {
-          uint32_t h[8];
-          #pragma unroll
-          for (int i = 0; i < 8; ++i) h[i] = valid ? pack_f16(pr[2 * i] * vsc, pr[2 * i + 1] * vsc) : 0u;
-          uint8_t* pp = pbuf + (key >> 3) * 128 + (key & 7) * 16;
-          *reinterpret_cast<uint4*>(pp) = make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4*>(pp + 2048) = make_uint4(h[4], h[5], h[6], h[7]);
-          // ---- V row of this key widened to f16 (exact), 8 head dims per 16-byte core-matrix row
-          const uint8_t* vr = sm + L::OFF_V + st * L::KCH + key * kTcD;
-          uint8_t* vd = sm + L::OFF_V16 + (key >> 3) * 128 + (key & 7) * 16;
-          #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (valid) w = *reinterpret_cast<const uint4*>(vr + ((cc ^ (key & 7)) << 4));  // codes d = 16cc ..
-            const uint4 lo = make_uint4(e4m3x2_to_f16x2(w.x & 0xffffu), e4m3x2_to_f16x2(w.x >> 16),
-                                        e4m3x2_to_f16x2(w.y & 0xffffu), e4m3x2_to_f16x2(w.y >> 16));
-            const uint4 hi = make_uint4(e4m3x2_to_f16x2(w.z & 0xffffu), e4m3x2_to_f16x2(w.z >> 16),
-                                        e4m3x2_to_f16x2(w.w & 0xffffu), e4m3x2_to_f16x2(w.w >> 16));
-            *reinterpret_cast<uint4*>(vd + (2 * cc) * 2048) = lo;
-            *reinterpret_cast<uint4*>(vd + (2 * cc + 1) * 2048) = hi;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar[kKvEmpty + st]);  // the V half of the stage has been read
         }
+        // the P^T buffer: Q8 writes buffer g & 1, which chunk g - 2's P V read; otherwise the single
+        // buffer, once the previous chunk's P V has read it (a tile's first chunk: the previous
+        // tile's epilogue waited for its last P V)
+        if (M::NPB == 2 ? (g >= 2 && !wait_pv(g - 2)) : (c > 0 && !wait_pv(g - 1))) { ok = false; break; }
+        uint8_t* pbuf = sm + L::OFF_P + (int)(g & (M::NPB - 1)) * L::PB;
+        #pragma unroll
+        for (int q = 0; q < M::PP; ++q)
+          *reinterpret_cast<uint4*>(pbuf + q * L::PPLANE + key * kTcN) =
+              make_uint4(w8[q][0], w8[q][1], w8[q][2], w8[q][3]);
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
@@ -712,14 +739,10 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       // ---- the next tile's q: the MMA warp starts that tile while this one's epilogue runs
       if (dnext.b >= 0 && !publish_q(qx, qp ^ 1)) { ok = false; break; }
 
-      // ---- epilogue: row sums over the tile, O^T / l, out or partial (after the tile's last P V)
-      if (!tc_wait_warp(&bar[kPvDone + ((g - 1) & 1)], (uint32_t)(((g - 1) >> 1) & 1), p.status, abort, wl)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // row sums over the warp's 32 keys by a butterfly reduce-scatter: after the five levels,
-      // lanes 2c and 2c + 1 hold column c's sum (Q8: the exact sums, then the rounded ones)
+      // ---- epilogue: row sums over the tile, O^T / l, out or partial
+      // row sums over the warp's 32 keys by a butterfly reduce-scatter (before the wait for the
+      // tile's last P V): after the five levels, lanes 2c and 2c + 1 hold column c's sum (Q8: the
+      // exact sums, then the rounded ones)
       auto warp_colsum = [&](const float (&in)[kTcN], float* dst) {
         float v[kTcN];
         #pragma unroll
@@ -740,8 +763,10 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       };
       warp_colsum(lacc, ered);
       if constexpr (Q8) warp_colsum(lrnd, ered + 4 * kTcN);
-      float o[kTcN];
-      tmem_ld16(tO, o);
+      if (!wait_pv(g - 1)) { ok = false; break; }
+      tc_fence_after();
+      float osum[kTcN];
+      o_sum(tO, osum);
       tc_fence_before();
       if (!gsync()) { ok = false; break; }
       // lane n: row n's sums, the reciprocal that normalises O^T and (one warp) its lse
@@ -751,7 +776,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         const float* er = ered + (Q8 ? 4 * kTcN : 0);
         lr_n = er[lane] + er[kTcN + lane] + er[2 * kTcN + lane] + er[3 * kTcN + lane];
       }
-      const float inv_n = lr_n > 0.f ? __fdividef(1.f, (Q8 ? c_ref : kTcPScale) * lr_n) : 0.f;
+      const float inv_n = lr_n > 0.f ? __fdividef(1.f, c_ref * lr_n) : 0.f;
       if (warp == 0 && lane < p.GT) {
         float mr = mref[0];
         #pragma unroll
@@ -764,9 +789,10 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       #pragma unroll
       for (int n = 0; n < kTcN; ++n) {
         if (n >= p.GT) break;
+        const float o = osum[n];
         const int64_t row = __shfl_sync(0xffffffffu, row_n, n);
         const float inv = __shfl_sync(0xffffffffu, inv_n, n);
-        base_out[row * kTcD + dd] = o[n] * inv;
+        base_out[row * kTcD + dd] = o * inv;
       }
       ++ut;
       d = dnext;
@@ -779,7 +805,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
   __syncthreads();
   tc_fence_after();
   if (warp == 5)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kTcTmemCols) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(M::TMEM) : "memory");
 }
 
 }  // namespace decattn
