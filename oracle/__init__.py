@@ -298,3 +298,89 @@ def append_rope(q_new, k_new, v_new, page_table, seq_lens, k_pages, v_pages, bas
                                B, T, Hq, Hkv, d, P, num_pages, int(tab.shape[1]), float(base), q_out.ctypes.data,
                                kp.ctypes.data, vp.ctypes.data)
     return q_out, kp, vp, int(n)
+
+
+# ---- the same pre-processing over an FP8 E4M3 cache: appending rows to a page with one scale
+
+def e4m3_codes(values) -> np.ndarray:
+    """The E4M3 code (uint8) of each value, which must be an E4M3 number (e.g. from e4m3_round)."""
+    v = np.asarray(values, dtype=np.float64)
+    tab = e4m3_table()
+    mag = np.abs(v)
+    idx = np.searchsorted(tab[:127], mag)        # codes 0x00 .. 0x7E hold 0 .. 448, increasing
+    assert np.all(tab[np.minimum(idx, 126)] == mag), "not an E4M3 value"
+    return (idx | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
+
+
+def append_rope_fp8(q_new, k_new, v_new, page_table, seq_lens, k_codes, v_codes, kv_scales, base: float = 10000.0):
+    """Rotary embedding of the T new q and k rows and their append to an E4M3 paged cache with one
+    fp32 scale per (page, KV head) for K and for V (the reading for FP8 pages; "PaddlePaddle/HALOps"
+    README, Highlights, GQA attention item: fused pre/post-processing, BF16 / FP8 KV cache).
+
+    The scale of a page and head covers its valid rows: |row value| <= 448 * scale (the encoding
+    reading of the pages' FP8 scales). Appending new rows keeps that and never re-rounds old rows
+    it does not have to:
+      * x: the new rows' values (k rotated exactly, in fp64; v as given), A = max |x| over the
+        page's new rows, rounded to fp32;
+      * the page's old rows are its slots before the first new one; with old rows the scale
+        becomes s' = max(s, A / 448), else s' = A / 448 (1 when A = 0), the divisions in fp32;
+      * if s' > s, each old code is re-rounded: E4M3(fp32(value(code) * fp32(s / s')));
+      * new rows: E4M3(fp32(fp32(x) / s'));
+    E4M3(.) rounds to the nearest E4M3 value, ties to even, saturating at 448: every rounding
+    decision is taken on the same fp32 numbers a single-precision implementation forms. q is
+    rotated and rounded to bf16 as in append_rope; rows at positions < 0 have no slot.
+    Inputs: q_new [B][T][Hq][d], k_new / v_new [B][T][Hkv][d] bf16 bits; k_codes / v_codes uint8
+    [num_pages][Hkv][P][d]; kv_scales float32 [2][num_pages][Hkv]. Returns (q_out, k_codes',
+    v_codes', kv_scales'), copies."""
+    qn = np.asarray(q_new, dtype=np.uint16)
+    kn = np.asarray(k_new, dtype=np.uint16)
+    vn = np.asarray(v_new, dtype=np.uint16)
+    tab = np.asarray(page_table, dtype=np.int64)
+    L = np.asarray(seq_lens, dtype=np.int64)
+    kc = np.array(k_codes, dtype=np.uint8, copy=True)
+    vc = np.array(v_codes, dtype=np.uint8, copy=True)
+    sc = np.array(kv_scales, dtype=np.float32, copy=True)
+    B, T, Hq, d = qn.shape
+    Hkv = kn.shape[2]
+    P = kc.shape[2]
+    f32 = np.float32
+    val = e4m3_table()
+
+    def to64(bits):
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    # q: the bf16 append's rotation
+    pos_all = L[:, None] - T + np.arange(T)[None, :]                     # [B][T]
+    q_out = np.empty_like(qn)
+    for b in range(B):
+        for t in range(T):
+            pos = max(int(pos_all[b, t]), 0)
+            q_out[b, t] = bf16_bits(rope_rows(to64(qn[b, t]), [pos] * Hq, base))
+    for b in range(B):
+        first = int(max(L[b] - T, 0))
+        if L[b] <= first:
+            continue
+        for pg in range(first // P, (int(L[b]) - 1) // P + 1):
+            lo, hi = max(first, pg * P), min(int(L[b]), pg * P + P)   # new positions in this page
+            pid = int(tab[b, pg])
+            ts = np.arange(lo, hi) - (int(L[b]) - T)                 # their token indices
+            s_first = lo - pg * P
+            for which, codes, new in ((0, kc, kn), (1, vc, vn)):
+                for h in range(Hkv):
+                    x = to64(new[b, ts, h])                            # [n][d]
+                    if which == 0:
+                        x = rope_rows(x, np.arange(lo, hi), base)
+                    x32 = x.astype(f32)
+                    A = f32(np.max(np.abs(x32)))
+                    s_old = f32(sc[which, pid, h])
+                    if s_first > 0:
+                        s_new = max(s_old, f32(A / f32(448)))
+                    else:
+                        s_new = f32(A / f32(448)) if A > 0 else f32(1)
+                    if s_first > 0 and s_new != s_old:
+                        r = f32(s_old / s_new)
+                        old = val[codes[pid, h, :s_first]].astype(f32)
+                        codes[pid, h, :s_first] = e4m3_codes(e4m3_round((old * r).astype(np.float64)))
+                    codes[pid, h, s_first:s_first + (hi - lo)] = e4m3_codes(e4m3_round((x32 / s_new).astype(np.float64)))
+                    sc[which, pid, h] = s_new
+    return q_out, kc, vc, sc
