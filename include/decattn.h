@@ -326,13 +326,37 @@ DECATTN_API const char *dec_attn_status_string(int status);
  *   status      optional device int32: a page id outside [0, num_pages), or a page past the
  *               row's max_pages_per_seq entries, skips that token's K/V write and sets
  *               DECATTN_EDEVICE here (first error wins; the caller zeroes it). May be NULL.
- * Returns DECATTN_ENOTSUP for FP8 KV (appending to an FP8 page would need its scale, which
- * covers the whole page) or another head_dim, DECATTN_EINVAL / DECATTN_EALIGN for bad
+ * Returns DECATTN_ENOTSUP for FP8 KV (dec_attn_append_rope_fp8 takes those pools and their
+ * scales) or another head_dim, DECATTN_EINVAL / DECATTN_EALIGN for bad
  * arguments (nothing enqueued), DECATTN_ECUDA if the launch fails. */
 DECATTN_API int dec_attn_append_rope(const dec_attn_shape *shape, const void *q_new, const void *k_new,
                                      const void *v_new, const int32_t *page_table, const int32_t *seq_lens,
                                      float rope_base, void *q_out, void *k_pages, void *v_pages, int32_t *status,
                                      void *stream);
+
+/* dec_attn_append_rope for an E4M3 cache (the same passage: fused pre/post-processing around
+ * paged-KV decode over a BF16 / FP8 KV cache). The pages give one scale per (page, KV head) and do
+ * not say how a page takes new rows; the reading implemented keeps the scale covering the page's
+ * valid rows (|value| <= 448 * scale) and re-rounds older rows only when it must:
+ *   - q rows: exactly as dec_attn_append_rope (rotated, rounded to bf16, into q_out);
+ *   - per page and KV head touched by the new tokens, separately for K and V: x = the new rows'
+ *     values (k rotated as above, in fp32), A = max |x| over the page's new rows; the page's older
+ *     rows are its slots before the first new one. The scale becomes s' = max(s, A / 448) when there
+ *     are older rows, else A / 448 (1 when A = 0). When s' > s every older code c is re-rounded to
+ *     E4M3(value(c) * (s / s')); the new rows are stored as E4M3(x / s'). E4M3(.) is fp32 rounded to
+ *     the nearest E4M3 value, ties to even, saturating at +-448.
+ * Arguments as dec_attn_append_rope, with shape->kv_dtype DECATTN_KV_FP8E4M3 (or _MMA8: the same
+ * pages), k_pages / v_pages E4M3 codes [num_pages][Hkv][P][d] (no alignment needed) and
+ *   kv_scales  device fp32 [2][num_pages][Hkv] (K scales, then V), updated in place, 4-byte aligned.
+ * Two kernels on `stream` (q rows, then the pages), each waiting for the previous kernel before it
+ * reads. Pages of different requests must be distinct (as for every entry point); a page id outside
+ * the pool sets DECATTN_EDEVICE in `status` and that page is left unwritten. Returns
+ * DECATTN_ENOTSUP for a bf16 shape or another head_dim, DECATTN_EINVAL / DECATTN_EALIGN for bad
+ * arguments (nothing enqueued), DECATTN_ECUDA if a launch fails. */
+DECATTN_API int dec_attn_append_rope_fp8(const dec_attn_shape *shape, const void *q_new, const void *k_new,
+                                         const void *v_new, const int32_t *page_table, const int32_t *seq_lens,
+                                         float rope_base, void *q_out, void *k_pages, void *v_pages, float *kv_scales,
+                                         int32_t *status, void *stream);
 
 /* Prefill: causal attention of many query rows per request over the paged KV cache (the
  * prefill side of "PaddlePaddle/HALOps" README, Highlights, GQA attention item: variable-length

@@ -28,7 +28,7 @@ OK, EINVAL, ENOTSUP, ESMALL, ECUDA, ETIMEOUT, EDEVICE, EALIGN, ECAPACITY = 0, -1
 KV_BF16, KV_FP8E4M3, KV_FP8E4M3_MMA8 = 0, 1, 2
 API = ("dec_attn_default_bins", "dec_attn_default_tile_len", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
-       "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_prefill",
+       "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_append_rope_fp8", "dec_attn_prefill",
        "dec_attn_prefill_varlen", "dec_attn_plan_sparse_bytes",
        "dec_attn_plan_sparse", "dec_attn_last_error", "dec_attn_test_set_waits")
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -104,6 +104,9 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_append_rope.restype = i32
         lib.dec_attn_prefill.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, vp, vp, vp]
         lib.dec_attn_prefill.restype = i32
+        lib.dec_attn_append_rope_fp8.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, C.c_float, vp, vp, vp, vp,
+                                                 vp, vp]
+        lib.dec_attn_append_rope_fp8.restype = i32
         lib.dec_attn_prefill_varlen.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp]
         lib.dec_attn_prefill_varlen.restype = i32
         lib.dec_attn_test_set_waits.argtypes = [C.c_uint64, C.c_int32]
@@ -322,6 +325,27 @@ def append_rope(q_new: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, p
                                   _ptr(status), _stream_handle(stream))
     if rc != OK:
         raise DecAttnError(rc, "dec_attn_append_rope")
+    return q_out
+
+
+def append_rope_fp8(q_new: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, page_table: torch.Tensor,
+                    seq_lens: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, kv_scales: torch.Tensor,
+                    *, rope_base: float = 10000.0, q_out: torch.Tensor | None = None,
+                    status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """dec_attn_append_rope_fp8: the fused pre-processing over an E4M3 cache (k_pages / v_pages uint8
+    or float8_e4m3fn codes [num_pages][Hkv][P][d], kv_scales fp32 [2][num_pages][Hkv], all updated in
+    place); returns the rotated q."""
+    lib = load_library()
+    B, T, Hq, d = q_new.shape
+    num_pages, Hkv, P, d2 = k_pages.shape
+    shape = ShapeT(B, Hq, Hkv, d, T, P, num_pages, int(page_table.shape[1]), KV_FP8E4M3, 0.0)
+    if q_out is None:
+        q_out = torch.empty_like(q_new)
+    rc = lib.dec_attn_append_rope_fp8(C.byref(shape), _ptr(q_new), _ptr(k_new), _ptr(v_new), _ptr(page_table),
+                                      _ptr(seq_lens), float(rope_base), _ptr(q_out), _ptr(k_pages), _ptr(v_pages),
+                                      _ptr(kv_scales), _ptr(status), _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_append_rope_fp8")
     return q_out
 
 

@@ -38,8 +38,25 @@ struct AppendParams {
   uint16_t* v_pages;
   int32_t* status;         // optional device word: DECATTN_EDEVICE for a bad page id
   int B, T, Hq, Hkv, P, num_pages, mpps;
+  int rows;                       // rows per token this kernel writes: Hq + 2 Hkv (bf16 pages) or Hq (FP8)
   int groups;                     // row groups of kAppendWarps rows per token
   double theta[kAppendMaxHalf];   // base^(-2i/d), i < d/2
+};
+
+// The K / V side of the step for E4M3 pages (one fp32 scale per (page, KV head) and K or V): one
+// block per (request, page touched by the new tokens, KV head, K or V), one thread per head dim.
+struct AppendFp8Params {
+  const uint16_t* k_new;   // bf16 [B][T][Hkv][D]
+  const uint16_t* v_new;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  uint8_t* k_pages;        // E4M3 codes [num_pages][Hkv][P][D]
+  uint8_t* v_pages;
+  float* kv_scales;        // [2][num_pages][Hkv]
+  int32_t* status;
+  int B, T, Hkv, P, num_pages, mpps;
+  int maxpg;                      // pages the T new tokens of a request can touch
+  double theta[kAppendMaxHalf];
 };
 
 template <int E>
@@ -64,7 +81,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
   // this warp's row (q heads, then k, then v): its loads go out before the shared work below
   const int lane = threadIdx.x & 31;
   const int r = grp * kAppendWarps + (threadIdx.x >> 5);
-  const bool has_row = r < p.Hq + 2 * p.Hkv;
+  const bool has_row = r < p.rows;
   const bool is_q = r < p.Hq, is_k = !is_q && r < p.Hq + p.Hkv;
   const int h = is_q ? 0 : is_k ? r - p.Hq : r - p.Hq - p.Hkv;
   const uint16_t* src = is_q ? p.q_new + ((int64_t)bt * p.Hq + r) * D
@@ -127,6 +144,89 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
   }
 }
 
+// E4M3 pages: the page's scale covers its valid rows (|value| <= 448 * scale). With x the new rows'
+// values (k rotated as in append_rope_kernel, in fp32) and A = max |x| over the page's new rows, the
+// scale becomes max(s, A / 448) if the page holds older rows (its slots before the first new one),
+// else A / 448 (1 when A = 0); older codes are re-rounded, E4M3(value * (s / s')), only when the
+// scale grows; new rows are E4M3(x / s'). Every rounding is fp32 then round-to-nearest-even
+// (saturating) to E4M3.
+template <int D>
+__global__ void __launch_bounds__(D) append_fp8_kernel(const AppendFp8Params p) {
+  constexpr int HALF = D / 2;
+  __shared__ float wmax[D / 32];
+  griddep_wait();  // the pages and scales were last touched by earlier kernels of the stream
+  const int b = blockIdx.x / p.maxpg, pi = blockIdx.x - b * p.maxpg;
+  const int h = blockIdx.y, which = blockIdx.z;  // 0: K, 1: V
+  const int L = p.seq_lens[b];
+  const int first = max(L - p.T, 0);  // the first new position with a slot
+  if (L <= first) return;
+  const int pg = first / p.P + pi;
+  if (pg * p.P >= L) return;
+  const int lo = max(first, pg * p.P), hi = min(L, pg * p.P + p.P);  // new positions in this page
+  const int s_first = lo - pg * p.P;
+  const int pid = pg < p.mpps ? p.page_table[(int64_t)b * p.mpps + pg] : -1;
+  if (pid < 0 || pid >= p.num_pages) {
+    if (threadIdx.x == 0) set_status(p.status, DECATTN_EDEVICE);
+    return;
+  }
+  const int d = threadIdx.x;
+  const uint16_t* src = which == 0 ? p.k_new : p.v_new;
+  auto bf = [](uint16_t u) { return __uint_as_float((uint32_t)u << 16); };
+  // element d of the new row at position pos (k: rotated)
+  auto value = [&](int pos) -> float {
+    const uint16_t* row = src + (((int64_t)b * p.T + (pos - (L - p.T))) * p.Hkv + h) * D;
+    const float x = bf(row[d]);
+    if (which == 1) return x;
+    const int i = d < HALF ? d : d - HALF;
+    const float xp = bf(row[d < HALF ? d + HALF : d - HALF]);
+    double sn, cs;
+    sincos((double)pos * p.theta[i], &sn, &cs);
+    const float c = (float)cs, sf = (float)sn;
+    return d < HALF ? x * c - xp * sf : x * c + xp * sf;
+  };
+  float amax = 0.f;
+  for (int pos = lo; pos < hi; ++pos) amax = fmaxf(amax, fabsf(value(pos)));
+  const int64_t si = ((int64_t)which * p.num_pages + pid) * p.Hkv + h;
+  const float s_old = p.kv_scales[si];  // read by every thread before the barrier below
+  #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((d & 31) == 0) wmax[d >> 5] = amax;
+  __syncthreads();
+  #pragma unroll
+  for (int w = 0; w < D / 32; ++w) amax = fmaxf(amax, wmax[w]);
+  const float s_new = s_first > 0 ? fmaxf(s_old, amax / 448.f) : (amax > 0.f ? amax / 448.f : 1.f);
+  uint8_t* base = (which == 0 ? p.k_pages : p.v_pages) + ((int64_t)pid * p.Hkv + h) * p.P * D;
+  if (s_first > 0 && s_new != s_old) {
+    const float r = s_old / s_new;
+    for (int sl = 0; sl < s_first; ++sl) {
+      const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(base[sl * D + d]), __NV_E4M3);
+      const float v = __half2float(__half(hr)) * r;
+      base[sl * D + d] = static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+    }
+  }
+  for (int pos = lo; pos < hi; ++pos)
+    base[(pos - pg * p.P) * D + d] = static_cast<uint8_t>(__nv_cvt_float_to_fp8(value(pos) / s_new, __NV_SATFINITE, __NV_E4M3));
+  if (d == 0) p.kv_scales[si] = s_new;
+}
+
+cudaError_t launch_append_fp8(const AppendFp8Params& p, int D, cudaStream_t st) {
+  const int64_t blocks = (int64_t)p.B * p.maxpg;
+  if (blocks <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks, (unsigned)p.Hkv, 2);
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (D == 128) return cudaLaunchKernelEx(&cfg, append_fp8_kernel<128>, p);
+  if (D == 64) return cudaLaunchKernelEx(&cfg, append_fp8_kernel<64>, p);
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t st) {
   const int64_t blocks = (int64_t)p.B * p.T * p.groups;
   if (blocks <= 0) return cudaSuccess;
@@ -145,6 +245,47 @@ cudaError_t launch_append(const AppendParams& p, int D, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
+// Argument checks shared by both entry points; fills the row kernel's parameters.
+static int append_setup(const dec_attn_shape* shape, const void* q_new, const void* k_new, const void* v_new,
+                        const int32_t* page_table, const int32_t* seq_lens, float rope_base, void* q_out,
+                        void* k_pages, void* v_pages, int32_t* status, bool fp8, AppendParams& p) {
+  if (!shape) return DECATTN_EINVAL;
+  const dec_attn_shape& s = *shape;
+  if (s.batch < 0 || s.q_tokens <= 0 || s.n_q_heads <= 0 || s.n_kv_heads <= 0 || s.page_size <= 0 ||
+      s.num_pages < 0 || s.max_pages_per_seq < 0 || s.n_q_heads % s.n_kv_heads != 0)
+    return DECATTN_EINVAL;
+  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return DECATTN_EINVAL;
+  if (fp8 ? (s.kv_dtype != DECATTN_KV_FP8E4M3 && s.kv_dtype != DECATTN_KV_FP8E4M3_MMA8)
+          : s.kv_dtype != DECATTN_KV_BF16)
+    return DECATTN_ENOTSUP;
+  if (s.head_dim != 64 && s.head_dim != 128) return DECATTN_ENOTSUP;
+  if (s.batch == 0) return DECATTN_OK;
+  if (!q_new || !k_new || !v_new || !page_table || !seq_lens || !q_out || !k_pages || !v_pages)
+    return DECATTN_EINVAL;
+  const uintptr_t need = s.head_dim == 128 ? 3 : 1;  // 4-byte (d = 128) or 2-byte lane accesses
+  for (const void* ptr : {q_new, k_new, v_new, (const void*)q_out})
+    if (reinterpret_cast<uintptr_t>(ptr) & need) return DECATTN_EALIGN;
+  if (!fp8)
+    for (const void* ptr : {(const void*)k_pages, (const void*)v_pages})
+      if (reinterpret_cast<uintptr_t>(ptr) & need) return DECATTN_EALIGN;
+  p.q_new = static_cast<const uint16_t*>(q_new);
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.v_new = static_cast<const uint16_t*>(v_new);
+  p.page_table = page_table;
+  p.seq_lens = seq_lens;
+  p.q_out = static_cast<uint16_t*>(q_out);
+  p.k_pages = fp8 ? nullptr : static_cast<uint16_t*>(k_pages);
+  p.v_pages = fp8 ? nullptr : static_cast<uint16_t*>(v_pages);
+  p.status = status;
+  p.B = s.batch; p.T = s.q_tokens; p.Hq = s.n_q_heads; p.Hkv = s.n_kv_heads; p.P = s.page_size;
+  p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
+  p.rows = fp8 ? s.n_q_heads : s.n_q_heads + 2 * s.n_kv_heads;
+  p.groups = (p.rows + kAppendWarps - 1) / kAppendWarps;
+  for (int i = 0; i < s.head_dim / 2; ++i) p.theta[i] = std::pow((double)rope_base, -2.0 * i / s.head_dim);
+  if ((int64_t)s.batch * s.q_tokens * p.groups > 0x7fffffff) return DECATTN_ENOTSUP;
+  return 1;  // arguments good, work to launch
+}
+
 }  // namespace decattn
 
 using namespace decattn;
@@ -153,35 +294,42 @@ extern "C" int dec_attn_append_rope(const dec_attn_shape* shape, const void* q_n
                                     const void* v_new, const int32_t* page_table, const int32_t* seq_lens,
                                     float rope_base, void* q_out, void* k_pages, void* v_pages, int32_t* status,
                                     void* stream) {
-  if (!shape) return DECATTN_EINVAL;
-  const dec_attn_shape& s = *shape;
-  if (s.batch < 0 || s.q_tokens <= 0 || s.n_q_heads <= 0 || s.n_kv_heads <= 0 || s.page_size <= 0 ||
-      s.num_pages < 0 || s.max_pages_per_seq < 0 || s.n_q_heads % s.n_kv_heads != 0)
-    return DECATTN_EINVAL;
-  if (!(rope_base > 0.f) || !std::isfinite(rope_base)) return DECATTN_EINVAL;
-  if (s.kv_dtype != DECATTN_KV_BF16) return DECATTN_ENOTSUP;  // an FP8 page's scale would need the whole page
-  if (s.head_dim != 64 && s.head_dim != 128) return DECATTN_ENOTSUP;
-  if (s.batch == 0) return DECATTN_OK;
-  if (!q_new || !k_new || !v_new || !page_table || !seq_lens || !q_out || !k_pages || !v_pages)
-    return DECATTN_EINVAL;
-  const uintptr_t need = s.head_dim == 128 ? 3 : 1;  // 4-byte (d = 128) or 2-byte lane accesses
-  for (const void* ptr : {q_new, k_new, v_new, (const void*)q_out, (const void*)k_pages, (const void*)v_pages})
-    if (reinterpret_cast<uintptr_t>(ptr) & need) return DECATTN_EALIGN;
   AppendParams p;
-  p.q_new = static_cast<const uint16_t*>(q_new);
-  p.k_new = static_cast<const uint16_t*>(k_new);
-  p.v_new = static_cast<const uint16_t*>(v_new);
-  p.page_table = page_table;
-  p.seq_lens = seq_lens;
-  p.q_out = static_cast<uint16_t*>(q_out);
-  p.k_pages = static_cast<uint16_t*>(k_pages);
-  p.v_pages = static_cast<uint16_t*>(v_pages);
-  p.status = status;
-  p.B = s.batch; p.T = s.q_tokens; p.Hq = s.n_q_heads; p.Hkv = s.n_kv_heads; p.P = s.page_size;
-  p.num_pages = s.num_pages; p.mpps = s.max_pages_per_seq;
-  p.groups = (s.n_q_heads + 2 * s.n_kv_heads + kAppendWarps - 1) / kAppendWarps;
-  for (int i = 0; i < s.head_dim / 2; ++i) p.theta[i] = std::pow((double)rope_base, -2.0 * i / s.head_dim);
-  if ((int64_t)s.batch * s.q_tokens * p.groups > 0x7fffffff) return DECATTN_ENOTSUP;
-  const cudaError_t e = launch_append(p, s.head_dim, static_cast<cudaStream_t>(stream));
+  const int rc = append_setup(shape, q_new, k_new, v_new, page_table, seq_lens, rope_base, q_out, k_pages, v_pages,
+                              status, false, p);
+  if (rc <= 0) return rc;
+  const cudaError_t e = launch_append(p, shape->head_dim, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DECATTN_OK : cuda_fail("append kernel launch", e);
+}
+
+extern "C" int dec_attn_append_rope_fp8(const dec_attn_shape* shape, const void* q_new, const void* k_new,
+                                        const void* v_new, const int32_t* page_table, const int32_t* seq_lens,
+                                        float rope_base, void* q_out, void* k_pages, void* v_pages, float* kv_scales,
+                                        int32_t* status, void* stream) {
+  AppendParams p;
+  const int rc = append_setup(shape, q_new, k_new, v_new, page_table, seq_lens, rope_base, q_out, k_pages, v_pages,
+                              status, true, p);
+  if (rc <= 0) return rc;
+  if (!kv_scales) return DECATTN_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(kv_scales) & 3) != 0) return DECATTN_EALIGN;
+  const dec_attn_shape& s = *shape;
+  AppendFp8Params f;
+  f.k_new = p.k_new;
+  f.v_new = p.v_new;
+  f.page_table = page_table;
+  f.seq_lens = seq_lens;
+  f.k_pages = static_cast<uint8_t*>(k_pages);
+  f.v_pages = static_cast<uint8_t*>(v_pages);
+  f.kv_scales = kv_scales;
+  f.status = status;
+  f.B = s.batch; f.T = s.q_tokens; f.Hkv = s.n_kv_heads; f.P = s.page_size; f.num_pages = s.num_pages;
+  f.mpps = s.max_pages_per_seq;
+  f.maxpg = (s.q_tokens + s.page_size - 1) / s.page_size + 1;
+  for (int i = 0; i < s.head_dim / 2; ++i) f.theta[i] = p.theta[i];
+  if ((int64_t)s.batch * f.maxpg > 0x7fffffff || s.n_kv_heads > 65535) return DECATTN_ENOTSUP;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_append(p, s.head_dim, st);  // q rows
+  if (e != cudaSuccess) return cuda_fail("append kernel launch", e);
+  e = launch_append_fp8(f, s.head_dim, st);          // K / V pages and scales
+  return e == cudaSuccess ? DECATTN_OK : cuda_fail("FP8 append kernel launch", e);
 }

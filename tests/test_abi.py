@@ -250,3 +250,16 @@ def test_default_tile_len_rule(lib):
     assert f(0, 8, 100, 16, 128, 4, da.KV_BF16, 592) == da.EINVAL
     assert f(4, 8, 100, 24, 128, 4, da.KV_BF16, 592) == da.EINVAL           # page not a multiple of 16
     assert f(4, 8, 100, 16, 128, 4, da.KV_BF16, 0) == da.EINVAL
+
+
+def test_append_rope_fp8_rejects_bad_args(lib):
+    def call(s, **kw):
+        args = dict(q=FAKE, k=FAKE, v=FAKE, tab=FAKE, lens=FAKE, qo=FAKE, kp=FAKE, vp=FAKE, sc=FAKE)
+        args.update(kw)
+        return lib.dec_attn_append_rope_fp8(C.byref(s), args["q"], args["k"], args["v"], args["tab"], args["lens"],
+                                            10000.0, args["qo"], args["kp"], args["vp"], args["sc"], None, None)
+    assert call(_shape(kv_dtype=da.KV_BF16)) == da.ENOTSUP          # bf16 pages go through dec_attn_append_rope
+    assert call(_shape(kv_dtype=da.KV_FP8E4M3, head_dim=96)) == da.ENOTSUP
+    assert call(_shape(kv_dtype=da.KV_FP8E4M3), sc=None) == da.EINVAL
+    assert call(_shape(kv_dtype=da.KV_FP8E4M3), sc=FAKE + 2) == da.EALIGN
+    assert call(_shape(kv_dtype=da.KV_FP8E4M3), q=FAKE + 2) == da.EALIGN

@@ -153,3 +153,83 @@ def test_append_plan_run_in_one_cuda_graph():
     pr2 = W.Problem(**{**pr.__dict__, "q": want_q, "k_pages": want_k, "v_pages": want_v})
     ref_o, ref_l = oracle.decode(pr2)
     U.check_rows(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, "graph: append + plan + run")
+
+
+# ---------------------------------------------------------------- E4M3 pages (dec_attn_append_rope_fp8)
+
+def _fp8_problem(seq_lens, *, Hq=8, Hkv=2, d=128, P=16, T=1, seed=7):
+    return W.make_problem(name="append_fp8", batch=len(seq_lens), n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d,
+                          seq_lens=seq_lens, page_size=P, q_tokens=T, kv_dtype="fp8e4m3", seed=seed, tile_len=64)
+
+
+def _run_append_fp8(pr, q_new, k_new, v_new, status=None, table=None):
+    tab = torch.from_numpy(np.ascontiguousarray(pr.page_table if table is None else table)).cuda()
+    lens = torch.from_numpy(pr.seq_lens.astype(np.int32)).cuda()
+    kp = torch.from_numpy(np.ascontiguousarray(pr.k_pages)).cuda()
+    vp = torch.from_numpy(np.ascontiguousarray(pr.v_pages)).cuda()
+    sc = torch.from_numpy(np.ascontiguousarray(pr.kv_scales)).cuda()
+    qn, kn, vn = _to_dev_bits(q_new), _to_dev_bits(k_new), _to_dev_bits(v_new)
+    q_out = da.append_rope_fp8(qn, kn, vn, tab, lens, kp, vp, sc, status=status)
+    torch.cuda.synchronize()
+    return q_out, kp, vp, sc, tab, lens
+
+
+def _e4m3_step(values, scale):
+    """One E4M3 step (3 mantissa bits, subnormal step 2^-9) at each value's magnitude, times scale."""
+    m = np.maximum(np.abs(values) / scale, 2.0 ** -6)
+    return np.maximum(2.0 ** (np.floor(np.log2(m)) - 3), 2.0 ** -9) * scale
+
+
+@pytest.mark.parametrize("T,P,d", [(1, 16, 128), (4, 16, 128), (8, 16, 64), (3, 32, 128), (8, 64, 128)])
+def test_append_fp8_matches_oracle(T, P, d):
+    # requests whose new tokens start a fresh page, continue a page (the scale may grow), span two
+    # pages, and sit partly before position 0 (L < T)
+    lens = [P * 3, P * 2 + 3, P + T + 5, max(T - 2, 1), 5 * P + P // 2]
+    pr = _fp8_problem(lens, T=T, P=P, d=d, seed=T * 10 + P)
+    q_new, k_new, v_new = W.make_step_inputs(pr)
+    # scale the new rows up for half the requests, so that their pages' scales grow
+    big = np.array([1, 0, 1, 0, 1], dtype=bool)[:, None, None, None]
+    kf, vf = _bits_to_f64(k_new), _bits_to_f64(v_new)
+    k_new = W.bf16_bits_from_f32(np.where(big, kf * 12, kf).astype(np.float32))
+    v_new = W.bf16_bits_from_f32(np.where(big, vf * 12, vf).astype(np.float32))
+    q_out, kp, vp, sc, tab, lens_d = _run_append_fp8(pr, q_new, k_new, v_new)
+    want_q, want_k, want_v, want_sc = oracle.append_rope_fp8(q_new, k_new, v_new, pr.page_table, pr.seq_lens,
+                                                             pr.k_pages, pr.v_pages, pr.kv_scales)
+    assert np.all(_within_one_ulp(_from_dev_bits(q_out), want_q))
+    got_k, got_v, got_sc = kp.cpu().numpy(), vp.cpu().numpy(), sc.cpu().numpy()
+    # V: exact inputs, every rounding decision on the same fp32 numbers -> bit-exact codes and scales
+    assert np.array_equal(got_v, want_v)
+    assert np.array_equal(got_sc[1], want_sc[1])
+    # K: rotated in fp32 on the GPU, exactly in the oracle -> scales within an fp32 unit, codes within one
+    # E4M3 step (a rounding decision can flip only next to a tie), and almost all codes equal
+    assert np.allclose(got_sc[0], want_sc[0], rtol=2.0 ** -22, atol=0)
+    tabv = oracle.e4m3_table()
+    gk = tabv[got_k] * got_sc[0][:, :, None, None]
+    wk = tabv[want_k] * want_sc[0][:, :, None, None]
+    assert np.all(np.abs(gk - wk) <= _e4m3_step(wk, want_sc[0][:, :, None, None]) * (1 + 1e-6))
+    assert np.mean(got_k != want_k) < 1e-3
+    # decode over the appended cache (its own values) meets the decode tolerances
+    pr2 = W.Problem(**{**pr.__dict__, "q": _from_dev_bits(q_out), "k_pages": got_k, "v_pages": got_v,
+                       "kv_scales": got_sc})
+    out, lse, _, st = U.run_problem(pr2)
+    assert st == da.OK
+    ref_o, ref_l = oracle.decode(pr2)
+    U.check_rows(out.cpu().numpy(), lse.cpu().numpy(), ref_o, ref_l, f"decode after FP8 append T{T} P{P} d{d}")
+
+
+def test_append_fp8_bad_page_id_reports_and_skips_the_page():
+    pr = _fp8_problem([40, 70], T=2)
+    q_new, k_new, v_new = W.make_step_inputs(pr)
+    table = pr.page_table.copy()
+    table[1, (70 - 2) // 16] = pr.num_pages + 3
+    st = torch.zeros((), dtype=torch.int32, device="cuda")
+    q_out, kp, vp, sc, _, _ = _run_append_fp8(pr, q_new, k_new, v_new, status=st, table=table)
+    assert int(st.item()) == da.EDEVICE
+    # request 0's page was written as the oracle writes it; every page of request 1 is unchanged
+    _, want_k, _, _ = oracle.append_rope_fp8(q_new, k_new, v_new, pr.page_table, pr.seq_lens, pr.k_pages,
+                                             pr.v_pages, pr.kv_scales)
+    got_k = kp.cpu().numpy()
+    pid0 = int(pr.page_table[0, (40 - 2) // 16])
+    assert np.mean(got_k[pid0] != want_k[pid0]) < 1e-3
+    for p_ in pr.page_table[1, :(70 + 15) // 16]:
+        assert np.array_equal(got_k[p_], pr.k_pages[p_])
