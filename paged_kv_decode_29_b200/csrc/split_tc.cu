@@ -14,9 +14,10 @@
 //  * O^T (128 head dims x 16 query rows, fp32 in tensor memory) += V^T P^T, A = the staged V codes
 //    (MN-major: head dims contiguous, 128-byte swizzle). B = P^T with P scaled by (V page scale) *
 //    C (C a power of two per chunk that keeps P within E4M3's range) and split into three E4M3
-//    parts hi, mid, lo side by side (N = 48; the three 16-column groups of O^T are added in the
-//    epilogue): about 12 significant bits, as close to P as an f16 P would be, so the result
-//    meets the same tolerance as the bf16 path. Q8: one part (N = 16) and its own tolerance.
+//    parts x = hi + mid / 16 + lo / 256 side by side (N = 48; the epilogue adds the three 16-column
+//    groups of O^T with those weights): about 12 significant bits, as close to P as an f16 P would
+//    be, so the result meets the same tolerance as the bf16 path. Q8: one part (N = 16) and its own
+//    tolerance.
 // Thread j of the 128-thread softmax group owns key j of the chunk (tensor-memory lane j) and
 // reads its scores with one tcgen05.ld, so the per-key work has no fragment shuffles.
 //
@@ -399,9 +400,6 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       // N = the P parts' columns
       constexpr uint32_t idS = umma_idesc(0, 0, 0, 0, kTcChunk, M::NS);
       constexpr uint32_t idO = umma_idesc(0, 0, 1, 1, kTcD, M::NO);
-      int us = 0; uint32_t uph = 0;
-      int64_t g = 0;  // chunks issued so far
-      int ut = 0;     // tiles started so far
       bool ok = true;
       // descriptors, built once: the start address is the low 14 bits (16-byte units), so a
       // stage or a k-step adds to the base descriptor.
@@ -415,49 +413,89 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       const uint64_t dV = umma_desc(base + L::OFF_V, 1024, 1024, 2);
       const uint64_t dP = umma_desc(base + L::OFF_P, 128, L::PPLANE, 0);
       const uint32_t tO = tmem + 2 * M::NS;
-      // O^T (+)= V^T P^T over chunk gg's 128 keys. A tile's first chunk overwrites O^T: the
-      // softmax group signals that chunk's P only after it has read the previous tile's O^T.
-      auto pv = [&](int64_t gg, bool first_of_tile) -> bool {
-        if (!tc_wait(&bar[kPReady + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl)) return false;
-        tc_fence_after();
-        const int sg = (int)(gg % kTcStages);
-        const uint64_t a0 = dV + (uint64_t)((sg * L::KCH) >> 4);
-        const uint64_t b0 = dP + (uint64_t)((((int)(gg & (M::NPB - 1))) * L::PB) >> 4);
-        #pragma unroll
-        for (int k = 0; k < kTcChunk / 32; ++k)  // 32 keys per instruction: 4 KB of V, 512 B per P part
-          umma_f8(tO, a0 + (uint64_t)(256 * k), b0 + (uint64_t)(32 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
-        umma_commit(&bar[kPvDone + (gg & 1)]);
-        umma_commit(&bar[kKvEmpty + sg]);  // K and V of the stage have both been read
-        return true;
-      };
+      // Two cursors, each taking its barriers' phases in order, issued in whichever order they
+      // become ready, so that neither waits for the other's operands:
+      //  * S^T of chunk gs (global chunk count) once its K has landed and the softmax group has read
+      //    the S^T buffer's previous contents; a new tile first needs its descriptor and its q;
+      //  * O^T (+)= V^T P^T of chunk gp once the softmax group has written its P^T. A tile's first
+      //    chunk overwrites O^T: the softmax group signals that chunk's P only after it has read the
+      //    previous tile's O^T.
+      int us = 0; uint32_t uph = 0;  // tile descriptor slot
+      int64_t gs = 0, gp = 0;        // next chunk for S^T / for P V
+      int ts = -1;                   // tiles opened by the S cursor, minus 1
+      int cs = 0, ncs = 0;           // the S cursor's chunk within its tile, and that tile's chunks
+      bool need_q = false;           // the S cursor's tile still waits for its q
+      bool done = false;             // the end-of-work descriptor has been read
+      int tp = 0, cp = 0;            // the P V cursor's tile and chunk within it
+      int nc_of[2] = {0, 0};         // chunks of the tiles opened, by tile parity
+      uint64_t dQ = dQ0;
+      uint64_t t_last = globaltimer_ns();
       for (;;) {
-        if (!tc_wait(&bar[kUFull + us], uph, p.status, abort, wl)) { ok = false; break; }
-        const Unit d = umeta[us];
-        mbar_arrive(&bar[kUEmpty + us]);
-        us ^= 1; if (us == 0) uph ^= 1;
-        if (d.b < 0) break;
-        const int nc = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
-        if (!tc_wait(&bar[kQReady], (uint32_t)(ut & 1), p.status, abort, wl)) { ok = false; break; }
-        const uint64_t dQ = dQ0 + (uint64_t)(((ut & 1) * L::QB) >> 4);
-        for (int c = 0; c < nc; ++c, ++g) {
-          const int st = (int)(g % kTcStages), sb = (int)(g & 1);
-          if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl) ||
-              !tc_wait(&bar[kSFree + sb], (uint32_t)(((g >> 1) & 1) ^ 1), p.status, abort, wl)) {
-            ok = false;
-            break;
+        bool progress = false;
+        // open the next tile for S^T (at most one tile ahead of the P V cursor: two q buffers)
+        if (!done && cs == ncs && ts + 1 - tp < 2 && mbar_test(&bar[kUFull + us], uph)) {
+          const Unit d = umeta[us];
+          mbar_arrive(&bar[kUEmpty + us]);
+          us ^= 1; if (us == 0) uph ^= 1;
+          if (d.b < 0) {
+            done = true;
+          } else {
+            ++ts;
+            cs = 0;
+            ncs = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
+            nc_of[ts & 1] = ncs;
+            need_q = true;
           }
-          tc_fence_after();
-          // S^T = K (q parts)^T: four 32-byte k-steps of the 128-byte swizzled rows
-          const uint64_t dK = dK0 + (uint64_t)((st * L::KCH) >> 4);
-          #pragma unroll
-          for (int kk = 0; kk < kTcD / 32; ++kk)
-            umma_f8(tmem + M::NS * sb, dK + (uint64_t)(2 * kk), dQ + (uint64_t)(2 * kk), idS, kk > 0 ? 1u : 0u);
-          umma_commit(&bar[kSFull + sb]);
-          if (c > 0 && !pv(g - 1, c == 1)) { ok = false; break; }
+          progress = true;
         }
-        if (!ok) break;
-        if (!pv(g - 1, nc == 1)) { ok = false; break; }
-        ++ut;
+        if (need_q && mbar_test(&bar[kQReady], (uint32_t)(ts & 1))) {
+          need_q = false;
+          dQ = dQ0 + (uint64_t)(((ts & 1) * L::QB) >> 4);
+          progress = true;
+        }
+        if (!need_q && cs < ncs) {
+          const int st = (int)(gs % kTcStages), sb = (int)(gs & 1);
+          if (mbar_test(&bar[kKvFull + st], (uint32_t)((gs / kTcStages) & 1)) &&
+              mbar_test(&bar[kSFree + sb], (uint32_t)(((gs >> 1) & 1) ^ 1))) {
+            tc_fence_after();
+            // S^T = K (q parts)^T: four 32-byte k-steps of the 128-byte swizzled rows
+            const uint64_t dK = dK0 + (uint64_t)((st * L::KCH) >> 4);
+            #pragma unroll
+            for (int kk = 0; kk < kTcD / 32; ++kk)
+              umma_f8(tmem + M::NS * sb, dK + (uint64_t)(2 * kk), dQ + (uint64_t)(2 * kk), idS, kk > 0 ? 1u : 0u);
+            umma_commit(&bar[kSFull + sb]);
+            ++cs;
+            ++gs;
+            progress = true;
+          }
+        }
+        if (gp < gs && mbar_test(&bar[kPReady + (gp & 1)], (uint32_t)((gp >> 1) & 1))) {
+          tc_fence_after();
+          const int sg = (int)(gp % kTcStages);
+          const uint64_t a0 = dV + (uint64_t)((sg * L::KCH) >> 4);
+          const uint64_t b0 = dP + (uint64_t)((((int)(gp & (M::NPB - 1))) * L::PB) >> 4);
+          const bool first_of_tile = cp == 0;
+          #pragma unroll
+          for (int k = 0; k < kTcChunk / 32; ++k)  // 32 keys per instruction: 4 KB of V, 512 B per P part
+            umma_f8(tO, a0 + (uint64_t)(256 * k), b0 + (uint64_t)(32 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
+          umma_commit(&bar[kPvDone + (gp & 1)]);
+          umma_commit(&bar[kKvEmpty + sg]);  // K and V of the stage have both been read
+          ++gp;
+          if (++cp == nc_of[tp & 1]) { ++tp; cp = 0; }
+          progress = true;
+        }
+        if (done && cs == ncs && gp == gs) break;  // every chunk's products issued
+        const uint64_t now = globaltimer_ns();
+        if (progress) {
+          t_last = now;
+        } else if (*abort) {
+          ok = false;
+          break;
+        } else if (now - t_last > wl) {  // nothing became ready within the wait limit
+          set_status(p.status, DECATTN_ETIMEOUT);
+          ok = false;
+          break;
+        }
       }
       if (!ok) *abort = 1;
       // every tensor-core operation of the CTA completes before the memory is freed
@@ -504,15 +542,16 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     auto wait_pv = [&](int64_t gg) -> bool {
       return tc_wait_warp(&bar[kPvDone + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl);
     };
-    // this thread's row of O^T (its head dim), the P parts' 16-column groups added
+    // this thread's row of O^T (its head dim): the P parts' 16-column groups, weighed 1, 1/16, 1/256
     auto o_sum = [&](uint32_t tO, float (&o)[kTcN]) {
       tmem_ld16(tO, o);
       #pragma unroll
       for (int q = 1; q < M::PP; ++q) {
         float t[kTcN];
         tmem_ld16(tO + kTcN * q, t);
+        const float wq = q == 1 ? 0.0625f : 0.00390625f;
         #pragma unroll
-        for (int n = 0; n < kTcN; ++n) o[n] += t[n];
+        for (int n = 0; n < kTcN; ++n) o[n] += wq * t[n];
       }
     };
     Unit d;
@@ -693,7 +732,14 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           lacc[n] += pr[n];
         }
         // ---- P^T row of this key, 16 query rows: x = P * (V page scale) * C rounded to E4M3 parts,
-        //      x = hi + mid + lo (Q8: hi alone), computed before the wait for the buffer
+        //      computed before the wait for the buffer.
+        //      Q8: one part, E4M3(x).
+        //      Otherwise x = hi + mid / 16 + lo / 256: hi is x rounded onto E4M3's grid (4 significant
+        //      bits, steps of 2^-9 below 2^-6) with fp32 multiply and adds, no conversion, so the rest
+        //      x - hi is exact; the rest times 16 gives mid the same way, and the next rest times 16
+        //      is rounded to E4M3 as lo. Each part stays in E4M3's normal range for x >= 2^-6 and lands
+        //      in its own 16-column group of O^T, which the epilogue weighs by 1, 1/16, 1/256: about
+        //      12 significant bits of P.
         const float xs = vsc * c_ref;
         uint32_t w8[M::PP][4];
         #pragma unroll
@@ -701,22 +747,33 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           float x[4] = {pr[4 * i] * xs, pr[4 * i + 1] * xs, pr[4 * i + 2] * xs, pr[4 * i + 3] * xs};
           #pragma unroll
           for (int q = 0; q < M::PP; ++q) {
-            const uint32_t lo = f32x2_to_e4m3x2(x[0], x[1]);
-            const uint32_t hi = f32x2_to_e4m3x2(x[2], x[3]);
-            w8[q][i] = valid ? (lo | (hi << 16)) : 0u;
-            if (Q8 || q + 1 < M::PP) {
-              const float2 a = f16x2_to_float2(e4m3x2_to_f16x2(lo)), b = f16x2_to_float2(e4m3x2_to_f16x2(hi));
-              if constexpr (Q8) {
-                // the output is normalised by the weights as rounded, so it stays a convex
-                // combination of V rows (a single visible key reproduces its V row); lse keeps the
-                // exact sums
-                if (valid) {
-                  const float rxs = 1.f / xs;
-                  lrnd[4 * i] += a.x * rxs; lrnd[4 * i + 1] += a.y * rxs;
-                  lrnd[4 * i + 2] += b.x * rxs; lrnd[4 * i + 3] += b.y * rxs;
-                }
+            float y[4];
+            #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              if (Q8 || q + 1 == M::PP) {
+                y[e] = x[e];
               } else {
-                x[0] -= a.x; x[1] -= a.y; x[2] -= b.x; x[3] -= b.y;  // exact: the next part rounds the rest
+                // (the _rn forms keep each operation rounded on its own: no fused multiply-add)
+                const float c = __fmul_rn(x[e], 1048577.f);                // 2^20 + 1
+                const float yn = __fsub_rn(c, __fsub_rn(c, x[e]));         // 4 significant bits
+                const float t = __fadd_rn(x[e], 24576.f);                  // 1.5 * 2^14: fp32 steps of 2^-9
+                const float ys = __fsub_rn(t, 24576.f);                    // a multiple of 2^-9
+                y[e] = fabsf(x[e]) < 0.015625f ? ys : yn;                  // E4M3's grid at x
+                x[e] = __fsub_rn(x[e], y[e]) * 16.f;                       // both exact
+              }
+            }
+            const uint32_t lo = f32x2_to_e4m3x2(y[0], y[1]);
+            const uint32_t hi = f32x2_to_e4m3x2(y[2], y[3]);
+            w8[q][i] = valid ? (lo | (hi << 16)) : 0u;
+            if constexpr (Q8) {
+              // the output is normalised by the weights as rounded, so it stays a convex
+              // combination of V rows (a single visible key reproduces its V row); lse keeps the
+              // exact sums
+              if (valid) {
+                const float2 a = f16x2_to_float2(e4m3x2_to_f16x2(lo)), b = f16x2_to_float2(e4m3x2_to_f16x2(hi));
+                const float rxs = 1.f / xs;
+                lrnd[4 * i] += a.x * rxs; lrnd[4 * i + 1] += a.y * rxs;
+                lrnd[4 * i + 2] += b.x * rxs; lrnd[4 * i + 3] += b.y * rxs;
               }
             }
           }
