@@ -21,8 +21,8 @@
 //    then an online softmax in
 //    fp32 (log2 domain), then O^T += V^T P^T (again keys as the contraction, head_dim on
 //    M). Probabilities go to the MMA as bf16 hi + bf16 lo (BF16 KV: two columns of the
-//    same MMA when G*T <= 4, two N tiles otherwise), or as f16 scaled by the page's V
-//    scale (FP8 KV).
+//    same MMA when G*T <= 4, two N tiles otherwise), or as f16 hi + lo scaled by the page's V
+//    scale (FP8 KV, two N tiles).
 //  * FP8 KV: S^T runs on E4M3 MMAs straight from the staged codes (K is never widened);
 //    V is widened to f16. With one consumer warp it is widened in registers; with several,
 //    each widens its share of every V block into a shared f16 block (laid out like a bf16
@@ -517,7 +517,7 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
       if (__any_sync(0xffffffffu, grew)) {
         #pragma unroll
         for (int j = 0; j < NPVW; ++j) {
-          const int nw = (KVT == 0 && !DUP) ? j / 2 : j;
+          const int nw = DUP ? j : j / 2;
           #pragma unroll
           for (int mt = 0; mt < D / 16; ++mt) {
             o[j][mt][0] *= alpha[nw][0]; o[j][mt][1] *= alpha[nw][1];
@@ -530,8 +530,15 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
       #pragma unroll
       for (int nw = 0; nw < NQW; ++nw) {
         if (KVT == 1) {
-          bp[nw][0] = movmatrix_t(pack_f16(pv[nw][0] * vsc, pv[nw][1] * vsc));
-          bp[nw][1] = movmatrix_t(pack_f16(pv[nw][2] * vsc, pv[nw][3] * vsc));
+          // f16 hi + lo of P * (V page scale) * kPScale: about 22 significant bits, so that P's
+          // rounding stays far below the tolerance even for large |v| (f16 alone: 2^-11 |v|)
+          const float x0 = pv[nw][0] * vsc, x1 = pv[nw][1] * vsc, x2 = pv[nw][2] * vsc, x3 = pv[nw][3] * vsc;
+          const uint32_t h01 = pack_f16(x0, x1), h23 = pack_f16(x2, x3);
+          const float2 f01 = f16x2_to_float2(h01), f23 = f16x2_to_float2(h23);
+          bp[2 * nw][0] = movmatrix_t(h01);
+          bp[2 * nw][1] = movmatrix_t(h23);
+          bp[2 * nw + 1][0] = movmatrix_t(pack_f16(x0 - f01.x, x1 - f01.y));
+          bp[2 * nw + 1][1] = movmatrix_t(pack_f16(x2 - f23.x, x3 - f23.y));
         } else {
           const uint32_t h01 = pack_bf16(pv[nw][0], pv[nw][1]);
           const uint32_t h23 = pack_bf16(pv[nw][2], pv[nw][3]);
@@ -620,24 +627,22 @@ split_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, const
         l += __shfl_xor_sync(0xffffffffu, l, 16);
         lrow[nw][e] = l;
       }
-    if (KVT == 0) {
-      if (DUP) {
+    if (DUP) {
+      #pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt)
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) o[0][mt][i] += __shfl_xor_sync(0xffffffffu, o[0][mt][i], 2);
+    } else {  // the products of P's hi and lo halves
+      #pragma unroll
+      for (int nw = 0; nw < NQW; ++nw)
         #pragma unroll
         for (int mt = 0; mt < D / 16; ++mt)
           #pragma unroll
-          for (int i = 0; i < 4; ++i) o[0][mt][i] += __shfl_xor_sync(0xffffffffu, o[0][mt][i], 2);
-      } else {
-        #pragma unroll
-        for (int nw = 0; nw < NQW; ++nw)
-          #pragma unroll
-          for (int mt = 0; mt < D / 16; ++mt)
-            #pragma unroll
-            for (int i = 0; i < 4; ++i) o[2 * nw][mt][i] += o[2 * nw + 1][mt][i];
-      }
+          for (int i = 0; i < 4; ++i) o[2 * nw][mt][i] += o[2 * nw + 1][mt][i];
     }
     #pragma unroll
     for (int nw = 0; nw < NQW; ++nw) {
-      const int j = (KVT == 0 && !DUP) ? 2 * nw : nw;
+      const int j = DUP ? nw : 2 * nw;
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int n = 8 * (nq0 + nw) + 2 * tig + e;
@@ -714,10 +719,10 @@ static cudaError_t launch_gt(const SplitParams& p, const CUtensorMap& tmK, const
     if (p.GT <= 32) return launch_variant<KVT, D, 4, 8, false, 4>(p, tmK, tmV, st);
     return launch_variant<KVT, D, 8, 16, false, 8>(p, tmK, tmV, st);
   } else {
-    if (p.GT <= 8) return launch_variant<KVT, D, 1, 1, false, 1>(p, tmK, tmV, st);
-    if (p.GT <= 16) return launch_variant<KVT, D, 2, 2, false, 2>(p, tmK, tmV, st);
-    if (p.GT <= 32) return launch_variant<KVT, D, 4, 4, false, 4>(p, tmK, tmV, st);
-    return launch_variant<KVT, D, 8, 8, false, 8>(p, tmK, tmV, st);
+    if (p.GT <= 8) return launch_variant<KVT, D, 1, 2, false, 1>(p, tmK, tmV, st);
+    if (p.GT <= 16) return launch_variant<KVT, D, 2, 4, false, 2>(p, tmK, tmV, st);
+    if (p.GT <= 32) return launch_variant<KVT, D, 4, 8, false, 4>(p, tmK, tmV, st);
+    return launch_variant<KVT, D, 8, 16, false, 8>(p, tmK, tmV, st);
   }
 }
 
