@@ -191,3 +191,15 @@ def test_repeated_runs_on_one_workspace_and_stage_calls():
     assert torch.equal(out, o1) and torch.equal(lse, l1)
     ref_o, ref_l = oracle.decode(pr)
     U.check_rows(o1.cpu().numpy(), l1.cpu().numpy(), ref_o, ref_l, "repeated")
+
+
+@pytest.mark.parametrize("d,G,T", [(64, 4, 1), (64, 4, 4), (64, 8, 4), (64, 8, 8), (128, 4, 4), (128, 8, 4), (128, 16, 4)])
+def test_fp8_large_values(d, G, T):
+    # V pages scaled by 12 and K pages by 3 (peakier softmax, |v| up to about 55): the absolute 2e-3
+    # must still hold, which needs P well beyond f16's 11 bits (every FP8 kernel variant)
+    pr = small(LENS, Hq=2 * G, Hkv=2, d=d, T=T, kv="fp8e4m3", seed=G + T + d)
+    sc = pr.kv_scales.copy()
+    sc[0] *= 3.0
+    sc[1] *= 12.0
+    pr.kv_scales = sc
+    check_all(pr)
