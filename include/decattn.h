@@ -126,8 +126,8 @@ DECATTN_API int dec_attn_default_bins(int device);
  * over n_bins bins, the estimate is
  *   ceil(U / n_bins) * (tl * 2 * head_dim * elem + 8192) + U * rows * (head_dim + 1) * 8 / n_bins
  * (elem = 2 for bf16, 1 for E4M3; rows = G * T query rows per KV head; 8192 = the fixed cost of a
- * tile in KV bytes). A candidate with U >= n_bins is preferred, then the smallest estimate, then
- * the shorter tile. Host only (no CUDA call): n_bins > 0 must be given, e.g.
+ * tile in KV bytes). The smallest estimate wins, the shorter tile on a tie. Host only (no CUDA
+ * call): n_bins > 0 must be given, e.g.
  * dec_attn_default_bins(device). Returns the tile length (a multiple of page_size and of 16), or
  * DECATTN_EINVAL for invalid arguments. */
 DECATTN_API int dec_attn_default_tile_len(int batch, int n_kv_heads, int64_t total_kv_tokens, int page_size,

@@ -341,21 +341,16 @@ extern "C" int dec_attn_default_tile_len(int batch, int n_kv_heads, int64_t tota
   const double tile_cost = 8192.0;  // fixed cost of a tile (q, epilogue, pipeline start) in KV-byte terms
   int best = 0;
   double best_est = 0.0;
-  bool best_fills = false;  // the candidate gives every bin a tile
   for (int tl = page_size; tl <= 8192; tl *= 2) {
     const double U = W / tl;  // tiles, as if every tile were full
-    const bool fills = U >= N;
     const double per_bin = U > 0 ? ceil(U / N) : 0.0;
     // the busiest bin's KV bytes and tile overheads, plus the partials every tile writes and the
     // combine reads back (fp32 o and lse per query row), spread over the bins
     const double est = per_bin * (tl * 2.0 * head_dim * elem + tile_cost) +
                        U * rows_per_kv_head * (head_dim + 1.0) * 8.0 / N;
-    // a candidate that fills every bin beats one that does not; then the smaller estimate, then
-    // the shorter tile
-    if (best == 0 || (fills && !best_fills) || (fills == best_fills && est < best_est)) {
+    if (best == 0 || est < best_est) {  // the smaller estimate; on a tie the shorter tile
       best = tl;
       best_est = est;
-      best_fills = fills;
     }
   }
   return best;

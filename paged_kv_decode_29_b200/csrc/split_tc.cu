@@ -400,6 +400,9 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       // N = the P parts' columns
       constexpr uint32_t idS = umma_idesc(0, 0, 0, 0, kTcChunk, M::NS);
       constexpr uint32_t idO = umma_idesc(0, 0, 1, 1, kTcD, M::NO);
+      int us = 0; uint32_t uph = 0;
+      int64_t g = 0;  // chunks issued so far
+      int ut = 0;     // tiles started so far
       bool ok = true;
       // descriptors, built once: the start address is the low 14 bits (16-byte units), so a
       // stage or a k-step adds to the base descriptor.
@@ -413,89 +416,49 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       const uint64_t dV = umma_desc(base + L::OFF_V, 1024, 1024, 2);
       const uint64_t dP = umma_desc(base + L::OFF_P, 128, L::PPLANE, 0);
       const uint32_t tO = tmem + 2 * M::NS;
-      // Two cursors, each taking its barriers' phases in order, issued in whichever order they
-      // become ready, so that neither waits for the other's operands:
-      //  * S^T of chunk gs (global chunk count) once its K has landed and the softmax group has read
-      //    the S^T buffer's previous contents; a new tile first needs its descriptor and its q;
-      //  * O^T (+)= V^T P^T of chunk gp once the softmax group has written its P^T. A tile's first
-      //    chunk overwrites O^T: the softmax group signals that chunk's P only after it has read the
-      //    previous tile's O^T.
-      int us = 0; uint32_t uph = 0;  // tile descriptor slot
-      int64_t gs = 0, gp = 0;        // next chunk for S^T / for P V
-      int ts = -1;                   // tiles opened by the S cursor, minus 1
-      int cs = 0, ncs = 0;           // the S cursor's chunk within its tile, and that tile's chunks
-      bool need_q = false;           // the S cursor's tile still waits for its q
-      bool done = false;             // the end-of-work descriptor has been read
-      int tp = 0, cp = 0;            // the P V cursor's tile and chunk within it
-      int nc_of[2] = {0, 0};         // chunks of the tiles opened, by tile parity
-      uint64_t dQ = dQ0;
-      uint64_t t_last = globaltimer_ns();
+      // O^T (+)= V^T P^T over chunk gg's 128 keys. A tile's first chunk overwrites O^T: the
+      // softmax group signals that chunk's P only after it has read the previous tile's O^T.
+      auto pv = [&](int64_t gg, bool first_of_tile) -> bool {
+        if (!tc_wait(&bar[kPReady + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl)) return false;
+        tc_fence_after();
+        const int sg = (int)(gg % kTcStages);
+        const uint64_t a0 = dV + (uint64_t)((sg * L::KCH) >> 4);
+        const uint64_t b0 = dP + (uint64_t)((((int)(gg & (M::NPB - 1))) * L::PB) >> 4);
+        #pragma unroll
+        for (int k = 0; k < kTcChunk / 32; ++k)  // 32 keys per instruction: 4 KB of V, 512 B per P part
+          umma_f8(tO, a0 + (uint64_t)(256 * k), b0 + (uint64_t)(32 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
+        umma_commit(&bar[kPvDone + (gg & 1)]);
+        umma_commit(&bar[kKvEmpty + sg]);  // K and V of the stage have both been read
+        return true;
+      };
       for (;;) {
-        bool progress = false;
-        // open the next tile for S^T (at most one tile ahead of the P V cursor: two q buffers)
-        if (!done && cs == ncs && ts + 1 - tp < 2 && mbar_test(&bar[kUFull + us], uph)) {
-          const Unit d = umeta[us];
-          mbar_arrive(&bar[kUEmpty + us]);
-          us ^= 1; if (us == 0) uph ^= 1;
-          if (d.b < 0) {
-            done = true;
-          } else {
-            ++ts;
-            cs = 0;
-            ncs = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
-            nc_of[ts & 1] = ncs;
-            need_q = true;
+        if (!tc_wait(&bar[kUFull + us], uph, p.status, abort, wl)) { ok = false; break; }
+        const Unit d = umeta[us];
+        mbar_arrive(&bar[kUEmpty + us]);
+        us ^= 1; if (us == 0) uph ^= 1;
+        if (d.b < 0) break;
+        const int nc = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
+        if (!tc_wait(&bar[kQReady], (uint32_t)(ut & 1), p.status, abort, wl)) { ok = false; break; }
+        const uint64_t dQ = dQ0 + (uint64_t)(((ut & 1) * L::QB) >> 4);
+        for (int c = 0; c < nc; ++c, ++g) {
+          const int st = (int)(g % kTcStages), sb = (int)(g & 1);
+          if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl) ||
+              !tc_wait(&bar[kSFree + sb], (uint32_t)(((g >> 1) & 1) ^ 1), p.status, abort, wl)) {
+            ok = false;
+            break;
           }
-          progress = true;
-        }
-        if (need_q && mbar_test(&bar[kQReady], (uint32_t)(ts & 1))) {
-          need_q = false;
-          dQ = dQ0 + (uint64_t)(((ts & 1) * L::QB) >> 4);
-          progress = true;
-        }
-        if (!need_q && cs < ncs) {
-          const int st = (int)(gs % kTcStages), sb = (int)(gs & 1);
-          if (mbar_test(&bar[kKvFull + st], (uint32_t)((gs / kTcStages) & 1)) &&
-              mbar_test(&bar[kSFree + sb], (uint32_t)(((gs >> 1) & 1) ^ 1))) {
-            tc_fence_after();
-            // S^T = K (q parts)^T: four 32-byte k-steps of the 128-byte swizzled rows
-            const uint64_t dK = dK0 + (uint64_t)((st * L::KCH) >> 4);
-            #pragma unroll
-            for (int kk = 0; kk < kTcD / 32; ++kk)
-              umma_f8(tmem + M::NS * sb, dK + (uint64_t)(2 * kk), dQ + (uint64_t)(2 * kk), idS, kk > 0 ? 1u : 0u);
-            umma_commit(&bar[kSFull + sb]);
-            ++cs;
-            ++gs;
-            progress = true;
-          }
-        }
-        if (gp < gs && mbar_test(&bar[kPReady + (gp & 1)], (uint32_t)((gp >> 1) & 1))) {
           tc_fence_after();
-          const int sg = (int)(gp % kTcStages);
-          const uint64_t a0 = dV + (uint64_t)((sg * L::KCH) >> 4);
-          const uint64_t b0 = dP + (uint64_t)((((int)(gp & (M::NPB - 1))) * L::PB) >> 4);
-          const bool first_of_tile = cp == 0;
+          // S^T = K (q parts)^T: four 32-byte k-steps of the 128-byte swizzled rows
+          const uint64_t dK = dK0 + (uint64_t)((st * L::KCH) >> 4);
           #pragma unroll
-          for (int k = 0; k < kTcChunk / 32; ++k)  // 32 keys per instruction: 4 KB of V, 512 B per P part
-            umma_f8(tO, a0 + (uint64_t)(256 * k), b0 + (uint64_t)(32 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
-          umma_commit(&bar[kPvDone + (gp & 1)]);
-          umma_commit(&bar[kKvEmpty + sg]);  // K and V of the stage have both been read
-          ++gp;
-          if (++cp == nc_of[tp & 1]) { ++tp; cp = 0; }
-          progress = true;
+          for (int kk = 0; kk < kTcD / 32; ++kk)
+            umma_f8(tmem + M::NS * sb, dK + (uint64_t)(2 * kk), dQ + (uint64_t)(2 * kk), idS, kk > 0 ? 1u : 0u);
+          umma_commit(&bar[kSFull + sb]);
+          if (c > 0 && !pv(g - 1, c == 1)) { ok = false; break; }
         }
-        if (done && cs == ncs && gp == gs) break;  // every chunk's products issued
-        const uint64_t now = globaltimer_ns();
-        if (progress) {
-          t_last = now;
-        } else if (*abort) {
-          ok = false;
-          break;
-        } else if (now - t_last > wl) {  // nothing became ready within the wait limit
-          set_status(p.status, DECATTN_ETIMEOUT);
-          ok = false;
-          break;
-        }
+        if (!ok) break;
+        if (!pv(g - 1, nc == 1)) { ok = false; break; }
+        ++ut;
       }
       if (!ok) *abort = 1;
       // every tensor-core operation of the CTA completes before the memory is freed
@@ -732,14 +695,10 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           lacc[n] += pr[n];
         }
         // ---- P^T row of this key, 16 query rows: x = P * (V page scale) * C rounded to E4M3 parts,
-        //      computed before the wait for the buffer.
-        //      Q8: one part, E4M3(x).
-        //      Otherwise x = hi + mid / 16 + lo / 256: hi is x rounded onto E4M3's grid (4 significant
-        //      bits, steps of 2^-9 below 2^-6) with fp32 multiply and adds, no conversion, so the rest
-        //      x - hi is exact; the rest times 16 gives mid the same way, and the next rest times 16
-        //      is rounded to E4M3 as lo. Each part stays in E4M3's normal range for x >= 2^-6 and lands
-        //      in its own 16-column group of O^T, which the epilogue weighs by 1, 1/16, 1/256: about
-        //      12 significant bits of P.
+        //      computed before the wait for the buffer. Q8: hi = E4M3(x) alone. Otherwise
+        //      x = hi + mid / 16 + lo / 256: each rest (x minus the parts so far, exact in fp32) is
+        //      scaled by 16 before it is rounded, so that the parts stay in E4M3's normal range for
+        //      x >= 2^-6; the epilogue weighs the parts' O^T column groups by 1, 1/16, 1/256
         const float xs = vsc * c_ref;
         uint32_t w8[M::PP][4];
         #pragma unroll
@@ -747,33 +706,23 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           float x[4] = {pr[4 * i] * xs, pr[4 * i + 1] * xs, pr[4 * i + 2] * xs, pr[4 * i + 3] * xs};
           #pragma unroll
           for (int q = 0; q < M::PP; ++q) {
-            float y[4];
-            #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              if (Q8 || q + 1 == M::PP) {
-                y[e] = x[e];
-              } else {
-                // (the _rn forms keep each operation rounded on its own: no fused multiply-add)
-                const float c = __fmul_rn(x[e], 1048577.f);                // 2^20 + 1
-                const float yn = __fsub_rn(c, __fsub_rn(c, x[e]));         // 4 significant bits
-                const float t = __fadd_rn(x[e], 24576.f);                  // 1.5 * 2^14: fp32 steps of 2^-9
-                const float ys = __fsub_rn(t, 24576.f);                    // a multiple of 2^-9
-                y[e] = fabsf(x[e]) < 0.015625f ? ys : yn;                  // E4M3's grid at x
-                x[e] = __fsub_rn(x[e], y[e]) * 16.f;                       // both exact
-              }
-            }
-            const uint32_t lo = f32x2_to_e4m3x2(y[0], y[1]);
-            const uint32_t hi = f32x2_to_e4m3x2(y[2], y[3]);
+            const uint32_t lo = f32x2_to_e4m3x2(x[0], x[1]);
+            const uint32_t hi = f32x2_to_e4m3x2(x[2], x[3]);
             w8[q][i] = valid ? (lo | (hi << 16)) : 0u;
-            if constexpr (Q8) {
-              // the output is normalised by the weights as rounded, so it stays a convex
-              // combination of V rows (a single visible key reproduces its V row); lse keeps the
-              // exact sums
-              if (valid) {
-                const float2 a = f16x2_to_float2(e4m3x2_to_f16x2(lo)), b = f16x2_to_float2(e4m3x2_to_f16x2(hi));
-                const float rxs = 1.f / xs;
-                lrnd[4 * i] += a.x * rxs; lrnd[4 * i + 1] += a.y * rxs;
-                lrnd[4 * i + 2] += b.x * rxs; lrnd[4 * i + 3] += b.y * rxs;
+            if (Q8 || q + 1 < M::PP) {
+              const float2 a = f16x2_to_float2(e4m3x2_to_f16x2(lo)), b = f16x2_to_float2(e4m3x2_to_f16x2(hi));
+              if constexpr (Q8) {
+                // the output is normalised by the weights as rounded, so it stays a convex
+                // combination of V rows (a single visible key reproduces its V row); lse keeps the
+                // exact sums
+                if (valid) {
+                  const float rxs = 1.f / xs;
+                  lrnd[4 * i] += a.x * rxs; lrnd[4 * i + 1] += a.y * rxs;
+                  lrnd[4 * i + 2] += b.x * rxs; lrnd[4 * i + 3] += b.y * rxs;
+                }
+              } else {  // the rest, exact, scaled by 16 (exact)
+                x[0] = (x[0] - a.x) * 16.f; x[1] = (x[1] - a.y) * 16.f;
+                x[2] = (x[2] - b.x) * 16.f; x[3] = (x[3] - b.y) * 16.f;
               }
             }
           }

@@ -5,9 +5,11 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 import paged_kv_decode_29_b200 as da
+import workloads as W
 from paged_kv_decode_29_b200 import build as dbuild
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -240,6 +242,13 @@ def test_default_tile_len_rule(lib):
     assert f(1, 8, 131072, 64, 128, 8, da.KV_BF16, 592) == 256             # long context, one request
     assert f(4, 8, 4 * 131072, 64, 128, 8, da.KV_BF16, 592) == 1024        # long context, four requests
     assert f(2, 1, 317, 16, 64, 4, da.KV_BF16, 592) == 16                  # too small to fill the bins
+    # every workload whose tile length the configs leave open uses the rule's length
+    for name in ("uniform", "long_b1", "long_b4", "fp8_spec"):
+        c = W.CONFIGS[name]
+        L = np.asarray(W.config_seq_lens(name), dtype=np.int64)
+        kv = da.KV_BF16 if c["kv_dtype"] == "bf16" else da.KV_FP8E4M3
+        rows = c["n_q_heads"] // c["n_kv_heads"] * c["q_tokens"]
+        assert f(len(L), c["n_kv_heads"], int(L.sum()), c["page_size"], c["head_dim"], rows, kv, 592) == c["tile_len"], name
     for P in (16, 32, 48, 64, 256):
         tl = f(8, 8, 100000, P, 128, 8, da.KV_BF16, 592)
         assert tl > 0 and tl % P == 0 and tl % 16 == 0
