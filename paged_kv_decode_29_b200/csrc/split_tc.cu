@@ -584,26 +584,45 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         }
         if (!tc_wait_warp(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort, wl)) { ok = false; break; }
         tc_fence_after();
+        // scores times the column factors f * 2^-E, in pairs
         float s[kTcN];
         if constexpr (M::QP == 2) {  // the q hi and lo halves of S^T, added
           float s2[2 * kTcN];
           tmem_ld32(tmem + lane_off + M::NS * sb, s2);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[kSFree + sb]);
           #pragma unroll
-          for (int n = 0; n < kTcN; ++n) s[n] = s2[n] + s2[kTcN + n];
+          for (int q4 = 0; q4 < kTcN / 4; ++q4) {
+            const float4 qc = qcs4[q4];
+            const int n = 4 * q4;
+            float f0, f1, f2, f3;
+            fmul2(f0, f1, qc.x, qc.y, f, f);
+            fmul2(f2, f3, qc.z, qc.w, f, f);
+            fadd2(s[n], s[n + 1], s2[n], s2[n + 1], s2[kTcN + n], s2[kTcN + n + 1]);
+            fadd2(s[n + 2], s[n + 3], s2[n + 2], s2[n + 3], s2[kTcN + n + 2], s2[kTcN + n + 3]);
+            fmul2(s[n], s[n + 1], s[n], s[n + 1], f0, f1);
+            fmul2(s[n + 2], s[n + 3], s[n + 2], s[n + 3], f2, f3);
+          }
         } else {
           tmem_ld16(tmem + lane_off + M::NS * sb, s);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[kSFree + sb]);
+          #pragma unroll
+          for (int q4 = 0; q4 < kTcN / 4; ++q4) {
+            const float4 qc = qcs4[q4];
+            const int n = 4 * q4;
+            float f0, f1, f2, f3;
+            fmul2(f0, f1, qc.x, qc.y, f, f);
+            fmul2(f2, f3, qc.z, qc.w, f, f);
+            fmul2(s[n], s[n + 1], s[n], s[n + 1], f0, f1);
+            fmul2(s[n + 2], s[n + 3], s[n + 2], s[n + 3], f2, f3);
+          }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[kSFree + sb]);
 
-        // ---- scale, mask; per-column maxima of the chunk
+        // ---- mask; per-column maxima of the chunk
         int* rw = red + ((sb * 4 + warp) * kTcN);
-        #pragma unroll
-        for (int q4 = 0; q4 < kTcN / 4; ++q4) {
-          const float4 qc = qcs4[q4];
-          s[4 * q4] *= f * qc.x; s[4 * q4 + 1] *= f * qc.y; s[4 * q4 + 2] *= f * qc.z; s[4 * q4 + 3] *= f * qc.w;
-        }
         const int over = j - causal_base;  // > 0 only for the last T - 1 keys of the request
         if (!valid) {
           #pragma unroll
@@ -690,9 +709,12 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         // ---- P = 2^(s - m_ref) (at most 2^kTcTau); row sums in fp32
         float (&pr)[kTcN] = s;  // in place
         #pragma unroll
-        for (int n = 0; n < kTcN; ++n) {
-          pr[n] = fast_exp2(s[n] - (mref[n] == -INFINITY ? 0.f : mref[n]));
-          lacc[n] += pr[n];
+        for (int n = 0; n < kTcN; n += 2) {
+          float d0, d1;
+          fadd2(d0, d1, s[n], s[n + 1], mref[n] == -INFINITY ? 0.f : -mref[n], mref[n + 1] == -INFINITY ? 0.f : -mref[n + 1]);
+          pr[n] = fast_exp2(d0);
+          pr[n + 1] = fast_exp2(d1);
+          fadd2(lacc[n], lacc[n + 1], lacc[n], lacc[n + 1], pr[n], pr[n + 1]);
         }
         // ---- P^T row of this key, 16 query rows: x = P * (V page scale) * C rounded to E4M3 parts,
         //      computed before the wait for the buffer. Q8: hi = E4M3(x) alone. Otherwise
@@ -703,7 +725,9 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         uint32_t w8[M::PP][4];
         #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          float x[4] = {pr[4 * i] * xs, pr[4 * i + 1] * xs, pr[4 * i + 2] * xs, pr[4 * i + 3] * xs};
+          float x[4];
+          fmul2(x[0], x[1], pr[4 * i], pr[4 * i + 1], xs, xs);
+          fmul2(x[2], x[3], pr[4 * i + 2], pr[4 * i + 3], xs, xs);
           #pragma unroll
           for (int q = 0; q < M::PP; ++q) {
             const uint32_t lo = f32x2_to_e4m3x2(x[0], x[1]);
@@ -720,9 +744,9 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
                   lrnd[4 * i] += a.x * rxs; lrnd[4 * i + 1] += a.y * rxs;
                   lrnd[4 * i + 2] += b.x * rxs; lrnd[4 * i + 3] += b.y * rxs;
                 }
-              } else {  // the rest, exact, scaled by 16 (exact)
-                x[0] = (x[0] - a.x) * 16.f; x[1] = (x[1] - a.y) * 16.f;
-                x[2] = (x[2] - b.x) * 16.f; x[3] = (x[3] - b.y) * 16.f;
+              } else {  // the rest times 16: 16 x - 16 part, one rounding of an exact result
+                ffma2(x[0], x[1], x[0], x[1], 16.f, 16.f, -16.f * a.x, -16.f * a.y);
+                ffma2(x[2], x[3], x[2], x[3], 16.f, 16.f, -16.f * b.x, -16.f * b.y);
               }
             }
           }
