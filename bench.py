@@ -137,12 +137,13 @@ def split_kernel_name(pr) -> str:
 # the ratio of algorithmic bytes (reads measured within 0.05% of the algorithmic bytes on every
 # captured case, so traffic grows in proportion): workload -> (requests captured, read, write).
 SPLIT_TRAFFIC_CAPTURED = {
-    "source_hash": "2cd4dd2d54b1c127",  # kernel_source_hash() of the sources these were captured on
+    "source_hash": "72bcac3874b68c0f",  # kernel_source_hash() of the sources these were captured on
     "configs": {
-        "uniform": (8, 134362368, 3598080),
-        "mixed": (16, 1039144960, 17676288),
-        "fp8_spec": (4, 167250432, 6338304),
-        "long_b4": (1, 536982272, 5664256),
+        "uniform": (8, 134362624, 3202816),
+        "mixed": (16, 1039146752, 17593088),
+        "fp8_spec": (4, 167686400, 4259072),
+        "long_b4": (1, 536969728, 5669632),
+        "long_b1": (1, 536979200, 15681280),
     },
 }
 # prefill_kernel on the full prefill workload (read, write): a few hundred MB on the device.
