@@ -147,7 +147,7 @@ SPLIT_TRAFFIC_CAPTURED = {
     },
 }
 # prefill_kernel on the full prefill workload (read, write): a few hundred MB on the device.
-PREFILL_TRAFFIC_CAPTURED = {"source_hash": "22fe69057deeaf7e", "read": 108316928, "write": 87724800}
+PREFILL_TRAFFIC_CAPTURED = {"source_hash": "1ae2fe489d1ff892", "read": 108431616, "write": 85455104}
 
 
 def config_algorithmic_bytes(name: str, batch: int | None = None) -> int:
