@@ -61,7 +61,6 @@ struct TcMode {
   static constexpr int PP = Q8 ? 1 : 3;            // E4M3 parts of P
   static constexpr int NS = QP * kTcN;             // S^T columns (per q part, 16 query rows)
   static constexpr int NO = PP * kTcN;             // O^T columns (per P part, 16 query rows)
-  static constexpr int NPB = Q8 ? 2 : 1;           // P^T buffers (Q8: one per chunk parity)
   static constexpr int TMEM = Q8 ? 64 : 128;       // columns: S^T double buffer + O^T, a power of 2
   static_assert(2 * NS + NO <= TMEM, "tensor-memory columns");
 };
@@ -75,11 +74,13 @@ struct TcSmem {
   static constexpr int QB = M::QP * kTcN * kTcD;             // q parts [part][16][128], E4M3
   static constexpr int PPLANE = kTcChunk * kTcN;             // one E4M3 part of P^T: 2 KB
   static constexpr int PB = M::PP * PPLANE;                  // P^T of one chunk: [part][128 keys][16]
+  // A chunk's P^T is written over its own K (MN-major interleaved, from the stage's start): the
+  // softmax group writes it only after S^T of the chunk, the last reader of that K, is complete,
+  // and the stage is refilled only after the chunk's P V.
   static constexpr int OFF_K = 0;                            // [stage][128 keys][128 B], 128-B swizzle
   static constexpr int OFF_V = OFF_K + STAGES * KCH;
   static constexpr int OFF_QB = OFF_V + STAGES * KCH;        // [tile parity] q parts, 128-B swizzle
-  static constexpr int OFF_P = OFF_QB + 2 * QB;              // [NPB] P^T, MN-major interleaved
-  static constexpr int OFF_SC = OFF_P + M::NPB * PB;         // per stage: 8 K scales, 8 V scales
+  static constexpr int OFF_SC = OFF_QB + 2 * QB;             // per stage: 8 K scales, 8 V scales
   static constexpr int OFF_QCS = OFF_SC + STAGES * 2 * kTcBlk * 4;  // [tile parity][16]: 2^-E of q rows
   static constexpr int OFF_FLG = OFF_QCS + 2 * kTcN * 4;     // [2][4] per-warp "passes the reference" flags
   static constexpr int OFF_RED = OFF_FLG + 2 * 4 * 4;        // [2][4][16] chunk maxima per warp
@@ -92,13 +93,15 @@ struct TcSmem {
   static constexpr int ALLOC = BYTES + 1024;                 // slack to align the base to 1024
   static_assert(OFF_QB % 1024 == 0 && QB % 1024 == 0, "swizzled q operands need 1024-byte bases");
   static_assert(OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
+  static_assert(PB <= KCH, "P^T fits in the K of its stage");
   static_assert(2 * (ALLOC + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
 // Barrier slots. The P / P V hand-off has one barrier per chunk parity: chunk g (counted over all
 // tiles of the CTA) signals kPReady + (g & 1) and its P V completes kPvDone + (g & 1), phase
-// (g >> 1) & 1, so that the softmax group can compute chunk g + 1's P while chunk g's P V runs
-// (Q8: and write it, into the other P^T buffer) without ever running two phases ahead of a waiter.
+// (g >> 1) & 1, so that the softmax group can compute and write chunk g + 1's P while chunk g's
+// P V runs without ever running two phases ahead of a waiter (the MMA warp issues S^T of chunk
+// g + 2 only after it has taken chunk g + 1's P).
 enum TcBar {
   kKvFull = 0,   // [stages] producer -> MMA, softmax: K, V and scales of a chunk landed
   kKvEmpty = 3,  // [stages] the stage may be refilled: the MMA commit after the chunk's P V
@@ -410,11 +413,12 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       //    parts are consecutive 16-row blocks, so N = 32 spans hi then lo.
       //  V^T: the staged V (E4M3, MN-major: head dims contiguous, 128-byte swizzle; 8-key groups
       //    1024 B apart, a 32-key k-step is 4 KB).
-      //  P^T: MN-major interleaved, key j of part q at q * 2 KB + 16 j: 8-key groups 128 B apart
-      //    (leading offset), the next 16 columns (the next part) 2 KB on (stride offset).
+      //  P^T: over the K of the chunk's stage, MN-major interleaved, key j of part q at
+      //    q * 2 KB + 16 j: 8-key groups 128 B apart (leading offset), the next 16 columns (the
+      //    next part) 2 KB on (stride offset).
       const uint64_t dK0 = umma_desc(base + L::OFF_K, 16, 1024, 2), dQ0 = umma_desc(base + L::OFF_QB, 16, 1024, 2);
       const uint64_t dV = umma_desc(base + L::OFF_V, 1024, 1024, 2);
-      const uint64_t dP = umma_desc(base + L::OFF_P, 128, L::PPLANE, 0);
+      const uint64_t dP = umma_desc(base + L::OFF_K, 128, L::PPLANE, 0);
       const uint32_t tO = tmem + 2 * M::NS;
       // O^T (+)= V^T P^T over chunk gg's 128 keys. A tile's first chunk overwrites O^T: the
       // softmax group signals that chunk's P only after it has read the previous tile's O^T.
@@ -423,7 +427,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         tc_fence_after();
         const int sg = (int)(gg % kTcStages);
         const uint64_t a0 = dV + (uint64_t)((sg * L::KCH) >> 4);
-        const uint64_t b0 = dP + (uint64_t)((((int)(gg & (M::NPB - 1))) * L::PB) >> 4);
+        const uint64_t b0 = dP + (uint64_t)((sg * L::KCH) >> 4);
         #pragma unroll
         for (int k = 0; k < kTcChunk / 32; ++k)  // 32 keys per instruction: 4 KB of V, 512 B per P part
           umma_f8(tO, a0 + (uint64_t)(256 * k), b0 + (uint64_t)(32 * k), idO, (first_of_tile && k == 0) ? 0u : 1u);
@@ -751,11 +755,9 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
             }
           }
         }
-        // the P^T buffer: Q8 writes buffer g & 1, which chunk g - 2's P V read; otherwise the single
-        // buffer, once the previous chunk's P V has read it (a tile's first chunk: the previous
-        // tile's epilogue waited for its last P V)
-        if (M::NPB == 2 ? (g >= 2 && !wait_pv(g - 2)) : (c > 0 && !wait_pv(g - 1))) { ok = false; break; }
-        uint8_t* pbuf = sm + L::OFF_P + (int)(g & (M::NPB - 1)) * L::PB;
+        // P^T over the chunk's K: S^T of the chunk (complete, its barrier was waited on above) was
+        // that K's last reader
+        uint8_t* pbuf = sm + L::OFF_K + st * L::KCH;
         #pragma unroll
         for (int q = 0; q < M::PP; ++q)
           *reinterpret_cast<uint4*>(pbuf + q * L::PPLANE + key * kTcN) =
