@@ -82,12 +82,12 @@ struct TcSmem {
   static constexpr int OFF_QB = OFF_V + STAGES * KCH;        // [tile parity] q parts, 128-B swizzle
   static constexpr int OFF_SC = OFF_QB + 2 * QB;             // per stage: 8 K scales, 8 V scales
   static constexpr int OFF_QCS = OFF_SC + STAGES * 2 * kTcBlk * 4;  // [tile parity][16]: 2^-E of q rows
-  static constexpr int OFF_FLG = OFF_QCS + 2 * kTcN * 4;     // [2][4] per-warp "passes the reference" flags
-  static constexpr int OFF_RED = OFF_FLG + 2 * 4 * 4;        // [2][4][16] chunk maxima per warp
+  static constexpr int OFF_FLG = OFF_QCS + 2 * kTcN * 4;     // [2][8] per warp: "passes the reference" flag, then largest V scale
+  static constexpr int OFF_RED = OFF_FLG + 2 * 8 * 4;        // [2][4][16] chunk maxima per warp
   static constexpr int OFF_ERED = OFF_RED + 2 * 4 * kTcN * 4;  // [2][4][16] row-sum partials (Q8: exact, rounded)
   static constexpr int OFF_UNIT = OFF_ERED + 2 * 4 * kTcN * 4;  // Unit x 2
   static constexpr int OFF_BAR = OFF_UNIT + 2 * (int)sizeof(Unit);
-  static constexpr int NBAR = 21;
+  static constexpr int NBAR = 18;
   static constexpr int OFF_MISC = OFF_BAR + 8 * NBAR;        // tensor-memory base, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;                 // slack to align the base to 1024
@@ -102,19 +102,22 @@ struct TcSmem {
 // (g >> 1) & 1, so that the softmax group can compute and write chunk g + 1's P while chunk g's
 // P V runs without ever running two phases ahead of a waiter (the MMA warp issues S^T of chunk
 // g + 2 only after it has taken chunk g + 1's P).
+// S^T has two tensor-memory buffers (chunk parity) and no "buffer read" barrier: S^T of chunk g + 2
+// goes into chunk g's buffer, and the MMA warp issues it only after it has taken chunk g's P (and
+// chunk g + 1's), which the softmax group signals after its last read of chunk g's S^T.
 enum TcBar {
   kKvFull = 0,   // [stages] producer -> MMA, softmax: K, V and scales of a chunk landed
   kKvEmpty = 3,  // [stages] the stage may be refilled: the MMA commit after the chunk's P V
   kSFull = 6,    // [2] MMA commit -> softmax: S^T of a chunk is in tensor memory
-  kSFree = 8,    // [2] 4 softmax warps -> MMA: that S^T buffer has been read
-  kPReady = 10,  // [chunk parity] 4 softmax warps -> MMA: P^T written, O^T rescaled
-  kPvDone = 12,  // [chunk parity] MMA commit -> softmax: O^T += V^T P^T of a chunk complete
-  kUFull = 14,   // [2] producer -> MMA, softmax: tile descriptor written
-  kUEmpty = 16,  // [2] MMA + 4 softmax warps -> producer: tile descriptor read
-  kQReady = 18,  // 4 softmax warps -> MMA: q hi / lo of the next tile written
-  kGroup = 19,   // 4 softmax warps: the group's own barrier (bounded, unlike bar.sync)
-  kFin = 20,     // MMA commit -> MMA: every tensor-core operation of the CTA complete
+  kPReady = 8,   // [chunk parity] 4 softmax warps -> MMA: P^T written, O^T rescaled
+  kPvDone = 10,  // [chunk parity] MMA commit -> softmax: O^T += V^T P^T of a chunk complete
+  kUFull = 12,   // [2] producer -> MMA, softmax: tile descriptor written
+  kUEmpty = 14,  // [2] MMA + 4 softmax warps -> producer: tile descriptor read
+  kQReady = 16,  // 4 softmax warps -> MMA: q hi / lo of the next tile written
+  kFin = 17,     // MMA commit -> MMA: every tensor-core operation of the CTA complete
 };
+// The softmax group's own barrier: named barrier 1 over its 128 threads.
+constexpr int kGroupBarrier = 1;
 
 }  // namespace decattn
 
@@ -212,14 +215,12 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[kSFull + s], 1);
-      mbar_init(&bar[kSFree + s], 4);
       mbar_init(&bar[kUFull + s], 1);
       mbar_init(&bar[kUEmpty + s], 1 + 4);
       mbar_init(&bar[kPReady + s], 4);
       mbar_init(&bar[kPvDone + s], 1);
     }
     mbar_init(&bar[kQReady], 4);
-    mbar_init(&bar[kGroup], 4);
     mbar_init(&bar[kFin], 1);
     *abort = 0;
     fence_mbar_init();
@@ -446,8 +447,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         const uint64_t dQ = dQ0 + (uint64_t)(((ut & 1) * L::QB) >> 4);
         for (int c = 0; c < nc; ++c, ++g) {
           const int st = (int)(g % kTcStages), sb = (int)(g & 1);
-          if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl) ||
-              !tc_wait(&bar[kSFree + sb], (uint32_t)(((g >> 1) & 1) ^ 1), p.status, abort, wl)) {
+          if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl)) {
             ok = false;
             break;
           }
@@ -477,17 +477,26 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     const float LN2 = 0.6931471805599453f;
     float* qcs_sm = reinterpret_cast<float*>(sm + L::OFF_QCS);   // [tile parity][16]
     int* red = reinterpret_cast<int*>(sm + L::OFF_RED);          // [2][4][16] chunk maxima (ordered ints)
-    int* flg = reinterpret_cast<int*>(sm + L::OFF_FLG);          // [2][4]
+    int* flg = reinterpret_cast<int*>(sm + L::OFF_FLG);          // [2][8]
     float* ered = reinterpret_cast<float*>(sm + L::OFF_ERED);    // [4][16] row-sum partials
     int us = 0; uint32_t uph = 0;
     int64_t g = 0;    // chunks processed so far
     int ut = 0;       // tiles processed so far
-    uint32_t gn = 0;  // group-barrier uses so far
-    bool ok = true;
-    auto gsync = [&]() -> bool {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar[kGroup]);
-      return tc_wait_warp(&bar[kGroup], (gn++) & 1u, p.status, abort, wl);
+    // The group's barrier, with the AND of the four warps' states. A warp whose wait gave up
+    // (which sets the abort flag) does not leave the loop on its own: it carries ok = false on
+    // to the group's next barrier, which every warp reaches in the same order, and the barrier's
+    // answer (the same in every thread) takes all four out together. The barrier thus always
+    // completes: it needs no time limit.
+    auto gsync = [&](bool mine) -> bool {
+      const uint32_t in = (mine && *abort == 0) ? 1u : 0u;
+      uint32_t all;
+      asm volatile(
+          "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+          "barrier.cta.red.and.aligned.pred po, %2, 128, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+          : "=r"(all)
+          : "r"(in), "n"(kGroupBarrier)
+          : "memory");
+      return all != 0u;
     };
     auto next_desc = [&](Unit& dd) -> bool {
       if (!tc_wait_warp(&bar[kUFull + us], uph, p.status, abort, wl)) return false;
@@ -497,12 +506,15 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       us ^= 1; if (us == 0) uph ^= 1;
       return true;
     };
-    // q of a tile into operand buffer `par`; the MMA warp may start the tile afterwards
-    auto publish_q = [&](const uint4 (&x)[2], int par) -> bool {
-      tc_store_q<M::QP>(x, sm + L::OFF_QB + par * L::QB, qcs_sm + kTcN * par);
-      fence_async_smem();
-      if (!gsync()) return false;
-      if (lane == 0) mbar_arrive(&bar[kQReady]);
+    // q of a tile (if there is one) into operand buffer `par`; the MMA warp may start the tile
+    // afterwards. The group's barrier is passed in either case.
+    auto publish_q = [&](const uint4 (&x)[2], int par, bool have, bool mine) -> bool {
+      if (have) {
+        tc_store_q<M::QP>(x, sm + L::OFF_QB + par * L::QB, qcs_sm + kTcN * par);
+        fence_async_smem();
+      }
+      if (!gsync(mine)) return false;
+      if (have && lane == 0) mbar_arrive(&bar[kQReady]);
       return true;
     };
     // waits on a chunk's P V: chunk gg's completes kPvDone + (gg & 1), phase (gg >> 1) & 1
@@ -523,11 +535,11 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     };
     Unit d;
     d.b = -1;
-    if (!next_desc(d)) ok = false;
-    if (ok && d.b >= 0) {
-      uint4 x[2];
-      tc_load_q(p, d, x);
-      ok = publish_q(x, 0);
+    bool ok = next_desc(d);
+    {
+      uint4 x[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+      if (ok && d.b >= 0) tc_load_q(p, d, x);
+      ok = publish_q(x, 0, ok && d.b >= 0, ok);
     }
     while (ok && d.b >= 0) {
       const int qp = ut & 1;
@@ -554,18 +566,17 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       dnext.b = -1;
       uint4 qx[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
       const int nc = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
+      bool fail = false;  // a group barrier found a warp that gave up: the four leave together
       for (int c = 0; c < nc; ++c, ++g) {
         const int st = (int)(g % kTcStages), sb = (int)(g & 1);
         if (c == nc - 1) {  // the next tile: its descriptor now, its q rows in flight meanwhile
-          if (!next_desc(dnext)) { ok = false; break; }
-          if (dnext.b >= 0) tc_load_q(p, dnext, qx);
+          if (!next_desc(dnext)) ok = false;
+          else if (dnext.b >= 0) tc_load_q(p, dnext, qx);
         }
         // ---- the chunk's K, V and scales have landed; V stays in the stage as the E4M3 operand
-        //      and the MMA warp frees the stage after the chunk's P V
-        if (!tc_wait_warp(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl)) {
-          ok = false;
-          break;
-        }
+        //      and the MMA warp frees the stage after the chunk's P V. (A wait that gives up
+        //      leaves ok = false for the next group barrier; see gsync.)
+        if (!tc_wait_warp(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl)) ok = false;
         const int j = d.tok_begin + c * kTcChunk + key;
         const bool valid = j < d.tok_end;
         // this key's page scales
@@ -573,29 +584,25 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         const float f = p.qk_scale_log2 * sc[st * 16 + blk];
         const float vsc = sc[st * 16 + 8 + blk];
         // P^T = P * (V page scale) * C with C a power of two such that the largest P (2^kTcTau)
-        // times the chunk's largest V scale lands in (224, 448]; the same in every thread. Only the
-        // blocks the producer filled for this chunk count (the other slots hold stale values).
-        float c_chunk;
-        {
-          const int nblk = min(kTcBlk, (d.tok_end - d.tok_begin - c * kTcChunk + 15) / 16);
-          float svmax = 0.f;
-          #pragma unroll
-          for (int i = 0; i < kTcBlk; ++i)
-            if (i < nblk) svmax = fmaxf(svmax, sc[st * 16 + 8 + i]);
+        // times the chunk's largest V scale lands in (224, 448]; the same in every thread. The
+        // largest scale of the keys in range (the producer filled their blocks; other slots hold
+        // stale values) is reduced per warp here and over the warps at the group's next barrier.
+        // V scales are >= 0, so their bit patterns order as the values.
+        const uint32_t wsv = __reduce_max_sync(0xffffffffu, valid ? __float_as_uint(vsc) : 0u);
+        auto chunk_c = [&]() -> float {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(flg + sb * 8 + 4);
+          const float svmax = __uint_as_float(max(max(v4.x, v4.y), max(v4.z, v4.w)));
           const float r = 448.f / ((float)(1 << kTcTau) * svmax);
           // the largest power of two <= r (exponent field only); 1 when no scale is usable
-          c_chunk = (svmax > 0.f && r < 1e30f) ? __int_as_float(__float_as_int(r) & 0x7f800000) : 1.f;
-        }
-        if (!tc_wait_warp(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort, wl)) { ok = false; break; }
+          return (svmax > 0.f && r < 1e30f) ? __int_as_float(__float_as_int(r) & 0x7f800000) : 1.f;
+        };
+        if (!tc_wait_warp(&bar[kSFull + sb], (uint32_t)((g >> 1) & 1), p.status, abort, wl)) ok = false;
         tc_fence_after();
         // scores times the column factors f * 2^-E, in pairs
         float s[kTcN];
         if constexpr (M::QP == 2) {  // the q hi and lo halves of S^T, added
           float s2[2 * kTcN];
           tmem_ld32(tmem + lane_off + M::NS * sb, s2);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar[kSFree + sb]);
           #pragma unroll
           for (int q4 = 0; q4 < kTcN / 4; ++q4) {
             const float4 qc = qcs4[q4];
@@ -610,9 +617,6 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           }
         } else {
           tmem_ld16(tmem + lane_off + M::NS * sb, s);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar[kSFree + sb]);
           #pragma unroll
           for (int q4 = 0; q4 < kTcN / 4; ++q4) {
             const float4 qc = qcs4[q4];
@@ -639,15 +643,17 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         // does any score of the chunk pass the reference by more than kTcTau? (one flag per warp)
         // (a tile's first chunk goes straight to the exact maxima: its reference is unset)
         bool upd = c == 0;
+        float c_chunk = 1.f;
         if (!upd) {
           bool over_ref = false;
           #pragma unroll
           for (int n = 0; n < kTcN; ++n) over_ref |= s[n] > mref[n] + (float)kTcTau;
           const int wflag = __any_sync(0xffffffffu, over_ref) ? 1 : 0;
-          if (lane == 0) flg[sb * 4 + warp] = wflag;
-          if (!gsync()) { ok = false; break; }
-          const int4 f4 = *reinterpret_cast<const int4*>(flg + sb * 4);
+          if (lane == 0) { flg[sb * 8 + warp] = wflag; flg[sb * 8 + 4 + warp] = (int)wsv; }
+          if (!gsync(ok)) { fail = true; break; }
+          const int4 f4 = *reinterpret_cast<const int4*>(flg + sb * 8);
           upd = (f4.x | f4.y | f4.z | f4.w) != 0;  // the same in every thread
+          c_chunk = chunk_c();
         }
         float cm[kTcN];
         if (upd) {
@@ -657,7 +663,9 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
             const int m = __reduce_max_sync(0xffffffffu, ordered_int(s[n]));
             if (lane == 0) rw[n] = m;
           }
-          if (!gsync()) { ok = false; break; }
+          if (c == 0 && lane == 0) flg[sb * 8 + 4 + warp] = (int)wsv;
+          if (!gsync(ok)) { fail = true; break; }
+          if (c == 0) c_chunk = chunk_c();
           const int4* r4 = reinterpret_cast<const int4*>(red + sb * 4 * kTcN);
           #pragma unroll
           for (int q4 = 0; q4 < kTcN / 4; ++q4) {
@@ -698,7 +706,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
           if (c > 0 && resc) {
             // O^T holds chunks 0 .. c-1 of this tile once the previous chunk's P V is done: rescale
             // every part's columns in place
-            if (!wait_pv(g - 1)) { ok = false; break; }
+            if (!wait_pv(g - 1)) ok = false;
             tc_fence_after();
             #pragma unroll
             for (int q = 0; q < M::PP; ++q) {
@@ -767,9 +775,9 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[kPReady + (g & 1)]);
       }
-      if (!ok) break;
+      if (fail) { ok = false; break; }
       // ---- the next tile's q: the MMA warp starts that tile while this one's epilogue runs
-      if (dnext.b >= 0 && !publish_q(qx, qp ^ 1)) { ok = false; break; }
+      if (!publish_q(qx, qp ^ 1, dnext.b >= 0, ok)) { ok = false; break; }
 
       // ---- epilogue: row sums over the tile, O^T / l, out or partial
       // row sums over the warp's 32 keys by a butterfly reduce-scatter (before the wait for the
@@ -795,12 +803,12 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       };
       warp_colsum(lacc, ered);
       if constexpr (Q8) warp_colsum(lrnd, ered + 4 * kTcN);
-      if (!wait_pv(g - 1)) { ok = false; break; }
+      if (!wait_pv(g - 1)) ok = false;
       tc_fence_after();
       float osum[kTcN];
       o_sum(tO, osum);
       tc_fence_before();
-      if (!gsync()) { ok = false; break; }
+      if (!gsync(ok)) { ok = false; break; }
       // lane n: row n's sums, the reciprocal that normalises O^T and (one warp) its lse
       float l_n = 0.f, lr_n = 0.f;
       if (lane < kTcN) {
