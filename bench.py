@@ -86,6 +86,9 @@ def parse():
                          "its own tolerance)")
     ap.add_argument("--bins", type=int, default=0,
                     help="bins of the plan (0: the library's default, SM count x 4)")
+    ap.add_argument("--fp8-kv", action="store_true",
+                    help="--config prefill: an E4M3 KV cache with per-(page, KV head) scales "
+                         "(dec_attn_prefill_fp8: a widening pass, then the bf16 prefill kernel)")
     ap.add_argument("--append", action="store_true",
                     help="each step starts with the fused pre-processing kernel (rotary embedding of the "
                          "step's new q / k rows and their KV append), and the decode reads the rotated q")
@@ -310,6 +313,8 @@ def make_workload(args):
     kw = dict(W.CONFIGS[args.config])
     if args.tile_len:
         kw["tile_len"] = args.tile_len
+    if getattr(args, "fp8_kv", False):
+        kw["kv_dtype"] = "fp8e4m3"
     lens = W.config_seq_lens(args.config)
     name = args.config
     if args.batch:
@@ -601,7 +606,8 @@ def run_ours(args, rank: int, world: int, local_rank: int, dist):
     line = {
         "metric": METRIC, "value": round(step_m, 3), "unit": "us/step", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_m / 1e3, 6), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": ("fp8e4m3 (q, P in e4m3)" if args.mma8 else "fp8e4m3->f16") if pr.kv_dtype == "fp8e4m3" else "bf16",
+        "scaling": "weak", "vs_baseline": None, "dtype": ("fp8e4m3 (q, P rounded to e4m3)" if args.mma8 else "fp8e4m3 (e4m3 products: q, P as exact e4m3 parts)")
+        if pr.kv_dtype == "fp8e4m3" else "bf16",
         "data": "synthetic",
         "config": {**bench_config(pr, world),
                    **({"products": "e4m3 tensor cores (q and P rounded to e4m3)"} if args.mma8 else {})},
@@ -696,10 +702,25 @@ def run_prefill(args, rank: int, world: int, local_rank: int, dist):
     log(f"[rank {rank}] prefill workload {pr.name}: B={pr.batch} Hq={pr.n_q_heads} Hkv={pr.n_kv_heads} "
         f"d={pr.head_dim} T={pr.q_tokens} P={pr.page_size} tokens={int(pr.seq_lens.sum())}")
     bf = torch.bfloat16
+    fp8 = pr.kv_dtype == "fp8e4m3"
     q = torch.from_numpy(pr.q.view(np.int16)).view(bf).to(dev)
-    k = torch.from_numpy(pr.k_pages.view(np.int16)).view(bf).to(dev)
-    v = torch.from_numpy(pr.v_pages.view(np.int16)).view(bf).to(dev)
+    if fp8:
+        k = torch.from_numpy(np.ascontiguousarray(pr.k_pages)).to(dev)
+        v = torch.from_numpy(np.ascontiguousarray(pr.v_pages)).to(dev)
+        sc = torch.from_numpy(np.ascontiguousarray(pr.kv_scales)).to(dev)
+    else:
+        k = torch.from_numpy(pr.k_pages.view(np.int16)).view(bf).to(dev)
+        v = torch.from_numpy(pr.v_pages.view(np.int16)).view(bf).to(dev)
     tab, lens = (torch.from_numpy(np.ascontiguousarray(a)).to(dev) for a in (pr.page_table, pr.seq_lens))
+    ws = None
+    if fp8:
+        ws = torch.empty(da.prefill_fp8_workspace_bytes(q.shape, k, tab, pr.q_tokens), dtype=torch.uint8, device=dev)
+
+    def attend():  # one prefill: FP8 KV = the widening pass + the bf16 prefill kernel
+        if fp8:
+            da.prefill_fp8(q, k, v, sc, tab, lens, sm_scale=pr.sm_scale, workspace=ws, out=out, lse=lse, status=status)
+        else:
+            da.prefill(q, k, v, tab, lens, sm_scale=pr.sm_scale, out=out, lse=lse, status=status)
     out = torch.empty((pr.batch, pr.q_tokens, pr.n_q_heads, pr.head_dim), dtype=torch.float32, device=dev)
     lse = torch.empty((pr.batch, pr.q_tokens, pr.n_q_heads), dtype=torch.float32, device=dev)
     status = torch.zeros((), dtype=torch.int32, device=dev)
@@ -711,7 +732,7 @@ def run_prefill(args, rank: int, world: int, local_rank: int, dist):
         torch.sum(flush, dim=0, out=flush_sink)
         torch.cuda._sleep(SLEEP_CYCLES)
         a.record(stream)
-        da.prefill(q, k, v, tab, lens, sm_scale=pr.sm_scale, out=out, lse=lse, status=status)
+        attend()
         b_.record(stream)
 
     def barrier():
@@ -767,7 +788,7 @@ def run_prefill(args, rank: int, world: int, local_rank: int, dist):
             q.copy_(hq, non_blocking=True)
             tab.copy_(htab, non_blocking=True)
             lens.copy_(hlens, non_blocking=True)
-            da.prefill(q, k, v, tab, lens, sm_scale=pr.sm_scale, out=out, lse=lse, status=status)
+            attend()
             hout.copy_(out, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
             b_.record(stream)
@@ -789,13 +810,15 @@ def run_prefill(args, rank: int, world: int, local_rank: int, dist):
         "metric": PREFILL_METRIC,
         "value": round(step_m, 3), "unit": "us/step", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(step_m / 1e3, 6), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (e4m3 KV widened to bf16)" if fp8 else "bf16",
+        "data": "synthetic",
         "config": bench_config(pr, world, prefill=True),
         "algorithmic_flops": flops,
-        "roofline": {"bound": "tensor", "kernel": "prefill_kernel", "achieved": round(tflops, 1), "peak": peak,
+        "roofline": {"bound": "tensor", "kernel": "widen_kv_kernel + prefill_kernel" if fp8 else "prefill_kernel",
+                     "achieved": round(tflops, 1), "peak": peak,
                      "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
-                     "traffic": prefill_traffic() if pr.name == "prefill" else None},
-        "gpu_launches": args.steps,  # one prefill kernel per timed step
+                     "traffic": prefill_traffic() if pr.name == "prefill" and not fp8 else None},
+        "gpu_launches": args.steps * (2 if fp8 else 1),  # per timed step: the prefill kernel (FP8: and the widening)
     }
     if sampler:
         line["clocks"] = sampler.summary()

@@ -406,6 +406,35 @@ DECATTN_API int dec_attn_prefill_varlen(const dec_attn_shape *shape, const void 
                                         const int32_t *cu_q_lens, int64_t total_q_rows, float *out, float *lse,
                                         int32_t *status, void *stream);
 
+/* Prefill over an FP8 (E4M3) KV cache (the same passage: prefill and paged-KV decode across
+ * BF16 / FP8 KV caches). The same attention as dec_attn_prefill / dec_attn_prefill_varlen over
+ * the dequantised cache, K = code * (page scale) and V likewise (the scales of
+ * dec_attn_run's DECATTN_KV_FP8E4M3). Two launches on the stream: a pass widens the pages each
+ * request uses into the workspace, K and V as RN_bf16(RN_fp32(code * scale)) (a relative error
+ * of at most 2^-9 per element against the exact product), in a bf16 pool laid out like the
+ * caller's (page i of request b at b * max_pages_per_seq + i) with its own page table; then the
+ * bf16 prefill kernel runs on it. So the result differs from attention over the exact products
+ * by the effect of that rounding on scores and values, besides the bf16 kernel's own.
+ *   shape         as dec_attn_prefill with kv_dtype DECATTN_KV_FP8E4M3;
+ *   q             device bf16 [B][T][Hq][128] (cu_q_lens NULL) or [total_q_rows][Hq][128] (packed);
+ *   k_pages, v_pages   device E4M3 [num_pages][Hkv][P][128], 16-byte aligned;
+ *   kv_scales     device fp32 [2][num_pages][Hkv] (K scales, then V), 4-byte aligned;
+ *   page_table, seq_lens   as dec_attn_run;
+ *   cu_q_lens     NULL: every request has q_tokens rows and total_q_rows must be batch * q_tokens;
+ *                 else as dec_attn_prefill_varlen;
+ *   workspace     device, 16-byte aligned, at least dec_attn_prefill_fp8_workspace_bytes(shape)
+ *                 bytes (caller-owned; its contents are overwritten);
+ *   out, lse, status   as dec_attn_prefill (status also reports a page id outside the pool seen by
+ *                 the widening pass).
+ * Returns DECATTN_ESMALL if the workspace is too small and otherwise as dec_attn_prefill; every
+ * check happens before the first launch (nothing is enqueued on an error). */
+DECATTN_API int64_t dec_attn_prefill_fp8_workspace_bytes(const dec_attn_shape *shape);
+DECATTN_API int dec_attn_prefill_fp8(const dec_attn_shape *shape, const void *q, const void *k_pages,
+                                     const void *v_pages, const float *kv_scales, const int32_t *page_table,
+                                     const int32_t *seq_lens, const int32_t *cu_q_lens, int64_t total_q_rows,
+                                     void *workspace, int64_t workspace_bytes, float *out, float *lse,
+                                     int32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,7 +29,8 @@ KV_BF16, KV_FP8E4M3, KV_FP8E4M3_MMA8 = 0, 1, 2
 API = ("dec_attn_default_bins", "dec_attn_default_tile_len", "dec_attn_plan_bytes", "dec_attn_plan", "dec_attn_plan_export",
        "dec_attn_workspace_bytes", "dec_attn_run", "dec_attn_split", "dec_attn_combine", "dec_attn_run_noalloc",
        "dec_attn_read_status", "dec_attn_status_string", "dec_attn_append_rope", "dec_attn_append_rope_fp8", "dec_attn_prefill",
-       "dec_attn_prefill_varlen", "dec_attn_plan_sparse_bytes",
+       "dec_attn_prefill_varlen", "dec_attn_prefill_fp8_workspace_bytes", "dec_attn_prefill_fp8",
+       "dec_attn_plan_sparse_bytes",
        "dec_attn_plan_sparse", "dec_attn_last_error", "dec_attn_test_set_waits")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -109,6 +110,11 @@ def load_library(path: str = LIB_PATH):
         lib.dec_attn_append_rope_fp8.restype = i32
         lib.dec_attn_prefill_varlen.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, i64, vp, vp, vp, vp]
         lib.dec_attn_prefill_varlen.restype = i32
+        lib.dec_attn_prefill_fp8_workspace_bytes.argtypes = [C.POINTER(ShapeT)]
+        lib.dec_attn_prefill_fp8_workspace_bytes.restype = i64
+        lib.dec_attn_prefill_fp8.argtypes = [C.POINTER(ShapeT), vp, vp, vp, vp, vp, vp, vp, i64, vp, i64, vp, vp, vp,
+                                             vp]
+        lib.dec_attn_prefill_fp8.restype = i32
         lib.dec_attn_test_set_waits.argtypes = [C.c_uint64, C.c_int32]
         lib.dec_attn_test_set_waits.restype = i32
         _lib = lib
@@ -392,6 +398,56 @@ def prefill_varlen(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor
     if rc != OK:
         raise DecAttnError(rc, "dec_attn_prefill_varlen")
     return out, lse
+
+
+def prefill_fp8(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, kv_scales: torch.Tensor,
+                page_table: torch.Tensor, seq_lens: torch.Tensor, *, cu_q_lens: torch.Tensor | None = None,
+                max_q_rows: int = 0, sm_scale: float = 0.0, workspace: torch.Tensor | None = None,
+                out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                status: torch.Tensor | None = None, stream=None):
+    """dec_attn_prefill_fp8: prefill over E4M3 pages (uint8 [num_pages][Hkv][P][128]) with fp32
+    kv_scales [2][num_pages][Hkv]. q is [B][T][Hq][128] (cu_q_lens None) or packed
+    [total][Hq][128] with cu_q_lens [B + 1] and ``max_q_rows`` bounding every request's rows.
+    ``workspace``: uint8 device buffer of at least prefill_fp8_workspace_bytes (allocated here if
+    None). Returns (out fp32, lse fp32) shaped like q's rows."""
+    lib = load_library()
+    if cu_q_lens is None:
+        B, T, Hq, d = q.shape
+        total = B * T
+        out_shape = (B, T, Hq, d)
+    else:
+        total, Hq, d = q.shape
+        B, T = page_table.shape[0], int(max_q_rows)
+        out_shape = (total, Hq, d)
+    shape = ShapeT(B, Hq, k_pages.shape[1], d, T, k_pages.shape[2], k_pages.shape[0], page_table.shape[1],
+                   KV_FP8E4M3, float(sm_scale))
+    need = int(lib.dec_attn_prefill_fp8_workspace_bytes(C.byref(shape)))
+    if need < 0:
+        raise DecAttnError(need, "dec_attn_prefill_fp8_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty(out_shape, dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(out_shape[:-1], dtype=torch.float32, device=q.device)
+    rc = lib.dec_attn_prefill_fp8(C.byref(shape), _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(kv_scales),
+                                  _ptr(page_table), _ptr(seq_lens), _ptr(cu_q_lens), int(total), _ptr(workspace),
+                                  int(workspace.numel() * workspace.element_size()), _ptr(out), _ptr(lse),
+                                  _ptr(status), _stream_handle(stream))
+    if rc != OK:
+        raise DecAttnError(rc, "dec_attn_prefill_fp8")
+    return out, lse
+
+
+def prefill_fp8_workspace_bytes(q_shape, k_pages: torch.Tensor, page_table: torch.Tensor, max_q_rows: int = 0) -> int:
+    """dec_attn_prefill_fp8_workspace_bytes for these pools (the workspace does not depend on q)."""
+    Hq, d = int(q_shape[-2]), int(q_shape[-1])
+    shape = ShapeT(page_table.shape[0], Hq, k_pages.shape[1], d, max(int(max_q_rows), 1), k_pages.shape[2],
+                   k_pages.shape[0], page_table.shape[1], KV_FP8E4M3, 0.0)
+    n = int(load_library().dec_attn_prefill_fp8_workspace_bytes(C.byref(shape)))
+    if n < 0:
+        raise DecAttnError(n, "dec_attn_prefill_fp8_workspace_bytes")
+    return n
 
 
 def test_set_waits(limit_ns: int = 0, skip_fill: int = -1) -> None:

@@ -258,10 +258,12 @@ static int enqueue(int stages, const dec_attn_shape* shape, const void* q, const
   return DECATTN_OK;
 }
 
-// Shared by dec_attn_prefill (cu_q null: T rows per request) and dec_attn_prefill_varlen.
+// Shared by dec_attn_prefill (cu_q null: T rows per request), dec_attn_prefill_varlen and the FP8
+// prefill (on its widened pool). check_only: every check and tensor map, no launch.
 static int prefill_enqueue(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
                            const int32_t* page_table, const int32_t* seq_lens, const int32_t* cu_q,
-                           int64_t total_rows, float* out, float* lse, int32_t* status, void* stream) {
+                           int64_t total_rows, float* out, float* lse, int32_t* status, void* stream,
+                           bool check_only = false) {
   if (!shape) return DECATTN_EINVAL;
   const dec_attn_shape& s = *shape;
   if (s.batch < 0 || s.q_tokens <= 0 || s.n_q_heads <= 0 || s.n_kv_heads <= 0 || s.page_size <= 0 ||
@@ -301,13 +303,81 @@ static int prefill_enqueue(const dec_attn_shape* shape, const void* q, const voi
   p.total_rows = total_rows;
   p.qk_scale_log2 = scale * 1.4426950408889634f;
   test_waits(&p.wait_ns, &p.skip_fill);
+  if (check_only) return DECATTN_OK;
   const cudaError_t e = launch_prefill(p, tmQ, tmK, tmV, tmO, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DECATTN_OK : cuda_fail("prefill kernel launch", e);
+}
+
+// FP8 prefill: widen the E4M3 pages each request uses into the workspace (bf16 pool with its own
+// page table), then the bf16 prefill on it. Every check happens before the first launch.
+static int prefill_fp8_enqueue(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
+                               const float* kv_scales, const int32_t* page_table, const int32_t* seq_lens,
+                               const int32_t* cu_q, int64_t total_rows, void* workspace, int64_t workspace_bytes,
+                               float* out, float* lse, int32_t* status, void* stream) {
+  if (!shape) return DECATTN_EINVAL;
+  const dec_attn_shape& s = *shape;
+  if (s.batch < 0 || s.q_tokens <= 0 || s.n_kv_heads <= 0 || s.page_size <= 0 || s.num_pages < 0 ||
+      s.max_pages_per_seq < 0 || total_rows < 0 || workspace_bytes < 0)
+    return DECATTN_EINVAL;
+  if (s.kv_dtype != DECATTN_KV_FP8E4M3 || s.head_dim != 128 || s.page_size % 16 != 0) return DECATTN_ENOTSUP;
+  if ((int64_t)s.batch * s.max_pages_per_seq >= (1ll << 31)) return DECATTN_ENOTSUP;
+  if (s.batch == 0 || total_rows == 0) return DECATTN_OK;
+  if (!k_pages || !v_pages || !kv_scales || !page_table || !seq_lens || !workspace) return DECATTN_EINVAL;
+  if (s.num_pages <= 0 || s.max_pages_per_seq <= 0) return DECATTN_EINVAL;
+  if (!aligned16(k_pages) || !aligned16(v_pages) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(kv_scales) & 3) != 0)
+    return DECATTN_EALIGN;
+  int64_t off_v = 0, off_pt = 0;
+  const int64_t need =
+      widen_scratch_bytes(s.batch, s.max_pages_per_seq, s.n_kv_heads, s.page_size, s.head_dim, &off_v, &off_pt);
+  if (workspace_bytes < need) return DECATTN_ESMALL;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  dec_attn_shape wide = s;  // the widened pool: bf16, page i of request b at b * max_pages_per_seq + i
+  wide.kv_dtype = DECATTN_KV_BF16;
+  wide.num_pages = s.batch * s.max_pages_per_seq;
+  const int32_t* wide_pt = reinterpret_cast<const int32_t*>(ws + off_pt);
+  int rc = prefill_enqueue(&wide, q, ws, ws + off_v, wide_pt, seq_lens, cu_q, total_rows, out, lse, status, stream,
+                           /*check_only=*/true);
+  if (rc != DECATTN_OK) return rc;
+  WidenParams w;
+  w.k_codes = static_cast<const uint8_t*>(k_pages);
+  w.v_codes = static_cast<const uint8_t*>(v_pages);
+  w.kv_scales = kv_scales;
+  w.page_table = page_table;
+  w.seq_lens = seq_lens;
+  w.k_out = reinterpret_cast<uint16_t*>(ws);
+  w.v_out = reinterpret_cast<uint16_t*>(ws + off_v);
+  w.pt_out = reinterpret_cast<int32_t*>(ws + off_pt);
+  w.status = status;
+  w.B = s.batch; w.Hkv = s.n_kv_heads; w.P = s.page_size; w.D = s.head_dim;
+  w.num_pages = s.num_pages; w.mpps = s.max_pages_per_seq;
+  const cudaError_t e = launch_widen_kv(w, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail("FP8 prefill widening launch", e);
+  return prefill_enqueue(&wide, q, ws, ws + off_v, wide_pt, seq_lens, cu_q, total_rows, out, lse, status, stream);
 }
 
 }  // namespace decattn
 
 using namespace decattn;
+
+extern "C" int64_t dec_attn_prefill_fp8_workspace_bytes(const dec_attn_shape* shape) {
+  if (!shape) return DECATTN_EINVAL;
+  const dec_attn_shape& s = *shape;
+  if (s.batch < 0 || s.n_kv_heads <= 0 || s.page_size <= 0 || s.max_pages_per_seq < 0 || s.head_dim <= 0)
+    return DECATTN_EINVAL;
+  return widen_scratch_bytes(s.batch, s.max_pages_per_seq, s.n_kv_heads, s.page_size, s.head_dim, nullptr, nullptr);
+}
+
+extern "C" int dec_attn_prefill_fp8(const dec_attn_shape* shape, const void* q, const void* k_pages,
+                                    const void* v_pages, const float* kv_scales, const int32_t* page_table,
+                                    const int32_t* seq_lens, const int32_t* cu_q_lens, int64_t total_q_rows,
+                                    void* workspace, int64_t workspace_bytes, float* out, float* lse,
+                                    int32_t* status, void* stream) {
+  if (!shape) return DECATTN_EINVAL;
+  if (!cu_q_lens && total_q_rows != (int64_t)shape->batch * shape->q_tokens) return DECATTN_EINVAL;
+  return prefill_fp8_enqueue(shape, q, k_pages, v_pages, kv_scales, page_table, seq_lens, cu_q_lens, total_q_rows,
+                             workspace, workspace_bytes, out, lse, status, stream);
+}
 
 extern "C" int dec_attn_prefill(const dec_attn_shape* shape, const void* q, const void* k_pages, const void* v_pages,
                                 const int32_t* page_table, const int32_t* seq_lens, float* out, float* lse,

@@ -198,6 +198,20 @@ struct PrefillParams {
   int32_t skip_fill;          // tests only: CTA 0's producer leaves this K block out (-1: none)
 };
 
+// FP8 prefill: the E4M3 pages each request uses, widened to a bf16 scratch pool (prefill_fp8.cu).
+struct WidenParams {
+  const uint8_t* k_codes;     // E4M3 [num_pages][Hkv][P][D]
+  const uint8_t* v_codes;
+  const float* kv_scales;     // [2][num_pages][Hkv]: K, then V
+  const int32_t* page_table;  // [B][mpps]
+  const int32_t* seq_lens;    // [B]
+  uint16_t* k_out;            // bf16 [B * mpps][Hkv][P][D]: page i of request b at b * mpps + i
+  uint16_t* v_out;
+  int32_t* pt_out;            // [B][mpps]: b * mpps + i
+  int32_t* status;            // optional device word
+  int B, Hkv, P, D, num_pages, mpps;
+};
+
 // Query rows of one KV head that a decode tile computes at once (G * T), and query tokens per
 // request (T), that dec_attn_run supports.
 constexpr int kMaxGT = 64;
@@ -473,5 +487,8 @@ cudaError_t launch_split_tc(const SplitParams& p, const CUtensorMap& tmK, const 
 cudaError_t launch_combine(const CombineParams& p, int device, cudaStream_t st);  // combine.cu
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const CUtensorMap& tmO, cudaStream_t st);  // prefill.cu
+// bytes of the widened pool (K, then V at *off_v, then the page table at *off_pt)   prefill_fp8.cu
+int64_t widen_scratch_bytes(int B, int mpps, int Hkv, int P, int D, int64_t* off_v, int64_t* off_pt);
+cudaError_t launch_widen_kv(const WidenParams& p, cudaStream_t st);  // prefill_fp8.cu
 
 }  // namespace decattn

@@ -272,3 +272,37 @@ def test_append_rope_fp8_rejects_bad_args(lib):
     assert call(_shape(kv_dtype=da.KV_FP8E4M3), sc=None) == da.EINVAL
     assert call(_shape(kv_dtype=da.KV_FP8E4M3), sc=FAKE + 2) == da.EALIGN
     assert call(_shape(kv_dtype=da.KV_FP8E4M3), q=FAKE + 2) == da.EALIGN
+
+
+def test_prefill_fp8_workspace_and_host_checks(lib):
+    # the widened pool: K and V bf16 [B * max_pages_per_seq][Hkv][P][128], then its page table
+    s = _shape(kv_dtype=da.KV_FP8E4M3, q_tokens=300)
+    B, mpps, Hkv, P, d = s.batch, s.max_pages_per_seq, s.n_kv_heads, s.page_size, s.head_dim
+    kv = -(-(B * mpps * Hkv * P * d * 2) // 256) * 256
+    need = lib.dec_attn_prefill_fp8_workspace_bytes(C.byref(s))
+    assert need == 2 * kv + -(-(B * mpps * 4) // 256) * 256
+    assert lib.dec_attn_prefill_fp8_workspace_bytes(None) == da.EINVAL
+
+    def call(shape, ws_bytes=need, total=None, **kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, sc=FAKE, tab=FAKE, lens=FAKE, cu=None, ws=FAKE, out=FAKE, lse=FAKE)
+        a.update(kw)
+        total = shape.batch * shape.q_tokens if total is None else total
+        return lib.dec_attn_prefill_fp8(C.byref(shape), a["q"], a["k"], a["v"], a["sc"], a["tab"], a["lens"], a["cu"],
+                                        total, a["ws"], ws_bytes, a["out"], a["lse"], None, None)
+    # every case fails a host check before any tensor map is built or a kernel launched
+    assert lib.dec_attn_prefill_fp8(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, FAKE, need, FAKE, FAKE,
+                                    None, None) == da.EINVAL
+    assert call(_shape(kv_dtype=da.KV_BF16, q_tokens=300)) == da.ENOTSUP      # bf16 pools: dec_attn_prefill
+    assert call(_shape(kv_dtype=da.KV_FP8E4M3_MMA8, q_tokens=300)) == da.ENOTSUP
+    assert call(_shape(kv_dtype=da.KV_FP8E4M3, q_tokens=300, head_dim=64)) == da.ENOTSUP
+    assert call(_shape(kv_dtype=da.KV_FP8E4M3, q_tokens=300, page_size=8)) == da.ENOTSUP
+    assert call(_shape(kv_dtype=da.KV_FP8E4M3, q_tokens=0)) == da.EINVAL
+    assert call(s, total=5) == da.EINVAL                  # no row offsets: batch * q_tokens rows
+    for name in ("k", "v", "sc", "tab", "lens", "ws"):
+        assert call(s, **{name: None}) == da.EINVAL
+    assert call(s, k=FAKE + 8) == da.EALIGN
+    assert call(s, ws=FAKE + 8) == da.EALIGN
+    assert call(s, sc=FAKE + 2) == da.EALIGN
+    assert call(s, ws_bytes=need - 1) == da.ESMALL
+    assert call(_shape(kv_dtype=da.KV_FP8E4M3, batch=0, q_tokens=300), q=None, k=None, v=None, sc=None, tab=None,
+                lens=None, ws=None, out=None, lse=None) == da.OK
