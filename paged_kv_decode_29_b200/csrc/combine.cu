@@ -11,8 +11,8 @@
 // cb_b chunks of up to kCombineChunk tiles; the items (b, row, chunk) are numbered request
 // by request (block-sparse plans: (request, KV head) pair by pair, since pairs keep their
 // own tiles). The kernel is persistent: every warp takes items w, w + #warps, ...
-//  * a warp loads the lse and the D floats of up to 16 partial rows (8 loads in flight per
-//    lane at a time) and folds them into (max, weight, weighted sum);
+//  * a warp loads the lse and the D floats of up to kCombineChunk (32) partial rows (8 loads in
+//    flight per lane at a time) and folds them into (max, weight, weighted sum);
 //  * a row made of one chunk is finished right there;
 //  * otherwise the warp publishes its chunk state and bumps the row's counter; the warp
 //    that brings the counter to cb_b merges the row's chunk states (8 at once, with an
@@ -137,16 +137,18 @@ __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_ke
       }
       const int64_t slot0 = slot_base + (int64_t)j * kCombineChunk;
       const int n = min(kCombineChunk, nt - j * kCombineChunk);
-      // ---- fold up to kCombineChunk partial rows, in two halves of loads in flight at once
-      //      (with every warp loading, the fold runs at DRAM bandwidth; halves keep the
-      //      registers below the occupancy limit)
+      // ---- fold up to kCombineChunk partial rows, kLoads loads in flight per lane at a time
+      //      (with every warp loading, the fold runs at DRAM bandwidth; batches of kLoads keep the
+      //      registers below the occupancy limit). Lane i holds the lse of row i of the chunk.
+      static_assert(kCombineChunk <= 32 && kCombineChunk % 8 == 0, "one lse per lane, whole batches");
       const float my_lse = lane < n ? p.part_lse[(slot0 + lane) * p.GT + r] : -INFINITY;
       const V* src = reinterpret_cast<const V*>(p.part_o + (slot0 * p.GT + r) * D) + lane;
       const int64_t stride = (int64_t)p.GT * (D / VEC);  // V elements between consecutive tiles' rows
-      constexpr int kHalf = kCombineChunk / 2;
-      V v[kHalf];
+      constexpr int kLoads = 8;
+      constexpr int kRounds = kCombineChunk / kLoads;
+      V v[kLoads];
       #pragma unroll
-      for (int i = 0; i < kHalf; ++i)
+      for (int i = 0; i < kLoads; ++i)
         if (i < n) v[i] = __ldcs(src + i * stride);
       float M = my_lse;
       #pragma unroll
@@ -156,17 +158,17 @@ __global__ void __launch_bounds__(kCombineThreads, kCombineCtasPerSm) combine_ke
       #pragma unroll
       for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
       #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        if (hf == 1) {
-          if (n <= kHalf) break;
+      for (int hf = 0; hf < kRounds; ++hf) {
+        if (hf > 0) {
+          if (n <= hf * kLoads) break;
           #pragma unroll
-          for (int i = 0; i < kHalf; ++i)
-            if (kHalf + i < n) v[i] = __ldcs(src + (kHalf + i) * stride);
+          for (int i = 0; i < kLoads; ++i)
+            if (hf * kLoads + i < n) v[i] = __ldcs(src + (hf * kLoads + i) * stride);
         }
         #pragma unroll
-        for (int i = 0; i < kHalf; ++i) {
-          const float wi = __shfl_sync(0xffffffffu, my_w, hf * kHalf + i);
-          if (hf * kHalf + i < n) {
+        for (int i = 0; i < kLoads; ++i) {
+          const float wi = __shfl_sync(0xffffffffu, my_w, hf * kLoads + i);
+          if (hf * kLoads + i < n) {
             const float* f = reinterpret_cast<const float*>(&v[i]);
             #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] += wi * f[e];

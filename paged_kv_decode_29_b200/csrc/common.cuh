@@ -220,7 +220,7 @@ constexpr int kMaxT = 8;
 // The combine kernel folds the partials of one query row in chunks of this many tiles.
 // A request with n_b tiles gives each of its rows cb_b = ceil(n_b / kCombineChunk) chunks
 // (1 if n_b == 0: the row is zero-filled; 0 if n_b == 1: the split kernel wrote the row).
-constexpr int kCombineChunk = 16;
+constexpr int kCombineChunk = 32;
 
 __host__ __device__ inline int combine_chunks(int64_t n_b) {
   return n_b == 0 ? 1 : n_b == 1 ? 0 : (int)((n_b + kCombineChunk - 1) / kCombineChunk);
