@@ -150,7 +150,7 @@ SPLIT_TRAFFIC_CAPTURED = {
     },
 }
 # prefill_kernel on the full prefill workload (read, write): a few hundred MB on the device.
-PREFILL_TRAFFIC_CAPTURED = {"source_hash": "1ae2fe489d1ff892", "read": 108431616, "write": 85455104}
+PREFILL_TRAFFIC_CAPTURED = {"source_hash": "3447e365c41c00d8", "read": 109325568, "write": 85145600}
 
 
 def config_algorithmic_bytes(name: str, batch: int | None = None) -> int:

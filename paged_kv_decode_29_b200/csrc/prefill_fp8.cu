@@ -16,49 +16,47 @@
 
 namespace decattn {
 
-constexpr int kWidenThreads = 256;
+constexpr int kWidenThreads = 128;
 
-// CTA w = b * mpps + i: scratch page w (page i of request b), every KV head, K then V. Pages past
-// the request's keys are never read by the prefill kernel and are left unwritten; a page id
-// outside the pool is reported (DECATTN_EDEVICE) and its scratch page is zero.
+// CTA (w, y): scratch page w = b * mpps + i (page i of request b), y = kv * Hkv + h: K (kv = 0) or V
+// of KV head h, one 16-code chunk per thread. Pages past the request's keys are never read by the
+// prefill kernel and are left unwritten; a page id outside the pool is reported (DECATTN_EDEVICE)
+// and its scratch page is zero.
 __global__ void __launch_bounds__(kWidenThreads) widen_kv_kernel(const WidenParams p) {
   const int64_t w = blockIdx.x;
+  const int kv = (int)blockIdx.y / p.Hkv, h = (int)blockIdx.y - kv * p.Hkv;
   const int b = (int)(w / p.mpps);
   const int i = (int)(w - (int64_t)b * p.mpps);
-  if (threadIdx.x == 0) p.pt_out[w] = (int32_t)w;
+  if (threadIdx.x == 0 && blockIdx.y == 0) p.pt_out[w] = (int32_t)w;
   const int Lb = p.seq_lens[b];
   if (Lb < 0) {
-    if (threadIdx.x == 0 && i == 0) set_status(p.status, DECATTN_EDEVICE);
+    if (threadIdx.x == 0 && i == 0 && blockIdx.y == 0) set_status(p.status, DECATTN_EDEVICE);
     return;
   }
   if ((int64_t)i * p.P >= Lb) return;
-  int pid = p.page_table[w];
+  const int pid = p.page_table[w];
   const bool good = pid >= 0 && pid < p.num_pages;
-  if (!good && threadIdx.x == 0) set_status(p.status, DECATTN_EDEVICE);
-  const int per_head = p.P * p.D / 16;  // 16-code chunks of one (page, KV head) slice
-  const int n = 2 * p.Hkv * per_head;
-  for (int t = threadIdx.x; t < n; t += kWidenThreads) {
-    const int kv = t / (p.Hkv * per_head);  // 0: K, 1: V
-    const int rem = t - kv * p.Hkv * per_head;
-    const int h = rem / per_head, c = rem - h * per_head;
+  if (!good && threadIdx.x == 0 && blockIdx.y == 0) set_status(p.status, DECATTN_EDEVICE);
+  const float s = good ? p.kv_scales[(int64_t)kv * p.num_pages * p.Hkv + (int64_t)pid * p.Hkv + h] : 0.f;
+  const uint8_t* src = (kv ? p.v_codes : p.k_codes) + ((int64_t)(good ? pid : 0) * p.Hkv + h) * p.P * p.D;
+  uint16_t* dst = (kv ? p.v_out : p.k_out) + (w * p.Hkv + h) * p.P * p.D;
+  const int per_slice = p.P * p.D / 16;  // 16-code chunks of the (page, KV head) slice
+  for (int c = threadIdx.x; c < per_slice; c += kWidenThreads) {
     uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (good) {
-      const uint8_t* src = (kv ? p.v_codes : p.k_codes) + ((int64_t)pid * p.Hkv + h) * p.P * p.D + 16 * c;
-      const float s = p.kv_scales[(int64_t)kv * p.num_pages * p.Hkv + (int64_t)pid * p.Hkv + h];
-      const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(src + 16 * c));
       const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
       #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int q = 0; q < 4; ++q) {
         #pragma unroll
         for (int half = 0; half < 2; ++half) {  // two codes at a time: exact in f16, then times s
-          const float2 f = f16x2_to_float2(e4m3x2_to_f16x2(half ? (xw[k] >> 16) : (xw[k] & 0xffffu)));
-          o[2 * k + half] = pack_bf16(f.x * s, f.y * s);
+          const float2 f = f16x2_to_float2(e4m3x2_to_f16x2(half ? (xw[q] >> 16) : (xw[q] & 0xffffu)));
+          o[2 * q + half] = pack_bf16(f.x * s, f.y * s);
         }
       }
     }
-    uint16_t* dst = (kv ? p.v_out : p.k_out) + (w * p.Hkv + h) * p.P * p.D + 16 * c;
-    reinterpret_cast<uint4*>(dst)[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    reinterpret_cast<uint4*>(dst)[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    reinterpret_cast<uint4*>(dst + 16 * c)[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<uint4*>(dst + 16 * c)[1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 
@@ -72,8 +70,8 @@ int64_t widen_scratch_bytes(int B, int mpps, int Hkv, int P, int D, int64_t* off
 cudaError_t launch_widen_kv(const WidenParams& p, cudaStream_t st) {
   const int64_t grid = (int64_t)p.B * p.mpps;
   if (grid <= 0) return cudaSuccess;
-  if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-  widen_kv_kernel<<<(unsigned)grid, kWidenThreads, 0, st>>>(p);
+  if (grid > 0x7fffffff || 2 * p.Hkv > 65535) return cudaErrorInvalidValue;
+  widen_kv_kernel<<<dim3((unsigned)grid, (unsigned)(2 * p.Hkv)), kWidenThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -300,7 +300,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
     };
     auto wait0 = [&](uint64_t* b, uint32_t par) -> bool {  // lane 0 waits, the warp follows
       int r = 1;
-      if (lane == 0) r = tc_wait(b, par, p.status, abort, wl) ? 1 : 0;
+      if (lane == 0) r = tc_wait_suspend(b, par, p.status, abort, wl) ? 1 : 0;
       return __shfl_sync(0xffffffffu, r, 0) != 0;
     };
     // lane l: page id of page l of a tile's first window of 32 pages (0 past the tile's pages)
@@ -424,7 +424,7 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
       // O^T (+)= V^T P^T over chunk gg's 128 keys. A tile's first chunk overwrites O^T: the
       // softmax group signals that chunk's P only after it has read the previous tile's O^T.
       auto pv = [&](int64_t gg, bool first_of_tile) -> bool {
-        if (!tc_wait(&bar[kPReady + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl)) return false;
+        if (!tc_wait_suspend(&bar[kPReady + (gg & 1)], (uint32_t)((gg >> 1) & 1), p.status, abort, wl)) return false;
         tc_fence_after();
         const int sg = (int)(gg % kTcStages);
         const uint64_t a0 = dV + (uint64_t)((sg * L::KCH) >> 4);
@@ -437,17 +437,17 @@ split_tc_kernel(const SplitParams p, const __grid_constant__ CUtensorMap tmK, co
         return true;
       };
       for (;;) {
-        if (!tc_wait(&bar[kUFull + us], uph, p.status, abort, wl)) { ok = false; break; }
+        if (!tc_wait_suspend(&bar[kUFull + us], uph, p.status, abort, wl)) { ok = false; break; }
         const Unit d = umeta[us];
         mbar_arrive(&bar[kUEmpty + us]);
         us ^= 1; if (us == 0) uph ^= 1;
         if (d.b < 0) break;
         const int nc = (d.tok_end - d.tok_begin + kTcChunk - 1) / kTcChunk;
-        if (!tc_wait(&bar[kQReady], (uint32_t)(ut & 1), p.status, abort, wl)) { ok = false; break; }
+        if (!tc_wait_suspend(&bar[kQReady], (uint32_t)(ut & 1), p.status, abort, wl)) { ok = false; break; }
         const uint64_t dQ = dQ0 + (uint64_t)(((ut & 1) * L::QB) >> 4);
         for (int c = 0; c < nc; ++c, ++g) {
           const int st = (int)(g % kTcStages), sb = (int)(g & 1);
-          if (!tc_wait(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl)) {
+          if (!tc_wait_suspend(&bar[kKvFull + st], (uint32_t)((g / kTcStages) & 1), p.status, abort, wl)) {
             ok = false;
             break;
           }
