@@ -140,13 +140,13 @@ def split_kernel_name(pr) -> str:
 # the ratio of algorithmic bytes (reads measured within 0.05% of the algorithmic bytes on every
 # captured case, so traffic grows in proportion): workload -> (requests captured, read, write).
 SPLIT_TRAFFIC_CAPTURED = {
-    "source_hash": "f977df437aa9655e",  # kernel_source_hash() of the sources these were captured on
+    "source_hash": "fa4bf76c34d9ec92",  # kernel_source_hash() of the sources these were captured on
     "configs": {
-        "uniform": (8, 134362112, 3442688),
-        "mixed": (16, 1039149056, 17764864),
-        "fp8_spec": (4, 167783168, 4456704),
-        "long_b4": (1, 537029120, 6024960),
-        "long_b1": (1, 537049088, 15755008),
+        "uniform": (8, 134365184, 3114752),
+        "mixed": (16, 1039181824, 17484288),
+        "fp8_spec": (4, 167784448, 4281856),
+        "long_b4": (1, 536983040, 6753536),
+        "long_b1": (1, 536993792, 16440320),
     },
 }
 # prefill_kernel on the full prefill workload (read, write): a few hundred MB on the device.
