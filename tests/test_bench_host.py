@@ -112,3 +112,17 @@ def test_both_arms_report_the_same_config():
     c = bench.bench_config(pr, 1)
     assert c["workload"] == "tiny" and "l2" in c and c["parallelism"] == "single GPU"
     assert "n_bins" not in c
+
+
+def test_fp8_kv_option_builds_the_same_workload_with_e4m3_pages():
+    # --fp8-kv keeps the workload's shape, lengths and seed and only changes the KV cache to E4M3
+    # pages with per-(page, head) scales (the prefill entry point then widens them)
+    import argparse
+    base = argparse.Namespace(config="prefill", tile_len=0, batch=1, fp8_kv=False)
+    fp8 = argparse.Namespace(config="prefill", tile_len=0, batch=1, fp8_kv=True)
+    a, b = bench.make_workload(base), bench.make_workload(fp8)
+    assert a.kv_dtype == "bf16" and b.kv_dtype == "fp8e4m3"
+    assert np.array_equal(a.seq_lens, b.seq_lens) and np.array_equal(a.q, b.q)
+    assert np.array_equal(a.page_table, b.page_table)
+    assert b.k_pages.dtype == np.uint8 and b.kv_scales.shape == (2, b.num_pages, b.n_kv_heads)
+    assert bench.bench_config(b, 1, prefill=True)["kv_dtype"] == "fp8e4m3"
