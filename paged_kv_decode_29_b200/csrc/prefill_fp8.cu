@@ -23,10 +23,12 @@ constexpr int kWidenThreads = 128;
 // prefill kernel and are left unwritten; a page id outside the pool is reported (DECATTN_EDEVICE)
 // and its scratch page is zero.
 __global__ void __launch_bounds__(kWidenThreads) widen_kv_kernel(const WidenParams p) {
-  const int64_t w = blockIdx.x;
+  // 32-bit index arithmetic (the page index is below 2^31: the grid's x size): a 64-bit division
+  // is a software routine, and every CTA converts only one slice
+  const int w = (int)blockIdx.x;
   const int kv = (int)blockIdx.y / p.Hkv, h = (int)blockIdx.y - kv * p.Hkv;
-  const int b = (int)(w / p.mpps);
-  const int i = (int)(w - (int64_t)b * p.mpps);
+  const int b = w / p.mpps;
+  const int i = w - b * p.mpps;
   if (threadIdx.x == 0 && blockIdx.y == 0) p.pt_out[w] = (int32_t)w;
   const int Lb = p.seq_lens[b];
   if (Lb < 0) {
@@ -39,7 +41,7 @@ __global__ void __launch_bounds__(kWidenThreads) widen_kv_kernel(const WidenPara
   if (!good && threadIdx.x == 0 && blockIdx.y == 0) set_status(p.status, DECATTN_EDEVICE);
   const float s = good ? p.kv_scales[(int64_t)kv * p.num_pages * p.Hkv + (int64_t)pid * p.Hkv + h] : 0.f;
   const uint8_t* src = (kv ? p.v_codes : p.k_codes) + ((int64_t)(good ? pid : 0) * p.Hkv + h) * p.P * p.D;
-  uint16_t* dst = (kv ? p.v_out : p.k_out) + (w * p.Hkv + h) * p.P * p.D;
+  uint16_t* dst = (kv ? p.v_out : p.k_out) + ((int64_t)w * p.Hkv + h) * p.P * p.D;
   const int per_slice = p.P * p.D / 16;  // 16-code chunks of the (page, KV head) slice
   for (int c = threadIdx.x; c < per_slice; c += kWidenThreads) {
     uint32_t o[8] = {0, 0, 0, 0, 0, 0, 0, 0};
