@@ -71,9 +71,10 @@ typedef enum {
 /* KV element type of the pools, and how the products are formed:
  *   DECATTN_KV_BF16          bf16 pages;
  *   DECATTN_KV_FP8E4M3       OCP E4M3 pages with fp32 per-(page, KV head) scales; q keeps bf16
- *                            precision (two E4M3 parts) and P enters P V as f16: the result is
- *                            checked against the fp64 oracle on the dequantised pages (out 2e-3,
- *                            lse 1e-4);
+ *                            precision (two E4M3 parts) and P keeps about 12 significant bits
+ *                            (three E4M3 parts on the tcgen05 kernel, head_dim 128 and G*T <= 16;
+ *                            f16 hi + lo on the warp-MMA kernel otherwise): the result is checked
+ *                            against the fp64 oracle on the dequantised pages (out 2e-3, lse 1e-4);
  *   DECATTN_KV_FP8E4M3_MMA8  the same pages and scales, with both products on E4M3 tensor cores
  *                            (the HPC-Ops article at sdftguanye.com, section on fine-grained task
  *                            scheduling and data rearrangement: an FP8 attention kernel): q rounded to
